@@ -1,0 +1,287 @@
+"""CPU oracle of the single-GPU MoE-layer forward (router -> top-k -> counts and
+scan -> stable permutation -> grouped SwiGLU FFN -> weighted combine).
+
+TEST INFRASTRUCTURE ONLY. Nothing on the product path may import, call or run
+this module: only ``tests/``, ``__graft_entry__.smoke()`` and ``bench.py``'s
+CPU-baseline / reference legs do. It shares no code with the CUDA library and
+imports nothing from it.
+
+Plain numpy, float64 arithmetic unless a step is an integer decision that the
+kernels take in fp32 (the top-k selection compares fp32 logits, as the kernels
+do). Slow and obviously correct is the goal: no blocking, no fusion, no
+reordering beyond what each definition states. Library primitives used as
+steps: ``numpy.matmul``/``dot`` (fp64), ``numpy.lexsort``, ``numpy.exp``.
+
+Sources (page title, section):
+  [P1] "Operators & compilers: MoE routing and sparse kernels"
+       (charles2530.github.io), sections 2-4: top-k routing, token permutation
+       by counting + prefix sum, capacity factor with drops.
+  [P2] "Two upstream innovations of MoE: Routing-Free and OmniMoE"
+       (chatdocs.ruinique.com), section 1.1 (Router -> Softmax -> TopK) and
+       section 2.3 (expert-centric scheduling: flatten the (token, expert)
+       tasks, sort by (expert, token), run grouped, scatter-add back).
+  [P4] "How AI chips support MoE", chapter 4, sections 4.2-4.3 (gating is a
+       linear map, then softmax, then top-K selection).
+  [P5] SonicMoE explainer (gitcode.csdn.net), section 1 (y = sum_i gate_i(x) *
+       expert_i(x) over the top-k experts), section 3 (the GPU pipeline:
+       route, regroup to expert-major, grouped GEMM, SwiGLU, second grouped
+       GEMM, scatter/combine), section 11 (expert-major metadata: per-expert
+       counts, expert-major slot -> token, token-major slot -> expert-major
+       slot).
+
+Readings where the pages are silent (each also listed in the design notes):
+  * top-k order: descending logit, ties to the lower expert id, +0 == -0;
+    selection is on the fp32 logits (softmax is monotone);
+  * weights: softmax restricted to the K selected, i.e. renormalised;
+  * capacity C = ceil(cf * T * K / E); an expert keeps its first C
+    assignments in token order and drops the rest;
+  * order inside an expert: ascending token id (the section 2.3 example of
+    [P2] shows it); dropped slots contribute 0 and are not re-renormalised;
+  * SwiGLU(g, u) = g / (1 + exp(-g)) * u with g from W_gate, u from W_up.
+"""
+from __future__ import annotations
+
+import math
+from typing import Optional
+
+import numpy as np
+
+F64 = np.float64
+
+
+def as_f64(a) -> np.ndarray:
+    """Widen an array (numpy, or a CPU torch tensor of any float dtype) to fp64."""
+    if hasattr(a, "detach"):  # torch tensor: bf16 has no numpy dtype
+        import torch
+        a = a.detach().to("cpu", torch.float64).numpy()
+    return np.asarray(a, dtype=F64)
+
+
+# --------------------------------------------------------------------------- router
+def router_logits(x, w_r, bias=None) -> np.ndarray:
+    """[P4] 4.2 / [P2] 1.1: router scores are a linear map, logits = x . W_r.
+
+    x[T, d], W_r[d, E]; fp64 products and sums, optional per-expert bias added
+    to every token's logits, then rounded to fp32 (the precision in which the
+    top-k decision is taken on both sides)."""
+    z = as_f64(x) @ as_f64(w_r)
+    if bias is not None:
+        z = z + as_f64(bias)[None, :]
+    return z.astype(np.float32)
+
+
+def topk_ids(logits_f32, K: int) -> np.ndarray:
+    """[P1] 2, [P4] 4.3: per token, the K experts with the largest logits.
+
+    Order key (logit descending, expert id ascending); slot 0 holds the best.
+    ``np.lexsort`` sorts by its last key first, so the keys are (id, -logit).
+    Comparisons are on fp32 values, where +0 and -0 are equal."""
+    lg = np.asarray(logits_f32, dtype=np.float32)
+    T, E = lg.shape
+    if not (1 <= K <= E):
+        raise ValueError("need 1 <= K <= E")
+    ids = np.broadcast_to(np.arange(E), (T, E))
+    neg = -lg.astype(F64)  # exact; -(+0) == -(-0) compare equal
+    order = np.lexsort((ids, neg), axis=1)
+    return order[:, :K].astype(np.int32)
+
+
+def topk_weights(logits_f32, ids, renormalize: bool = True) -> np.ndarray:
+    """[P2] 1.1 Router -> Softmax -> TopK, with the top-K probabilities renormalised.
+
+    w_k = exp(l_k - m) / sum_{j in S} exp(l_j - m), m the token's largest
+    logit, S = the K selected experts (renormalised) or all E experts (plain
+    softmax, ``renormalize=False``). fp64, rounded to fp32."""
+    lg = np.asarray(logits_f32, dtype=np.float32).astype(F64)
+    T, E = lg.shape
+    m = lg.max(axis=1, keepdims=True)
+    p = np.exp(lg - m)
+    sel = np.take_along_axis(p, np.asarray(ids, dtype=np.int64), axis=1)
+    den = sel.sum(axis=1, keepdims=True) if renormalize else p.sum(axis=1, keepdims=True)
+    return (sel / den).astype(np.float32)
+
+
+def route(logits_f32, K: int, renormalize: bool = True):
+    ids = topk_ids(logits_f32, K)
+    return ids, topk_weights(logits_f32, ids, renormalize)
+
+
+# --------------------------------------------------------------------------- dispatch
+def capacity(capacity_factor: float, T: int, K: int, E: int) -> Optional[int]:
+    """[P1] 4: an upper bound on the tokens one expert receives.
+
+    C = ceil(cf * T * K / E), computed in double from the fp32 factor; cf <= 0
+    means no limit (None)."""
+    cf = float(np.float32(capacity_factor))
+    if cf <= 0.0:
+        return None
+    return int(math.ceil(cf * T * K / E))
+
+
+def permute(topk_ids_, E: int, C: Optional[int] = None):
+    """[P1] 3 (counting + prefix sum), [P2] 2.3 (sort tasks by (expert, token)),
+    [P5] 11 (expert-major metadata).
+
+    Flat assignment a = t*K + k. For each expert e, its assignments in
+    ascending a (= ascending token t, since one token picks an expert once);
+    the first C are kept, the rest dropped.
+      counts[e]          raw number of assignments to e (sums to T*K)
+      offsets[E+1]       exclusive scan of kept counts min(counts, C)
+      perm_to_assign[p]  expert-major slot -> a   (first offsets[E] valid, rest -1)
+      assign_to_perm[a]  a -> expert-major slot, or -1 when dropped
+    """
+    ids = np.asarray(topk_ids_, dtype=np.int64).reshape(-1)
+    A = ids.size
+    if A and (ids.min() < 0 or ids.max() >= E):
+        raise ValueError("expert id out of range")
+    counts = np.zeros(E, dtype=np.int64)
+    kept = np.zeros(E, dtype=np.int64)
+    members = []
+    for e in range(E):
+        a_e = np.nonzero(ids == e)[0]  # ascending flat index
+        counts[e] = a_e.size
+        keep = a_e if C is None else a_e[:C]
+        kept[e] = keep.size
+        members.append(keep)
+    offsets = np.zeros(E + 1, dtype=np.int64)
+    for e in range(E):
+        offsets[e + 1] = offsets[e] + kept[e]
+    perm_to_assign = np.full(A, -1, dtype=np.int64)
+    assign_to_perm = np.full(A, -1, dtype=np.int64)
+    for e in range(E):
+        for r, a in enumerate(members[e]):
+            p = offsets[e] + r
+            perm_to_assign[p] = a
+            assign_to_perm[a] = p
+    return (counts.astype(np.int32), offsets.astype(np.int32),
+            assign_to_perm.astype(np.int32), perm_to_assign.astype(np.int32))
+
+
+def expert_of_slot(offsets, p: int) -> int:
+    """The expert that owns expert-major slot p (offsets[e] <= p < offsets[e+1])."""
+    off = np.asarray(offsets)
+    for e in range(off.size - 1):
+        if off[e] <= p < off[e + 1]:
+            return e
+    raise IndexError(p)
+
+
+def gather_rows(x, perm_to_assign, offsets, K: int) -> np.ndarray:
+    """[P5] 6.2 "pre-gather": X_perm[p] = x[token(p)] for the kept slots
+    (a pure data move, compared bit-exactly)."""
+    xa = np.asarray(x)
+    n_kept = int(np.asarray(offsets)[-1])
+    tok = np.asarray(perm_to_assign[:n_kept], dtype=np.int64) // K
+    return xa[tok]
+
+
+# --------------------------------------------------------------------------- experts
+def swiglu(g, u) -> np.ndarray:
+    """[P5] 3 item 4 (activation between the GEMMs, SwiGLU):
+    silu(g) * u with silu(g) = g / (1 + exp(-g))."""
+    g = as_f64(g)
+    return g / (1.0 + np.exp(-g)) * as_f64(u)
+
+
+def expert_ffn(x_rows, w_gate_e, w_up_e, w_down_e) -> np.ndarray:
+    """[P5] 3 items 3-5 for one expert: (SwiGLU(x W_gate, x W_up)) W_down, fp64."""
+    xr = as_f64(x_rows)
+    g = xr @ as_f64(w_gate_e)
+    u = xr @ as_f64(w_up_e)
+    return swiglu(g, u) @ as_f64(w_down_e)
+
+
+def grouped_ffn(x, perm_to_assign, offsets, K: int, w_gate, w_up, w_down):
+    """[P5] 3 items 3-5 and 6.2: for each expert e, the rows p in
+    [offsets[e], offsets[e+1]) hold token perm_to_assign[p] // K; both GEMMs
+    run on them. Returns (a_act, y_perm) in fp64 (no intermediate rounding)."""
+    off = np.asarray(offsets, dtype=np.int64)
+    E = off.size - 1
+    n_kept = int(off[-1])
+    xa = as_f64(x)
+    n = w_gate.shape[2]
+    d = w_down.shape[2]
+    a_act = np.zeros((n_kept, n), dtype=F64)
+    y_perm = np.zeros((n_kept, d), dtype=F64)
+    for e in range(E):
+        lo, hi = int(off[e]), int(off[e + 1])
+        if hi == lo:
+            continue
+        tok = np.asarray(perm_to_assign[lo:hi], dtype=np.int64) // K
+        xr = xa[tok]
+        g = xr @ as_f64(w_gate[e])
+        u = xr @ as_f64(w_up[e])
+        a_act[lo:hi] = swiglu(g, u)
+        y_perm[lo:hi] = a_act[lo:hi] @ as_f64(w_down[e])
+    return a_act, y_perm
+
+
+def combine(y_perm, assign_to_perm, topk_w, T: int, K: int) -> np.ndarray:
+    """[P5] 1 and 3 item 6: out[t] = sum_k w[t,k] * y[assign_to_perm[t*K+k]],
+    summed in k order; a dropped slot (-1) adds nothing and the other weights
+    are not rescaled. fp64."""
+    y = as_f64(y_perm)
+    a2p = np.asarray(assign_to_perm, dtype=np.int64).reshape(T, K)
+    w = as_f64(topk_w).reshape(T, K)
+    out = np.zeros((T, y.shape[1]), dtype=F64)
+    for k in range(K):
+        p = a2p[:, k]
+        keep = p >= 0
+        out[keep] += w[keep, k, None] * y[p[keep]]
+    return out
+
+
+# --------------------------------------------------------------------------- layer
+def forward(x, w_r, w_gate, w_up, w_down, K: int, capacity_factor: float = 0.0,
+            bias=None, logits=None, renormalize: bool = True):
+    """The whole layer forward ([P5] section 3 pipeline), every intermediate kept.
+
+    ``logits`` (fp32 [T, E]) replaces x . W_r + bias when given: this is how
+    ids/counts/permutation parity is checked on identical logits."""
+    T = x.shape[0]
+    lg = router_logits(x, w_r, bias) if logits is None else np.asarray(logits, np.float32)
+    E = lg.shape[1]
+    ids, w = route(lg, K, renormalize)
+    C = capacity(capacity_factor, T, K, E)
+    counts, offsets, a2p, p2a = permute(ids, E, C)
+    a_act, y_perm = grouped_ffn(x, p2a, offsets, K, w_gate, w_up, w_down)
+    out = combine(y_perm, a2p, w, T, K)
+    return dict(logits=lg, topk_ids=ids, topk_w=w, counts=counts, offsets=offsets,
+                assign_to_perm=a2p, perm_to_assign=p2a, a_act=a_act, y_perm=y_perm,
+                out=out, capacity=C)
+
+
+def forward_rows(tokens, x, w_gate, w_up, w_down, topk_ids_, topk_w_, assign_to_perm, K: int):
+    """Layer output for a few chosen tokens only (the sampled full-size check):
+    out[t] = sum over kept slots k of w[t,k] * FFN_{id[t,k]}(x[t]), in k order."""
+    tokens = np.asarray(tokens, dtype=np.int64)
+    ids = np.asarray(topk_ids_).reshape(-1, K)
+    w = as_f64(topk_w_).reshape(-1, K)
+    a2p = np.asarray(assign_to_perm).reshape(-1, K)
+    d = w_down.shape[2]
+    out = np.zeros((tokens.size, d), dtype=F64)
+    for i, t in enumerate(tokens):
+        xt = as_f64(x[int(t):int(t) + 1])
+        for k in range(K):
+            if a2p[t, k] < 0:
+                continue
+            e = int(ids[t, k])
+            out[i] += w[t, k] * expert_ffn(xt, w_gate[e], w_up[e], w_down[e])[0]
+    return out
+
+
+def dense_reference(x, w_gate, w_up, w_down, topk_ids_, topk_w_, E: int) -> np.ndarray:
+    """[P5] 1 read literally: y_t = sum over ALL E experts of gate_{t,e} * expert_e(x_t),
+    with gate_{t,e} the routed weight when e is among the token's top-K and 0
+    otherwise. No permutation or capacity (used with no capacity limit)."""
+    xa = as_f64(x)
+    T = xa.shape[0]
+    K = np.asarray(topk_ids_).shape[1]
+    gate = np.zeros((T, E), dtype=F64)
+    for t in range(T):
+        for k in range(K):
+            gate[t, int(topk_ids_[t, k])] = float(topk_w_[t, k])
+    out = np.zeros((T, w_down.shape[2]), dtype=F64)
+    for e in range(E):
+        out += gate[:, e:e + 1] * expert_ffn(xa, w_gate[e], w_up[e], w_down[e])
+    return out

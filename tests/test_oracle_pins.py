@@ -1,0 +1,377 @@
+"""Pins of the CPU oracle to facts fixed by the pages and by mathematics
+(worked examples, closed forms, invariants, library special cases, brute
+force), so that a plausible slip in the oracle fails at least one of them.
+CPU only."""
+import math
+import os
+
+import numpy as np
+import pytest
+import scipy.special
+import torch
+
+import moe_inputs as mi
+from oracle import moe_oracle as orc
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def _rand(seed, *shape):
+    return np.random.default_rng(seed).standard_normal(shape)
+
+
+# ----------------------------------------------------------------- router GEMM
+def test_router_logits_one_hot_rows_pick_rows_of_wr():
+    d, E = 7, 5  # d != E: a transposed operand cannot pass
+    w_r = _rand(1, d, E)
+    x = np.eye(d)
+    lg = orc.router_logits(x, w_r)
+    assert lg.shape == (d, E) and lg.dtype == np.float32
+    np.testing.assert_array_equal(lg, w_r.astype(np.float32))
+
+
+def test_router_logits_linear_and_bias():
+    x, w_r = _rand(2, 9, 6), _rand(3, 6, 4)
+    b = np.array([0.5, -1.0, 2.0, 0.0])
+    a = orc.router_logits(x, w_r).astype(np.float64)
+    ab = orc.router_logits(x, w_r, b).astype(np.float64)
+    np.testing.assert_allclose(ab - a, np.broadcast_to(b, a.shape), atol=1e-6)
+    two = orc.router_logits(2 * x, w_r).astype(np.float64)
+    np.testing.assert_allclose(two, 2 * a, rtol=1e-6, atol=1e-6)
+    # column sums for an all-ones token
+    ones = orc.router_logits(np.ones((1, 6)), w_r)[0]
+    np.testing.assert_allclose(ones, w_r.sum(axis=0), rtol=1e-6)
+
+
+# ----------------------------------------------------------------- top-k
+def _brute_topk(row, K):
+    # python's own stable sort on the (value desc, id asc) key
+    return sorted(range(len(row)), key=lambda e: (-float(row[e]), e))[:K]
+
+
+@pytest.mark.parametrize("seed", range(5))
+def test_topk_matches_brute_force(seed):
+    rng = np.random.default_rng(seed)
+    E = int(rng.integers(1, 20))
+    K = int(rng.integers(1, E + 1))
+    lg = rng.integers(-3, 4, size=(40, E)).astype(np.float32)  # many ties
+    ids = orc.topk_ids(lg, K)
+    for t in range(lg.shape[0]):
+        assert list(ids[t]) == _brute_topk(lg[t], K)
+
+
+def test_topk_all_equal_gives_lowest_ids():
+    ids = orc.topk_ids(np.zeros((3, 8), np.float32), 3)
+    np.testing.assert_array_equal(ids, np.tile([0, 1, 2], (3, 1)))
+
+
+def test_topk_signed_zero_is_a_tie():
+    lg = np.array([[-0.0, 0.0, -1.0, 0.0]], np.float32)
+    np.testing.assert_array_equal(orc.topk_ids(lg, 3), [[0, 1, 3]])
+
+
+def test_topk_k_equals_e_is_a_descending_sort():
+    lg = _rand(4, 6, 9).astype(np.float32)
+    ids = orc.topk_ids(lg, 9)
+    for t in range(6):
+        assert sorted(ids[t]) == list(range(9))
+        vals = lg[t, ids[t]]
+        assert np.all(np.diff(vals) <= 0)
+
+
+# ----------------------------------------------------------------- weights
+def test_weights_sum_to_one_renormalised():
+    lg = (3 * _rand(5, 100, 16)).astype(np.float32)
+    ids, w = orc.route(lg, 4)
+    assert np.all(np.abs(w.astype(np.float64).sum(1) - 1.0) <= 1e-6)
+    assert np.all(w > 0)
+    assert np.all(np.diff(w, axis=1) <= 0)  # descending with the logits
+
+
+def test_weights_k_equals_e_is_full_softmax():
+    lg = _rand(6, 20, 7).astype(np.float32)
+    ids, w = orc.route(lg, 7)
+    sm = scipy.special.softmax(lg.astype(np.float64), axis=1)
+    np.testing.assert_allclose(w, np.take_along_axis(sm, ids.astype(np.int64), 1), rtol=1e-6)
+
+
+def test_weights_not_renormalised_is_softmax_at_selected():
+    lg = _rand(7, 20, 10).astype(np.float32)
+    ids, w = orc.route(lg, 3, renormalize=False)
+    sm = scipy.special.softmax(lg.astype(np.float64), axis=1)
+    np.testing.assert_allclose(w, np.take_along_axis(sm, ids.astype(np.int64), 1), rtol=1e-6)
+    assert np.all(w.sum(1) < 1.0)
+
+
+def test_weights_k1_is_one_and_two_experts_is_logistic():
+    lg = _rand(8, 30, 5).astype(np.float32)
+    _, w1 = orc.route(lg, 1)
+    np.testing.assert_array_equal(w1, np.ones((30, 1), np.float32))
+    l2 = _rand(9, 30, 2).astype(np.float32)
+    ids, w = orc.route(l2, 2)
+    hi = np.take_along_axis(l2, ids[:, :1].astype(np.int64), 1)[:, 0].astype(np.float64)
+    lo = np.take_along_axis(l2, ids[:, 1:].astype(np.int64), 1)[:, 0].astype(np.float64)
+    np.testing.assert_allclose(w[:, 0], 1.0 / (1.0 + np.exp(lo - hi)), rtol=1e-6)
+
+
+# ----------------------------------------------------------------- capacity
+def test_capacity_values():
+    assert orc.capacity(1.25, 8192, 4, 32) == 1280  # the skewed workload
+    assert orc.capacity(0.0, 100, 2, 8) is None
+    assert orc.capacity(-1.0, 100, 2, 8) is None
+    assert orc.capacity(1.0, 10, 3, 4) == math.ceil(7.5)
+
+
+# ----------------------------------------------------------------- permutation
+def _read_golden():
+    routing, expert_tokens, sec = {}, {}, None
+    with open(os.path.join(GOLDEN, "omnimoe_expert_centric_example.txt")) as f:
+        for line in f:
+            line = line.strip()
+            if not line or line.startswith("#"):
+                continue
+            if line.startswith("["):
+                sec = line
+                continue
+            k, v = line.split(":")
+            vals = [int(s) for s in v.split()]
+            (routing if sec == "[routing]" else expert_tokens)[int(k)] = vals
+    return routing, expert_tokens
+
+
+def test_permutation_worked_example():
+    routing, printed = _read_golden()
+    T = len(routing)
+    K = len(routing[0])
+    uniq = sorted({e for v in routing.values() for e in v})
+    dense = {e: i for i, e in enumerate(uniq)}  # order-preserving remap to 0..E-1
+    ids = np.array([[dense[e] for e in routing[t]] for t in range(T)], np.int32)
+    counts, offsets, a2p, p2a = orc.permute(ids, len(uniq), None)
+    got = {}
+    for orig, e in dense.items():
+        lo, hi = offsets[e], offsets[e + 1]
+        got[orig] = [int(a) // K for a in p2a[lo:hi]]
+    for orig, toks in printed.items():
+        assert got[orig] == toks
+    for orig in set(uniq) - set(printed):
+        assert len(got[orig]) == 1
+    assert counts.sum() == T * K
+
+
+def _check_perm_invariants(ids, E, C):
+    T, K = ids.shape
+    counts, offsets, a2p, p2a = orc.permute(ids, E, C)
+    flat = ids.reshape(-1)
+    np.testing.assert_array_equal(counts, np.bincount(flat, minlength=E))
+    kept = counts if C is None else np.minimum(counts, C)
+    np.testing.assert_array_equal(offsets, np.concatenate([[0], np.cumsum(kept)]))
+    nk = offsets[-1]
+    # bijection between kept assignments and slots [0, nk)
+    assert np.all(p2a[nk:] == -1)
+    assert sorted(p2a[:nk]) == sorted(np.nonzero(a2p >= 0)[0])
+    np.testing.assert_array_equal(a2p[p2a[:nk]], np.arange(nk))
+    # expert ids non-decreasing along p; tokens strictly increasing in an expert
+    ex = flat[p2a[:nk]]
+    assert np.all(np.diff(ex) >= 0)
+    for e in range(E):
+        tok = p2a[offsets[e]:offsets[e + 1]] // K
+        assert np.all(np.diff(tok) > 0)
+        assert np.all(ex[offsets[e]:offsets[e + 1]] == e)
+        if C is not None:
+            dropped = [a // K for a in np.nonzero((flat == e) & (a2p < 0))[0]]
+            if len(tok) and dropped:
+                assert min(dropped) > tok.max()
+    return counts, offsets, a2p, p2a
+
+
+@pytest.mark.parametrize("seed", range(6))
+def test_permutation_invariants(seed):
+    rng = np.random.default_rng(100 + seed)
+    E = int(rng.integers(1, 12))
+    K = int(rng.integers(1, E + 1))
+    T = int(rng.integers(1, 60))
+    ids = np.stack([rng.permutation(E)[:K] for _ in range(T)]).astype(np.int32)
+    _check_perm_invariants(ids, E, None)
+    for C in (0, 1, 3, T):
+        _check_perm_invariants(ids, E, C)
+
+
+def test_permutation_is_the_stable_sort():
+    rng = np.random.default_rng(11)
+    E, K, T = 9, 3, 200
+    ids = np.stack([rng.permutation(E)[:K] for _ in range(T)]).astype(np.int32)
+    _, _, a2p, p2a = orc.permute(ids, E, None)
+    np.testing.assert_array_equal(p2a, np.argsort(ids.reshape(-1), kind="stable"))
+
+
+def test_capacity_large_enough_changes_nothing():
+    rng = np.random.default_rng(12)
+    E, K, T = 6, 2, 80
+    ids = np.stack([rng.permutation(E)[:K] for _ in range(T)]).astype(np.int32)
+    a = orc.permute(ids, E, None)
+    b = orc.permute(ids, E, int(np.bincount(ids.reshape(-1)).max()))
+    for u, v in zip(a, b):
+        np.testing.assert_array_equal(u, v)
+
+
+def test_capacity_drops_in_token_order_direct_rule():
+    rng = np.random.default_rng(13)
+    E, K, T, C = 5, 2, 50, 7
+    ids = np.stack([rng.permutation(E)[:K] for _ in range(T)]).astype(np.int32)
+    _, _, a2p, _ = orc.permute(ids, E, C)
+    seen = np.zeros(E, int)
+    for t in range(T):  # direct rule: an assignment survives iff fewer than C earlier tokens hold e
+        for k in range(K):
+            e = ids[t, k]
+            assert (a2p[t * K + k] >= 0) == (seen[e] < C)
+        for k in range(K):
+            seen[ids[t, k]] += 1
+
+
+def test_gather_rows_moves_token_rows():
+    rng = np.random.default_rng(14)
+    E, K, T = 4, 2, 10
+    ids = np.stack([rng.permutation(E)[:K] for _ in range(T)]).astype(np.int32)
+    x = np.arange(T * 3, dtype=np.float32).reshape(T, 3)
+    _, offsets, a2p, p2a = orc.permute(ids, E, None)
+    xp = orc.gather_rows(x, p2a, offsets, K)
+    for t in range(T):
+        for k in range(K):
+            np.testing.assert_array_equal(xp[a2p[t * K + k]], x[t])
+
+
+# ----------------------------------------------------------------- experts and layer
+def test_swiglu_is_torch_silu_times_up():
+    g, u = _rand(15, 50), _rand(16, 50)
+    ref = torch.nn.functional.silu(torch.from_numpy(g)) * torch.from_numpy(u)
+    np.testing.assert_allclose(orc.swiglu(g, u), ref.numpy(), rtol=1e-13, atol=1e-15)
+
+
+def test_single_expert_is_dense_swiglu_mlp():
+    T, d, n = 12, 8, 5  # d != n so a transposed weight cannot pass
+    x, wg, wu, wd = _rand(17, T, d), _rand(18, 1, d, n), _rand(19, 1, d, n), _rand(20, 1, n, d)
+    w_r = _rand(21, d, 1)
+    res = orc.forward(x, w_r, wg, wu, wd, K=1)
+    xt = torch.from_numpy(x)
+    ref = (torch.nn.functional.silu(xt @ torch.from_numpy(wg[0])) * (xt @ torch.from_numpy(wu[0]))
+           ) @ torch.from_numpy(wd[0])
+    np.testing.assert_allclose(res["out"], ref.numpy(), rtol=1e-12, atol=1e-12)
+
+
+@pytest.mark.parametrize("seed", range(4))
+def test_layer_equals_dense_sum_over_all_experts(seed):
+    rng = np.random.default_rng(200 + seed)
+    E = int(rng.integers(2, 7))
+    K = int(rng.integers(1, E + 1))
+    T, d, n = int(rng.integers(1, 24)), 6, 4
+    x, w_r = rng.standard_normal((T, d)), rng.standard_normal((d, E))
+    wg, wu = rng.standard_normal((E, d, n)), rng.standard_normal((E, d, n))
+    wd = rng.standard_normal((E, n, d))
+    res = orc.forward(x, w_r, wg, wu, wd, K=K)
+    dense = orc.dense_reference(x, wg, wu, wd, res["topk_ids"], res["topk_w"], E)
+    np.testing.assert_allclose(res["out"], dense, rtol=1e-12, atol=1e-12)
+    rows = orc.forward_rows(np.arange(T), x, wg, wu, wd, res["topk_ids"], res["topk_w"],
+                            res["assign_to_perm"], K)
+    np.testing.assert_allclose(rows, dense, rtol=1e-12, atol=1e-12)
+
+
+def test_layer_with_capacity_equals_dense_with_dropped_gates_zeroed():
+    rng = np.random.default_rng(300)
+    E, K, T, d, n = 4, 2, 30, 5, 3
+    x, w_r = rng.standard_normal((T, d)), rng.standard_normal((d, E))
+    w_r[:, 0] += 2.0  # skew toward expert 0 so it overflows
+    wg, wu = rng.standard_normal((E, d, n)), rng.standard_normal((E, d, n))
+    wd = rng.standard_normal((E, n, d))
+    cf = 0.5
+    res = orc.forward(x, w_r, wg, wu, wd, K=K, capacity_factor=cf)
+    C = orc.capacity(cf, T, K, E)
+    w = res["topk_w"].astype(np.float64).copy()
+    seen = np.zeros(E, int)
+    for t in range(T):
+        for k in range(K):
+            if seen[res["topk_ids"][t, k]] >= C:
+                w[t, k] = 0.0
+        for k in range(K):
+            seen[res["topk_ids"][t, k]] += 1
+    assert (w == 0).any()
+    dense = orc.dense_reference(x, wg, wu, wd, res["topk_ids"], w, E)
+    np.testing.assert_allclose(res["out"], dense, rtol=1e-12, atol=1e-12)
+
+
+def test_identity_experts_give_back_x():
+    """Dispatch/combine-only workload: identity experts, sum of weights 1 => out = x."""
+    cfg = mi.DISPATCH_COMBINE.with_T(64)
+    inp = mi.make_inputs(cfg)
+    x = orc.as_f64(inp.x)
+    ids, w = orc.route(inp.logits.numpy(), cfg.K)
+    _, offsets, a2p, p2a = orc.permute(ids, cfg.E, None)
+    xp = orc.gather_rows(x, p2a, offsets, cfg.K)
+    out = orc.combine(xp, a2p, w, cfg.T, cfg.K)
+    np.testing.assert_allclose(out, x, rtol=1e-6, atol=1e-6)
+
+
+def test_tiny_workload_forward_is_self_consistent():
+    cfg = mi.TINY_FP32
+    inp = mi.make_inputs(cfg)
+    res = orc.forward(inp.x.numpy(), inp.w_r.numpy(), inp.w_gate.numpy(), inp.w_up.numpy(),
+                      inp.w_down.numpy(), cfg.K)
+    assert res["counts"].sum() == cfg.T * cfg.K
+    dense = orc.dense_reference(inp.x.numpy(), inp.w_gate.numpy(), inp.w_up.numpy(),
+                                inp.w_down.numpy(), res["topk_ids"], res["topk_w"], cfg.E)
+    np.testing.assert_allclose(res["out"], dense, rtol=1e-12, atol=1e-12)
+
+
+def test_zipf_alpha_reaches_five_times_mean_load():
+    cfg = mi.SKEWED_CAPACITY_BF16
+    inp = mi.make_inputs(cfg, with_experts=False)
+    lg = orc.router_logits(inp.x, inp.w_r, inp.bias.numpy())
+    counts, _, _, _ = orc.permute(orc.topk_ids(lg, cfg.K), cfg.E, None)
+    ratio = counts.max() / (cfg.T * cfg.K / cfg.E)
+    assert abs(ratio - 5.0) <= 0.1
+    assert int(np.argmax(counts)) == 0
+
+
+# ----------------------------------------------------------------- planted mistakes
+def test_planted_mistakes_are_caught(monkeypatch):
+    """Mutate the oracle on the CPU and check that a pin above notices."""
+    rng = np.random.default_rng(400)
+    E, K, T, d, n = 4, 2, 9, 5, 3
+    x, w_r = rng.standard_normal((T, d)), rng.standard_normal((d, E))
+    wg, wu = rng.standard_normal((E, d, n)), rng.standard_normal((E, d, n))
+    wd = rng.standard_normal((E, n, d))
+
+    def dense_ok():
+        res = orc.forward(x, w_r, wg, wu, wd, K=K)
+        dense = orc.dense_reference(x, wg, wu, wd, res["topk_ids"], res["topk_w"], E)
+        return np.allclose(res["out"], dense, rtol=1e-12, atol=1e-12)
+
+    assert dense_ok()
+    real_combine = orc.combine
+
+    def combine_drops_last_slot(y, a2p, w, T_, K_):
+        a2p = np.asarray(a2p).reshape(T_, K_).copy()
+        a2p[:, -1] = -1
+        return real_combine(y, a2p.reshape(-1), w, T_, K_)
+
+    monkeypatch.setattr(orc, "combine", combine_drops_last_slot)
+    assert not dense_ok()
+    monkeypatch.undo()
+
+    real_permute = orc.permute
+
+    def permute_off_by_one(ids, E_, C_):
+        c, o, a2p, p2a = real_permute(ids, E_, C_)
+        nk = o[-1]
+        p2a = p2a.copy()
+        p2a[:nk] = np.roll(p2a[:nk], 1)
+        return c, o, a2p, p2a
+
+    monkeypatch.setattr(orc, "permute", permute_off_by_one)
+    assert not dense_ok()
+    monkeypatch.undo()
+
+    g, u = rng.standard_normal(20), rng.standard_normal(20)
+    wrong = g / (1.0 + np.exp(g)) * u  # sign slip inside silu
+    ref = (torch.nn.functional.silu(torch.from_numpy(g)) * torch.from_numpy(u)).numpy()
+    assert not np.allclose(wrong, ref)
+    assert np.allclose(orc.swiglu(g, u), ref)
