@@ -1,0 +1,384 @@
+"""Benchmark of the MoE-layer forward on B200.
+
+python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                [--workload mixtral_bf16]
+
+One step = one whole layer forward (route -> permute -> gate/up GEMM with fused gather and
+SwiGLU -> down GEMM -> combine) over one batch of seeded synthetic input, through
+moe_forward. Default workload: Mixtral-like, T=4096 d=4096 E=8 K=2 n=14336 bf16.
+For N > 1 (torchrun, one rank per GPU) every rank runs an independent replica: the layer
+shards by tokens with replicated weights and needs no collective; timing is the max over
+ranks and `value` counts the tokens of all ranks (weak scaling).
+
+--impl reference times the CPU oracle (numpy, fp64) as it stands on this host's cores, each
+step a bounded sample of the same workload (a few tokens through the whole layer); rank 0
+only.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import moe_inputs as mi  # noqa: E402
+
+METRIC = "MoE layer fwd tokens/s at 1 B200; dispatch+combine GB/s and GEMM % of peak"
+PEAKS_FILE = os.path.join(ROOT, "MEASURED_PEAKS.json")
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "traffic.json")
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=100)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="mixtral_bf16")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-tokens", type=int, default=8, help="tokens in the CPU oracle sample")
+    return ap.parse_args()
+
+
+# ------------------------------------------------------------------ distributed plumbing
+def dist_init(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        return rank, world, local  # rank 0 alone times the oracle; no process group
+    if world > 1:
+        import datetime
+        backend = "nccl" if args.impl == "ours" else "gloo"
+        if backend == "nccl":
+            torch.cuda.set_device(local)
+        torch.distributed.init_process_group(backend, timeout=datetime.timedelta(seconds=300))
+    elif args.impl == "ours":
+        torch.cuda.set_device(0)
+    return rank, world, local
+
+
+def barrier(world):
+    if world > 1:
+        torch.distributed.barrier()
+
+
+def max_over_ranks(v: float, world: int) -> float:
+    if world == 1:
+        return v
+    t = torch.tensor([v], dtype=torch.float64,
+                     device="cuda" if torch.distributed.get_backend() == "nccl" else "cpu")
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ------------------------------------------------------------------ measurement helpers
+def load_peaks():
+    if os.path.exists(PEAKS_FILE):
+        with open(PEAKS_FILE) as f:
+            p = json.load(f)
+        return p, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled during the timed region."""
+
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.Q}",
+                 "--format=csv,noheader,nounits", "-lms", "50"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            time.sleep(0.3)
+        except OSError:
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            time.sleep(0.1)
+            self.proc.terminate()
+            try:
+                self.out, _ = self.proc.communicate(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+                self.out, _ = self.proc.communicate()
+
+    def summary(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in (self.out or "").splitlines():
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                smax.append(float(f[2]))
+            except ValueError:
+                continue
+            for nm, v in zip(names, f[5:9]):
+                if v.lower() == "active":
+                    reasons.add(nm)
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(smax) if smax else None, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    for name in ("ffn_tc.cu", "common.cuh"):
+        with open(os.path.join(ROOT, "token_dispatch_router_b200", "csrc", name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def traffic_for(kernel: str, workload: str):
+    """ncu DRAM bytes per launch for `kernel`, if taken on the current kernel source."""
+    if not os.path.exists(TRAFFIC_FILE):
+        return None
+    with open(TRAFFIC_FILE) as f:
+        rec = json.load(f)
+    r = rec.get(workload, {}).get(kernel)
+    if not r or r.get("source_hash") != kernel_source_hash():
+        return None
+    return r.get("bytes_per_launch")
+
+
+# ------------------------------------------------------------------ CPU oracle leg
+def cpu_oracle_tokens_per_s(inp, n_tokens: int, start: int = 0, wide=None):
+    """The oracle on a bounded sample: n_tokens tokens through the whole layer (router
+    logits, softmax/top-k, counts/scan/permutation of the sample, expert FFNs, combine).
+    Expert weights are widened to fp64 once (outside the timing) in `wide`."""
+    from oracle import moe_oracle as orc
+    cfg = inp.cfg
+    if wide is None:
+        wide = {}
+    tok = (start + np.arange(n_tokens)) % cfg.T
+    x = orc.as_f64(inp.x[torch.from_numpy(tok)])
+    # widen the weights of the experts this sample uses, untimed
+    lg0 = orc.router_logits(x, inp.w_r, None if inp.bias is None else inp.bias.numpy())
+    for e in np.unique(orc.topk_ids(lg0, cfg.K)):
+        if int(e) not in wide:
+            wide[int(e)] = tuple(orc.as_f64(w[int(e)]) for w in (inp.w_gate, inp.w_up, inp.w_down))
+    t0 = time.perf_counter()
+    lg = orc.router_logits(x, inp.w_r, None if inp.bias is None else inp.bias.numpy())
+    ids, w = orc.route(lg, cfg.K)
+    C = orc.capacity(cfg.capacity_factor, n_tokens, cfg.K, cfg.E)
+    _, offsets, a2p, p2a = orc.permute(ids, cfg.E, C)
+    E = cfg.E
+    wg = [wide.get(e, (None,) * 3)[0] for e in range(E)]
+    wu = [wide.get(e, (None,) * 3)[1] for e in range(E)]
+    wd = [wide.get(e, (None,) * 3)[2] for e in range(E)]
+    off = np.asarray(offsets)
+    y = np.zeros((int(off[-1]), cfg.d))
+    for e in range(E):
+        lo, hi = int(off[e]), int(off[e + 1])
+        if hi > lo:
+            rows = x[np.asarray(p2a[lo:hi]) // cfg.K]
+            y[lo:hi] = orc.expert_ffn(rows, wg[e], wu[e], wd[e])
+    orc.combine(y, a2p, w, n_tokens, cfg.K)
+    dt = time.perf_counter() - t0
+    return n_tokens / dt, dt, wide
+
+
+def cpu_cores() -> int:
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:
+        return os.cpu_count() or 1
+
+
+# ------------------------------------------------------------------ reference arm
+def run_reference(args, rank, world):
+    if rank != 0:
+        return
+    cfg = mi.CONFIGS[args.workload]
+    inp = mi.make_inputs(cfg)
+    wide = {}
+    per_step = max(1, args.cpu_tokens // 4)
+    for i in range(args.warmup):
+        cpu_oracle_tokens_per_s(inp, per_step, start=i * per_step, wide=wide)
+    total_t, total_tok = 0.0, 0
+    for i in range(args.steps):
+        _, dt, wide = cpu_oracle_tokens_per_s(inp, per_step, start=(args.warmup + i) * per_step,
+                                              wide=wide)
+        total_t += dt
+        total_tok += per_step
+    value = total_tok / total_t
+    sample = f"{per_step} tokens per step through the whole layer (oracle, fp64)"
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1e3 * total_t / args.steps, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": cfg.name, "T": cfg.T, "d": cfg.d, "E": cfg.E, "K": cfg.K,
+                   "n": cfg.n},
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cpu_cores(),
+                         "kind": "oracle", "sample": sample},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+# ------------------------------------------------------------------ our arm
+def run_ours(args, rank, world, local):
+    import token_dispatch_router_b200 as tdr
+    tdr.load_library()  # fails loudly if the CUDA library is missing
+    cfg = mi.CONFIGS[args.workload]
+    dt = torch.bfloat16 if cfg.dtype == "bf16" else torch.float32
+    inp = mi.make_inputs(cfg)
+    dev = torch.device("cuda", torch.cuda.current_device())
+    x = inp.x.to(dev)
+    w_r = inp.w_r.to(dev)
+    wg, wu, wd = inp.w_gate.to(dev), inp.w_up.to(dev), inp.w_down.to(dev)
+    bias = None if inp.bias is None else inp.bias.to(dev)
+    s = tdr.make_shape(cfg.T, cfg.d, cfg.E, cfg.K, cfg.n, cfg.capacity_factor, True, dt)
+    ws = torch.empty(tdr.forward_workspace_size(s), dtype=torch.uint8, device=dev)
+    out = torch.empty(cfg.T, cfg.d, dtype=dt, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def step():
+        tdr.forward(s, x, w_r, wg, wu, wd, bias=bias, out=out, workspace=ws)
+
+    for _ in range(max(3, args.warmup)):
+        step()
+    torch.cuda.synchronize()
+    if tdr.device_status() != 0:
+        raise RuntimeError("device status set during warm-up")
+
+    # ---- timed region: K whole-layer steps, per-kernel events recorded by the library
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    launches0 = tdr.launch_count()
+    prof = tdr.Profiler()
+    with ClockSampler(local) as clocks:
+        barrier(world)
+        torch.cuda.synchronize()
+        with prof:
+            ev0.record(stream)
+            for _ in range(args.steps):
+                step()
+            ev1.record(stream)
+            torch.cuda.synchronize()
+        barrier(world)
+    launches = tdr.launch_count() - launches0
+    ms_total = ev0.elapsed_time(ev1)
+    ms_total = max_over_ranks(ms_total, world)
+    ms_step = ms_total / args.steps
+    value = cfg.T * world * args.steps / (ms_total / 1e3)
+    kern = prof.results()
+    if tdr.device_status() != 0:
+        raise RuntimeError("device status set during the timed region")
+
+    # ---- roofline of the dominant kernel (gate/up grouped GEMM, tensor cores)
+    v = tdr.workspace_views(s, ws)
+    a_kept = int(v["offsets"][cfg.E].item())
+    peaks, peak_src = load_peaks()
+    flops_gateup = 4.0 * cfg.d * cfg.n * a_kept
+    flops_down = 2.0 * cfg.d * cfg.n * a_kept
+    n_g, ms_g = kern.get("gateup_tc", (0, 0.0))
+    n_d, ms_d = kern.get("down_tc", (0, 0.0))
+    avg_g = ms_g / max(n_g, 1)
+    avg_d = ms_d / max(n_d, 1)
+    peak_t = float(peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"]))
+    ach_g = flops_gateup / (avg_g / 1e3) / 1e12 if avg_g > 0 else 0.0
+    ach_d = flops_down / (avg_d / 1e3) / 1e12 if avg_d > 0 else 0.0
+    ach_gemm = (flops_gateup + flops_down) / ((avg_g + avg_d) / 1e3) / 1e12 if avg_g > 0 else 0.0
+    roofline = {"bound": "tensor", "kernel": "gateup_tc", "achieved": round(ach_g, 2),
+                "peak": peak_t, "unit": "TFLOP/s", "frac": round(ach_g / peak_t, 4),
+                "traffic": traffic_for("gateup_tc", cfg.name),
+                "peak_source": f"{peak_src} bf16_tflops_sustained (kernel timed inside a long "
+                               "step loop)",
+                "algorithmic": "4*d*n*A_kept FLOP per launch (gate and up GEMMs)",
+                "avg_launch_ms": round(avg_g, 4)}
+
+    # ---- end to end through the public API with host buffers
+    x_host = inp.x.pin_memory()
+    out_host = torch.empty(cfg.T, cfg.d, dtype=dt).pin_memory()
+    e2e_steps = max(3, min(args.steps, 50))
+
+    def e2e_step():
+        x.copy_(x_host, non_blocking=True)
+        tdr.forward(s, x, w_r, wg, wu, wd, bias=bias, out=out, workspace=ws)
+        out_host.copy_(out, non_blocking=True)
+
+    for _ in range(2):
+        e2e_step()
+    torch.cuda.synchronize()
+    barrier(world)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1), world)
+    elem = 2 if dt == torch.bfloat16 else 4
+    e2e = {"value": cfg.T * world * e2e_steps / (e2e_ms / 1e3), "unit": "tokens/s",
+           "h2d_bytes_per_step": cfg.T * cfg.d * elem, "d2h_bytes_per_step": cfg.T * cfg.d * elem}
+
+    # ---- per-kernel breakdown (ms per step) and the two secondary figures of the metric
+    per_kernel = {k: round(ms / args.steps, 4) for k, (n, ms) in kern.items()}
+    gemm = {"achieved_tflops": round(ach_gemm, 2), "frac": round(ach_gemm / peak_t, 4),
+            "gateup_tflops": round(ach_g, 2), "down_tflops": round(ach_d, 2)}
+    result = {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16"
+        if dt == torch.bfloat16 else "f32", "data": "synthetic",
+        "config": {"workload": cfg.name, "T": cfg.T, "d": cfg.d, "E": cfg.E, "K": cfg.K,
+                   "n": cfg.n, "global_batch": cfg.T * world, "parallelism": f"replicas{world}",
+                   "l2": "inputs larger than L2: the 2.82 GB of expert weights stream every step"},
+        "roofline": roofline, "gemm": gemm, "kernel_ms_per_step": per_kernel,
+        "gpu_launches": int(launches), "e2e": e2e,
+    }
+    result["clocks"] = clocks.summary()
+
+    # ---- CPU oracle baseline (rank 0, N = 1 only)
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        v_cpu, dt_cpu, _ = cpu_oracle_tokens_per_s(inp, args.cpu_tokens)
+        result["cpu_baseline"] = {
+            "value": v_cpu, "unit": "tokens/s", "cores": cpu_cores(), "kind": "oracle",
+            "sample": f"{args.cpu_tokens} tokens through the whole layer (oracle numpy fp64, "
+                      f"{dt_cpu:.1f} s; expert weights widened to fp64 outside the timing)"}
+    if rank == 0:
+        print(json.dumps(result), flush=True)
+
+
+def main():
+    args = parse()
+    rank, world, local = dist_init(args)
+    try:
+        if args.impl == "reference":
+            run_reference(args, rank, world)
+        else:
+            run_ours(args, rank, world, local)
+    finally:
+        if world > 1 and torch.distributed.is_initialized():
+            torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

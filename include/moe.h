@@ -1,0 +1,230 @@
+/*
+ * moe.h - C ABI of the single-GPU MoE-layer forward for NVIDIA B200 (sm_100a).
+ *
+ * The layer (SonicMoE explainer, gitcode.csdn.net, sections 1 and 3):
+ *     y_t = sum over the token's top-K experts e of  w_{t,e} * FFN_e(x_t),
+ *     FFN_e(x) = (silu(x W_gate[e]) * (x W_up[e])) W_down[e],
+ * computed as router GEMM -> softmax -> top-K -> per-expert count + exclusive
+ * scan -> stable permutation into expert-major order -> grouped gate/up GEMM
+ * with the token gather fused into the operand load and SwiGLU in the epilogue
+ * -> grouped down GEMM -> weighted combine back to token order.
+ *
+ * Conventions shared by every entry point:
+ *  - Ownership: the caller allocates and owns every buffer. Pointers named
+ *    "device" must be device-accessible memory of the current CUDA device; the
+ *    library never allocates, frees or synchronises, except moe_get_device_status
+ *    and the profiling queries, which synchronise.
+ *  - Layout: every tensor is dense row-major. Indices are int32.
+ *  - Dtypes: MOE_F32 - x, weights, outputs and intermediates are fp32.
+ *    MOE_BF16 - x, W_r, W_gate, W_up, W_down, x_perm, a_act, y_perm and out are
+ *    bf16; logits, bias and top-k weights are fp32; all sums accumulate in fp32.
+ *  - Asynchrony: work is enqueued on `stream` (a cudaStream_t; NULL = legacy
+ *    default stream) and returns at once.
+ *  - Errors: argument errors (null required pointer, bad sizes, unsupported
+ *    shape, short workspace) are returned synchronously and nothing is
+ *    enqueued. A launch failure returns MOE_ERR_CUDA. Faults found on the
+ *    device (an expert id out of range, a bounded wait that ran out) set a
+ *    device status word that moe_get_device_status() reads and clears.
+ *  - Thread safety: calls are reentrant; the only global state is the device
+ *    status word, a per-device cache of SM counts and the opt-in profiler.
+ */
+#ifndef MOE_B200_H
+#define MOE_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st* moe_stream_t; /* same handle as cudaStream_t */
+
+typedef enum {
+  MOE_OK = 0,
+  MOE_ERR_INVALID_ARG = 1, /* null pointer, bad size, K > E, ...          */
+  MOE_ERR_UNSUPPORTED = 2, /* valid but not implemented (e.g. E > 256)      */
+  MOE_ERR_CUDA = 3,        /* a CUDA runtime/driver call failed            */
+  MOE_ERR_WORKSPACE = 4,   /* workspace missing or smaller than required   */
+  MOE_ERR_TIMEOUT = 5,     /* device: a bounded wait ran out               */
+  MOE_ERR_DEVICE_INDEX = 6 /* device: an index read was out of range       */
+} moe_status;
+
+typedef enum { MOE_F32 = 0, MOE_BF16 = 1 } moe_dtype;
+
+/* Problem size. T tokens of width d, E experts, top-K per token, expert
+ * intermediate width n. capacity_factor <= 0 means no limit; otherwise each
+ * expert keeps at most C = ceil(capacity_factor * T * K / E) assignments,
+ * the first C in token order ("Operators & compilers: MoE routing and sparse
+ * kernels", section 4: capacity factor bounds the tokens per expert, the
+ * overflow is dropped). renormalize != 0: top-K weights are the softmax
+ * restricted to the K selected experts (they sum to 1); 0: plain softmax
+ * over all E experts, read at the selected ones. Limits: 1 <= K <= E <= 256,
+ * K <= 32, T >= 0. MOE_BF16 also needs d % 64 == 0 and n % 64 == 0 (TMA
+ * tiles); MOE_F32 needs d % 4 == 0 and n % 4 == 0. */
+typedef struct {
+  int32_t T, d, E, K, n;
+  float capacity_factor;
+  int32_t renormalize;
+  int32_t dtype; /* moe_dtype */
+} moe_shape;
+
+/* ----------------------------------------------------------------------------
+ * Workspace sizes (bytes). The caller passes a device buffer at least this big
+ * (256-byte aligned) to moe_permute / moe_forward. Returns 0 on a bad shape.
+ * moe_permute_workspace_size: scratch of the histogram / scan / scatter
+ *   kernels (per-chunk expert counts and rank bases).
+ * moe_forward_workspace_size: everything moe_forward keeps between kernels:
+ *   logits, top-K ids and weights, counts, offsets, both permutation indices,
+ *   the permute scratch, a_act[T*K, n] and y_perm[T*K, d].
+ */
+size_t moe_permute_workspace_size(const moe_shape* shape);
+size_t moe_forward_workspace_size(const moe_shape* shape);
+
+/* ----------------------------------------------------------------------------
+ * moe_route - router logits, softmax and top-K.
+ * "Two upstream innovations of MoE: Routing-Free and OmniMoE"
+ * (chatdocs.ruinique.com), section 1.1: x -> Router(x) -> Softmax -> TopK;
+ * "How AI chips support MoE", chapter 4, sections 4.2-4.3: the gate is a
+ * small dense linear map followed by softmax and a top-K selection.
+ *
+ *   x          [T, d]  device, dtype; ignored when logits_in != NULL
+ *   w_r        [d, E]  device, dtype; ignored when logits_in != NULL
+ *   bias       [E]     device fp32 or NULL; added to every token's logits
+ *   logits_in  [T, E]  device fp32 or NULL: use these logits instead of x W_r
+ *   logits_out [T, E]  device fp32 or NULL: receives the logits the top-K saw
+ *                      (x W_r + bias, or a copy of logits_in)
+ *   topk_ids   [T, K]  device int32 out: slot 0 = largest logit; ties go to
+ *                      the lower expert id (+0 and -0 are equal)
+ *   topk_w     [T, K]  device fp32 out: weights (see renormalize)
+ * Selection compares the fp32 logits; NaN logits give unspecified ids.
+ */
+moe_status moe_route(const moe_shape* shape, const void* x, const void* w_r, const float* bias,
+                     const float* logits_in, float* logits_out, int32_t* topk_ids,
+                     float* topk_w, moe_stream_t stream);
+
+/* ----------------------------------------------------------------------------
+ * moe_permute - per-expert counts, exclusive scan and the stable permutation.
+ * "Operators & compilers: MoE routing and sparse kernels"
+ * (charles2530.github.io), section 3: regrouping tokens by expert is an
+ * index/scatter/gather problem solved with counting and a prefix sum;
+ * "Two upstream innovations of MoE: Routing-Free and OmniMoE", section 2.3:
+ * the (token, expert) tasks sorted by (expert, token);
+ * SonicMoE explainer, section 11: the expert-major metadata.
+ * Atomic-free and deterministic: flat assignment a = t*K + k; inside an expert
+ * the assignments keep ascending a (= token) order.
+ *
+ *   topk_ids        [T, K]   device int32 in, each in [0, E) (an id out of range
+ *                            is skipped and flags MOE_ERR_DEVICE_INDEX)
+ *   counts          [E]      device int32 out: raw assignments per expert
+ *   offsets         [E + 1]  device int32 out: exclusive scan of min(counts, C);
+ *                            offsets[E] = kept assignments
+ *   assign_to_perm  [T * K]  device int32 out: a -> expert-major slot, -1 if dropped
+ *   perm_to_assign  [T * K]  device int32 out: slot -> a for slots < offsets[E];
+ *                            the tail is left unwritten
+ *   x               [T, d]   device dtype or NULL  \ both non-NULL: also write the
+ *   x_perm          [T*K, d] device dtype or NULL  / gathered rows x_perm[p] =
+ *                            x[perm_to_assign[p] / K] for p < offsets[E]
+ *   workspace, ws_bytes      >= moe_permute_workspace_size(shape)
+ */
+moe_status moe_permute(const moe_shape* shape, const int32_t* topk_ids, int32_t* counts,
+                       int32_t* offsets, int32_t* assign_to_perm, int32_t* perm_to_assign,
+                       const void* x, void* x_perm, void* workspace, size_t ws_bytes,
+                       moe_stream_t stream);
+
+/* ----------------------------------------------------------------------------
+ * moe_grouped_ffn - the grouped SwiGLU expert FFN on the expert-major rows.
+ * SonicMoE explainer, section 3 items 3-5 (grouped GEMM with a different M
+ * per expert, SwiGLU, second grouped GEMM), section 6.2 (the gather of x is
+ * fused into the GEMM's operand load: no [T*K, d] gathered copy of x is made)
+ * and section 6.3 (SwiGLU runs in the epilogue while the accumulator is on chip).
+ * For expert e, rows p in [offsets[e], offsets[e+1]) hold token
+ * t = perm_to_assign[p] / K:
+ *     a_act[p]  = silu(x[t] W_gate[e]) * (x[t] W_up[e])     (n wide)
+ *     y_perm[p] = a_act[p] W_down[e]                        (d wide)
+ *
+ *   x               [T, d]      device dtype
+ *   offsets         [E + 1]     device int32 (from moe_permute)
+ *   perm_to_assign  [T * K]     device int32 (from moe_permute)
+ *   w_gate, w_up    [E, d, n]   device dtype
+ *   w_down          [E, n, d]   device dtype
+ *   a_act           [T * K, n]  device dtype out (rows >= offsets[E] unwritten)
+ *   y_perm          [T * K, d]  device dtype out (rows >= offsets[E] unwritten)
+ * MOE_BF16 runs on the tcgen05 tensor cores (fp32 accumulation in TMEM);
+ * MOE_F32 runs an fp32 FMA path.
+ */
+moe_status moe_grouped_ffn(const moe_shape* shape, const void* x, const int32_t* offsets,
+                           const int32_t* perm_to_assign, const void* w_gate, const void* w_up,
+                           const void* w_down, void* a_act, void* y_perm, moe_stream_t stream);
+
+/* ----------------------------------------------------------------------------
+ * moe_combine - weighted scatter-combine back to token order.
+ * SonicMoE explainer, section 3 item 6 (scatter/combine to token-major) and
+ * section 6.1 (the aggregation fuses the scatter and the weighted sum).
+ *     out[t] = sum_{k=0..K-1, assign_to_perm[t*K+k] >= 0} topk_w[t,k] * y_perm[assign_to_perm[t*K+k]]
+ * summed in fp32 in k order (deterministic); dropped slots add nothing and the
+ * remaining weights are not rescaled; a token with every slot dropped gets 0.
+ *
+ *   y_perm          [T * K, d]  device dtype
+ *   assign_to_perm  [T * K]     device int32 (values >= T*K flag MOE_ERR_DEVICE_INDEX)
+ *   topk_w          [T, K]      device fp32
+ *   out             [T, d]      device dtype out
+ */
+moe_status moe_combine(const moe_shape* shape, const void* y_perm, const int32_t* assign_to_perm,
+                       const float* topk_w, void* out, moe_stream_t stream);
+
+/* ----------------------------------------------------------------------------
+ * moe_forward - the whole layer: moe_route, moe_permute (no x_perm),
+ * moe_grouped_ffn and moe_combine chained on `stream` with no host sync.
+ *
+ *   x [T, d], w_r [d, E], bias [E] or NULL, logits_in [T, E] or NULL,
+ *   w_gate/w_up [E, d, n], w_down [E, n, d]: as above
+ *   out        [T, d]  device dtype out
+ *   workspace, ws_bytes >= moe_forward_workspace_size(shape)
+ *   layout of the workspace (byte offsets from moe_forward_workspace_layout)
+ *   lets a caller read the intermediates after the call.
+ */
+moe_status moe_forward(const moe_shape* shape, const void* x, const void* w_r, const float* bias,
+                       const float* logits_in, const void* w_gate, const void* w_up,
+                       const void* w_down, void* out, void* workspace, size_t ws_bytes,
+                       moe_stream_t stream);
+
+/* Byte offsets of the intermediates inside moe_forward's workspace. */
+typedef struct {
+  size_t logits, topk_ids, topk_w, counts, offsets, assign_to_perm, perm_to_assign,
+      permute_scratch, a_act, y_perm, total;
+} moe_workspace_layout;
+moe_status moe_forward_workspace_layout(const moe_shape* shape, moe_workspace_layout* layout);
+
+/* ----------------------------------------------------------------------------
+ * Device status: synchronises `stream`, returns the first device-side fault
+ * recorded since the last call (MOE_OK if none) and clears it.
+ */
+moe_status moe_get_device_status(moe_stream_t stream);
+const char* moe_status_string(moe_status status);
+
+/* ----------------------------------------------------------------------------
+ * Opt-in per-kernel timing (host state, not thread safe). While enabled,
+ * every kernel launch the library makes is bracketed by CUDA events on its
+ * stream. moe_profile_query synchronises on the recorded events and returns,
+ * for kernel `id` in [0, moe_kernel_count()), its launch count and total
+ * device milliseconds since the last reset; moe_kernel_name names it.
+ * moe_launch_count counts every kernel launch made by the library (always on).
+ */
+moe_status moe_profile_enable(int on);
+moe_status moe_profile_reset(void);
+int moe_kernel_count(void);
+const char* moe_kernel_name(int id);
+moe_status moe_profile_query(int id, int64_t* launches, double* total_ms);
+int64_t moe_launch_count(void);
+
+/* Test hook for the failure-detection path: launches one block that waits on
+ * an mbarrier nothing will complete, bounded by `limit_ns` nanoseconds, then
+ * records MOE_ERR_TIMEOUT in the device status word and returns (no trap, no
+ * hang). Read the result with moe_get_device_status. */
+moe_status moe_selftest_timeout(uint64_t limit_ns, moe_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* MOE_B200_H */

@@ -253,20 +253,28 @@ def forward(x, w_r, w_gate, w_up, w_down, K: int, capacity_factor: float = 0.0,
 
 def forward_rows(tokens, x, w_gate, w_up, w_down, topk_ids_, topk_w_, assign_to_perm, K: int):
     """Layer output for a few chosen tokens only (the sampled full-size check):
-    out[t] = sum over kept slots k of w[t,k] * FFN_{id[t,k]}(x[t]), in k order."""
+    out[t] = sum over kept slots k of w[t,k] * FFN_{id[t,k]}(x[t]), summed in k order.
+    Each expert's FFN runs once on all chosen tokens routed to it, so its weights are
+    widened to fp64 once."""
     tokens = np.asarray(tokens, dtype=np.int64)
     ids = np.asarray(topk_ids_).reshape(-1, K)
     w = as_f64(topk_w_).reshape(-1, K)
     a2p = np.asarray(assign_to_perm).reshape(-1, K)
     d = w_down.shape[2]
-    out = np.zeros((tokens.size, d), dtype=F64)
+    per_slot = np.zeros((tokens.size, K, d), dtype=F64)
+    pairs = {}
     for i, t in enumerate(tokens):
-        xt = as_f64(x[int(t):int(t) + 1])
         for k in range(K):
-            if a2p[t, k] < 0:
-                continue
-            e = int(ids[t, k])
-            out[i] += w[t, k] * expert_ffn(xt, w_gate[e], w_up[e], w_down[e])[0]
+            if a2p[t, k] >= 0:
+                pairs.setdefault(int(ids[t, k]), []).append((i, k))
+    for e, lst in pairs.items():
+        rows = np.array([tokens[i] for i, _ in lst], dtype=np.int64)
+        y = expert_ffn(as_f64(x[rows]), w_gate[e], w_up[e], w_down[e])
+        for j, (i, k) in enumerate(lst):
+            per_slot[i, k] = w[tokens[i], k] * y[j]
+    out = np.zeros((tokens.size, d), dtype=F64)
+    for k in range(K):
+        out += per_slot[:, k]
     return out
 
 

@@ -1,0 +1,374 @@
+"""GPU parity: every stage of the CUDA path, called through the C ABI, against the
+CPU oracle on the same seeded inputs.
+
+Bars (stated by the workloads): top-k ids, counts, offsets and both permutation maps
+bit-exact given identical router logits (the oracle routes on the logits the GPU
+produced); top-k weights within 1e-6; layer output max abs error <= 1e-4 for fp32
+shapes; for bf16 shapes max|err| / max|ref| <= 2e-2 and ||err|| / ||ref|| <= 2e-2.
+Pure data moves (the materialised gather) are bit-exact."""
+import numpy as np
+import pytest
+import torch
+
+import moe_inputs as mi
+from oracle import moe_oracle as orc
+
+pytestmark = pytest.mark.gpu
+
+BF16_REL = 2e-2
+F32_ABS = 1e-4
+W_ABS = 1e-6
+
+
+# ------------------------------------------------------------------ helpers
+def cuda(t):
+    return None if t is None else t.cuda()
+
+
+def shape_of(cfg, tdr, T=None):
+    dt = torch.bfloat16 if cfg.dtype == "bf16" else torch.float32
+    return tdr.make_shape(cfg.T if T is None else T, cfg.d, cfg.E, cfg.K, cfg.n,
+                          cfg.capacity_factor, True, dt)
+
+
+def assert_status_ok(tdr):
+    assert tdr.device_status() == 0
+
+
+def rel_errors(got, ref):
+    got = np.asarray(got, np.float64)
+    ref = np.asarray(ref, np.float64)
+    diff = got - ref
+    scale = max(np.abs(ref).max(), 1e-30)
+    l2 = np.linalg.norm(diff) / max(np.linalg.norm(ref), 1e-30)
+    return np.abs(diff).max() / scale, l2
+
+
+def assert_bf16_close(got, ref, what):
+    mx, l2 = rel_errors(got, ref)
+    assert mx <= BF16_REL and l2 <= BF16_REL, f"{what}: max-rel {mx:.3e} l2-rel {l2:.3e}"
+
+
+def check_routing(tdr, logits_gpu, ids_gpu, w_gpu, K, renorm=True):
+    lg = logits_gpu.cpu().numpy()
+    ids_ref, w_ref = orc.route(lg, K, renorm)
+    np.testing.assert_array_equal(ids_gpu.cpu().numpy(), ids_ref)
+    assert np.abs(w_gpu.cpu().numpy().astype(np.float64) - w_ref).max() <= W_ABS
+    return ids_ref, w_ref
+
+
+def check_permutation(perm, ids, E, C):
+    counts, offsets, a2p, p2a = orc.permute(ids, E, C)
+    np.testing.assert_array_equal(perm["counts"].cpu().numpy(), counts)
+    np.testing.assert_array_equal(perm["offsets"].cpu().numpy(), offsets)
+    np.testing.assert_array_equal(perm["assign_to_perm"].cpu().numpy(), a2p)
+    nk = int(offsets[-1])
+    np.testing.assert_array_equal(perm["perm_to_assign"].cpu().numpy()[:nk], p2a[:nk])
+    return counts, offsets, a2p, p2a
+
+
+_INPUTS = {}
+
+
+def inputs_for(cfg):
+    if cfg.name not in _INPUTS:
+        _INPUTS.clear()  # keep one large workload in host memory at a time
+        _INPUTS[cfg.name] = mi.make_inputs(cfg)
+    return _INPUTS[cfg.name]
+
+
+# ------------------------------------------------------------------ failure detection
+def test_bounded_wait_times_out_and_reports(cuda_lib):
+    tdr = cuda_lib
+    assert tdr.device_status() == 0
+    assert tdr.selftest_timeout(2_000_000) == 5  # 2 ms limit, nothing completes the barrier
+    assert tdr.device_status() == 0  # cleared by the read
+    x = torch.ones(4, device="cuda")
+    assert float(x.sum()) == 4.0  # the context is still usable
+
+
+# ------------------------------------------------------------------ route
+@pytest.mark.parametrize("T,d,E,K,dtype,bias,renorm", [
+    (256, 128, 8, 2, "f32", False, True),      # the tiny workload's router
+    (300, 4096, 8, 2, "bf16", False, True),
+    (257, 2048, 128, 8, "bf16", False, True),
+    (500, 2880, 32, 4, "bf16", True, True),
+    (100, 128, 256, 32, "bf16", False, True),
+    (33, 64, 6, 3, "f32", False, False),
+    (1, 64, 1, 1, "bf16", False, True),
+    (129, 192, 64, 6, "bf16", True, False),
+])
+def test_route_matches_oracle(cuda_lib, T, d, E, K, dtype, bias, renorm):
+    tdr = cuda_lib
+    cfg = mi.MoEConfig("route", T=T, d=d, E=E, K=K, n=64, dtype=dtype, seed=T + E)
+    inp = mi.make_inputs(cfg, with_experts=False)
+    b = mi.zipf_bias(E, 1.2, 1.75) if bias else None
+    s = tdr.make_shape(T, d, E, K, 64, 0.0, renorm,
+                       torch.bfloat16 if dtype == "bf16" else torch.float32)
+    lo = torch.empty(T, E, dtype=torch.float32, device="cuda")
+    ids, w, _ = tdr.route(s, cuda(inp.x), cuda(inp.w_r), bias=cuda(b), logits_out=lo)
+    ref_lg = orc.router_logits(inp.x, inp.w_r, None if b is None else b.numpy())
+    np.testing.assert_allclose(lo.cpu().numpy(), ref_lg, rtol=1e-4, atol=2e-4)
+    check_routing(tdr, lo, ids, w, K, renorm)
+    assert_status_ok(tdr)
+
+
+def test_route_ties_go_to_lower_id(cuda_lib):
+    tdr = cuda_lib
+    g = np.random.default_rng(5)
+    T, E, K = 777, 64, 6
+    lg = g.integers(-2, 3, size=(T, E)).astype(np.float32)  # heavy ties
+    lg[0] = 0.0
+    lg[1, ::2] = -0.0  # signed zeros tie with +0
+    s = tdr.make_shape(T, 64, E, K, 64, 0.0, True, torch.bfloat16)
+    ids, w, lo = tdr.route(s, logits_in=torch.from_numpy(lg).cuda(),
+                           logits_out=torch.empty(T, E, device="cuda"))
+    np.testing.assert_array_equal(lo.cpu().numpy(), lg)
+    ids_ref, _ = check_routing(tdr, lo, ids, w, K)
+    np.testing.assert_array_equal(ids_ref[0], np.arange(K))
+    assert_status_ok(tdr)
+
+
+@pytest.mark.parametrize("T", mi.DISPATCH_COMBINE_T)
+def test_route_given_logits_sweep(cuda_lib, T):
+    tdr = cuda_lib
+    cfg = mi.DISPATCH_COMBINE.with_T(T)
+    inp = mi.make_inputs(cfg)
+    s = shape_of(cfg, tdr)
+    ids, w, _ = tdr.route(s, logits_in=cuda(inp.logits))
+    check_routing(tdr, inp.logits, ids, w, cfg.K)
+    assert_status_ok(tdr)
+
+
+# ------------------------------------------------------------------ permute
+def _random_ids(rng, T, E, K, skew=0.0):
+    if T == 0:
+        return np.zeros((0, K), np.int32)
+    scores = rng.standard_normal((T, E)) + skew * (np.arange(E)[None, :] == 0)
+    return np.argsort(-scores, axis=1, kind="stable")[:, :K].astype(np.int32)
+
+
+@pytest.mark.parametrize("T,E,K,cf,skew", [
+    (1, 1, 1, 0.0, 0.0),
+    (37, 8, 2, 0.0, 0.0),
+    (4095, 8, 2, 0.0, 0.0),
+    (5000, 64, 6, 0.0, 0.0),
+    (16384, 128, 8, 0.0, 0.0),
+    (8192, 32, 4, 1.25, 3.0),
+    (3001, 256, 32, 0.5, 0.0),
+    (700, 16, 4, 0.3, 5.0),
+    (65536, 64, 6, 0.0, 0.0),
+])
+def test_permute_matches_oracle(cuda_lib, T, E, K, cf, skew):
+    tdr = cuda_lib
+    rng = np.random.default_rng(T * 31 + E)
+    ids = _random_ids(rng, T, E, K, skew)
+    s = tdr.make_shape(T, 64, E, K, 64, cf, True, torch.bfloat16)
+    perm = tdr.permute(s, torch.from_numpy(ids).cuda())
+    check_permutation(perm, ids, E, orc.capacity(cf, T, K, E))
+    assert_status_ok(tdr)
+
+
+def test_permute_materialised_gather_is_exact(cuda_lib):
+    tdr = cuda_lib
+    rng = np.random.default_rng(9)
+    T, E, K, d = 1234, 16, 3, 256
+    ids = _random_ids(rng, T, E, K, 1.0)
+    x = torch.randn(T, d).to(torch.bfloat16)
+    s = tdr.make_shape(T, d, E, K, 64, 0.9, True, torch.bfloat16)
+    perm = tdr.permute(s, torch.from_numpy(ids).cuda(), x=x.cuda(), materialize=True)
+    _, offsets, _, p2a = check_permutation(perm, ids, E, orc.capacity(0.9, T, K, E))
+    nk = int(offsets[-1])
+    ref = orc.gather_rows(x.float().numpy(), p2a, offsets, K)
+    np.testing.assert_array_equal(perm["x_perm"][:nk].float().cpu().numpy(), ref)
+    assert_status_ok(tdr)
+
+
+def test_permute_flags_out_of_range_ids(cuda_lib):
+    tdr = cuda_lib
+    T, E, K = 100, 8, 2
+    ids = np.tile(np.array([[0, 1]], np.int32), (T, 1))
+    ids[7, 1] = E  # out of range: skipped and reported, never used as an index
+    s = tdr.make_shape(T, 64, E, K, 64, 0.0, True, torch.bfloat16)
+    perm = tdr.permute(s, torch.from_numpy(ids).cuda())
+    assert tdr.device_status() == 6
+    a2p = perm["assign_to_perm"].cpu().numpy()
+    assert a2p[7 * K + 1] == -1
+    assert int(perm["counts"].cpu().sum()) == T * K - 1
+
+
+# ------------------------------------------------------------------ combine
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_combine_matches_oracle(cuda_lib, dtype):
+    tdr = cuda_lib
+    rng = np.random.default_rng(21)
+    T, E, K, d = 999, 16, 4, 192
+    ids = _random_ids(rng, T, E, K, 2.0)
+    C = orc.capacity(0.8, T, K, E)
+    _, offsets, a2p, _ = orc.permute(ids, E, C)
+    w = rng.random((T, K)).astype(np.float32)
+    tdt = torch.bfloat16 if dtype == "bf16" else torch.float32
+    y = torch.randn(T * K, d).to(tdt)
+    s = tdr.make_shape(T, d, E, K, 64, 0.8, True, tdt)
+    out = tdr.combine(s, y.cuda(), torch.from_numpy(a2p).cuda(), torch.from_numpy(w).cuda())
+    ref = orc.combine(y.float().numpy(), a2p, w, T, K)
+    got = out.float().cpu().numpy()
+    if dtype == "f32":
+        np.testing.assert_allclose(got, ref, rtol=1e-5, atol=1e-5)
+    else:  # fp32 sum rounded once to bf16: within half a bf16 ulp plus fp32 rounding
+        np.testing.assert_allclose(got, ref, rtol=2 ** -8, atol=1e-6)
+    assert_status_ok(tdr)
+
+
+# ------------------------------------------------------------------ grouped FFN
+def _ffn_case(tdr, T, d, n, E, K, cf, dtype, seed):
+    cfg = mi.MoEConfig("ffn", T=T, d=d, E=E, K=K, n=n, dtype=dtype, capacity_factor=cf,
+                       seed=seed)
+    inp = mi.make_inputs(cfg)
+    s = shape_of(cfg, tdr)
+    lo = torch.empty(T, E, dtype=torch.float32, device="cuda")
+    ids, w, _ = tdr.route(s, cuda(inp.x), cuda(inp.w_r), logits_out=lo)
+    perm = tdr.permute(s, ids)
+    a_act, y_perm = tdr.grouped_ffn(s, cuda(inp.x), perm["offsets"], perm["perm_to_assign"],
+                                    cuda(inp.w_gate), cuda(inp.w_up), cuda(inp.w_down))
+    out = tdr.combine(s, y_perm, perm["assign_to_perm"], w)
+    ids_ref, w_ref = check_routing(tdr, lo, ids, w, K)
+    _, offsets, a2p, p2a = check_permutation(perm, ids_ref, E, orc.capacity(cf, T, K, E))
+    a_ref, y_ref = orc.grouped_ffn(inp.x, p2a, offsets, K, inp.w_gate, inp.w_up, inp.w_down)
+    out_ref = orc.combine(y_ref, a2p, w_ref, T, K)
+    nk = int(offsets[-1])
+    return (a_act[:nk].float().cpu().numpy(), a_ref, y_perm[:nk].float().cpu().numpy(), y_ref,
+            out.float().cpu().numpy(), out_ref)
+
+
+def test_grouped_ffn_fp32_tiny_workload(cuda_lib):
+    tdr = cuda_lib
+    c = mi.TINY_FP32
+    a, a_ref, y, y_ref, out, out_ref = _ffn_case(tdr, c.T, c.d, c.n, c.E, c.K, 0.0, "f32", 0)
+    assert np.abs(a - a_ref).max() <= 1e-5
+    assert np.abs(y - y_ref).max() <= F32_ABS
+    assert np.abs(out - out_ref).max() <= F32_ABS
+    assert_status_ok(tdr)
+
+
+@pytest.mark.parametrize("T,d,n,E,K,cf", [
+    (300, 256, 384, 4, 2, 0.0),     # gate/up tail tile of 128 columns (n = 3 x 128)
+    (1000, 512, 192, 16, 4, 1.1),   # n = 192: last gate/up tile half valid; capacity drops
+    (64, 128, 128, 8, 8, 0.0),      # K = E; down tile wider than d
+    (2500, 320, 256, 3, 1, 0.0),    # d = 320: down tile 256 + ragged 64
+    (129, 64, 64, 1, 1, 0.0),       # one expert; one k-block; 2 M-tiles, the last has 1 row
+])
+def test_grouped_ffn_bf16_tensor_cores(cuda_lib, T, d, n, E, K, cf):
+    tdr = cuda_lib
+    a, a_ref, y, y_ref, out, out_ref = _ffn_case(tdr, T, d, n, E, K, cf, "bf16", T + d)
+    assert_bf16_close(a, a_ref, "a_act")
+    assert_bf16_close(y, y_ref, "y_perm")
+    assert_bf16_close(out, out_ref, "out")
+    assert_status_ok(tdr)
+
+
+# ------------------------------------------------------------------ whole layer
+def test_forward_tiny_fp32(cuda_lib):
+    tdr = cuda_lib
+    cfg = mi.TINY_FP32
+    inp = mi.make_inputs(cfg)
+    s = shape_of(cfg, tdr)
+    out, ws = tdr.forward(s, cuda(inp.x), cuda(inp.w_r), cuda(inp.w_gate), cuda(inp.w_up),
+                          cuda(inp.w_down))
+    v = tdr.workspace_views(s, ws)
+    ref = orc.forward(inp.x.numpy(), inp.w_r.numpy(), inp.w_gate.numpy(), inp.w_up.numpy(),
+                      inp.w_down.numpy(), cfg.K, logits=v["logits"].cpu().numpy())
+    np.testing.assert_array_equal(v["topk_ids"].cpu().numpy(), ref["topk_ids"])
+    assert np.abs(out.cpu().numpy() - ref["out"]).max() <= F32_ABS
+    dense = orc.dense_reference(inp.x.numpy(), inp.w_gate.numpy(), inp.w_up.numpy(),
+                                inp.w_down.numpy(), ref["topk_ids"], ref["topk_w"], cfg.E)
+    assert np.abs(out.cpu().numpy() - dense).max() <= F32_ABS
+    assert_status_ok(tdr)
+
+
+@pytest.mark.parametrize("name", ["mixtral_bf16", "fine_grained_bf16", "skewed_capacity_bf16"])
+def test_forward_full_size_workloads(cuda_lib, name):
+    tdr = cuda_lib
+    cfg = mi.CONFIGS[name]
+    inp = inputs_for(cfg)
+    s = shape_of(cfg, tdr)
+    out, ws = tdr.forward(s, cuda(inp.x), cuda(inp.w_r), cuda(inp.w_gate), cuda(inp.w_up),
+                          cuda(inp.w_down), bias=cuda(inp.bias))
+    torch.cuda.synchronize()
+    assert_status_ok(tdr)
+    v = tdr.workspace_views(s, ws)
+    lg = v["logits"].cpu().numpy()
+    rng = np.random.default_rng(7)
+    sample = np.sort(rng.choice(cfg.T, size=64, replace=False))
+    ref_lg = orc.router_logits(inp.x[sample], inp.w_r,
+                               None if inp.bias is None else inp.bias.numpy())
+    np.testing.assert_allclose(lg[sample], ref_lg, rtol=1e-4, atol=2e-4)
+    ids_ref, w_ref = check_routing(tdr, v["logits"], v["topk_ids"], v["topk_w"], cfg.K)
+    C = orc.capacity(cfg.capacity_factor, cfg.T, cfg.K, cfg.E)
+    _, offsets, a2p, _ = check_permutation(v, ids_ref, cfg.E, C)
+    if C is not None:
+        assert (a2p < 0).any()  # the skewed workload really drops
+    tokens = sample[:16]
+    ref_rows = orc.forward_rows(tokens, inp.x, inp.w_gate, inp.w_up, inp.w_down, ids_ref, w_ref,
+                                a2p, cfg.K)
+    assert_bf16_close(out[torch.from_numpy(tokens).cuda()].float().cpu().numpy(), ref_rows,
+                      f"{name} out")
+
+
+@pytest.mark.parametrize("T", mi.DISPATCH_COMBINE_T)
+def test_dispatch_combine_identity_experts(cuda_lib, T):
+    """route (given logits) -> permute with x_perm -> combine(y_perm = x_perm) returns x."""
+    tdr = cuda_lib
+    cfg = mi.DISPATCH_COMBINE.with_T(T)
+    inp = mi.make_inputs(cfg)
+    s = shape_of(cfg, tdr)
+    x = cuda(inp.x)
+    ids, w, _ = tdr.route(s, logits_in=cuda(inp.logits))
+    perm = tdr.permute(s, ids, x=x, materialize=True)
+    out = tdr.combine(s, perm["x_perm"], perm["assign_to_perm"], w)
+    ids_ref, w_ref = check_routing(tdr, inp.logits, ids, w, cfg.K)
+    check_permutation(perm, ids_ref, cfg.E, None)
+    got = out.float().cpu().numpy()
+    xr = inp.x.float().numpy()
+    ulp = np.abs(xr) * 2.0 ** -8 + 1e-30
+    assert np.all(np.abs(got - xr) <= ulp)
+    assert_status_ok(tdr)
+
+
+def test_forward_edge_cases(cuda_lib):
+    tdr = cuda_lib
+    # one token; one expert with K = 1; all tokens forced onto one expert; tiny capacity
+    for (T, d, n, E, K, cf, force) in [(1, 64, 64, 4, 2, 0.0, False),
+                                       (77, 64, 128, 1, 1, 0.0, False),
+                                       (300, 128, 64, 8, 2, 0.0, True),
+                                       (300, 128, 64, 8, 2, 0.1, True)]:
+        cfg = mi.MoEConfig("edge", T=T, d=d, E=E, K=K, n=n, dtype="bf16", capacity_factor=cf,
+                           seed=T + E)
+        inp = mi.make_inputs(cfg)
+        s = shape_of(cfg, tdr)
+        logits = None
+        if force:
+            lg = np.zeros((T, E), np.float32)
+            lg[:, 3] = 5.0
+            lg[:, 5] = 4.0
+            logits = torch.from_numpy(lg)
+        out, ws = tdr.forward(s, cuda(inp.x), cuda(inp.w_r), cuda(inp.w_gate), cuda(inp.w_up),
+                              cuda(inp.w_down), logits_in=cuda(logits))
+        v = tdr.workspace_views(s, ws)
+        ref = orc.forward(inp.x, inp.w_r, inp.w_gate, inp.w_up, inp.w_down, K,
+                          capacity_factor=cf, logits=v["logits"].cpu().numpy())
+        np.testing.assert_array_equal(v["topk_ids"].cpu().numpy(), ref["topk_ids"])
+        np.testing.assert_array_equal(v["assign_to_perm"].cpu().numpy(), ref["assign_to_perm"])
+        got = out.float().cpu().numpy()
+        if np.abs(ref["out"]).max() == 0:
+            assert np.abs(got).max() == 0
+        else:
+            assert_bf16_close(got, ref["out"], f"edge T={T} E={E} cf={cf}")
+        assert_status_ok(tdr)
+    s0 = tdr.make_shape(0, 64, 4, 2, 64, 0.0, True, torch.bfloat16)
+    z = torch.empty(0, 64, dtype=torch.bfloat16, device="cuda")
+    w = torch.zeros(64, 4, dtype=torch.bfloat16, device="cuda")
+    wg = torch.zeros(4, 64, 64, dtype=torch.bfloat16, device="cuda")
+    out0, _ = tdr.forward(s0, z, w, wg, wg, wg)
+    assert out0.shape == (0, 64)
+    assert_status_ok(tdr)

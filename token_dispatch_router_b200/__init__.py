@@ -1,0 +1,317 @@
+"""Python binding of the B200 MoE-layer forward library (libmoe_b200.so).
+
+Argument marshalling only: every step of the layer runs in the library's CUDA kernels.
+The functions take torch CUDA tensors (PyTorch is used for device memory and streams),
+check dtype/shape/contiguity, and call the C ABI of include/moe.h through ctypes on the
+current torch stream. There is no CPU fallback: without the compiled library, or without
+a CUDA device, every call raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libmoe_b200.so")
+
+MOE_F32, MOE_BF16 = 0, 1
+STATUS = {0: "ok", 1: "invalid argument", 2: "unsupported shape", 3: "CUDA error",
+          4: "workspace missing or too small", 5: "device wait timed out",
+          6: "device index out of range"}
+
+
+class MoEError(RuntimeError):
+    def __init__(self, code: int, where: str):
+        super().__init__(f"{where}: {STATUS.get(code, code)} ({code})")
+        self.code = code
+
+
+class moe_shape(ctypes.Structure):
+    _fields_ = [("T", ctypes.c_int32), ("d", ctypes.c_int32), ("E", ctypes.c_int32),
+                ("K", ctypes.c_int32), ("n", ctypes.c_int32),
+                ("capacity_factor", ctypes.c_float), ("renormalize", ctypes.c_int32),
+                ("dtype", ctypes.c_int32)]
+
+
+class moe_workspace_layout(ctypes.Structure):
+    _fields_ = [(f, ctypes.c_size_t) for f in (
+        "logits", "topk_ids", "topk_w", "counts", "offsets", "assign_to_perm",
+        "perm_to_assign", "permute_scratch", "a_act", "y_perm", "total")]
+
+
+_P = ctypes.c_void_p
+_S = ctypes.POINTER(moe_shape)
+_SIGS = {
+    "moe_permute_workspace_size": (ctypes.c_size_t, [_S]),
+    "moe_forward_workspace_size": (ctypes.c_size_t, [_S]),
+    "moe_forward_workspace_layout": (ctypes.c_int, [_S, ctypes.POINTER(moe_workspace_layout)]),
+    "moe_route": (ctypes.c_int, [_S, _P, _P, _P, _P, _P, _P, _P, _P]),
+    "moe_permute": (ctypes.c_int, [_S, _P, _P, _P, _P, _P, _P, _P, _P, ctypes.c_size_t, _P]),
+    "moe_grouped_ffn": (ctypes.c_int, [_S, _P, _P, _P, _P, _P, _P, _P, _P, _P]),
+    "moe_combine": (ctypes.c_int, [_S, _P, _P, _P, _P, _P]),
+    "moe_forward": (ctypes.c_int, [_S, _P, _P, _P, _P, _P, _P, _P, _P, _P, ctypes.c_size_t, _P]),
+    "moe_get_device_status": (ctypes.c_int, [_P]),
+    "moe_status_string": (ctypes.c_char_p, [ctypes.c_int]),
+    "moe_profile_enable": (ctypes.c_int, [ctypes.c_int]),
+    "moe_profile_reset": (ctypes.c_int, []),
+    "moe_kernel_count": (ctypes.c_int, []),
+    "moe_kernel_name": (ctypes.c_char_p, [ctypes.c_int]),
+    "moe_profile_query": (ctypes.c_int, [ctypes.c_int, ctypes.POINTER(ctypes.c_int64),
+                                         ctypes.POINTER(ctypes.c_double)]),
+    "moe_launch_count": (ctypes.c_int64, []),
+    "moe_selftest_timeout": (ctypes.c_int, [ctypes.c_uint64, _P]),
+}
+
+_lib: Optional[ctypes.CDLL] = None
+
+
+def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
+    """Load (once) and type the C ABI. Raises if the library is missing."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(path):
+        raise RuntimeError(f"CUDA library not built: {path} (run python -m "
+                           "token_dispatch_router_b200.build)")
+    lib = ctypes.CDLL(path)
+    for name, (res, args) in _SIGS.items():
+        fn = getattr(lib, name)
+        fn.restype = res
+        fn.argtypes = args
+    _lib = lib
+    return lib
+
+
+def _check(code: int, where: str) -> None:
+    if code != 0:
+        raise MoEError(code, where)
+
+
+def make_shape(T: int, d: int, E: int, K: int, n: int = 0, capacity_factor: float = 0.0,
+               renormalize: bool = True, dtype=torch.bfloat16) -> moe_shape:
+    dt = MOE_BF16 if dtype == torch.bfloat16 else MOE_F32
+    return moe_shape(T, d, E, K, n, float(capacity_factor), 1 if renormalize else 0, dt)
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream() -> ctypes.c_void_p:
+    return ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+
+
+def _dev(t: torch.Tensor, name: str, dtype=None, shape=None) -> None:
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if dtype is not None and t.dtype != dtype:
+        raise ValueError(f"{name} must be {dtype}, got {t.dtype}")
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
+
+
+def _act_dtype(shape: moe_shape):
+    return torch.bfloat16 if shape.dtype == MOE_BF16 else torch.float32
+
+
+def permute_workspace_size(shape: moe_shape) -> int:
+    return int(load_library().moe_permute_workspace_size(ctypes.byref(shape)))
+
+
+def forward_workspace_size(shape: moe_shape) -> int:
+    return int(load_library().moe_forward_workspace_size(ctypes.byref(shape)))
+
+
+def forward_workspace_layout(shape: moe_shape) -> moe_workspace_layout:
+    L = moe_workspace_layout()
+    _check(load_library().moe_forward_workspace_layout(ctypes.byref(shape), ctypes.byref(L)),
+           "moe_forward_workspace_layout")
+    return L
+
+
+def route(shape: moe_shape, x=None, w_r=None, bias=None, logits_in=None, logits_out=None,
+          topk_ids=None, topk_w=None):
+    """moe_route. Returns (topk_ids [T,K] int32, topk_w [T,K] fp32, logits_out or None)."""
+    lib = load_library()
+    T, E, K = shape.T, shape.E, shape.K
+    dev = (logits_in if logits_in is not None else x).device
+    dt = _act_dtype(shape)
+    if logits_in is None:
+        _dev(x, "x", dt, (T, shape.d))
+        _dev(w_r, "w_r", dt, (shape.d, E))
+    else:
+        _dev(logits_in, "logits_in", torch.float32, (T, E))
+    if bias is not None:
+        _dev(bias, "bias", torch.float32, (E,))
+    if topk_ids is None:
+        topk_ids = torch.empty(T, K, dtype=torch.int32, device=dev)
+    if topk_w is None:
+        topk_w = torch.empty(T, K, dtype=torch.float32, device=dev)
+    if logits_out is not None:
+        _dev(logits_out, "logits_out", torch.float32, (T, E))
+    _check(lib.moe_route(ctypes.byref(shape), _ptr(x), _ptr(w_r), _ptr(bias), _ptr(logits_in),
+                         _ptr(logits_out), _ptr(topk_ids), _ptr(topk_w), _stream()), "moe_route")
+    return topk_ids, topk_w, logits_out
+
+
+def permute(shape: moe_shape, topk_ids: torch.Tensor, x=None, materialize: bool = False,
+            workspace=None):
+    """moe_permute. Returns dict(counts, offsets, assign_to_perm, perm_to_assign[, x_perm])."""
+    lib = load_library()
+    T, E, K = shape.T, shape.E, shape.K
+    dev = topk_ids.device
+    _dev(topk_ids, "topk_ids", torch.int32, (T, K))
+    counts = torch.empty(E, dtype=torch.int32, device=dev)
+    offsets = torch.empty(E + 1, dtype=torch.int32, device=dev)
+    a2p = torch.empty(T * K, dtype=torch.int32, device=dev)
+    p2a = torch.full((T * K,), -1, dtype=torch.int32, device=dev)
+    x_perm = None
+    if materialize:
+        _dev(x, "x", _act_dtype(shape), (T, shape.d))
+        x_perm = torch.empty(T * K, shape.d, dtype=x.dtype, device=dev)
+    need = permute_workspace_size(shape)
+    if workspace is None:
+        workspace = torch.empty(max(need, 256), dtype=torch.uint8, device=dev)
+    _check(lib.moe_permute(ctypes.byref(shape), _ptr(topk_ids), _ptr(counts), _ptr(offsets),
+                           _ptr(a2p), _ptr(p2a), _ptr(x if materialize else None), _ptr(x_perm),
+                           _ptr(workspace), workspace.numel(), _stream()), "moe_permute")
+    out = dict(counts=counts, offsets=offsets, assign_to_perm=a2p, perm_to_assign=p2a)
+    if materialize:
+        out["x_perm"] = x_perm
+    return out
+
+
+def grouped_ffn(shape: moe_shape, x, offsets, perm_to_assign, w_gate, w_up, w_down,
+                a_act=None, y_perm=None):
+    """moe_grouped_ffn. Returns (a_act [T*K, n], y_perm [T*K, d])."""
+    lib = load_library()
+    T, d, E, K, n = shape.T, shape.d, shape.E, shape.K, shape.n
+    dt = _act_dtype(shape)
+    _dev(x, "x", dt, (T, d))
+    _dev(offsets, "offsets", torch.int32, (E + 1,))
+    _dev(perm_to_assign, "perm_to_assign", torch.int32, (T * K,))
+    _dev(w_gate, "w_gate", dt, (E, d, n))
+    _dev(w_up, "w_up", dt, (E, d, n))
+    _dev(w_down, "w_down", dt, (E, n, d))
+    if a_act is None:
+        a_act = torch.empty(T * K, n, dtype=dt, device=x.device)
+    if y_perm is None:
+        y_perm = torch.empty(T * K, d, dtype=dt, device=x.device)
+    _check(lib.moe_grouped_ffn(ctypes.byref(shape), _ptr(x), _ptr(offsets), _ptr(perm_to_assign),
+                               _ptr(w_gate), _ptr(w_up), _ptr(w_down), _ptr(a_act), _ptr(y_perm),
+                               _stream()), "moe_grouped_ffn")
+    return a_act, y_perm
+
+
+def combine(shape: moe_shape, y_perm, assign_to_perm, topk_w, out=None):
+    """moe_combine. Returns out [T, d]."""
+    lib = load_library()
+    T, d, K = shape.T, shape.d, shape.K
+    dt = _act_dtype(shape)
+    _dev(y_perm, "y_perm", dt)
+    if y_perm.dim() != 2 or y_perm.shape[1] != d or y_perm.shape[0] < T * K:
+        raise ValueError("y_perm must be [>= T*K, d]")
+    _dev(assign_to_perm, "assign_to_perm", torch.int32, (T * K,))
+    _dev(topk_w, "topk_w", torch.float32, (T, K))
+    if out is None:
+        out = torch.empty(T, d, dtype=dt, device=y_perm.device)
+    _check(lib.moe_combine(ctypes.byref(shape), _ptr(y_perm), _ptr(assign_to_perm), _ptr(topk_w),
+                           _ptr(out), _stream()), "moe_combine")
+    return out
+
+
+def forward(shape: moe_shape, x, w_r, w_gate, w_up, w_down, bias=None, logits_in=None, out=None,
+            workspace=None):
+    """moe_forward (the whole layer). Returns (out [T, d], workspace)."""
+    lib = load_library()
+    T, d, E, n = shape.T, shape.d, shape.E, shape.n
+    dt = _act_dtype(shape)
+    _dev(x, "x", dt, (T, d))
+    if logits_in is None:
+        _dev(w_r, "w_r", dt, (d, E))
+    else:
+        _dev(logits_in, "logits_in", torch.float32, (T, E))
+    _dev(w_gate, "w_gate", dt, (E, d, n))
+    _dev(w_up, "w_up", dt, (E, d, n))
+    _dev(w_down, "w_down", dt, (E, n, d))
+    if bias is not None:
+        _dev(bias, "bias", torch.float32, (E,))
+    need = forward_workspace_size(shape)
+    if need == 0:
+        raise MoEError(1, "moe_forward_workspace_size")
+    if workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=x.device)
+    if out is None:
+        out = torch.empty(T, d, dtype=dt, device=x.device)
+    _check(lib.moe_forward(ctypes.byref(shape), _ptr(x), _ptr(w_r), _ptr(bias), _ptr(logits_in),
+                           _ptr(w_gate), _ptr(w_up), _ptr(w_down), _ptr(out), _ptr(workspace),
+                           workspace.numel(), _stream()), "moe_forward")
+    return out, workspace
+
+
+def workspace_views(shape: moe_shape, workspace: torch.Tensor) -> dict:
+    """Typed views of moe_forward's intermediates inside its workspace."""
+    L = forward_workspace_layout(shape)
+    T, E, K, d, n = shape.T, shape.E, shape.K, shape.d, shape.n
+    A = T * K
+    dt = _act_dtype(shape)
+    eb = 2 if dt == torch.bfloat16 else 4
+
+    def view(off, count, dtype, shp, esz):
+        return workspace[off:off + count * esz].view(dtype).view(*shp)
+
+    return dict(logits=view(L.logits, T * E, torch.float32, (T, E), 4),
+                topk_ids=view(L.topk_ids, A, torch.int32, (T, K), 4),
+                topk_w=view(L.topk_w, A, torch.float32, (T, K), 4),
+                counts=view(L.counts, E, torch.int32, (E,), 4),
+                offsets=view(L.offsets, E + 1, torch.int32, (E + 1,), 4),
+                assign_to_perm=view(L.assign_to_perm, A, torch.int32, (A,), 4),
+                perm_to_assign=view(L.perm_to_assign, A, torch.int32, (A,), 4),
+                a_act=view(L.a_act, A * n, dt, (A, n), eb),
+                y_perm=view(L.y_perm, A * d, dt, (A, d), eb))
+
+
+def device_status() -> int:
+    return int(load_library().moe_get_device_status(_stream()))
+
+
+def selftest_timeout(limit_ns: int) -> int:
+    """Run the bounded-wait self test; returns the device status it leaves (5 = timeout)."""
+    lib = load_library()
+    _check(lib.moe_selftest_timeout(int(limit_ns), _stream()), "moe_selftest_timeout")
+    return device_status()
+
+
+class Profiler:
+    """Per-kernel device time from the library's opt-in event profiler."""
+
+    def __init__(self):
+        self.lib = load_library()
+
+    def __enter__(self):
+        self.lib.moe_profile_reset()
+        self.lib.moe_profile_enable(1)
+        return self
+
+    def __exit__(self, *exc):
+        self.lib.moe_profile_enable(0)
+
+    def results(self) -> dict:
+        out = {}
+        for i in range(self.lib.moe_kernel_count()):
+            n = ctypes.c_int64(0)
+            ms = ctypes.c_double(0.0)
+            _check(self.lib.moe_profile_query(i, ctypes.byref(n), ctypes.byref(ms)),
+                   "moe_profile_query")
+            if n.value:
+                out[self.lib.moe_kernel_name(i).decode()] = (int(n.value), float(ms.value))
+        return out
+
+
+def launch_count() -> int:
+    return int(load_library().moe_launch_count())

@@ -1,0 +1,355 @@
+// C ABI of the MoE-layer forward: argument checks, workspace layout, the device status
+// word, the opt-in profiler and the entry points declared in include/moe.h.
+#include <math.h>
+#include <string.h>
+
+#include <mutex>
+#include <vector>
+
+#include "common.cuh"
+
+namespace moe {
+
+moe_status launch_route(const moe_shape& s, const void* x, const void* w_r, const float* bias,
+                        const float* logits_in, float* logits_out, int32_t* ids, float* w,
+                        cudaStream_t st);
+size_t permute_scratch_bytes(const moe_shape& s);
+moe_status launch_permute(const moe_shape& s, const int32_t* ids, int32_t* counts,
+                          int32_t* offsets, int32_t* a2p, int32_t* p2a, const void* x,
+                          void* x_perm, void* scratch, cudaStream_t st);
+moe_status launch_ffn_simt(const moe_shape& s, const void* x, const int32_t* offsets,
+                           const int32_t* p2a, const void* w_gate, const void* w_up,
+                           const void* w_down, void* a_act, void* y_perm, cudaStream_t st);
+moe_status launch_ffn_tc(const moe_shape& s, const void* x, const int32_t* offsets,
+                         const int32_t* p2a, const void* w_gate, const void* w_up,
+                         const void* w_down, void* a_act, void* y_perm, cudaStream_t st);
+moe_status launch_combine(const moe_shape& s, const void* y_perm, const int32_t* a2p,
+                          const float* topk_w, void* out, cudaStream_t st);
+moe_status launch_selftest_timeout(uint64_t limit_ns, cudaStream_t st);
+
+// ------------------------------------------------------------------ device state
+__device__ unsigned int g_device_status;
+
+namespace {
+constexpr int kMaxDev = 64;
+unsigned int* g_status_ptr[kMaxDev];
+int g_sms[kMaxDev];
+std::mutex g_dev_mu;
+
+int cur_dev() {
+  int d = 0;
+  cudaGetDevice(&d);
+  return (d >= 0 && d < kMaxDev) ? d : 0;
+}
+}  // namespace
+
+unsigned int* device_status_ptr() {
+  const int d = cur_dev();
+  std::lock_guard<std::mutex> lk(g_dev_mu);
+  if (g_status_ptr[d] == nullptr) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_device_status) == cudaSuccess) g_status_ptr[d] = (unsigned*)p;
+  }
+  return g_status_ptr[d];
+}
+
+int sm_count() {
+  const int d = cur_dev();
+  std::lock_guard<std::mutex> lk(g_dev_mu);
+  if (g_sms[d] == 0) {
+    int n = 0;
+    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, d);
+    g_sms[d] = n > 0 ? n : 1;
+  }
+  return g_sms[d];
+}
+
+// ------------------------------------------------------------------ profiler
+namespace {
+const char* kKernelNames[K_COUNT] = {
+    "route",        "hist",          "scan",           "scatter",     "gather_rows", "gateup_tc",
+    "down_tc",      "gateup_simt",   "down_simt",      "combine",     "selftest_timeout"};
+
+struct ProfRec {
+  int kid;
+  cudaEvent_t a, b;
+};
+bool g_prof_on = false;
+std::vector<ProfRec> g_recs;
+std::vector<cudaEvent_t> g_pool;
+long long g_launches = 0;
+std::mutex g_prof_mu;
+
+cudaEvent_t take_event() {
+  if (!g_pool.empty()) {
+    cudaEvent_t e = g_pool.back();
+    g_pool.pop_back();
+    return e;
+  }
+  cudaEvent_t e = nullptr;
+  cudaEventCreate(&e);
+  return e;
+}
+}  // namespace
+
+void launch_begin(int kid, cudaStream_t s) {
+  std::lock_guard<std::mutex> lk(g_prof_mu);
+  ++g_launches;
+  if (!g_prof_on) return;
+  ProfRec r{kid, take_event(), take_event()};
+  cudaEventRecord(r.a, s);
+  g_recs.push_back(r);
+}
+
+moe_status launch_end(int kid, cudaStream_t s) {
+  const cudaError_t err = cudaGetLastError();
+  {
+    std::lock_guard<std::mutex> lk(g_prof_mu);
+    if (g_prof_on && !g_recs.empty() && g_recs.back().kid == kid) cudaEventRecord(g_recs.back().b, s);
+  }
+  return err == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
+// ------------------------------------------------------------------ checks and layout
+namespace {
+
+size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
+
+int elem_bytes(const moe_shape& s) { return s.dtype == MOE_BF16 ? 2 : 4; }
+
+moe_status check_shape(const moe_shape* s, bool need_d, bool need_ffn) {
+  if (s == nullptr) return MOE_ERR_INVALID_ARG;
+  if (s->dtype != MOE_F32 && s->dtype != MOE_BF16) return MOE_ERR_INVALID_ARG;
+  if (s->T < 0 || s->E < 1 || s->K < 1 || s->K > s->E) return MOE_ERR_INVALID_ARG;
+  if (s->E > 256 || s->K > 32) return MOE_ERR_UNSUPPORTED;
+  if ((long long)s->T * s->K > 0x7fffffffLL) return MOE_ERR_UNSUPPORTED;
+  if (isnan(s->capacity_factor)) return MOE_ERR_INVALID_ARG;
+  if (need_d) {
+    if (s->d < 64 || s->d % 64 != 0) return MOE_ERR_INVALID_ARG;
+  }
+  if (need_ffn) {
+    const int nq = s->dtype == MOE_BF16 ? 64 : 16;
+    if (s->n < nq || s->n % nq != 0) return MOE_ERR_INVALID_ARG;
+  }
+  return MOE_OK;
+}
+
+bool layout_of(const moe_shape& s, moe_workspace_layout* L) {
+  const size_t T = (size_t)s.T, E = (size_t)s.E, K = (size_t)s.K, A = T * K;
+  const size_t eb = (size_t)elem_bytes(s);
+  size_t o = 0;
+  L->logits = o;
+  o = align256(o + T * E * 4);
+  L->topk_ids = o;
+  o = align256(o + A * 4);
+  L->topk_w = o;
+  o = align256(o + A * 4);
+  L->counts = o;
+  o = align256(o + E * 4);
+  L->offsets = o;
+  o = align256(o + (E + 1) * 4);
+  L->assign_to_perm = o;
+  o = align256(o + A * 4);
+  L->perm_to_assign = o;
+  o = align256(o + A * 4);
+  L->permute_scratch = o;
+  o = align256(o + permute_scratch_bytes(s));
+  L->a_act = o;
+  o = align256(o + A * (size_t)s.n * eb);
+  L->y_perm = o;
+  o = align256(o + A * (size_t)s.d * eb);
+  L->total = o;
+  return true;
+}
+
+bool aligned16(const void* p) { return ((uintptr_t)p & 15) == 0; }
+
+}  // namespace
+}  // namespace moe
+
+using namespace moe;
+
+extern "C" {
+
+size_t moe_permute_workspace_size(const moe_shape* s) {
+  if (check_shape(s, false, false) != MOE_OK) return 0;
+  return align256(permute_scratch_bytes(*s)) + 256;
+}
+
+size_t moe_forward_workspace_size(const moe_shape* s) {
+  if (check_shape(s, true, true) != MOE_OK) return 0;
+  moe_workspace_layout L;
+  layout_of(*s, &L);
+  return L.total;
+}
+
+moe_status moe_forward_workspace_layout(const moe_shape* s, moe_workspace_layout* L) {
+  if (L == nullptr) return MOE_ERR_INVALID_ARG;
+  const moe_status r = check_shape(s, true, true);
+  if (r != MOE_OK) return r;
+  layout_of(*s, L);
+  return MOE_OK;
+}
+
+moe_status moe_route(const moe_shape* s, const void* x, const void* w_r, const float* bias,
+                     const float* logits_in, float* logits_out, int32_t* topk_ids, float* topk_w,
+                     moe_stream_t stream) {
+  moe_status r = check_shape(s, logits_in == nullptr, false);
+  if (r != MOE_OK) return r;
+  if (topk_ids == nullptr || topk_w == nullptr) return MOE_ERR_INVALID_ARG;
+  if (logits_in == nullptr && (x == nullptr || w_r == nullptr)) return MOE_ERR_INVALID_ARG;
+  if (logits_in == nullptr && !aligned16(x)) return MOE_ERR_INVALID_ARG;
+  if (s->T == 0) return MOE_OK;
+  return launch_route(*s, x, w_r, bias, logits_in, logits_out, topk_ids, topk_w,
+                      (cudaStream_t)stream);
+}
+
+moe_status moe_permute(const moe_shape* s, const int32_t* topk_ids, int32_t* counts,
+                       int32_t* offsets, int32_t* assign_to_perm, int32_t* perm_to_assign,
+                       const void* x, void* x_perm, void* workspace, size_t ws_bytes,
+                       moe_stream_t stream) {
+  const bool gather = (x != nullptr && x_perm != nullptr);
+  moe_status r = check_shape(s, gather, false);
+  if (r != MOE_OK) return r;
+  if (topk_ids == nullptr || counts == nullptr || offsets == nullptr || assign_to_perm == nullptr ||
+      perm_to_assign == nullptr)
+    return MOE_ERR_INVALID_ARG;
+  if ((x == nullptr) != (x_perm == nullptr)) return MOE_ERR_INVALID_ARG;
+  if (gather && (!aligned16(x) || !aligned16(x_perm))) return MOE_ERR_INVALID_ARG;
+  const size_t need = permute_scratch_bytes(*s);
+  if (need > 0 && (workspace == nullptr || ws_bytes < need)) return MOE_ERR_WORKSPACE;
+  return launch_permute(*s, topk_ids, counts, offsets, assign_to_perm, perm_to_assign, x, x_perm,
+                        workspace, (cudaStream_t)stream);
+}
+
+moe_status moe_grouped_ffn(const moe_shape* s, const void* x, const int32_t* offsets,
+                           const int32_t* perm_to_assign, const void* w_gate, const void* w_up,
+                           const void* w_down, void* a_act, void* y_perm, moe_stream_t stream) {
+  moe_status r = check_shape(s, true, true);
+  if (r != MOE_OK) return r;
+  if (!x || !offsets || !perm_to_assign || !w_gate || !w_up || !w_down || !a_act || !y_perm)
+    return MOE_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(w_gate) || !aligned16(w_up) || !aligned16(w_down) ||
+      !aligned16(a_act) || !aligned16(y_perm))
+    return MOE_ERR_INVALID_ARG;
+  if (s->T == 0) return MOE_OK;
+  if (s->dtype == MOE_BF16)
+    return launch_ffn_tc(*s, x, offsets, perm_to_assign, w_gate, w_up, w_down, a_act, y_perm,
+                         (cudaStream_t)stream);
+  return launch_ffn_simt(*s, x, offsets, perm_to_assign, w_gate, w_up, w_down, a_act, y_perm,
+                         (cudaStream_t)stream);
+}
+
+moe_status moe_combine(const moe_shape* s, const void* y_perm, const int32_t* assign_to_perm,
+                       const float* topk_w, void* out, moe_stream_t stream) {
+  moe_status r = check_shape(s, true, false);
+  if (r != MOE_OK) return r;
+  if (!y_perm || !assign_to_perm || !topk_w || !out) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(y_perm) || !aligned16(out)) return MOE_ERR_INVALID_ARG;
+  return launch_combine(*s, y_perm, assign_to_perm, topk_w, out, (cudaStream_t)stream);
+}
+
+moe_status moe_forward(const moe_shape* s, const void* x, const void* w_r, const float* bias,
+                       const float* logits_in, const void* w_gate, const void* w_up,
+                       const void* w_down, void* out, void* workspace, size_t ws_bytes,
+                       moe_stream_t stream) {
+  moe_status r = check_shape(s, true, true);
+  if (r != MOE_OK) return r;
+  if (!x || (!w_r && !logits_in) || !w_gate || !w_up || !w_down || !out) return MOE_ERR_INVALID_ARG;
+  moe_workspace_layout L;
+  layout_of(*s, &L);
+  if (workspace == nullptr || ws_bytes < L.total) return MOE_ERR_WORKSPACE;
+  if (((uintptr_t)workspace & 255) != 0) return MOE_ERR_INVALID_ARG;
+  if (s->T == 0) return MOE_OK;
+  uint8_t* ws = (uint8_t*)workspace;
+  const cudaStream_t st = (cudaStream_t)stream;
+  float* logits = (float*)(ws + L.logits);
+  int32_t* ids = (int32_t*)(ws + L.topk_ids);
+  float* w = (float*)(ws + L.topk_w);
+  int32_t* counts = (int32_t*)(ws + L.counts);
+  int32_t* offsets = (int32_t*)(ws + L.offsets);
+  int32_t* a2p = (int32_t*)(ws + L.assign_to_perm);
+  int32_t* p2a = (int32_t*)(ws + L.perm_to_assign);
+  if ((r = moe_route(s, x, w_r, bias, logits_in, logits, ids, w, stream)) != MOE_OK) return r;
+  if ((r = launch_permute(*s, ids, counts, offsets, a2p, p2a, nullptr, nullptr,
+                          ws + L.permute_scratch, st)) != MOE_OK)
+    return r;
+  if ((r = moe_grouped_ffn(s, x, offsets, p2a, w_gate, w_up, w_down, ws + L.a_act, ws + L.y_perm,
+                           stream)) != MOE_OK)
+    return r;
+  return launch_combine(*s, ws + L.y_perm, a2p, w, out, st);
+}
+
+moe_status moe_get_device_status(moe_stream_t stream) {
+  if (cudaStreamSynchronize((cudaStream_t)stream) != cudaSuccess) return MOE_ERR_CUDA;
+  unsigned int v = 0;
+  if (cudaMemcpyFromSymbol(&v, g_device_status, sizeof(v)) != cudaSuccess) return MOE_ERR_CUDA;
+  const unsigned int zero = 0;
+  if (cudaMemcpyToSymbol(g_device_status, &zero, sizeof(zero)) != cudaSuccess) return MOE_ERR_CUDA;
+  return (moe_status)v;
+}
+
+const char* moe_status_string(moe_status st) {
+  switch (st) {
+    case MOE_OK: return "ok";
+    case MOE_ERR_INVALID_ARG: return "invalid argument";
+    case MOE_ERR_UNSUPPORTED: return "unsupported shape";
+    case MOE_ERR_CUDA: return "CUDA error";
+    case MOE_ERR_WORKSPACE: return "workspace missing or too small";
+    case MOE_ERR_TIMEOUT: return "device wait timed out";
+    case MOE_ERR_DEVICE_INDEX: return "device index out of range";
+  }
+  return "unknown status";
+}
+
+moe_status moe_profile_enable(int on) {
+  std::lock_guard<std::mutex> lk(g_prof_mu);
+  g_prof_on = on != 0;
+  return MOE_OK;
+}
+
+moe_status moe_profile_reset(void) {
+  std::lock_guard<std::mutex> lk(g_prof_mu);
+  for (auto& r : g_recs) {
+    cudaEventSynchronize(r.b);
+    g_pool.push_back(r.a);
+    g_pool.push_back(r.b);
+  }
+  g_recs.clear();
+  return MOE_OK;
+}
+
+int moe_kernel_count(void) { return K_COUNT; }
+
+const char* moe_kernel_name(int id) { return (id >= 0 && id < K_COUNT) ? kKernelNames[id] : ""; }
+
+moe_status moe_profile_query(int id, int64_t* launches, double* total_ms) {
+  if (id < 0 || id >= K_COUNT || launches == nullptr || total_ms == nullptr)
+    return MOE_ERR_INVALID_ARG;
+  std::lock_guard<std::mutex> lk(g_prof_mu);
+  int64_t n = 0;
+  double ms = 0.0;
+  for (auto& r : g_recs) {
+    if (r.kid != id) continue;
+    if (cudaEventSynchronize(r.b) != cudaSuccess) return MOE_ERR_CUDA;
+    float f = 0.f;
+    if (cudaEventElapsedTime(&f, r.a, r.b) != cudaSuccess) return MOE_ERR_CUDA;
+    ++n;
+    ms += f;
+  }
+  *launches = n;
+  *total_ms = ms;
+  return MOE_OK;
+}
+
+int64_t moe_launch_count(void) {
+  std::lock_guard<std::mutex> lk(g_prof_mu);
+  return g_launches;
+}
+
+moe_status moe_selftest_timeout(uint64_t limit_ns, moe_stream_t stream) {
+  if (limit_ns == 0 || limit_ns > 10000000000ull) return MOE_ERR_INVALID_ARG;
+  return launch_selftest_timeout(limit_ns, (cudaStream_t)stream);
+}
+
+}  // extern "C"

@@ -1,0 +1,97 @@
+// Shared device/host helpers of the MoE-layer library (sm_100a only).
+#pragma once
+
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/moe.h"
+
+namespace moe {
+
+typedef __nv_bfloat16 bf16;
+
+// ---------------------------------------------------------------- status word
+// Kernels receive a pointer to the library's device status word and record
+// the first fault there (atomicCAS from 0), never trapping.
+__device__ __forceinline__ void report(unsigned int* status, unsigned int code) {
+  if (status) atomicCAS(status, 0u, code);
+}
+
+// ---------------------------------------------------------------- dtype helpers
+template <typename T> struct Vec16;  // 16-byte vector of T
+template <> struct Vec16<float> {
+  static constexpr int N = 4;
+};
+template <> struct Vec16<bf16> {
+  static constexpr int N = 8;
+};
+
+__device__ __forceinline__ float to_f32(float v) { return v; }
+__device__ __forceinline__ float to_f32(bf16 v) { return __bfloat162float(v); }
+
+__device__ __forceinline__ void unpack16(const uint4& u, float* f, float) {
+  f[0] = __uint_as_float(u.x);
+  f[1] = __uint_as_float(u.y);
+  f[2] = __uint_as_float(u.z);
+  f[3] = __uint_as_float(u.w);
+}
+__device__ __forceinline__ void unpack16(const uint4& u, float* f, bf16) {
+  const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    f[2 * i] = __uint_as_float(w[i] << 16);
+    f[2 * i + 1] = __uint_as_float(w[i] & 0xffff0000u);
+  }
+}
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+  __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);  // RNE
+  return *reinterpret_cast<uint32_t*>(&h);
+}
+__device__ __forceinline__ uint4 pack16(const float* f, float) {
+  return make_uint4(__float_as_uint(f[0]), __float_as_uint(f[1]), __float_as_uint(f[2]),
+                    __float_as_uint(f[3]));
+}
+__device__ __forceinline__ uint4 pack16(const float* f, bf16) {
+  return make_uint4(pack_bf16x2(f[0], f[1]), pack_bf16x2(f[2], f[3]), pack_bf16x2(f[4], f[5]),
+                    pack_bf16x2(f[6], f[7]));
+}
+
+__device__ __forceinline__ uint32_t lanemask_lt() {
+  uint32_t m;
+  asm volatile("mov.u32 %0, %%lanemask_lt;" : "=r"(m));
+  return m;
+}
+
+__device__ __forceinline__ uint64_t globaltimer_ns() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+
+// ---------------------------------------------------------------- host side
+// Kernel ids of the opt-in profiler (order = moe_kernel_name).
+enum KernelId {
+  K_ROUTE = 0,
+  K_HIST,
+  K_SCAN,
+  K_SCATTER,
+  K_GATHER,
+  K_GATEUP_TC,
+  K_DOWN_TC,
+  K_GATEUP_SIMT,
+  K_DOWN_SIMT,
+  K_COMBINE,
+  K_SELFTEST,
+  K_COUNT
+};
+
+unsigned int* device_status_ptr();  // status word of the current device
+int sm_count();                     // SMs of the current device (cached)
+void launch_begin(int kernel_id, cudaStream_t s);
+moe_status launch_end(int kernel_id, cudaStream_t s);  // checks cudaGetLastError
+
+constexpr uint64_t kWaitLimitNs = 2000000000ull;  // bounded waits: 2 s
+
+}  // namespace moe

@@ -1,0 +1,250 @@
+// Dispatch metadata: per-expert counts, capacity clamp, exclusive scan and the stable
+// permutation between token-major assignments and expert-major slots.
+//
+// "Operators & compilers: MoE routing and sparse kernels" (charles2530.github.io),
+// section 3: regrouping tokens by expert is an index/scatter/gather problem that needs
+// counting and a prefix sum; section 4: a capacity factor bounds each expert's tokens and
+// the overflow is dropped. "Two upstream innovations of MoE: Routing-Free and OmniMoE"
+// (chatdocs.ruinique.com), section 2.3: tasks sorted by (expert, token). SonicMoE explainer
+// (gitcode.csdn.net), section 11: counts per expert, slot -> token, token slot -> slot.
+//
+// Atomic-free and deterministic. The T*K flat assignments are cut into chunks of
+// kChunk; a CTA owns a chunk and each of its 8 warps a contiguous slice of it.
+//   hist    : per warp, 32 ids at a time, __match_any_sync groups equal ids and the
+//             group's lowest lane adds the group size to the warp's private counter row
+//             (no two lanes touch one address); the CTA sums its 8 rows per expert.
+//   scan    : one CTA; per expert the chunk counts are scanned in chunk order (rank base
+//             of each chunk inside the expert), counts[e] is the total, kept = min(count,
+//             C) and offsets = exclusive scan of kept over experts.
+//   scatter : recomputes the warp rows, turns them into rank bases (chunk base + earlier
+//             warps), then walks the slice again: rank = base + (lanes of the group below
+//             me); rank < C -> slot offsets[e] + rank, else dropped (-1).
+// Inside an expert the slots follow ascending flat index a = t*K + k, i.e. token order.
+#include "common.cuh"
+
+namespace moe {
+
+namespace {
+
+constexpr int kWarps = 8;
+constexpr int kIters = 16;                   // 32-id groups per warp
+constexpr int kSlice = 32 * kIters;          // ids per warp
+constexpr int kChunk = kWarps * kSlice;      // ids per CTA
+constexpr int kMaxE = 256;
+
+__device__ __forceinline__ int load_id(const int32_t* ids, long long a, long long A, int E,
+                                       unsigned* status) {
+  if (a >= A) return -1;
+  const int id = ids[a];
+  if (id < 0 || id >= E) {
+    report(status, MOE_ERR_DEVICE_INDEX);
+    return -1;
+  }
+  return id;
+}
+
+// Counts of this warp's slice into its private row (plain shared-memory adds by unique lanes).
+__device__ __forceinline__ void warp_histogram(const int32_t* ids, long long slice0, long long A,
+                                               int E, int* row, unsigned* status) {
+  const int lane = threadIdx.x & 31;
+  int v[kIters];
+#pragma unroll
+  for (int it = 0; it < kIters; ++it) v[it] = load_id(ids, slice0 + it * 32 + lane, A, E, status);
+#pragma unroll
+  for (int it = 0; it < kIters; ++it) {
+    const unsigned m = __match_any_sync(0xffffffffu, v[it]);
+    if (v[it] >= 0 && lane == __ffs(m) - 1) row[v[it]] += __popc(m);
+    __syncwarp();
+  }
+}
+
+__global__ void __launch_bounds__(kWarps * 32) hist_kernel(const int32_t* __restrict__ ids,
+                                                           long long A, int E,
+                                                           int32_t* __restrict__ chunk_counts,
+                                                           unsigned* status) {
+  __shared__ int rows[kWarps][kMaxE];
+  const int tid = threadIdx.x, warp = tid >> 5;
+  for (int i = tid; i < kWarps * kMaxE; i += blockDim.x) (&rows[0][0])[i] = 0;
+  __syncthreads();
+  const long long slice0 = (long long)blockIdx.x * kChunk + (long long)warp * kSlice;
+  warp_histogram(ids, slice0, A, E, rows[warp], status);
+  __syncthreads();
+  for (int e = tid; e < E; e += blockDim.x) {
+    int s = 0;
+#pragma unroll
+    for (int w = 0; w < kWarps; ++w) s += rows[w][e];
+    chunk_counts[(size_t)blockIdx.x * E + e] = s;
+  }
+}
+
+// One CTA of kMaxE threads: thread e walks the chunks of expert e in order.
+__global__ void __launch_bounds__(kMaxE) scan_kernel(const int32_t* __restrict__ chunk_counts,
+                                                     int32_t* __restrict__ chunk_base, int nchunks,
+                                                     int E, long long cap,
+                                                     int32_t* __restrict__ counts,
+                                                     int32_t* __restrict__ offsets) {
+  __shared__ long long kept_s[kMaxE];
+  const int e = threadIdx.x;
+  long long run = 0;
+  if (e < E) {
+    int c = 0;
+    for (; c + 8 <= nchunks; c += 8) {  // 8 independent loads in flight
+      int v[8];
+#pragma unroll
+      for (int j = 0; j < 8; ++j) v[j] = chunk_counts[(size_t)(c + j) * E + e];
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        chunk_base[(size_t)(c + j) * E + e] = (int32_t)run;
+        run += v[j];
+      }
+    }
+    for (; c < nchunks; ++c) {
+      const int v = chunk_counts[(size_t)c * E + e];
+      chunk_base[(size_t)c * E + e] = (int32_t)run;
+      run += v;
+    }
+    counts[e] = (int32_t)run;
+  }
+  kept_s[e] = (e < E) ? (cap >= 0 && run > cap ? cap : run) : 0;
+  __syncthreads();
+  // exclusive scan of kept over experts (Hillis-Steele on kMaxE entries)
+  for (int off = 1; off < kMaxE; off <<= 1) {
+    const long long add = (e >= off) ? kept_s[e - off] : 0;
+    __syncthreads();
+    kept_s[e] += add;
+    __syncthreads();
+  }
+  if (e < E) {
+    const long long incl = kept_s[e];
+    const long long mine = (cap >= 0 && run > cap) ? cap : run;
+    offsets[e] = (int32_t)(incl - mine);
+    if (e == E - 1) offsets[E] = (int32_t)incl;
+  }
+}
+
+__global__ void __launch_bounds__(kWarps * 32) scatter_kernel(
+    const int32_t* __restrict__ ids, long long A, int E, long long cap,
+    const int32_t* __restrict__ chunk_base, const int32_t* __restrict__ offsets,
+    int32_t* __restrict__ assign_to_perm, int32_t* __restrict__ perm_to_assign, unsigned* status) {
+  __shared__ int rows[kWarps][kMaxE];
+  __shared__ int offs[kMaxE];
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  for (int i = tid; i < kWarps * kMaxE; i += blockDim.x) (&rows[0][0])[i] = 0;
+  for (int e = tid; e < E; e += blockDim.x) offs[e] = offsets[e];
+  __syncthreads();
+  const long long slice0 = (long long)blockIdx.x * kChunk + (long long)warp * kSlice;
+  warp_histogram(ids, slice0, A, E, rows[warp], nullptr);
+  __syncthreads();
+  // rank base of each warp row: chunk base + counts of the earlier warps of this chunk
+  for (int e = tid; e < E; e += blockDim.x) {
+    int run = chunk_base[(size_t)blockIdx.x * E + e];
+#pragma unroll
+    for (int w = 0; w < kWarps; ++w) {
+      const int c = rows[w][e];
+      rows[w][e] = run;
+      run += c;
+    }
+  }
+  __syncthreads();
+  int* base = rows[warp];
+  const unsigned lt = lanemask_lt();
+  int v[kIters];
+#pragma unroll
+  for (int it = 0; it < kIters; ++it) v[it] = load_id(ids, slice0 + it * 32 + lane, A, E, nullptr);
+#pragma unroll
+  for (int it = 0; it < kIters; ++it) {
+    const long long a = slice0 + it * 32 + lane;
+    const int id = v[it];
+    const unsigned m = __match_any_sync(0xffffffffu, id);
+    int rank = 0;
+    if (id >= 0) rank = base[id] + __popc(m & lt);
+    __syncwarp();
+    if (id >= 0 && lane == __ffs(m) - 1) base[id] += __popc(m);
+    __syncwarp();
+    if (id >= 0) {
+      int p = -1;
+      if (cap < 0 || rank < cap) {
+        p = offs[id] + rank;
+        perm_to_assign[p] = (int32_t)a;
+      }
+      assign_to_perm[a] = p;
+    } else if (a < A) {
+      assign_to_perm[a] = -1;  // id out of range (already reported)
+    }
+  }
+}
+
+// x_perm[p] = x[perm_to_assign[p] / K] for p < offsets[E]; 16-byte vectors.
+__global__ void __launch_bounds__(256) gather_rows_kernel(const uint4* __restrict__ x,
+                                                          const int32_t* __restrict__ p2a,
+                                                          const int32_t* __restrict__ n_kept_ptr,
+                                                          int K, int T, int vec_per_row,
+                                                          uint4* __restrict__ x_perm,
+                                                          unsigned* status) {
+  const long long n_kept = *n_kept_ptr;
+  const long long total = n_kept * vec_per_row;
+  for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < total;
+       i += (long long)gridDim.x * blockDim.x) {
+    const long long p = i / vec_per_row;
+    const int v = (int)(i - p * vec_per_row);
+    const int a = p2a[p];
+    const int t = a / K;
+    if (a < 0 || t >= T) {
+      report(status, MOE_ERR_DEVICE_INDEX);
+      continue;
+    }
+    x_perm[i] = x[(size_t)t * vec_per_row + v];
+  }
+}
+
+}  // namespace
+
+size_t permute_scratch_bytes(const moe_shape& s) {
+  const long long A = (long long)s.T * s.K;
+  const long long nchunks = (A + kChunk - 1) / kChunk;
+  return (size_t)(2 * nchunks * s.E) * sizeof(int32_t);
+}
+
+moe_status launch_permute(const moe_shape& s, const int32_t* ids, int32_t* counts,
+                          int32_t* offsets, int32_t* a2p, int32_t* p2a, const void* x,
+                          void* x_perm, void* scratch, cudaStream_t st) {
+  const long long A = (long long)s.T * s.K;
+  const int nchunks = (int)((A + kChunk - 1) / kChunk);
+  int32_t* chunk_counts = (int32_t*)scratch;
+  int32_t* chunk_base = chunk_counts + (size_t)nchunks * s.E;
+  const long long cap =
+      (s.capacity_factor > 0.f)
+          ? (long long)ceil((double)s.capacity_factor * (double)s.T * (double)s.K / (double)s.E)
+          : -1;
+  unsigned* status = device_status_ptr();
+  moe_status r;
+  if (nchunks > 0) {
+    launch_begin(K_HIST, st);
+    hist_kernel<<<nchunks, kWarps * 32, 0, st>>>(ids, A, s.E, chunk_counts, status);
+    if ((r = launch_end(K_HIST, st)) != MOE_OK) return r;
+  }
+  launch_begin(K_SCAN, st);
+  scan_kernel<<<1, kMaxE, 0, st>>>(chunk_counts, chunk_base, nchunks, s.E, cap, counts, offsets);
+  if ((r = launch_end(K_SCAN, st)) != MOE_OK) return r;
+  if (nchunks > 0) {
+    launch_begin(K_SCATTER, st);
+    scatter_kernel<<<nchunks, kWarps * 32, 0, st>>>(ids, A, s.E, cap, chunk_base, offsets, a2p,
+                                                    p2a, status);
+    if ((r = launch_end(K_SCATTER, st)) != MOE_OK) return r;
+  }
+  if (x != nullptr && x_perm != nullptr && A > 0) {
+    const int elem = (s.dtype == MOE_BF16) ? 2 : 4;
+    const int vec_per_row = s.d * elem / 16;
+    const long long total = A * vec_per_row;
+    long long blocks = (total + 255) / 256;
+    const long long cap_blocks = (long long)sm_count() * 16;
+    if (blocks > cap_blocks) blocks = cap_blocks;
+    launch_begin(K_GATHER, st);
+    gather_rows_kernel<<<(int)blocks, 256, 0, st>>>((const uint4*)x, p2a, offsets + s.E, s.K, s.T,
+                                                    vec_per_row, (uint4*)x_perm, status);
+    if ((r = launch_end(K_GATHER, st)) != MOE_OK) return r;
+  }
+  return MOE_OK;
+}
+
+}  // namespace moe

@@ -1,0 +1,219 @@
+// Router: logits = x W_r (+ bias), softmax, top-K with ties to the lower expert id.
+//
+// "Two upstream innovations of MoE: Routing-Free and OmniMoE" (chatdocs.ruinique.com),
+// section 1.1: x -> Router(x) -> Softmax -> TopK. "How AI chips support MoE", chapter 4,
+// section 4.2: the gate is a small dense linear map every token passes through; 4.3: the
+// top-K is a partial sort per token.
+//
+// One CTA owns TM tokens. Phase 1 is a register-tiled fp32 FMA GEMM (x tile and W_r tile
+// staged through shared memory, fp32 accumulation) that leaves the TM x E logits in shared
+// memory; with logits_in the tile is loaded instead. Phase 2 gives one warp per token: each
+// lane holds E/32 logits in registers and K rounds of a warp arg-max under the total order
+// (value descending, id ascending) pick the top-K. Selection compares fp32 logits, so +0 and
+// -0 tie. Weights: exp(l - l_max) over the selected (renormalised) or over all E.
+#include <math.h>
+
+#include "common.cuh"
+
+namespace moe {
+
+namespace {
+
+constexpr int kThreads = 256;
+constexpr int kDK = 64;
+
+template <typename Tin, int CT, int CPT, int RPT>
+__global__ void __launch_bounds__(kThreads) route_kernel(
+    const Tin* __restrict__ x, const Tin* __restrict__ w_r, const float* __restrict__ bias,
+    const float* __restrict__ logits_in, float* __restrict__ logits_out,
+    int32_t* __restrict__ topk_ids, float* __restrict__ topk_w, int T, int d, int E, int K,
+    int renorm) {
+  constexpr int RT = kThreads / CT;
+  constexpr int TM = RT * RPT;
+  constexpr int EP = CT * CPT;
+  constexpr int LDL = EP + 1;
+  constexpr int VPL = (EP + 31) / 32;
+  extern __shared__ float smem[];
+  float* lg = smem;  // [TM][LDL]
+  const int tid = threadIdx.x;
+  const int t0 = blockIdx.x * TM;
+
+  if (logits_in == nullptr) {
+    constexpr int VEC = Vec16<Tin>::N;
+    float* xs = lg + TM * LDL;          // [TM][kDK + 1]
+    float* ws = xs + TM * (kDK + 1);    // [kDK][EP]
+    const int tc = tid % CT, tr = tid / CT;
+    float acc[RPT][CPT];
+#pragma unroll
+    for (int i = 0; i < RPT; ++i)
+#pragma unroll
+      for (int j = 0; j < CPT; ++j) acc[i][j] = 0.f;
+
+    for (int k0 = 0; k0 < d; k0 += kDK) {
+      // x tile: TM rows x kDK columns, 16-byte vector loads (d is a multiple of kDK)
+      for (int i = tid; i < TM * (kDK / VEC); i += kThreads) {
+        const int r = i / (kDK / VEC), c = (i % (kDK / VEC)) * VEC;
+        const int t = t0 + r;
+        float f[VEC];
+        if (t < T) {
+          const uint4 u = *reinterpret_cast<const uint4*>(x + (size_t)t * d + k0 + c);
+          unpack16(u, f, Tin());
+        } else {
+#pragma unroll
+          for (int v = 0; v < VEC; ++v) f[v] = 0.f;
+        }
+#pragma unroll
+        for (int v = 0; v < VEC; ++v) xs[r * (kDK + 1) + c + v] = f[v];
+      }
+      // W_r tile: kDK rows x EP columns (zero past E)
+      for (int i = tid; i < kDK * EP; i += kThreads) {
+        const int r = i / EP, c = i % EP;
+        ws[i] = (c < E) ? to_f32(w_r[(size_t)(k0 + r) * E + c]) : 0.f;
+      }
+      __syncthreads();
+#pragma unroll 8
+      for (int k = 0; k < kDK; ++k) {
+        float a[RPT], b[CPT];
+#pragma unroll
+        for (int i = 0; i < RPT; ++i) a[i] = xs[(tr + i * RT) * (kDK + 1) + k];
+#pragma unroll
+        for (int j = 0; j < CPT; ++j) b[j] = ws[k * EP + tc + j * CT];
+#pragma unroll
+        for (int i = 0; i < RPT; ++i)
+#pragma unroll
+          for (int j = 0; j < CPT; ++j) acc[i][j] = fmaf(a[i], b[j], acc[i][j]);
+      }
+      __syncthreads();
+    }
+#pragma unroll
+    for (int i = 0; i < RPT; ++i)
+#pragma unroll
+      for (int j = 0; j < CPT; ++j) {
+        const int e = tc + j * CT;
+        const float bb = (bias != nullptr && e < E) ? bias[e] : 0.f;
+        lg[(tr + i * RT) * LDL + e] = acc[i][j] + bb;
+      }
+  } else {
+    for (int i = tid; i < TM * E; i += kThreads) {
+      const int r = i / E, c = i % E;
+      const int t = t0 + r;
+      lg[r * LDL + c] = (t < T) ? logits_in[(size_t)t * E + c] : 0.f;
+    }
+  }
+  __syncthreads();
+
+  if (logits_out != nullptr && logits_out != logits_in) {
+    for (int i = tid; i < TM * E; i += kThreads) {
+      const int r = i / E, c = i % E;
+      const int t = t0 + r;
+      if (t < T) logits_out[(size_t)t * E + c] = lg[r * LDL + c];
+    }
+  }
+
+  const int warp = tid >> 5, lane = tid & 31;
+  for (int r = warp; r < TM; r += kThreads / 32) {
+    const int t = t0 + r;
+    if (t >= T) break;
+    float v[VPL];
+    bool taken[VPL];
+#pragma unroll
+    for (int j = 0; j < VPL; ++j) {
+      const int e = lane + 32 * j;
+      v[j] = (e < E) ? lg[r * LDL + e] : -INFINITY;
+      taken[j] = (e >= E);
+    }
+    float vmax = 0.f, selv = 0.f;
+    int sele = 0;
+    for (int k = 0; k < K; ++k) {
+      float bv = -INFINITY;
+      int be = 0x7fffffff;
+#pragma unroll
+      for (int j = 0; j < VPL; ++j) {
+        const int e = lane + 32 * j;
+        if (!taken[j] && (v[j] > bv || (v[j] == bv && e < be))) {
+          bv = v[j];
+          be = e;
+        }
+      }
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) {
+        const float ov = __shfl_xor_sync(0xffffffffu, bv, off);
+        const int oe = __shfl_xor_sync(0xffffffffu, be, off);
+        if (ov > bv || (ov == bv && oe < be)) {
+          bv = ov;
+          be = oe;
+        }
+      }
+#pragma unroll
+      for (int j = 0; j < VPL; ++j)
+        if (lane + 32 * j == be) taken[j] = true;
+      if (k == 0) vmax = bv;
+      if (lane == k) {
+        selv = bv;
+        sele = be;
+      }
+    }
+    const float ex = (lane < K) ? expf(selv - vmax) : 0.f;
+    float den;
+    if (renorm) {
+      den = ex;
+    } else {
+      den = 0.f;
+#pragma unroll
+      for (int j = 0; j < VPL; ++j)
+        if (lane + 32 * j < E) den += expf(v[j] - vmax);
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) den += __shfl_xor_sync(0xffffffffu, den, off);
+    if (lane < K) {
+      topk_ids[(size_t)t * K + lane] = sele;
+      topk_w[(size_t)t * K + lane] = ex / den;
+    }
+  }
+}
+
+template <typename Tin, int CT, int CPT, int RPT>
+moe_status launch_route_t(const moe_shape& s, const void* x, const void* w_r, const float* bias,
+                          const float* logits_in, float* logits_out, int32_t* ids, float* w,
+                          cudaStream_t st) {
+  constexpr int RT = kThreads / CT;
+  constexpr int TM = RT * RPT;
+  constexpr int EP = CT * CPT;
+  size_t smem = (size_t)TM * (EP + 1) * sizeof(float);
+  if (logits_in == nullptr) smem += ((size_t)TM * (kDK + 1) + (size_t)kDK * EP) * sizeof(float);
+  auto kern = route_kernel<Tin, CT, CPT, RPT>;
+  if (smem > 48 * 1024) {
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
+        cudaSuccess)
+      return MOE_ERR_CUDA;
+  }
+  const int grid = (s.T + TM - 1) / TM;
+  if (grid == 0) return MOE_OK;
+  launch_begin(K_ROUTE, st);
+  kern<<<grid, kThreads, smem, st>>>((const Tin*)x, (const Tin*)w_r, bias, logits_in, logits_out,
+                                     ids, w, s.T, s.d, s.E, s.K, s.renormalize);
+  return launch_end(K_ROUTE, st);
+}
+
+template <typename Tin>
+moe_status launch_route_dt(const moe_shape& s, const void* x, const void* w_r, const float* bias,
+                           const float* li, float* lo, int32_t* ids, float* w, cudaStream_t st) {
+  if (s.E <= 8) return launch_route_t<Tin, 8, 1, 2>(s, x, w_r, bias, li, lo, ids, w, st);
+  if (s.E <= 16) return launch_route_t<Tin, 16, 1, 4>(s, x, w_r, bias, li, lo, ids, w, st);
+  if (s.E <= 32) return launch_route_t<Tin, 32, 1, 8>(s, x, w_r, bias, li, lo, ids, w, st);
+  if (s.E <= 64) return launch_route_t<Tin, 32, 2, 8>(s, x, w_r, bias, li, lo, ids, w, st);
+  if (s.E <= 128) return launch_route_t<Tin, 32, 4, 4>(s, x, w_r, bias, li, lo, ids, w, st);
+  return launch_route_t<Tin, 32, 8, 2>(s, x, w_r, bias, li, lo, ids, w, st);
+}
+
+}  // namespace
+
+moe_status launch_route(const moe_shape& s, const void* x, const void* w_r, const float* bias,
+                        const float* logits_in, float* logits_out, int32_t* ids, float* w,
+                        cudaStream_t st) {
+  if (s.dtype == MOE_BF16)
+    return launch_route_dt<bf16>(s, x, w_r, bias, logits_in, logits_out, ids, w, st);
+  return launch_route_dt<float>(s, x, w_r, bias, logits_in, logits_out, ids, w, st);
+}
+
+}  // namespace moe
