@@ -25,6 +25,8 @@
  *    enqueued. A launch failure returns MOE_ERR_CUDA. Faults found on the
  *    device (an expert id out of range, a bounded wait that ran out) set a
  *    device status word that moe_get_device_status() reads and clears.
+ *  - T = 0 is valid: nothing is read or written (moe_permute still zeroes counts
+ *    and offsets) and data pointers may be NULL.
  *  - Thread safety: calls are reentrant; the only global state is the device
  *    status word, a per-device cache of SM counts and the opt-in profiler.
  */
@@ -60,8 +62,8 @@ typedef enum { MOE_F32 = 0, MOE_BF16 = 1 } moe_dtype;
  * overflow is dropped). renormalize != 0: top-K weights are the softmax
  * restricted to the K selected experts (they sum to 1); 0: plain softmax
  * over all E experts, read at the selected ones. Limits: 1 <= K <= E <= 256,
- * K <= 32, T >= 0. MOE_BF16 also needs d % 64 == 0 and n % 64 == 0 (TMA
- * tiles); MOE_F32 needs d % 4 == 0 and n % 4 == 0. */
+ * K <= 32, T >= 0, T * K < 2^31, d % 64 == 0 (router tiles, TMA boxes);
+ * n % 64 == 0 for MOE_BF16 and n % 16 == 0 for MOE_F32. */
 typedef struct {
   int32_t T, d, E, K, n;
   float capacity_factor;
@@ -90,7 +92,8 @@ size_t moe_forward_workspace_size(const moe_shape* shape);
  *
  *   x          [T, d]  device, dtype; ignored when logits_in != NULL
  *   w_r        [d, E]  device, dtype; ignored when logits_in != NULL
- *   bias       [E]     device fp32 or NULL; added to every token's logits
+ *   bias       [E]     device fp32 or NULL; added to every token's x W_r
+ *                      (not to logits_in)
  *   logits_in  [T, E]  device fp32 or NULL: use these logits instead of x W_r
  *   logits_out [T, E]  device fp32 or NULL: receives the logits the top-K saw
  *                      (x W_r + bias, or a copy of logits_in)

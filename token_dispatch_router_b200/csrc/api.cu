@@ -196,10 +196,10 @@ moe_status moe_route(const moe_shape* s, const void* x, const void* w_r, const f
                      moe_stream_t stream) {
   moe_status r = check_shape(s, logits_in == nullptr, false);
   if (r != MOE_OK) return r;
+  if (s->T == 0) return MOE_OK;  // nothing to read or write; pointers may be NULL
   if (topk_ids == nullptr || topk_w == nullptr) return MOE_ERR_INVALID_ARG;
   if (logits_in == nullptr && (x == nullptr || w_r == nullptr)) return MOE_ERR_INVALID_ARG;
   if (logits_in == nullptr && !aligned16(x)) return MOE_ERR_INVALID_ARG;
-  if (s->T == 0) return MOE_OK;
   return launch_route(*s, x, w_r, bias, logits_in, logits_out, topk_ids, topk_w,
                       (cudaStream_t)stream);
 }
@@ -211,6 +211,14 @@ moe_status moe_permute(const moe_shape* s, const int32_t* topk_ids, int32_t* cou
   const bool gather = (x != nullptr && x_perm != nullptr);
   moe_status r = check_shape(s, gather, false);
   if (r != MOE_OK) return r;
+  if (s->T == 0) {  // no assignments: only counts and offsets (all zero) are written
+    if (counts == nullptr || offsets == nullptr) return MOE_ERR_INVALID_ARG;
+    const cudaStream_t st = (cudaStream_t)stream;
+    if (cudaMemsetAsync(counts, 0, sizeof(int32_t) * s->E, st) != cudaSuccess ||
+        cudaMemsetAsync(offsets, 0, sizeof(int32_t) * (s->E + 1), st) != cudaSuccess)
+      return MOE_ERR_CUDA;
+    return MOE_OK;
+  }
   if (topk_ids == nullptr || counts == nullptr || offsets == nullptr || assign_to_perm == nullptr ||
       perm_to_assign == nullptr)
     return MOE_ERR_INVALID_ARG;
@@ -227,12 +235,12 @@ moe_status moe_grouped_ffn(const moe_shape* s, const void* x, const int32_t* off
                            const void* w_down, void* a_act, void* y_perm, moe_stream_t stream) {
   moe_status r = check_shape(s, true, true);
   if (r != MOE_OK) return r;
+  if (s->T == 0) return MOE_OK;
   if (!x || !offsets || !perm_to_assign || !w_gate || !w_up || !w_down || !a_act || !y_perm)
     return MOE_ERR_INVALID_ARG;
   if (!aligned16(x) || !aligned16(w_gate) || !aligned16(w_up) || !aligned16(w_down) ||
       !aligned16(a_act) || !aligned16(y_perm))
     return MOE_ERR_INVALID_ARG;
-  if (s->T == 0) return MOE_OK;
   if (s->dtype == MOE_BF16)
     return launch_ffn_tc(*s, x, offsets, perm_to_assign, w_gate, w_up, w_down, a_act, y_perm,
                          (cudaStream_t)stream);
@@ -244,6 +252,7 @@ moe_status moe_combine(const moe_shape* s, const void* y_perm, const int32_t* as
                        const float* topk_w, void* out, moe_stream_t stream) {
   moe_status r = check_shape(s, true, false);
   if (r != MOE_OK) return r;
+  if (s->T == 0) return MOE_OK;
   if (!y_perm || !assign_to_perm || !topk_w || !out) return MOE_ERR_INVALID_ARG;
   if (!aligned16(y_perm) || !aligned16(out)) return MOE_ERR_INVALID_ARG;
   return launch_combine(*s, y_perm, assign_to_perm, topk_w, out, (cudaStream_t)stream);
@@ -255,12 +264,12 @@ moe_status moe_forward(const moe_shape* s, const void* x, const void* w_r, const
                        moe_stream_t stream) {
   moe_status r = check_shape(s, true, true);
   if (r != MOE_OK) return r;
+  if (s->T == 0) return MOE_OK;
   if (!x || (!w_r && !logits_in) || !w_gate || !w_up || !w_down || !out) return MOE_ERR_INVALID_ARG;
   moe_workspace_layout L;
   layout_of(*s, &L);
   if (workspace == nullptr || ws_bytes < L.total) return MOE_ERR_WORKSPACE;
   if (((uintptr_t)workspace & 255) != 0) return MOE_ERR_INVALID_ARG;
-  if (s->T == 0) return MOE_OK;
   uint8_t* ws = (uint8_t*)workspace;
   const cudaStream_t st = (cudaStream_t)stream;
   float* logits = (float*)(ws + L.logits);
