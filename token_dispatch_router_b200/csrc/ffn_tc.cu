@@ -8,11 +8,17 @@
 //                         chip (here in TMEM) before anything goes back to HBM.
 //
 // One persistent kernel per GEMM (grid = #SMs, one CTA per SM), warp-specialised:
-//   warp 0     TMA producer: A tile 128 x 64 bf16 (gate/up: 32 `tile::gather4` loads of
-//              four x rows each, row = perm_to_assign[p] / K; down: one tiled load of
-//              a_act rows) and the B tile 64 x 256 bf16 as four 64 x 64 boxes of the
-//              expert's weights, all into a 4-stage shared-memory ring (48 KB a stage,
-//              128-byte swizzle) signalled through mbarrier transaction counts;
+//   warp 0     TMA producer: the B tile 64 x 256 bf16 as four 64 x 64 boxes of the
+//              expert's weights (and, for the down GEMM, the A tile: one tiled load of
+//              128 a_act rows) into a 4-stage shared-memory ring (48 KB a stage, 128-byte
+//              swizzle) signalled through mbarrier transaction counts;
+//   warps 6-9  (gate/up only) the gathered A tile 128 x 64 bf16: each lane copies 16-byte
+//              pieces of x rows, row = perm_to_assign[p] / K, with cp.async straight into
+//              the 128-byte-swizzled layout the MMA descriptor expects, and signals the
+//              stage with cp.async.mbarrier.arrive.noinc. Eight lanes cover one 128-byte
+//              row segment, so each warp instruction moves four whole segments. (The
+//              tensor-map gather4 form measured 2.6x slower here: 128 row requests per
+//              stage starve the tensor pipe.)
 //   warp 1     TMEM allocator and MMA issuer: one thread issues tcgen05.mma (M=128,
 //              N=256, K=16, bf16 in, fp32 accumulate) four times per stage and commits
 //              each stage back to the producer; two 256-column accumulators in TMEM
@@ -38,7 +44,10 @@ constexpr int A_BYTES = BM * BK * 2;           // 16 KB
 constexpr int B_CHUNK = BK * 64 * 2;           // one 64 x 64 bf16 box, 8 KB
 constexpr int B_BYTES = 4 * B_CHUNK;           // 32 KB
 constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
-constexpr int THREADS = 192;
+constexpr int THREADS_DOWN = 192;   // producer, MMA, 4 epilogue warps
+constexpr int THREADS_GATEUP = 320; // + 4 gather warps
+constexpr int GATHER_WARP0 = 6;
+constexpr int GATHER_THREADS = 128;
 constexpr uint32_t TMEM_COLS = 512;
 constexpr int MAXE = 256;
 constexpr int SMEM_TAIL = 4096;  // barriers, TMEM slot, abort flag, tile table
@@ -53,6 +62,8 @@ constexpr uint32_t IDESC = (1u << 4) | (1u << 7) | (1u << 10) | (1u << 16) |
 struct GemmArgs {
   const int32_t* offsets;
   const int32_t* p2a;
+  const uint8_t* x;  // gate/up: token rows gathered by cp.async
+  long long x_row_bytes;
   bf16* out;
   int ld_out;    // elements per output row
   int n_out;     // valid output columns
@@ -120,14 +131,20 @@ __device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* map
       "l"((uint64_t)map), "r"(c0), "r"(c1), "r"(c2), "r"(bar)
       : "memory");
 }
-// Four rows r0..r3 of a 2-D map (box one row high), columns [c0, c0 + box) -> 4 x 128 B.
-__device__ __forceinline__ void tma_gather4(uint32_t dst, const CUtensorMap* map, int c0, int r0,
-                                            int r1, int r2, int r3, uint32_t bar) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes"
-      " [%0], [%1, {%2, %3, %4, %5, %6}], [%7];" ::"r"(dst),
-      "l"((uint64_t)map), "r"(c0), "r"(r0), "r"(r1), "r"(r2), "r"(r3), "r"(bar)
-      : "memory");
+// 16 bytes global -> shared, cached in L2 only; completion tracked per thread.
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src) {
+  asm volatile("cp.async.cg.shared.global.L2::128B [%0], [%1], 16;" ::"r"(dst), "l"(src)
+               : "memory");
+}
+// The barrier receives one arrival once every cp.async this thread issued so far landed.
+__device__ __forceinline__ void cp_async_arrive_noinc(uint32_t bar) {
+  asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(bar) : "memory");
+}
+__device__ __forceinline__ void cp_async_wait_all() {
+  asm volatile("cp.async.wait_all;" ::: "memory");
+}
+__device__ __forceinline__ void fence_proxy_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 __device__ __forceinline__ void tc_fence_before() {
   asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
@@ -197,7 +214,7 @@ __device__ __forceinline__ Tile decode_tile(int w, const int* s_off, const int* 
 }
 
 template <bool GATEUP>
-__global__ void __launch_bounds__(THREADS, 1)
+__global__ void __launch_bounds__(GATEUP ? THREADS_GATEUP : THREADS_DOWN, 1)
     grouped_gemm_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB0,
                     const __grid_constant__ CUtensorMap tmB1, const GemmArgs g) {
   extern __shared__ uint8_t smem_raw[];
@@ -217,10 +234,14 @@ __global__ void __launch_bounds__(THREADS, 1)
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int E = g.E;
+  constexpr int NTHREADS = GATEUP ? THREADS_GATEUP : THREADS_DOWN;
+  // full[s]: the TMA thread's expect_tx arrival (+ one noinc arrival per gather thread)
+  constexpr uint32_t FULL_COUNT = GATEUP ? 1 + GATHER_THREADS : 1;
+  constexpr uint32_t TMA_BYTES = GATEUP ? B_BYTES : STAGE_BYTES;
 
   if (tid == 0) {
     for (int s = 0; s < STAGES; ++s) {
-      mbar_init(saddr(&full[s]), 1);
+      mbar_init(saddr(&full[s]), FULL_COUNT);
       mbar_init(saddr(&empty[s]), 1);
     }
     for (int b = 0; b < 2; ++b) {
@@ -238,7 +259,7 @@ __global__ void __launch_bounds__(THREADS, 1)
                  : "memory");
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
   }
-  for (int i = tid; i <= E; i += THREADS) s_off[i] = g.offsets[i];
+  for (int i = tid; i <= E; i += NTHREADS) s_off[i] = g.offsets[i];
   __syncthreads();
   if (warp == 0) {  // tile table: s_mt[e] = ceil(kept_e / BM); s_cum = n_tiles * prefix
     constexpr int PER = MAXE / 32;
@@ -281,21 +302,6 @@ __global__ void __launch_bounds__(THREADS, 1)
     uint32_t issued_mask = 0, issued_par = 0;  // per stage: ever issued, parity of last issue
     for (int w = blockIdx.x; w < total; w += gridDim.x) {
       const Tile t = decode_tile(w, s_off, s_cum, s_mt, E, g.out_tile);
-      int tok[4] = {0, 0, 0, 0};
-      if (GATEUP) {
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          const int r = lane * 4 + j;
-          const int p = t.m0 + (r < t.rows ? r : 0);  // padding rows reuse the tile's first row
-          const int a = g.p2a[p];
-          int tk = a / g.K;
-          if (a < 0 || tk >= g.T) {
-            report(g.status, MOE_ERR_DEVICE_INDEX);
-            tk = 0;
-          }
-          tok[j] = tk;
-        }
-      }
       bool ok = true;
       for (int kb = 0; kb < g.kblocks; ++kb) {
         int w_ok = 0;
@@ -306,15 +312,11 @@ __global__ void __launch_bounds__(THREADS, 1)
           break;
         }
         const uint32_t fb = saddr(&full[stage]);
-        if (lane == 0) mbar_expect_tx(fb, STAGE_BYTES);
+        if (lane == 0) mbar_expect_tx(fb, TMA_BYTES);
         __syncwarp();
         const uint32_t a_dst = saddr(ring + stage * STAGE_BYTES);
         const uint32_t b_dst = a_dst + A_BYTES;
-        if (GATEUP) {
-          tma_gather4(a_dst + lane * 4 * 128, &tmA, kb * BK, tok[0], tok[1], tok[2], tok[3], fb);
-        } else if (lane == 0) {
-          tma_load_2d(a_dst, &tmA, kb * BK, t.m0, fb);
-        }
+        if (!GATEUP && lane == 0) tma_load_2d(a_dst, &tmA, kb * BK, t.m0, fb);
         if (lane < 4) {
           if (GATEUP) {
             const CUtensorMap* mp = (lane < 2) ? &tmB0 : &tmB1;
@@ -360,6 +362,7 @@ __global__ void __launch_bounds__(THREADS, 1)
             ok = false;
             break;
           }
+          if (GATEUP) fence_proxy_async_smem();  // cp.async (generic) writes -> MMA reads
           tc_fence_after();
           const uint32_t a_addr = saddr(ring + stage * STAGE_BYTES);
           const uint32_t b_addr = a_addr + A_BYTES;
@@ -383,6 +386,51 @@ __global__ void __launch_bounds__(THREADS, 1)
       while (!mbar_try(saddr(done), 0) && globaltimer_ns() - t0 < limit) {
       }
     }
+  } else if (GATEUP && warp >= GATHER_WARP0) {
+    // ------------------------------------------------------------ A gather (warps 6-9)
+    const int gw = warp - GATHER_WARP0;  // rows [32 gw, 32 gw + 32)
+    const int c = lane & 7;              // 16-byte piece of the 128-byte row segment
+    const int rg = lane >> 3;            // rows 32 gw + rg + 4 i, i < 8
+    int stage = 0;
+    uint32_t phase = 0;
+    for (int w = blockIdx.x; w < total; w += gridDim.x) {
+      const Tile t = decode_tile(w, s_off, s_cum, s_mt, E, g.out_tile);
+      const uint8_t* src[8];
+      uint32_t dst[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const int r = gw * 32 + rg + 4 * i;
+        const int p = t.m0 + (r < t.rows ? r : 0);  // padding rows reuse the tile's first row
+        const int a = g.p2a[p];
+        int tk = a / g.K;
+        if (a < 0 || tk >= g.T) {
+          report(g.status, MOE_ERR_DEVICE_INDEX);
+          tk = 0;
+        }
+        src[i] = g.x + (size_t)tk * g.x_row_bytes + c * 16;
+        dst[i] = (uint32_t)(r * 128 + ((c ^ (r & 7)) << 4));  // 128-byte swizzle
+      }
+      bool ok = true;
+      for (int kb = 0; kb < g.kblocks; ++kb) {
+        int w_ok = 0;
+        if (lane == 0) w_ok = mbar_wait(saddr(&empty[stage]), phase ^ 1u, abort_flag, g, limit);
+        w_ok = __shfl_sync(0xffffffffu, w_ok, 0);
+        if (!w_ok) {
+          ok = false;
+          break;
+        }
+        const uint32_t a_dst = saddr(ring + stage * STAGE_BYTES);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) cp_async16(a_dst + dst[i], src[i] + (size_t)kb * (BK * 2));
+        cp_async_arrive_noinc(saddr(&full[stage]));
+        if (++stage == STAGES) {
+          stage = 0;
+          phase ^= 1u;
+        }
+      }
+      if (!ok) break;
+    }
+    cp_async_wait_all();  // nothing of ours lands after the CTA exits
   } else {
     // ------------------------------------------------------------ epilogue (warps 2-5)
     const int q = warp & 3;  // TMEM lanes 32q..32q+31 are reachable from this warp
@@ -500,7 +548,7 @@ moe_status run_gemm(const CUtensorMap& a, const CUtensorMap& b0, const CUtensorM
       cudaSuccess)
     return MOE_ERR_CUDA;
   launch_begin(kid, st);
-  kern<<<sm_count(), THREADS, SMEM_BYTES, st>>>(a, b0, b1, args);
+  kern<<<sm_count(), GATEUP ? THREADS_GATEUP : THREADS_DOWN, SMEM_BYTES, st>>>(a, b0, b1, args);
   return launch_end(kid, st);
 }
 
@@ -538,12 +586,7 @@ moe_status launch_ffn_tc(const moe_shape& s, const void* x, const int32_t* offse
   const long long A = (long long)s.T * s.K;
   if (A == 0) return MOE_OK;
   const uint64_t T = s.T, d = s.d, n = s.n, E = s.E;
-  CUtensorMap mx, mg, mu, ma, md;
-  {
-    const uint64_t dims[2] = {d, T}, str[1] = {d * 2};
-    const uint32_t box[2] = {64, 1};
-    if (!make_map(&mx, x, 2, dims, str, box)) return MOE_ERR_CUDA;
-  }
+  CUtensorMap mg, mu, ma, md;
   {
     const uint64_t dims[3] = {n, d, E}, str[2] = {n * 2, d * n * 2};
     const uint32_t box[3] = {64, 64, 1};
@@ -563,6 +606,8 @@ moe_status launch_ffn_tc(const moe_shape& s, const void* x, const int32_t* offse
   GemmArgs ga;
   ga.offsets = offsets;
   ga.p2a = p2a;
+  ga.x = (const uint8_t*)x;
+  ga.x_row_bytes = (long long)s.d * 2;
   ga.E = s.E;
   ga.K = s.K;
   ga.T = s.T;
@@ -575,7 +620,7 @@ moe_status launch_ffn_tc(const moe_shape& s, const void* x, const int32_t* offse
   ga.out_tile = 128;
   ga.n_tiles = (s.n + 127) / 128;
   ga.kblocks = s.d / BK;
-  moe_status r = run_gemm<true>(mx, mg, mu, ga, st, K_GATEUP_TC);
+  moe_status r = run_gemm<true>(mg, mg, mu, ga, st, K_GATEUP_TC);
   if (r != MOE_OK) return r;
 
   GemmArgs gd = ga;
