@@ -26,6 +26,9 @@ moe_status launch_ffn_tc(const moe_shape& s, const void* x, const int32_t* offse
 moe_status launch_combine(const moe_shape& s, const void* y_perm, const int32_t* a2p,
                           const float* topk_w, void* out, cudaStream_t st);
 moe_status launch_selftest_timeout(uint64_t limit_ns, cudaStream_t st);
+bool route_tc_supported(const moe_shape& s);
+moe_status launch_route_tc(const moe_shape& s, const void* x, const void* w_r, const float* bias,
+                           float* logits_out, int32_t* ids, float* w, cudaStream_t st);
 
 // ------------------------------------------------------------------ device state
 __device__ unsigned int g_device_status;
@@ -68,7 +71,8 @@ int sm_count() {
 namespace {
 const char* kKernelNames[K_COUNT] = {
     "route",        "hist",          "scan",           "scatter",     "gather_rows", "gateup_tc",
-    "down_tc",      "gateup_simt",   "down_simt",      "combine",     "selftest_timeout"};
+    "down_tc",      "gateup_simt",   "down_simt",      "combine",     "selftest_timeout",
+    "route_tc"};
 
 struct ProfRec {
   int kid;
@@ -200,6 +204,8 @@ moe_status moe_route(const moe_shape* s, const void* x, const void* w_r, const f
   if (topk_ids == nullptr || topk_w == nullptr) return MOE_ERR_INVALID_ARG;
   if (logits_in == nullptr && (x == nullptr || w_r == nullptr)) return MOE_ERR_INVALID_ARG;
   if (logits_in == nullptr && !aligned16(x)) return MOE_ERR_INVALID_ARG;
+  if (logits_in == nullptr && route_tc_supported(*s) && aligned16(w_r))
+    return launch_route_tc(*s, x, w_r, bias, logits_out, topk_ids, topk_w, (cudaStream_t)stream);
   return launch_route(*s, x, w_r, bias, logits_in, logits_out, topk_ids, topk_w,
                       (cudaStream_t)stream);
 }

@@ -84,6 +84,7 @@ enum KernelId {
   K_DOWN_SIMT,
   K_COMBINE,
   K_SELFTEST,
+  K_ROUTE_TC,
   K_COUNT
 };
 

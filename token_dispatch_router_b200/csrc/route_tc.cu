@@ -1,0 +1,442 @@
+// Router on the tensor cores for bf16 shapes: logits = x W_r (+ bias) with tcgen05, then
+// softmax and top-K in the epilogue, one token per thread.
+//
+// "How AI chips support MoE", chapter 4, section 4.2: the gate is a small dense linear map
+// that every token passes through and that the experts wait on; section 4.3: top-K is a
+// partial sort per token. "Two upstream innovations of MoE: Routing-Free and OmniMoE",
+// section 1.1: Router -> Softmax -> TopK.
+//
+// The router GEMM (M = T tokens, N = E experts, K = d) has an arithmetic intensity of about
+// E FLOP per byte of x, so at E >= 32 fp32 FMA units cannot keep up with HBM; tcgen05 can.
+// Layout: one 128-token tile per cluster of S CTAs (S <= 8). The S CTAs split the d
+// contraction (k-blocks of 64); each accumulates its partial 128 x N tile in TMEM
+// (N = E rounded up to 16, fp32), copies it column-major into its shared memory, and
+// after a cluster barrier CTA rank 0 adds the partials of ranks 0..S-1 in that fixed
+// order through distributed shared memory (deterministic, no atomics, no global
+// scratch). Rank 0's 128 threads then own one token each: + bias, optional logits
+// store, register top-K by insertion (value descending, ties to the lower id, +0 == -0),
+// softmax weights over the selected (renormalised) or over all E with an online sum.
+// Roles per CTA (128 threads): warp 0 lane 0 issues the TMA loads (x tile 128 x 64 and
+// the W_r tile 64 x N, 128-byte swizzle), warp 1 lane 0 issues the MMAs (M=128, N, K=16,
+// A K-major, B MN-major), then all four warps read TMEM (warp w owns lanes 32w..32w+31).
+// Every mbarrier wait is bounded; on expiry the status word records MOE_ERR_TIMEOUT.
+#include <math.h>
+
+#include "common.cuh"
+
+namespace moe {
+
+namespace {
+
+constexpr int RBM = 128, RBK = 64, RSTAGES = 4;
+constexpr int RA_BYTES = RBM * RBK * 2;  // 16 KB
+constexpr int RB_CHUNK = RBK * 64 * 2;   // 8 KB: 64 k-rows x 64 experts
+constexpr int R_THREADS = 128;
+constexpr int KMAX = 8;
+
+struct RouteArgs {
+  const float* bias;
+  float* logits_out;
+  int32_t* topk_ids;
+  float* topk_w;
+  int T, E, K, renorm, kblocks, S;
+  unsigned* status;
+  unsigned long long limit_ns;
+};
+
+__device__ __forceinline__ uint32_t saddr(const void* p) {
+  return (uint32_t)__cvta_generic_to_shared(p);
+}
+__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
+}
+__device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes)
+               : "memory");
+}
+__device__ __forceinline__ bool mbar_try(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}\n"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, unsigned* status,
+                                          uint64_t limit) {
+  if (mbar_try(bar, parity)) return true;
+  const uint64_t t0 = globaltimer_ns();
+  while (!mbar_try(bar, parity)) {
+    if (globaltimer_ns() - t0 > limit) {
+      report(status, MOE_ERR_TIMEOUT);
+      return false;
+    }
+  }
+  return true;
+}
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, int c0, int c1,
+                                            uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%2, %3}], [%4];" ::"r"(dst),
+      "l"((uint64_t)map), "r"(c0), "r"(c1), "r"(bar)
+      : "memory");
+}
+__device__ __forceinline__ uint64_t desc_sw128(uint32_t addr, uint32_t lbo, uint32_t sbo) {
+  return (uint64_t)((addr >> 4) & 0x3FFFu) | ((uint64_t)((lbo >> 4) & 0x3FFFu) << 16) |
+         ((uint64_t)((sbo >> 4) & 0x3FFFu) << 32) | (1ull << 46) | (2ull << 61);
+}
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&v)[16]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+      "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15}, [%16];"
+      : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]),
+        "=r"(v[7]), "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]),
+        "=r"(v[14]), "=r"(v[15])
+      : "r"(taddr));
+}
+__device__ __forceinline__ uint32_t cluster_rank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+__device__ __forceinline__ uint32_t cluster_id_x() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%clusterid.x;" : "=r"(r));
+  return r;
+}
+__device__ __forceinline__ void cluster_sync() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::
+                   : "memory");
+}
+// Address of the same shared-memory location in CTA `rank` of this cluster.
+__device__ __forceinline__ uint32_t map_rank(uint32_t local_addr, uint32_t rank) {
+  uint32_t remote;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(remote) : "r"(local_addr), "r"(rank));
+  return remote;
+}
+__device__ __forceinline__ float ld_dsmem(uint32_t remote_addr) {
+  float v;
+  asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(remote_addr) : "memory");
+  return v;
+}
+
+// Insert (v, e) into the descending list (ids arrive in ascending order, so an equal value
+// goes behind the ones already held: ties keep the lower id).
+__device__ __forceinline__ void topk_insert(float (&bv)[KMAX], int (&be)[KMAX], int& cnt, int K,
+                                            float v, int e) {
+  float kth = 0.f;  // the K-th value once the list is full (unrolled select: no local memory)
+#pragma unroll
+  for (int j = 0; j < KMAX; ++j)
+    if (j == K - 1) kth = bv[j];
+  if (cnt == K && !(v > kth)) return;
+  float cv = v;
+  int ce = e;
+  bool placed = false;
+#pragma unroll
+  for (int j = 0; j < KMAX; ++j) {
+    if (j < K && !placed) {
+      if (j >= cnt) {
+        bv[j] = cv;
+        be[j] = ce;
+        placed = true;
+      } else if (cv > bv[j]) {
+        const float tv = bv[j];
+        const int te = be[j];
+        bv[j] = cv;
+        be[j] = ce;
+        cv = tv;
+        ce = te;
+      }
+    }
+  }
+  if (cnt < K) ++cnt;
+}
+
+template <int N>  // MMA N = E rounded up to 16
+__global__ void __launch_bounds__(R_THREADS) route_tc_kernel(const __grid_constant__ CUtensorMap tmX,
+                                                             const __grid_constant__ CUtensorMap tmW,
+                                                             const RouteArgs g) {
+  constexpr int NCH = (N + 63) / 64;         // B chunks of 64 experts
+  constexpr int B_BYTES = NCH * RB_CHUNK;
+  constexpr int STAGE = RA_BYTES + B_BYTES;
+  constexpr uint32_t TCOLS = N <= 32 ? 32 : (N <= 64 ? 64 : (N <= 128 ? 128 : 256));
+  constexpr uint32_t IDESC = (1u << 4) | (1u << 7) | (1u << 10) | (1u << 16) |
+                             ((uint32_t)(N >> 3) << 17) | ((uint32_t)(RBM >> 4) << 24);
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* base = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+  uint8_t* ring = base;
+  uint64_t* bars = (uint64_t*)(base + RSTAGES * STAGE);
+  uint64_t* full = bars;
+  uint64_t* empty = bars + RSTAGES;
+  uint64_t* accf = bars + 2 * RSTAGES;
+  uint32_t* tmem_slot = (uint32_t*)(bars + 2 * RSTAGES + 1);
+  float* part = (float*)ring;  // after the mainloop: this CTA's partial, [N][128]
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const uint32_t rank = cluster_rank();
+  const int tile = (int)cluster_id_x();
+  const int S = g.S;
+  const int kb0 = (int)(rank * g.kblocks / S), kb1 = (int)((rank + 1) * g.kblocks / S);
+
+  if (tid == 0) {
+    for (int s = 0; s < RSTAGES; ++s) {
+      mbar_init(saddr(&full[s]), 1);
+      mbar_init(saddr(&empty[s]), 1);
+    }
+    mbar_init(saddr(accf), 1);
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  if (warp == 1) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                     saddr(tmem_slot)),
+                 "r"(TCOLS)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  }
+  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+  __syncthreads();
+  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+  const uint32_t tmem = *tmem_slot;
+  bool ok = true;
+
+  if (warp == 0 && lane == 0) {
+    int stage = 0;
+    uint32_t phase = 0;
+    for (int kb = kb0; kb < kb1; ++kb) {
+      if (!mbar_wait(saddr(&empty[stage]), phase ^ 1u, g.status, g.limit_ns)) {
+        ok = false;
+        break;
+      }
+      const uint32_t fb = saddr(&full[stage]);
+      mbar_expect_tx(fb, STAGE);
+      const uint32_t a = saddr(ring + stage * STAGE);
+      tma_load_2d(a, &tmX, kb * RBK, tile * RBM, fb);
+#pragma unroll
+      for (int c = 0; c < NCH; ++c) tma_load_2d(a + RA_BYTES + c * RB_CHUNK, &tmW, c * 64, kb * RBK, fb);
+      if (++stage == RSTAGES) {
+        stage = 0;
+        phase ^= 1u;
+      }
+    }
+  } else if (warp == 1 && lane == 0) {
+    int stage = 0;
+    uint32_t phase = 0;
+    for (int kb = kb0; kb < kb1; ++kb) {
+      if (!mbar_wait(saddr(&full[stage]), phase, g.status, g.limit_ns)) {
+        ok = false;
+        break;
+      }
+      asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+      const uint32_t a = saddr(ring + stage * STAGE);
+#pragma unroll
+      for (int kk = 0; kk < RBK / 16; ++kk) {
+        const uint64_t ad = desc_sw128(a + kk * 32, 16, 1024);
+        const uint64_t bd = desc_sw128(a + RA_BYTES + kk * 2048, RB_CHUNK, 1024);
+        const uint32_t acc = (kb > kb0 || kk > 0) ? 1u : 0u;
+        asm volatile(
+            "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+            "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(tmem),
+            "l"(ad), "l"(bd), "r"(IDESC), "r"(acc)
+            : "memory");
+      }
+      asm volatile(
+          "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+              saddr(&empty[stage]))
+          : "memory");
+      if (++stage == RSTAGES) {
+        stage = 0;
+        phase ^= 1u;
+      }
+    }
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+                     saddr(accf))
+                 : "memory");
+  }
+  __syncwarp();
+  // every thread: the accumulator of this CTA is complete (bounded)
+  int w_ok = 0;
+  if (lane == 0) w_ok = mbar_wait(saddr(accf), 0, g.status, g.limit_ns);
+  w_ok = __shfl_sync(0xffffffffu, w_ok, 0);
+  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+  const bool have = w_ok && (kb1 > kb0);
+  const int r = warp * 32 + lane;  // token row of this thread inside the tile
+  const uint32_t trow = tmem + ((uint32_t)(warp * 32) << 16);
+
+  if (S > 1 && rank != 0) {
+    // publish this CTA's partial (column-major) for rank 0, then wait until it was read
+#pragma unroll
+    for (int c0 = 0; c0 < N; c0 += 16) {
+      uint32_t v[16];
+      tmem_ld16(trow + c0, v);
+      asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+      for (int j = 0; j < 16; ++j) part[(c0 + j) * RBM + r] = have ? __uint_as_float(v[j]) : 0.f;
+    }
+    cluster_sync();
+    cluster_sync();
+  } else {
+    if (S > 1) cluster_sync();  // partials of ranks 1..S-1 are in their shared memory
+    const int t = tile * RBM + r;
+    const int E = g.E, K = g.K;
+    float bv[KMAX];
+    int be[KMAX];
+    int cnt = 0;
+    float m = -INFINITY, ssum = 0.f;  // online max / sum of exp for the plain softmax
+#pragma unroll 1
+    for (int c0 = 0; c0 < N; c0 += 16) {
+      uint32_t v[16];
+      tmem_ld16(trow + c0, v);
+      asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+      float lv[16];
+#pragma unroll
+      for (int j = 0; j < 16; ++j) lv[j] = have ? __uint_as_float(v[j]) : 0.f;
+      for (int q = 1; q < S; ++q) {  // partials of the other ranks, added in rank order
+        const uint32_t rbase = map_rank(saddr(&part[c0 * RBM + r]), (uint32_t)q);
+        float pv[16];
+#pragma unroll
+        for (int j = 0; j < 16; ++j) pv[j] = ld_dsmem(rbase + (uint32_t)(j * RBM * 4));
+#pragma unroll
+        for (int j = 0; j < 16; ++j) lv[j] += pv[j];
+      }
+#pragma unroll
+      for (int j = 0; j < 16; ++j) {
+        const int e = c0 + j;
+        float l = lv[j];
+        if (e < E) {
+          if (g.bias != nullptr) l += g.bias[e];
+          if (t < g.T) {
+            if (g.logits_out != nullptr) g.logits_out[(size_t)t * E + e] = l;
+            topk_insert(bv, be, cnt, K, l, e);
+            if (!g.renorm) {
+              if (l > m) {
+                ssum = ssum * expf(m - l) + 1.f;
+                m = l;
+              } else {
+                ssum += expf(l - m);
+              }
+            }
+          }
+        }
+      }
+    }
+    if (t < g.T) {
+      const float top = bv[0];
+      float den = 0.f;
+#pragma unroll
+      for (int k = 0; k < KMAX; ++k)
+        if (k < K) den += expf(bv[k] - top);
+      if (!g.renorm) den = ssum * expf(m - top);
+#pragma unroll
+      for (int k = 0; k < KMAX; ++k) {
+        if (k < K) {
+          g.topk_ids[(size_t)t * K + k] = be[k];
+          g.topk_w[(size_t)t * K + k] = expf(bv[k] - top) / den;
+        }
+      }
+    }
+    if (S > 1) cluster_sync();  // peers may exit now
+  }
+  (void)ok;
+  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+  __syncthreads();
+  if (warp == 1) {
+    asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(TCOLS)
+                 : "memory");
+  }
+}
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+bool make_map_2d(CUtensorMap* m, const void* ptr, uint64_t inner, uint64_t outer, uint32_t box0,
+                 uint32_t box1) {
+  static EncodeTiledFn fn = nullptr;
+  if (fn == nullptr) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) !=
+            cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+      return false;
+    fn = (EncodeTiledFn)p;
+  }
+  cuuint64_t gd[2] = {inner, outer}, gs[1] = {inner * 2};
+  cuuint32_t bx[2] = {box0, box1}, es[2] = {1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), gd, gs, bx, es,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <int N>
+moe_status launch_n(const CUtensorMap& mx, const CUtensorMap& mw, const RouteArgs& a, int tiles,
+                    cudaStream_t st) {
+  constexpr int NCH = (N + 63) / 64;
+  constexpr int STAGE = RA_BYTES + NCH * RB_CHUNK;
+  const int smem = RSTAGES * STAGE + 1024 + 256;
+  auto kern = route_tc_kernel<N>;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)(tiles * a.S));
+  cfg.blockDim = dim3(R_THREADS);
+  cfg.dynamicSmemBytes = (size_t)smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = (unsigned)a.S;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  launch_begin(K_ROUTE_TC, st);
+  cudaLaunchKernelEx(&cfg, kern, mx, mw, a);
+  return launch_end(K_ROUTE_TC, st);
+}
+
+}  // namespace
+
+bool route_tc_supported(const moe_shape& s) {
+  return s.dtype == MOE_BF16 && s.E % 8 == 0 && s.E <= 256 && s.K <= KMAX && s.d % 64 == 0;
+}
+
+moe_status launch_route_tc(const moe_shape& s, const void* x, const void* w_r, const float* bias,
+                           float* logits_out, int32_t* ids, float* w, cudaStream_t st) {
+  const int tiles = (s.T + RBM - 1) / RBM;
+  const int kblocks = s.d / RBK;
+  int S = (sm_count() + tiles - 1) / tiles;  // split d so that about one CTA per SM works
+  if (S > 8) S = 8;
+  if (S > kblocks) S = kblocks;
+  if (S < 1) S = 1;
+  const int N = ((s.E + 15) / 16) * 16;  // MMA N (a multiple of 16 for M = 128)
+  CUtensorMap mx, mw;
+  if (!make_map_2d(&mx, x, (uint64_t)s.d, (uint64_t)s.T, 64, 128)) return MOE_ERR_CUDA;
+  if (!make_map_2d(&mw, w_r, (uint64_t)s.E, (uint64_t)s.d, 64, 64)) return MOE_ERR_CUDA;
+  RouteArgs a;
+  a.bias = bias;
+  a.logits_out = logits_out;
+  a.topk_ids = ids;
+  a.topk_w = w;
+  a.T = s.T;
+  a.E = s.E;
+  a.K = s.K;
+  a.renorm = s.renormalize;
+  a.kblocks = kblocks;
+  a.S = S;
+  a.status = device_status_ptr();
+  a.limit_ns = kWaitLimitNs;
+  // instantiations cover N up to the next of 16/32/64/128/256; columns past E read zeros
+  if (N <= 16) return launch_n<16>(mx, mw, a, tiles, st);
+  if (N <= 32) return launch_n<32>(mx, mw, a, tiles, st);
+  if (N <= 64) return launch_n<64>(mx, mw, a, tiles, st);
+  if (N <= 128) return launch_n<128>(mx, mw, a, tiles, st);
+  return launch_n<256>(mx, mw, a, tiles, st);
+}
+
+}  // namespace moe
