@@ -585,7 +585,7 @@ moe_status launch_ffn_tc(const moe_shape& s, const void* x, const int32_t* offse
                          const void* w_down, void* a_act, void* y_perm, cudaStream_t st) {
   const long long A = (long long)s.T * s.K;
   if (A == 0) return MOE_OK;
-  const uint64_t T = s.T, d = s.d, n = s.n, E = s.E;
+  const uint64_t d = s.d, n = s.n, E = s.E;
   CUtensorMap mg, mu, ma, md;
   {
     const uint64_t dims[3] = {n, d, E}, str[2] = {n * 2, d * n * 2};

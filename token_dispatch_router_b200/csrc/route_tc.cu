@@ -282,6 +282,11 @@ __global__ void __launch_bounds__(R_THREADS) route_tc_kernel(const __grid_consta
     if (S > 1) cluster_sync();  // partials of ranks 1..S-1 are in their shared memory
     const int t = tile * RBM + r;
     const int E = g.E, K = g.K;
+    // Outputs are staged in this CTA's (idle) ring and written back coalesced: the tile's
+    // logits rows are one contiguous [128, E] block, its ids and weights [128, K] blocks.
+    float* st_l = (float*)ring;                         // [128][E + 1]
+    int32_t* st_i = (int32_t*)(st_l + RBM * (E + 1));   // [128][K]
+    float* st_w = (float*)(st_i + RBM * K);             // [128][K]
     float bv[KMAX];
     int be[KMAX];
     int cnt = 0;
@@ -309,7 +314,7 @@ __global__ void __launch_bounds__(R_THREADS) route_tc_kernel(const __grid_consta
         if (e < E) {
           if (g.bias != nullptr) l += g.bias[e];
           if (t < g.T) {
-            if (g.logits_out != nullptr) g.logits_out[(size_t)t * E + e] = l;
+            st_l[r * (E + 1) + e] = l;
             topk_insert(bv, be, cnt, K, l, e);
             if (!g.renorm) {
               if (l > m) {
@@ -333,10 +338,20 @@ __global__ void __launch_bounds__(R_THREADS) route_tc_kernel(const __grid_consta
 #pragma unroll
       for (int k = 0; k < KMAX; ++k) {
         if (k < K) {
-          g.topk_ids[(size_t)t * K + k] = be[k];
-          g.topk_w[(size_t)t * K + k] = expf(bv[k] - top) / den;
+          st_i[r * K + k] = be[k];
+          st_w[r * K + k] = expf(bv[k] - top) / den;
         }
       }
+    }
+    __syncthreads();
+    const int rows = min(RBM, g.T - tile * RBM);
+    const size_t t0 = (size_t)tile * RBM;
+    if (g.logits_out != nullptr)
+      for (int i = tid; i < rows * E; i += R_THREADS)
+        g.logits_out[t0 * E + i] = st_l[(i / E) * (E + 1) + i % E];
+    for (int i = tid; i < rows * K; i += R_THREADS) {
+      g.topk_ids[t0 * K + i] = st_i[i];
+      g.topk_w[t0 * K + i] = st_w[i];
     }
     if (S > 1) cluster_sync();  // peers may exit now
   }
