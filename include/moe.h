@@ -136,6 +136,36 @@ moe_status moe_permute(const moe_shape* shape, const int32_t* topk_ids, int32_t*
                        moe_stream_t stream);
 
 /* ----------------------------------------------------------------------------
+ * moe_permute_static - moe_permute for callers that cannot allocate device memory.
+ * The pages have no counterpart: this is a deployment variant, not part of the method.
+ * Some callers may not call cudaMalloc while they run: a serving engine that plans its
+ * whole memory budget at start-up and forbids allocation on the request path, an embedded
+ * runtime with a fixed arena, or code that runs where an allocation would synchronise the
+ * device. This entry point takes the same arguments as moe_permute minus the workspace:
+ * its scratch (per-chunk expert counts and rank bases) lives in a file-scope device array
+ * of MOE_PERMUTE_STATIC_SCRATCH_BYTES inside the library, which every GPU that loads the
+ * library holds until the process exits. It allocates nothing and calls no allocating
+ * routine. Results are identical to moe_permute.
+ *  - Limit: needs 2 * ceil(T*K / 4096) * E * 4 bytes of scratch (= moe_permute_workspace_size
+ *    minus its 256-byte slack); larger problems return MOE_ERR_UNSUPPORTED and enqueue
+ *    nothing. With the default 1 MiB: T*K up to about 2 million assignments at E = 256,
+ *    8 million at E = 64.
+ *  - Set-up: the first call on each device (with that device current) resolves the array's
+ *    device address with cudaGetSymbolAddress; make that first call before any stream
+ *    capture.
+ *  - Sharing: every call uses the same array, which keeps the last call's contents (the
+ *    kernels overwrite every entry they read, so nothing must start at zero). Calls whose
+ *    kernels overlap on the GPU (other streams, other host threads) race on it: serialise
+ *    them.
+ */
+#ifndef MOE_PERMUTE_STATIC_SCRATCH_BYTES
+#define MOE_PERMUTE_STATIC_SCRATCH_BYTES (1u << 20)
+#endif
+moe_status moe_permute_static(const moe_shape* shape, const int32_t* topk_ids, int32_t* counts,
+                              int32_t* offsets, int32_t* assign_to_perm, int32_t* perm_to_assign,
+                              const void* x, void* x_perm, moe_stream_t stream);
+
+/* ----------------------------------------------------------------------------
  * moe_grouped_ffn - the grouped SwiGLU expert FFN on the expert-major rows.
  * SonicMoE explainer, section 3 items 3-5 (grouped GEMM with a different M
  * per expert, SwiGLU, second grouped GEMM), section 6.2 (the gather of x is

@@ -50,6 +50,7 @@ _SIGS = {
     "moe_forward_workspace_layout": (ctypes.c_int, [_S, ctypes.POINTER(moe_workspace_layout)]),
     "moe_route": (ctypes.c_int, [_S, _P, _P, _P, _P, _P, _P, _P, _P]),
     "moe_permute": (ctypes.c_int, [_S, _P, _P, _P, _P, _P, _P, _P, _P, ctypes.c_size_t, _P]),
+    "moe_permute_static": (ctypes.c_int, [_S, _P, _P, _P, _P, _P, _P, _P, _P]),
     "moe_grouped_ffn": (ctypes.c_int, [_S, _P, _P, _P, _P, _P, _P, _P, _P, _P]),
     "moe_combine": (ctypes.c_int, [_S, _P, _P, _P, _P, _P]),
     "moe_forward": (ctypes.c_int, [_S, _P, _P, _P, _P, _P, _P, _P, _P, _P, ctypes.c_size_t, _P]),
@@ -180,6 +181,33 @@ def permute(shape: moe_shape, topk_ids: torch.Tensor, x=None, materialize: bool 
     _check(lib.moe_permute(ctypes.byref(shape), _ptr(topk_ids), _ptr(counts), _ptr(offsets),
                            _ptr(a2p), _ptr(p2a), _ptr(x if materialize else None), _ptr(x_perm),
                            _ptr(workspace), workspace.numel(), _stream()), "moe_permute")
+    out = dict(counts=counts, offsets=offsets, assign_to_perm=a2p, perm_to_assign=p2a)
+    if materialize:
+        out["x_perm"] = x_perm
+    return out
+
+
+def permute_static(shape: moe_shape, topk_ids: torch.Tensor, x=None, materialize: bool = False):
+    """moe_permute_static: moe_permute without a workspace, for callers that may not
+    allocate device memory while they run (its scratch is a fixed array inside the
+    library; see include/moe.h for the size limit and the sharing rules). The output
+    tensors here are allocated by torch only for the convenience of this binding."""
+    lib = load_library()
+    T, E, K = shape.T, shape.E, shape.K
+    dev = topk_ids.device
+    _dev(topk_ids, "topk_ids", torch.int32, (T, K))
+    counts = torch.empty(E, dtype=torch.int32, device=dev)
+    offsets = torch.empty(E + 1, dtype=torch.int32, device=dev)
+    a2p = torch.empty(T * K, dtype=torch.int32, device=dev)
+    p2a = torch.full((T * K,), -1, dtype=torch.int32, device=dev)
+    x_perm = None
+    if materialize:
+        _dev(x, "x", _act_dtype(shape), (T, shape.d))
+        x_perm = torch.empty(T * K, shape.d, dtype=x.dtype, device=dev)
+    _check(lib.moe_permute_static(ctypes.byref(shape), _ptr(topk_ids), _ptr(counts),
+                                  _ptr(offsets), _ptr(a2p), _ptr(p2a),
+                                  _ptr(x if materialize else None), _ptr(x_perm), _stream()),
+           "moe_permute_static")
     out = dict(counts=counts, offsets=offsets, assign_to_perm=a2p, perm_to_assign=p2a)
     if materialize:
         out["x_perm"] = x_perm

@@ -27,6 +27,9 @@ moe_status launch_combine(const moe_shape& s, const void* y_perm, const int32_t*
                           const float* topk_w, void* out, cudaStream_t st);
 moe_status launch_selftest_timeout(uint64_t limit_ns, cudaStream_t st);
 bool route_tc_supported(const moe_shape& s);
+moe_status launch_permute_static(const moe_shape& s, const int32_t* ids, int32_t* counts,
+                                 int32_t* offsets, int32_t* a2p, int32_t* p2a, const void* x,
+                                 void* x_perm, cudaStream_t st);
 moe_status launch_route_tc(const moe_shape& s, const void* x, const void* w_r, const float* bias,
                            float* logits_out, int32_t* ids, float* w, cudaStream_t st);
 
@@ -234,6 +237,28 @@ moe_status moe_permute(const moe_shape* s, const int32_t* topk_ids, int32_t* cou
   if (need > 0 && (workspace == nullptr || ws_bytes < need)) return MOE_ERR_WORKSPACE;
   return launch_permute(*s, topk_ids, counts, offsets, assign_to_perm, perm_to_assign, x, x_perm,
                         workspace, (cudaStream_t)stream);
+}
+
+moe_status moe_permute_static(const moe_shape* s, const int32_t* topk_ids, int32_t* counts,
+                              int32_t* offsets, int32_t* assign_to_perm, int32_t* perm_to_assign,
+                              const void* x, void* x_perm, moe_stream_t stream) {
+  const bool gather = (x != nullptr && x_perm != nullptr);
+  moe_status r = check_shape(s, gather, false);
+  if (r != MOE_OK) return r;
+  if (topk_ids == nullptr || counts == nullptr || offsets == nullptr || assign_to_perm == nullptr ||
+      perm_to_assign == nullptr)
+    return MOE_ERR_INVALID_ARG;
+  if ((x == nullptr) != (x_perm == nullptr)) return MOE_ERR_INVALID_ARG;
+  if (gather && (!aligned16(x) || !aligned16(x_perm))) return MOE_ERR_INVALID_ARG;
+  if (s->T == 0) {
+    const cudaStream_t st = (cudaStream_t)stream;
+    if (cudaMemsetAsync(counts, 0, sizeof(int32_t) * s->E, st) != cudaSuccess ||
+        cudaMemsetAsync(offsets, 0, sizeof(int32_t) * (s->E + 1), st) != cudaSuccess)
+      return MOE_ERR_CUDA;
+    return MOE_OK;
+  }
+  return launch_permute_static(*s, topk_ids, counts, offsets, assign_to_perm, perm_to_assign, x,
+                               x_perm, (cudaStream_t)stream);
 }
 
 moe_status moe_grouped_ffn(const moe_shape* s, const void* x, const int32_t* offsets,

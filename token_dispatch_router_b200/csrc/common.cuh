@@ -95,4 +95,7 @@ moe_status launch_end(int kernel_id, cudaStream_t s);  // checks cudaGetLastErro
 
 constexpr uint64_t kWaitLimitNs = 2000000000ull;  // bounded waits: 2 s
 
+// Size of the static scratch behind moe_permute_static (see moe.h).
+constexpr size_t kPermuteStaticScratchBytes = MOE_PERMUTE_STATIC_SCRATCH_BYTES;
+
 }  // namespace moe

@@ -20,6 +20,8 @@
 //             warps), then walks the slice again: rank = base + (lanes of the group below
 //             me); rank < C -> slot offsets[e] + rank, else dropped (-1).
 // Inside an expert the slots follow ascending flat index a = t*K + k, i.e. token order.
+#include <mutex>
+
 #include "common.cuh"
 
 namespace moe {
@@ -245,6 +247,49 @@ moe_status launch_permute(const moe_shape& s, const int32_t* ids, int32_t* count
     if ((r = launch_end(K_GATHER, st)) != MOE_OK) return r;
   }
   return MOE_OK;
+}
+
+// ------------------------------------------------------------------ no-allocation variant
+// For callers that may not allocate device memory while they run: a serving engine that
+// plans its whole memory budget at start-up and forbids allocation on the request path, an
+// embedded runtime with a fixed arena, or code that runs where cudaMalloc would synchronise
+// the device. Their permute scratch lives in this file-scope device array instead of a
+// caller workspace. Every GPU that loads the library holds it until the process exits.
+// All calls share it and it keeps the last call's contents; the histogram kernel writes
+// every per-chunk count and the scan kernel every rank base before either is read, so
+// nothing in it has to start at zero. Calls whose kernels overlap on the GPU (different
+// streams, or several host threads) race on it and must be serialised by the caller.
+static __device__ __align__(256) unsigned char g_permute_static_scratch[kPermuteStaticScratchBytes];
+
+namespace {
+std::mutex g_static_mu;
+void* g_static_ptr[64];  // device address of the array, per device
+}  // namespace
+
+// Device address of the static scratch on the current device. The first call on a device
+// resolves it with cudaGetSymbolAddress (with that device current); later calls reuse it.
+static moe_status static_scratch_ptr(void** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return MOE_ERR_CUDA;
+  std::lock_guard<std::mutex> lk(g_static_mu);
+  if (g_static_ptr[dev] == nullptr) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_permute_static_scratch) != cudaSuccess || p == nullptr)
+      return MOE_ERR_CUDA;
+    g_static_ptr[dev] = p;
+  }
+  *out = g_static_ptr[dev];
+  return MOE_OK;
+}
+
+moe_status launch_permute_static(const moe_shape& s, const int32_t* ids, int32_t* counts,
+                                 int32_t* offsets, int32_t* a2p, int32_t* p2a, const void* x,
+                                 void* x_perm, cudaStream_t st) {
+  if (permute_scratch_bytes(s) > (size_t)kPermuteStaticScratchBytes) return MOE_ERR_UNSUPPORTED;
+  void* scratch = nullptr;
+  const moe_status r = static_scratch_ptr(&scratch);
+  if (r != MOE_OK) return r;
+  return launch_permute(s, ids, counts, offsets, a2p, p2a, x, x_perm, scratch, st);
 }
 
 }  // namespace moe
