@@ -35,7 +35,7 @@ import moe_inputs as mi  # noqa: E402
 
 METRIC = "MoE layer fwd tokens/s at 1 B200; dispatch+combine GB/s and GEMM % of peak"
 PEAKS_FILE = os.path.join(ROOT, "MEASURED_PEAKS.json")
-TRAFFIC_FILE = os.path.join(ROOT, "profiles", "traffic.json")
+PROFILES_DIR = os.path.join(ROOT, "profiles")
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 
@@ -155,15 +155,20 @@ def kernel_source_hash() -> str:
 
 
 def traffic_for(kernel: str, workload: str):
-    """ncu DRAM bytes per launch for `kernel`, if taken on the current kernel source."""
-    if not os.path.exists(TRAFFIC_FILE):
-        return None
-    with open(TRAFFIC_FILE) as f:
-        rec = json.load(f)
-    r = rec.get(workload, {}).get(kernel)
-    if not r or r.get("source_hash") != kernel_source_hash():
-        return None
-    return r.get("bytes_per_launch")
+    """ncu DRAM bytes per launch for `kernel` from a `bench-record:` line of a profiles/*.md
+    summary, reported only if it was taken on the current kernel source."""
+    import glob
+    want = kernel_source_hash()
+    for path in sorted(glob.glob(os.path.join(PROFILES_DIR, "*.md"))):
+        with open(path) as f:
+            for line in f:
+                if not line.startswith("bench-record:"):
+                    continue
+                kv = dict(item.split("=", 1) for item in line.split()[1:] if "=" in item)
+                if (kv.get("workload") == workload and kv.get("kernel") == kernel
+                        and kv.get("source_hash") == want):
+                    return int(kv["bytes_per_launch"])
+    return None
 
 
 # ------------------------------------------------------------------ CPU oracle leg
