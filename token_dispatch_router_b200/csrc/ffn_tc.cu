@@ -393,10 +393,9 @@ __global__ void __launch_bounds__(GATEUP ? THREADS_GATEUP : THREADS_DOWN, 1)
     const int rg = lane >> 3;            // rows 32 gw + rg + 4 i, i < 8
     int stage = 0;
     uint32_t phase = 0;
-    for (int w = blockIdx.x; w < total; w += gridDim.x) {
+    // token rows of a tile: row r of the tile reads x[perm_to_assign[m0 + r] / K]
+    auto rows_of = [&](int w, const uint8_t* (&src)[8]) {
       const Tile t = decode_tile(w, s_off, s_cum, s_mt, E, g.out_tile);
-      const uint8_t* src[8];
-      uint32_t dst[8];
 #pragma unroll
       for (int i = 0; i < 8; ++i) {
         const int r = gw * 32 + rg + 4 * i;
@@ -408,8 +407,20 @@ __global__ void __launch_bounds__(GATEUP ? THREADS_GATEUP : THREADS_DOWN, 1)
           tk = 0;
         }
         src[i] = g.x + (size_t)tk * g.x_row_bytes + c * 16;
-        dst[i] = (uint32_t)(r * 128 + ((c ^ (r & 7)) << 4));  // 128-byte swizzle
       }
+    };
+    uint32_t dst[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const int r = gw * 32 + rg + 4 * i;
+      dst[i] = (uint32_t)(r * 128 + ((c ^ (r & 7)) << 4));  // 128-byte swizzle
+    }
+    const uint8_t* src[8];
+    if (blockIdx.x < (unsigned)total) rows_of(blockIdx.x, src);
+    for (int w = blockIdx.x; w < total; w += gridDim.x) {
+      // the next tile's rows are loaded now, one tile ahead of their use
+      const uint8_t* nsrc[8];
+      if (w + (int)gridDim.x < total) rows_of(w + gridDim.x, nsrc);
       bool ok = true;
       for (int kb = 0; kb < g.kblocks; ++kb) {
         int w_ok = 0;
@@ -429,6 +440,8 @@ __global__ void __launch_bounds__(GATEUP ? THREADS_GATEUP : THREADS_DOWN, 1)
         }
       }
       if (!ok) break;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) src[i] = nsrc[i];
     }
     cp_async_wait_all();  // nothing of ours lands after the CTA exits
   } else {
