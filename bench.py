@@ -248,6 +248,60 @@ def run_reference(args, rank, world):
     print(json.dumps(line), flush=True)
 
 
+# ------------------------------------------------------------------ dispatch + combine
+def dispatch_combine_bytes(cfg) -> int:
+    """Algorithmic bytes of route + permute (gathered rows materialised) + combine:
+    route reads x and writes logits, ids and weights; permute reads ids and writes both
+    index maps, reads x and writes x_perm; combine reads x_perm, ids/weights and writes out."""
+    b = 2 if cfg.dtype == "bf16" else 4
+    T, d, E, K = cfg.T, cfg.d, cfg.E, cfg.K
+    A = T * K
+    route = T * d * b + d * E * b + T * E * 4 + T * K * 8
+    permute = A * 4 + A * 8 + E * 8 + T * d * b + A * d * b
+    combine = A * d * b + A * 8 + T * d * b
+    return route + permute + combine
+
+
+def dispatch_combine(tdr, s, cfg, x, w_r, bias, steps, world, peaks):
+    """Time route -> permute (x_perm) -> combine(x_perm) at the layer's shape."""
+    dev = x.device
+    T, d, E, K = cfg.T, cfg.d, cfg.E, cfg.K
+    ids = torch.empty(T, K, dtype=torch.int32, device=dev)
+    w = torch.empty(T, K, dtype=torch.float32, device=dev)
+    lo = torch.empty(T, E, dtype=torch.float32, device=dev)
+    pws = torch.empty(max(tdr.permute_workspace_size(s), 256), dtype=torch.uint8, device=dev)
+    out = torch.empty(T, d, dtype=x.dtype, device=dev)
+
+    def once():
+        tdr.route(s, x, w_r, bias=bias, logits_out=lo, topk_ids=ids, topk_w=w)
+        p = tdr.permute(s, ids, x=x, materialize=True, workspace=pws)
+        tdr.combine(s, p["x_perm"], p["assign_to_perm"], w, out=out)
+
+    for _ in range(3):
+        once()
+    torch.cuda.synchronize()
+    n = max(10, min(steps, 100))
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    prof = tdr.Profiler()
+    with prof:
+        e0.record()
+        for _ in range(n):
+            once()
+        e1.record()
+        torch.cuda.synchronize()
+    ms = max_over_ranks(e0.elapsed_time(e1) / n, world)
+    kern = {k: round(v[1] / n, 4) for k, v in prof.results().items()}
+    kern_ms = sum(kern.values())
+    nbytes = dispatch_combine_bytes(cfg)
+    peak = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
+    gbs = nbytes / (kern_ms / 1e3) / 1e9 if kern_ms > 0 else 0.0
+    return {"bytes": nbytes, "ms_kernels": round(kern_ms, 4), "ms_wall": round(ms, 4),
+            "achieved_gbs": round(gbs, 1), "peak_gbs": peak, "frac": round(gbs / peak, 4),
+            "kernels_ms": kern,
+            "note": "route + permute with x_perm materialised + combine(x_perm); GB/s over "
+                    "the summed kernel time (CUDA events around each launch)"}
+
+
 # ------------------------------------------------------------------ our arm
 def run_ours(args, rank, world, local):
     import token_dispatch_router_b200 as tdr
@@ -344,6 +398,10 @@ def run_ours(args, rank, world, local):
     e2e = {"value": cfg.T * world * e2e_steps / (e2e_ms / 1e3), "unit": "tokens/s",
            "h2d_bytes_per_step": cfg.T * cfg.d * elem, "d2h_bytes_per_step": cfg.T * cfg.d * elem}
 
+    # ---- dispatch + combine byte stream at the same shape (route, permute with the gathered
+    # rows materialised, combine of those rows as identity experts): the unfused traffic
+    dc = dispatch_combine(tdr, s, cfg, x, w_r, bias, args.steps, world, peaks)
+
     # ---- per-kernel breakdown (ms per step) and the two secondary figures of the metric
     per_kernel = {k: round(ms / args.steps, 4) for k, (n, ms) in kern.items()}
     gemm = {"achieved_tflops": round(ach_gemm, 2), "frac": round(ach_gemm / peak_t, 4),
@@ -356,7 +414,8 @@ def run_ours(args, rank, world, local):
         "config": {"workload": cfg.name, "T": cfg.T, "d": cfg.d, "E": cfg.E, "K": cfg.K,
                    "n": cfg.n, "global_batch": cfg.T * world, "parallelism": f"replicas{world}",
                    "l2": "inputs larger than L2: the 2.82 GB of expert weights stream every step"},
-        "roofline": roofline, "gemm": gemm, "kernel_ms_per_step": per_kernel,
+        "roofline": roofline, "gemm": gemm, "dispatch_combine": dc,
+        "kernel_ms_per_step": per_kernel,
         "gpu_launches": int(launches), "e2e": e2e,
     }
     result["clocks"] = clocks.summary()

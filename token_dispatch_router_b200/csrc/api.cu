@@ -75,7 +75,7 @@ namespace {
 const char* kKernelNames[K_COUNT] = {
     "route",        "hist",          "scan",           "scatter",     "gather_rows", "gateup_tc",
     "down_tc",      "gateup_simt",   "down_simt",      "combine",     "selftest_timeout",
-    "route_tc"};
+    "route_tc",     "permute_small"};
 
 struct ProfRec {
   int kid;

@@ -5,9 +5,11 @@
 //   out[t] = sum_{k, assign_to_perm[t*K+k] >= 0} topk_w[t,k] * y_perm[assign_to_perm[t*K+k]]
 // fp32 accumulation in k order (deterministic); dropped slots add nothing.
 //
-// HBM-bound. One thread per (token, 16-byte column vector): the K expert rows are read
-// with independent 128-bit loads (K loads in flight per thread), consecutive threads take
-// consecutive vectors of one row, so every warp access is 512 contiguous bytes.
+// HBM-bound. One warp owns a 2 KB segment (128 16-byte vectors) of one token's output row:
+// the token's K slots and weights are loaded once per lane (same addresses across the warp),
+// then for each pair of slots every lane issues eight independent 128-bit loads (4 vectors
+// x 2 rows; every warp-wide load covers 512 contiguous bytes), accumulates in fp32 in slot
+// order, and writes its four vectors.
 #include "common.cuh"
 
 namespace moe {
@@ -21,42 +23,57 @@ __global__ void __launch_bounds__(256) combine_kernel(const uint4* __restrict__ 
                                                       int K, int vec_per_row, long long n_rows,
                                                       uint4* __restrict__ out, unsigned* status) {
   constexpr int V = Vec16<Tv>::N;
-  const long long total = (long long)T * vec_per_row;
-  for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < total;
-       i += (long long)gridDim.x * blockDim.x) {
-    const long long t = i / vec_per_row;
-    const int v = (int)(i - t * vec_per_row);
-    float acc[V];
+  const int segs = (vec_per_row + 127) / 128;
+  const long long units = (long long)T * segs;
+  const int lane = threadIdx.x & 31;
+  const long long warps = (long long)gridDim.x * (blockDim.x >> 5);
+  for (long long u = (long long)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); u < units;
+       u += warps) {
+    const long long t = u / segs;
+    const int v0 = (int)(u - t * segs) * 128 + lane;
+    float acc[4][V];
 #pragma unroll
-    for (int j = 0; j < V; ++j) acc[j] = 0.f;
-    for (int k0 = 0; k0 < K; k0 += 4) {  // up to 4 rows in flight
-      uint4 u[4];
-      float w[4];
-      bool ok[4];
+    for (int j = 0; j < 4; ++j)
 #pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        const int k = k0 + j;
-        ok[j] = false;
-        if (k < K) {
-          const long long p = a2p[t * K + k];
-          if (p >= n_rows) report(status, MOE_ERR_DEVICE_INDEX);
-          if (p >= 0 && p < n_rows) {
-            ok[j] = true;
-            w[j] = topk_w[t * K + k];
-            u[j] = y_perm[p * vec_per_row + v];
+      for (int q = 0; q < V; ++q) acc[j][q] = 0.f;
+    for (int k0 = 0; k0 < K; k0 += 2) {
+      long long p[2];
+      float w[2];
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        p[h] = -1;
+        w[h] = 0.f;
+        if (k0 + h < K) {
+          p[h] = a2p[t * K + k0 + h];
+          if (p[h] >= n_rows) {
+            if (lane == 0) report(status, MOE_ERR_DEVICE_INDEX);
+            p[h] = -1;
           }
+          if (p[h] >= 0) w[h] = topk_w[t * K + k0 + h];
         }
       }
+      uint4 r[2][4];
 #pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        if (!ok[j]) continue;
-        float f[V];
-        unpack16(u[j], f, Tv());
+      for (int h = 0; h < 2; ++h)
 #pragma unroll
-        for (int q = 0; q < V; ++q) acc[q] = fmaf(w[j], f[q], acc[q]);
+        for (int j = 0; j < 4; ++j)
+          if (p[h] >= 0 && v0 + 32 * j < vec_per_row) r[h][j] = y_perm[p[h] * vec_per_row + v0 + 32 * j];
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        if (p[h] < 0) continue;
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          if (v0 + 32 * j >= vec_per_row) continue;
+          float f[V];
+          unpack16(r[h][j], f, Tv());
+#pragma unroll
+          for (int q = 0; q < V; ++q) acc[j][q] = fmaf(w[h], f[q], acc[j][q]);
+        }
       }
     }
-    out[i] = pack16(acc, Tv());
+#pragma unroll
+    for (int j = 0; j < 4; ++j)
+      if (v0 + 32 * j < vec_per_row) out[t * vec_per_row + v0 + 32 * j] = pack16(acc[j], Tv());
   }
 }
 
@@ -66,9 +83,9 @@ moe_status launch_combine(const moe_shape& s, const void* y_perm, const int32_t*
                           const float* topk_w, void* out, cudaStream_t st) {
   const int elem = (s.dtype == MOE_BF16) ? 2 : 4;
   const int vec_per_row = s.d * elem / 16;
-  const long long total = (long long)s.T * vec_per_row;
-  if (total == 0) return MOE_OK;
-  long long blocks = (total + 255) / 256;
+  const long long units = (long long)s.T * ((vec_per_row + 127) / 128);  // one warp each
+  if (units == 0) return MOE_OK;
+  long long blocks = (units + 7) / 8;
   const long long cap_blocks = (long long)sm_count() * 8;
   if (blocks > cap_blocks) blocks = cap_blocks;
   const long long n_rows = (long long)s.T * s.K;

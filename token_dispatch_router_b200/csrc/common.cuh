@@ -85,6 +85,7 @@ enum KernelId {
   K_COMBINE,
   K_SELFTEST,
   K_ROUTE_TC,
+  K_PERMUTE_SMALL,
   K_COUNT
 };
 

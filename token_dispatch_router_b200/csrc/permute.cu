@@ -176,7 +176,87 @@ __global__ void __launch_bounds__(kWarps * 32) scatter_kernel(
   }
 }
 
-// x_perm[p] = x[perm_to_assign[p] / K] for p < offsets[E]; 16-byte vectors.
+// Small problems (T*K <= kSmallMax): histogram, scan and scatter in one CTA of 32 warps,
+// one launch instead of three. Same algorithm and same result as the three kernels: each
+// warp owns a contiguous slice, counts it into its private row, the rows are turned into
+// rank bases in warp order, and the slice is walked again to place each assignment.
+constexpr int kSmallWarps = 32;
+constexpr long long kSmallMax = 32768;
+
+__global__ void __launch_bounds__(kSmallWarps * 32) permute_small_kernel(
+    const int32_t* __restrict__ ids, long long A, int E, long long cap, int32_t* __restrict__ counts,
+    int32_t* __restrict__ offsets, int32_t* __restrict__ assign_to_perm,
+    int32_t* __restrict__ perm_to_assign, unsigned* status) {
+  __shared__ int rows[kSmallWarps][kMaxE];
+  __shared__ long long kept_s[kMaxE];
+  __shared__ int offs[kMaxE];
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const long long slice = ((A + kSmallWarps * 32 - 1) / (kSmallWarps * 32)) * 32;  // ids per warp
+  const long long s0 = (long long)warp * slice;
+  for (int i = tid; i < kSmallWarps * kMaxE; i += blockDim.x) (&rows[0][0])[i] = 0;
+  __syncthreads();
+  int* row = rows[warp];
+  for (long long a0 = s0; a0 < s0 + slice; a0 += 32) {
+    const int id = load_id(ids, a0 + lane, A, E, status);
+    const unsigned m = __match_any_sync(0xffffffffu, id);
+    if (id >= 0 && lane == __ffs(m) - 1) row[id] += __popc(m);
+    __syncwarp();
+  }
+  __syncthreads();
+  long long run = 0;
+  if (tid < kMaxE) {
+    const int e = tid;
+    if (e < E) {
+      for (int w = 0; w < kSmallWarps; ++w) {
+        const int c = rows[w][e];
+        rows[w][e] = (int)run;
+        run += c;
+      }
+      counts[e] = (int32_t)run;
+    }
+    kept_s[e] = (e < E) ? (cap >= 0 && run > cap ? cap : run) : 0;
+  }
+  __syncthreads();
+  for (int off = 1; off < kMaxE; off <<= 1) {  // inclusive scan of kept over experts
+    long long add = 0;
+    if (tid < kMaxE && tid >= off) add = kept_s[tid - off];
+    __syncthreads();
+    if (tid < kMaxE) kept_s[tid] += add;
+    __syncthreads();
+  }
+  if (tid < E) {
+    const long long mine = (cap >= 0 && run > cap) ? cap : run;
+    offs[tid] = (int)(kept_s[tid] - mine);
+    offsets[tid] = (int32_t)(kept_s[tid] - mine);
+    if (tid == E - 1) offsets[E] = (int32_t)kept_s[tid];
+  }
+  __syncthreads();
+  const unsigned lt = lanemask_lt();
+  for (long long a0 = s0; a0 < s0 + slice; a0 += 32) {
+    const long long a = a0 + lane;
+    const int id = load_id(ids, a, A, E, nullptr);
+    const unsigned m = __match_any_sync(0xffffffffu, id);
+    int rank = 0;
+    if (id >= 0) rank = row[id] + __popc(m & lt);
+    __syncwarp();
+    if (id >= 0 && lane == __ffs(m) - 1) row[id] += __popc(m);
+    __syncwarp();
+    if (id >= 0) {
+      int p = -1;
+      if (cap < 0 || rank < cap) {
+        p = offs[id] + rank;
+        perm_to_assign[p] = (int32_t)a;
+      }
+      assign_to_perm[a] = p;
+    } else if (a < A) {
+      assign_to_perm[a] = -1;
+    }
+  }
+}
+
+// x_perm[p] = x[perm_to_assign[p] / K] for p < offsets[E]; 16-byte vectors. One warp moves
+// a 2 KB segment (128 vectors) of one row: the row's source token is loaded once per lane
+// and each lane keeps four independent 16-byte loads in flight.
 __global__ void __launch_bounds__(256) gather_rows_kernel(const uint4* __restrict__ x,
                                                           const int32_t* __restrict__ p2a,
                                                           const int32_t* __restrict__ n_kept_ptr,
@@ -184,18 +264,29 @@ __global__ void __launch_bounds__(256) gather_rows_kernel(const uint4* __restric
                                                           uint4* __restrict__ x_perm,
                                                           unsigned* status) {
   const long long n_kept = *n_kept_ptr;
-  const long long total = n_kept * vec_per_row;
-  for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < total;
-       i += (long long)gridDim.x * blockDim.x) {
-    const long long p = i / vec_per_row;
-    const int v = (int)(i - p * vec_per_row);
+  const int segs = (vec_per_row + 127) / 128;
+  const long long units = n_kept * segs;
+  const int lane = threadIdx.x & 31;
+  const long long warps = (long long)gridDim.x * (blockDim.x >> 5);
+  for (long long u = (long long)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); u < units;
+       u += warps) {
+    const long long p = u / segs;
+    const int v0 = (int)(u - p * segs) * 128 + lane;
     const int a = p2a[p];
     const int t = a / K;
     if (a < 0 || t >= T) {
-      report(status, MOE_ERR_DEVICE_INDEX);
+      if (lane == 0) report(status, MOE_ERR_DEVICE_INDEX);
       continue;
     }
-    x_perm[i] = x[(size_t)t * vec_per_row + v];
+    const uint4* src = x + (size_t)t * vec_per_row;
+    uint4* dst = x_perm + (size_t)p * vec_per_row;
+    uint4 r[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j)
+      if (v0 + 32 * j < vec_per_row) r[j] = src[v0 + 32 * j];
+#pragma unroll
+    for (int j = 0; j < 4; ++j)
+      if (v0 + 32 * j < vec_per_row) dst[v0 + 32 * j] = r[j];
   }
 }
 
@@ -220,15 +311,19 @@ moe_status launch_permute(const moe_shape& s, const int32_t* ids, int32_t* count
           : -1;
   unsigned* status = device_status_ptr();
   moe_status r;
-  if (nchunks > 0) {
+  if (A > 0 && A <= kSmallMax) {
+    launch_begin(K_PERMUTE_SMALL, st);
+    permute_small_kernel<<<1, kSmallWarps * 32, 0, st>>>(ids, A, s.E, cap, counts, offsets, a2p,
+                                                         p2a, status);
+    if ((r = launch_end(K_PERMUTE_SMALL, st)) != MOE_OK) return r;
+  } else if (nchunks > 0) {
     launch_begin(K_HIST, st);
     hist_kernel<<<nchunks, kWarps * 32, 0, st>>>(ids, A, s.E, chunk_counts, status);
     if ((r = launch_end(K_HIST, st)) != MOE_OK) return r;
-  }
-  launch_begin(K_SCAN, st);
-  scan_kernel<<<1, kMaxE, 0, st>>>(chunk_counts, chunk_base, nchunks, s.E, cap, counts, offsets);
-  if ((r = launch_end(K_SCAN, st)) != MOE_OK) return r;
-  if (nchunks > 0) {
+    launch_begin(K_SCAN, st);
+    scan_kernel<<<1, kMaxE, 0, st>>>(chunk_counts, chunk_base, nchunks, s.E, cap, counts,
+                                     offsets);
+    if ((r = launch_end(K_SCAN, st)) != MOE_OK) return r;
     launch_begin(K_SCATTER, st);
     scatter_kernel<<<nchunks, kWarps * 32, 0, st>>>(ids, A, s.E, cap, chunk_base, offsets, a2p,
                                                     p2a, status);
@@ -237,9 +332,9 @@ moe_status launch_permute(const moe_shape& s, const int32_t* ids, int32_t* count
   if (x != nullptr && x_perm != nullptr && A > 0) {
     const int elem = (s.dtype == MOE_BF16) ? 2 : 4;
     const int vec_per_row = s.d * elem / 16;
-    const long long total = A * vec_per_row;
-    long long blocks = (total + 255) / 256;
-    const long long cap_blocks = (long long)sm_count() * 16;
+    const long long units = A * ((vec_per_row + 127) / 128);  // one warp each
+    long long blocks = (units + 7) / 8;
+    const long long cap_blocks = (long long)sm_count() * 8;
     if (blocks > cap_blocks) blocks = cap_blocks;
     launch_begin(K_GATHER, st);
     gather_rows_kernel<<<(int)blocks, 256, 0, st>>>((const uint4*)x, p2a, offsets + s.E, s.K, s.T,

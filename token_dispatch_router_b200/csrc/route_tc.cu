@@ -125,13 +125,10 @@ __device__ __forceinline__ float ld_dsmem(uint32_t remote_addr) {
 }
 
 // Insert (v, e) into the descending list (ids arrive in ascending order, so an equal value
-// goes behind the ones already held: ties keep the lower id).
-__device__ __forceinline__ void topk_insert(float (&bv)[KMAX], int (&be)[KMAX], int& cnt, int K,
-                                            float v, int e) {
-  float kth = 0.f;  // the K-th value once the list is full (unrolled select: no local memory)
-#pragma unroll
-  for (int j = 0; j < KMAX; ++j)
-    if (j == K - 1) kth = bv[j];
+// goes behind the ones already held: ties keep the lower id). `kth` caches the K-th value
+// once the list is full, so a value that does not enter costs one comparison.
+__device__ __forceinline__ void topk_insert(float (&bv)[KMAX], int (&be)[KMAX], int& cnt,
+                                            float& kth, int K, float v, int e) {
   if (cnt == K && !(v > kth)) return;
   float cv = v;
   int ce = e;
@@ -154,6 +151,11 @@ __device__ __forceinline__ void topk_insert(float (&bv)[KMAX], int (&be)[KMAX], 
     }
   }
   if (cnt < K) ++cnt;
+  if (cnt == K) {
+#pragma unroll
+    for (int j = 0; j < KMAX; ++j)
+      if (j == K - 1) kth = bv[j];
+  }
 }
 
 template <int N>  // MMA N = E rounded up to 16
@@ -290,6 +292,7 @@ __global__ void __launch_bounds__(R_THREADS) route_tc_kernel(const __grid_consta
     float bv[KMAX];
     int be[KMAX];
     int cnt = 0;
+    float kth = -INFINITY;
     float m = -INFINITY, ssum = 0.f;  // online max / sum of exp for the plain softmax
 #pragma unroll 1
     for (int c0 = 0; c0 < N; c0 += 16) {
@@ -315,7 +318,7 @@ __global__ void __launch_bounds__(R_THREADS) route_tc_kernel(const __grid_consta
           if (g.bias != nullptr) l += g.bias[e];
           if (t < g.T) {
             st_l[r * (E + 1) + e] = l;
-            topk_insert(bv, be, cnt, K, l, e);
+            topk_insert(bv, be, cnt, kth, K, l, e);
             if (!g.renorm) {
               if (l > m) {
                 ssum = ssum * expf(m - l) + 1.f;
