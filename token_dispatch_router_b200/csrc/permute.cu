@@ -34,10 +34,14 @@ constexpr int kSlice = 32 * kIters;          // ids per warp
 constexpr int kChunk = kWarps * kSlice;      // ids per CTA
 constexpr int kMaxE = 256;
 
-__device__ __forceinline__ int load_id(const int32_t* ids, long long a, long long A, int E,
-                                       unsigned* status) {
-  if (a >= A) return -1;
-  const int id = ids[a];
+// Ids are fetched with plain non-coherent loads first and validated afterwards, so that a
+// group of loads is issued back to back (a status report between loads would serialise
+// them). An id outside [0, E) is reported and treated as absent.
+__device__ __forceinline__ int raw_id(const int32_t* __restrict__ ids, long long a, long long A) {
+  return a < A ? __ldg(ids + a) : -1;
+}
+__device__ __forceinline__ int checked_id(int id, bool real, int E, unsigned* status) {
+  if (!real) return -1;
   if (id < 0 || id >= E) {
     report(status, MOE_ERR_DEVICE_INDEX);
     return -1;
@@ -51,7 +55,9 @@ __device__ __forceinline__ void warp_histogram(const int32_t* ids, long long sli
   const int lane = threadIdx.x & 31;
   int v[kIters];
 #pragma unroll
-  for (int it = 0; it < kIters; ++it) v[it] = load_id(ids, slice0 + it * 32 + lane, A, E, status);
+  for (int it = 0; it < kIters; ++it) v[it] = raw_id(ids, slice0 + it * 32 + lane, A);
+#pragma unroll
+  for (int it = 0; it < kIters; ++it) v[it] = checked_id(v[it], slice0 + it * 32 + lane < A, E, status);
 #pragma unroll
   for (int it = 0; it < kIters; ++it) {
     const unsigned m = __match_any_sync(0xffffffffu, v[it]);
@@ -152,7 +158,9 @@ __global__ void __launch_bounds__(kWarps * 32) scatter_kernel(
   const unsigned lt = lanemask_lt();
   int v[kIters];
 #pragma unroll
-  for (int it = 0; it < kIters; ++it) v[it] = load_id(ids, slice0 + it * 32 + lane, A, E, nullptr);
+  for (int it = 0; it < kIters; ++it) v[it] = raw_id(ids, slice0 + it * 32 + lane, A);
+#pragma unroll
+  for (int it = 0; it < kIters; ++it) v[it] = checked_id(v[it], slice0 + it * 32 + lane < A, E, nullptr);
 #pragma unroll
   for (int it = 0; it < kIters; ++it) {
     const long long a = slice0 + it * 32 + lane;
@@ -181,7 +189,9 @@ __global__ void __launch_bounds__(kWarps * 32) scatter_kernel(
 // warp owns a contiguous slice, counts it into its private row, the rows are turned into
 // rank bases in warp order, and the slice is walked again to place each assignment.
 constexpr int kSmallWarps = 32;
-constexpr long long kSmallMax = 32768;
+constexpr int kSmallIters = 32;  // 32-id groups per warp
+constexpr int kGroup = 16;       // of which loaded together
+constexpr long long kSmallMax = (long long)kSmallWarps * 32 * kSmallIters;  // 32768
 
 __global__ void __launch_bounds__(kSmallWarps * 32) permute_small_kernel(
     const int32_t* __restrict__ ids, long long A, int E, long long cap, int32_t* __restrict__ counts,
@@ -191,16 +201,27 @@ __global__ void __launch_bounds__(kSmallWarps * 32) permute_small_kernel(
   __shared__ long long kept_s[kMaxE];
   __shared__ int offs[kMaxE];
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const long long slice = ((A + kSmallWarps * 32 - 1) / (kSmallWarps * 32)) * 32;  // ids per warp
-  const long long s0 = (long long)warp * slice;
+  const int iters = (int)((A + kSmallWarps * 32 - 1) / (kSmallWarps * 32));  // <= kSmallIters
+  const long long s0 = (long long)warp * iters * 32;
   for (int i = tid; i < kSmallWarps * kMaxE; i += blockDim.x) (&rows[0][0])[i] = 0;
   __syncthreads();
   int* row = rows[warp];
-  for (long long a0 = s0; a0 < s0 + slice; a0 += 32) {
-    const int id = load_id(ids, a0 + lane, A, E, status);
-    const unsigned m = __match_any_sync(0xffffffffu, id);
-    if (id >= 0 && lane == __ffs(m) - 1) row[id] += __popc(m);
-    __syncwarp();
+  // the slice is read in groups of kGroup ids per lane, each group one round of
+  // independent loads
+  for (int g0 = 0; g0 < iters; g0 += kGroup) {
+    int v[kGroup];
+#pragma unroll
+    for (int j = 0; j < kGroup; ++j)
+      v[j] = g0 + j < iters ? raw_id(ids, s0 + (g0 + j) * 32 + lane, A) : -1;
+#pragma unroll
+    for (int j = 0; j < kGroup; ++j)
+      v[j] = checked_id(v[j], g0 + j < iters && s0 + (g0 + j) * 32 + lane < A, E, status);
+#pragma unroll
+    for (int j = 0; j < kGroup; ++j) {
+      const unsigned m = __match_any_sync(0xffffffffu, v[j]);
+      if (v[j] >= 0 && lane == __ffs(m) - 1) row[v[j]] += __popc(m);
+      __syncwarp();
+    }
   }
   __syncthreads();
   long long run = 0;
@@ -232,24 +253,35 @@ __global__ void __launch_bounds__(kSmallWarps * 32) permute_small_kernel(
   }
   __syncthreads();
   const unsigned lt = lanemask_lt();
-  for (long long a0 = s0; a0 < s0 + slice; a0 += 32) {
-    const long long a = a0 + lane;
-    const int id = load_id(ids, a, A, E, nullptr);
-    const unsigned m = __match_any_sync(0xffffffffu, id);
-    int rank = 0;
-    if (id >= 0) rank = row[id] + __popc(m & lt);
-    __syncwarp();
-    if (id >= 0 && lane == __ffs(m) - 1) row[id] += __popc(m);
-    __syncwarp();
-    if (id >= 0) {
-      int p = -1;
-      if (cap < 0 || rank < cap) {
-        p = offs[id] + rank;
-        perm_to_assign[p] = (int32_t)a;
+  for (int g0 = 0; g0 < iters; g0 += kGroup) {
+    int v[kGroup];
+#pragma unroll
+    for (int j = 0; j < kGroup; ++j)
+      v[j] = g0 + j < iters ? raw_id(ids, s0 + (g0 + j) * 32 + lane, A) : -1;
+#pragma unroll
+    for (int j = 0; j < kGroup; ++j)
+      v[j] = checked_id(v[j], g0 + j < iters && s0 + (g0 + j) * 32 + lane < A, E, nullptr);
+#pragma unroll
+    for (int j = 0; j < kGroup; ++j) {
+      if (g0 + j >= iters) break;  // past this warp's slice (warp-uniform)
+      const long long a = s0 + (g0 + j) * 32 + lane;
+      const int id = v[j];
+      const unsigned m = __match_any_sync(0xffffffffu, id);
+      int rank = 0;
+      if (id >= 0) rank = row[id] + __popc(m & lt);
+      __syncwarp();
+      if (id >= 0 && lane == __ffs(m) - 1) row[id] += __popc(m);
+      __syncwarp();
+      if (id >= 0) {
+        int p = -1;
+        if (cap < 0 || rank < cap) {
+          p = offs[id] + rank;
+          perm_to_assign[p] = (int32_t)a;
+        }
+        assign_to_perm[a] = p;
+      } else if (a < A) {
+        assign_to_perm[a] = -1;
       }
-      assign_to_perm[a] = p;
-    } else if (a < A) {
-      assign_to_perm[a] = -1;
     }
   }
 }

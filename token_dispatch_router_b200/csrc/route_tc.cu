@@ -124,37 +124,30 @@ __device__ __forceinline__ float ld_dsmem(uint32_t remote_addr) {
   return v;
 }
 
-// Insert (v, e) into the descending list (ids arrive in ascending order, so an equal value
-// goes behind the ones already held: ties keep the lower id). `kth` caches the K-th value
-// once the list is full, so a value that does not enter costs one comparison.
-__device__ __forceinline__ void topk_insert(float (&bv)[KMAX], int (&be)[KMAX], int& cnt,
-                                            float& kth, int K, float v, int e) {
-  if (cnt == K && !(v > kth)) return;
-  float cv = v;
-  int ce = e;
-  bool placed = false;
+// Top-8 list, descending by (value, then lower id); empty slots have id -1. Ids arrive in
+// ascending order, so an existing entry with an equal value stays above the new one (ties
+// go to the lower id, +0 == -0). The top-K for K <= 8 is the first K slots. Every index is
+// a compile-time constant, so the list lives in registers.
+__device__ __forceinline__ void top8_insert(float (&bv)[KMAX], int (&be)[KMAX], float v, int e) {
+  if (be[KMAX - 1] >= 0 && !(v > bv[KMAX - 1])) return;  // does not enter
+  bool above[KMAX];  // the entry in slot j stays above the new one
 #pragma unroll
-  for (int j = 0; j < KMAX; ++j) {
-    if (j < K && !placed) {
-      if (j >= cnt) {
-        bv[j] = cv;
-        be[j] = ce;
-        placed = true;
-      } else if (cv > bv[j]) {
-        const float tv = bv[j];
-        const int te = be[j];
-        bv[j] = cv;
-        be[j] = ce;
-        cv = tv;
-        ce = te;
+  for (int j = 0; j < KMAX; ++j) above[j] = be[j] >= 0 && !(v > bv[j]);
+#pragma unroll
+  for (int j = KMAX - 1; j >= 1; --j) {
+    if (!above[j]) {
+      if (above[j - 1]) {
+        bv[j] = v;
+        be[j] = e;
+      } else {
+        bv[j] = bv[j - 1];
+        be[j] = be[j - 1];
       }
     }
   }
-  if (cnt < K) ++cnt;
-  if (cnt == K) {
-#pragma unroll
-    for (int j = 0; j < KMAX; ++j)
-      if (j == K - 1) kth = bv[j];
+  if (!above[0]) {
+    bv[0] = v;
+    be[0] = e;
   }
 }
 
@@ -291,8 +284,11 @@ __global__ void __launch_bounds__(R_THREADS) route_tc_kernel(const __grid_consta
     float* st_w = (float*)(st_i + RBM * K);             // [128][K]
     float bv[KMAX];
     int be[KMAX];
-    int cnt = 0;
-    float kth = -INFINITY;
+#pragma unroll
+    for (int k = 0; k < KMAX; ++k) {
+      bv[k] = -INFINITY;
+      be[k] = -1;
+    }
     float m = -INFINITY, ssum = 0.f;  // online max / sum of exp for the plain softmax
 #pragma unroll 1
     for (int c0 = 0; c0 < N; c0 += 16) {
@@ -318,7 +314,7 @@ __global__ void __launch_bounds__(R_THREADS) route_tc_kernel(const __grid_consta
           if (g.bias != nullptr) l += g.bias[e];
           if (t < g.T) {
             st_l[r * (E + 1) + e] = l;
-            topk_insert(bv, be, cnt, kth, K, l, e);
+            top8_insert(bv, be, l, e);
             if (!g.renorm) {
               if (l > m) {
                 ssum = ssum * expf(m - l) + 1.f;
@@ -428,7 +424,15 @@ moe_status launch_route_tc(const moe_shape& s, const void* x, const void* w_r, c
                            float* logits_out, int32_t* ids, float* w, cudaStream_t st) {
   const int tiles = (s.T + RBM - 1) / RBM;
   const int kblocks = s.d / RBK;
-  int S = (sm_count() + tiles - 1) / tiles;  // split d so that about one CTA per SM works
+  // Split d over S CTAs so that about one CTA per SM works, but never beyond the CTAs that
+  // can be resident at once (a second wave costs more than the split saves).
+  const int npad = ((s.E + 15) / 16) * 16;
+  const int nmma = npad <= 16 ? 16 : npad <= 32 ? 32 : npad <= 64 ? 64 : npad <= 128 ? 128 : 256;
+  const int smem_cta = RSTAGES * (RA_BYTES + ((nmma + 63) / 64) * RB_CHUNK) + 1024 + 256;
+  const int per_sm = (227 * 1024) / smem_cta;
+  int S = (sm_count() + tiles - 1) / tiles;
+  const int resident = sm_count() * (per_sm > 0 ? per_sm : 1);
+  if (S > resident / tiles) S = resident / tiles;
   if (S > 8) S = 8;
   if (S > kblocks) S = kblocks;
   if (S < 1) S = 1;
