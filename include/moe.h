@@ -146,10 +146,10 @@ moe_status moe_permute(const moe_shape* shape, const int32_t* topk_ids, int32_t*
  * of MOE_PERMUTE_STATIC_SCRATCH_BYTES inside the library, which every GPU that loads the
  * library holds until the process exits. It allocates nothing and calls no allocating
  * routine. Results are identical to moe_permute.
- *  - Limit: needs 2 * ceil(T*K / 4096) * E * 4 bytes of scratch (= moe_permute_workspace_size
+ *  - Limit: needs 2 * ceil(T*K / 1024) * E * 4 bytes of scratch (= moe_permute_workspace_size
  *    minus its 256-byte slack); larger problems return MOE_ERR_UNSUPPORTED and enqueue
- *    nothing. With the default 1 MiB: T*K up to about 2 million assignments at E = 256,
- *    8 million at E = 64.
+ *    nothing. With the default 1 MiB: T*K up to about 0.5 million assignments at E = 256,
+ *    2 million at E = 64.
  *  - Set-up: the first call on each device (with that device current) resolves the array's
  *    device address with cudaGetSymbolAddress; make that first call before any stream
  *    capture.
@@ -250,6 +250,13 @@ int moe_kernel_count(void);
 const char* moe_kernel_name(int id);
 moe_status moe_profile_query(int id, int64_t* launches, double* total_ms);
 int64_t moe_launch_count(void);
+
+/* Tile variant of the bf16 grouped GEMMs (process-wide, not thread safe): 0 = automatic
+ * (CTA-pair 256 x 256 tiles when T*K >= 512*E, else single-CTA 128 x 256 tiles), 1 = always
+ * single-CTA, 2 = always CTA pairs. Both compute the same result; the choice trades row
+ * padding (256-row tiles pad more) against traffic per SM (pairs move a third less). */
+moe_status moe_set_ffn_variant(int variant);
+int moe_get_ffn_variant(void);
 
 /* Test hook for the failure-detection path: launches one block that waits on
  * an mbarrier nothing will complete, bounded by `limit_ns` nanoseconds, then

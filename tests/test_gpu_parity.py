@@ -70,6 +70,14 @@ def check_permutation(perm, ids, E, C):
 _INPUTS = {}
 
 
+@pytest.fixture(params=[1, 2], ids=["single_cta", "cta_pair"])
+def ffn_variant(request, cuda_lib):
+    """Run a test with the single-CTA and with the CTA-pair grouped GEMM."""
+    cuda_lib.set_ffn_variant(request.param)
+    yield request.param
+    cuda_lib.set_ffn_variant(0)
+
+
 def inputs_for(cfg):
     if cfg.name not in _INPUTS:
         _INPUTS.clear()  # keep one large workload in host memory at a time
@@ -258,7 +266,7 @@ def test_grouped_ffn_fp32_tiny_workload(cuda_lib):
     (2500, 320, 256, 3, 1, 0.0),    # d = 320: down tile 256 + ragged 64
     (129, 64, 64, 1, 1, 0.0),       # one expert; one k-block; 2 M-tiles, the last has 1 row
 ])
-def test_grouped_ffn_bf16_tensor_cores(cuda_lib, T, d, n, E, K, cf):
+def test_grouped_ffn_bf16_tensor_cores(cuda_lib, ffn_variant, T, d, n, E, K, cf):
     tdr = cuda_lib
     a, a_ref, y, y_ref, out, out_ref = _ffn_case(tdr, T, d, n, E, K, cf, "bf16", T + d)
     assert_bf16_close(a, a_ref, "a_act")
@@ -287,7 +295,7 @@ def test_forward_tiny_fp32(cuda_lib):
 
 
 @pytest.mark.parametrize("name", ["mixtral_bf16", "fine_grained_bf16", "skewed_capacity_bf16"])
-def test_forward_full_size_workloads(cuda_lib, name):
+def test_forward_full_size_workloads(cuda_lib, ffn_variant, name):
     tdr = cuda_lib
     cfg = mi.CONFIGS[name]
     inp = inputs_for(cfg)
@@ -335,7 +343,7 @@ def test_dispatch_combine_identity_experts(cuda_lib, T):
     assert_status_ok(tdr)
 
 
-def test_forward_edge_cases(cuda_lib):
+def test_forward_edge_cases(cuda_lib, ffn_variant):
     tdr = cuda_lib
     # one token; one expert with K = 1; all tokens forced onto one expert; tiny capacity
     for (T, d, n, E, K, cf, force) in [(1, 64, 64, 4, 2, 0.0, False),

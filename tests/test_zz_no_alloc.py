@@ -52,7 +52,7 @@ def test_static_scratch_permute_matches_workspace_permute(cuda_lib, calls):
 def test_static_scratch_rejects_sizes_beyond_its_limit(cuda_lib):
     tdr = cuda_lib
     lib = tdr.load_library()
-    # 2 * ceil(T*K / 4096) * E * 4 bytes > 1 MiB
+    # 2 * ceil(T*K / 1024) * E * 4 bytes > 1 MiB
     s = tdr.make_shape(2_000_000, 64, 256, 8, 64, 0.0, True, torch.bfloat16)
     dummy = ctypes.c_void_p(256)  # never used: the size check fails first
     r = lib.moe_permute_static(ctypes.byref(s), dummy, dummy, dummy, dummy, dummy, None, None,

@@ -64,6 +64,8 @@ _SIGS = {
                                          ctypes.POINTER(ctypes.c_double)]),
     "moe_launch_count": (ctypes.c_int64, []),
     "moe_selftest_timeout": (ctypes.c_int, [ctypes.c_uint64, _P]),
+    "moe_set_ffn_variant": (ctypes.c_int, [ctypes.c_int]),
+    "moe_get_ffn_variant": (ctypes.c_int, []),
 }
 
 _lib: Optional[ctypes.CDLL] = None
@@ -339,6 +341,15 @@ class Profiler:
             if n.value:
                 out[self.lib.moe_kernel_name(i).decode()] = (int(n.value), float(ms.value))
         return out
+
+
+def set_ffn_variant(variant: int) -> None:
+    """0 = automatic, 1 = single-CTA 128 x 256 tiles, 2 = CTA-pair 256 x 256 tiles."""
+    _check(load_library().moe_set_ffn_variant(int(variant)), "moe_set_ffn_variant")
+
+
+def get_ffn_variant() -> int:
+    return int(load_library().moe_get_ffn_variant())
 
 
 def launch_count() -> int:

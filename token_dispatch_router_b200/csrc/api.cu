@@ -27,6 +27,9 @@ moe_status launch_combine(const moe_shape& s, const void* y_perm, const int32_t*
                           const float* topk_w, void* out, cudaStream_t st);
 moe_status launch_selftest_timeout(uint64_t limit_ns, cudaStream_t st);
 bool route_tc_supported(const moe_shape& s);
+moe_status launch_ffn_tc2(const moe_shape& s, const void* x, const int32_t* offsets,
+                          const int32_t* p2a, const void* w_gate, const void* w_up,
+                          const void* w_down, void* a_act, void* y_perm, cudaStream_t st);
 moe_status launch_permute_static(const moe_shape& s, const int32_t* ids, int32_t* counts,
                                  int32_t* offsets, int32_t* a2p, int32_t* p2a, const void* x,
                                  void* x_perm, cudaStream_t st);
@@ -75,7 +78,7 @@ namespace {
 const char* kKernelNames[K_COUNT] = {
     "route",        "hist",          "scan",           "scatter",     "gather_rows", "gateup_tc",
     "down_tc",      "gateup_simt",   "down_simt",      "combine",     "selftest_timeout",
-    "route_tc",     "permute_small"};
+    "route_tc",     "permute_small", "gateup_tc2",   "down_tc2"};
 
 struct ProfRec {
   int kid;
@@ -170,6 +173,16 @@ bool layout_of(const moe_shape& s, moe_workspace_layout* L) {
 }
 
 bool aligned16(const void* p) { return ((uintptr_t)p & 15) == 0; }
+
+int g_ffn_variant = 0;  // 0 auto, 1 single-CTA tiles, 2 CTA-pair tiles
+
+// CTA-pair tiles are 256 rows: worth their extra row padding only when the experts hold
+// several hundred rows on average.
+bool use_pair_gemm(const moe_shape& s) {
+  if (g_ffn_variant == 1) return false;
+  if (g_ffn_variant == 2) return true;
+  return (long long)s.T * s.K >= 512LL * s.E;
+}
 
 }  // namespace
 }  // namespace moe
@@ -272,9 +285,13 @@ moe_status moe_grouped_ffn(const moe_shape* s, const void* x, const int32_t* off
   if (!aligned16(x) || !aligned16(w_gate) || !aligned16(w_up) || !aligned16(w_down) ||
       !aligned16(a_act) || !aligned16(y_perm))
     return MOE_ERR_INVALID_ARG;
-  if (s->dtype == MOE_BF16)
+  if (s->dtype == MOE_BF16) {
+    if (use_pair_gemm(*s))
+      return launch_ffn_tc2(*s, x, offsets, perm_to_assign, w_gate, w_up, w_down, a_act, y_perm,
+                            (cudaStream_t)stream);
     return launch_ffn_tc(*s, x, offsets, perm_to_assign, w_gate, w_up, w_down, a_act, y_perm,
                          (cudaStream_t)stream);
+  }
   return launch_ffn_simt(*s, x, offsets, perm_to_assign, w_gate, w_up, w_down, a_act, y_perm,
                          (cudaStream_t)stream);
 }
@@ -386,6 +403,14 @@ int64_t moe_launch_count(void) {
   std::lock_guard<std::mutex> lk(g_prof_mu);
   return g_launches;
 }
+
+moe_status moe_set_ffn_variant(int variant) {
+  if (variant < 0 || variant > 2) return MOE_ERR_INVALID_ARG;
+  g_ffn_variant = variant;
+  return MOE_OK;
+}
+
+int moe_get_ffn_variant(void) { return g_ffn_variant; }
 
 moe_status moe_selftest_timeout(uint64_t limit_ns, moe_stream_t stream) {
   if (limit_ns == 0 || limit_ns > 10000000000ull) return MOE_ERR_INVALID_ARG;

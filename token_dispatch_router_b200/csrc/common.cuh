@@ -86,6 +86,8 @@ enum KernelId {
   K_SELFTEST,
   K_ROUTE_TC,
   K_PERMUTE_SMALL,
+  K_GATEUP_TC2,
+  K_DOWN_TC2,
   K_COUNT
 };
 

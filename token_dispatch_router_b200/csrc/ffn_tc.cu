@@ -517,6 +517,8 @@ __global__ void __launch_bounds__(GATEUP ? THREADS_GATEUP : THREADS_DOWN, 1)
   }
 }
 
+}  // namespace
+
 // ------------------------------------------------------------------ host: tensor maps
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
@@ -552,6 +554,8 @@ bool make_map(CUtensorMap* m, const void* ptr, int rank, const uint64_t* dims,
             bx, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
+
+namespace {
 
 template <bool GATEUP>
 moe_status run_gemm(const CUtensorMap& a, const CUtensorMap& b0, const CUtensorMap& b1,

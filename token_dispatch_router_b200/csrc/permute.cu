@@ -9,16 +9,19 @@
 // (gitcode.csdn.net), section 11: counts per expert, slot -> token, token slot -> slot.
 //
 // Atomic-free and deterministic. The T*K flat assignments are cut into chunks of
-// kChunk; a CTA owns a chunk and each of its 8 warps a contiguous slice of it.
+// kChunk (1024); a CTA owns a chunk and each of its 8 warps a contiguous slice of it.
 //   hist    : per warp, 32 ids at a time, __match_any_sync groups equal ids and the
 //             group's lowest lane adds the group size to the warp's private counter row
 //             (no two lanes touch one address); the CTA sums its 8 rows per expert.
-//   scan    : one CTA; per expert the chunk counts are scanned in chunk order (rank base
-//             of each chunk inside the expert), counts[e] is the total, kept = min(count,
-//             C) and offsets = exclusive scan of kept over experts.
+//   scan    : one CTA of 1024 threads, several per expert: each sums a run of chunks, a
+//             segmented prefix over the runs gives every chunk's rank base inside its
+//             expert; counts[e] is the total, kept = min(count, C) and offsets = exclusive
+//             scan of kept over experts. When chunks x experts is small the scatter CTAs
+//             derive their own bases and the offsets instead (two launches, not three).
 //   scatter : recomputes the warp rows, turns them into rank bases (chunk base + earlier
 //             warps), then walks the slice again: rank = base + (lanes of the group below
 //             me); rank < C -> slot offsets[e] + rank, else dropped (-1).
+// Problems of at most kSmallMax assignments run all three phases in one CTA.
 // Inside an expert the slots follow ascending flat index a = t*K + k, i.e. token order.
 #include <mutex>
 
@@ -29,7 +32,7 @@ namespace moe {
 namespace {
 
 constexpr int kWarps = 8;
-constexpr int kIters = 16;                   // 32-id groups per warp
+constexpr int kIters = 4;                    // 32-id groups per warp
 constexpr int kSlice = 32 * kIters;          // ids per warp
 constexpr int kChunk = kWarps * kSlice;      // ids per CTA
 constexpr int kMaxE = 256;
@@ -85,67 +88,129 @@ __global__ void __launch_bounds__(kWarps * 32) hist_kernel(const int32_t* __rest
   }
 }
 
-// One CTA of kMaxE threads: thread e walks the chunks of expert e in order.
-__global__ void __launch_bounds__(kMaxE) scan_kernel(const int32_t* __restrict__ chunk_counts,
-                                                     int32_t* __restrict__ chunk_base, int nchunks,
-                                                     int E, long long cap,
-                                                     int32_t* __restrict__ counts,
-                                                     int32_t* __restrict__ offsets) {
+// Chunk rank bases for many chunks: one CTA of kScanThreads threads, kScanThreads / Epad
+// of them per expert (Epad = E rounded up to a power of two), each owning a run of
+// consecutive chunks.
+constexpr int kScanThreads = 1024;
+constexpr long long kFusedScanMax = 8192;  // chunks x experts summed by every scatter CTA
+
+__global__ void __launch_bounds__(kScanThreads) scan_kernel(
+    const int32_t* __restrict__ chunk_counts, int32_t* __restrict__ chunk_base, int nchunks, int E,
+    int Epad, long long cap, int32_t* __restrict__ counts, int32_t* __restrict__ offsets) {
+  __shared__ long long part[kScanThreads];
   __shared__ long long kept_s[kMaxE];
-  const int e = threadIdx.x;
-  long long run = 0;
+  const int tid = threadIdx.x;
+  const int tpe = kScanThreads / Epad;  // threads per expert
+  const int e = tid / tpe, j = tid % tpe;
+  const int seg = (nchunks + tpe - 1) / tpe;
+  const int c0 = min(nchunks, j * seg), c1 = min(nchunks, c0 + seg);
+  long long sum = 0;
   if (e < E) {
-    int c = 0;
-    for (; c + 8 <= nchunks; c += 8) {  // 8 independent loads in flight
+    int c = c0;
+    for (; c + 8 <= c1; c += 8) {  // eight independent loads in flight
       int v[8];
 #pragma unroll
-      for (int j = 0; j < 8; ++j) v[j] = chunk_counts[(size_t)(c + j) * E + e];
+      for (int q = 0; q < 8; ++q) v[q] = chunk_counts[(size_t)(c + q) * E + e];
 #pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        chunk_base[(size_t)(c + j) * E + e] = (int32_t)run;
-        run += v[j];
-      }
+      for (int q = 0; q < 8; ++q) sum += v[q];
     }
-    for (; c < nchunks; ++c) {
-      const int v = chunk_counts[(size_t)c * E + e];
-      chunk_base[(size_t)c * E + e] = (int32_t)run;
-      run += v;
-    }
-    counts[e] = (int32_t)run;
+    for (; c < c1; ++c) sum += chunk_counts[(size_t)c * E + e];
   }
-  kept_s[e] = (e < E) ? (cap >= 0 && run > cap ? cap : run) : 0;
+  part[tid] = sum;
   __syncthreads();
-  // exclusive scan of kept over experts (Hillis-Steele on kMaxE entries)
-  for (int off = 1; off < kMaxE; off <<= 1) {
-    const long long add = (e >= off) ? kept_s[e - off] : 0;
+  for (int off = 1; off < tpe; off <<= 1) {  // inclusive prefix inside each expert's group
+    const long long add = (j >= off) ? part[tid - off] : 0;
     __syncthreads();
-    kept_s[e] += add;
+    part[tid] += add;
     __syncthreads();
   }
   if (e < E) {
-    const long long incl = kept_s[e];
-    const long long mine = (cap >= 0 && run > cap) ? cap : run;
-    offsets[e] = (int32_t)(incl - mine);
-    if (e == E - 1) offsets[E] = (int32_t)incl;
+    long long run = part[tid] - sum;  // exclusive: chunks before this run
+    for (int c = c0; c < c1; ++c) {
+      chunk_base[(size_t)c * E + e] = (int32_t)run;
+      run += chunk_counts[(size_t)c * E + e];
+    }
+  }
+  if (j == tpe - 1 && e < kMaxE) {
+    const long long total = (e < E) ? part[tid] : 0;
+    if (e < E) counts[e] = (int32_t)total;
+    kept_s[e] = (e < E) ? (cap >= 0 && total > cap ? cap : total) : 0;
+  }
+  __syncthreads();
+  for (int off = 1; off < Epad; off <<= 1) {  // inclusive scan of kept over experts
+    long long add = 0;
+    if (tid < Epad && tid >= off) add = kept_s[tid - off];
+    __syncthreads();
+    if (tid < Epad) kept_s[tid] += add;
+    __syncthreads();
+  }
+  if (tid < E) {
+    const long long prev = tid > 0 ? kept_s[tid - 1] : 0;
+    offsets[tid] = (int32_t)prev;
+    if (tid == E - 1) offsets[E] = (int32_t)kept_s[tid];
   }
 }
 
+// fused_scan: chunk_base is not given; every CTA sums the chunk counts itself (its bases:
+// chunks before it; the offsets: all chunks) and CTA 0 also writes counts and offsets.
 __global__ void __launch_bounds__(kWarps * 32) scatter_kernel(
     const int32_t* __restrict__ ids, long long A, int E, long long cap,
-    const int32_t* __restrict__ chunk_base, const int32_t* __restrict__ offsets,
+    const int32_t* __restrict__ chunk_counts, const int32_t* __restrict__ chunk_base,
+    int nchunks, int fused_scan, int32_t* __restrict__ counts, int32_t* __restrict__ offsets,
     int32_t* __restrict__ assign_to_perm, int32_t* __restrict__ perm_to_assign, unsigned* status) {
   __shared__ int rows[kWarps][kMaxE];
   __shared__ int offs[kMaxE];
+  __shared__ int cbase[kMaxE];
+  __shared__ long long kept_s[kMaxE];
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   for (int i = tid; i < kWarps * kMaxE; i += blockDim.x) (&rows[0][0])[i] = 0;
-  for (int e = tid; e < E; e += blockDim.x) offs[e] = offsets[e];
+  if (!fused_scan) {
+    for (int e = tid; e < E; e += blockDim.x) {
+      offs[e] = offsets[e];
+      cbase[e] = chunk_base[(size_t)blockIdx.x * E + e];
+    }
+  } else {
+    for (int e = tid; e < kMaxE; e += blockDim.x) {
+      long long before = 0, total = 0;
+      if (e < E) {
+        for (int c = 0; c < nchunks; ++c) {
+          const int v = chunk_counts[(size_t)c * E + e];
+          if (c < (int)blockIdx.x) before += v;
+          total += v;
+        }
+        if (blockIdx.x == 0) counts[e] = (int32_t)total;
+      }
+      cbase[e] = (int)before;
+      kept_s[e] = (e < E) ? (cap >= 0 && total > cap ? cap : total) : 0;
+    }
+    __syncthreads();
+    for (int off = 1; off < kMaxE; off <<= 1) {  // inclusive scan of kept over experts
+      long long add[kMaxE / (kWarps * 32)];
+#pragma unroll
+      for (int q = 0; q < kMaxE / (kWarps * 32); ++q) {
+        const int e = tid + q * kWarps * 32;
+        add[q] = e >= off ? kept_s[e - off] : 0;
+      }
+      __syncthreads();
+#pragma unroll
+      for (int q = 0; q < kMaxE / (kWarps * 32); ++q) kept_s[tid + q * kWarps * 32] += add[q];
+      __syncthreads();
+    }
+    for (int e = tid; e < E; e += blockDim.x) {
+      offs[e] = (int)(e > 0 ? kept_s[e - 1] : 0);
+      if (blockIdx.x == 0) {
+        offsets[e] = offs[e];
+        if (e == E - 1) offsets[E] = (int32_t)kept_s[e];
+      }
+    }
+  }
   __syncthreads();
   const long long slice0 = (long long)blockIdx.x * kChunk + (long long)warp * kSlice;
   warp_histogram(ids, slice0, A, E, rows[warp], nullptr);
   __syncthreads();
   // rank base of each warp row: chunk base + counts of the earlier warps of this chunk
   for (int e = tid; e < E; e += blockDim.x) {
-    int run = chunk_base[(size_t)blockIdx.x * E + e];
+    int run = cbase[e];
 #pragma unroll
     for (int w = 0; w < kWarps; ++w) {
       const int c = rows[w][e];
@@ -189,9 +254,9 @@ __global__ void __launch_bounds__(kWarps * 32) scatter_kernel(
 // warp owns a contiguous slice, counts it into its private row, the rows are turned into
 // rank bases in warp order, and the slice is walked again to place each assignment.
 constexpr int kSmallWarps = 32;
-constexpr int kSmallIters = 32;  // 32-id groups per warp
-constexpr int kGroup = 16;       // of which loaded together
-constexpr long long kSmallMax = (long long)kSmallWarps * 32 * kSmallIters;  // 32768
+constexpr int kSmallIters = 2;  // 32-id groups per warp
+constexpr int kGroup = 2;       // of which loaded together
+constexpr long long kSmallMax = (long long)kSmallWarps * 32 * kSmallIters;  // 2048
 
 __global__ void __launch_bounds__(kSmallWarps * 32) permute_small_kernel(
     const int32_t* __restrict__ ids, long long A, int E, long long cap, int32_t* __restrict__ counts,
@@ -352,13 +417,19 @@ moe_status launch_permute(const moe_shape& s, const int32_t* ids, int32_t* count
     launch_begin(K_HIST, st);
     hist_kernel<<<nchunks, kWarps * 32, 0, st>>>(ids, A, s.E, chunk_counts, status);
     if ((r = launch_end(K_HIST, st)) != MOE_OK) return r;
-    launch_begin(K_SCAN, st);
-    scan_kernel<<<1, kMaxE, 0, st>>>(chunk_counts, chunk_base, nchunks, s.E, cap, counts,
-                                     offsets);
-    if ((r = launch_end(K_SCAN, st)) != MOE_OK) return r;
+    const int fused = (long long)nchunks * s.E <= kFusedScanMax;
+    if (!fused) {
+      int epad = 1;
+      while (epad < s.E) epad <<= 1;
+      launch_begin(K_SCAN, st);
+      scan_kernel<<<1, kScanThreads, 0, st>>>(chunk_counts, chunk_base, nchunks, s.E, epad, cap,
+                                              counts, offsets);
+      if ((r = launch_end(K_SCAN, st)) != MOE_OK) return r;
+    }
     launch_begin(K_SCATTER, st);
-    scatter_kernel<<<nchunks, kWarps * 32, 0, st>>>(ids, A, s.E, cap, chunk_base, offsets, a2p,
-                                                    p2a, status);
+    scatter_kernel<<<nchunks, kWarps * 32, 0, st>>>(ids, A, s.E, cap, chunk_counts, chunk_base,
+                                                    nchunks, fused, counts, offsets, a2p, p2a,
+                                                    status);
     if ((r = launch_end(K_SCATTER, st)) != MOE_OK) return r;
   }
   if (x != nullptr && x_perm != nullptr && A > 0) {
