@@ -364,17 +364,20 @@ def run_ours(args, rank, world, local):
     peaks, peak_src = load_peaks()
     flops_gateup = 4.0 * cfg.d * cfg.n * a_kept
     flops_down = 2.0 * cfg.d * cfg.n * a_kept
-    n_g, ms_g = kern.get("gateup_tc", (0, 0.0))
-    n_d, ms_d = kern.get("down_tc", (0, 0.0))
+    # the grouped GEMMs run as single-CTA (`*_tc`) or CTA-pair (`*_tc2`) kernels
+    g_name = "gateup_tc2" if "gateup_tc2" in kern else "gateup_tc"
+    d_name = "down_tc2" if "down_tc2" in kern else "down_tc"
+    n_g, ms_g = kern.get(g_name, (0, 0.0))
+    n_d, ms_d = kern.get(d_name, (0, 0.0))
     avg_g = ms_g / max(n_g, 1)
     avg_d = ms_d / max(n_d, 1)
     peak_t = float(peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"]))
     ach_g = flops_gateup / (avg_g / 1e3) / 1e12 if avg_g > 0 else 0.0
     ach_d = flops_down / (avg_d / 1e3) / 1e12 if avg_d > 0 else 0.0
     ach_gemm = (flops_gateup + flops_down) / ((avg_g + avg_d) / 1e3) / 1e12 if avg_g > 0 else 0.0
-    roofline = {"bound": "tensor", "kernel": "gateup_tc", "achieved": round(ach_g, 2),
+    roofline = {"bound": "tensor", "kernel": g_name, "achieved": round(ach_g, 2),
                 "peak": peak_t, "unit": "TFLOP/s", "frac": round(ach_g / peak_t, 4),
-                "traffic": traffic_for("gateup_tc", cfg.name),
+                "traffic": traffic_for(g_name, cfg.name),
                 "peak_source": f"{peak_src} bf16_tflops_sustained (kernel timed inside a long "
                                "step loop)",
                 "algorithmic": "4*d*n*A_kept FLOP per launch (gate and up GEMMs)",

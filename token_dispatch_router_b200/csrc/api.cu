@@ -20,16 +20,14 @@ moe_status launch_permute(const moe_shape& s, const int32_t* ids, int32_t* count
 moe_status launch_ffn_simt(const moe_shape& s, const void* x, const int32_t* offsets,
                            const int32_t* p2a, const void* w_gate, const void* w_up,
                            const void* w_down, void* a_act, void* y_perm, cudaStream_t st);
-moe_status launch_ffn_tc(const moe_shape& s, const void* x, const int32_t* offsets,
-                         const int32_t* p2a, const void* w_gate, const void* w_up,
-                         const void* w_down, void* a_act, void* y_perm, cudaStream_t st);
 moe_status launch_combine(const moe_shape& s, const void* y_perm, const int32_t* a2p,
                           const float* topk_w, void* out, cudaStream_t st);
 moe_status launch_selftest_timeout(uint64_t limit_ns, cudaStream_t st);
 bool route_tc_supported(const moe_shape& s);
-moe_status launch_ffn_tc2(const moe_shape& s, const void* x, const int32_t* offsets,
-                          const int32_t* p2a, const void* w_gate, const void* w_up,
-                          const void* w_down, void* a_act, void* y_perm, cudaStream_t st);
+moe_status launch_ffn_tc_mixed(const moe_shape& s, const void* x, const int32_t* offsets,
+                               const int32_t* p2a, const void* w_gate, const void* w_up,
+                               const void* w_down, void* a_act, void* y_perm, bool pair_gateup,
+                               bool pair_down, cudaStream_t st);
 moe_status launch_permute_static(const moe_shape& s, const int32_t* ids, int32_t* counts,
                                  int32_t* offsets, int32_t* a2p, int32_t* p2a, const void* x,
                                  void* x_perm, cudaStream_t st);
@@ -176,13 +174,15 @@ bool aligned16(const void* p) { return ((uintptr_t)p & 15) == 0; }
 
 int g_ffn_variant = 0;  // 0 auto, 1 single-CTA tiles, 2 CTA-pair tiles
 
-// CTA-pair tiles are 256 rows: worth their extra row padding only when the experts hold
-// several hundred rows on average.
-bool use_pair_gemm(const moe_shape& s) {
-  if (g_ffn_variant == 1) return false;
-  if (g_ffn_variant == 2) return true;
+// Automatic choice, from measurements on B200: the gate/up GEMM runs single-CTA tiles
+// (its gathered A operand gains nothing from pairing, and 256-row tiles pad twice as many
+// rows); the down GEMM runs on CTA pairs once experts average at least 512 rows, where the
+// pair's deeper pipeline beats the extra padding.
+bool use_pair_down(const moe_shape& s) {
+  if (g_ffn_variant != 0) return g_ffn_variant == 2;
   return (long long)s.T * s.K >= 512LL * s.E;
 }
+bool use_pair_gateup() { return g_ffn_variant == 2; }
 
 }  // namespace
 }  // namespace moe
@@ -285,13 +285,9 @@ moe_status moe_grouped_ffn(const moe_shape* s, const void* x, const int32_t* off
   if (!aligned16(x) || !aligned16(w_gate) || !aligned16(w_up) || !aligned16(w_down) ||
       !aligned16(a_act) || !aligned16(y_perm))
     return MOE_ERR_INVALID_ARG;
-  if (s->dtype == MOE_BF16) {
-    if (use_pair_gemm(*s))
-      return launch_ffn_tc2(*s, x, offsets, perm_to_assign, w_gate, w_up, w_down, a_act, y_perm,
-                            (cudaStream_t)stream);
-    return launch_ffn_tc(*s, x, offsets, perm_to_assign, w_gate, w_up, w_down, a_act, y_perm,
-                         (cudaStream_t)stream);
-  }
+  if (s->dtype == MOE_BF16)
+    return launch_ffn_tc_mixed(*s, x, offsets, perm_to_assign, w_gate, w_up, w_down, a_act, y_perm,
+                               use_pair_gateup(), use_pair_down(*s), (cudaStream_t)stream);
   return launch_ffn_simt(*s, x, offsets, perm_to_assign, w_gate, w_up, w_down, a_act, y_perm,
                          (cudaStream_t)stream);
 }

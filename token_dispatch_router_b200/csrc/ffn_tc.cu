@@ -33,7 +33,7 @@
 // sync. Every mbarrier wait is bounded (kWaitLimitNs); on expiry the CTA records
 // MOE_ERR_TIMEOUT, stops issuing, waits (bounded) for its copies and MMAs in flight,
 // frees its TMEM and returns.
-#include "common.cuh"
+#include "ffn_args.cuh"
 
 namespace moe {
 
@@ -59,21 +59,6 @@ constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 + SMEM_TAIL;
 constexpr uint32_t IDESC = (1u << 4) | (1u << 7) | (1u << 10) | (1u << 16) |
                            ((uint32_t)(BN >> 3) << 17) | ((uint32_t)(BM >> 4) << 24);
 
-struct GemmArgs {
-  const int32_t* offsets;
-  const int32_t* p2a;
-  const uint8_t* x;  // gate/up: token rows gathered by cp.async
-  long long x_row_bytes;
-  bf16* out;
-  int ld_out;    // elements per output row
-  int n_out;     // valid output columns
-  int out_tile;  // output columns per tile (128 gate/up, 256 down)
-  int n_tiles;
-  int kblocks;   // contraction / 64
-  int E, K, T;
-  unsigned* status;
-  unsigned long long limit_ns;
-};
 
 // ------------------------------------------------------------------ PTX wrappers
 __device__ __forceinline__ uint32_t saddr(const void* p) {
@@ -475,8 +460,8 @@ __global__ void __launch_bounds__(GATEUP ? THREADS_GATEUP : THREADS_DOWN, 1)
             for (int j = 0; j < 16; ++j) {
               const float g0 = __uint_as_float(gv[2 * j]), g1 = __uint_as_float(gv[2 * j + 1]);
               const float u0 = __uint_as_float(uv[2 * j]), u1 = __uint_as_float(uv[2 * j + 1]);
-              const float h0 = g0 / (1.f + expf(-g0)) * u0;
-              const float h1 = g1 / (1.f + expf(-g1)) * u1;
+              const float h0 = __fdividef(g0, 1.f + __expf(-g0)) * u0;
+              const float h1 = __fdividef(g1, 1.f + __expf(-g1)) * u1;
               pk[j] = pack_bf16x2(h0, h1);
             }
             uint4* dst = reinterpret_cast<uint4*>(orow + col);
@@ -538,7 +523,6 @@ EncodeTiledFn encode_fn() {
   return fn;
 }
 
-// bf16 tensor of `rank` dims (innermost first), 128-byte swizzle, zero fill out of bounds.
 bool make_map(CUtensorMap* m, const void* ptr, int rank, const uint64_t* dims,
               const uint64_t* strides_bytes, const uint32_t* box) {
   EncodeTiledFn fn = encode_fn();
@@ -597,30 +581,33 @@ moe_status launch_selftest_timeout(uint64_t limit_ns, cudaStream_t st) {
   return launch_end(K_SELFTEST, st);
 }
 
-moe_status launch_ffn_tc(const moe_shape& s, const void* x, const int32_t* offsets,
-                         const int32_t* p2a, const void* w_gate, const void* w_up,
-                         const void* w_down, void* a_act, void* y_perm, cudaStream_t st) {
-  const long long A = (long long)s.T * s.K;
-  if (A == 0) return MOE_OK;
-  const uint64_t d = s.d, n = s.n, E = s.E;
+// Tensor maps and arguments of both GEMMs for one call.
+struct FfnMaps {
   CUtensorMap mg, mu, ma, md;
+  GemmArgs gate_up, down;
+};
+
+static moe_status prepare_ffn(const moe_shape& s, const void* x, const int32_t* offsets,
+                              const int32_t* p2a, const void* w_gate, const void* w_up,
+                              const void* w_down, void* a_act, void* y_perm, FfnMaps& f) {
+  const uint64_t d = s.d, n = s.n, E = s.E, A = (uint64_t)s.T * s.K;
   {
     const uint64_t dims[3] = {n, d, E}, str[2] = {n * 2, d * n * 2};
     const uint32_t box[3] = {64, 64, 1};
-    if (!make_map(&mg, w_gate, 3, dims, str, box)) return MOE_ERR_CUDA;
-    if (!make_map(&mu, w_up, 3, dims, str, box)) return MOE_ERR_CUDA;
+    if (!make_map(&f.mg, w_gate, 3, dims, str, box)) return MOE_ERR_CUDA;
+    if (!make_map(&f.mu, w_up, 3, dims, str, box)) return MOE_ERR_CUDA;
   }
   {
-    const uint64_t dims[2] = {n, (uint64_t)A}, str[1] = {n * 2};
+    const uint64_t dims[2] = {n, A}, str[1] = {n * 2};
     const uint32_t box[2] = {64, 128};
-    if (!make_map(&ma, a_act, 2, dims, str, box)) return MOE_ERR_CUDA;
+    if (!make_map(&f.ma, a_act, 2, dims, str, box)) return MOE_ERR_CUDA;
   }
   {
     const uint64_t dims[3] = {d, n, E}, str[2] = {d * 2, n * d * 2};
     const uint32_t box[3] = {64, 64, 1};
-    if (!make_map(&md, w_down, 3, dims, str, box)) return MOE_ERR_CUDA;
+    if (!make_map(&f.md, w_down, 3, dims, str, box)) return MOE_ERR_CUDA;
   }
-  GemmArgs ga;
+  GemmArgs& ga = f.gate_up;
   ga.offsets = offsets;
   ga.p2a = p2a;
   ga.x = (const uint8_t*)x;
@@ -630,24 +617,39 @@ moe_status launch_ffn_tc(const moe_shape& s, const void* x, const int32_t* offse
   ga.T = s.T;
   ga.status = device_status_ptr();
   ga.limit_ns = kWaitLimitNs;
-
   ga.out = (bf16*)a_act;
   ga.ld_out = s.n;
   ga.n_out = s.n;
   ga.out_tile = 128;
   ga.n_tiles = (s.n + 127) / 128;
   ga.kblocks = s.d / BK;
-  moe_status r = run_gemm<true>(mg, mg, mu, ga, st, K_GATEUP_TC);
-  if (r != MOE_OK) return r;
-
-  GemmArgs gd = ga;
+  GemmArgs& gd = f.down;
+  gd = ga;
   gd.out = (bf16*)y_perm;
   gd.ld_out = s.d;
   gd.n_out = s.d;
   gd.out_tile = BN;
   gd.n_tiles = (s.d + BN - 1) / BN;
   gd.kblocks = s.n / BK;
-  return run_gemm<false>(ma, md, md, gd, st, K_DOWN_TC);
+  return MOE_OK;
+}
+
+moe_status launch_ffn_tc2_gemm(bool gateup, const CUtensorMap& a, const CUtensorMap& b0,
+                               const CUtensorMap& b1, const GemmArgs& args, cudaStream_t st);
+
+moe_status launch_ffn_tc_mixed(const moe_shape& s, const void* x, const int32_t* offsets,
+                               const int32_t* p2a, const void* w_gate, const void* w_up,
+                               const void* w_down, void* a_act, void* y_perm, bool pair_gateup,
+                               bool pair_down, cudaStream_t st) {
+  if ((long long)s.T * s.K == 0) return MOE_OK;
+  FfnMaps f;
+  moe_status r = prepare_ffn(s, x, offsets, p2a, w_gate, w_up, w_down, a_act, y_perm, f);
+  if (r != MOE_OK) return r;
+  r = pair_gateup ? launch_ffn_tc2_gemm(true, f.mg, f.mg, f.mu, f.gate_up, st)
+                  : run_gemm<true>(f.mg, f.mg, f.mu, f.gate_up, st, K_GATEUP_TC);
+  if (r != MOE_OK) return r;
+  return pair_down ? launch_ffn_tc2_gemm(false, f.ma, f.md, f.md, f.down, st)
+                   : run_gemm<false>(f.ma, f.md, f.md, f.down, st, K_DOWN_TC);
 }
 
 }  // namespace moe

@@ -17,12 +17,10 @@
 // (peer); the leader commits each stage to both CTAs' empty barriers and each tile to both
 // CTAs' accumulator-full barriers; both CTAs' epilogue warps arrive on the leader's
 // accumulator-empty barrier. Every wait is bounded (MOE_ERR_TIMEOUT on expiry).
+#include "ffn_args.cuh"
 #include "tc_ptx.cuh"
 
 namespace moe {
-
-bool make_map(CUtensorMap* m, const void* ptr, int rank, const uint64_t* dims,
-              const uint64_t* strides_bytes, const uint32_t* box);
 
 namespace {
 
@@ -45,17 +43,6 @@ constexpr int SMEM_TAIL = 4096;
 constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 + SMEM_TAIL;
 constexpr uint32_t IDESC = idesc_bf16(PAIR_M, BN);
 
-struct Args2 {
-  const int32_t* offsets;
-  const int32_t* p2a;
-  const uint8_t* x;
-  long long x_row_bytes;
-  bf16* out;
-  int ld_out, n_out, out_tile, n_tiles, kblocks;
-  int E, K, T;
-  unsigned* status;
-  unsigned long long limit_ns;
-};
 
 struct Tile2 {
   int e, m0, rows, n0, m0_pair;  // m0 / rows: this CTA's half of the pair's 256 rows
@@ -84,7 +71,7 @@ template <bool GATEUP>
 __global__ void __launch_bounds__(GATEUP ? THREADS_GATEUP : THREADS_DOWN, 1)
     grouped_gemm_tc2(const __grid_constant__ CUtensorMap tmA,
                      const __grid_constant__ CUtensorMap tmB0,
-                     const __grid_constant__ CUtensorMap tmB1, const Args2 g) {
+                     const __grid_constant__ CUtensorMap tmB1, const GemmArgs g) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* base = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
   uint8_t* ring = base;
@@ -102,8 +89,11 @@ __global__ void __launch_bounds__(GATEUP ? THREADS_GATEUP : THREADS_DOWN, 1)
   int* s_mt = s_cum + MAXE + 1;
 
   constexpr int NTHREADS = GATEUP ? THREADS_GATEUP : THREADS_DOWN;
-  // leader's full[s]: one expect_tx arrival per CTA (+ leader gathers + peer relay)
-  constexpr uint32_t FULL_COUNT = GATEUP ? 2 + GATHER_THREADS + 1 : 2;
+  // leader's full[s]: the leader's expect_tx arrival for the TMA bytes of both CTAs (+ the
+  // leader's gather threads + the peer's relay). The peer's loads complete on it without
+  // an arrival of their own: a transaction count may run ahead of its expect_tx, and the
+  // phase cannot complete before the leader's arrival anyway.
+  constexpr uint32_t FULL_COUNT = GATEUP ? 1 + GATHER_THREADS + 1 : 1;
   constexpr uint32_t TMA_BYTES = GATEUP ? B_HALF : STAGE_BYTES;  // per CTA and stage
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -182,7 +172,7 @@ __global__ void __launch_bounds__(GATEUP ? THREADS_GATEUP : THREADS_DOWN, 1)
           break;
         }
         const uint32_t fb = map_rank(saddr(&full[stage]), 0);  // the leader's barrier
-        if (lane == 0) mbar_expect_tx_remote(fb, TMA_BYTES);
+        if (leader && lane == 0) mbar_expect_tx(saddr(&full[stage]), 2 * TMA_BYTES);
         __syncwarp();
         const uint32_t a_dst = saddr(ring + stage * STAGE_BYTES);
         const uint32_t b_dst = a_dst + A_BYTES;
@@ -374,7 +364,7 @@ __global__ void __launch_bounds__(GATEUP ? THREADS_GATEUP : THREADS_DOWN, 1)
             for (int j = 0; j < 16; ++j) {
               const float g0 = __uint_as_float(gv[2 * j]), g1 = __uint_as_float(gv[2 * j + 1]);
               const float u0 = __uint_as_float(uv[2 * j]), u1 = __uint_as_float(uv[2 * j + 1]);
-              pk[j] = pack_bf16x2(g0 / (1.f + expf(-g0)) * u0, g1 / (1.f + expf(-g1)) * u1);
+              pk[j] = pack_bf16x2(__fdividef(g0, 1.f + __expf(-g0)) * u0, __fdividef(g1, 1.f + __expf(-g1)) * u1);
             }
             uint4* dst = reinterpret_cast<uint4*>(orow + col);
 #pragma unroll
@@ -417,7 +407,7 @@ __global__ void __launch_bounds__(GATEUP ? THREADS_GATEUP : THREADS_DOWN, 1)
 
 template <bool GATEUP>
 moe_status run_gemm2(const CUtensorMap& a, const CUtensorMap& b0, const CUtensorMap& b1,
-                     const Args2& args, cudaStream_t st, int kid) {
+                     const GemmArgs& args, cudaStream_t st, int kid) {
   auto kern = grouped_gemm_tc2<GATEUP>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES) !=
       cudaSuccess)
@@ -442,55 +432,10 @@ moe_status run_gemm2(const CUtensorMap& a, const CUtensorMap& b0, const CUtensor
 
 }  // namespace
 
-moe_status launch_ffn_tc2(const moe_shape& s, const void* x, const int32_t* offsets,
-                          const int32_t* p2a, const void* w_gate, const void* w_up,
-                          const void* w_down, void* a_act, void* y_perm, cudaStream_t st) {
-  const long long A = (long long)s.T * s.K;
-  if (A == 0) return MOE_OK;
-  const uint64_t d = s.d, n = s.n, E = s.E;
-  CUtensorMap mg, mu, ma, md;
-  {
-    const uint64_t dims[3] = {n, d, E}, str[2] = {n * 2, d * n * 2};
-    const uint32_t box[3] = {64, 64, 1};
-    if (!make_map(&mg, w_gate, 3, dims, str, box)) return MOE_ERR_CUDA;
-    if (!make_map(&mu, w_up, 3, dims, str, box)) return MOE_ERR_CUDA;
-  }
-  {
-    const uint64_t dims[2] = {n, (uint64_t)A}, str[1] = {n * 2};
-    const uint32_t box[2] = {64, 128};
-    if (!make_map(&ma, a_act, 2, dims, str, box)) return MOE_ERR_CUDA;
-  }
-  {
-    const uint64_t dims[3] = {d, n, E}, str[2] = {d * 2, n * d * 2};
-    const uint32_t box[3] = {64, 64, 1};
-    if (!make_map(&md, w_down, 3, dims, str, box)) return MOE_ERR_CUDA;
-  }
-  Args2 ga;
-  ga.offsets = offsets;
-  ga.p2a = p2a;
-  ga.x = (const uint8_t*)x;
-  ga.x_row_bytes = (long long)s.d * 2;
-  ga.E = s.E;
-  ga.K = s.K;
-  ga.T = s.T;
-  ga.status = device_status_ptr();
-  ga.limit_ns = kWaitLimitNs;
-  ga.out = (bf16*)a_act;
-  ga.ld_out = s.n;
-  ga.n_out = s.n;
-  ga.out_tile = 128;
-  ga.n_tiles = (s.n + 127) / 128;
-  ga.kblocks = s.d / BK;
-  moe_status r = run_gemm2<true>(mg, mg, mu, ga, st, K_GATEUP_TC2);
-  if (r != MOE_OK) return r;
-  Args2 gd = ga;
-  gd.out = (bf16*)y_perm;
-  gd.ld_out = s.d;
-  gd.n_out = s.d;
-  gd.out_tile = BN;
-  gd.n_tiles = (s.d + BN - 1) / BN;
-  gd.kblocks = s.n / BK;
-  return run_gemm2<false>(ma, md, md, gd, st, K_DOWN_TC2);
+moe_status launch_ffn_tc2_gemm(bool gateup, const CUtensorMap& a, const CUtensorMap& b0,
+                               const CUtensorMap& b1, const GemmArgs& args, cudaStream_t st) {
+  return gateup ? run_gemm2<true>(a, b0, b1, args, st, K_GATEUP_TC2)
+                : run_gemm2<false>(a, b0, b1, args, st, K_DOWN_TC2);
 }
 
 }  // namespace moe
