@@ -47,7 +47,10 @@ def parse():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="mixtral_bf16")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--cpu-tokens", type=int, default=8, help="tokens in the CPU oracle sample")
+    ap.add_argument("--cpu-tokens", type=int, default=1024,
+                    help="tokens in the CPU oracle sample (about 10-30 s of host work)")
+    ap.add_argument("--ref-tokens", type=int, default=64,
+                    help="tokens per step of the reference arm (the CPU oracle)")
     return ap.parse_args()
 
 
@@ -229,7 +232,7 @@ def run_reference(args, rank, world):
     cfg = mi.CONFIGS[args.workload]
     inp = mi.make_inputs(cfg)
     wide = {}
-    per_step = max(1, args.cpu_tokens // 4)
+    per_step = max(1, args.ref_tokens)
     for i in range(args.warmup):
         cpu_oracle_tokens_per_s(inp, per_step, start=i * per_step, wide=wide)
     total_t, total_tok = 0.0, 0

@@ -172,7 +172,7 @@ def permute(shape: moe_shape, topk_ids: torch.Tensor, x=None, materialize: bool 
     counts = torch.empty(E, dtype=torch.int32, device=dev)
     offsets = torch.empty(E + 1, dtype=torch.int32, device=dev)
     a2p = torch.empty(T * K, dtype=torch.int32, device=dev)
-    p2a = torch.full((T * K,), -1, dtype=torch.int32, device=dev)
+    p2a = torch.empty(T * K, dtype=torch.int32, device=dev)  # tail past offsets[E] unwritten
     x_perm = None
     if materialize:
         _dev(x, "x", _act_dtype(shape), (T, shape.d))
@@ -201,7 +201,7 @@ def permute_static(shape: moe_shape, topk_ids: torch.Tensor, x=None, materialize
     counts = torch.empty(E, dtype=torch.int32, device=dev)
     offsets = torch.empty(E + 1, dtype=torch.int32, device=dev)
     a2p = torch.empty(T * K, dtype=torch.int32, device=dev)
-    p2a = torch.full((T * K,), -1, dtype=torch.int32, device=dev)
+    p2a = torch.empty(T * K, dtype=torch.int32, device=dev)  # tail past offsets[E] unwritten
     x_perm = None
     if materialize:
         _dev(x, "x", _act_dtype(shape), (T, shape.d))
