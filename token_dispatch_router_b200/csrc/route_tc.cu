@@ -28,11 +28,14 @@ namespace moe {
 
 namespace {
 
-constexpr int RBM = 128, RBK = 64, RSTAGES = 4;
+constexpr int RBM = 128, RBK = 64;
 constexpr int RA_BYTES = RBM * RBK * 2;  // 16 KB
 constexpr int RB_CHUNK = RBK * 64 * 2;   // 8 KB: 64 k-rows x 64 experts
 constexpr int R_THREADS = 128;
 constexpr int KMAX = 8;
+
+// Pipeline depth: the x stream is latency-bound per CTA, so small-N stages (24 KB) go 8 deep.
+__host__ __device__ constexpr int route_stages(int N) { return N <= 64 ? 8 : (N <= 128 ? 6 : 4); }
 
 struct RouteArgs {
   const float* bias;
@@ -158,6 +161,7 @@ __global__ void __launch_bounds__(R_THREADS) route_tc_kernel(const __grid_consta
   constexpr int NCH = (N + 63) / 64;         // B chunks of 64 experts
   constexpr int B_BYTES = NCH * RB_CHUNK;
   constexpr int STAGE = RA_BYTES + B_BYTES;
+  constexpr int RSTAGES = route_stages(N);
   constexpr uint32_t TCOLS = N <= 32 ? 32 : (N <= 64 ? 64 : (N <= 128 ? 128 : 256));
   constexpr uint32_t IDESC = (1u << 4) | (1u << 7) | (1u << 10) | (1u << 16) |
                              ((uint32_t)(N >> 3) << 17) | ((uint32_t)(RBM >> 4) << 24);
@@ -393,7 +397,7 @@ moe_status launch_n(const CUtensorMap& mx, const CUtensorMap& mw, const RouteArg
                     cudaStream_t st) {
   constexpr int NCH = (N + 63) / 64;
   constexpr int STAGE = RA_BYTES + NCH * RB_CHUNK;
-  const int smem = RSTAGES * STAGE + 1024 + 256;
+  const int smem = route_stages(N) * STAGE + 1024 + 256;
   auto kern = route_tc_kernel<N>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
     return MOE_ERR_CUDA;
@@ -428,7 +432,8 @@ moe_status launch_route_tc(const moe_shape& s, const void* x, const void* w_r, c
   // can be resident at once (a second wave costs more than the split saves).
   const int npad = ((s.E + 15) / 16) * 16;
   const int nmma = npad <= 16 ? 16 : npad <= 32 ? 32 : npad <= 64 ? 64 : npad <= 128 ? 128 : 256;
-  const int smem_cta = RSTAGES * (RA_BYTES + ((nmma + 63) / 64) * RB_CHUNK) + 1024 + 256;
+  const int smem_cta =
+      route_stages(nmma) * (RA_BYTES + ((nmma + 63) / 64) * RB_CHUNK) + 1024 + 256;
   const int per_sm = (227 * 1024) / smem_cta;
   int S = (sm_count() + tiles - 1) / tiles;
   const int resident = sm_count() * (per_sm > 0 ? per_sm : 1);
