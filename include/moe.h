@@ -251,11 +251,13 @@ const char* moe_kernel_name(int id);
 moe_status moe_profile_query(int id, int64_t* launches, double* total_ms);
 int64_t moe_launch_count(void);
 
-/* Tile variant of the bf16 grouped GEMMs (process-wide, not thread safe): 0 = automatic
- * (currently the single-CTA 128 x 256 tiles), 1 = always single-CTA, 2 = always CTA pairs
- * (256 x 256 tiles on two SMs, tcgen05 cta_group::2). Both compute the same result; the
- * choice trades row padding (256-row tiles pad more) against traffic per SM (pairs move a
- * third less). */
+/* Tile variant of the bf16 grouped GEMMs (process-wide, not thread safe): 0 = automatic,
+ * 1 = always single-CTA 128 x 256 tiles, 2 = always CTA pairs (256 x 256 tiles on two SMs,
+ * tcgen05 cta_group::2) with the gate/up A rows gathered inside the GEMM, 3 = CTA pairs with
+ * the gate/up A rows first copied expert-major into the y_perm buffer by one gather kernel
+ * and loaded from there by TMA. All compute the same result; the choice trades row padding
+ * (256-row tiles pad more) and the extra copy against traffic per SM (pairs move a third
+ * less). */
 moe_status moe_set_ffn_variant(int variant);
 int moe_get_ffn_variant(void);
 

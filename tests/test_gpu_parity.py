@@ -70,9 +70,10 @@ def check_permutation(perm, ids, E, C):
 _INPUTS = {}
 
 
-@pytest.fixture(params=[1, 2], ids=["single_cta", "cta_pair"])
+@pytest.fixture(params=[1, 2, 3], ids=["single_cta", "cta_pair", "cta_pair_tma_a"])
 def ffn_variant(request, cuda_lib):
-    """Run a test with the single-CTA and with the CTA-pair grouped GEMM."""
+    """Run a test with the single-CTA grouped GEMM, the CTA-pair one gathering its rows, and
+    the CTA-pair one reading rows copied expert-major beforehand."""
     cuda_lib.set_ffn_variant(request.param)
     yield request.param
     cuda_lib.set_ffn_variant(0)
@@ -105,6 +106,12 @@ def test_bounded_wait_times_out_and_reports(cuda_lib):
     (33, 64, 6, 3, "f32", False, False),
     (1, 64, 1, 1, "bf16", False, True),
     (129, 192, 64, 6, "bf16", True, False),
+    # bf16 with few experts: ragged tiles, E below 8, K up to E, long d
+    (301, 2880, 8, 3, "bf16", True, False),
+    (5, 2048, 4, 4, "bf16", True, True),
+    (1027, 256, 7, 2, "bf16", False, False),
+    (9001, 4096, 8, 8, "bf16", True, True),
+    (70, 4160, 8, 2, "bf16", False, True),
 ])
 def test_route_matches_oracle(cuda_lib, T, d, E, K, dtype, bias, renorm):
     tdr = cuda_lib
@@ -137,6 +144,31 @@ def test_route_ties_go_to_lower_id(cuda_lib):
     assert_status_ok(tdr)
 
 
+@pytest.mark.parametrize("d", [1024, 4096])
+def test_route_identical_router_columns_tie_exactly(cuda_lib, d):
+    """Experts with identical router columns get bit-identical logits from x, so their
+    order is decided by the id alone."""
+    tdr = cuda_lib
+    T, E, K = 203, 8, 4
+    cfg = mi.MoEConfig("ties", T=T, d=d, E=E, K=K, n=64, dtype="bf16", seed=11)
+    inp = mi.make_inputs(cfg, with_experts=False)
+    w_r = inp.w_r.clone()
+    for e in (1, 3, 6):
+        w_r[:, e] = w_r[:, 5]
+    s = tdr.make_shape(T, d, E, K, 64, 0.0, True, torch.bfloat16)
+    lo = torch.empty(T, E, dtype=torch.float32, device="cuda")
+    ids, w, _ = tdr.route(s, cuda(inp.x), cuda(w_r), logits_out=lo)
+    lg = lo.cpu().numpy()
+    for e in (1, 3, 6):
+        np.testing.assert_array_equal(lg[:, e], lg[:, 5])
+    ids_ref, _ = check_routing(tdr, lo, ids, w, K)
+    got = ids.cpu().numpy()
+    for t in range(T):  # a tied group appears in ascending id order
+        tied = [e for e in got[t] if e in (1, 3, 5, 6)]
+        assert tied == sorted(tied)
+    assert_status_ok(tdr)
+
+
 @pytest.mark.parametrize("T", mi.DISPATCH_COMBINE_T)
 def test_route_given_logits_sweep(cuda_lib, T):
     tdr = cuda_lib
@@ -166,6 +198,10 @@ def _random_ids(rng, T, E, K, skew=0.0):
     (3001, 256, 32, 0.5, 0.0),
     (700, 16, 4, 0.3, 5.0),
     (65536, 64, 6, 0.0, 0.0),
+    # around the one-launch cluster path's bounds (2048 < T*K <= 32768 assignments)
+    (1025, 8, 2, 0.0, 0.0),
+    (4097, 8, 2, 1.0, 2.0),
+    (4097, 8, 8, 0.0, 0.0),
 ])
 def test_permute_matches_oracle(cuda_lib, T, E, K, cf, skew):
     tdr = cuda_lib

@@ -344,7 +344,8 @@ class Profiler:
 
 
 def set_ffn_variant(variant: int) -> None:
-    """0 = automatic, 1 = single-CTA 128 x 256 tiles, 2 = CTA-pair 256 x 256 tiles."""
+    """0 = automatic, 1 = single-CTA 128 x 256 tiles, 2 = CTA-pair 256 x 256 tiles with
+    the gate/up rows gathered in the GEMM, 3 = CTA pairs with the rows copied first."""
     _check(load_library().moe_set_ffn_variant(int(variant)), "moe_set_ffn_variant")
 
 

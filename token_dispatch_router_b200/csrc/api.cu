@@ -26,7 +26,7 @@ moe_status launch_selftest_timeout(uint64_t limit_ns, cudaStream_t st);
 bool route_tc_supported(const moe_shape& s);
 moe_status launch_ffn_tc_mixed(const moe_shape& s, const void* x, const int32_t* offsets,
                                const int32_t* p2a, const void* w_gate, const void* w_up,
-                               const void* w_down, void* a_act, void* y_perm, bool pair_gateup,
+                               const void* w_down, void* a_act, void* y_perm, int gateup_mode,
                                bool pair_down, cudaStream_t st);
 moe_status launch_permute_static(const moe_shape& s, const int32_t* ids, int32_t* counts,
                                  int32_t* offsets, int32_t* a2p, int32_t* p2a, const void* x,
@@ -76,7 +76,8 @@ namespace {
 const char* kKernelNames[K_COUNT] = {
     "route",        "hist",          "scan",           "scatter",     "gather_rows", "gateup_tc",
     "down_tc",      "gateup_simt",   "down_simt",      "combine",     "selftest_timeout",
-    "route_tc",     "permute_small", "gateup_tc2",   "down_tc2"};
+    "route_tc",     "permute_small", "gateup_tc2",   "down_tc2",
+    "permute_cluster"};
 
 struct ProfRec {
   int kid;
@@ -172,17 +173,17 @@ bool layout_of(const moe_shape& s, moe_workspace_layout* L) {
 
 bool aligned16(const void* p) { return ((uintptr_t)p & 15) == 0; }
 
-int g_ffn_variant = 0;  // 0 auto, 1 single-CTA tiles, 2 CTA-pair tiles
+int g_ffn_variant = 0;  // 0 auto, 1 single-CTA tiles, 2 CTA-pair tiles, 3 CTA pairs, A by TMA
 
 // Automatic choice, from measurements on B200: the gate/up GEMM runs single-CTA tiles
 // (its gathered A operand gains nothing from pairing, and 256-row tiles pad twice as many
 // rows); the down GEMM runs on CTA pairs once experts average at least 512 rows, where the
 // pair's deeper pipeline beats the extra padding.
 bool use_pair_down(const moe_shape& s) {
-  if (g_ffn_variant != 0) return g_ffn_variant == 2;
+  if (g_ffn_variant != 0) return g_ffn_variant >= 2;
   return (long long)s.T * s.K >= 512LL * s.E;
 }
-bool use_pair_gateup() { return g_ffn_variant == 2; }
+int gateup_mode() { return g_ffn_variant == 2 ? 1 : g_ffn_variant == 3 ? 2 : 0; }
 
 }  // namespace
 }  // namespace moe
@@ -287,7 +288,7 @@ moe_status moe_grouped_ffn(const moe_shape* s, const void* x, const int32_t* off
     return MOE_ERR_INVALID_ARG;
   if (s->dtype == MOE_BF16)
     return launch_ffn_tc_mixed(*s, x, offsets, perm_to_assign, w_gate, w_up, w_down, a_act, y_perm,
-                               use_pair_gateup(), use_pair_down(*s), (cudaStream_t)stream);
+                               gateup_mode(), use_pair_down(*s), (cudaStream_t)stream);
   return launch_ffn_simt(*s, x, offsets, perm_to_assign, w_gate, w_up, w_down, a_act, y_perm,
                          (cudaStream_t)stream);
 }
@@ -401,7 +402,7 @@ int64_t moe_launch_count(void) {
 }
 
 moe_status moe_set_ffn_variant(int variant) {
-  if (variant < 0 || variant > 2) return MOE_ERR_INVALID_ARG;
+  if (variant < 0 || variant > 3) return MOE_ERR_INVALID_ARG;
   g_ffn_variant = variant;
   return MOE_OK;
 }

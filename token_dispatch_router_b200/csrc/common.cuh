@@ -88,6 +88,7 @@ enum KernelId {
   K_PERMUTE_SMALL,
   K_GATEUP_TC2,
   K_DOWN_TC2,
+  K_PERMUTE_CLUSTER,
   K_COUNT
 };
 

@@ -634,21 +634,36 @@ static moe_status prepare_ffn(const moe_shape& s, const void* x, const int32_t* 
   return MOE_OK;
 }
 
-moe_status launch_ffn_tc2_gemm(bool gateup, const CUtensorMap& a, const CUtensorMap& b0,
+moe_status launch_ffn_tc2_gemm(int mode, const CUtensorMap& a, const CUtensorMap& b0,
                                const CUtensorMap& b1, const GemmArgs& args, cudaStream_t st);
+moe_status launch_gather_rows(const moe_shape& s, const void* x, const int32_t* p2a,
+                              const int32_t* offsets, void* x_perm, cudaStream_t st);
 
+// gateup_mode 0: single-CTA tiles, A rows gathered in the kernel; 1: CTA pairs, A rows
+// gathered in the kernel; 2: the rows are first copied expert-major into y_perm (which the
+// down GEMM overwrites only later), then CTA pairs load A from there by TMA.
 moe_status launch_ffn_tc_mixed(const moe_shape& s, const void* x, const int32_t* offsets,
                                const int32_t* p2a, const void* w_gate, const void* w_up,
-                               const void* w_down, void* a_act, void* y_perm, bool pair_gateup,
+                               const void* w_down, void* a_act, void* y_perm, int gateup_mode,
                                bool pair_down, cudaStream_t st) {
   if ((long long)s.T * s.K == 0) return MOE_OK;
   FfnMaps f;
   moe_status r = prepare_ffn(s, x, offsets, p2a, w_gate, w_up, w_down, a_act, y_perm, f);
   if (r != MOE_OK) return r;
-  r = pair_gateup ? launch_ffn_tc2_gemm(true, f.mg, f.mg, f.mu, f.gate_up, st)
-                  : run_gemm<true>(f.mg, f.mg, f.mu, f.gate_up, st, K_GATEUP_TC);
+  if (gateup_mode == 2) {
+    if ((r = launch_gather_rows(s, x, p2a, offsets, y_perm, st)) != MOE_OK) return r;
+    CUtensorMap mx;
+    const uint64_t dims[2] = {(uint64_t)s.d, (uint64_t)s.T * s.K}, str[1] = {(uint64_t)s.d * 2};
+    const uint32_t box[2] = {64, 128};
+    if (!make_map(&mx, y_perm, 2, dims, str, box)) return MOE_ERR_CUDA;
+    r = launch_ffn_tc2_gemm(2, mx, f.mg, f.mu, f.gate_up, st);
+  } else if (gateup_mode == 1) {
+    r = launch_ffn_tc2_gemm(1, f.mg, f.mg, f.mu, f.gate_up, st);
+  } else {
+    r = run_gemm<true>(f.mg, f.mg, f.mu, f.gate_up, st, K_GATEUP_TC);
+  }
   if (r != MOE_OK) return r;
-  return pair_down ? launch_ffn_tc2_gemm(false, f.ma, f.md, f.md, f.down, st)
+  return pair_down ? launch_ffn_tc2_gemm(0, f.ma, f.md, f.md, f.down, st)
                    : run_gemm<false>(f.ma, f.md, f.md, f.down, st, K_DOWN_TC);
 }
 

@@ -67,8 +67,11 @@ __device__ __forceinline__ Tile2 decode2(int w, const int* s_off, const int* s_c
   return t;
 }
 
-template <bool GATEUP>
-__global__ void __launch_bounds__(GATEUP ? THREADS_GATEUP : THREADS_DOWN, 1)
+// MODE 0: down GEMM (A = the activations, by TMA); 1: gate/up GEMM with the A rows
+// gathered from x by cp.async; 2: gate/up GEMM with A = rows already gathered into an
+// expert-major buffer, by TMA (no gather warps, no relay).
+template <int MODE>
+__global__ void __launch_bounds__(MODE == 1 ? THREADS_GATEUP : THREADS_DOWN, 1)
     grouped_gemm_tc2(const __grid_constant__ CUtensorMap tmA,
                      const __grid_constant__ CUtensorMap tmB0,
                      const __grid_constant__ CUtensorMap tmB1, const GemmArgs g) {
@@ -88,13 +91,15 @@ __global__ void __launch_bounds__(GATEUP ? THREADS_GATEUP : THREADS_DOWN, 1)
   int* s_cum = s_off + MAXE + 1;
   int* s_mt = s_cum + MAXE + 1;
 
-  constexpr int NTHREADS = GATEUP ? THREADS_GATEUP : THREADS_DOWN;
+  constexpr bool GATEUP = MODE != 0;
+  constexpr bool GATHER = MODE == 1;
+  constexpr int NTHREADS = GATHER ? THREADS_GATEUP : THREADS_DOWN;
   // leader's full[s]: the leader's expect_tx arrival for the TMA bytes of both CTAs (+ the
   // leader's gather threads + the peer's relay). The peer's loads complete on it without
   // an arrival of their own: a transaction count may run ahead of its expect_tx, and the
   // phase cannot complete before the leader's arrival anyway.
-  constexpr uint32_t FULL_COUNT = GATEUP ? 1 + GATHER_THREADS + 1 : 1;
-  constexpr uint32_t TMA_BYTES = GATEUP ? B_HALF : STAGE_BYTES;  // per CTA and stage
+  constexpr uint32_t FULL_COUNT = GATHER ? 1 + GATHER_THREADS + 1 : 1;
+  constexpr uint32_t TMA_BYTES = GATHER ? B_HALF : STAGE_BYTES;  // per CTA and stage
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const uint32_t rank = cluster_rank();
@@ -176,7 +181,7 @@ __global__ void __launch_bounds__(GATEUP ? THREADS_GATEUP : THREADS_DOWN, 1)
         __syncwarp();
         const uint32_t a_dst = saddr(ring + stage * STAGE_BYTES);
         const uint32_t b_dst = a_dst + A_BYTES;
-        if (!GATEUP && lane == 0) tma_load_2d_pair(a_dst, &tmA, kb * BK, t.m0, fb);
+        if (!GATHER && lane == 0) tma_load_2d_pair(a_dst, &tmA, kb * BK, t.m0, fb);
         if (lane < 2) {
           if (GATEUP)
             tma_load_3d_pair(b_dst + lane * B_CHUNK, leader ? &tmB0 : &tmB1, t.n0 + lane * 64,
@@ -225,7 +230,7 @@ __global__ void __launch_bounds__(GATEUP ? THREADS_GATEUP : THREADS_DOWN, 1)
             ok = false;
             break;
           }
-          if (GATEUP) fence_proxy_async_smem();  // this CTA's cp.async rows -> MMA reads
+          if (GATHER) fence_proxy_async_smem();  // this CTA's cp.async rows -> MMA reads
           tc_fence_after();
           const uint32_t a_addr = saddr(ring + stage * STAGE_BYTES);
           const uint32_t b_addr = a_addr + A_BYTES;
@@ -251,7 +256,7 @@ __global__ void __launch_bounds__(GATEUP ? THREADS_GATEUP : THREADS_DOWN, 1)
       const uint64_t t0 = globaltimer_ns();
       while (!mbar_try(saddr(done), 0) && globaltimer_ns() - t0 < limit) {
       }
-    } else if (GATEUP && !leader && lane == 0) {
+    } else if (GATHER && !leader && lane == 0) {
       // ---------------------------------------------------------- gather relay (peer)
       int stage = 0;
       uint32_t phase = 0;
@@ -272,7 +277,7 @@ __global__ void __launch_bounds__(GATEUP ? THREADS_GATEUP : THREADS_DOWN, 1)
         if (!ok) break;
       }
     }
-  } else if (GATEUP && warp >= GATHER_WARP0) {
+  } else if (GATHER && warp >= GATHER_WARP0) {
     // ------------------------------------------------------------ A gather (both CTAs)
     const int gw = warp - GATHER_WARP0;
     const int c = lane & 7;
@@ -405,17 +410,17 @@ __global__ void __launch_bounds__(GATEUP ? THREADS_GATEUP : THREADS_DOWN, 1)
   }
 }
 
-template <bool GATEUP>
+template <int MODE>
 moe_status run_gemm2(const CUtensorMap& a, const CUtensorMap& b0, const CUtensorMap& b1,
                      const GemmArgs& args, cudaStream_t st, int kid) {
-  auto kern = grouped_gemm_tc2<GATEUP>;
+  auto kern = grouped_gemm_tc2<MODE>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES) !=
       cudaSuccess)
     return MOE_ERR_CUDA;
   const int pairs = sm_count() / 2;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((unsigned)(2 * (pairs > 0 ? pairs : 1)));
-  cfg.blockDim = dim3(GATEUP ? THREADS_GATEUP : THREADS_DOWN);
+  cfg.blockDim = dim3(MODE == 1 ? THREADS_GATEUP : THREADS_DOWN);
   cfg.dynamicSmemBytes = (size_t)SMEM_BYTES;
   cfg.stream = st;
   cudaLaunchAttribute attr[1];
@@ -432,10 +437,11 @@ moe_status run_gemm2(const CUtensorMap& a, const CUtensorMap& b0, const CUtensor
 
 }  // namespace
 
-moe_status launch_ffn_tc2_gemm(bool gateup, const CUtensorMap& a, const CUtensorMap& b0,
+moe_status launch_ffn_tc2_gemm(int mode, const CUtensorMap& a, const CUtensorMap& b0,
                                const CUtensorMap& b1, const GemmArgs& args, cudaStream_t st) {
-  return gateup ? run_gemm2<true>(a, b0, b1, args, st, K_GATEUP_TC2)
-                : run_gemm2<false>(a, b0, b1, args, st, K_DOWN_TC2);
+  if (mode == 1) return run_gemm2<1>(a, b0, b1, args, st, K_GATEUP_TC2);
+  if (mode == 2) return run_gemm2<2>(a, b0, b1, args, st, K_GATEUP_TC2);
+  return run_gemm2<0>(a, b0, b1, args, st, K_DOWN_TC2);
 }
 
 }  // namespace moe

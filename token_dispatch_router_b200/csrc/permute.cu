@@ -25,7 +25,7 @@
 // Inside an expert the slots follow ascending flat index a = t*K + k, i.e. token order.
 #include <mutex>
 
-#include "common.cuh"
+#include "tc_ptx.cuh"
 
 namespace moe {
 
@@ -351,6 +351,147 @@ __global__ void __launch_bounds__(kSmallWarps * 32) permute_small_kernel(
   }
 }
 
+// Medium problems (kSmallMax < T*K <= kClusterMax): histogram, scan and scatter in one
+// launch of a cluster of C <= 8 CTAs of 32 warps, CTA c owning the contiguous chunk
+// [c * 1024 * ITERS, (c + 1) * 1024 * ITERS) and each warp a slice of ITERS x 32 ids inside
+// it. Same algorithm and result as the three kernels; the ids stay in registers between the
+// counting and the placing walk, and the chunk counts are exchanged through distributed
+// shared memory instead of global memory: after one cluster barrier thread e of every CTA
+// reads the C counts of expert e (its rank base = the counts of the earlier CTAs, the
+// expert's total = all of them), and a second barrier ends all remote reads before any CTA
+// can exit.
+constexpr int kClusterWarps = 32;
+constexpr int kClusterMaxCtas = 8;
+constexpr int kClusterMaxIters = 4;  // beyond, the three-kernel path is faster (measured)
+constexpr long long kClusterMax = (long long)kClusterMaxCtas * kClusterWarps * 32 * kClusterMaxIters;
+
+template <int ITERS>
+__global__ void __launch_bounds__(kClusterWarps * 32) permute_cluster_kernel(
+    const int32_t* __restrict__ ids, long long A, int E, long long cap, int C,
+    int32_t* __restrict__ counts, int32_t* __restrict__ offsets,
+    int32_t* __restrict__ assign_to_perm, int32_t* __restrict__ perm_to_assign, unsigned* status) {
+  __shared__ int rows[kClusterWarps][kMaxE];
+  __shared__ int ctot[kMaxE];   // this CTA's count per expert (read by every CTA)
+  __shared__ int cbase[kMaxE];  // counts of the earlier CTAs
+  __shared__ int offs[kMaxE];
+  __shared__ int wsum[kMaxE / 32];
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const uint32_t rank = ptx::cluster_rank();
+  const long long s0 = ((long long)rank * kClusterWarps + warp) * (32LL * ITERS);
+  for (int i = tid; i < kClusterWarps * kMaxE; i += blockDim.x) (&rows[0][0])[i] = 0;
+  __syncthreads();
+  int v[ITERS];
+#pragma unroll
+  for (int it = 0; it < ITERS; ++it) v[it] = raw_id(ids, s0 + it * 32 + lane, A);
+#pragma unroll
+  for (int it = 0; it < ITERS; ++it) v[it] = checked_id(v[it], s0 + it * 32 + lane < A, E, status);
+  int* row = rows[warp];
+#pragma unroll
+  for (int it = 0; it < ITERS; ++it) {
+    const unsigned m = __match_any_sync(0xffffffffu, v[it]);
+    if (v[it] >= 0 && lane == __ffs(m) - 1) row[v[it]] += __popc(m);
+    __syncwarp();
+  }
+  __syncthreads();
+  if (tid < E) {  // per-warp exclusive bases inside the CTA, and the CTA's total
+    int run = 0;
+    for (int w = 0; w < kClusterWarps; ++w) {
+      const int c = rows[w][tid];
+      rows[w][tid] = run;
+      run += c;
+    }
+    ctot[tid] = run;
+  }
+  ptx::cluster_sync();  // every CTA's totals are complete
+  int total = 0;
+  if (tid < E) {
+    int cv[kClusterMaxCtas];
+    const uint32_t mine = ptx::saddr(&ctot[tid]);
+#pragma unroll
+    for (int q = 0; q < kClusterMaxCtas; ++q)
+      cv[q] = q < C ? ptx::ld_dsmem_s32(ptx::map_rank(mine, (uint32_t)q)) : 0;
+    int before = 0;
+#pragma unroll
+    for (int q = 0; q < kClusterMaxCtas; ++q) {
+      if (q < (int)rank) before += cv[q];
+      total += cv[q];
+    }
+    cbase[tid] = before;
+    if (rank == 0) counts[tid] = total;
+  }
+  ptx::cluster_sync();  // no CTA reads another's shared memory after this point
+  // exclusive scan of kept = min(total, cap) over the experts (threads 0..255)
+  int kept = 0, incl = 0;
+  if (tid < kMaxE) {
+    kept = (tid < E) ? (int)((cap >= 0 && total > cap) ? cap : total) : 0;
+    incl = kept;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, incl, off);
+      if (lane >= off) incl += y;
+    }
+    if (lane == 31) wsum[warp] = incl;
+  }
+  __syncthreads();
+  if (tid < kMaxE) {
+    int pre = 0;
+    for (int w = 0; w < warp; ++w) pre += wsum[w];
+    incl += pre;
+    if (tid < E) {
+      offs[tid] = incl - kept;
+      if (rank == 0) {
+        offsets[tid] = incl - kept;
+        if (tid == E - 1) offsets[E] = incl;
+      }
+    }
+  }
+  __syncthreads();
+  const unsigned lt = lanemask_lt();
+#pragma unroll
+  for (int it = 0; it < ITERS; ++it) {
+    const long long a = s0 + it * 32 + lane;
+    const int id = v[it];
+    const unsigned m = __match_any_sync(0xffffffffu, id);
+    int r = 0;
+    if (id >= 0) r = cbase[id] + row[id] + __popc(m & lt);
+    __syncwarp();
+    if (id >= 0 && lane == __ffs(m) - 1) row[id] += __popc(m);
+    __syncwarp();
+    if (id >= 0) {
+      int p = -1;
+      if (cap < 0 || r < cap) {
+        p = offs[id] + r;
+        perm_to_assign[p] = (int32_t)a;
+      }
+      assign_to_perm[a] = p;
+    } else if (a < A) {
+      assign_to_perm[a] = -1;
+    }
+  }
+}
+
+template <int ITERS>
+moe_status launch_cluster_permute(const int32_t* ids, long long A, int E, long long cap, int C,
+                                  int32_t* counts, int32_t* offsets, int32_t* a2p, int32_t* p2a,
+                                  unsigned* status, cudaStream_t st) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)C);
+  cfg.blockDim = dim3(kClusterWarps * 32);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = (unsigned)C;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  launch_begin(K_PERMUTE_CLUSTER, st);
+  cudaLaunchKernelEx(&cfg, permute_cluster_kernel<ITERS>, ids, A, E, cap, C, counts, offsets, a2p,
+                     p2a, status);
+  return launch_end(K_PERMUTE_CLUSTER, st);
+}
+
 // x_perm[p] = x[perm_to_assign[p] / K] for p < offsets[E]; 16-byte vectors. One warp moves
 // a 2 KB segment (128 vectors) of one row: the row's source token is loaded once per lane
 // and each lane keeps four independent 16-byte loads in flight.
@@ -389,6 +530,9 @@ __global__ void __launch_bounds__(256) gather_rows_kernel(const uint4* __restric
 
 }  // namespace
 
+moe_status launch_gather_rows(const moe_shape& s, const void* x, const int32_t* p2a,
+                              const int32_t* offsets, void* x_perm, cudaStream_t st);
+
 size_t permute_scratch_bytes(const moe_shape& s) {
   const long long A = (long long)s.T * s.K;
   const long long nchunks = (A + kChunk - 1) / kChunk;
@@ -413,6 +557,18 @@ moe_status launch_permute(const moe_shape& s, const int32_t* ids, int32_t* count
     permute_small_kernel<<<1, kSmallWarps * 32, 0, st>>>(ids, A, s.E, cap, counts, offsets, a2p,
                                                          p2a, status);
     if ((r = launch_end(K_PERMUTE_SMALL, st)) != MOE_OK) return r;
+  } else if (A > 0 && A <= kClusterMax) {
+    // fewest ids per warp that still fit the chunks into one cluster of <= 8 CTAs
+    int iters = 1;
+    while ((long long)kClusterMaxCtas * kClusterWarps * 32 * iters < A) iters <<= 1;
+    const int per_cta = kClusterWarps * 32 * iters;
+    const int C = (int)((A + per_cta - 1) / per_cta);
+    switch (iters) {
+      case 1: r = launch_cluster_permute<1>(ids, A, s.E, cap, C, counts, offsets, a2p, p2a, status, st); break;
+      case 2: r = launch_cluster_permute<2>(ids, A, s.E, cap, C, counts, offsets, a2p, p2a, status, st); break;
+      default: r = launch_cluster_permute<4>(ids, A, s.E, cap, C, counts, offsets, a2p, p2a, status, st); break;
+    }
+    if (r != MOE_OK) return r;
   } else if (nchunks > 0) {
     launch_begin(K_HIST, st);
     hist_kernel<<<nchunks, kWarps * 32, 0, st>>>(ids, A, s.E, chunk_counts, status);
@@ -432,19 +588,25 @@ moe_status launch_permute(const moe_shape& s, const int32_t* ids, int32_t* count
                                                     status);
     if ((r = launch_end(K_SCATTER, st)) != MOE_OK) return r;
   }
-  if (x != nullptr && x_perm != nullptr && A > 0) {
-    const int elem = (s.dtype == MOE_BF16) ? 2 : 4;
-    const int vec_per_row = s.d * elem / 16;
-    const long long units = A * ((vec_per_row + 127) / 128);  // one warp each
-    long long blocks = (units + 7) / 8;
-    const long long cap_blocks = (long long)sm_count() * 8;
-    if (blocks > cap_blocks) blocks = cap_blocks;
-    launch_begin(K_GATHER, st);
-    gather_rows_kernel<<<(int)blocks, 256, 0, st>>>((const uint4*)x, p2a, offsets + s.E, s.K, s.T,
-                                                    vec_per_row, (uint4*)x_perm, status);
-    if ((r = launch_end(K_GATHER, st)) != MOE_OK) return r;
-  }
+  if (x != nullptr && x_perm != nullptr && A > 0)
+    return launch_gather_rows(s, x, p2a, offsets, x_perm, st);
   return MOE_OK;
+}
+
+moe_status launch_gather_rows(const moe_shape& s, const void* x, const int32_t* p2a,
+                              const int32_t* offsets, void* x_perm, cudaStream_t st) {
+  const long long A = (long long)s.T * s.K;
+  if (A == 0) return MOE_OK;
+  const int elem = (s.dtype == MOE_BF16) ? 2 : 4;
+  const int vec_per_row = s.d * elem / 16;
+  const long long units = A * ((vec_per_row + 127) / 128);  // one warp each
+  long long blocks = (units + 7) / 8;
+  const long long cap_blocks = (long long)sm_count() * 8;
+  if (blocks > cap_blocks) blocks = cap_blocks;
+  launch_begin(K_GATHER, st);
+  gather_rows_kernel<<<(int)blocks, 256, 0, st>>>((const uint4*)x, p2a, offsets + s.E, s.K, s.T,
+                                                  vec_per_row, (uint4*)x_perm, device_status_ptr());
+  return launch_end(K_GATHER, st);
 }
 
 // ------------------------------------------------------------------ no-allocation variant

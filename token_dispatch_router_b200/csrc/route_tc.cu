@@ -127,17 +127,18 @@ __device__ __forceinline__ float ld_dsmem(uint32_t remote_addr) {
   return v;
 }
 
-// Top-8 list, descending by (value, then lower id); empty slots have id -1. Ids arrive in
-// ascending order, so an existing entry with an equal value stays above the new one (ties
-// go to the lower id, +0 == -0). The top-K for K <= 8 is the first K slots. Every index is
-// a compile-time constant, so the list lives in registers.
-__device__ __forceinline__ void top8_insert(float (&bv)[KMAX], int (&be)[KMAX], float v, int e) {
-  if (be[KMAX - 1] >= 0 && !(v > bv[KMAX - 1])) return;  // does not enter
-  bool above[KMAX];  // the entry in slot j stays above the new one
+// Top-KM list (KM = 2, 4 or 8 >= K), descending by (value, then lower id); empty slots
+// have id -1. Ids arrive in ascending order, so an existing entry with an equal value stays
+// above the new one (ties go to the lower id, +0 == -0). The top-K is the first K slots.
+// Every index is a compile-time constant, so the list lives in registers.
+template <int KM>
+__device__ __forceinline__ void top_insert(float (&bv)[KM], int (&be)[KM], float v, int e) {
+  if (be[KM - 1] >= 0 && !(v > bv[KM - 1])) return;  // does not enter
+  bool above[KM];  // the entry in slot j stays above the new one
 #pragma unroll
-  for (int j = 0; j < KMAX; ++j) above[j] = be[j] >= 0 && !(v > bv[j]);
+  for (int j = 0; j < KM; ++j) above[j] = be[j] >= 0 && !(v > bv[j]);
 #pragma unroll
-  for (int j = KMAX - 1; j >= 1; --j) {
+  for (int j = KM - 1; j >= 1; --j) {
     if (!above[j]) {
       if (above[j - 1]) {
         bv[j] = v;
@@ -154,7 +155,7 @@ __device__ __forceinline__ void top8_insert(float (&bv)[KMAX], int (&be)[KMAX], 
   }
 }
 
-template <int N>  // MMA N = E rounded up to 16
+template <int N, int KM>  // MMA N = E rounded up to 16; KM >= K, a power of two <= 8
 __global__ void __launch_bounds__(R_THREADS) route_tc_kernel(const __grid_constant__ CUtensorMap tmX,
                                                              const __grid_constant__ CUtensorMap tmW,
                                                              const RouteArgs g) {
@@ -286,10 +287,10 @@ __global__ void __launch_bounds__(R_THREADS) route_tc_kernel(const __grid_consta
     float* st_l = (float*)ring;                         // [128][E + 1]
     int32_t* st_i = (int32_t*)(st_l + RBM * (E + 1));   // [128][K]
     float* st_w = (float*)(st_i + RBM * K);             // [128][K]
-    float bv[KMAX];
-    int be[KMAX];
+    float bv[KM];
+    int be[KM];
 #pragma unroll
-    for (int k = 0; k < KMAX; ++k) {
+    for (int k = 0; k < KM; ++k) {
       bv[k] = -INFINITY;
       be[k] = -1;
     }
@@ -302,13 +303,22 @@ __global__ void __launch_bounds__(R_THREADS) route_tc_kernel(const __grid_consta
       float lv[16];
 #pragma unroll
       for (int j = 0; j < 16; ++j) lv[j] = have ? __uint_as_float(v[j]) : 0.f;
-      for (int q = 1; q < S; ++q) {  // partials of the other ranks, added in rank order
-        const uint32_t rbase = map_rank(saddr(&part[c0 * RBM + r]), (uint32_t)q);
-        float pv[16];
+      // partials of the other ranks, added in rank order; up to four ranks' loads in flight
+      for (int q0 = 1; q0 < S; q0 += 4) {
+        float pv[4][16];
 #pragma unroll
-        for (int j = 0; j < 16; ++j) pv[j] = ld_dsmem(rbase + (uint32_t)(j * RBM * 4));
+        for (int qq = 0; qq < 4; ++qq) {
+          if (q0 + qq < S) {
+            const uint32_t rbase = map_rank(saddr(&part[c0 * RBM + r]), (uint32_t)(q0 + qq));
 #pragma unroll
-        for (int j = 0; j < 16; ++j) lv[j] += pv[j];
+            for (int j = 0; j < 16; ++j) pv[qq][j] = ld_dsmem(rbase + (uint32_t)(j * RBM * 4));
+          }
+        }
+#pragma unroll
+        for (int qq = 0; qq < 4; ++qq)
+          if (q0 + qq < S)
+#pragma unroll
+            for (int j = 0; j < 16; ++j) lv[j] += pv[qq][j];
       }
 #pragma unroll
       for (int j = 0; j < 16; ++j) {
@@ -318,7 +328,7 @@ __global__ void __launch_bounds__(R_THREADS) route_tc_kernel(const __grid_consta
           if (g.bias != nullptr) l += g.bias[e];
           if (t < g.T) {
             st_l[r * (E + 1) + e] = l;
-            top8_insert(bv, be, l, e);
+            top_insert<KM>(bv, be, l, e);
             if (!g.renorm) {
               if (l > m) {
                 ssum = ssum * expf(m - l) + 1.f;
@@ -335,11 +345,11 @@ __global__ void __launch_bounds__(R_THREADS) route_tc_kernel(const __grid_consta
       const float top = bv[0];
       float den = 0.f;
 #pragma unroll
-      for (int k = 0; k < KMAX; ++k)
+      for (int k = 0; k < KM; ++k)
         if (k < K) den += expf(bv[k] - top);
       if (!g.renorm) den = ssum * expf(m - top);
 #pragma unroll
-      for (int k = 0; k < KMAX; ++k) {
+      for (int k = 0; k < KM; ++k) {
         if (k < K) {
           st_i[r * K + k] = be[k];
           st_w[r * K + k] = expf(bv[k] - top) / den;
@@ -392,13 +402,13 @@ bool make_map_2d(CUtensorMap* m, const void* ptr, uint64_t inner, uint64_t outer
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int N>
-moe_status launch_n(const CUtensorMap& mx, const CUtensorMap& mw, const RouteArgs& a, int tiles,
+template <int N, int KM>
+moe_status launch_nk(const CUtensorMap& mx, const CUtensorMap& mw, const RouteArgs& a, int tiles,
                     cudaStream_t st) {
   constexpr int NCH = (N + 63) / 64;
   constexpr int STAGE = RA_BYTES + NCH * RB_CHUNK;
   const int smem = route_stages(N) * STAGE + 1024 + 256;
-  auto kern = route_tc_kernel<N>;
+  auto kern = route_tc_kernel<N, KM>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
     return MOE_ERR_CUDA;
   cudaLaunchConfig_t cfg = {};
@@ -416,6 +426,16 @@ moe_status launch_n(const CUtensorMap& mx, const CUtensorMap& mw, const RouteArg
   launch_begin(K_ROUTE_TC, st);
   cudaLaunchKernelEx(&cfg, kern, mx, mw, a);
   return launch_end(K_ROUTE_TC, st);
+}
+
+template <int KM>
+moe_status launch_n(int N, const CUtensorMap& mx, const CUtensorMap& mw, const RouteArgs& a,
+                    int tiles, cudaStream_t st) {
+  if (N <= 16) return launch_nk<16, KM>(mx, mw, a, tiles, st);
+  if (N <= 32) return launch_nk<32, KM>(mx, mw, a, tiles, st);
+  if (N <= 64) return launch_nk<64, KM>(mx, mw, a, tiles, st);
+  if (N <= 128) return launch_nk<128, KM>(mx, mw, a, tiles, st);
+  return launch_nk<256, KM>(mx, mw, a, tiles, st);
 }
 
 }  // namespace
@@ -459,11 +479,9 @@ moe_status launch_route_tc(const moe_shape& s, const void* x, const void* w_r, c
   a.status = device_status_ptr();
   a.limit_ns = kWaitLimitNs;
   // instantiations cover N up to the next of 16/32/64/128/256; columns past E read zeros
-  if (N <= 16) return launch_n<16>(mx, mw, a, tiles, st);
-  if (N <= 32) return launch_n<32>(mx, mw, a, tiles, st);
-  if (N <= 64) return launch_n<64>(mx, mw, a, tiles, st);
-  if (N <= 128) return launch_n<128>(mx, mw, a, tiles, st);
-  return launch_n<256>(mx, mw, a, tiles, st);
+  if (s.K <= 2) return launch_n<2>(N, mx, mw, a, tiles, st);
+  if (s.K <= 4) return launch_n<4>(N, mx, mw, a, tiles, st);
+  return launch_n<8>(N, mx, mw, a, tiles, st);
 }
 
 }  // namespace moe
