@@ -22,6 +22,8 @@ __global__ void __launch_bounds__(256) combine_kernel(const uint4* __restrict__ 
                                                       const float* __restrict__ topk_w, int T,
                                                       int K, int vec_per_row, long long n_rows,
                                                       uint4* __restrict__ out, unsigned* status) {
+  pdl_wait();  // the previous kernel in the stream has completed
+  pdl_trigger();
   constexpr int V = Vec16<Tv>::N;
   const int segs = (vec_per_row + 127) / 128;
   const long long units = (long long)T * segs;
@@ -91,13 +93,13 @@ moe_status launch_combine(const moe_shape& s, const void* y_perm, const int32_t*
   const long long n_rows = (long long)s.T * s.K;
   launch_begin(K_COMBINE, st);
   if (s.dtype == MOE_BF16)
-    combine_kernel<bf16><<<(int)blocks, 256, 0, st>>>((const uint4*)y_perm, a2p, topk_w, s.T, s.K,
-                                                      vec_per_row, n_rows, (uint4*)out,
-                                                      device_status_ptr());
+    launch_kernel(combine_kernel<bf16>, dim3((unsigned)blocks), dim3(256), 0, st, 1,
+                  (const uint4*)y_perm, a2p, topk_w, s.T, s.K, vec_per_row, n_rows, (uint4*)out,
+                  device_status_ptr());
   else
-    combine_kernel<float><<<(int)blocks, 256, 0, st>>>((const uint4*)y_perm, a2p, topk_w, s.T, s.K,
-                                                       vec_per_row, n_rows, (uint4*)out,
-                                                       device_status_ptr());
+    launch_kernel(combine_kernel<float>, dim3((unsigned)blocks), dim3(256), 0, st, 1,
+                  (const uint4*)y_perm, a2p, topk_w, s.T, s.K, vec_per_row, n_rows, (uint4*)out,
+                  device_status_ptr());
   return launch_end(K_COMBINE, st);
 }
 

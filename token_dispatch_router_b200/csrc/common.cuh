@@ -6,6 +6,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <utility>
+
 #include "moe.h"
 
 namespace moe {
@@ -64,6 +66,17 @@ __device__ __forceinline__ uint32_t lanemask_lt() {
   return m;
 }
 
+// Programmatic dependent launch. Every kernel of the library is launched with programmatic
+// stream serialisation, so the GPU may schedule it while the kernel before it in the stream
+// is still running. pdl_wait() returns once that kernel has completed and its writes are
+// visible: every kernel calls it before its first global-memory access (read or write).
+// pdl_trigger() allows the next kernel to be scheduled once every CTA of this one has called
+// it (or exited); it does not make this kernel's writes visible early.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 __device__ __forceinline__ uint64_t globaltimer_ns() {
   uint64_t t;
   asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
@@ -98,6 +111,33 @@ void launch_begin(int kernel_id, cudaStream_t s);
 moe_status launch_end(int kernel_id, cudaStream_t s);  // checks cudaGetLastError
 
 constexpr uint64_t kWaitLimitNs = 2000000000ull;  // bounded waits: 2 s
+
+// Launches `kern` on `st` with programmatic stream serialisation (see pdl_wait) and, when
+// cluster_x > 1, thread-block clusters of cluster_x CTAs along x.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_kernel(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                          cudaStream_t st, unsigned cluster_x, Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[2];
+  unsigned n = 0;
+  attr[n].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[n].val.programmaticStreamSerializationAllowed = 1;
+  ++n;
+  if (cluster_x > 1) {
+    attr[n].id = cudaLaunchAttributeClusterDimension;
+    attr[n].val.clusterDim.x = cluster_x;
+    attr[n].val.clusterDim.y = 1;
+    attr[n].val.clusterDim.z = 1;
+    ++n;
+  }
+  cfg.attrs = attr;
+  cfg.numAttrs = n;
+  return cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
+}
 
 // Size of the static scratch behind moe_permute_static (see moe.h).
 constexpr size_t kPermuteStaticScratchBytes = MOE_PERMUTE_STATIC_SCRATCH_BYTES;

@@ -52,6 +52,8 @@ __global__ void __launch_bounds__(kThreads) ffn_simt_kernel(
     const float* __restrict__ a_src, const int32_t* __restrict__ offsets,
     const int32_t* __restrict__ p2a, const float* __restrict__ w0, const float* __restrict__ w1,
     float* __restrict__ out, int E, int K, int T, int kdim, int ncols, unsigned* status) {
+  pdl_wait();  // the previous kernel in the stream has completed
+  pdl_trigger();
   __shared__ int s_off[kMaxE + 1], s_cum[kMaxE + 1];
   __shared__ long long s_src[SBM];
   __shared__ float As[SBK][SBM + 4];
@@ -153,15 +155,15 @@ moe_status launch_ffn_simt(const moe_shape& s, const void* x, const int32_t* off
   moe_status r;
   dim3 g1((s.n + SBN - 1) / SBN, (unsigned)mtiles);
   launch_begin(K_GATEUP_SIMT, st);
-  ffn_simt_kernel<true><<<g1, kThreads, 0, st>>>((const float*)x, offsets, p2a,
-                                                 (const float*)w_gate, (const float*)w_up,
-                                                 (float*)a_act, s.E, s.K, s.T, s.d, s.n, status);
+  launch_kernel(ffn_simt_kernel<true>, g1, dim3(kThreads), 0, st, 1, (const float*)x, offsets, p2a,
+                (const float*)w_gate, (const float*)w_up, (float*)a_act, s.E, s.K, s.T, s.d, s.n,
+                status);
   if ((r = launch_end(K_GATEUP_SIMT, st)) != MOE_OK) return r;
   dim3 g2((s.d + SBN - 1) / SBN, (unsigned)mtiles);
   launch_begin(K_DOWN_SIMT, st);
-  ffn_simt_kernel<false><<<g2, kThreads, 0, st>>>((const float*)a_act, offsets, p2a,
-                                                  (const float*)w_down, nullptr, (float*)y_perm,
-                                                  s.E, s.K, s.T, s.n, s.d, status);
+  launch_kernel(ffn_simt_kernel<false>, g2, dim3(kThreads), 0, st, 1, (const float*)a_act, offsets,
+                p2a, (const float*)w_down, (const float*)nullptr, (float*)y_perm, s.E, s.K, s.T,
+                s.n, s.d, status);
   return launch_end(K_DOWN_SIMT, st);
 }
 

@@ -244,6 +244,8 @@ __global__ void __launch_bounds__(GATEUP ? THREADS_GATEUP : THREADS_DOWN, 1)
                  : "memory");
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
   }
+  pdl_wait();  // the previous kernel in the stream has completed
+  pdl_trigger();
   for (int i = tid; i <= E; i += NTHREADS) s_off[i] = g.offsets[i];
   __syncthreads();
   if (warp == 0) {  // tile table: s_mt[e] = ceil(kept_e / BM); s_cum = n_tiles * prefix
@@ -549,7 +551,8 @@ moe_status run_gemm(const CUtensorMap& a, const CUtensorMap& b0, const CUtensorM
       cudaSuccess)
     return MOE_ERR_CUDA;
   launch_begin(kid, st);
-  kern<<<sm_count(), GATEUP ? THREADS_GATEUP : THREADS_DOWN, SMEM_BYTES, st>>>(a, b0, b1, args);
+  launch_kernel(kern, dim3((unsigned)sm_count()), dim3(GATEUP ? THREADS_GATEUP : THREADS_DOWN),
+                SMEM_BYTES, st, 1, a, b0, b1, args);
   return launch_end(kid, st);
 }
 

@@ -122,6 +122,8 @@ __global__ void __launch_bounds__(MODE == 1 ? THREADS_GATEUP : THREADS_DOWN, 1)
     mbar_init_fence();
   }
   if (warp == 1) tmem_alloc<2>(saddr(tmem_slot), TMEM_COLS);
+  pdl_wait();  // the previous kernel in the stream has completed
+  pdl_trigger();
   for (int i = tid; i <= E; i += NTHREADS) s_off[i] = g.offsets[i];
   __syncthreads();
   if (warp == 0) {  // tile table: s_mt[e] = ceil(kept_e / 256); s_cum = n_tiles * prefix
@@ -418,20 +420,10 @@ moe_status run_gemm2(const CUtensorMap& a, const CUtensorMap& b0, const CUtensor
       cudaSuccess)
     return MOE_ERR_CUDA;
   const int pairs = sm_count() / 2;
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3((unsigned)(2 * (pairs > 0 ? pairs : 1)));
-  cfg.blockDim = dim3(MODE == 1 ? THREADS_GATEUP : THREADS_DOWN);
-  cfg.dynamicSmemBytes = (size_t)SMEM_BYTES;
-  cfg.stream = st;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = 2;
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
   launch_begin(kid, st);
-  cudaLaunchKernelEx(&cfg, kern, a, b0, b1, args);
+  launch_kernel(kern, dim3((unsigned)(2 * (pairs > 0 ? pairs : 1))),
+                dim3(MODE == 1 ? THREADS_GATEUP : THREADS_DOWN), (size_t)SMEM_BYTES, st, 2, a, b0,
+                b1, args);
   return launch_end(kid, st);
 }
 

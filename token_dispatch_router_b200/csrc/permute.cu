@@ -73,6 +73,8 @@ __global__ void __launch_bounds__(kWarps * 32) hist_kernel(const int32_t* __rest
                                                            long long A, int E,
                                                            int32_t* __restrict__ chunk_counts,
                                                            unsigned* status) {
+  pdl_wait();  // the previous kernel in the stream has completed
+  pdl_trigger();
   __shared__ int rows[kWarps][kMaxE];
   const int tid = threadIdx.x, warp = tid >> 5;
   for (int i = tid; i < kWarps * kMaxE; i += blockDim.x) (&rows[0][0])[i] = 0;
@@ -97,6 +99,8 @@ constexpr long long kFusedScanMax = 8192;  // chunks x experts summed by every s
 __global__ void __launch_bounds__(kScanThreads) scan_kernel(
     const int32_t* __restrict__ chunk_counts, int32_t* __restrict__ chunk_base, int nchunks, int E,
     int Epad, long long cap, int32_t* __restrict__ counts, int32_t* __restrict__ offsets) {
+  pdl_wait();  // the previous kernel in the stream has completed
+  pdl_trigger();
   __shared__ long long part[kScanThreads];
   __shared__ long long kept_s[kMaxE];
   const int tid = threadIdx.x;
@@ -158,6 +162,8 @@ __global__ void __launch_bounds__(kWarps * 32) scatter_kernel(
     const int32_t* __restrict__ chunk_counts, const int32_t* __restrict__ chunk_base,
     int nchunks, int fused_scan, int32_t* __restrict__ counts, int32_t* __restrict__ offsets,
     int32_t* __restrict__ assign_to_perm, int32_t* __restrict__ perm_to_assign, unsigned* status) {
+  pdl_wait();  // the previous kernel in the stream has completed
+  pdl_trigger();
   __shared__ int rows[kWarps][kMaxE];
   __shared__ int offs[kMaxE];
   __shared__ int cbase[kMaxE];
@@ -262,6 +268,8 @@ __global__ void __launch_bounds__(kSmallWarps * 32) permute_small_kernel(
     const int32_t* __restrict__ ids, long long A, int E, long long cap, int32_t* __restrict__ counts,
     int32_t* __restrict__ offsets, int32_t* __restrict__ assign_to_perm,
     int32_t* __restrict__ perm_to_assign, unsigned* status) {
+  pdl_wait();  // the previous kernel in the stream has completed
+  pdl_trigger();
   __shared__ int rows[kSmallWarps][kMaxE];
   __shared__ long long kept_s[kMaxE];
   __shared__ int offs[kMaxE];
@@ -370,6 +378,8 @@ __global__ void __launch_bounds__(kClusterWarps * 32) permute_cluster_kernel(
     const int32_t* __restrict__ ids, long long A, int E, long long cap, int C,
     int32_t* __restrict__ counts, int32_t* __restrict__ offsets,
     int32_t* __restrict__ assign_to_perm, int32_t* __restrict__ perm_to_assign, unsigned* status) {
+  pdl_wait();  // the previous kernel in the stream has completed
+  pdl_trigger();
   __shared__ int rows[kClusterWarps][kMaxE];
   __shared__ int ctot[kMaxE];   // this CTA's count per expert (read by every CTA)
   __shared__ int cbase[kMaxE];  // counts of the earlier CTAs
@@ -474,21 +484,9 @@ template <int ITERS>
 moe_status launch_cluster_permute(const int32_t* ids, long long A, int E, long long cap, int C,
                                   int32_t* counts, int32_t* offsets, int32_t* a2p, int32_t* p2a,
                                   unsigned* status, cudaStream_t st) {
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3((unsigned)C);
-  cfg.blockDim = dim3(kClusterWarps * 32);
-  cfg.dynamicSmemBytes = 0;
-  cfg.stream = st;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = (unsigned)C;
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
   launch_begin(K_PERMUTE_CLUSTER, st);
-  cudaLaunchKernelEx(&cfg, permute_cluster_kernel<ITERS>, ids, A, E, cap, C, counts, offsets, a2p,
-                     p2a, status);
+  launch_kernel(permute_cluster_kernel<ITERS>, dim3((unsigned)C), dim3(kClusterWarps * 32), 0, st,
+                (unsigned)C, ids, A, E, cap, C, counts, offsets, a2p, p2a, status);
   return launch_end(K_PERMUTE_CLUSTER, st);
 }
 
@@ -501,6 +499,8 @@ __global__ void __launch_bounds__(256) gather_rows_kernel(const uint4* __restric
                                                           int K, int T, int vec_per_row,
                                                           uint4* __restrict__ x_perm,
                                                           unsigned* status) {
+  pdl_wait();  // the previous kernel in the stream has completed
+  pdl_trigger();
   const long long n_kept = *n_kept_ptr;
   const int segs = (vec_per_row + 127) / 128;
   const long long units = n_kept * segs;
@@ -554,8 +554,8 @@ moe_status launch_permute(const moe_shape& s, const int32_t* ids, int32_t* count
   moe_status r;
   if (A > 0 && A <= kSmallMax) {
     launch_begin(K_PERMUTE_SMALL, st);
-    permute_small_kernel<<<1, kSmallWarps * 32, 0, st>>>(ids, A, s.E, cap, counts, offsets, a2p,
-                                                         p2a, status);
+    launch_kernel(permute_small_kernel, dim3(1), dim3(kSmallWarps * 32), 0, st, 1, ids, A, s.E, cap,
+                  counts, offsets, a2p, p2a, status);
     if ((r = launch_end(K_PERMUTE_SMALL, st)) != MOE_OK) return r;
   } else if (A > 0 && A <= kClusterMax) {
     // fewest ids per warp that still fit the chunks into one cluster of <= 8 CTAs
@@ -571,21 +571,23 @@ moe_status launch_permute(const moe_shape& s, const int32_t* ids, int32_t* count
     if (r != MOE_OK) return r;
   } else if (nchunks > 0) {
     launch_begin(K_HIST, st);
-    hist_kernel<<<nchunks, kWarps * 32, 0, st>>>(ids, A, s.E, chunk_counts, status);
+    launch_kernel(hist_kernel, dim3((unsigned)nchunks), dim3(kWarps * 32), 0, st, 1, ids, A, s.E,
+                  chunk_counts, status);
     if ((r = launch_end(K_HIST, st)) != MOE_OK) return r;
     const int fused = (long long)nchunks * s.E <= kFusedScanMax;
     if (!fused) {
       int epad = 1;
       while (epad < s.E) epad <<= 1;
       launch_begin(K_SCAN, st);
-      scan_kernel<<<1, kScanThreads, 0, st>>>(chunk_counts, chunk_base, nchunks, s.E, epad, cap,
-                                              counts, offsets);
+      launch_kernel(scan_kernel, dim3(1), dim3(kScanThreads), 0, st, 1,
+                    (const int32_t*)chunk_counts, chunk_base, nchunks, s.E, epad, cap, counts,
+                    offsets);
       if ((r = launch_end(K_SCAN, st)) != MOE_OK) return r;
     }
     launch_begin(K_SCATTER, st);
-    scatter_kernel<<<nchunks, kWarps * 32, 0, st>>>(ids, A, s.E, cap, chunk_counts, chunk_base,
-                                                    nchunks, fused, counts, offsets, a2p, p2a,
-                                                    status);
+    launch_kernel(scatter_kernel, dim3((unsigned)nchunks), dim3(kWarps * 32), 0, st, 1, ids, A,
+                  s.E, cap, (const int32_t*)chunk_counts, (const int32_t*)chunk_base, nchunks,
+                  fused, counts, offsets, a2p, p2a, status);
     if ((r = launch_end(K_SCATTER, st)) != MOE_OK) return r;
   }
   if (x != nullptr && x_perm != nullptr && A > 0)
@@ -604,8 +606,9 @@ moe_status launch_gather_rows(const moe_shape& s, const void* x, const int32_t* 
   const long long cap_blocks = (long long)sm_count() * 8;
   if (blocks > cap_blocks) blocks = cap_blocks;
   launch_begin(K_GATHER, st);
-  gather_rows_kernel<<<(int)blocks, 256, 0, st>>>((const uint4*)x, p2a, offsets + s.E, s.K, s.T,
-                                                  vec_per_row, (uint4*)x_perm, device_status_ptr());
+  launch_kernel(gather_rows_kernel, dim3((unsigned)blocks), dim3(256), 0, st, 1, (const uint4*)x,
+                p2a, (const int32_t*)(offsets + s.E), s.K, s.T, vec_per_row, (uint4*)x_perm,
+                device_status_ptr());
   return launch_end(K_GATHER, st);
 }
 

@@ -28,6 +28,8 @@ __global__ void __launch_bounds__(kThreads) route_kernel(
     const float* __restrict__ logits_in, float* __restrict__ logits_out,
     int32_t* __restrict__ topk_ids, float* __restrict__ topk_w, int T, int d, int E, int K,
     int renorm) {
+  pdl_wait();  // the previous kernel in the stream has completed
+  pdl_trigger();
   constexpr int RT = kThreads / CT;
   constexpr int TM = RT * RPT;
   constexpr int EP = CT * CPT;
@@ -190,8 +192,9 @@ moe_status launch_route_t(const moe_shape& s, const void* x, const void* w_r, co
   const int grid = (s.T + TM - 1) / TM;
   if (grid == 0) return MOE_OK;
   launch_begin(K_ROUTE, st);
-  kern<<<grid, kThreads, smem, st>>>((const Tin*)x, (const Tin*)w_r, bias, logits_in, logits_out,
-                                     ids, w, s.T, s.d, s.E, s.K, s.renormalize);
+  launch_kernel(kern, dim3((unsigned)grid), dim3(kThreads), smem, st, 1, (const Tin*)x,
+                (const Tin*)w_r, bias, logits_in, logits_out, ids, w, s.T, s.d, s.E, s.K,
+                s.renormalize);
   return launch_end(K_ROUTE, st);
 }
 

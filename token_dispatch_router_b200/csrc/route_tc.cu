@@ -202,6 +202,8 @@ __global__ void __launch_bounds__(R_THREADS) route_tc_kernel(const __grid_consta
   asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
   const uint32_t tmem = *tmem_slot;
   bool ok = true;
+  pdl_wait();  // the previous kernel in the stream has completed
+  pdl_trigger();
 
   if (warp == 0 && lane == 0) {
     int stage = 0;
@@ -411,20 +413,9 @@ moe_status launch_nk(const CUtensorMap& mx, const CUtensorMap& mw, const RouteAr
   auto kern = route_tc_kernel<N, KM>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
     return MOE_ERR_CUDA;
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3((unsigned)(tiles * a.S));
-  cfg.blockDim = dim3(R_THREADS);
-  cfg.dynamicSmemBytes = (size_t)smem;
-  cfg.stream = st;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = (unsigned)a.S;
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
   launch_begin(K_ROUTE_TC, st);
-  cudaLaunchKernelEx(&cfg, kern, mx, mw, a);
+  launch_kernel(kern, dim3((unsigned)(tiles * a.S)), dim3(R_THREADS), (size_t)smem, st,
+                (unsigned)a.S, mx, mw, a);
   return launch_end(K_ROUTE_TC, st);
 }
 
