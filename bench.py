@@ -156,9 +156,16 @@ class ClockSampler:
                 "samples": len(sm)}
 
 
-def kernel_source_hash() -> str:
+# Source file of each kernel a profiles/ record may describe; the shared headers count too.
+KERNEL_SOURCES = {"gateup_tc": "ffn_tc.cu", "down_tc": "ffn_tc.cu", "gateup_tc2": "ffn_tc2.cu",
+                  "down_tc2": "ffn_tc2.cu", "route_tc": "route_tc.cu", "combine": "combine.cu",
+                  "gather_rows": "permute.cu", "permute_cluster": "permute.cu"}
+KERNEL_HEADERS = ("common.cuh", "tc_ptx.cuh", "ffn_args.cuh")
+
+
+def kernel_source_hash(kernel: str) -> str:
     h = hashlib.sha256()
-    for name in ("ffn_tc.cu", "common.cuh"):
+    for name in (KERNEL_SOURCES.get(kernel, "ffn_tc.cu"),) + KERNEL_HEADERS:
         with open(os.path.join(ROOT, "token_dispatch_router_b200", "csrc", name), "rb") as f:
             h.update(f.read())
     return h.hexdigest()[:16]
@@ -168,7 +175,7 @@ def traffic_for(kernel: str, workload: str):
     """ncu DRAM bytes per launch for `kernel` from a `bench-record:` line of a profiles/*.md
     summary, reported only if it was taken on the current kernel source."""
     import glob
-    want = kernel_source_hash()
+    want = kernel_source_hash(kernel)
     for path in sorted(glob.glob(os.path.join(PROFILES_DIR, "*.md"))):
         with open(path) as f:
             for line in f:
