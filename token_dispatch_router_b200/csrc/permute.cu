@@ -360,39 +360,47 @@ __global__ void __launch_bounds__(kSmallWarps * 32) permute_small_kernel(
 }
 
 // Medium problems (kSmallMax < T*K <= kClusterMax): histogram, scan and scatter in one
-// launch of a cluster of C <= 8 CTAs of 32 warps, CTA c owning the contiguous chunk
-// [c * 1024 * ITERS, (c + 1) * 1024 * ITERS) and each warp a slice of ITERS x 32 ids inside
-// it. Same algorithm and result as the three kernels; the ids stay in registers between the
-// counting and the placing walk, and the chunk counts are exchanged through distributed
-// shared memory instead of global memory: after one cluster barrier thread e of every CTA
-// reads the C counts of expert e (its rank base = the counts of the earlier CTAs, the
-// expert's total = all of them), and a second barrier ends all remote reads before any CTA
-// can exit.
-constexpr int kClusterWarps = 32;
+// launch of a cluster of C <= 8 CTAs of WARPS warps, CTA c owning the contiguous chunk
+// [c * WARPS * 32 * ITERS, (c + 1) * WARPS * 32 * ITERS) and each warp a slice of
+// ITERS x 32 ids inside it. Same algorithm and result as the three kernels; the ids stay in
+// registers between the counting and the placing walk, and the chunk counts are exchanged
+// through distributed shared memory instead of global memory: after one cluster barrier
+// thread e of every CTA reads the C counts of expert e (its rank base = the counts of the
+// earlier CTAs, the expert's total = all of them). Each CTA then arrives on a second
+// cluster barrier and waits on it only before exiting, so no CTA leaves while another may
+// still read its counts, and nobody stalls for it in between.
 constexpr int kClusterMaxCtas = 8;
-constexpr int kClusterMaxIters = 4;  // beyond, the three-kernel path is faster (measured)
-constexpr long long kClusterMax = (long long)kClusterMaxCtas * kClusterWarps * 32 * kClusterMaxIters;
+constexpr long long kClusterMax = (long long)kClusterMaxCtas * 32 * 32 * 4;  // 32 warps x 4
 
-template <int ITERS>
-__global__ void __launch_bounds__(kClusterWarps * 32) permute_cluster_kernel(
+__device__ __forceinline__ void cluster_arrive() {
+  asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void cluster_wait() {
+  asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+
+template <int WARPS, int ITERS>
+__global__ void __launch_bounds__(WARPS * 32) permute_cluster_kernel(
     const int32_t* __restrict__ ids, long long A, int E, long long cap, int C,
     int32_t* __restrict__ counts, int32_t* __restrict__ offsets,
     int32_t* __restrict__ assign_to_perm, int32_t* __restrict__ perm_to_assign, unsigned* status) {
-  pdl_wait();  // the previous kernel in the stream has completed
-  pdl_trigger();
-  __shared__ int rows[kClusterWarps][kMaxE];
+  constexpr int NT = WARPS * 32;
+  static_assert(NT >= kMaxE, "one thread per expert in the scan");
+  __shared__ int rows[WARPS][kMaxE];
   __shared__ int ctot[kMaxE];   // this CTA's count per expert (read by every CTA)
   __shared__ int cbase[kMaxE];  // counts of the earlier CTAs
   __shared__ int offs[kMaxE];
   __shared__ int wsum[kMaxE / 32];
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const uint32_t rank = ptx::cluster_rank();
-  const long long s0 = ((long long)rank * kClusterWarps + warp) * (32LL * ITERS);
-  for (int i = tid; i < kClusterWarps * kMaxE; i += blockDim.x) (&rows[0][0])[i] = 0;
-  __syncthreads();
+  const long long s0 = ((long long)rank * WARPS + warp) * (32LL * ITERS);
+  for (int i = tid; i < WARPS * kMaxE; i += NT) (&rows[0][0])[i] = 0;
+  pdl_wait();  // the previous kernel in the stream has completed
+  pdl_trigger();
   int v[ITERS];
 #pragma unroll
   for (int it = 0; it < ITERS; ++it) v[it] = raw_id(ids, s0 + it * 32 + lane, A);
+  __syncthreads();  // rows zeroed
 #pragma unroll
   for (int it = 0; it < ITERS; ++it) v[it] = checked_id(v[it], s0 + it * 32 + lane < A, E, status);
   int* row = rows[warp];
@@ -403,14 +411,18 @@ __global__ void __launch_bounds__(kClusterWarps * 32) permute_cluster_kernel(
     __syncwarp();
   }
   __syncthreads();
-  if (tid < E) {  // per-warp exclusive bases inside the CTA, and the CTA's total
-    int run = 0;
-    for (int w = 0; w < kClusterWarps; ++w) {
-      const int c = rows[w][tid];
-      rows[w][tid] = run;
-      run += c;
+  // per-warp exclusive bases inside the CTA and the CTA's total: warp w takes experts
+  // w, w + WARPS, ...; lane l holds warp l's count and a shuffle scan runs over the lanes
+  for (int e = warp; e < E; e += WARPS) {
+    const int c = lane < WARPS ? rows[lane][e] : 0;
+    int incl = c;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, incl, off);
+      if (lane >= off) incl += y;
     }
-    ctot[tid] = run;
+    if (lane < WARPS) rows[lane][e] = incl - c;
+    if (lane == 31) ctot[e] = incl;
   }
   ptx::cluster_sync();  // every CTA's totals are complete
   int total = 0;
@@ -429,7 +441,7 @@ __global__ void __launch_bounds__(kClusterWarps * 32) permute_cluster_kernel(
     cbase[tid] = before;
     if (rank == 0) counts[tid] = total;
   }
-  ptx::cluster_sync();  // no CTA reads another's shared memory after this point
+  cluster_arrive();  // this CTA's remote reads are done (waited on before exit)
   // exclusive scan of kept = min(total, cap) over the experts (threads 0..255)
   int kept = 0, incl = 0;
   if (tid < kMaxE) {
@@ -478,14 +490,15 @@ __global__ void __launch_bounds__(kClusterWarps * 32) permute_cluster_kernel(
       assign_to_perm[a] = -1;
     }
   }
+  cluster_wait();  // every CTA of the cluster has finished reading this CTA's counts
 }
 
-template <int ITERS>
+template <int WARPS, int ITERS>
 moe_status launch_cluster_permute(const int32_t* ids, long long A, int E, long long cap, int C,
                                   int32_t* counts, int32_t* offsets, int32_t* a2p, int32_t* p2a,
                                   unsigned* status, cudaStream_t st) {
   launch_begin(K_PERMUTE_CLUSTER, st);
-  launch_kernel(permute_cluster_kernel<ITERS>, dim3((unsigned)C), dim3(kClusterWarps * 32), 0, st,
+  launch_kernel(permute_cluster_kernel<WARPS, ITERS>, dim3((unsigned)C), dim3(WARPS * 32), 0, st,
                 (unsigned)C, ids, A, E, cap, C, counts, offsets, a2p, p2a, status);
   return launch_end(K_PERMUTE_CLUSTER, st);
 }
@@ -558,16 +571,25 @@ moe_status launch_permute(const moe_shape& s, const int32_t* ids, int32_t* count
                   counts, offsets, a2p, p2a, status);
     if ((r = launch_end(K_PERMUTE_SMALL, st)) != MOE_OK) return r;
   } else if (A > 0 && A <= kClusterMax) {
-    // fewest ids per warp that still fit the chunks into one cluster of <= 8 CTAs
-    int iters = 1;
-    while ((long long)kClusterMaxCtas * kClusterWarps * 32 * iters < A) iters <<= 1;
-    const int per_cta = kClusterWarps * 32 * iters;
-    const int C = (int)((A + per_cta - 1) / per_cta);
-    switch (iters) {
-      case 1: r = launch_cluster_permute<1>(ids, A, s.E, cap, C, counts, offsets, a2p, p2a, status, st); break;
-      case 2: r = launch_cluster_permute<2>(ids, A, s.E, cap, C, counts, offsets, a2p, p2a, status, st); break;
-      default: r = launch_cluster_permute<4>(ids, A, s.E, cap, C, counts, offsets, a2p, p2a, status, st); break;
+    // one cluster of <= 8 CTAs: 8-warp CTAs with 1, 2 or 4 groups of 32 ids per warp up to
+    // 8192 assignments, 32-warp CTAs with 2 or 4 groups beyond
+    int warps = 8, iters = 1;
+    while ((long long)kClusterMaxCtas * warps * 32 * iters < A) {
+      if (iters < 4) iters <<= 1;
+      else {
+        warps = 32;
+        iters = 2;
+      }
     }
+    const int per_cta = warps * 32 * iters;
+    const int C = (int)((A + per_cta - 1) / per_cta);
+    if (warps == 8)
+      r = iters == 1 ? launch_cluster_permute<8, 1>(ids, A, s.E, cap, C, counts, offsets, a2p, p2a, status, st)
+        : iters == 2 ? launch_cluster_permute<8, 2>(ids, A, s.E, cap, C, counts, offsets, a2p, p2a, status, st)
+                     : launch_cluster_permute<8, 4>(ids, A, s.E, cap, C, counts, offsets, a2p, p2a, status, st);
+    else
+      r = iters == 2 ? launch_cluster_permute<32, 2>(ids, A, s.E, cap, C, counts, offsets, a2p, p2a, status, st)
+                     : launch_cluster_permute<32, 4>(ids, A, s.E, cap, C, counts, offsets, a2p, p2a, status, st);
     if (r != MOE_OK) return r;
   } else if (nchunks > 0) {
     launch_begin(K_HIST, st);

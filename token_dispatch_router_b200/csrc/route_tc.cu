@@ -182,6 +182,10 @@ __global__ void __launch_bounds__(R_THREADS) route_tc_kernel(const __grid_consta
   const int S = g.S;
   const int kb0 = (int)(rank * g.kblocks / S), kb1 = (int)((rank + 1) * g.kblocks / S);
 
+  if (tid == 32) {  // fetch both tensor maps while the barriers are set up
+    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmX)) : "memory");
+    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmW)) : "memory");
+  }
   if (tid == 0) {
     for (int s = 0; s < RSTAGES; ++s) {
       mbar_init(saddr(&full[s]), 1);
