@@ -166,6 +166,26 @@ moe_status moe_permute_static(const moe_shape* shape, const int32_t* topk_ids, i
                               const void* x, void* x_perm, moe_stream_t stream);
 
 /* ----------------------------------------------------------------------------
+ * moe_dispatch - moe_route followed by moe_permute, in one call.
+ * The steps are those of the two calls ("How AI chips support MoE", chapter 4,
+ * sections 4.2-4.3; "Operators & compilers: MoE routing and sparse kernels", section 3);
+ * the pages describe no separate dispatch operation, this is a launch-count saving for
+ * the decode regime. Arguments are the union of both calls' (x serves the router and
+ * the optional gather); every output equals what moe_route then moe_permute write.
+ * When logits_in is given, T*K <= 8192, E <= 256 and K <= 32, one kernel (one
+ * cluster of up to 8 CTAs) routes and permutes without a round trip of the ids through
+ * global memory; otherwise the two calls' kernels run in turn. bias is added only to
+ * x W_r, as in moe_route.
+ *   workspace, ws_bytes  >= moe_permute_workspace_size(shape)
+ * Errors: those of moe_route and moe_permute.
+ */
+moe_status moe_dispatch(const moe_shape* shape, const void* x, const void* w_r, const float* bias,
+                        const float* logits_in, float* logits_out, int32_t* topk_ids,
+                        float* topk_w, int32_t* counts, int32_t* offsets,
+                        int32_t* assign_to_perm, int32_t* perm_to_assign, void* x_perm,
+                        void* workspace, size_t ws_bytes, moe_stream_t stream);
+
+/* ----------------------------------------------------------------------------
  * moe_grouped_ffn - the grouped SwiGLU expert FFN on the expert-major rows.
  * SonicMoE explainer, section 3 items 3-5 (grouped GEMM with a different M
  * per expert, SwiGLU, second grouped GEMM), section 6.2 (the gather of x is

@@ -99,3 +99,24 @@ def test_null_pointers_and_short_workspace_rejected(lib):
                         None, 0, None)
     assert r == 4
     assert lib.moe_selftest_timeout(0, None) == 1
+
+
+def test_dispatch_argument_checks_on_host(lib):
+    s = tdr.make_shape(16, 128, 8, 2, 128)
+    dummy = ctypes.c_void_p(256)  # never dereferenced: every check below fails first
+    # a missing output
+    r = lib.moe_dispatch(ctypes.byref(s), None, None, None, dummy, None, None, dummy, dummy,
+                         dummy, dummy, dummy, None, None, 0, None)
+    assert r == 1
+    # routable from the given logits in one kernel, but no workspace for the permute scratch
+    r = lib.moe_dispatch(ctypes.byref(s), None, None, None, dummy, None, dummy, dummy, dummy,
+                         dummy, dummy, dummy, None, None, 0, None)
+    assert r == 4
+    # a gather without x
+    r = lib.moe_dispatch(ctypes.byref(s), None, None, None, dummy, None, dummy, dummy, dummy,
+                         dummy, dummy, dummy, dummy, None, 0, None)
+    assert r == 1
+    bad = tdr.make_shape(16, 128, 8, 9, 128)  # K > E
+    r = lib.moe_dispatch(ctypes.byref(bad), None, None, None, dummy, None, dummy, dummy, dummy,
+                         dummy, dummy, dummy, None, None, 0, None)
+    assert r == 1

@@ -241,6 +241,61 @@ def test_permute_flags_out_of_range_ids(cuda_lib):
     assert int(perm["counts"].cpu().sum()) == T * K - 1
 
 
+# ------------------------------------------------------------------ dispatch (route + permute)
+@pytest.mark.parametrize("T,E,K,cf,renorm,ties", [
+    (64, 64, 6, 0.0, True, False),      # the dispatch workload's decode-regime sizes
+    (256, 64, 6, 0.0, True, False),
+    (1024, 64, 6, 0.0, True, False),
+    (1, 1, 1, 0.0, True, False),
+    (33, 8, 2, 1.0, False, False),
+    (1365, 64, 6, 1.25, True, False),   # 8190 assignments over 8 ragged CTAs
+    (256, 256, 32, 0.0, True, True),    # E = 256, K = 32, integer logits (ties)
+    (1000, 37, 5, 0.5, False, True),
+    (1366, 64, 6, 0.0, True, False),    # 8196 assignments: the two-call path
+])
+def test_dispatch_matches_oracle_and_the_two_calls(cuda_lib, T, E, K, cf, renorm, ties):
+    tdr = cuda_lib
+    rng = np.random.default_rng(T * 7 + E)
+    if ties:
+        lg = rng.integers(-3, 4, size=(T, E)).astype(np.float32)
+        lg[0, ::2] = -0.0
+    else:
+        lg = rng.standard_normal((T, E)).astype(np.float32)
+    s = tdr.make_shape(T, 64, E, K, 64, cf, renorm, torch.bfloat16)
+    lgd = torch.from_numpy(lg).cuda()
+    lo = torch.empty(T, E, device="cuda")
+    out = tdr.dispatch(s, logits_in=lgd, logits_out=lo)
+    np.testing.assert_array_equal(lo.cpu().numpy(), lg)
+    ids_ref, w_ref = orc.route(lg, K, renorm)
+    np.testing.assert_array_equal(out["topk_ids"].cpu().numpy(), ids_ref)
+    assert np.abs(out["topk_w"].cpu().numpy().astype(np.float64) - w_ref).max() <= W_ABS
+    _, offsets, _, _ = check_permutation(out, ids_ref, E, orc.capacity(cf, T, K, E))
+    ids2, w2, _ = tdr.route(s, logits_in=lgd)
+    p2 = tdr.permute(s, ids2)
+    assert torch.equal(out["topk_ids"], ids2) and torch.equal(out["topk_w"], w2)
+    nk = int(offsets[-1])
+    for k in ("counts", "offsets", "assign_to_perm"):
+        assert torch.equal(out[k], p2[k])
+    assert torch.equal(out["perm_to_assign"][:nk], p2["perm_to_assign"][:nk])
+    assert_status_ok(tdr)
+
+
+def test_dispatch_materialised_gather_is_exact(cuda_lib):
+    tdr = cuda_lib
+    rng = np.random.default_rng(17)
+    T, E, K, d = 300, 16, 3, 256
+    lg = rng.standard_normal((T, E)).astype(np.float32)
+    x = torch.randn(T, d).to(torch.bfloat16)
+    s = tdr.make_shape(T, d, E, K, 64, 0.9, True, torch.bfloat16)
+    out = tdr.dispatch(s, x=x.cuda(), logits_in=torch.from_numpy(lg).cuda(), materialize=True)
+    ids_ref, _ = orc.route(lg, K, True)
+    _, offsets, _, p2a = check_permutation(out, ids_ref, E, orc.capacity(0.9, T, K, E))
+    nk = int(offsets[-1])
+    ref = orc.gather_rows(x.float().numpy(), p2a, offsets, K)
+    np.testing.assert_array_equal(out["x_perm"][:nk].float().cpu().numpy(), ref)
+    assert_status_ok(tdr)
+
+
 # ------------------------------------------------------------------ combine
 @pytest.mark.parametrize("dtype", ["f32", "bf16"])
 def test_combine_matches_oracle(cuda_lib, dtype):

@@ -51,6 +51,8 @@ _SIGS = {
     "moe_route": (ctypes.c_int, [_S, _P, _P, _P, _P, _P, _P, _P, _P]),
     "moe_permute": (ctypes.c_int, [_S, _P, _P, _P, _P, _P, _P, _P, _P, ctypes.c_size_t, _P]),
     "moe_permute_static": (ctypes.c_int, [_S, _P, _P, _P, _P, _P, _P, _P, _P]),
+    "moe_dispatch": (ctypes.c_int, [_S, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P,
+                                    ctypes.c_size_t, _P]),
     "moe_grouped_ffn": (ctypes.c_int, [_S, _P, _P, _P, _P, _P, _P, _P, _P, _P]),
     "moe_combine": (ctypes.c_int, [_S, _P, _P, _P, _P, _P]),
     "moe_forward": (ctypes.c_int, [_S, _P, _P, _P, _P, _P, _P, _P, _P, _P, ctypes.c_size_t, _P]),
@@ -187,6 +189,58 @@ def permute(shape: moe_shape, topk_ids: torch.Tensor, x=None, materialize: bool 
     if materialize:
         out["x_perm"] = x_perm
     return out
+
+
+def dispatch(shape: moe_shape, x=None, w_r=None, bias=None, logits_in=None, logits_out=None,
+             materialize: bool = False, workspace=None, out=None):
+    """moe_dispatch (moe_route then moe_permute in one call). Returns dict(topk_ids, topk_w,
+    counts, offsets, assign_to_perm, perm_to_assign[, x_perm][, logits_out]); `out` may hold
+    preallocated tensors under those names."""
+    lib = load_library()
+    T, E, K = shape.T, shape.E, shape.K
+    src = logits_in if logits_in is not None else x
+    dev = src.device
+    dt = _act_dtype(shape)
+    if logits_in is None:
+        _dev(x, "x", dt, (T, shape.d))
+        _dev(w_r, "w_r", dt, (shape.d, E))
+    else:
+        _dev(logits_in, "logits_in", torch.float32, (T, E))
+    if bias is not None:
+        _dev(bias, "bias", torch.float32, (E,))
+    if logits_out is not None:
+        _dev(logits_out, "logits_out", torch.float32, (T, E))
+    o = dict(out or {})
+
+    def get(name, shape_, dtype):
+        if name not in o:
+            o[name] = torch.empty(*shape_, dtype=dtype, device=dev)
+        return o[name]
+
+    ids = get("topk_ids", (T, K), torch.int32)
+    w = get("topk_w", (T, K), torch.float32)
+    counts = get("counts", (E,), torch.int32)
+    offsets = get("offsets", (E + 1,), torch.int32)
+    a2p = get("assign_to_perm", (T * K,), torch.int32)
+    p2a = get("perm_to_assign", (T * K,), torch.int32)
+    x_perm = None
+    if materialize:
+        _dev(x, "x", dt, (T, shape.d))
+        x_perm = get("x_perm", (T * K, shape.d), x.dtype)
+    need = permute_workspace_size(shape)
+    if workspace is None:
+        workspace = torch.empty(max(need, 256), dtype=torch.uint8, device=dev)
+    _check(lib.moe_dispatch(ctypes.byref(shape), _ptr(x), _ptr(w_r), _ptr(bias), _ptr(logits_in),
+                            _ptr(logits_out), _ptr(ids), _ptr(w), _ptr(counts), _ptr(offsets),
+                            _ptr(a2p), _ptr(p2a), _ptr(x_perm), _ptr(workspace),
+                            workspace.numel(), _stream()), "moe_dispatch")
+    res = dict(topk_ids=ids, topk_w=w, counts=counts, offsets=offsets, assign_to_perm=a2p,
+               perm_to_assign=p2a)
+    if materialize:
+        res["x_perm"] = x_perm
+    if logits_out is not None:
+        res["logits_out"] = logits_out
+    return res
 
 
 def permute_static(shape: moe_shape, topk_ids: torch.Tensor, x=None, materialize: bool = False):

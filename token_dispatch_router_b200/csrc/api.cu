@@ -33,6 +33,12 @@ moe_status launch_permute_static(const moe_shape& s, const int32_t* ids, int32_t
                                  void* x_perm, cudaStream_t st);
 moe_status launch_route_tc(const moe_shape& s, const void* x, const void* w_r, const float* bias,
                            float* logits_out, int32_t* ids, float* w, cudaStream_t st);
+bool route_permute_fusable(const moe_shape& s, const float* logits_in);
+moe_status launch_route_permute(const moe_shape& s, const float* logits_in, float* logits_out,
+                                int32_t* ids, float* w, int32_t* counts, int32_t* offsets,
+                                int32_t* a2p, int32_t* p2a, cudaStream_t st);
+moe_status launch_gather_rows(const moe_shape& s, const void* x, const int32_t* p2a,
+                              const int32_t* offsets, void* x_perm, cudaStream_t st);
 
 // ------------------------------------------------------------------ device state
 __device__ unsigned int g_device_status;
@@ -77,7 +83,7 @@ const char* kKernelNames[K_COUNT] = {
     "route",        "hist",          "scan",           "scatter",     "gather_rows", "gateup_tc",
     "down_tc",      "gateup_simt",   "down_simt",      "combine",     "selftest_timeout",
     "route_tc",     "permute_small", "gateup_tc2",   "down_tc2",
-    "permute_cluster"};
+    "permute_cluster", "route_permute"};
 
 struct ProfRec {
   int kid;
@@ -275,6 +281,36 @@ moe_status moe_permute_static(const moe_shape* s, const int32_t* topk_ids, int32
                                x_perm, (cudaStream_t)stream);
 }
 
+moe_status moe_dispatch(const moe_shape* s, const void* x, const void* w_r, const float* bias,
+                        const float* logits_in, float* logits_out, int32_t* topk_ids,
+                        float* topk_w, int32_t* counts, int32_t* offsets,
+                        int32_t* assign_to_perm, int32_t* perm_to_assign, void* x_perm,
+                        void* workspace, size_t ws_bytes, moe_stream_t stream) {
+  const bool gather = x_perm != nullptr;
+  moe_status r = check_shape(s, logits_in == nullptr || gather, false);
+  if (r != MOE_OK) return r;
+  if (s->T == 0)
+    return moe_permute(s, topk_ids, counts, offsets, assign_to_perm, perm_to_assign, nullptr,
+                       nullptr, workspace, ws_bytes, stream);
+  if (!topk_ids || !topk_w || !counts || !offsets || !assign_to_perm || !perm_to_assign)
+    return MOE_ERR_INVALID_ARG;
+  if (gather && (x == nullptr || !aligned16(x) || !aligned16(x_perm))) return MOE_ERR_INVALID_ARG;
+  if (!route_permute_fusable(*s, logits_in)) {
+    if ((r = moe_route(s, x, w_r, bias, logits_in, logits_out, topk_ids, topk_w, stream)) != MOE_OK)
+      return r;
+    return moe_permute(s, topk_ids, counts, offsets, assign_to_perm, perm_to_assign,
+                       gather ? x : nullptr, x_perm, workspace, ws_bytes, stream);
+  }
+  const size_t need = permute_scratch_bytes(*s);
+  if (need > 0 && (workspace == nullptr || ws_bytes < need)) return MOE_ERR_WORKSPACE;
+  const cudaStream_t st = (cudaStream_t)stream;
+  if ((r = launch_route_permute(*s, logits_in, logits_out, topk_ids, topk_w, counts, offsets,
+                                assign_to_perm, perm_to_assign, st)) != MOE_OK)
+    return r;
+  if (gather) return launch_gather_rows(*s, x, perm_to_assign, offsets, x_perm, st);
+  return MOE_OK;
+}
+
 moe_status moe_grouped_ffn(const moe_shape* s, const void* x, const int32_t* offsets,
                            const int32_t* perm_to_assign, const void* w_gate, const void* w_up,
                            const void* w_down, void* a_act, void* y_perm, moe_stream_t stream) {
@@ -324,10 +360,16 @@ moe_status moe_forward(const moe_shape* s, const void* x, const void* w_r, const
   int32_t* offsets = (int32_t*)(ws + L.offsets);
   int32_t* a2p = (int32_t*)(ws + L.assign_to_perm);
   int32_t* p2a = (int32_t*)(ws + L.perm_to_assign);
-  if ((r = moe_route(s, x, w_r, bias, logits_in, logits, ids, w, stream)) != MOE_OK) return r;
-  if ((r = launch_permute(*s, ids, counts, offsets, a2p, p2a, nullptr, nullptr,
-                          ws + L.permute_scratch, st)) != MOE_OK)
-    return r;
+  if (route_permute_fusable(*s, logits_in)) {
+    if ((r = launch_route_permute(*s, logits_in, logits, ids, w, counts, offsets, a2p, p2a, st)) !=
+        MOE_OK)
+      return r;
+  } else {
+    if ((r = moe_route(s, x, w_r, bias, logits_in, logits, ids, w, stream)) != MOE_OK) return r;
+    if ((r = launch_permute(*s, ids, counts, offsets, a2p, p2a, nullptr, nullptr,
+                            ws + L.permute_scratch, st)) != MOE_OK)
+      return r;
+  }
   if ((r = moe_grouped_ffn(s, x, offsets, p2a, w_gate, w_up, w_down, ws + L.a_act, ws + L.y_perm,
                            stream)) != MOE_OK)
     return r;

@@ -102,6 +102,7 @@ enum KernelId {
   K_GATEUP_TC2,
   K_DOWN_TC2,
   K_PERMUTE_CLUSTER,
+  K_ROUTE_PERMUTE,
   K_COUNT
 };
 

@@ -503,6 +503,206 @@ moe_status launch_cluster_permute(const int32_t* ids, long long A, int E, long l
   return launch_end(K_PERMUTE_CLUSTER, st);
 }
 
+// Routing and permutation in one launch, for given router logits and at most
+// kFusedMax assignments (the decode regime: a few hundred to a thousand tokens).
+// "How AI chips support MoE", chapter 4, sections 4.2-4.3 (softmax, top-K) and
+// "Operators & compilers: MoE routing and sparse kernels", section 3 (count, prefix sum,
+// scatter): the steps are those of the router and of the cluster permute above, run by one
+// cluster of C <= 8 CTAs of 8 warps without a round trip of the ids through global memory.
+// CTA c owns the tokens [c * tpc, (c + 1) * tpc) and so the assignments
+// [c * tpc * K, (c + 1) * tpc * K). Routing: one warp per token, each lane holding up to 8
+// logits (e = lane + 32 j), K rounds of a warp arg-max under (value descending, id
+// ascending; +0 == -0), weights exp(l - l_max) over the selected (renormalised) or over all
+// E; the ids also go to shared memory. Permutation: each warp owns ITERS x 32 of the CTA's
+// assignments, and the histogram, cluster exchange of counts, scan and scatter follow the
+// cluster permute exactly.
+constexpr int kFusedWarps = 8;
+constexpr long long kFusedMax = (long long)kClusterMaxCtas * kFusedWarps * 32 * 4;  // 8192
+
+template <int ITERS>
+__global__ void __launch_bounds__(kFusedWarps * 32) route_permute_kernel(
+    const float* __restrict__ logits_in, float* __restrict__ logits_out, int T, int E, int K,
+    int renorm, int tpc, long long cap, int C, int32_t* __restrict__ topk_ids,
+    float* __restrict__ topk_w, int32_t* __restrict__ counts, int32_t* __restrict__ offsets,
+    int32_t* __restrict__ assign_to_perm, int32_t* __restrict__ perm_to_assign) {
+  constexpr int WARPS = kFusedWarps, NT = WARPS * 32;
+  constexpr int CHUNK = NT * ITERS;  // assignments a CTA can own
+  __shared__ int rows[WARPS][kMaxE];
+  __shared__ int ctot[kMaxE];
+  __shared__ int cbase[kMaxE];
+  __shared__ int offs[kMaxE];
+  __shared__ int wsum[kMaxE / 32];
+  __shared__ int sid[CHUNK];  // this CTA's ids, in flat assignment order
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const uint32_t rank = C > 1 ? ptx::cluster_rank() : 0u;
+  const int t0 = (int)rank * tpc;
+  const int ntok = max(0, min(tpc, T - t0));
+  const int na = ntok * K;                      // assignments of this CTA
+  const long long a0 = (long long)t0 * K;       // the first one's flat index
+  for (int i = tid; i < WARPS * kMaxE; i += NT) (&rows[0][0])[i] = 0;
+  pdl_wait();  // the previous kernel in the stream has completed
+  pdl_trigger();
+
+  // ---------------------------------------------------------------- routing
+  for (int r = warp; r < ntok; r += WARPS) {
+    const int t = t0 + r;
+    float v[8];
+    bool taken[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const int e = lane + 32 * j;
+      v[j] = (e < E) ? logits_in[(size_t)t * E + e] : -INFINITY;
+      taken[j] = (e >= E);
+      if (logits_out != nullptr && e < E) logits_out[(size_t)t * E + e] = v[j];
+    }
+    float vmax = 0.f, selv = 0.f;
+    int sele = 0;
+    for (int k = 0; k < K; ++k) {
+      float bv = -INFINITY;
+      int be = 0x7fffffff;
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        const int e = lane + 32 * j;
+        if (!taken[j] && (v[j] > bv || (v[j] == bv && e < be))) {
+          bv = v[j];
+          be = e;
+        }
+      }
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) {
+        const float ov = __shfl_xor_sync(0xffffffffu, bv, off);
+        const int oe = __shfl_xor_sync(0xffffffffu, be, off);
+        if (ov > bv || (ov == bv && oe < be)) {
+          bv = ov;
+          be = oe;
+        }
+      }
+#pragma unroll
+      for (int j = 0; j < 8; ++j)
+        if (lane + 32 * j == be) taken[j] = true;
+      if (k == 0) vmax = bv;
+      if (lane == k) {
+        selv = bv;
+        sele = be;
+      }
+    }
+    const float ex = (lane < K) ? expf(selv - vmax) : 0.f;
+    float den;
+    if (renorm) {
+      den = ex;
+    } else {
+      den = 0.f;
+#pragma unroll
+      for (int j = 0; j < 8; ++j)
+        if (lane + 32 * j < E) den += expf(v[j] - vmax);
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) den += __shfl_xor_sync(0xffffffffu, den, off);
+    if (lane < K) {
+      topk_ids[(size_t)t * K + lane] = sele;
+      topk_w[(size_t)t * K + lane] = ex / den;
+      sid[r * K + lane] = sele;
+    }
+  }
+  __syncthreads();  // the CTA's ids are in shared memory; rows are zeroed
+
+  // ---------------------------------------------------------------- permutation
+  const int l0 = warp * 32 * ITERS;  // this warp's slice of the CTA's assignments
+  int v[ITERS];
+#pragma unroll
+  for (int it = 0; it < ITERS; ++it) {
+    const int l = l0 + it * 32 + lane;
+    v[it] = l < na ? sid[l] : -1;
+  }
+  int* row = rows[warp];
+#pragma unroll
+  for (int it = 0; it < ITERS; ++it) {
+    const unsigned m = __match_any_sync(0xffffffffu, v[it]);
+    if (v[it] >= 0 && lane == __ffs(m) - 1) row[v[it]] += __popc(m);
+    __syncwarp();
+  }
+  __syncthreads();
+  for (int e = warp; e < E; e += WARPS) {
+    const int c = lane < WARPS ? rows[lane][e] : 0;
+    int incl = c;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, incl, off);
+      if (lane >= off) incl += y;
+    }
+    if (lane < WARPS) rows[lane][e] = incl - c;
+    if (lane == 31) ctot[e] = incl;
+  }
+  if (C > 1) ptx::cluster_sync();  // every CTA's totals are complete
+  else __syncthreads();
+  int total = 0;
+  if (tid < E) {
+    int cv[kClusterMaxCtas];
+    const uint32_t mine = ptx::saddr(&ctot[tid]);
+#pragma unroll
+    for (int q = 0; q < kClusterMaxCtas; ++q)
+      cv[q] = q == (int)rank ? ctot[tid]
+              : q < C        ? ptx::ld_dsmem_s32(ptx::map_rank(mine, (uint32_t)q))
+                             : 0;
+    int before = 0;
+#pragma unroll
+    for (int q = 0; q < kClusterMaxCtas; ++q) {
+      if (q < (int)rank) before += cv[q];
+      total += cv[q];
+    }
+    cbase[tid] = before;
+    if (rank == 0) counts[tid] = total;
+  }
+  if (C > 1) cluster_arrive();  // remote reads done (waited on before exit)
+  int kept = 0, incl = 0;
+  if (tid < kMaxE) {
+    kept = (tid < E) ? (int)((cap >= 0 && total > cap) ? cap : total) : 0;
+    incl = kept;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, incl, off);
+      if (lane >= off) incl += y;
+    }
+    if (lane == 31) wsum[warp] = incl;
+  }
+  __syncthreads();
+  if (tid < kMaxE) {
+    int pre = 0;
+    for (int w = 0; w < warp; ++w) pre += wsum[w];
+    incl += pre;
+    if (tid < E) {
+      offs[tid] = incl - kept;
+      if (rank == 0) {
+        offsets[tid] = incl - kept;
+        if (tid == E - 1) offsets[E] = incl;
+      }
+    }
+  }
+  __syncthreads();
+  const unsigned lt = lanemask_lt();
+#pragma unroll
+  for (int it = 0; it < ITERS; ++it) {
+    const int l = l0 + it * 32 + lane;
+    const long long a = a0 + l;
+    const int id = v[it];
+    const unsigned m = __match_any_sync(0xffffffffu, id);
+    int r = 0;
+    if (id >= 0) r = cbase[id] + row[id] + __popc(m & lt);
+    __syncwarp();
+    if (id >= 0 && lane == __ffs(m) - 1) row[id] += __popc(m);
+    __syncwarp();
+    if (id >= 0) {
+      int p = -1;
+      if (cap < 0 || r < cap) {
+        p = offs[id] + r;
+        perm_to_assign[p] = (int32_t)a;
+      }
+      assign_to_perm[a] = p;
+    }
+  }
+  if (C > 1) cluster_wait();  // every CTA has finished reading this CTA's counts
+}
+
 // x_perm[p] = x[perm_to_assign[p] / K] for p < offsets[E]; 16-byte vectors. One warp moves
 // a 2 KB segment (128 vectors) of one row: the row's source token is loaded once per lane
 // and each lane keeps four independent 16-byte loads in flight.
@@ -632,6 +832,50 @@ moe_status launch_gather_rows(const moe_shape& s, const void* x, const int32_t* 
                 p2a, (const int32_t*)(offsets + s.E), s.K, s.T, vec_per_row, (uint4*)x_perm,
                 device_status_ptr());
   return launch_end(K_GATHER, st);
+}
+
+namespace {
+// CTAs of the fused kernel: about 32 tokens (4 a warp) per CTA, at most 8 CTAs; false if a
+// CTA would own more than 4 x 32 assignments per warp
+bool fused_grid(const moe_shape& s, int* C_out, int* tpc_out, int* iters_out) {
+  int C = (s.T + 31) / 32;
+  if (C > kClusterMaxCtas) C = kClusterMaxCtas;
+  if (C < 1) C = 1;
+  const int tpc = (s.T + C - 1) / C;
+  const long long per = (long long)tpc * s.K;  // assignments per CTA
+  if (per > (long long)kFusedWarps * 32 * 4) return false;
+  *C_out = C;
+  *tpc_out = tpc;
+  *iters_out = per <= kFusedWarps * 32 ? 1 : per <= kFusedWarps * 64 ? 2 : 4;
+  return true;
+}
+}  // namespace
+
+bool route_permute_fusable(const moe_shape& s, const float* logits_in) {
+  int C, tpc, iters;
+  return logits_in != nullptr && s.T > 0 && s.E <= kMaxE && s.K <= 32 &&
+         (long long)s.T * s.K <= kFusedMax && fused_grid(s, &C, &tpc, &iters);
+}
+
+moe_status launch_route_permute(const moe_shape& s, const float* logits_in, float* logits_out,
+                                int32_t* ids, float* w, int32_t* counts, int32_t* offsets,
+                                int32_t* a2p, int32_t* p2a, cudaStream_t st) {
+  const long long cap =
+      (s.capacity_factor > 0.f)
+          ? (long long)ceil((double)s.capacity_factor * (double)s.T * (double)s.K / (double)s.E)
+          : -1;
+  int C, tpc, iters;
+  if (!fused_grid(s, &C, &tpc, &iters)) return MOE_ERR_UNSUPPORTED;
+  launch_begin(K_ROUTE_PERMUTE, st);
+  auto go = [&](auto kern) {
+    launch_kernel(kern, dim3((unsigned)C), dim3(kFusedWarps * 32), 0, st, (unsigned)C, logits_in,
+                  logits_out, s.T, s.E, s.K, s.renormalize, tpc, cap, C, ids, w, counts, offsets,
+                  a2p, p2a);
+  };
+  if (iters == 1) go(route_permute_kernel<1>);
+  else if (iters == 2) go(route_permute_kernel<2>);
+  else go(route_permute_kernel<4>);
+  return launch_end(K_ROUTE_PERMUTE, st);
 }
 
 // ------------------------------------------------------------------ no-allocation variant
