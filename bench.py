@@ -266,6 +266,14 @@ def run_reference(args, rank, world):
 
 
 # ------------------------------------------------------------------ dispatch + combine
+def hold_gpu(us: float = 200.0):
+    """Keep the GPU busy for `us` microseconds so that the host has queued the next timed
+    sequence before the GPU reaches it (the timed region then holds no host time)."""
+    sleep = getattr(torch.cuda, "_sleep", None)
+    if sleep is not None:
+        sleep(int(us * 2000))  # cycles at about 2 GHz
+
+
 def dispatch_combine_bytes(cfg) -> int:
     """Algorithmic bytes of route + permute (gathered rows materialised) + combine:
     route reads x and writes logits, ids and weights; permute reads ids and writes both
@@ -307,6 +315,7 @@ def dispatch_combine(tdr, s, cfg, x, w_r, bias, steps, world, peaks):
           for _ in range(n)]
     for a, b in ev:
         flush.sum()
+        hold_gpu()
         a.record()
         once()
         b.record()
@@ -337,6 +346,58 @@ def dispatch_combine(tdr, s, cfg, x, w_r, bias, steps, world, peaks):
             "note": "route + permute with x_perm materialised + combine(x_perm) at the layer's "
                     "shape; GB/s = algorithmic bytes over the device time of one sequence after "
                     "an L2 flush (launch gaps inside the sequence included)"}
+
+
+def decode_dispatch(tdr, world, Ts=(64, 256, 512, 1024)):
+    """Dispatch workload (given N(0,1) logits, E=64 K=6 d=4096 bf16) in the decode regime:
+    route + permute with x_perm materialised + combine of those rows, per L2-flushed
+    sequence with CUDA events around it, through the two calls (moe_route, moe_permute) and
+    through moe_dispatch (one kernel for routing and permutation)."""
+    base = mi.CONFIGS["dispatch_combine"]
+    dev = torch.device("cuda", torch.cuda.current_device())
+    flush = torch.ones(64 << 20, dtype=torch.int64, device=dev)
+    res = {}
+    for T in Ts:
+        cfg = base.with_T(T)
+        inp = mi.make_inputs(cfg)
+        x, lg = inp.x.to(dev), inp.logits.to(dev)
+        s = tdr.make_shape(T, cfg.d, cfg.E, cfg.K, 64, 0.0, True, torch.bfloat16)
+        pws = torch.empty(max(tdr.permute_workspace_size(s), 256), dtype=torch.uint8, device=dev)
+        out = torch.empty(T, cfg.d, dtype=x.dtype, device=dev)
+        bufs = {}
+
+        def two_calls():
+            ids, w, _ = tdr.route(s, logits_in=lg)
+            p = tdr.permute(s, ids, x=x, materialize=True, workspace=pws)
+            tdr.combine(s, p["x_perm"], p["assign_to_perm"], w, out=out)
+
+        def one_call():
+            r = tdr.dispatch(s, x=x, logits_in=lg, materialize=True, workspace=pws, out=bufs)
+            bufs.update(r)
+            tdr.combine(s, r["x_perm"], r["assign_to_perm"], r["topk_w"], out=out)
+
+        row = {}
+        for name, fn in (("two_calls_us", two_calls), ("moe_dispatch_us", one_call)):
+            for _ in range(3):
+                fn()
+            torch.cuda.synchronize()
+            n = 50
+            ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                  for _ in range(n)]
+            for a, b in ev:
+                flush.sum()
+                hold_gpu()
+                a.record()
+                fn()
+                b.record()
+            torch.cuda.synchronize()
+            row[name] = round(1e3 * max_over_ranks(sum(a.elapsed_time(b) for a, b in ev) / n,
+                                                   world), 2)
+        res[f"T={T}"] = row
+    del flush
+    return {"workload": "dispatch_combine (E=64 K=6 d=4096 bf16, given logits)", "latency": res,
+            "note": "route + permute with x_perm + combine, one sequence per L2-flushed "
+                    "iteration, CUDA events, launch gaps included"}
 
 
 # ------------------------------------------------------------------ our arm
@@ -467,6 +528,7 @@ def run_ours(args, rank, world, local):
     # ---- dispatch + combine byte stream at the same shape (route, permute with the gathered
     # rows materialised, combine of those rows as identity experts): the unfused traffic
     dc = dispatch_combine(tdr, s, cfg, x, w_r, bias, args.steps, world, peaks)
+    dd = decode_dispatch(tdr, world)
 
     # ---- per-kernel breakdown (ms per step) and the two secondary figures of the metric
     per_kernel = {k: round(ms / args.steps, 4) for k, (n, ms) in kern.items()}
@@ -480,7 +542,7 @@ def run_ours(args, rank, world, local):
         "config": {"workload": cfg.name, "T": cfg.T, "d": cfg.d, "E": cfg.E, "K": cfg.K,
                    "n": cfg.n, "global_batch": cfg.T * world, "parallelism": f"replicas{world}",
                    "l2": "inputs larger than L2: the 2.82 GB of expert weights stream every step"},
-        "roofline": roofline, "gemm": gemm, "dispatch_combine": dc,
+        "roofline": roofline, "gemm": gemm, "dispatch_combine": dc, "decode_dispatch": dd,
         "kernel_ms_per_step": per_kernel,
         "gpu_launches": int(launches), "e2e": e2e,
     }

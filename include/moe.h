@@ -172,7 +172,7 @@ moe_status moe_permute_static(const moe_shape* shape, const int32_t* topk_ids, i
  * the pages describe no separate dispatch operation, this is a launch-count saving for
  * the decode regime. Arguments are the union of both calls' (x serves the router and
  * the optional gather); every output equals what moe_route then moe_permute write.
- * When logits_in is given, T*K <= 8192, E <= 256 and K <= 32, one kernel (one
+ * When logits_in is given, T*K <= 4096, E <= 256 and K <= 32, one kernel (one
  * cluster of up to 8 CTAs) routes and permutes without a round trip of the ids through
  * global memory; otherwise the two calls' kernels run in turn. bias is added only to
  * x W_r, as in moe_route.

@@ -248,10 +248,11 @@ def test_permute_flags_out_of_range_ids(cuda_lib):
     (1024, 64, 6, 0.0, True, False),
     (1, 1, 1, 0.0, True, False),
     (33, 8, 2, 1.0, False, False),
-    (1365, 64, 6, 1.25, True, False),   # 8190 assignments over 8 ragged CTAs
-    (256, 256, 32, 0.0, True, True),    # E = 256, K = 32, integer logits (ties)
-    (1000, 37, 5, 0.5, False, True),
-    (1366, 64, 6, 0.0, True, False),    # 8196 assignments: the two-call path
+    (682, 64, 6, 1.25, True, False),    # 4092 assignments over 8 ragged CTAs of 32 warps
+    (128, 256, 32, 0.0, True, True),    # E = 256, K = 32, integer logits (ties)
+    (800, 37, 5, 0.5, False, True),     # 4000 assignments
+    (683, 64, 6, 0.0, True, False),     # 4098 assignments: the two-call path
+    (1365, 64, 6, 1.25, True, False),
 ])
 def test_dispatch_matches_oracle_and_the_two_calls(cuda_lib, T, E, K, cf, renorm, ties):
     tdr = cuda_lib

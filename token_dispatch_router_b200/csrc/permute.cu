@@ -504,11 +504,12 @@ moe_status launch_cluster_permute(const int32_t* ids, long long A, int E, long l
 }
 
 // Routing and permutation in one launch, for given router logits and at most
-// kFusedMax assignments (the decode regime: a few hundred to a thousand tokens).
+// kFusedMax assignments (the decode regime: up to several hundred tokens).
 // "How AI chips support MoE", chapter 4, sections 4.2-4.3 (softmax, top-K) and
 // "Operators & compilers: MoE routing and sparse kernels", section 3 (count, prefix sum,
 // scatter): the steps are those of the router and of the cluster permute above, run by one
-// cluster of C <= 8 CTAs of 8 warps without a round trip of the ids through global memory.
+// cluster of C <= 8 CTAs of 8 or 32 warps without a round trip of the ids through global
+// memory.
 // CTA c owns the tokens [c * tpc, (c + 1) * tpc) and so the assignments
 // [c * tpc * K, (c + 1) * tpc * K). Routing: one warp per token, each lane holding up to 8
 // logits (e = lane + 32 j), K rounds of a warp arg-max under (value descending, id
@@ -516,17 +517,18 @@ moe_status launch_cluster_permute(const int32_t* ids, long long A, int E, long l
 // E; the ids also go to shared memory. Permutation: each warp owns ITERS x 32 of the CTA's
 // assignments, and the histogram, cluster exchange of counts, scan and scatter follow the
 // cluster permute exactly.
-constexpr int kFusedWarps = 8;
-constexpr long long kFusedMax = (long long)kClusterMaxCtas * kFusedWarps * 32 * 4;  // 8192
+constexpr long long kFusedMax = 4096;  // assignments (above, the two launches were faster)
+constexpr int kFusedTpw = 4;           // tokens a warp routes
 
-template <int ITERS>
-__global__ void __launch_bounds__(kFusedWarps * 32) route_permute_kernel(
+template <int WARPS, int ITERS>
+__global__ void __launch_bounds__(WARPS * 32) route_permute_kernel(
     const float* __restrict__ logits_in, float* __restrict__ logits_out, int T, int E, int K,
     int renorm, int tpc, long long cap, int C, int32_t* __restrict__ topk_ids,
     float* __restrict__ topk_w, int32_t* __restrict__ counts, int32_t* __restrict__ offsets,
     int32_t* __restrict__ assign_to_perm, int32_t* __restrict__ perm_to_assign) {
-  constexpr int WARPS = kFusedWarps, NT = WARPS * 32;
+  constexpr int NT = WARPS * 32;
   constexpr int CHUNK = NT * ITERS;  // assignments a CTA can own
+  static_assert(NT >= kMaxE, "one thread per expert in the scan");
   __shared__ int rows[WARPS][kMaxE];
   __shared__ int ctot[kMaxE];
   __shared__ int cbase[kMaxE];
@@ -544,14 +546,29 @@ __global__ void __launch_bounds__(kFusedWarps * 32) route_permute_kernel(
   pdl_trigger();
 
   // ---------------------------------------------------------------- routing
-  for (int r = warp; r < ntok; r += WARPS) {
+  // a warp routes the tokens warp, warp + WARPS, ... (at most kFusedTpw); all their logits
+  // are loaded before the first is ranked
+  float lv[kFusedTpw][8];
+#pragma unroll
+  for (int i = 0; i < kFusedTpw; ++i) {
+    const int r = warp + i * WARPS;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const int e = lane + 32 * j;
+      lv[i][j] = (r < ntok && e < E) ? logits_in[(size_t)(t0 + r) * E + e] : -INFINITY;
+    }
+  }
+#pragma unroll
+  for (int i = 0; i < kFusedTpw; ++i) {
+    const int r = warp + i * WARPS;
+    if (r >= ntok) break;  // warp-uniform
     const int t = t0 + r;
     float v[8];
     bool taken[8];
 #pragma unroll
     for (int j = 0; j < 8; ++j) {
       const int e = lane + 32 * j;
-      v[j] = (e < E) ? logits_in[(size_t)t * E + e] : -INFINITY;
+      v[j] = lv[i][j];
       taken[j] = (e >= E);
       if (logits_out != nullptr && e < E) logits_out[(size_t)t * E + e] = v[j];
     }
@@ -835,26 +852,32 @@ moe_status launch_gather_rows(const moe_shape& s, const void* x, const int32_t* 
 }
 
 namespace {
-// CTAs of the fused kernel: about 32 tokens (4 a warp) per CTA, at most 8 CTAs; false if a
-// CTA would own more than 4 x 32 assignments per warp
-bool fused_grid(const moe_shape& s, int* C_out, int* tpc_out, int* iters_out) {
+// CTAs of the fused kernel: about 32 tokens per CTA up to 8 CTAs; 8 warps per CTA, or 32
+// when a CTA owns more than 32 tokens (routing runs one token per warp at a time); false if
+// a warp would own more assignments than the instantiated shapes hold (4 x 32 with 8 warps,
+// 2 x 32 with 32)
+bool fused_grid(const moe_shape& s, int* C_out, int* tpc_out, int* warps_out, int* iters_out) {
   int C = (s.T + 31) / 32;
   if (C > kClusterMaxCtas) C = kClusterMaxCtas;
   if (C < 1) C = 1;
   const int tpc = (s.T + C - 1) / C;
+  const int warps = tpc > 32 ? 32 : 8;
+  if (tpc > warps * kFusedTpw) return false;
   const long long per = (long long)tpc * s.K;  // assignments per CTA
-  if (per > (long long)kFusedWarps * 32 * 4) return false;
+  const long long lanes = (long long)warps * 32;
+  if (per > lanes * (warps == 32 ? 2 : 4)) return false;  // the instantiated shapes
   *C_out = C;
   *tpc_out = tpc;
-  *iters_out = per <= kFusedWarps * 32 ? 1 : per <= kFusedWarps * 64 ? 2 : 4;
+  *warps_out = warps;
+  *iters_out = per <= lanes ? 1 : per <= 2 * lanes ? 2 : 4;
   return true;
 }
 }  // namespace
 
 bool route_permute_fusable(const moe_shape& s, const float* logits_in) {
-  int C, tpc, iters;
+  int C, tpc, warps, iters;
   return logits_in != nullptr && s.T > 0 && s.E <= kMaxE && s.K <= 32 &&
-         (long long)s.T * s.K <= kFusedMax && fused_grid(s, &C, &tpc, &iters);
+         (long long)s.T * s.K <= kFusedMax && fused_grid(s, &C, &tpc, &warps, &iters);
 }
 
 moe_status launch_route_permute(const moe_shape& s, const float* logits_in, float* logits_out,
@@ -864,17 +887,22 @@ moe_status launch_route_permute(const moe_shape& s, const float* logits_in, floa
       (s.capacity_factor > 0.f)
           ? (long long)ceil((double)s.capacity_factor * (double)s.T * (double)s.K / (double)s.E)
           : -1;
-  int C, tpc, iters;
-  if (!fused_grid(s, &C, &tpc, &iters)) return MOE_ERR_UNSUPPORTED;
+  int C, tpc, warps, iters;
+  if (!fused_grid(s, &C, &tpc, &warps, &iters)) return MOE_ERR_UNSUPPORTED;
   launch_begin(K_ROUTE_PERMUTE, st);
-  auto go = [&](auto kern) {
-    launch_kernel(kern, dim3((unsigned)C), dim3(kFusedWarps * 32), 0, st, (unsigned)C, logits_in,
+  auto go = [&](auto kern, int nwarps) {
+    launch_kernel(kern, dim3((unsigned)C), dim3(nwarps * 32), 0, st, (unsigned)C, logits_in,
                   logits_out, s.T, s.E, s.K, s.renormalize, tpc, cap, C, ids, w, counts, offsets,
                   a2p, p2a);
   };
-  if (iters == 1) go(route_permute_kernel<1>);
-  else if (iters == 2) go(route_permute_kernel<2>);
-  else go(route_permute_kernel<4>);
+  if (warps == 8) {
+    if (iters == 1) go(route_permute_kernel<8, 1>, 8);
+    else if (iters == 2) go(route_permute_kernel<8, 2>, 8);
+    else go(route_permute_kernel<8, 4>, 8);
+  } else {
+    if (iters == 1) go(route_permute_kernel<32, 1>, 32);
+    else go(route_permute_kernel<32, 2>, 32);
+  }
   return launch_end(K_ROUTE_PERMUTE, st);
 }
 
