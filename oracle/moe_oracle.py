@@ -37,7 +37,11 @@ Readings where the pages are silent (each also listed in the design notes):
     assignments in token order and drops the rest;
   * order inside an expert: ascending token id (the section 2.3 example of
     [P2] shows it); dropped slots contribute 0 and are not re-renormalised;
-  * SwiGLU(g, u) = g / (1 + exp(-g)) * u with g from W_gate, u from W_up.
+  * SwiGLU(g, u) = g / (1 + exp(-g)) * u with g from W_gate, u from W_up;
+  * tile-aware token rounding ([P5] 6.5 names it without a rule): an expert
+    with c >= R routed assignments keeps R * floor(c / R) of them, those with
+    the largest router logit for that expert, among equal logits the earlier
+    token; experts with c < R keep all; nothing is added (rounding down only).
 """
 from __future__ import annotations
 
@@ -118,13 +122,43 @@ def capacity(capacity_factor: float, T: int, K: int, E: int) -> Optional[int]:
     return int(math.ceil(cf * T * K / E))
 
 
-def permute(topk_ids_, E: int, C: Optional[int] = None):
+def tile_round_keep(topk_ids_, logits_f32, E: int, R: int) -> np.ndarray:
+    """[P5] 6.5: routing that takes the GEMM's M tile into account, so that each
+    expert's row count fits whole tiles. Reading (the pages give no rule):
+    expert e with c_e >= R routed assignments keeps R * floor(c_e / R) of them,
+    the ones whose router logit for e is largest; among equal logits the
+    earlier token is kept and the later one dropped; an expert with c_e < R
+    keeps all of its assignments. Nothing is added.
+    Returns keep[T, K] (bool): False marks a dropped assignment."""
+    ids = np.asarray(topk_ids_, dtype=np.int64)
+    lg = np.asarray(logits_f32, dtype=np.float32)
+    T, K = ids.shape
+    keep = np.ones((T, K), dtype=bool)
+    if R <= 1:
+        return keep
+    for e in range(E):
+        tok, slot = np.nonzero(ids == e)  # ascending token
+        c = tok.size
+        if c < R or c % R == 0:
+            continue
+        n_drop = c % R
+        score = lg[tok, e].astype(F64)
+        # ascending by (score, -token): the first n_drop are the weakest
+        order = np.lexsort((-tok, score))
+        drop = order[:n_drop]
+        keep[tok[drop], slot[drop]] = False
+    return keep
+
+
+def permute(topk_ids_, E: int, C: Optional[int] = None, keep=None):
     """[P1] 3 (counting + prefix sum), [P2] 2.3 (sort tasks by (expert, token)),
     [P5] 11 (expert-major metadata).
 
     Flat assignment a = t*K + k. For each expert e, its assignments in
     ascending a (= ascending token t, since one token picks an expert once);
     the first C are kept, the rest dropped.
+    ``keep`` (optional, [T, K] or [T*K] bool) removes assignments first (token
+    rounding); they count in ``counts`` and are dropped like capacity overflow.
       counts[e]          raw number of assignments to e (sums to T*K)
       offsets[E+1]       exclusive scan of kept counts min(counts, C)
       perm_to_assign[p]  expert-major slot -> a   (first offsets[E] valid, rest -1)
@@ -134,15 +168,18 @@ def permute(topk_ids_, E: int, C: Optional[int] = None):
     A = ids.size
     if A and (ids.min() < 0 or ids.max() >= E):
         raise ValueError("expert id out of range")
+    keep_mask = None if keep is None else np.asarray(keep, dtype=bool).reshape(-1)
     counts = np.zeros(E, dtype=np.int64)
     kept = np.zeros(E, dtype=np.int64)
     members = []
     for e in range(E):
         a_e = np.nonzero(ids == e)[0]  # ascending flat index
         counts[e] = a_e.size
-        keep = a_e if C is None else a_e[:C]
-        kept[e] = keep.size
-        members.append(keep)
+        if keep_mask is not None:  # assignments removed by token rounding
+            a_e = a_e[keep_mask[a_e]]
+        kept_e = a_e if C is None else a_e[:C]
+        kept[e] = kept_e.size
+        members.append(kept_e)
     offsets = np.zeros(E + 1, dtype=np.int64)
     for e in range(E):
         offsets[e + 1] = offsets[e] + kept[e]
@@ -233,17 +270,23 @@ def combine(y_perm, assign_to_perm, topk_w, T: int, K: int) -> np.ndarray:
 
 # --------------------------------------------------------------------------- layer
 def forward(x, w_r, w_gate, w_up, w_down, K: int, capacity_factor: float = 0.0,
-            bias=None, logits=None, renormalize: bool = True):
+            bias=None, logits=None, renormalize: bool = True, tile_round: int = 0):
     """The whole layer forward ([P5] section 3 pipeline), every intermediate kept.
 
     ``logits`` (fp32 [T, E]) replaces x . W_r + bias when given: this is how
-    ids/counts/permutation parity is checked on identical logits."""
+    ids/counts/permutation parity is checked on identical logits. ``tile_round``
+    = R > 0 applies token rounding to R-row tiles (see tile_round_keep)."""
     T = x.shape[0]
     lg = router_logits(x, w_r, bias) if logits is None else np.asarray(logits, np.float32)
     E = lg.shape[1]
     ids, w = route(lg, K, renormalize)
     C = capacity(capacity_factor, T, K, E)
-    counts, offsets, a2p, p2a = permute(ids, E, C)
+    keep = None
+    if tile_round > 0:
+        if C is not None:
+            raise ValueError("token rounding and a capacity limit are exclusive")
+        keep = tile_round_keep(ids, lg, E, tile_round)
+    counts, offsets, a2p, p2a = permute(ids, E, C, keep)
     a_act, y_perm = grouped_ffn(x, p2a, offsets, K, w_gate, w_up, w_down)
     out = combine(y_perm, a2p, w, T, K)
     return dict(logits=lg, topk_ids=ids, topk_w=w, counts=counts, offsets=offsets,

@@ -359,8 +359,8 @@ def test_planted_mistakes_are_caught(monkeypatch):
 
     real_permute = orc.permute
 
-    def permute_off_by_one(ids, E_, C_):
-        c, o, a2p, p2a = real_permute(ids, E_, C_)
+    def permute_off_by_one(ids, E_, C_, keep=None):
+        c, o, a2p, p2a = real_permute(ids, E_, C_, keep)
         nk = o[-1]
         p2a = p2a.copy()
         p2a[:nk] = np.roll(p2a[:nk], 1)
@@ -375,3 +375,131 @@ def test_planted_mistakes_are_caught(monkeypatch):
     ref = (torch.nn.functional.silu(torch.from_numpy(g)) * torch.from_numpy(u)).numpy()
     assert not np.allclose(wrong, ref)
     assert np.allclose(orc.swiglu(g, u), ref)
+
+
+# ------------------------------------------------------------------ token rounding
+# SonicMoE explainer (gitcode.csdn.net), section 6.5 names tile-aware token rounding
+# without a rule; the rule pinned here is this build's reading: an expert with c >= R
+# routed assignments keeps R * floor(c / R) of them, the ones with the largest logit for
+# that expert (equal logits: the earlier token stays), experts with c < R keep all.
+def _hand_logits():
+    # K = 1: t0 t1 t3 t5 t6 pick e0 (scores 3 2 2 5 2), t2 t4 pick e1 (4, 1), t7 picks e2
+    lg = np.zeros((8, 3), np.float32)
+    for t, (e, v) in enumerate([(0, 3), (0, 2), (1, 4), (0, 2), (1, 1), (0, 5), (0, 2), (2, 7)]):
+        lg[t, e] = v
+    return lg
+
+
+@pytest.mark.parametrize("R,dropped_tokens", [
+    (1, []),        # nothing to round
+    (2, [6]),       # e0: 5 -> 4; the weakest logit 2 is held by t1, t3, t6: the latest goes
+    (3, [3, 6]),    # e0: 5 -> 3: t6 then t3; e1 (2 < 3) and e2 keep theirs
+    (4, [6]),       # e0: 5 -> 4
+    (8, []),        # every expert below R
+])
+def test_token_rounding_hand_worked(R, dropped_tokens):
+    lg = _hand_logits()
+    ids, _ = orc.route(lg, 1)
+    np.testing.assert_array_equal(ids[:, 0], [0, 0, 1, 0, 1, 0, 0, 2])
+    keep = orc.tile_round_keep(ids, lg, 3, R)
+    assert sorted(np.nonzero(~keep[:, 0])[0].tolist()) == dropped_tokens
+
+
+def test_token_rounding_hand_worked_two_slots():
+    # K = 2; t3 ties e0 and e2 at 2 (both picked, e0 first). e0 gets t0(3) t1(1) t3(2):
+    # 3 -> 2 drops t1's slot 1; e1 gets t0(2) t2(4): kept; e2 gets t1(5) t2(1) t3(2):
+    # 3 -> 2 drops t2's slot 1.
+    lg = np.array([[3, 2, 0], [1, 0, 5], [0, 4, 1], [2, 0, 2]], np.float32)
+    ids, _ = orc.route(lg, 2)
+    np.testing.assert_array_equal(ids, [[0, 1], [2, 0], [1, 2], [0, 2]])
+    keep = orc.tile_round_keep(ids, lg, 3, 2)
+    np.testing.assert_array_equal(keep, [[True, True], [True, False], [True, False],
+                                         [True, True]])
+
+
+def _rounding_brute_force(ids, lg, E, R):
+    """Every subset of the right size whose kept members all outrank its dropped members by
+    (logit, then earlier token); exactly one exists per expert."""
+    import itertools
+    T, K = ids.shape
+    keep = np.ones((T, K), bool)
+    for e in range(E):
+        members = [(t, k) for t in range(T) for k in range(K) if ids[t, k] == e]
+        c = len(members)
+        if c < R:
+            continue
+        r = (c // R) * R
+        found = []
+        for kept in itertools.combinations(range(c), r):
+            dropped = [i for i in range(c) if i not in kept]
+
+            def outranks(i, j):
+                (ti, ki), (tj, kj) = members[i], members[j]
+                si, sj = lg[ti, e], lg[tj, e]
+                return si > sj or (si == sj and ti < tj)
+            if all(outranks(i, j) for i in kept for j in dropped):
+                found.append(dropped)
+        assert len(found) == 1
+        for i in found[0]:
+            keep[members[i]] = False
+    return keep
+
+
+@pytest.mark.parametrize("seed", range(6))
+def test_token_rounding_matches_brute_force(seed):
+    rng = np.random.default_rng(seed)
+    T, E, K, R = 9, 3, 2, 2 + seed % 3
+    lg = rng.integers(-2, 3, size=(T, E)).astype(np.float32)  # many ties
+    ids, _ = orc.route(lg, K)
+    np.testing.assert_array_equal(orc.tile_round_keep(ids, lg, E, R),
+                                  _rounding_brute_force(ids, lg, E, R))
+
+
+@pytest.mark.parametrize("seed", range(4))
+def test_token_rounding_invariants(seed):
+    rng = np.random.default_rng(100 + seed)
+    T, E, K, R = 500, 8, 2, 16
+    lg = rng.standard_normal((T, E)).astype(np.float32)
+    ids, _ = orc.route(lg, K)
+    keep = orc.tile_round_keep(ids, lg, E, R)
+    counts, offsets, a2p, p2a = orc.permute(ids, E, None, keep)
+    assert counts.sum() == T * K
+    kept = np.diff(offsets)
+    for e in range(E):
+        c = int(counts[e])
+        assert kept[e] == (c if c < R else (c // R) * R)
+        mask = ids == e
+        ks, ds = lg[:, e][(mask & keep).any(1)], lg[:, e][(mask & ~keep).any(1)]
+        if ds.size:
+            assert ks.min() >= ds.max()
+    assert np.all(a2p.reshape(T, K)[~keep] == -1)
+    assert np.all(a2p.reshape(T, K)[keep] >= 0)
+
+
+def test_token_rounding_by_one_changes_nothing_and_excludes_capacity():
+    rng = np.random.default_rng(3)
+    E, K, T, d, n = 4, 2, 30, 6, 4
+    x, w_r = rng.standard_normal((T, d)), rng.standard_normal((d, E))
+    wg, wu = rng.standard_normal((E, d, n)), rng.standard_normal((E, d, n))
+    wd = rng.standard_normal((E, n, d))
+    a = orc.forward(x, w_r, wg, wu, wd, K=K)
+    b = orc.forward(x, w_r, wg, wu, wd, K=K, tile_round=1)
+    np.testing.assert_array_equal(a["assign_to_perm"], b["assign_to_perm"])
+    np.testing.assert_array_equal(a["out"], b["out"])
+    with pytest.raises(ValueError):
+        orc.forward(x, w_r, wg, wu, wd, K=K, capacity_factor=1.0, tile_round=4)
+
+
+def test_token_rounding_planted_mistake_is_caught(monkeypatch):
+    lg = _hand_logits()
+    E, K, R = 3, 1, 3
+    ids, _ = orc.route(lg, K)
+    real = np.lexsort
+
+    def keeps_the_weakest(keys):  # a reversed sort inside the rounding
+        return real(keys)[::-1]
+
+    monkeypatch.setattr(orc.np, "lexsort", keeps_the_weakest)
+    wrong = orc.tile_round_keep(ids, lg, E, R)
+    monkeypatch.undo()
+    assert not np.array_equal(wrong, _rounding_brute_force(ids, lg, E, R))
