@@ -63,19 +63,29 @@ typedef enum { MOE_F32 = 0, MOE_BF16 = 1 } moe_dtype;
  * restricted to the K selected experts (they sum to 1); 0: plain softmax
  * over all E experts, read at the selected ones. Limits: 1 <= K <= E <= 256,
  * K <= 32, T >= 0, T * K < 2^31, d % 64 == 0 (router tiles, TMA boxes);
- * n % 64 == 0 for MOE_BF16 and n % 16 == 0 for MOE_F32. */
+ * n % 64 == 0 for MOE_BF16 and n % 16 == 0 for MOE_F32.
+ * tile_round = R > 0: tile-aware token rounding (SonicMoE explainer, section 6.5, names
+ * it without a rule; this is the library's reading): an expert with c >= R routed
+ * assignments keeps R * floor(c / R) of them, the ones with the largest router logit for
+ * that expert (equal logits: the earlier token stays), and drops the rest like capacity
+ * overflow (assign_to_perm = -1, no re-normalisation); an expert with c < R keeps all.
+ * Nothing is added. Needs the router logits, so it applies in moe_forward and
+ * moe_dispatch (moe_permute returns MOE_ERR_UNSUPPORTED); exclusive with
+ * capacity_factor > 0. 0 = off. */
 typedef struct {
   int32_t T, d, E, K, n;
   float capacity_factor;
   int32_t renormalize;
-  int32_t dtype; /* moe_dtype */
+  int32_t dtype;      /* moe_dtype */
+  int32_t tile_round; /* 0, or the row tile R that each expert's kept count is rounded to */
 } moe_shape;
 
 /* ----------------------------------------------------------------------------
  * Workspace sizes (bytes). The caller passes a device buffer at least this big
  * (256-byte aligned) to moe_permute / moe_forward. Returns 0 on a bad shape.
  * moe_permute_workspace_size: scratch of the histogram / scan / scatter
- *   kernels (per-chunk expert counts and rank bases).
+ *   kernels (per-chunk expert counts and rank bases), plus, when tile_round > 0,
+ *   the rounded copy of the ids and the kept counts (used by moe_dispatch).
  * moe_forward_workspace_size: everything moe_forward keeps between kernels:
  *   logits, top-K ids and weights, counts, offsets, both permutation indices,
  *   the permute scratch, a_act[T*K, n] and y_perm[T*K, d].
@@ -245,7 +255,7 @@ moe_status moe_forward(const moe_shape* shape, const void* x, const void* w_r, c
 /* Byte offsets of the intermediates inside moe_forward's workspace. */
 typedef struct {
   size_t logits, topk_ids, topk_w, counts, offsets, assign_to_perm, perm_to_assign,
-      permute_scratch, a_act, y_perm, total;
+      permute_scratch, a_act, y_perm, round_ids, round_counts, total;
 } moe_workspace_layout;
 moe_status moe_forward_workspace_layout(const moe_shape* shape, moe_workspace_layout* layout);
 

@@ -120,3 +120,22 @@ def test_dispatch_argument_checks_on_host(lib):
     r = lib.moe_dispatch(ctypes.byref(bad), None, None, None, dummy, None, dummy, dummy, dummy,
                          dummy, dummy, dummy, None, None, 0, None)
     assert r == 1
+
+
+def test_token_rounding_shape_checks(lib):
+    ok = tdr.make_shape(4096, 128, 8, 2, 128, 0.0, True, tile_round=128)
+    plain = tdr.make_shape(4096, 128, 8, 2, 128)
+    assert lib.moe_forward_workspace_size(ctypes.byref(ok)) > \
+        lib.moe_forward_workspace_size(ctypes.byref(plain))
+    assert lib.moe_permute_workspace_size(ctypes.byref(ok)) >= \
+        lib.moe_permute_workspace_size(ctypes.byref(plain)) + 4096 * 2 * 4
+    neg = tdr.make_shape(16, 128, 8, 2, 128, 0.0, True, tile_round=-1)
+    both = tdr.make_shape(16, 128, 8, 2, 128, 1.0, True, tile_round=16)
+    for s in (neg, both):
+        assert lib.moe_forward_workspace_size(ctypes.byref(s)) == 0
+        assert lib.moe_forward(ctypes.byref(s), None, None, None, None, None, None, None, None,
+                               None, 0, None) == 1
+    dummy = ctypes.c_void_p(256)
+    r = lib.moe_permute(ctypes.byref(ok), dummy, dummy, dummy, dummy, dummy, None, None, dummy,
+                        1 << 30, None)
+    assert r == 2  # rounding needs the logits: not available to moe_permute

@@ -415,6 +415,83 @@ def test_forward_full_size_workloads(cuda_lib, ffn_variant, name):
                       f"{name} out")
 
 
+# ------------------------------------------------------------------ token rounding
+def _rounded_reference(lg, ids_ref, E, R):
+    keep = orc.tile_round_keep(ids_ref, lg, E, R)
+    return keep, orc.permute(ids_ref, E, None, keep)
+
+
+@pytest.mark.parametrize("T,E,K,R,ties", [
+    (1000, 8, 2, 64, False),
+    (4096, 8, 2, 128, False),      # the Mixtral-like routing shape
+    (3001, 32, 4, 128, True),      # integer logits: equal scores split by token order
+    (300, 4, 1, 128, False),       # experts below R keep everything
+    (16384, 128, 8, 128, False),   # three-kernel permutation
+    (500, 16, 3, 1, False),        # R = 1 changes nothing
+])
+def test_dispatch_token_rounding_matches_oracle(cuda_lib, T, E, K, R, ties):
+    tdr = cuda_lib
+    rng = np.random.default_rng(T + E + R)
+    if ties:
+        lg = rng.integers(-3, 4, size=(T, E)).astype(np.float32)
+    else:
+        lg = rng.standard_normal((T, E)).astype(np.float32)
+    s = tdr.make_shape(T, 64, E, K, 64, 0.0, True, torch.bfloat16, tile_round=R)
+    out = tdr.dispatch(s, logits_in=torch.from_numpy(lg).cuda())
+    ids_ref, w_ref = orc.route(lg, K, True)
+    np.testing.assert_array_equal(out["topk_ids"].cpu().numpy(), ids_ref)
+    keep, (counts, offsets, a2p, p2a) = _rounded_reference(lg, ids_ref, E, R)
+    np.testing.assert_array_equal(out["counts"].cpu().numpy(), counts)
+    np.testing.assert_array_equal(out["offsets"].cpu().numpy(), offsets)
+    np.testing.assert_array_equal(out["assign_to_perm"].cpu().numpy(), a2p)
+    nk = int(offsets[-1])
+    np.testing.assert_array_equal(out["perm_to_assign"].cpu().numpy()[:nk], p2a[:nk])
+    kept = np.diff(offsets)
+    assert all(k % R == 0 or c < R for k, c in zip(kept, counts))
+    if R > 1 and T >= 1000:
+        assert (~keep).any()  # the case really rounds
+    assert_status_ok(tdr)
+
+
+def test_forward_token_rounding_full_size(cuda_lib):
+    tdr = cuda_lib
+    cfg = mi.CONFIGS["mixtral_bf16"]
+    inp = inputs_for(cfg)
+    s = tdr.make_shape(cfg.T, cfg.d, cfg.E, cfg.K, cfg.n, 0.0, True, torch.bfloat16,
+                       tile_round=128)
+    out, ws = tdr.forward(s, cuda(inp.x), cuda(inp.w_r), cuda(inp.w_gate), cuda(inp.w_up),
+                          cuda(inp.w_down))
+    torch.cuda.synchronize()
+    assert_status_ok(tdr)
+    v = tdr.workspace_views(s, ws)
+    lg = v["logits"].cpu().numpy()
+    ids_ref, w_ref = check_routing(tdr, v["logits"], v["topk_ids"], v["topk_w"], cfg.K)
+    keep, (counts, offsets, a2p, p2a) = _rounded_reference(lg, ids_ref, cfg.E, 128)
+    np.testing.assert_array_equal(v["counts"].cpu().numpy(), counts)
+    np.testing.assert_array_equal(v["offsets"].cpu().numpy(), offsets)
+    np.testing.assert_array_equal(v["assign_to_perm"].cpu().numpy(), a2p)
+    assert np.all(np.diff(offsets) % 128 == 0) and (~keep).any()
+    rng = np.random.default_rng(11)
+    dropped_tok = np.nonzero((~keep).any(1))[0]
+    tokens = np.unique(np.concatenate([rng.choice(cfg.T, size=12, replace=False),
+                                       dropped_tok[:4]]))
+    ref_rows = orc.forward_rows(tokens, inp.x, inp.w_gate, inp.w_up, inp.w_down, ids_ref, w_ref,
+                                a2p, cfg.K)
+    assert_bf16_close(out[torch.from_numpy(tokens).cuda()].float().cpu().numpy(), ref_rows,
+                      "rounded forward out")
+
+
+def test_token_rounding_rejected_where_it_cannot_apply(cuda_lib):
+    tdr = cuda_lib
+    s = tdr.make_shape(64, 64, 8, 2, 64, 0.0, True, torch.bfloat16, tile_round=16)
+    ids = torch.zeros(64, 2, dtype=torch.int32, device="cuda")
+    with pytest.raises(tdr.MoEError):
+        tdr.permute(s, ids)  # no logits: unsupported
+    bad = tdr.make_shape(64, 64, 8, 2, 64, 1.0, True, torch.bfloat16, tile_round=16)
+    with pytest.raises(tdr.MoEError):
+        tdr.dispatch(bad, logits_in=torch.zeros(64, 8, device="cuda"))
+
+
 @pytest.mark.parametrize("T", mi.DISPATCH_COMBINE_T)
 def test_dispatch_combine_identity_experts(cuda_lib, T):
     """route (given logits) -> permute with x_perm -> combine(y_perm = x_perm) returns x."""

@@ -33,13 +33,14 @@ class moe_shape(ctypes.Structure):
     _fields_ = [("T", ctypes.c_int32), ("d", ctypes.c_int32), ("E", ctypes.c_int32),
                 ("K", ctypes.c_int32), ("n", ctypes.c_int32),
                 ("capacity_factor", ctypes.c_float), ("renormalize", ctypes.c_int32),
-                ("dtype", ctypes.c_int32)]
+                ("dtype", ctypes.c_int32), ("tile_round", ctypes.c_int32)]
 
 
 class moe_workspace_layout(ctypes.Structure):
     _fields_ = [(f, ctypes.c_size_t) for f in (
         "logits", "topk_ids", "topk_w", "counts", "offsets", "assign_to_perm",
-        "perm_to_assign", "permute_scratch", "a_act", "y_perm", "total")]
+        "perm_to_assign", "permute_scratch", "a_act", "y_perm", "round_ids", "round_counts",
+        "total")]
 
 
 _P = ctypes.c_void_p
@@ -96,9 +97,11 @@ def _check(code: int, where: str) -> None:
 
 
 def make_shape(T: int, d: int, E: int, K: int, n: int = 0, capacity_factor: float = 0.0,
-               renormalize: bool = True, dtype=torch.bfloat16) -> moe_shape:
+               renormalize: bool = True, dtype=torch.bfloat16, tile_round: int = 0) -> moe_shape:
+    """tile_round = R > 0 rounds each expert's kept count down to whole R-row tiles."""
     dt = MOE_BF16 if dtype == torch.bfloat16 else MOE_F32
-    return moe_shape(T, d, E, K, n, float(capacity_factor), 1 if renormalize else 0, dt)
+    return moe_shape(T, d, E, K, n, float(capacity_factor), 1 if renormalize else 0, dt,
+                     int(tile_round))
 
 
 def _ptr(t: Optional[torch.Tensor]):
@@ -210,6 +213,8 @@ def dispatch(shape: moe_shape, x=None, w_r=None, bias=None, logits_in=None, logi
         _dev(bias, "bias", torch.float32, (E,))
     if logits_out is not None:
         _dev(logits_out, "logits_out", torch.float32, (T, E))
+    elif logits_in is None and shape.tile_round > 0:  # rounding reads the router logits
+        logits_out = torch.empty(T, E, dtype=torch.float32, device=dev)
     o = dict(out or {})
 
     def get(name, shape_, dtype):

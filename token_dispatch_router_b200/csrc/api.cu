@@ -39,6 +39,10 @@ moe_status launch_route_permute(const moe_shape& s, const float* logits_in, floa
                                 int32_t* a2p, int32_t* p2a, cudaStream_t st);
 moe_status launch_gather_rows(const moe_shape& s, const void* x, const int32_t* p2a,
                               const int32_t* offsets, void* x_perm, cudaStream_t st);
+moe_status launch_permute_rounded(const moe_shape& s, const int32_t* ids, const float* logits,
+                                  int32_t* counts, int32_t* offsets, int32_t* a2p, int32_t* p2a,
+                                  const void* x, void* x_perm, void* scratch, int32_t* round_ids,
+                                  int32_t* round_counts, cudaStream_t st);
 
 // ------------------------------------------------------------------ device state
 __device__ unsigned int g_device_status;
@@ -83,7 +87,7 @@ const char* kKernelNames[K_COUNT] = {
     "route",        "hist",          "scan",           "scatter",     "gather_rows", "gateup_tc",
     "down_tc",      "gateup_simt",   "down_simt",      "combine",     "selftest_timeout",
     "route_tc",     "permute_small", "gateup_tc2",   "down_tc2",
-    "permute_cluster", "route_permute"};
+    "permute_cluster", "route_permute", "tile_round"};
 
 struct ProfRec {
   int kid;
@@ -139,6 +143,8 @@ moe_status check_shape(const moe_shape* s, bool need_d, bool need_ffn) {
   if (s->E > 256 || s->K > 32) return MOE_ERR_UNSUPPORTED;
   if ((long long)s->T * s->K > 0x7fffffffLL) return MOE_ERR_UNSUPPORTED;
   if (isnan(s->capacity_factor)) return MOE_ERR_INVALID_ARG;
+  if (s->tile_round < 0 || (s->tile_round > 0 && s->capacity_factor > 0.f))
+    return MOE_ERR_INVALID_ARG;  // token rounding and a capacity limit are exclusive
   if (need_d) {
     if (s->d < 64 || s->d % 64 != 0) return MOE_ERR_INVALID_ARG;
   }
@@ -173,6 +179,10 @@ bool layout_of(const moe_shape& s, moe_workspace_layout* L) {
   o = align256(o + A * (size_t)s.n * eb);
   L->y_perm = o;
   o = align256(o + A * (size_t)s.d * eb);
+  L->round_ids = o;
+  if (s.tile_round > 0) o = align256(o + A * 4);
+  L->round_counts = o;
+  if (s.tile_round > 0) o = align256(o + E * 4);
   L->total = o;
   return true;
 }
@@ -200,7 +210,10 @@ extern "C" {
 
 size_t moe_permute_workspace_size(const moe_shape* s) {
   if (check_shape(s, false, false) != MOE_OK) return 0;
-  return align256(permute_scratch_bytes(*s)) + 256;
+  size_t bytes = align256(permute_scratch_bytes(*s));
+  if (s->tile_round > 0)  // the rounded ids and the kept counts (moe_dispatch)
+    bytes += align256((size_t)s->T * s->K * 4) + align256((size_t)s->E * 4);
+  return bytes + 256;
 }
 
 size_t moe_forward_workspace_size(const moe_shape* s) {
@@ -240,6 +253,7 @@ moe_status moe_permute(const moe_shape* s, const int32_t* topk_ids, int32_t* cou
   const bool gather = (x != nullptr && x_perm != nullptr);
   moe_status r = check_shape(s, gather, false);
   if (r != MOE_OK) return r;
+  if (s->tile_round > 0) return MOE_ERR_UNSUPPORTED;  // rounding needs the router logits
   if (s->T == 0) {  // no assignments: only counts and offsets (all zero) are written
     if (counts == nullptr || offsets == nullptr) return MOE_ERR_INVALID_ARG;
     const cudaStream_t st = (cudaStream_t)stream;
@@ -265,6 +279,7 @@ moe_status moe_permute_static(const moe_shape* s, const int32_t* topk_ids, int32
   const bool gather = (x != nullptr && x_perm != nullptr);
   moe_status r = check_shape(s, gather, false);
   if (r != MOE_OK) return r;
+  if (s->tile_round > 0) return MOE_ERR_UNSUPPORTED;  // rounding needs the router logits
   if (topk_ids == nullptr || counts == nullptr || offsets == nullptr || assign_to_perm == nullptr ||
       perm_to_assign == nullptr)
     return MOE_ERR_INVALID_ARG;
@@ -295,6 +310,22 @@ moe_status moe_dispatch(const moe_shape* s, const void* x, const void* w_r, cons
   if (!topk_ids || !topk_w || !counts || !offsets || !assign_to_perm || !perm_to_assign)
     return MOE_ERR_INVALID_ARG;
   if (gather && (x == nullptr || !aligned16(x) || !aligned16(x_perm))) return MOE_ERR_INVALID_ARG;
+  if (s->tile_round > 0) {  // route, then the rounded permutation on the logits it saw
+    const float* lg = logits_in != nullptr ? logits_in : logits_out;
+    if (lg == nullptr) return MOE_ERR_INVALID_ARG;  // rounding reads the logits
+    const size_t sb = align256(permute_scratch_bytes(*s));
+    const size_t need = sb + align256((size_t)s->T * s->K * 4) + align256((size_t)s->E * 4);
+    if (workspace == nullptr || ws_bytes < need || ((uintptr_t)workspace & 255) != 0)
+      return MOE_ERR_WORKSPACE;
+    if ((r = moe_route(s, x, w_r, bias, logits_in, logits_out, topk_ids, topk_w, stream)) != MOE_OK)
+      return r;
+    uint8_t* ws = (uint8_t*)workspace;
+    return launch_permute_rounded(*s, topk_ids, lg, counts, offsets, assign_to_perm,
+                                  perm_to_assign, gather ? x : nullptr, x_perm, ws,
+                                  (int32_t*)(ws + sb),
+                                  (int32_t*)(ws + sb + align256((size_t)s->T * s->K * 4)),
+                                  (cudaStream_t)stream);
+  }
   if (!route_permute_fusable(*s, logits_in)) {
     if ((r = moe_route(s, x, w_r, bias, logits_in, logits_out, topk_ids, topk_w, stream)) != MOE_OK)
       return r;
@@ -360,7 +391,13 @@ moe_status moe_forward(const moe_shape* s, const void* x, const void* w_r, const
   int32_t* offsets = (int32_t*)(ws + L.offsets);
   int32_t* a2p = (int32_t*)(ws + L.assign_to_perm);
   int32_t* p2a = (int32_t*)(ws + L.perm_to_assign);
-  if (route_permute_fusable(*s, logits_in)) {
+  if (s->tile_round > 0) {
+    if ((r = moe_route(s, x, w_r, bias, logits_in, logits, ids, w, stream)) != MOE_OK) return r;
+    if ((r = launch_permute_rounded(*s, ids, logits, counts, offsets, a2p, p2a, nullptr, nullptr,
+                                    ws + L.permute_scratch, (int32_t*)(ws + L.round_ids),
+                                    (int32_t*)(ws + L.round_counts), st)) != MOE_OK)
+      return r;
+  } else if (route_permute_fusable(*s, logits_in)) {
     if ((r = launch_route_permute(*s, logits_in, logits, ids, w, counts, offsets, a2p, p2a, st)) !=
         MOE_OK)
       return r;

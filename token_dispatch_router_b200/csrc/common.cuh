@@ -103,6 +103,7 @@ enum KernelId {
   K_DOWN_TC2,
   K_PERMUTE_CLUSTER,
   K_ROUTE_PERMUTE,
+  K_TILE_ROUND,
   K_COUNT
 };
 

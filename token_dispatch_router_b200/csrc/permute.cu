@@ -44,7 +44,7 @@ __device__ __forceinline__ int raw_id(const int32_t* __restrict__ ids, long long
   return a < A ? __ldg(ids + a) : -1;
 }
 __device__ __forceinline__ int checked_id(int id, bool real, int E, unsigned* status) {
-  if (!real) return -1;
+  if (!real || id == -1) return -1;  // -1: no expert (an assignment removed by rounding)
   if (id < 0 || id >= E) {
     report(status, MOE_ERR_DEVICE_INDEX);
     return -1;
@@ -904,6 +904,124 @@ moe_status launch_route_permute(const moe_shape& s, const float* logits_in, floa
     else go(route_permute_kernel<32, 2>, 32);
   }
   return launch_end(K_ROUTE_PERMUTE, st);
+}
+
+// ------------------------------------------------------------------ token rounding
+// Tile-aware token rounding (SonicMoE explainer, section 6.5; the rule is the library's
+// reading): an expert with c >= R routed assignments keeps R * floor(c / R) of them, those
+// with the largest router logit for it (equal logits: the earlier token stays), and drops
+// the m = c mod R weakest. One CTA per expert, after an uncapped permutation (its slots
+// [offsets[e], offsets[e] + c) hold the assignments in token order): each slot's key is
+// (logit as an order-preserving 32-bit integer, +0 for both zeros) << 32 | (2^32 - 1 - t),
+// so ascending keys run from the weakest assignment up and every key is distinct; an
+// 8-pass radix select (8 bits a pass, a 256-bin shared histogram) finds the m-th smallest
+// key, and every slot at or below it marks its assignment -1 in the copy of the ids that
+// the second permutation reads.
+namespace {
+
+__device__ __forceinline__ uint64_t round_key(const int32_t* p2a, const float* logits, int slot,
+                                              int K, int E, int e) {
+  const int a = p2a[slot];
+  const int t = a / K;
+  float v = logits[(size_t)t * E + e];
+  if (v == 0.f) v = 0.f;  // -0 and +0 are one value
+  uint32_t u = __float_as_uint(v);
+  u = (u & 0x80000000u) ? ~u : (u | 0x80000000u);  // ascending order of the floats
+  return ((uint64_t)u << 32) | (uint64_t)(0xffffffffu - (uint32_t)t);
+}
+
+__global__ void __launch_bounds__(256) tile_round_kernel(const int32_t* __restrict__ counts,
+                                                         const int32_t* __restrict__ offsets,
+                                                         const int32_t* __restrict__ p2a,
+                                                         const float* __restrict__ logits,
+                                                         int K, int E, int R,
+                                                         int32_t* __restrict__ round_ids) {
+  __shared__ unsigned hist[256];
+  __shared__ unsigned long long s_pre;
+  __shared__ int s_need;
+  pdl_wait();  // the previous kernel in the stream has completed
+  pdl_trigger();
+  const int e = blockIdx.x, tid = threadIdx.x;
+  const int c = counts[e];
+  if (c < R || c % R == 0) return;  // uniform across the CTA
+  const int off = offsets[e];
+  uint64_t pre = 0;
+  int need = c % R;  // rank of the wanted key among the keys matching `pre` so far
+  for (int d = 7; d >= 0; --d) {
+    const uint64_t hi = d == 7 ? 0ull : (~0ull << (8 * (d + 1)));
+    hist[tid] = 0;
+    __syncthreads();
+    for (int j = tid; j < c; j += 256) {
+      const uint64_t key = round_key(p2a, logits, off + j, K, E, e);
+      if (((key ^ pre) & hi) == 0) atomicAdd(&hist[(key >> (8 * d)) & 255u], 1u);
+    }
+    __syncthreads();
+    if (tid < 32) {  // warp 0: the bin where the running count reaches `need`
+      const int lane = tid;
+      unsigned v[8], ls = 0;
+#pragma unroll
+      for (int q = 0; q < 8; ++q) {
+        v[q] = hist[lane * 8 + q];
+        ls += v[q];
+      }
+      unsigned incl = ls;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const unsigned y = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += y;
+      }
+      const unsigned excl = incl - ls;
+      const unsigned hit = __ballot_sync(0xffffffffu, excl < (unsigned)need && incl >= (unsigned)need);
+      if (lane == __ffs(hit) - 1) {
+        unsigned run = excl;
+        int b = lane * 8 + 7;
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {
+          if (run + v[q] >= (unsigned)need) {
+            b = lane * 8 + q;
+            break;
+          }
+          run += v[q];
+        }
+        s_need = need - (int)run;
+        s_pre = pre | ((uint64_t)b << (8 * d));
+      }
+    }
+    __syncthreads();
+    pre = s_pre;
+    need = s_need;
+    __syncthreads();
+  }
+  // `pre` is the m-th smallest key: drop it and every smaller one
+  for (int j = tid; j < c; j += 256) {
+    const uint64_t key = round_key(p2a, logits, off + j, K, E, e);
+    if (key <= pre) round_ids[p2a[off + j]] = -1;
+  }
+}
+
+}  // namespace
+
+moe_status launch_permute_rounded(const moe_shape& s, const int32_t* ids, const float* logits,
+                                  int32_t* counts, int32_t* offsets, int32_t* a2p, int32_t* p2a,
+                                  const void* x, void* x_perm, void* scratch, int32_t* round_ids,
+                                  int32_t* round_counts, cudaStream_t st) {
+  moe_status r;
+  // 1. uncapped permutation: raw counts, each expert's assignments in token order
+  if ((r = launch_permute(s, ids, counts, offsets, a2p, p2a, nullptr, nullptr, scratch, st)) !=
+      MOE_OK)
+    return r;
+  // 2. the ids again, with the rounded-away assignments set to -1
+  const size_t A = (size_t)s.T * s.K;
+  if (cudaMemcpyAsync(round_ids, ids, A * sizeof(int32_t), cudaMemcpyDeviceToDevice, st) !=
+      cudaSuccess)
+    return MOE_ERR_CUDA;
+  launch_begin(K_TILE_ROUND, st);
+  launch_kernel(tile_round_kernel, dim3((unsigned)s.E), dim3(256), 0, st, 1,
+                (const int32_t*)counts, (const int32_t*)offsets, (const int32_t*)p2a, logits, s.K,
+                s.E, s.tile_round, round_ids);
+  if ((r = launch_end(K_TILE_ROUND, st)) != MOE_OK) return r;
+  // 3. the final permutation of what is kept (its counts are the kept ones: not returned)
+  return launch_permute(s, round_ids, round_counts, offsets, a2p, p2a, x, x_perm, scratch, st);
 }
 
 // ------------------------------------------------------------------ no-allocation variant
