@@ -400,6 +400,55 @@ def decode_dispatch(tdr, world, Ts=(64, 256, 512, 1024)):
                     "iteration, CUDA events, launch gaps included"}
 
 
+def token_rounding_figure(tdr, cfg, x, w_r, wg, wu, wd, bias, world, R=128, rounds=5, per=10):
+    """The layer with tile-aware token rounding (each expert's kept rows rounded down to whole
+    R-row tiles, its weakest assignments dropped) against the plain layer: blocks of `per`
+    steps alternate between the two `rounds` times (the power-capped clock drifts), CUDA
+    events; reports both step times, the kept share of the assignments and the 128-row
+    tile rows the gate/up GEMM computes in each case."""
+    if cfg.capacity_factor > 0:
+        return None
+    dev = x.device
+    dt = x.dtype
+    out = torch.empty(cfg.T, cfg.d, dtype=dt, device=dev)
+    shapes = {"plain": tdr.make_shape(cfg.T, cfg.d, cfg.E, cfg.K, cfg.n, 0.0, True, dt),
+              "rounded": tdr.make_shape(cfg.T, cfg.d, cfg.E, cfg.K, cfg.n, 0.0, True, dt,
+                                        tile_round=R)}
+    wss = {k: torch.empty(tdr.forward_workspace_size(v), dtype=torch.uint8, device=dev)
+           for k, v in shapes.items()}
+    ms = {k: 0.0 for k in shapes}
+    for k in shapes:
+        for _ in range(3):
+            tdr.forward(shapes[k], x, w_r, wg, wu, wd, bias=bias, out=out, workspace=wss[k])
+    torch.cuda.synchronize()
+    for _ in range(rounds):
+        for k in shapes:
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            for _ in range(per):
+                tdr.forward(shapes[k], x, w_r, wg, wu, wd, bias=bias, out=out, workspace=wss[k])
+            e1.record()
+            torch.cuda.synchronize()
+            ms[k] += e0.elapsed_time(e1)
+    if tdr.device_status() != 0:
+        raise RuntimeError("device status set during the token-rounding runs")
+    res = {}
+    for k in shapes:
+        step = max_over_ranks(ms[k] / (rounds * per), world)
+        offs = tdr.workspace_views(shapes[k], wss[k])["offsets"].cpu().numpy()
+        kept = np.diff(offs)
+        res[k] = {"ms_per_step": round(step, 4),
+                  "tokens_per_s": cfg.T * world / (step / 1e3),
+                  "kept_assignments": int(offs[-1]),
+                  "gemm_tile_rows": int(sum(-(-int(c) // 128) * 128 for c in kept))}
+    res["R"] = R
+    res["kept_share"] = round(res["rounded"]["kept_assignments"] / (cfg.T * cfg.K), 4)
+    res["speedup"] = round(res["plain"]["ms_per_step"] / res["rounded"]["ms_per_step"], 4)
+    res["note"] = ("a different layer output: the dropped assignments add nothing; same "
+                   "weights, inputs and kernels otherwise")
+    return res
+
+
 # ------------------------------------------------------------------ our arm
 def run_ours(args, rank, world, local):
     import token_dispatch_router_b200 as tdr
@@ -529,6 +578,7 @@ def run_ours(args, rank, world, local):
     # rows materialised, combine of those rows as identity experts): the unfused traffic
     dc = dispatch_combine(tdr, s, cfg, x, w_r, bias, args.steps, world, peaks)
     dd = decode_dispatch(tdr, world)
+    tr = token_rounding_figure(tdr, cfg, x, w_r, wg, wu, wd, bias, world)
 
     # ---- per-kernel breakdown (ms per step) and the two secondary figures of the metric
     per_kernel = {k: round(ms / args.steps, 4) for k, (n, ms) in kern.items()}
@@ -543,6 +593,7 @@ def run_ours(args, rank, world, local):
                    "n": cfg.n, "global_batch": cfg.T * world, "parallelism": f"replicas{world}",
                    "l2": "inputs larger than L2: the 2.82 GB of expert weights stream every step"},
         "roofline": roofline, "gemm": gemm, "dispatch_combine": dc, "decode_dispatch": dd,
+        "token_rounding": tr,
         "kernel_ms_per_step": per_kernel,
         "gpu_launches": int(launches), "e2e": e2e,
     }
