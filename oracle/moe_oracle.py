@@ -25,9 +25,10 @@ Sources (page title, section):
   [P5] SonicMoE explainer (gitcode.csdn.net), section 1 (y = sum_i gate_i(x) *
        expert_i(x) over the top-k experts), section 3 (the GPU pipeline:
        route, regroup to expert-major, grouped GEMM, SwiGLU, second grouped
-       GEMM, scatter/combine), section 11 (expert-major metadata: per-expert
-       counts, expert-major slot -> token, token-major slot -> expert-major
-       slot).
+       GEMM, scatter/combine), section 6.4 (the backward without caching Y:
+       dA' = dO W_down^T, dS = <dA', A>), section 11 (expert-major metadata:
+       per-expert counts, expert-major slot -> token, token-major slot ->
+       expert-major slot).
 
 Readings where the pages are silent (each also listed in the design notes):
   * top-k order: descending logit, ties to the lower expert id, +0 == -0;
@@ -251,6 +252,65 @@ def grouped_ffn(x, perm_to_assign, offsets, K: int, w_gate, w_up, w_down):
         a_act[lo:hi] = swiglu(g, u)
         y_perm[lo:hi] = a_act[lo:hi] @ as_f64(w_down[e])
     return a_act, y_perm
+
+
+def gate_up_preact(x, perm_to_assign, offsets, K: int, w_gate, w_up):
+    """[P5] 3 item 3: the pre-activations of the kept slots, g[p] = x[tok(p)] W_gate[e] and
+    u[p] = x[tok(p)] W_up[e] (fp64), which the backward below reads."""
+    off = np.asarray(offsets, dtype=np.int64)
+    E = off.size - 1
+    n_kept = int(off[-1])
+    xa = as_f64(x)
+    n = w_gate.shape[2]
+    g = np.zeros((n_kept, n), dtype=F64)
+    u = np.zeros((n_kept, n), dtype=F64)
+    for e in range(E):
+        lo, hi = int(off[e]), int(off[e + 1])
+        if hi == lo:
+            continue
+        tok = np.asarray(perm_to_assign[lo:hi], dtype=np.int64) // K
+        g[lo:hi] = xa[tok] @ as_f64(w_gate[e])
+        u[lo:hi] = xa[tok] @ as_f64(w_up[e])
+    return g, u
+
+
+def backward_act(d_out, topk_w_, assign_to_perm, perm_to_assign, offsets, K: int, w_down, g, u):
+    """[P5] 6.4, the backward of the expert half of the layer without caching Y: for the
+    kept slot p of expert e holding token t's slot k (a = t*K + k = perm_to_assign[p]),
+      dA'[p] = dO[t] W_down[e]^T               (the rows of dO gathered by token)
+      dS[p]  = <dA'[p], A[p]>, A = silu(g) * u   (= dL/dw[t, k]: out = sum_k w y, y = A W_down)
+      dA[p]  = w[t, k] dA'[p]
+      dG[p]  = dA[p] * u * silu'(g),  silu'(g) = s (1 + g (1 - s)),  s = 1 / (1 + e^-g)
+      dU[p]  = dA[p] * silu(g)
+    Returns dG, dU ([kept, n], fp64) and d_w ([T, K], fp64; 0 at dropped slots)."""
+    off = np.asarray(offsets, dtype=np.int64)
+    E = off.size - 1
+    dO = as_f64(d_out)
+    T = dO.shape[0]
+    w = as_f64(topk_w_).reshape(-1)
+    a2p = np.asarray(assign_to_perm, dtype=np.int64)
+    n_kept = int(off[-1])
+    n = g.shape[1]
+    dG = np.zeros((n_kept, n), dtype=F64)
+    dU = np.zeros((n_kept, n), dtype=F64)
+    dS = np.zeros(n_kept, dtype=F64)
+    for e in range(E):
+        lo, hi = int(off[e]), int(off[e + 1])
+        if hi == lo:
+            continue
+        a = np.asarray(perm_to_assign[lo:hi], dtype=np.int64)
+        dA1 = dO[a // K] @ as_f64(w_down[e]).T
+        ge, ue = g[lo:hi], u[lo:hi]
+        sg = 1.0 / (1.0 + np.exp(-ge))
+        silu = ge * sg
+        dS[lo:hi] = np.sum(dA1 * (silu * ue), axis=1)
+        dA = w[a][:, None] * dA1
+        dG[lo:hi] = dA * ue * sg * (1.0 + ge * (1.0 - sg))
+        dU[lo:hi] = dA * silu
+    d_w = np.zeros(T * K, dtype=F64)
+    kept = a2p >= 0
+    d_w[kept] = dS[a2p[kept]]
+    return dG, dU, d_w.reshape(T, K)
 
 
 def combine(y_perm, assign_to_perm, topk_w, T: int, K: int) -> np.ndarray:

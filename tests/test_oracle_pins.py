@@ -503,3 +503,81 @@ def test_token_rounding_planted_mistake_is_caught(monkeypatch):
     wrong = orc.tile_round_keep(ids, lg, E, R)
     monkeypatch.undo()
     assert not np.array_equal(wrong, _rounding_brute_force(ids, lg, E, R))
+
+
+# ------------------------------------------------------------------ backward (expert half)
+def _autograd_backward(x, lg, wg, wu, wd, K, cf, d_out):
+    """The same layer written with torch ops in fp64 and differentiated by autograd: the
+    gradients of <d_out, out> with respect to the pre-activations (g, u) of every kept
+    slot and to the routing weights."""
+    T, E = lg.shape
+    ids, w = orc.route(lg, K)
+    counts, offsets, a2p, p2a = orc.permute(ids, E, orc.capacity(cf, T, K, E))
+    nk = int(offsets[-1])
+    xt = torch.from_numpy(np.asarray(x, np.float64))
+    G = torch.zeros(nk, wg.shape[2], dtype=torch.float64)
+    U = torch.zeros(nk, wg.shape[2], dtype=torch.float64)
+    for e in range(E):
+        lo, hi = int(offsets[e]), int(offsets[e + 1])
+        tok = torch.from_numpy(np.asarray(p2a[lo:hi], np.int64) // K)
+        G[lo:hi] = xt[tok] @ torch.from_numpy(wg[e])
+        U[lo:hi] = xt[tok] @ torch.from_numpy(wu[e])
+    G.requires_grad_(True)
+    U.requires_grad_(True)
+    W = torch.from_numpy(np.asarray(w, np.float64)).requires_grad_(True)
+    A = torch.nn.functional.silu(G) * U
+    Y = torch.zeros(nk, wd.shape[2], dtype=torch.float64)
+    for e in range(E):
+        lo, hi = int(offsets[e]), int(offsets[e + 1])
+        Y[lo:hi] = A[lo:hi] @ torch.from_numpy(wd[e])
+    out = torch.zeros(T, wd.shape[2], dtype=torch.float64)
+    for t in range(T):
+        for k in range(K):
+            p = int(a2p[t * K + k])
+            if p >= 0:
+                out[t] = out[t] + W[t, k] * Y[p]
+    (out * torch.from_numpy(d_out)).sum().backward()
+    return (G.detach().numpy(), U.detach().numpy(), G.grad.numpy(), U.grad.numpy(),
+            W.grad.numpy(), (offsets, a2p, p2a, w))
+
+
+@pytest.mark.parametrize("cf", [0.0, 0.7])
+def test_backward_matches_autograd(cf):
+    rng = np.random.default_rng(31)
+    T, d, n, E, K = 11, 6, 5, 4, 2
+    x = rng.standard_normal((T, d))
+    lg = rng.standard_normal((T, E)).astype(np.float32)
+    wg, wu = rng.standard_normal((E, d, n)), rng.standard_normal((E, d, n))
+    wd = rng.standard_normal((E, n, d))
+    d_out = rng.standard_normal((T, d))
+    g, u, gg, gu, gw, (offsets, a2p, p2a, w) = _autograd_backward(x, lg, wg, wu, wd, K, cf, d_out)
+    g2, u2 = orc.gate_up_preact(x, p2a, offsets, K, wg, wu)
+    np.testing.assert_allclose(g2, g, rtol=1e-13, atol=1e-13)
+    np.testing.assert_allclose(u2, u, rtol=1e-13, atol=1e-13)
+    dG, dU, d_w = orc.backward_act(d_out, w, a2p, p2a, offsets, K, wd, g2, u2)
+    np.testing.assert_allclose(dG, gg, rtol=1e-11, atol=1e-12)
+    np.testing.assert_allclose(dU, gu, rtol=1e-11, atol=1e-12)
+    np.testing.assert_allclose(d_w, gw, rtol=1e-11, atol=1e-12)
+    if cf > 0:
+        assert np.all(d_w.reshape(-1)[a2p < 0] == 0)  # dropped slots carry no gradient
+        assert (a2p < 0).any()
+
+
+def test_backward_planted_mistake_is_caught(monkeypatch):
+    rng = np.random.default_rng(32)
+    T, d, n, E, K = 9, 4, 3, 3, 2
+    x = rng.standard_normal((T, d))
+    lg = rng.standard_normal((T, E)).astype(np.float32)
+    wg, wu = rng.standard_normal((E, d, n)), rng.standard_normal((E, d, n))
+    wd = rng.standard_normal((E, n, d))
+    d_out = rng.standard_normal((T, d))
+    g, u, gg, gu, gw, (offsets, a2p, p2a, w) = _autograd_backward(x, lg, wg, wu, wd, K, 0.0, d_out)
+    real_exp = orc.np.exp
+
+    def exp_sign_slip(v):  # s = 1 / (1 + e^{+g}) instead of e^{-g}
+        return real_exp(-v)
+
+    monkeypatch.setattr(orc.np, "exp", exp_sign_slip)
+    dG, _, _ = orc.backward_act(d_out, w, a2p, p2a, offsets, K, wd, g, u)
+    monkeypatch.undo()
+    assert not np.allclose(dG, gg, rtol=1e-6, atol=1e-8)
