@@ -260,6 +260,40 @@ typedef struct {
 moe_status moe_forward_workspace_layout(const moe_shape* shape, moe_workspace_layout* layout);
 
 /* ----------------------------------------------------------------------------
+ * moe_forward_h - moe_forward that also keeps, for the backward, the gate/up
+ * pre-activations of every kept slot: h [T*K, 2n] bf16, row p = (g | u) with
+ * g = x[tok(p)] W_gate[e], u = x[tok(p)] W_up[e] (rows past offsets[E] unwritten).
+ * The routing outputs stay in the workspace (moe_forward_workspace_layout).
+ * bf16 only (MOE_ERR_UNSUPPORTED otherwise); h 16-byte aligned.
+ *
+ * moe_backward_act - the backward of the expert half of the layer without caching
+ * Y or dY (SonicMoE explainer, section 6.4; the gather of dO by routing index
+ * fused into the GEMM's operand load, section 6.2; the SwiGLU backward in the
+ * epilogue, section 6.3). For the kept slot p of expert e holding token t's slot k
+ * (a = perm_to_assign[p] = t*K + k):
+ *   dA'[p] = d_out[t] W_down[e]^T          (tensor cores, fp32 accumulate)
+ *   d_w[t, k] = <dA'[p], silu(g) * u>      (the routing-weight gradient; 0 if dropped)
+ *   dA = topk_w[t, k] dA',  s = 1 / (1 + e^-g)
+ *   d_h[p] = (dA u s (1 + g (1 - s)) | dA silu(g))   (dG | dU, bf16)
+ *   d_out  [T, d] bf16; topk_w [T, K] fp32; offsets, perm_to_assign,
+ *   assign_to_perm as moe_permute wrote them; w_down [E, n, d] bf16;
+ *   h [T*K, 2n] from moe_forward_h; d_h [T*K, 2n] bf16 out; d_w [T, K] fp32 out;
+ *   workspace >= moe_backward_workspace_size(shape) (per-slot partial sums).
+ * d_w sums each slot's 256-column parts in a fixed order (deterministic).
+ * bf16 only; d_out, w_down, h, d_h 16-byte aligned.
+ */
+moe_status moe_forward_h(const moe_shape* shape, const void* x, const void* w_r,
+                         const float* bias, const float* logits_in, const void* w_gate,
+                         const void* w_up, const void* w_down, void* out, void* h,
+                         void* workspace, size_t ws_bytes, moe_stream_t stream);
+size_t moe_backward_workspace_size(const moe_shape* shape);
+moe_status moe_backward_act(const moe_shape* shape, const void* d_out, const float* topk_w,
+                            const int32_t* offsets, const int32_t* perm_to_assign,
+                            const int32_t* assign_to_perm, const void* w_down, const void* h,
+                            void* d_h, float* d_w, void* workspace, size_t ws_bytes,
+                            moe_stream_t stream);
+
+/* ----------------------------------------------------------------------------
  * Device status: synchronises `stream`, returns the first device-side fault
  * recorded since the last call (MOE_OK if none) and clears it.
  */

@@ -492,6 +492,90 @@ def test_token_rounding_rejected_where_it_cannot_apply(cuda_lib):
         tdr.dispatch(bad, logits_in=torch.zeros(64, 8, device="cuda"))
 
 
+# ------------------------------------------------------------------ backward (expert half)
+def _bwd_case(tdr, cfg, seed):
+    inp = mi.make_inputs(cfg)
+    s = shape_of(cfg, tdr)
+    out_h, ws, h = tdr.forward_h(s, cuda(inp.x), cuda(inp.w_r), cuda(inp.w_gate), cuda(inp.w_up),
+                                 cuda(inp.w_down), bias=cuda(inp.bias))
+    v = tdr.workspace_views(s, ws)
+    rng = np.random.default_rng(seed)
+    d_out = torch.from_numpy(rng.standard_normal((cfg.T, cfg.d)).astype(np.float32)).to(
+        torch.bfloat16)
+    d_h, d_w = tdr.backward_act(s, d_out.cuda(), v["topk_w"], v["offsets"], v["perm_to_assign"],
+                                v["assign_to_perm"], cuda(inp.w_down), h)
+    torch.cuda.synchronize()
+    assert_status_ok(tdr)
+    return inp, s, out_h, v, h, d_out, d_h, d_w
+
+
+@pytest.mark.parametrize("T,d,n,E,K,cf", [
+    (300, 128, 128, 8, 2, 0.0),
+    (513, 256, 384, 4, 2, 0.8),    # a half n-tile, capacity drops
+    (1000, 512, 768, 16, 4, 0.0),
+])
+def test_backward_act_matches_oracle(cuda_lib, T, d, n, E, K, cf):
+    tdr = cuda_lib
+    cfg = mi.MoEConfig("bwd", T=T, d=d, E=E, K=K, n=n, dtype="bf16", capacity_factor=cf,
+                       seed=T + n)
+    inp, s, out_h, v, h, d_out, d_h, d_w = _bwd_case(tdr, cfg, 5)
+    # the forward is the plain one, and h holds the pre-activations
+    out_plain, _ = tdr.forward(s, cuda(inp.x), cuda(inp.w_r), cuda(inp.w_gate), cuda(inp.w_up),
+                               cuda(inp.w_down))
+    assert torch.equal(out_plain, out_h)
+    offsets = v["offsets"].cpu().numpy()
+    p2a = v["perm_to_assign"].cpu().numpy()
+    a2p = v["assign_to_perm"].cpu().numpy()
+    nk = int(offsets[-1])
+    g, u = orc.gate_up_preact(inp.x, p2a, offsets, K, inp.w_gate, inp.w_up)
+    hh = h[:nk].float().cpu().numpy()
+    assert_bf16_close(hh[:, :n], g, "h (g)")
+    assert_bf16_close(hh[:, n:], u, "h (u)")
+    dG, dU, dw_ref = orc.backward_act(d_out.float().numpy(), v["topk_w"].cpu().numpy(), a2p, p2a,
+                                      offsets, K, inp.w_down, g, u)
+    dh = d_h[:nk].float().cpu().numpy()
+    assert_bf16_close(dh[:, :n], dG, "dG")
+    assert_bf16_close(dh[:, n:], dU, "dU")
+    assert_bf16_close(d_w.cpu().numpy(), dw_ref, "d_w")
+    if cf > 0:
+        assert np.all(d_w.cpu().numpy().reshape(-1)[a2p < 0] == 0)
+
+
+def test_backward_act_full_size_sampled_slots(cuda_lib):
+    tdr = cuda_lib
+    cfg = mi.CONFIGS["mixtral_bf16"]
+    inp, s, _, v, h, d_out, d_h, d_w = _bwd_case(tdr, cfg, 9)
+    offsets = v["offsets"].cpu().numpy()
+    p2a = v["perm_to_assign"].cpu().numpy()
+    w = v["topk_w"].cpu().numpy().reshape(-1)
+    rng = np.random.default_rng(4)
+    slots = np.sort(rng.choice(int(offsets[-1]), size=12, replace=False))
+    K, n = cfg.K, cfg.n
+    dO = d_out.float().numpy().astype(np.float64)
+    dh = d_h.float().cpu().numpy()
+    got_g, got_u, ref_g, ref_u, got_w, ref_w = [], [], [], [], [], []
+    for p in slots:
+        e = orc.expert_of_slot(offsets, int(p))
+        a = int(p2a[p])
+        t = a // K
+        xt = orc.as_f64(inp.x[t])
+        g = xt @ orc.as_f64(inp.w_gate[e])
+        u = xt @ orc.as_f64(inp.w_up[e])
+        dA1 = dO[t] @ orc.as_f64(inp.w_down[e]).T
+        sg = 1.0 / (1.0 + np.exp(-g))
+        silu = g * sg
+        ref_w.append(float(np.dot(dA1, silu * u)))
+        dA = w[a] * dA1
+        ref_g.append(dA * u * sg * (1.0 + g * (1.0 - sg)))
+        ref_u.append(dA * silu)
+        got_g.append(dh[p, :n])
+        got_u.append(dh[p, n:])
+        got_w.append(float(d_w.reshape(-1)[a]))
+    assert_bf16_close(np.array(got_g), np.array(ref_g), "full-size dG")
+    assert_bf16_close(np.array(got_u), np.array(ref_u), "full-size dU")
+    assert_bf16_close(np.array(got_w), np.array(ref_w), "full-size d_w")
+
+
 @pytest.mark.parametrize("T", mi.DISPATCH_COMBINE_T)
 def test_dispatch_combine_identity_experts(cuda_lib, T):
     """route (given logits) -> permute with x_perm -> combine(y_perm = x_perm) returns x."""

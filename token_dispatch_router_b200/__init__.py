@@ -57,6 +57,11 @@ _SIGS = {
     "moe_grouped_ffn": (ctypes.c_int, [_S, _P, _P, _P, _P, _P, _P, _P, _P, _P]),
     "moe_combine": (ctypes.c_int, [_S, _P, _P, _P, _P, _P]),
     "moe_forward": (ctypes.c_int, [_S, _P, _P, _P, _P, _P, _P, _P, _P, _P, ctypes.c_size_t, _P]),
+    "moe_forward_h": (ctypes.c_int, [_S, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P,
+                                     ctypes.c_size_t, _P]),
+    "moe_backward_workspace_size": (ctypes.c_size_t, [_S]),
+    "moe_backward_act": (ctypes.c_int, [_S, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P,
+                                        ctypes.c_size_t, _P]),
     "moe_get_device_status": (ctypes.c_int, [_P]),
     "moe_status_string": (ctypes.c_char_p, [ctypes.c_int]),
     "moe_profile_enable": (ctypes.c_int, [ctypes.c_int]),
@@ -341,6 +346,62 @@ def forward(shape: moe_shape, x, w_r, w_gate, w_up, w_down, bias=None, logits_in
                            _ptr(w_gate), _ptr(w_up), _ptr(w_down), _ptr(out), _ptr(workspace),
                            workspace.numel(), _stream()), "moe_forward")
     return out, workspace
+
+
+def forward_h(shape: moe_shape, x, w_r, w_gate, w_up, w_down, bias=None, logits_in=None,
+              out=None, workspace=None, h=None):
+    """moe_forward_h: the layer, keeping the gate/up pre-activations for the backward.
+    Returns (out [T, d], workspace, h [T*K, 2n])."""
+    lib = load_library()
+    T, d, E, n, K = shape.T, shape.d, shape.E, shape.n, shape.K
+    dt = _act_dtype(shape)
+    _dev(x, "x", dt, (T, d))
+    if logits_in is None:
+        _dev(w_r, "w_r", dt, (d, E))
+    else:
+        _dev(logits_in, "logits_in", torch.float32, (T, E))
+    _dev(w_gate, "w_gate", dt, (E, d, n))
+    _dev(w_up, "w_up", dt, (E, d, n))
+    _dev(w_down, "w_down", dt, (E, n, d))
+    if bias is not None:
+        _dev(bias, "bias", torch.float32, (E,))
+    need = forward_workspace_size(shape)
+    if need == 0:
+        raise MoEError(1, "moe_forward_workspace_size")
+    if workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=x.device)
+    if out is None:
+        out = torch.empty(T, d, dtype=dt, device=x.device)
+    if h is None:
+        h = torch.empty(T * K, 2 * n, dtype=dt, device=x.device)
+    _check(lib.moe_forward_h(ctypes.byref(shape), _ptr(x), _ptr(w_r), _ptr(bias), _ptr(logits_in),
+                             _ptr(w_gate), _ptr(w_up), _ptr(w_down), _ptr(out), _ptr(h),
+                             _ptr(workspace), workspace.numel(), _stream()), "moe_forward_h")
+    return out, workspace, h
+
+
+def backward_act(shape: moe_shape, d_out, topk_w, offsets, perm_to_assign, assign_to_perm,
+                 w_down, h, d_h=None, d_w=None, workspace=None):
+    """moe_backward_act. Returns (d_h [T*K, 2n] = dG | dU per kept slot, d_w [T, K])."""
+    lib = load_library()
+    T, d, E, n, K = shape.T, shape.d, shape.E, shape.n, shape.K
+    dt = _act_dtype(shape)
+    _dev(d_out, "d_out", dt, (T, d))
+    _dev(w_down, "w_down", dt, (E, n, d))
+    _dev(h, "h", dt, (T * K, 2 * n))
+    dev = d_out.device
+    if d_h is None:
+        d_h = torch.empty(T * K, 2 * n, dtype=dt, device=dev)
+    if d_w is None:
+        d_w = torch.empty(T, K, dtype=torch.float32, device=dev)
+    need = int(lib.moe_backward_workspace_size(ctypes.byref(shape)))
+    if workspace is None:
+        workspace = torch.empty(max(need, 256), dtype=torch.uint8, device=dev)
+    _check(lib.moe_backward_act(ctypes.byref(shape), _ptr(d_out), _ptr(topk_w), _ptr(offsets),
+                                _ptr(perm_to_assign), _ptr(assign_to_perm), _ptr(w_down), _ptr(h),
+                                _ptr(d_h), _ptr(d_w), _ptr(workspace), workspace.numel(),
+                                _stream()), "moe_backward_act")
+    return d_h, d_w
 
 
 def workspace_views(shape: moe_shape, workspace: torch.Tensor) -> dict:

@@ -27,7 +27,12 @@ bool route_tc_supported(const moe_shape& s);
 moe_status launch_ffn_tc_mixed(const moe_shape& s, const void* x, const int32_t* offsets,
                                const int32_t* p2a, const void* w_gate, const void* w_up,
                                const void* w_down, void* a_act, void* y_perm, int gateup_mode,
-                               bool pair_down, cudaStream_t st);
+                               bool pair_down, void* h_out, cudaStream_t st);
+size_t backward_scratch_bytes(const moe_shape& s);
+moe_status launch_backward_act(const moe_shape& s, const void* d_out, const float* topk_w,
+                               const int32_t* offsets, const int32_t* p2a, const int32_t* a2p,
+                               const void* w_down, const void* h, void* d_h, float* d_w,
+                               void* scratch, cudaStream_t st);
 moe_status launch_permute_static(const moe_shape& s, const int32_t* ids, int32_t* counts,
                                  int32_t* offsets, int32_t* a2p, int32_t* p2a, const void* x,
                                  void* x_perm, cudaStream_t st);
@@ -87,7 +92,7 @@ const char* kKernelNames[K_COUNT] = {
     "route",        "hist",          "scan",           "scatter",     "gather_rows", "gateup_tc",
     "down_tc",      "gateup_simt",   "down_simt",      "combine",     "selftest_timeout",
     "route_tc",     "permute_small", "gateup_tc2",   "down_tc2",
-    "permute_cluster", "route_permute", "tile_round"};
+    "permute_cluster", "route_permute", "tile_round", "bwd_act", "bwd_dw"};
 
 struct ProfRec {
   int kid;
@@ -201,6 +206,60 @@ bool use_pair_down(const moe_shape& s) {
 }
 int gateup_mode() { return g_ffn_variant == 2 ? 1 : g_ffn_variant == 3 ? 2 : 0; }
 
+}  // namespace
+}  // namespace moe
+
+namespace moe {
+namespace {
+moe_status forward_impl(const moe_shape* s, const void* x, const void* w_r, const float* bias,
+                        const float* logits_in, const void* w_gate, const void* w_up,
+                        const void* w_down, void* out, void* h_out, void* workspace,
+                        size_t ws_bytes, moe_stream_t stream) {
+  moe_status r = check_shape(s, true, true);
+  if (r != MOE_OK) return r;
+  if (s->T == 0) return MOE_OK;
+  if (!x || (!w_r && !logits_in) || !w_gate || !w_up || !w_down || !out) return MOE_ERR_INVALID_ARG;
+  moe_workspace_layout L;
+  layout_of(*s, &L);
+  if (workspace == nullptr || ws_bytes < L.total) return MOE_ERR_WORKSPACE;
+  if (((uintptr_t)workspace & 255) != 0) return MOE_ERR_INVALID_ARG;
+  uint8_t* ws = (uint8_t*)workspace;
+  const cudaStream_t st = (cudaStream_t)stream;
+  float* logits = (float*)(ws + L.logits);
+  int32_t* ids = (int32_t*)(ws + L.topk_ids);
+  float* w = (float*)(ws + L.topk_w);
+  int32_t* counts = (int32_t*)(ws + L.counts);
+  int32_t* offsets = (int32_t*)(ws + L.offsets);
+  int32_t* a2p = (int32_t*)(ws + L.assign_to_perm);
+  int32_t* p2a = (int32_t*)(ws + L.perm_to_assign);
+  if (s->tile_round > 0) {
+    if ((r = moe_route(s, x, w_r, bias, logits_in, logits, ids, w, stream)) != MOE_OK) return r;
+    if ((r = launch_permute_rounded(*s, ids, logits, counts, offsets, a2p, p2a, nullptr, nullptr,
+                                    ws + L.permute_scratch, (int32_t*)(ws + L.round_ids),
+                                    (int32_t*)(ws + L.round_counts), st)) != MOE_OK)
+      return r;
+  } else if (route_permute_fusable(*s, logits_in)) {
+    if ((r = launch_route_permute(*s, logits_in, logits, ids, w, counts, offsets, a2p, p2a, st)) !=
+        MOE_OK)
+      return r;
+  } else {
+    if ((r = moe_route(s, x, w_r, bias, logits_in, logits, ids, w, stream)) != MOE_OK) return r;
+    if ((r = launch_permute(*s, ids, counts, offsets, a2p, p2a, nullptr, nullptr,
+                            ws + L.permute_scratch, st)) != MOE_OK)
+      return r;
+  }
+  if (h_out != nullptr) {  // keep the gate/up pre-activations (single-CTA gate/up tiles)
+    if (!aligned16(x) || !aligned16(w_gate) || !aligned16(w_up) || !aligned16(w_down))
+      return MOE_ERR_INVALID_ARG;
+    r = launch_ffn_tc_mixed(*s, x, offsets, p2a, w_gate, w_up, w_down, ws + L.a_act,
+                            ws + L.y_perm, 0, use_pair_down(*s), h_out, st);
+  } else {
+    r = moe_grouped_ffn(s, x, offsets, p2a, w_gate, w_up, w_down, ws + L.a_act, ws + L.y_perm,
+                        stream);
+  }
+  if (r != MOE_OK) return r;
+  return launch_combine(*s, ws + L.y_perm, a2p, w, out, st);
+}
 }  // namespace
 }  // namespace moe
 
@@ -355,7 +414,7 @@ moe_status moe_grouped_ffn(const moe_shape* s, const void* x, const int32_t* off
     return MOE_ERR_INVALID_ARG;
   if (s->dtype == MOE_BF16)
     return launch_ffn_tc_mixed(*s, x, offsets, perm_to_assign, w_gate, w_up, w_down, a_act, y_perm,
-                               gateup_mode(), use_pair_down(*s), (cudaStream_t)stream);
+                               gateup_mode(), use_pair_down(*s), nullptr, (cudaStream_t)stream);
   return launch_ffn_simt(*s, x, offsets, perm_to_assign, w_gate, w_up, w_down, a_act, y_perm,
                          (cudaStream_t)stream);
 }
@@ -370,47 +429,48 @@ moe_status moe_combine(const moe_shape* s, const void* y_perm, const int32_t* as
   return launch_combine(*s, y_perm, assign_to_perm, topk_w, out, (cudaStream_t)stream);
 }
 
+
 moe_status moe_forward(const moe_shape* s, const void* x, const void* w_r, const float* bias,
                        const float* logits_in, const void* w_gate, const void* w_up,
                        const void* w_down, void* out, void* workspace, size_t ws_bytes,
                        moe_stream_t stream) {
+  return forward_impl(s, x, w_r, bias, logits_in, w_gate, w_up, w_down, out, nullptr, workspace,
+                      ws_bytes, stream);
+}
+
+moe_status moe_forward_h(const moe_shape* s, const void* x, const void* w_r, const float* bias,
+                         const float* logits_in, const void* w_gate, const void* w_up,
+                         const void* w_down, void* out, void* h, void* workspace,
+                         size_t ws_bytes, moe_stream_t stream) {
+  if (s != nullptr && s->dtype != MOE_BF16) return MOE_ERR_UNSUPPORTED;
+  if (h == nullptr || !aligned16(h)) return MOE_ERR_INVALID_ARG;
+  return forward_impl(s, x, w_r, bias, logits_in, w_gate, w_up, w_down, out, h, workspace,
+                      ws_bytes, stream);
+}
+
+size_t moe_backward_workspace_size(const moe_shape* s) {
+  if (check_shape(s, true, true) != MOE_OK) return 0;
+  return align256(backward_scratch_bytes(*s)) + 256;
+}
+
+moe_status moe_backward_act(const moe_shape* s, const void* d_out, const float* topk_w,
+                            const int32_t* offsets, const int32_t* perm_to_assign,
+                            const int32_t* assign_to_perm, const void* w_down, const void* h,
+                            void* d_h, float* d_w, void* workspace, size_t ws_bytes,
+                            moe_stream_t stream) {
   moe_status r = check_shape(s, true, true);
   if (r != MOE_OK) return r;
+  if (s->dtype != MOE_BF16) return MOE_ERR_UNSUPPORTED;
   if (s->T == 0) return MOE_OK;
-  if (!x || (!w_r && !logits_in) || !w_gate || !w_up || !w_down || !out) return MOE_ERR_INVALID_ARG;
-  moe_workspace_layout L;
-  layout_of(*s, &L);
-  if (workspace == nullptr || ws_bytes < L.total) return MOE_ERR_WORKSPACE;
-  if (((uintptr_t)workspace & 255) != 0) return MOE_ERR_INVALID_ARG;
-  uint8_t* ws = (uint8_t*)workspace;
-  const cudaStream_t st = (cudaStream_t)stream;
-  float* logits = (float*)(ws + L.logits);
-  int32_t* ids = (int32_t*)(ws + L.topk_ids);
-  float* w = (float*)(ws + L.topk_w);
-  int32_t* counts = (int32_t*)(ws + L.counts);
-  int32_t* offsets = (int32_t*)(ws + L.offsets);
-  int32_t* a2p = (int32_t*)(ws + L.assign_to_perm);
-  int32_t* p2a = (int32_t*)(ws + L.perm_to_assign);
-  if (s->tile_round > 0) {
-    if ((r = moe_route(s, x, w_r, bias, logits_in, logits, ids, w, stream)) != MOE_OK) return r;
-    if ((r = launch_permute_rounded(*s, ids, logits, counts, offsets, a2p, p2a, nullptr, nullptr,
-                                    ws + L.permute_scratch, (int32_t*)(ws + L.round_ids),
-                                    (int32_t*)(ws + L.round_counts), st)) != MOE_OK)
-      return r;
-  } else if (route_permute_fusable(*s, logits_in)) {
-    if ((r = launch_route_permute(*s, logits_in, logits, ids, w, counts, offsets, a2p, p2a, st)) !=
-        MOE_OK)
-      return r;
-  } else {
-    if ((r = moe_route(s, x, w_r, bias, logits_in, logits, ids, w, stream)) != MOE_OK) return r;
-    if ((r = launch_permute(*s, ids, counts, offsets, a2p, p2a, nullptr, nullptr,
-                            ws + L.permute_scratch, st)) != MOE_OK)
-      return r;
-  }
-  if ((r = moe_grouped_ffn(s, x, offsets, p2a, w_gate, w_up, w_down, ws + L.a_act, ws + L.y_perm,
-                           stream)) != MOE_OK)
-    return r;
-  return launch_combine(*s, ws + L.y_perm, a2p, w, out, st);
+  if (!d_out || !topk_w || !offsets || !perm_to_assign || !assign_to_perm || !w_down || !h ||
+      !d_h || !d_w)
+    return MOE_ERR_INVALID_ARG;
+  if (!aligned16(d_out) || !aligned16(w_down) || !aligned16(h) || !aligned16(d_h))
+    return MOE_ERR_INVALID_ARG;
+  const size_t need = backward_scratch_bytes(*s);
+  if (workspace == nullptr || ws_bytes < need) return MOE_ERR_WORKSPACE;
+  return launch_backward_act(*s, d_out, topk_w, offsets, perm_to_assign, assign_to_perm, w_down,
+                             h, d_h, d_w, workspace, (cudaStream_t)stream);
 }
 
 moe_status moe_get_device_status(moe_stream_t stream) {

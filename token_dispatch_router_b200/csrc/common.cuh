@@ -104,6 +104,8 @@ enum KernelId {
   K_PERMUTE_CLUSTER,
   K_ROUTE_PERMUTE,
   K_TILE_ROUND,
+  K_BWD_ACT,
+  K_BWD_DW,
   K_COUNT
 };
 

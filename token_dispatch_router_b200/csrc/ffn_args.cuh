@@ -20,6 +20,7 @@ struct GemmArgs {
   int E, K, T;
   unsigned* status;
   unsigned long long limit_ns;
+  bf16* h_out;  // gate/up, single CTA: if not NULL, also the pre-activations (g | u) per row
 };
 
 // bf16 tensor of `rank` dims (innermost first), 128-byte swizzle, zero fill out of bounds.

@@ -470,6 +470,22 @@ __global__ void __launch_bounds__(GATEUP ? THREADS_GATEUP : THREADS_DOWN, 1)
 #pragma unroll
             for (int j = 0; j < 4; ++j)
               dst[j] = make_uint4(pk[4 * j], pk[4 * j + 1], pk[4 * j + 2], pk[4 * j + 3]);
+            if (g.h_out != nullptr) {  // keep (g | u) for the backward
+              bf16* hrow = g.h_out + (size_t)(t.m0 + r) * (2 * (size_t)g.n_out);
+              uint4* hg = reinterpret_cast<uint4*>(hrow + col);
+              uint4* hu = reinterpret_cast<uint4*>(hrow + g.n_out + col);
+#pragma unroll
+              for (int j = 0; j < 4; ++j) {
+                hg[j] = make_uint4(pack_bf16x2(__uint_as_float(gv[8 * j]), __uint_as_float(gv[8 * j + 1])),
+                                   pack_bf16x2(__uint_as_float(gv[8 * j + 2]), __uint_as_float(gv[8 * j + 3])),
+                                   pack_bf16x2(__uint_as_float(gv[8 * j + 4]), __uint_as_float(gv[8 * j + 5])),
+                                   pack_bf16x2(__uint_as_float(gv[8 * j + 6]), __uint_as_float(gv[8 * j + 7])));
+                hu[j] = make_uint4(pack_bf16x2(__uint_as_float(uv[8 * j]), __uint_as_float(uv[8 * j + 1])),
+                                   pack_bf16x2(__uint_as_float(uv[8 * j + 2]), __uint_as_float(uv[8 * j + 3])),
+                                   pack_bf16x2(__uint_as_float(uv[8 * j + 4]), __uint_as_float(uv[8 * j + 5])),
+                                   pack_bf16x2(__uint_as_float(uv[8 * j + 6]), __uint_as_float(uv[8 * j + 7])));
+              }
+            }
           }
         }
       } else {
@@ -620,6 +636,7 @@ static moe_status prepare_ffn(const moe_shape& s, const void* x, const int32_t* 
   ga.T = s.T;
   ga.status = device_status_ptr();
   ga.limit_ns = kWaitLimitNs;
+  ga.h_out = nullptr;
   ga.out = (bf16*)a_act;
   ga.ld_out = s.n;
   ga.n_out = s.n;
@@ -642,17 +659,21 @@ moe_status launch_ffn_tc2_gemm(int mode, const CUtensorMap& a, const CUtensorMap
 moe_status launch_gather_rows(const moe_shape& s, const void* x, const int32_t* p2a,
                               const int32_t* offsets, void* x_perm, cudaStream_t st);
 
-// gateup_mode 0: single-CTA tiles, A rows gathered in the kernel; 1: CTA pairs, A rows
+// h_out (nullable): the gate/up pre-activations (g | u) of every kept row, for the backward
+// (single-CTA tiles then). gateup_mode 0: single-CTA tiles, A rows gathered in the kernel;
+// 1: CTA pairs, A rows
 // gathered in the kernel; 2: the rows are first copied expert-major into y_perm (which the
 // down GEMM overwrites only later), then CTA pairs load A from there by TMA.
 moe_status launch_ffn_tc_mixed(const moe_shape& s, const void* x, const int32_t* offsets,
                                const int32_t* p2a, const void* w_gate, const void* w_up,
                                const void* w_down, void* a_act, void* y_perm, int gateup_mode,
-                               bool pair_down, cudaStream_t st) {
+                               bool pair_down, void* h_out, cudaStream_t st) {
   if ((long long)s.T * s.K == 0) return MOE_OK;
   FfnMaps f;
   moe_status r = prepare_ffn(s, x, offsets, p2a, w_gate, w_up, w_down, a_act, y_perm, f);
   if (r != MOE_OK) return r;
+  f.gate_up.h_out = (bf16*)h_out;
+  if (h_out != nullptr) gateup_mode = 0;  // the single-CTA epilogue keeps the pre-activations
   if (gateup_mode == 2) {
     if ((r = launch_gather_rows(s, x, p2a, offsets, y_perm, st)) != MOE_OK) return r;
     CUtensorMap mx;
