@@ -17,6 +17,7 @@ only.
 from __future__ import annotations
 
 import argparse
+import ctypes
 import hashlib
 import json
 import os
@@ -449,6 +450,55 @@ def token_rounding_figure(tdr, cfg, x, w_r, wg, wu, wd, bias, world, R=128, roun
     return res
 
 
+def backward_figure(tdr, cfg, s, x, w_r, wg, wu, wd, bias, world, peak_t, steps=20):
+    """The expert-half backward (moe_backward_act: dA' = dO W_down^T with dO gathered by
+    token, dS, dSwiGLU in the epilogue, then d_w) at the layer's shape, after a
+    moe_forward_h: CUDA events over `steps` calls; TFLOP/s on the algorithmic 2*d*n per kept
+    slot of the GEMM."""
+    if cfg.dtype != "bf16":
+        return None
+    dev = x.device
+    out, ws, h = tdr.forward_h(s, x, w_r, wg, wu, wd, bias=bias)
+    v = tdr.workspace_views(s, ws)
+    d_out = torch.randn(cfg.T, cfg.d, dtype=torch.bfloat16, device=dev,
+                        generator=torch.Generator(device=dev).manual_seed(0))
+    d_h = torch.empty_like(h)
+    d_w = torch.empty(cfg.T, cfg.K, dtype=torch.float32, device=dev)
+    bws = torch.empty(max(int(tdr.load_library().moe_backward_workspace_size(
+        ctypes.byref(s))), 256), dtype=torch.uint8, device=dev)
+
+    def call():
+        tdr.backward_act(s, d_out, v["topk_w"], v["offsets"], v["perm_to_assign"],
+                         v["assign_to_perm"], wd, h, d_h=d_h, d_w=d_w, workspace=bws)
+
+    for _ in range(3):
+        call()
+    torch.cuda.synchronize()
+    prof = tdr.Profiler()
+    with prof:
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(steps):
+            call()
+        e1.record()
+        torch.cuda.synchronize()
+    if tdr.device_status() != 0:
+        raise RuntimeError("device status set during the backward runs")
+    ms = max_over_ranks(e0.elapsed_time(e1) / steps, world)
+    k = prof.results()
+    a_kept = int(v["offsets"][cfg.E].item())
+    flops = 2.0 * cfg.d * cfg.n * a_kept
+    n_b, ms_b = k.get("bwd_act", (0, 0.0))
+    gemm_ms = ms_b / max(n_b, 1)
+    tf = flops / (gemm_ms / 1e3) / 1e12 if gemm_ms > 0 else 0.0
+    return {"ms_per_call": round(ms, 4), "gemm_ms": round(gemm_ms, 4),
+            "gemm_tflops": round(tf, 2), "gemm_frac_of_sustained_peak": round(tf / peak_t, 4),
+            "dw_ms": round(k.get("bwd_dw", (1, 0.0))[1] / max(k.get("bwd_dw", (1, 0.0))[0], 1), 4),
+            "bytes_epilogue": 2 * a_kept * 2 * cfg.n * 2,
+            "note": "dA' GEMM with dS and the SwiGLU backward in its epilogue (reads h, writes "
+                    "d_h), then the fixed-order d_w reduction"}
+
+
 # ------------------------------------------------------------------ our arm
 def run_ours(args, rank, world, local):
     import token_dispatch_router_b200 as tdr
@@ -579,6 +629,7 @@ def run_ours(args, rank, world, local):
     dc = dispatch_combine(tdr, s, cfg, x, w_r, bias, args.steps, world, peaks)
     dd = decode_dispatch(tdr, world)
     tr = token_rounding_figure(tdr, cfg, x, w_r, wg, wu, wd, bias, world)
+    bw = backward_figure(tdr, cfg, s, x, w_r, wg, wu, wd, bias, world, peak_t)
 
     # ---- per-kernel breakdown (ms per step) and the two secondary figures of the metric
     per_kernel = {k: round(ms / args.steps, 4) for k, (n, ms) in kern.items()}
@@ -593,7 +644,7 @@ def run_ours(args, rank, world, local):
                    "n": cfg.n, "global_batch": cfg.T * world, "parallelism": f"replicas{world}",
                    "l2": "inputs larger than L2: the 2.82 GB of expert weights stream every step"},
         "roofline": roofline, "gemm": gemm, "dispatch_combine": dc, "decode_dispatch": dd,
-        "token_rounding": tr,
+        "token_rounding": tr, "backward_act": bw,
         "kernel_ms_per_step": per_kernel,
         "gpu_launches": int(launches), "e2e": e2e,
     }
