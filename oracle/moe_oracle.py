@@ -313,6 +313,30 @@ def backward_act(d_out, topk_w_, assign_to_perm, perm_to_assign, offsets, K: int
     return dG, dU, d_w.reshape(T, K)
 
 
+def backward_dx(dG, dU, assign_to_perm, perm_to_assign, offsets, K: int, T: int, w_gate, w_up):
+    """[P5] 6.4 continued: the input gradient through the experts (routing held fixed),
+      dX_perm[p] = dG[p] W_gate[e]^T + dU[p] W_up[e]^T
+      dx[t]      = sum over t's kept slots k of dX_perm[assign_to_perm[t*K + k]], in k order.
+    Returns dx [T, d] (fp64)."""
+    off = np.asarray(offsets, dtype=np.int64)
+    E = off.size - 1
+    d = w_gate.shape[1]
+    n_kept = int(off[-1])
+    dXp = np.zeros((n_kept, d), dtype=F64)
+    for e in range(E):
+        lo, hi = int(off[e]), int(off[e + 1])
+        if hi == lo:
+            continue
+        dXp[lo:hi] = (as_f64(dG[lo:hi]) @ as_f64(w_gate[e]).T
+                      + as_f64(dU[lo:hi]) @ as_f64(w_up[e]).T)
+    a2p = np.asarray(assign_to_perm, dtype=np.int64).reshape(T, K)
+    dx = np.zeros((T, d), dtype=F64)
+    for k in range(K):
+        kept = a2p[:, k] >= 0
+        dx[kept] += dXp[a2p[kept, k]]
+    return dx
+
+
 def combine(y_perm, assign_to_perm, topk_w, T: int, K: int) -> np.ndarray:
     """[P5] 1 and 3 item 6: out[t] = sum_k w[t,k] * y[assign_to_perm[t*K+k]],
     summed in k order; a dropped slot (-1) adds nothing and the other weights

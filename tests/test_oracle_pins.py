@@ -526,6 +526,15 @@ def _autograd_backward(x, lg, wg, wu, wd, K, cf, d_out):
     U.requires_grad_(True)
     W = torch.from_numpy(np.asarray(w, np.float64)).requires_grad_(True)
     A = torch.nn.functional.silu(G) * U
+    # the same pre-activations as functions of x (routing held fixed), for the input gradient
+    Xl = xt.clone().requires_grad_(True)
+    G2 = torch.zeros_like(G)
+    U2 = torch.zeros_like(U)
+    for e in range(E):
+        lo, hi = int(offsets[e]), int(offsets[e + 1])
+        tok = torch.from_numpy(np.asarray(p2a[lo:hi], np.int64) // K)
+        G2[lo:hi] = Xl[tok] @ torch.from_numpy(wg[e])
+        U2[lo:hi] = Xl[tok] @ torch.from_numpy(wu[e])
     Y = torch.zeros(nk, wd.shape[2], dtype=torch.float64)
     for e in range(E):
         lo, hi = int(offsets[e]), int(offsets[e + 1])
@@ -537,6 +546,9 @@ def _autograd_backward(x, lg, wg, wu, wd, K, cf, d_out):
             if p >= 0:
                 out[t] = out[t] + W[t, k] * Y[p]
     (out * torch.from_numpy(d_out)).sum().backward()
+    # dx: d<d_out, out>/dx through G2, U2 with the upstream gradients G.grad, U.grad
+    (G2 * G.grad).sum().add_((U2 * U.grad).sum()).backward()
+    _autograd_backward.dx = Xl.grad.numpy()
     return (G.detach().numpy(), U.detach().numpy(), G.grad.numpy(), U.grad.numpy(),
             W.grad.numpy(), (offsets, a2p, p2a, w))
 
@@ -558,6 +570,8 @@ def test_backward_matches_autograd(cf):
     np.testing.assert_allclose(dG, gg, rtol=1e-11, atol=1e-12)
     np.testing.assert_allclose(dU, gu, rtol=1e-11, atol=1e-12)
     np.testing.assert_allclose(d_w, gw, rtol=1e-11, atol=1e-12)
+    dx = orc.backward_dx(dG, dU, a2p, p2a, offsets, K, T, wg, wu)
+    np.testing.assert_allclose(dx, _autograd_backward.dx, rtol=1e-11, atol=1e-12)
     if cf > 0:
         assert np.all(d_w.reshape(-1)[a2p < 0] == 0)  # dropped slots carry no gradient
         assert (a2p < 0).any()
