@@ -451,10 +451,9 @@ def token_rounding_figure(tdr, cfg, x, w_r, wg, wu, wd, bias, world, R=128, roun
 
 
 def backward_figure(tdr, cfg, s, x, w_r, wg, wu, wd, bias, world, peak_t, steps=20):
-    """The expert-half backward (moe_backward_act: dA' = dO W_down^T with dO gathered by
-    token, dS, dSwiGLU in the epilogue, then d_w) at the layer's shape, after a
-    moe_forward_h: CUDA events over `steps` calls; TFLOP/s on the algorithmic 2*d*n per kept
-    slot of the GEMM."""
+    """The expert-half backward (moe_backward with the input gradient) at the layer's shape,
+    after a moe_forward_h: CUDA events over `steps` calls, per-kernel times from the
+    library's event profiler."""
     if cfg.dtype != "bf16":
         return None
     dev = x.device
@@ -467,9 +466,12 @@ def backward_figure(tdr, cfg, s, x, w_r, wg, wu, wd, bias, world, peak_t, steps=
     bws = torch.empty(max(int(tdr.load_library().moe_backward_workspace_size(
         ctypes.byref(s))), 256), dtype=torch.uint8, device=dev)
 
+    d_x = torch.empty(cfg.T, cfg.d, dtype=torch.bfloat16, device=dev)
+
     def call():
-        tdr.backward_act(s, d_out, v["topk_w"], v["offsets"], v["perm_to_assign"],
-                         v["assign_to_perm"], wd, h, d_h=d_h, d_w=d_w, workspace=bws)
+        tdr.backward(s, d_out, v["topk_w"], v["offsets"], v["perm_to_assign"],
+                     v["assign_to_perm"], wd, h, w_gate=wg, w_up=wu, d_h=d_h, d_w=d_w, d_x=d_x,
+                     input_grad=True, workspace=bws)
 
     for _ in range(3):
         call()
@@ -488,15 +490,23 @@ def backward_figure(tdr, cfg, s, x, w_r, wg, wu, wd, bias, world, peak_t, steps=
     k = prof.results()
     a_kept = int(v["offsets"][cfg.E].item())
     flops = 2.0 * cfg.d * cfg.n * a_kept
-    n_b, ms_b = k.get("bwd_act", (0, 0.0))
-    gemm_ms = ms_b / max(n_b, 1)
-    tf = flops / (gemm_ms / 1e3) / 1e12 if gemm_ms > 0 else 0.0
-    return {"ms_per_call": round(ms, 4), "gemm_ms": round(gemm_ms, 4),
-            "gemm_tflops": round(tf, 2), "gemm_frac_of_sustained_peak": round(tf / peak_t, 4),
-            "dw_ms": round(k.get("bwd_dw", (1, 0.0))[1] / max(k.get("bwd_dw", (1, 0.0))[0], 1), 4),
-            "bytes_epilogue": 2 * a_kept * 2 * cfg.n * 2,
-            "note": "dA' GEMM with dS and the SwiGLU backward in its epilogue (reads h, writes "
-                    "d_h), then the fixed-order d_w reduction"}
+    def avg(name):
+        c, t = k.get(name, (0, 0.0))
+        return t / max(c, 1)
+
+    act_ms, dx_ms = avg("bwd_act"), avg("bwd_dx")
+    tf_act = flops / (act_ms / 1e3) / 1e12 if act_ms > 0 else 0.0
+    tf_dx = 2 * flops / (dx_ms / 1e3) / 1e12 if dx_ms > 0 else 0.0
+    return {"ms_per_call": round(ms, 4),
+            "dact_gemm_ms": round(act_ms, 4), "dact_tflops": round(tf_act, 2),
+            "dact_frac_of_sustained_peak": round(tf_act / peak_t, 4),
+            "dx_gemm_ms": round(dx_ms, 4), "dx_tflops": round(tf_dx, 2),
+            "dx_frac_of_sustained_peak": round(tf_dx / peak_t, 4),
+            "dw_ms": round(avg("bwd_dw"), 4), "scatter_add_ms": round(avg("combine"), 4),
+            "note": "dA' = dO W_down^T (dO gathered by token; dS and the SwiGLU backward in the "
+                    "epilogue: reads h, writes d_h), d_w reduction, dX_perm = (dG|dU) "
+                    "(W_gate|W_up)^T, scatter-add to tokens; TFLOP/s on 2*d*n (dA') and "
+                    "4*d*n (dX) per kept slot"}
 
 
 # ------------------------------------------------------------------ our arm

@@ -266,32 +266,39 @@ moe_status moe_forward_workspace_layout(const moe_shape* shape, moe_workspace_la
  * The routing outputs stay in the workspace (moe_forward_workspace_layout).
  * bf16 only (MOE_ERR_UNSUPPORTED otherwise); h 16-byte aligned.
  *
- * moe_backward_act - the backward of the expert half of the layer without caching
+ * moe_backward - the backward of the expert half of the layer without caching
  * Y or dY (SonicMoE explainer, section 6.4; the gather of dO by routing index
  * fused into the GEMM's operand load, section 6.2; the SwiGLU backward in the
- * epilogue, section 6.3). For the kept slot p of expert e holding token t's slot k
- * (a = perm_to_assign[p] = t*K + k):
+ * epilogue, section 6.3), routing held fixed. For the kept slot p of expert e
+ * holding token t's slot k (a = perm_to_assign[p] = t*K + k):
  *   dA'[p] = d_out[t] W_down[e]^T          (tensor cores, fp32 accumulate)
  *   d_w[t, k] = <dA'[p], silu(g) * u>      (the routing-weight gradient; 0 if dropped)
  *   dA = topk_w[t, k] dA',  s = 1 / (1 + e^-g)
  *   d_h[p] = (dA u s (1 + g (1 - s)) | dA silu(g))   (dG | dU, bf16)
+ * and, when d_x is not NULL, the input gradient through the experts:
+ *   dX_perm[p] = dG[p] W_gate[e]^T + dU[p] W_up[e]^T  (tensor cores, K = 2n)
+ *   d_x[t] = sum over t's kept slots of dX_perm      (fp32 sum in slot order, bf16)
  *   d_out  [T, d] bf16; topk_w [T, K] fp32; offsets, perm_to_assign,
- *   assign_to_perm as moe_permute wrote them; w_down [E, n, d] bf16;
+ *   assign_to_perm as moe_permute wrote them; w_gate, w_up [E, d, n] and
+ *   w_down [E, n, d] bf16 (w_gate, w_up may be NULL when d_x is NULL);
  *   h [T*K, 2n] from moe_forward_h; d_h [T*K, 2n] bf16 out; d_w [T, K] fp32 out;
- *   workspace >= moe_backward_workspace_size(shape) (per-slot partial sums).
- * d_w sums each slot's 256-column parts in a fixed order (deterministic).
- * bf16 only; d_out, w_down, h, d_h 16-byte aligned.
+ *   d_x [T, d] bf16 out or NULL;
+ *   workspace >= moe_backward_workspace_size(shape), 256-byte aligned (per-slot partial
+ *   sums, and the dX_perm rows).
+ * d_w sums each slot's 256-column parts in a fixed order (deterministic). The router's
+ * own backward (through the softmax and top-K to the logits, W_r and x) and the weight
+ * gradients are not computed. bf16 only; d_out, w_*, h, d_h, d_x 16-byte aligned.
  */
 moe_status moe_forward_h(const moe_shape* shape, const void* x, const void* w_r,
                          const float* bias, const float* logits_in, const void* w_gate,
                          const void* w_up, const void* w_down, void* out, void* h,
                          void* workspace, size_t ws_bytes, moe_stream_t stream);
 size_t moe_backward_workspace_size(const moe_shape* shape);
-moe_status moe_backward_act(const moe_shape* shape, const void* d_out, const float* topk_w,
-                            const int32_t* offsets, const int32_t* perm_to_assign,
-                            const int32_t* assign_to_perm, const void* w_down, const void* h,
-                            void* d_h, float* d_w, void* workspace, size_t ws_bytes,
-                            moe_stream_t stream);
+moe_status moe_backward(const moe_shape* shape, const void* d_out, const float* topk_w,
+                        const int32_t* offsets, const int32_t* perm_to_assign,
+                        const int32_t* assign_to_perm, const void* w_gate, const void* w_up,
+                        const void* w_down, const void* h, void* d_h, float* d_w, void* d_x,
+                        void* workspace, size_t ws_bytes, moe_stream_t stream);
 
 /* ----------------------------------------------------------------------------
  * Device status: synchronises `stream`, returns the first device-side fault

@@ -502,11 +502,12 @@ def _bwd_case(tdr, cfg, seed):
     rng = np.random.default_rng(seed)
     d_out = torch.from_numpy(rng.standard_normal((cfg.T, cfg.d)).astype(np.float32)).to(
         torch.bfloat16)
-    d_h, d_w = tdr.backward_act(s, d_out.cuda(), v["topk_w"], v["offsets"], v["perm_to_assign"],
-                                v["assign_to_perm"], cuda(inp.w_down), h)
+    d_h, d_w, d_x = tdr.backward(s, d_out.cuda(), v["topk_w"], v["offsets"], v["perm_to_assign"],
+                                 v["assign_to_perm"], cuda(inp.w_down), h,
+                                 w_gate=cuda(inp.w_gate), w_up=cuda(inp.w_up), input_grad=True)
     torch.cuda.synchronize()
     assert_status_ok(tdr)
-    return inp, s, out_h, v, h, d_out, d_h, d_w
+    return inp, s, out_h, v, h, d_out, d_h, d_w, d_x
 
 
 @pytest.mark.parametrize("T,d,n,E,K,cf", [
@@ -518,7 +519,7 @@ def test_backward_act_matches_oracle(cuda_lib, T, d, n, E, K, cf):
     tdr = cuda_lib
     cfg = mi.MoEConfig("bwd", T=T, d=d, E=E, K=K, n=n, dtype="bf16", capacity_factor=cf,
                        seed=T + n)
-    inp, s, out_h, v, h, d_out, d_h, d_w = _bwd_case(tdr, cfg, 5)
+    inp, s, out_h, v, h, d_out, d_h, d_w, d_x = _bwd_case(tdr, cfg, 5)
     # the forward is the plain one, and h holds the pre-activations
     out_plain, _ = tdr.forward(s, cuda(inp.x), cuda(inp.w_r), cuda(inp.w_gate), cuda(inp.w_up),
                                cuda(inp.w_down))
@@ -537,6 +538,8 @@ def test_backward_act_matches_oracle(cuda_lib, T, d, n, E, K, cf):
     assert_bf16_close(dh[:, :n], dG, "dG")
     assert_bf16_close(dh[:, n:], dU, "dU")
     assert_bf16_close(d_w.cpu().numpy(), dw_ref, "d_w")
+    dx_ref = orc.backward_dx(dG, dU, a2p, p2a, offsets, K, T, inp.w_gate, inp.w_up)
+    assert_bf16_close(d_x.float().cpu().numpy(), dx_ref, "d_x")
     if cf > 0:
         assert np.all(d_w.cpu().numpy().reshape(-1)[a2p < 0] == 0)
 
@@ -544,7 +547,7 @@ def test_backward_act_matches_oracle(cuda_lib, T, d, n, E, K, cf):
 def test_backward_act_full_size_sampled_slots(cuda_lib):
     tdr = cuda_lib
     cfg = mi.CONFIGS["mixtral_bf16"]
-    inp, s, _, v, h, d_out, d_h, d_w = _bwd_case(tdr, cfg, 9)
+    inp, s, _, v, h, d_out, d_h, d_w, d_x = _bwd_case(tdr, cfg, 9)
     offsets = v["offsets"].cpu().numpy()
     p2a = v["perm_to_assign"].cpu().numpy()
     w = v["topk_w"].cpu().numpy().reshape(-1)
@@ -574,6 +577,26 @@ def test_backward_act_full_size_sampled_slots(cuda_lib):
     assert_bf16_close(np.array(got_g), np.array(ref_g), "full-size dG")
     assert_bf16_close(np.array(got_u), np.array(ref_u), "full-size dU")
     assert_bf16_close(np.array(got_w), np.array(ref_w), "full-size d_w")
+    # the input gradient of a few tokens: every kept slot of the token, in slot order
+    a2p = v["assign_to_perm"].cpu().numpy().reshape(cfg.T, K)
+    ids = v["topk_ids"].cpu().numpy()
+    toks = rng.choice(cfg.T, size=3, replace=False)
+    ref_dx = np.zeros((toks.size, cfg.d))
+    for i, t in enumerate(toks):
+        xt = orc.as_f64(inp.x[t])
+        for k in range(K):
+            if a2p[t, k] < 0:
+                continue
+            e = int(ids[t, k])
+            g = xt @ orc.as_f64(inp.w_gate[e])
+            u = xt @ orc.as_f64(inp.w_up[e])
+            sg = 1.0 / (1.0 + np.exp(-g))
+            dA = w[t * K + k] * (dO[t] @ orc.as_f64(inp.w_down[e]).T)
+            dG = dA * u * sg * (1.0 + g * (1.0 - sg))
+            dU = dA * g * sg
+            ref_dx[i] += dG @ orc.as_f64(inp.w_gate[e]).T + dU @ orc.as_f64(inp.w_up[e]).T
+    assert_bf16_close(d_x[torch.from_numpy(toks).cuda()].float().cpu().numpy(), ref_dx,
+                      "full-size d_x")
 
 
 @pytest.mark.parametrize("T", mi.DISPATCH_COMBINE_T)

@@ -60,8 +60,8 @@ _SIGS = {
     "moe_forward_h": (ctypes.c_int, [_S, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P,
                                      ctypes.c_size_t, _P]),
     "moe_backward_workspace_size": (ctypes.c_size_t, [_S]),
-    "moe_backward_act": (ctypes.c_int, [_S, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P,
-                                        ctypes.c_size_t, _P]),
+    "moe_backward": (ctypes.c_int, [_S, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P,
+                                    ctypes.c_size_t, _P]),
     "moe_get_device_status": (ctypes.c_int, [_P]),
     "moe_status_string": (ctypes.c_char_p, [ctypes.c_int]),
     "moe_profile_enable": (ctypes.c_int, [ctypes.c_int]),
@@ -380,9 +380,11 @@ def forward_h(shape: moe_shape, x, w_r, w_gate, w_up, w_down, bias=None, logits_
     return out, workspace, h
 
 
-def backward_act(shape: moe_shape, d_out, topk_w, offsets, perm_to_assign, assign_to_perm,
-                 w_down, h, d_h=None, d_w=None, workspace=None):
-    """moe_backward_act. Returns (d_h [T*K, 2n] = dG | dU per kept slot, d_w [T, K])."""
+def backward(shape: moe_shape, d_out, topk_w, offsets, perm_to_assign, assign_to_perm,
+             w_down, h, w_gate=None, w_up=None, d_h=None, d_w=None, d_x=None,
+             input_grad: bool = False, workspace=None):
+    """moe_backward. Returns (d_h [T*K, 2n] = dG | dU per kept slot, d_w [T, K], d_x [T, d]
+    or None); the input gradient is computed when input_grad (then w_gate, w_up needed)."""
     lib = load_library()
     T, d, E, n, K = shape.T, shape.d, shape.E, shape.n, shape.K
     dt = _act_dtype(shape)
@@ -394,14 +396,21 @@ def backward_act(shape: moe_shape, d_out, topk_w, offsets, perm_to_assign, assig
         d_h = torch.empty(T * K, 2 * n, dtype=dt, device=dev)
     if d_w is None:
         d_w = torch.empty(T, K, dtype=torch.float32, device=dev)
+    if input_grad:
+        _dev(w_gate, "w_gate", dt, (E, d, n))
+        _dev(w_up, "w_up", dt, (E, d, n))
+        if d_x is None:
+            d_x = torch.empty(T, d, dtype=dt, device=dev)
+    else:
+        d_x = None
     need = int(lib.moe_backward_workspace_size(ctypes.byref(shape)))
     if workspace is None:
         workspace = torch.empty(max(need, 256), dtype=torch.uint8, device=dev)
-    _check(lib.moe_backward_act(ctypes.byref(shape), _ptr(d_out), _ptr(topk_w), _ptr(offsets),
-                                _ptr(perm_to_assign), _ptr(assign_to_perm), _ptr(w_down), _ptr(h),
-                                _ptr(d_h), _ptr(d_w), _ptr(workspace), workspace.numel(),
-                                _stream()), "moe_backward_act")
-    return d_h, d_w
+    _check(lib.moe_backward(ctypes.byref(shape), _ptr(d_out), _ptr(topk_w), _ptr(offsets),
+                            _ptr(perm_to_assign), _ptr(assign_to_perm), _ptr(w_gate), _ptr(w_up),
+                            _ptr(w_down), _ptr(h), _ptr(d_h), _ptr(d_w), _ptr(d_x),
+                            _ptr(workspace), workspace.numel(), _stream()), "moe_backward")
+    return d_h, d_w, d_x
 
 
 def workspace_views(shape: moe_shape, workspace: torch.Tensor) -> dict:

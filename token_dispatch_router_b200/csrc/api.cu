@@ -28,11 +28,12 @@ moe_status launch_ffn_tc_mixed(const moe_shape& s, const void* x, const int32_t*
                                const int32_t* p2a, const void* w_gate, const void* w_up,
                                const void* w_down, void* a_act, void* y_perm, int gateup_mode,
                                bool pair_down, void* h_out, cudaStream_t st);
-size_t backward_scratch_bytes(const moe_shape& s);
-moe_status launch_backward_act(const moe_shape& s, const void* d_out, const float* topk_w,
-                               const int32_t* offsets, const int32_t* p2a, const int32_t* a2p,
-                               const void* w_down, const void* h, void* d_h, float* d_w,
-                               void* scratch, cudaStream_t st);
+size_t backward_scratch_bytes(const moe_shape& s, bool with_dx);
+moe_status launch_backward(const moe_shape& s, const void* d_out, const float* topk_w,
+                           const int32_t* offsets, const int32_t* p2a, const int32_t* a2p,
+                           const void* w_gate, const void* w_up, const void* w_down,
+                           const void* h, void* d_h, float* d_w, void* d_x, void* scratch,
+                           cudaStream_t st);
 moe_status launch_permute_static(const moe_shape& s, const int32_t* ids, int32_t* counts,
                                  int32_t* offsets, int32_t* a2p, int32_t* p2a, const void* x,
                                  void* x_perm, cudaStream_t st);
@@ -92,7 +93,7 @@ const char* kKernelNames[K_COUNT] = {
     "route",        "hist",          "scan",           "scatter",     "gather_rows", "gateup_tc",
     "down_tc",      "gateup_simt",   "down_simt",      "combine",     "selftest_timeout",
     "route_tc",     "permute_small", "gateup_tc2",   "down_tc2",
-    "permute_cluster", "route_permute", "tile_round", "bwd_act", "bwd_dw"};
+    "permute_cluster", "route_permute", "tile_round", "bwd_act", "bwd_dw", "bwd_dx"};
 
 struct ProfRec {
   int kid;
@@ -450,14 +451,14 @@ moe_status moe_forward_h(const moe_shape* s, const void* x, const void* w_r, con
 
 size_t moe_backward_workspace_size(const moe_shape* s) {
   if (check_shape(s, true, true) != MOE_OK) return 0;
-  return align256(backward_scratch_bytes(*s)) + 256;
+  return align256(backward_scratch_bytes(*s, true)) + 256;
 }
 
-moe_status moe_backward_act(const moe_shape* s, const void* d_out, const float* topk_w,
-                            const int32_t* offsets, const int32_t* perm_to_assign,
-                            const int32_t* assign_to_perm, const void* w_down, const void* h,
-                            void* d_h, float* d_w, void* workspace, size_t ws_bytes,
-                            moe_stream_t stream) {
+moe_status moe_backward(const moe_shape* s, const void* d_out, const float* topk_w,
+                        const int32_t* offsets, const int32_t* perm_to_assign,
+                        const int32_t* assign_to_perm, const void* w_gate, const void* w_up,
+                        const void* w_down, const void* h, void* d_h, float* d_w, void* d_x,
+                        void* workspace, size_t ws_bytes, moe_stream_t stream) {
   moe_status r = check_shape(s, true, true);
   if (r != MOE_OK) return r;
   if (s->dtype != MOE_BF16) return MOE_ERR_UNSUPPORTED;
@@ -467,10 +468,14 @@ moe_status moe_backward_act(const moe_shape* s, const void* d_out, const float* 
     return MOE_ERR_INVALID_ARG;
   if (!aligned16(d_out) || !aligned16(w_down) || !aligned16(h) || !aligned16(d_h))
     return MOE_ERR_INVALID_ARG;
-  const size_t need = backward_scratch_bytes(*s);
-  if (workspace == nullptr || ws_bytes < need) return MOE_ERR_WORKSPACE;
-  return launch_backward_act(*s, d_out, topk_w, offsets, perm_to_assign, assign_to_perm, w_down,
-                             h, d_h, d_w, workspace, (cudaStream_t)stream);
+  if (d_x != nullptr && (!w_gate || !w_up || !aligned16(w_gate) || !aligned16(w_up) ||
+                         !aligned16(d_x)))
+    return MOE_ERR_INVALID_ARG;
+  const size_t need = backward_scratch_bytes(*s, d_x != nullptr);
+  if (workspace == nullptr || ws_bytes < need || ((uintptr_t)workspace & 255) != 0)
+    return MOE_ERR_WORKSPACE;
+  return launch_backward(*s, d_out, topk_w, offsets, perm_to_assign, assign_to_perm, w_gate,
+                         w_up, w_down, h, d_h, d_w, d_x, workspace, (cudaStream_t)stream);
 }
 
 moe_status moe_get_device_status(moe_stream_t stream) {

@@ -3,7 +3,8 @@
 // SonicMoE explainer (gitcode.csdn.net), section 3 item 6: scatter/combine back to the
 // token-major layout; section 6.1: the aggregation kernel fuses the scatter and the sum.
 //   out[t] = sum_{k, assign_to_perm[t*K+k] >= 0} topk_w[t,k] * y_perm[assign_to_perm[t*K+k]]
-// fp32 accumulation in k order (deterministic); dropped slots add nothing.
+// fp32 accumulation in k order (deterministic); dropped slots add nothing. With no weights
+// (topk_w NULL, the backward's scatter-add of the input gradient) every slot counts once.
 //
 // HBM-bound. One warp owns a 2 KB segment (128 16-byte vectors) of one token's output row:
 // the token's K slots and weights are loaded once per lane (same addresses across the warp),
@@ -51,7 +52,7 @@ __global__ void __launch_bounds__(256) combine_kernel(const uint4* __restrict__ 
             if (lane == 0) report(status, MOE_ERR_DEVICE_INDEX);
             p[h] = -1;
           }
-          if (p[h] >= 0) w[h] = topk_w[t * K + k0 + h];
+          if (p[h] >= 0) w[h] = topk_w != nullptr ? topk_w[t * K + k0 + h] : 1.f;
         }
       }
       uint4 r[2][4];

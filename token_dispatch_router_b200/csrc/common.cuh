@@ -106,6 +106,7 @@ enum KernelId {
   K_TILE_ROUND,
   K_BWD_ACT,
   K_BWD_DW,
+  K_BWD_DX,
   K_COUNT
 };
 

@@ -23,6 +23,8 @@
 //              partial[p][n-tile] (fp32).
 // A second kernel adds each slot's parts in n-tile order (deterministic) and writes the
 // routing-weight gradient d_w[t, k] (0 at dropped slots). Every mbarrier wait is bounded.
+#include <string.h>
+
 #include "ffn_args.cuh"
 #include "tc_ptx.cuh"
 
@@ -36,7 +38,8 @@ constexpr int BM = 128, BK = 64, BN = 256, STAGES = 4;
 constexpr int A_BYTES = BM * BK * 2;  // 16 KB: 128 dO rows x 64 of d
 constexpr int B_BYTES = BN * BK * 2;  // 32 KB: 256 W_down rows (n) x 64 of d
 constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
-constexpr int THREADS = 320;
+constexpr int THREADS_DACT = 320;  // producer, MMA, 4 epilogue warps, 4 gather warps
+constexpr int THREADS_DX = 192;    // producer, MMA, 4 epilogue warps
 constexpr int GATHER_WARP0 = 6;
 constexpr int GATHER_THREADS = 128;
 constexpr uint32_t TMEM_COLS = 512;
@@ -51,13 +54,15 @@ constexpr uint32_t IDESC =
 struct BwdArgs {
   const int32_t* offsets;    // [E + 1]
   const int32_t* p2a;        // slot -> flat assignment
-  const uint8_t* d_out;      // [T, d] rows gathered by token
+  const uint8_t* d_out;      // dA': [T, d] rows gathered by token
   long long row_bytes;       // d * 2
   const float* topk_w;       // [T * K]
   const bf16* h;             // [rows, 2n]: g | u per kept slot
-  bf16* d_h;                 // [rows, 2n]: dG | dU per kept slot
-  float* partial;            // [rows, n_tiles]
-  int n, n_tiles, kblocks, E, K, T;
+  bf16* d_h;                 // dA': [rows, 2n] out (dG | dU); dX: unused
+  float* partial;            // dA': [rows, n_tiles]
+  bf16* dx_perm;             // dX: [rows, d] out
+  int n;                     // dA': output columns (n); dX: output columns (d)
+  int n_tiles, kblocks, kb_split, E, K, T;  // dX: k-blocks < kb_split read W_gate, then W_up
   unsigned* status;
   unsigned long long limit_ns;
 };
@@ -85,8 +90,14 @@ __device__ __forceinline__ Tile decode(int w, const int* s_off, const int* s_cum
   return t;
 }
 
-__global__ void __launch_bounds__(THREADS, 1)
-    grouped_gemm_bwd(const __grid_constant__ CUtensorMap tmB, const BwdArgs g) {
+// MODE 0 (dA'): A = rows of dO gathered by token, B = W_down[e] (K = d), epilogue above.
+// MODE 1 (dX): A = the (dG | dU) rows by TMA, B = W_gate[e] for the first n of K and W_up[e]
+// for the second (K = 2n), both read K-major in place; epilogue: bf16 dX_perm rows.
+template <int MODE>
+__global__ void __launch_bounds__(MODE == 0 ? THREADS_DACT : THREADS_DX, 1)
+    grouped_gemm_bwd(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                     const __grid_constant__ CUtensorMap tmB2, const BwdArgs g) {
+  constexpr int THREADS = MODE == 0 ? THREADS_DACT : THREADS_DX;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* base = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
   uint8_t* ring = base;
@@ -104,7 +115,9 @@ __global__ void __launch_bounds__(THREADS, 1)
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int E = g.E;
-  constexpr uint32_t FULL_COUNT = 1 + GATHER_THREADS;  // TMA expect_tx + gather threads
+  // TMA expect_tx (+ the gather threads' cp.async arrivals in MODE 0)
+  constexpr uint32_t FULL_COUNT = MODE == 0 ? 1 + GATHER_THREADS : 1;
+  constexpr uint32_t TMA_BYTES = MODE == 0 ? B_BYTES : STAGE_BYTES;
 
   if (tid == 0) {
     for (int s = 0; s < STAGES; ++s) {
@@ -119,7 +132,13 @@ __global__ void __launch_bounds__(THREADS, 1)
     *abort_flag = 0;
     mbar_init_fence();
   }
-  if (tid == 32) asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmB)) : "memory");
+  if (tid == 32) {
+    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmB)) : "memory");
+    if (MODE == 1) {
+      asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmA)) : "memory");
+      asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmB2)) : "memory");
+    }
+  }
   if (warp == 1) tmem_alloc<1>(saddr(tmem_slot), TMEM_COLS);
   pdl_wait();  // the previous kernel in the stream has completed
   pdl_trigger();
@@ -178,8 +197,17 @@ __global__ void __launch_bounds__(THREADS, 1)
         }
         if (lane == 0) {
           const uint32_t fb = saddr(&full[stage]);
-          mbar_expect_tx(fb, B_BYTES);
-          tma_load_3d(saddr(ring + stage * STAGE_BYTES) + A_BYTES, &tmB, kb * BK, t.n0, t.e, fb);
+          const uint32_t a_dst = saddr(ring + stage * STAGE_BYTES);
+          mbar_expect_tx(fb, TMA_BYTES);
+          if (MODE == 0) {
+            tma_load_3d(a_dst + A_BYTES, &tmB, kb * BK, t.n0, t.e, fb);
+          } else {
+            tma_load_2d(a_dst, &tmA, kb * BK, t.m0, fb);
+            if (kb < g.kb_split)
+              tma_load_3d(a_dst + A_BYTES, &tmB, kb * BK, t.n0, t.e, fb);
+            else
+              tma_load_3d(a_dst + A_BYTES, &tmB2, (kb - g.kb_split) * BK, t.n0, t.e, fb);
+          }
         }
         issued_mask |= 1u << stage;
         issued_par = (issued_par & ~(1u << stage)) | (phase << stage);
@@ -217,7 +245,7 @@ __global__ void __launch_bounds__(THREADS, 1)
             ok = false;
             break;
           }
-          fence_proxy_async_smem();  // cp.async (generic) writes -> MMA reads
+          if (MODE == 0) fence_proxy_async_smem();  // cp.async (generic) writes -> MMA reads
           tc_fence_after();
           const uint32_t a_addr = saddr(ring + stage * STAGE_BYTES);
           const uint32_t b_addr = a_addr + A_BYTES;
@@ -240,7 +268,7 @@ __global__ void __launch_bounds__(THREADS, 1)
       while (!mbar_try(saddr(done), 0) && globaltimer_ns() - t0 < limit) {
       }
     }
-  } else if (warp >= GATHER_WARP0) {
+  } else if (MODE == 0 && warp >= GATHER_WARP0) {
     // ------------------------------------------------------------ A gather: rows of dO
     const int gw = warp - GATHER_WARP0;
     const int c = lane & 7;
@@ -315,6 +343,29 @@ __global__ void __launch_bounds__(THREADS, 1)
       const uint32_t tb = tmem_base + (uint32_t)(buf * BN) + ((uint32_t)(q * 32) << 16);
       const bool row_ok = r < t.rows;
       const int p = t.m0 + (row_ok ? r : 0);
+      if (MODE == 1) {  // dX_perm rows, bf16
+        bf16* orow = g.dx_perm + (size_t)p * g.n;
+#pragma unroll 1
+        for (int c = 0; c < BN / 32; ++c) {
+          uint32_t v[32];
+          tmem_ld32(tb + c * 32, v);
+          tmem_ld_wait();
+          const int col = t.n0 + c * 32;
+          if (row_ok && col < g.n) {
+            uint32_t pk[16];
+#pragma unroll
+            for (int j = 0; j < 16; ++j)
+              pk[j] = pack_bf16x2(__uint_as_float(v[2 * j]), __uint_as_float(v[2 * j + 1]));
+            uint4* dst = reinterpret_cast<uint4*>(orow + col);
+#pragma unroll
+            for (int j = 0; j < 4; ++j)
+              dst[j] = make_uint4(pk[4 * j], pk[4 * j + 1], pk[4 * j + 2], pk[4 * j + 3]);
+          }
+        }
+        tc_fence_before();
+        mbar_arrive(saddr(&tempty[buf]));
+        continue;
+      }
       const float wt = row_ok ? g.topk_w[g.p2a[p]] : 0.f;
       const bf16* hrow = g.h + (size_t)p * ld;
       bf16* drow = g.d_h + (size_t)p * ld;
@@ -397,18 +448,31 @@ __global__ void __launch_bounds__(256) dw_kernel(const int32_t* __restrict__ a2p
 
 }  // namespace
 
-size_t backward_scratch_bytes(const moe_shape& s) {
+namespace {
+size_t align256b(size_t v) { return (v + 255) & ~(size_t)255; }
+}  // namespace
+
+// Scratch: the per-slot partial sums of dS, then (when the input gradient is wanted) the
+// dX_perm rows.
+size_t backward_scratch_bytes(const moe_shape& s, bool with_dx) {
   const size_t n_tiles = (size_t)(s.n + BN - 1) / BN;
-  return (size_t)s.T * s.K * n_tiles * sizeof(float);
+  size_t b = align256b((size_t)s.T * s.K * n_tiles * sizeof(float));
+  if (with_dx) b += align256b((size_t)s.T * s.K * s.d * 2);
+  return b;
 }
 
-moe_status launch_backward_act(const moe_shape& s, const void* d_out, const float* topk_w,
-                               const int32_t* offsets, const int32_t* p2a, const int32_t* a2p,
-                               const void* w_down, const void* h, void* d_h, float* d_w,
-                               void* scratch, cudaStream_t st) {
+moe_status launch_combine(const moe_shape& s, const void* y_perm, const int32_t* a2p,
+                          const float* topk_w, void* out, cudaStream_t st);
+
+moe_status launch_backward(const moe_shape& s, const void* d_out, const float* topk_w,
+                           const int32_t* offsets, const int32_t* p2a, const int32_t* a2p,
+                           const void* w_gate, const void* w_up, const void* w_down,
+                           const void* h, void* d_h, float* d_w, void* d_x, void* scratch,
+                           cudaStream_t st) {
   const long long A = (long long)s.T * s.K;
   if (A == 0) return MOE_OK;
-  CUtensorMap mb;
+  CUtensorMap mb, none;
+  memset(&none, 0, sizeof(none));
   {
     const uint64_t dims[3] = {(uint64_t)s.d, (uint64_t)s.n, (uint64_t)s.E};
     const uint64_t str[2] = {(uint64_t)s.d * 2, (uint64_t)s.n * s.d * 2};
@@ -424,20 +488,22 @@ moe_status launch_backward_act(const moe_shape& s, const void* d_out, const floa
   a.h = (const bf16*)h;
   a.d_h = (bf16*)d_h;
   a.partial = (float*)scratch;
+  a.dx_perm = nullptr;
   a.n = s.n;
   a.n_tiles = (s.n + BN - 1) / BN;
   a.kblocks = s.d / BK;
+  a.kb_split = a.kblocks;
   a.E = s.E;
   a.K = s.K;
   a.T = s.T;
   a.status = device_status_ptr();
   a.limit_ns = kWaitLimitNs;
-  if (cudaFuncSetAttribute(grouped_gemm_bwd, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  if (cudaFuncSetAttribute(grouped_gemm_bwd<0>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            SMEM_BYTES) != cudaSuccess)
     return MOE_ERR_CUDA;
   launch_begin(K_BWD_ACT, st);
-  launch_kernel(grouped_gemm_bwd, dim3((unsigned)sm_count()), dim3(THREADS), (size_t)SMEM_BYTES,
-                st, 1, mb, a);
+  launch_kernel(grouped_gemm_bwd<0>, dim3((unsigned)sm_count()), dim3(THREADS_DACT),
+                (size_t)SMEM_BYTES, st, 1, none, mb, none, a);
   moe_status r = launch_end(K_BWD_ACT, st);
   if (r != MOE_OK) return r;
   long long blocks = (A + 255) / 256;
@@ -445,7 +511,38 @@ moe_status launch_backward_act(const moe_shape& s, const void* d_out, const floa
   launch_begin(K_BWD_DW, st);
   launch_kernel(dw_kernel, dim3((unsigned)blocks), dim3(256), 0, st, 1, a2p,
                 (const float*)scratch, a.n_tiles, A, d_w);
-  return launch_end(K_BWD_DW, st);
+  if ((r = launch_end(K_BWD_DW, st)) != MOE_OK) return r;
+  if (d_x == nullptr) return MOE_OK;
+  // input gradient: dX_perm = (dG | dU) [W_gate | W_up]^T per expert, then the scatter-add
+  bf16* dx_perm = (bf16*)((uint8_t*)scratch + backward_scratch_bytes(s, false));
+  CUtensorMap ma, mg, mu;
+  {
+    const uint64_t dims[2] = {2 * (uint64_t)s.n, (uint64_t)A};
+    const uint64_t str[1] = {2 * (uint64_t)s.n * 2};
+    const uint32_t box[2] = {BK, BM};
+    if (!make_map(&ma, d_h, 2, dims, str, box)) return MOE_ERR_CUDA;
+  }
+  {
+    const uint64_t dims[3] = {(uint64_t)s.n, (uint64_t)s.d, (uint64_t)s.E};
+    const uint64_t str[2] = {(uint64_t)s.n * 2, (uint64_t)s.d * s.n * 2};
+    const uint32_t box[3] = {BK, BN, 1};
+    if (!make_map(&mg, w_gate, 3, dims, str, box)) return MOE_ERR_CUDA;
+    if (!make_map(&mu, w_up, 3, dims, str, box)) return MOE_ERR_CUDA;
+  }
+  BwdArgs b = a;
+  b.dx_perm = dx_perm;
+  b.n = s.d;
+  b.n_tiles = (s.d + BN - 1) / BN;
+  b.kblocks = 2 * s.n / BK;
+  b.kb_split = s.n / BK;
+  if (cudaFuncSetAttribute(grouped_gemm_bwd<1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           SMEM_BYTES) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  launch_begin(K_BWD_DX, st);
+  launch_kernel(grouped_gemm_bwd<1>, dim3((unsigned)sm_count()), dim3(THREADS_DX),
+                (size_t)SMEM_BYTES, st, 1, ma, mg, mu, b);
+  if ((r = launch_end(K_BWD_DX, st)) != MOE_OK) return r;
+  return launch_combine(s, dx_perm, a2p, nullptr, d_x, st);  // unit weights: a plain sum
 }
 
 }  // namespace moe
