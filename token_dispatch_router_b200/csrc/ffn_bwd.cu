@@ -370,21 +370,29 @@ __global__ void __launch_bounds__(MODE == 0 ? THREADS_DACT : THREADS_DX, 1)
       const bf16* hrow = g.h + (size_t)p * ld;
       bf16* drow = g.d_h + (size_t)p * ld;
       float ds = 0.f;
-#pragma unroll 1
-      for (int c = 0; c < BN / 32; ++c) {
-        uint32_t v[32];
-        tmem_ld32(tb + c * 32, v);
-        tmem_ld_wait();
+      // g and u of the chunk are loaded one chunk ahead of their use
+      uint4 gq[4], uq[4], gn[4], un[4];
+      auto load_h = [&](int c, uint4 (&gd)[4], uint4 (&ud)[4]) {
         const int col = t.n0 + c * 32;
         if (row_ok && col < g.n) {
-          uint4 gq[4], uq[4];
           const uint4* gs = reinterpret_cast<const uint4*>(hrow + col);
           const uint4* us = reinterpret_cast<const uint4*>(hrow + g.n + col);
 #pragma unroll
           for (int j = 0; j < 4; ++j) {
-            gq[j] = gs[j];
-            uq[j] = us[j];
+            gd[j] = gs[j];
+            ud[j] = us[j];
           }
+        }
+      };
+      load_h(0, gq, uq);
+#pragma unroll 1
+      for (int c = 0; c < BN / 32; ++c) {
+        uint32_t v[32];
+        tmem_ld32(tb + c * 32, v);
+        if (c + 1 < BN / 32) load_h(c + 1, gn, un);
+        tmem_ld_wait();
+        const int col = t.n0 + c * 32;
+        if (row_ok && col < g.n) {
           uint32_t pg[16], pu[16];
 #pragma unroll
           for (int j = 0; j < 4; ++j) {
@@ -416,6 +424,11 @@ __global__ void __launch_bounds__(MODE == 0 ? THREADS_DACT : THREADS_DX, 1)
             gd[j] = make_uint4(pg[4 * j], pg[4 * j + 1], pg[4 * j + 2], pg[4 * j + 3]);
             ud[j] = make_uint4(pu[4 * j], pu[4 * j + 1], pu[4 * j + 2], pu[4 * j + 3]);
           }
+        }
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          gq[j] = gn[j];
+          uq[j] = un[j];
         }
       }
       if (row_ok) g.partial[(size_t)p * g.n_tiles + t.nt] = ds;
