@@ -337,6 +337,46 @@ def backward_dx(dG, dU, assign_to_perm, perm_to_assign, offsets, K: int, T: int,
     return dx
 
 
+def backward_router(d_w, topk_ids_, logits_f32, x, w_r, renormalize: bool = True):
+    """The router's backward with the top-K selection held fixed ([P2] 1.1 Router ->
+    Softmax -> TopK read backwards; [P4] 4.2: the gate is the linear map x W_r + bias).
+      renormalised: w_k = exp(l_{i_k}) / sum_{j in S} exp(l_{i_j})  =>
+        dL/dl_{i_j} = w_j (d_w_j - sum_k w_k d_w_k), 0 off the selected set S;
+      plain: w_k = p_{i_k}, p = softmax over all E  =>
+        dL/dl_e = p_e (g_e - sum_k w_k d_w_k), g_e = d_w of e if selected else 0.
+    Then d_W_r = x^T dL/dl, d_bias = sum_t dL/dl_t, and the router's term of the input
+    gradient d_x = dL/dl W_r^T. Returns (d_logits [T, E], d_w_r [d, E], d_bias [E],
+    d_x [T, d]), fp64."""
+    ids = np.asarray(topk_ids_, dtype=np.int64)
+    T, K = ids.shape
+    lg = as_f64(logits_f32)
+    E = lg.shape[1]
+    gw = as_f64(d_w).reshape(T, K)
+    if renormalize:
+        sel = np.take_along_axis(lg, ids, axis=1)
+        m = sel[:, :1]
+        ex = np.exp(sel - m)
+        w = ex / ex.sum(axis=1, keepdims=True)
+    else:
+        m = lg.max(axis=1, keepdims=True)
+        p = np.exp(lg - m)
+        p /= p.sum(axis=1, keepdims=True)
+        w = np.take_along_axis(p, ids, axis=1)
+    s = np.sum(w * gw, axis=1, keepdims=True)
+    d_logits = np.zeros((T, E), dtype=F64)
+    if renormalize:
+        np.put_along_axis(d_logits, ids, w * (gw - s), axis=1)
+    else:
+        g = np.zeros((T, E), dtype=F64)
+        np.put_along_axis(g, ids, gw, axis=1)
+        d_logits = p * (g - s)
+    xa = as_f64(x)
+    d_w_r = xa.T @ d_logits
+    d_bias = d_logits.sum(axis=0)
+    d_x = d_logits @ as_f64(w_r).T
+    return d_logits, d_w_r, d_bias, d_x
+
+
 def combine(y_perm, assign_to_perm, topk_w, T: int, K: int) -> np.ndarray:
     """[P5] 1 and 3 item 6: out[t] = sum_k w[t,k] * y[assign_to_perm[t*K+k]],
     summed in k order; a dropped slot (-1) adds nothing and the other weights

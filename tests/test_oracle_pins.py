@@ -595,3 +595,39 @@ def test_backward_planted_mistake_is_caught(monkeypatch):
     dG, _, _ = orc.backward_act(d_out, w, a2p, p2a, offsets, K, wd, g, u)
     monkeypatch.undo()
     assert not np.allclose(dG, gg, rtol=1e-6, atol=1e-8)
+
+
+@pytest.mark.parametrize("renorm", [True, False])
+def test_router_backward_matches_autograd(renorm):
+    rng = np.random.default_rng(41)
+    T, d, E, K = 10, 6, 5, 2
+    x = rng.standard_normal((T, d))
+    w_r = rng.standard_normal((d, E))
+    bias = rng.standard_normal(E)
+    d_w = rng.standard_normal((T, K))
+    lg32 = orc.router_logits(x, w_r, bias)
+    ids, _ = orc.route(lg32, K, renorm)
+    # autograd: the weights as a function of x, W_r and the bias with the selection fixed
+    X = torch.from_numpy(x).requires_grad_(True)
+    W = torch.from_numpy(w_r).requires_grad_(True)
+    B = torch.from_numpy(bias).requires_grad_(True)
+    L = X @ W + B
+    L.retain_grad()
+    idx = torch.from_numpy(ids.astype(np.int64))
+    if renorm:
+        wts = torch.softmax(torch.gather(L, 1, idx), dim=1)
+    else:
+        wts = torch.gather(torch.softmax(L, dim=1), 1, idx)
+    (wts * torch.from_numpy(d_w)).sum().backward()
+    # the oracle differentiates at the fp32 logits the selection saw; autograd at the fp64
+    # ones: the same function of nearly the same point
+    d_logits, d_w_r, d_bias, d_x = orc.backward_router(d_w, ids, lg32, x, w_r, renorm)
+    np.testing.assert_allclose(d_logits, L.grad.numpy(), rtol=1e-5, atol=1e-6)
+    np.testing.assert_allclose(d_w_r, W.grad.numpy(), rtol=1e-5, atol=1e-6)
+    np.testing.assert_allclose(d_bias, B.grad.numpy(), rtol=1e-5, atol=1e-6)
+    np.testing.assert_allclose(d_x, X.grad.numpy(), rtol=1e-5, atol=1e-6)
+    if renorm:  # only the selected logits receive a gradient, and each row sums to zero
+        mask = np.zeros((T, E), bool)
+        np.put_along_axis(mask, ids, True, axis=1)
+        assert np.all(d_logits[~mask] == 0)
+    np.testing.assert_allclose(d_logits.sum(axis=1), 0.0, atol=1e-12)
