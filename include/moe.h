@@ -301,6 +301,29 @@ moe_status moe_backward(const moe_shape* shape, const void* d_out, const float* 
                         void* workspace, size_t ws_bytes, moe_stream_t stream);
 
 /* ----------------------------------------------------------------------------
+ * moe_backward_router - the router's backward with the top-K selection held fixed
+ * ("Routing-Free and OmniMoE", section 1.1, Router -> Softmax -> TopK, and "How AI
+ * chips support MoE", chapter 4, section 4.2, the gate x W_r + bias, read backwards).
+ * With s_t = sum_k topk_w[t, k] d_w[t, k]:
+ *   renormalize != 0: d_logits[t, e] = topk_w[t, k] (d_w[t, k] - s_t) at e = topk_ids[t, k],
+ *                     0 at the experts not selected;
+ *   renormalize == 0: d_logits[t, e] = p[t, e] (g - s_t), p = softmax(logits[t]) over all E,
+ *                     g = d_w[t, k] at e = topk_ids[t, k], 0 elsewhere;
+ *   d_w_r = x^T d_logits, d_bias = sum over tokens of d_logits, and (d_x not NULL)
+ *   d_x += d_logits W_r^T (the router's term of the input gradient, added in fp32 to the
+ *   bf16 d_x, e.g. the experts' term from moe_backward).
+ *   x [T, d], w_r [d, E] bf16; logits [T, E] fp32 (read only when renormalize == 0);
+ *   topk_ids, topk_w [T, K] from the forward; d_w [T, K] from moe_backward;
+ *   d_logits [T, E] fp32 out (also the intermediate); d_w_r [d, E] fp32 out;
+ *   d_bias [E] fp32 out or NULL; d_x [T, d] bf16 in/out or NULL (16-byte aligned).
+ * Sums over tokens run in a fixed order (deterministic). bf16 only.
+ */
+moe_status moe_backward_router(const moe_shape* shape, const void* x, const void* w_r,
+                               const float* logits, const int32_t* topk_ids, const float* topk_w,
+                               const float* d_w, float* d_logits, float* d_w_r, float* d_bias,
+                               void* d_x, moe_stream_t stream);
+
+/* ----------------------------------------------------------------------------
  * Device status: synchronises `stream`, returns the first device-side fault
  * recorded since the last call (MOE_OK if none) and clears it.
  */

@@ -599,6 +599,41 @@ def test_backward_act_full_size_sampled_slots(cuda_lib):
                       "full-size d_x")
 
 
+@pytest.mark.parametrize("renorm", [True, False])
+def test_backward_router_matches_oracle(cuda_lib, renorm):
+    tdr = cuda_lib
+    T, d, n, E, K = 700, 256, 128, 16, 3
+    cfg = mi.MoEConfig("rbwd", T=T, d=d, E=E, K=K, n=n, dtype="bf16", seed=77)
+    inp = mi.make_inputs(cfg)
+    bias = mi.zipf_bias(E, 1.2, 1.75)
+    s = tdr.make_shape(T, d, E, K, n, 0.0, renorm, torch.bfloat16)
+    _, ws, h = tdr.forward_h(s, cuda(inp.x), cuda(inp.w_r), cuda(inp.w_gate), cuda(inp.w_up),
+                             cuda(inp.w_down), bias=cuda(bias))
+    v = tdr.workspace_views(s, ws)
+    rng = np.random.default_rng(8)
+    d_out = torch.from_numpy(rng.standard_normal((T, d)).astype(np.float32)).to(torch.bfloat16)
+    d_h, d_w, d_x = tdr.backward(s, d_out.cuda(), v["topk_w"], v["offsets"], v["perm_to_assign"],
+                                 v["assign_to_perm"], cuda(inp.w_down), h, w_gate=cuda(inp.w_gate),
+                                 w_up=cuda(inp.w_up), input_grad=True)
+    dx_experts = d_x.float().cpu().numpy()
+    d_logits, d_w_r, d_bias = tdr.backward_router(s, cuda(inp.x), cuda(inp.w_r), v["topk_ids"],
+                                                  v["topk_w"], d_w, logits=v["logits"], d_x=d_x,
+                                                  with_bias=True)
+    torch.cuda.synchronize()
+    assert_status_ok(tdr)
+    ref = orc.backward_router(d_w.cpu().numpy(), v["topk_ids"].cpu().numpy(),
+                              v["logits"].cpu().numpy(), inp.x, inp.w_r, renorm)
+    np.testing.assert_allclose(d_logits.cpu().numpy(), ref[0], rtol=1e-4, atol=1e-6)
+    np.testing.assert_allclose(d_w_r.cpu().numpy(), ref[1], rtol=1e-3, atol=1e-4)
+    np.testing.assert_allclose(d_bias.cpu().numpy(), ref[2], rtol=1e-3, atol=1e-4)
+    assert_bf16_close(d_x.float().cpu().numpy() - dx_experts, ref[3], "router term of d_x")
+    if renorm:
+        ids = v["topk_ids"].cpu().numpy()
+        mask = np.zeros((T, E), bool)
+        np.put_along_axis(mask, ids, True, axis=1)
+        assert np.all(d_logits.cpu().numpy()[~mask] == 0)
+
+
 @pytest.mark.parametrize("T", mi.DISPATCH_COMBINE_T)
 def test_dispatch_combine_identity_experts(cuda_lib, T):
     """route (given logits) -> permute with x_perm -> combine(y_perm = x_perm) returns x."""

@@ -60,6 +60,7 @@ _SIGS = {
     "moe_forward_h": (ctypes.c_int, [_S, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P,
                                      ctypes.c_size_t, _P]),
     "moe_backward_workspace_size": (ctypes.c_size_t, [_S]),
+    "moe_backward_router": (ctypes.c_int, [_S, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P]),
     "moe_backward": (ctypes.c_int, [_S, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P,
                                     ctypes.c_size_t, _P]),
     "moe_get_device_status": (ctypes.c_int, [_P]),
@@ -411,6 +412,28 @@ def backward(shape: moe_shape, d_out, topk_w, offsets, perm_to_assign, assign_to
                             _ptr(w_down), _ptr(h), _ptr(d_h), _ptr(d_w), _ptr(d_x),
                             _ptr(workspace), workspace.numel(), _stream()), "moe_backward")
     return d_h, d_w, d_x
+
+
+def backward_router(shape: moe_shape, x, w_r, topk_ids, topk_w, d_w, logits=None, d_x=None,
+                    with_bias: bool = False):
+    """moe_backward_router. Adds the router's term into d_x when given. Returns (d_logits
+    [T, E], d_w_r [d, E], d_bias [E] or None)."""
+    lib = load_library()
+    T, d, E = shape.T, shape.d, shape.E
+    dt = _act_dtype(shape)
+    _dev(x, "x", dt, (T, d))
+    _dev(w_r, "w_r", dt, (d, E))
+    dev = x.device
+    d_logits = torch.empty(T, E, dtype=torch.float32, device=dev)
+    d_w_r = torch.empty(d, E, dtype=torch.float32, device=dev)
+    d_bias = torch.empty(E, dtype=torch.float32, device=dev) if with_bias else None
+    if d_x is not None:
+        _dev(d_x, "d_x", dt, (T, d))
+    _check(lib.moe_backward_router(ctypes.byref(shape), _ptr(x), _ptr(w_r), _ptr(logits),
+                                   _ptr(topk_ids), _ptr(topk_w), _ptr(d_w), _ptr(d_logits),
+                                   _ptr(d_w_r), _ptr(d_bias), _ptr(d_x), _stream()),
+           "moe_backward_router")
+    return d_logits, d_w_r, d_bias
 
 
 def workspace_views(shape: moe_shape, workspace: torch.Tensor) -> dict:

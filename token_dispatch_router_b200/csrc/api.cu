@@ -29,6 +29,10 @@ moe_status launch_ffn_tc_mixed(const moe_shape& s, const void* x, const int32_t*
                                const void* w_down, void* a_act, void* y_perm, int gateup_mode,
                                bool pair_down, void* h_out, cudaStream_t st);
 size_t backward_scratch_bytes(const moe_shape& s, bool with_dx);
+moe_status launch_router_backward(const moe_shape& s, const void* x, const void* w_r,
+                                  const float* logits, const int32_t* ids, const float* topk_w,
+                                  const float* d_w, float* d_logits, float* d_w_r,
+                                  float* d_bias, void* d_x, cudaStream_t st);
 moe_status launch_backward(const moe_shape& s, const void* d_out, const float* topk_w,
                            const int32_t* offsets, const int32_t* p2a, const int32_t* a2p,
                            const void* w_gate, const void* w_up, const void* w_down,
@@ -93,7 +97,8 @@ const char* kKernelNames[K_COUNT] = {
     "route",        "hist",          "scan",           "scatter",     "gather_rows", "gateup_tc",
     "down_tc",      "gateup_simt",   "down_simt",      "combine",     "selftest_timeout",
     "route_tc",     "permute_small", "gateup_tc2",   "down_tc2",
-    "permute_cluster", "route_permute", "tile_round", "bwd_act", "bwd_dw", "bwd_dx"};
+    "permute_cluster", "route_permute", "tile_round", "bwd_act", "bwd_dw", "bwd_dx",
+    "router_dlogits", "router_dwr", "router_dx"};
 
 struct ProfRec {
   int kid;
@@ -476,6 +481,29 @@ moe_status moe_backward(const moe_shape* s, const void* d_out, const float* topk
     return MOE_ERR_WORKSPACE;
   return launch_backward(*s, d_out, topk_w, offsets, perm_to_assign, assign_to_perm, w_gate,
                          w_up, w_down, h, d_h, d_w, d_x, workspace, (cudaStream_t)stream);
+}
+
+moe_status moe_backward_router(const moe_shape* s, const void* x, const void* w_r,
+                               const float* logits, const int32_t* topk_ids, const float* topk_w,
+                               const float* d_w, float* d_logits, float* d_w_r, float* d_bias,
+                               void* d_x, moe_stream_t stream) {
+  moe_status r = check_shape(s, true, false);
+  if (r != MOE_OK) return r;
+  if (s->dtype != MOE_BF16) return MOE_ERR_UNSUPPORTED;
+  if (s->T == 0) {  // nothing routed: the weight and bias gradients are zero
+    if (d_w_r == nullptr) return MOE_ERR_INVALID_ARG;
+    const cudaStream_t st = (cudaStream_t)stream;
+    if (cudaMemsetAsync(d_w_r, 0, sizeof(float) * (size_t)s->d * s->E, st) != cudaSuccess)
+      return MOE_ERR_CUDA;
+    if (d_bias != nullptr && cudaMemsetAsync(d_bias, 0, sizeof(float) * s->E, st) != cudaSuccess)
+      return MOE_ERR_CUDA;
+    return MOE_OK;
+  }
+  if (!x || !w_r || !topk_ids || !topk_w || !d_w || !d_logits || !d_w_r) return MOE_ERR_INVALID_ARG;
+  if (!s->renormalize && logits == nullptr) return MOE_ERR_INVALID_ARG;  // the plain softmax
+  if (d_x != nullptr && !aligned16(d_x)) return MOE_ERR_INVALID_ARG;
+  return launch_router_backward(*s, x, w_r, logits, topk_ids, topk_w, d_w, d_logits, d_w_r,
+                                d_bias, d_x, (cudaStream_t)stream);
 }
 
 moe_status moe_get_device_status(moe_stream_t stream) {

@@ -107,6 +107,9 @@ enum KernelId {
   K_BWD_ACT,
   K_BWD_DW,
   K_BWD_DX,
+  K_ROUTER_DLOGITS,
+  K_ROUTER_DWR,
+  K_ROUTER_DX,
   K_COUNT
 };
 

@@ -1,0 +1,229 @@
+// The router's backward with the top-K selection held fixed.
+//
+// "Two upstream innovations of MoE: Routing-Free and OmniMoE", section 1.1 (Router ->
+// Softmax -> TopK) and "How AI chips support MoE", chapter 4, section 4.2 (the gate is the
+// linear map x W_r + bias), read backwards. With d_w = dL/dw[t, k] (from the expert half's
+// backward) and s_t = sum_k w[t, k] d_w[t, k]:
+//   renormalised top-K softmax: dL/dl[t, e] = w[t, k] (d_w[t, k] - s_t) if e = id[t, k],
+//                               0 for an expert that was not selected;
+//   plain softmax over all E:   dL/dl[t, e] = p[t, e] (g[t, e] - s_t), g = d_w at the
+//                               selected experts, 0 elsewhere;
+//   d_W_r = x^T dL/dl, d_bias = sum_t dL/dl[t, :], and the router's term of the input
+//   gradient dL/dl W_r^T, added to d_x.
+// Three kernels: one warp per token for dL/dl (the K selections are held one per lane and
+// broadcast by shuffles; a warp max and sum give the plain softmax); d_W_r and d_bias by
+// CTAs that own 32 columns of W_r and EC experts and sum over all tokens in a fixed order
+// (eight token groups, then the groups in order: deterministic); the input-gradient term
+// by CTAs that own 64 columns of d with that slice of W_r in shared memory, 8 threads per
+// token row slice, fp32 sums added to the bf16 d_x.
+#include <math.h>
+
+#include "common.cuh"
+
+namespace moe {
+
+namespace {
+
+__global__ void __launch_bounds__(256) router_dlogits_kernel(
+    const int32_t* __restrict__ ids, const float* __restrict__ topk_w,
+    const float* __restrict__ d_w, const float* __restrict__ logits, int T, int E, int K,
+    int renorm, float* __restrict__ d_logits) {
+  pdl_wait();  // the previous kernel in the stream has completed
+  pdl_trigger();
+  const int lane = threadIdx.x & 31;
+  const int warps = (int)(gridDim.x * (blockDim.x >> 5));
+  for (int t = (int)(blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5)); t < T; t += warps) {
+    int id = -1;
+    float w = 0.f, g = 0.f;
+    if (lane < K) {
+      id = ids[(size_t)t * K + lane];
+      w = topk_w[(size_t)t * K + lane];
+      g = d_w[(size_t)t * K + lane];
+    }
+    float s = w * g;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+    // plain softmax: p over all E (max and sum over the warp)
+    float m = -INFINITY, den = 0.f;
+    if (!renorm) {
+      for (int e = lane; e < E; e += 32) m = fmaxf(m, logits[(size_t)t * E + e]);
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+      for (int e = lane; e < E; e += 32) den += expf(logits[(size_t)t * E + e] - m);
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) den += __shfl_xor_sync(0xffffffffu, den, o);
+    }
+    for (int e0 = 0; e0 < E; e0 += 32) {  // warp-uniform
+      const int e = e0 + lane;
+      float ge = 0.f, we = 0.f;
+      bool sel = false;
+      for (int k = 0; k < K; ++k) {
+        const int ik = __shfl_sync(0xffffffffu, id, k);
+        const float wk = __shfl_sync(0xffffffffu, w, k);
+        const float gk = __shfl_sync(0xffffffffu, g, k);
+        if (ik == e) {
+          sel = true;
+          we = wk;
+          ge = gk;
+        }
+      }
+      if (e < E) {
+        float v;
+        if (renorm) v = sel ? we * (ge - s) : 0.f;
+        else v = expf(logits[(size_t)t * E + e] - m) / den * (ge - s);
+        d_logits[(size_t)t * E + e] = v;
+      }
+    }
+  }
+}
+
+// d_W_r[j, e] = sum_t x[t, j] dl[t, e]; d_bias[e] = sum_t dl[t, e] (CTAs of column block 0).
+// CTA: 32 columns of x (one per lane) x EC experts; warp w sums the tokens t = w (mod 8).
+template <int EC>
+__global__ void __launch_bounds__(256) router_dwr_kernel(const bf16* __restrict__ x,
+                                                         const float* __restrict__ dl, int T,
+                                                         int d, int E, float* __restrict__ d_w_r,
+                                                         float* __restrict__ d_bias) {
+  __shared__ float red[8][32][EC + 1];
+  __shared__ float redb[8][EC + 1];
+  pdl_wait();  // the previous kernel in the stream has completed
+  pdl_trigger();
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int j = blockIdx.x * 32 + lane;  // column of x / row of W_r
+  const int e0 = blockIdx.y * EC;
+  const bool bias_cta = blockIdx.x == 0 && d_bias != nullptr;
+  float acc[EC], accb[EC];
+#pragma unroll
+  for (int q = 0; q < EC; ++q) acc[q] = accb[q] = 0.f;
+  for (int t = warp; t < T; t += 8) {
+    const float xv = j < d ? __bfloat162float(x[(size_t)t * d + j]) : 0.f;
+    const float dv = (lane < EC && e0 + lane < E) ? dl[(size_t)t * E + e0 + lane] : 0.f;
+#pragma unroll
+    for (int q = 0; q < EC; ++q) {
+      const float dq = __shfl_sync(0xffffffffu, dv, q);
+      acc[q] = fmaf(xv, dq, acc[q]);
+      if (bias_cta) accb[q] += dq;
+    }
+  }
+#pragma unroll
+  for (int q = 0; q < EC; ++q) red[warp][lane][q] = acc[q];
+  if (bias_cta && lane == 0)
+#pragma unroll
+    for (int q = 0; q < EC; ++q) redb[warp][q] = accb[q];
+  __syncthreads();
+  for (int i = threadIdx.x; i < 32 * EC; i += 256) {
+    const int c = i / EC, q = i % EC;
+    float v = 0.f;
+#pragma unroll
+    for (int w = 0; w < 8; ++w) v += red[w][c][q];  // token groups in order
+    const int jj = blockIdx.x * 32 + c, e = e0 + q;
+    if (jj < d && e < E) d_w_r[(size_t)jj * E + e] = v;
+  }
+  if (bias_cta && threadIdx.x < EC && e0 + (int)threadIdx.x < E) {
+    float v = 0.f;
+#pragma unroll
+    for (int w = 0; w < 8; ++w) v += redb[w][threadIdx.x];
+    d_bias[e0 + threadIdx.x] = v;
+  }
+}
+
+// d_x[t, j] += sum_e dl[t, e] W_r[j, e]. CTA: 64 columns of d (its W_r slice in shared
+// memory, fp32, expert-major), 8 threads per token row slice (8 columns each, one 16-byte
+// vector of d_x).
+__global__ void __launch_bounds__(256) router_dx_kernel(const bf16* __restrict__ w_r,
+                                                        const float* __restrict__ dl, int T,
+                                                        int d, int E, int tokens_per_cta,
+                                                        bf16* __restrict__ d_x) {
+  extern __shared__ float wsl[];  // [E][64]: expert-major, a thread's 8 columns contiguous
+  pdl_wait();  // the previous kernel in the stream has completed
+  pdl_trigger();
+  const int j0 = blockIdx.x * 64;
+  for (int i = threadIdx.x; i < 64 * E; i += 256) {
+    const int r = i / E, e = i % E;
+    wsl[e * 64 + r] = (j0 + r < d) ? __bfloat162float(w_r[(size_t)(j0 + r) * E + e]) : 0.f;
+  }
+  __syncthreads();
+  const int sub = threadIdx.x & 7;   // 8 columns [j0 + 8 sub, +8)
+  const int row = threadIdx.x >> 3;  // 32 tokens per pass
+  const int t_begin = blockIdx.y * tokens_per_cta;
+  const int t_end = min(T, t_begin + tokens_per_cta);
+  const int jj = j0 + sub * 8;
+  if (jj >= d) return;
+  for (int t = t_begin + row; t < t_end; t += 32) {
+    float acc[8];
+#pragma unroll
+    for (int c = 0; c < 8; ++c) acc[c] = 0.f;
+    const float* dlt = dl + (size_t)t * E;
+    for (int e = 0; e < E; ++e) {
+      const float v = dlt[e];
+      const float4 w0 = *reinterpret_cast<const float4*>(wsl + e * 64 + sub * 8);
+      const float4 w1 = *reinterpret_cast<const float4*>(wsl + e * 64 + sub * 8 + 4);
+      acc[0] = fmaf(v, w0.x, acc[0]);
+      acc[1] = fmaf(v, w0.y, acc[1]);
+      acc[2] = fmaf(v, w0.z, acc[2]);
+      acc[3] = fmaf(v, w0.w, acc[3]);
+      acc[4] = fmaf(v, w1.x, acc[4]);
+      acc[5] = fmaf(v, w1.y, acc[5]);
+      acc[6] = fmaf(v, w1.z, acc[6]);
+      acc[7] = fmaf(v, w1.w, acc[7]);
+    }
+    uint4* px = reinterpret_cast<uint4*>(d_x + (size_t)t * d + jj);
+    float cur[8];
+    unpack16(*px, cur, bf16());
+#pragma unroll
+    for (int c = 0; c < 8; ++c) cur[c] += acc[c];
+    *px = pack16(cur, bf16());
+  }
+}
+
+}  // namespace
+
+moe_status launch_router_backward(const moe_shape& s, const void* x, const void* w_r,
+                                  const float* logits, const int32_t* ids, const float* topk_w,
+                                  const float* d_w, float* d_logits, float* d_w_r,
+                                  float* d_bias, void* d_x, cudaStream_t st) {
+  const int T = s.T, d = s.d, E = s.E, K = s.K;
+  moe_status r;
+  {
+    long long blocks = ((long long)T + 7) / 8;
+    if (blocks > (long long)sm_count() * 8) blocks = (long long)sm_count() * 8;
+    launch_begin(K_ROUTER_DLOGITS, st);
+    launch_kernel(router_dlogits_kernel, dim3((unsigned)blocks), dim3(256), 0, st, 1, ids, topk_w,
+                  d_w, logits, T, E, K, s.renormalize, d_logits);
+    if ((r = launch_end(K_ROUTER_DLOGITS, st)) != MOE_OK) return r;
+  }
+  {
+    const int EC = E <= 8 ? 8 : (E <= 16 ? 16 : 32);
+    const dim3 grid((unsigned)((d + 31) / 32), (unsigned)((E + EC - 1) / EC));
+    launch_begin(K_ROUTER_DWR, st);
+    if (EC == 8)
+      launch_kernel(router_dwr_kernel<8>, grid, dim3(256), 0, st, 1, (const bf16*)x,
+                    (const float*)d_logits, T, d, E, d_w_r, d_bias);
+    else if (EC == 16)
+      launch_kernel(router_dwr_kernel<16>, grid, dim3(256), 0, st, 1, (const bf16*)x,
+                    (const float*)d_logits, T, d, E, d_w_r, d_bias);
+    else
+      launch_kernel(router_dwr_kernel<32>, grid, dim3(256), 0, st, 1, (const bf16*)x,
+                    (const float*)d_logits, T, d, E, d_w_r, d_bias);
+    if ((r = launch_end(K_ROUTER_DWR, st)) != MOE_OK) return r;
+  }
+  if (d_x != nullptr) {
+    const int smem = 64 * E * (int)sizeof(float);
+    if (cudaFuncSetAttribute(router_dx_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             smem) != cudaSuccess)
+      return MOE_ERR_CUDA;
+    const int col_blocks = (d + 63) / 64;
+    int tok_blocks = (sm_count() * 4 + col_blocks - 1) / col_blocks;
+    if (tok_blocks < 1) tok_blocks = 1;
+    const int tpc = (T + tok_blocks - 1) / tok_blocks;
+    tok_blocks = (T + tpc - 1) / tpc;
+    launch_begin(K_ROUTER_DX, st);
+    launch_kernel(router_dx_kernel, dim3((unsigned)col_blocks, (unsigned)tok_blocks), dim3(256),
+                  (size_t)smem, st, 1, (const bf16*)w_r, (const float*)d_logits, T, d, E, tpc,
+                  (bf16*)d_x);
+    if ((r = launch_end(K_ROUTER_DX, st)) != MOE_OK) return r;
+  }
+  return MOE_OK;
+}
+
+}  // namespace moe
