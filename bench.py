@@ -451,9 +451,9 @@ def token_rounding_figure(tdr, cfg, x, w_r, wg, wu, wd, bias, world, R=128, roun
 
 
 def backward_figure(tdr, cfg, s, x, w_r, wg, wu, wd, bias, world, peak_t, steps=20):
-    """The expert-half backward (moe_backward with the input gradient) at the layer's shape,
-    after a moe_forward_h: CUDA events over `steps` calls, per-kernel times from the
-    library's event profiler."""
+    """The layer's backward at its shape, after a moe_forward_h: moe_backward with the input
+    gradient, then moe_backward_router (its term added to d_x); CUDA events over `steps`
+    calls, per-kernel times from the library's event profiler."""
     if cfg.dtype != "bf16":
         return None
     dev = x.device
@@ -473,15 +473,20 @@ def backward_figure(tdr, cfg, s, x, w_r, wg, wu, wd, bias, world, peak_t, steps=
                      v["assign_to_perm"], wd, h, w_gate=wg, w_up=wu, d_h=d_h, d_w=d_w, d_x=d_x,
                      input_grad=True, workspace=bws)
 
-    for _ in range(3):
+    def call_all():
         call()
+        tdr.backward_router(s, x, w_r, v["topk_ids"], v["topk_w"], d_w, logits=v["logits"],
+                            d_x=d_x, with_bias=bias is not None)
+
+    for _ in range(3):
+        call_all()
     torch.cuda.synchronize()
     prof = tdr.Profiler()
     with prof:
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record()
         for _ in range(steps):
-            call()
+            call_all()
         e1.record()
         torch.cuda.synchronize()
     if tdr.device_status() != 0:
@@ -503,10 +508,12 @@ def backward_figure(tdr, cfg, s, x, w_r, wg, wu, wd, bias, world, peak_t, steps=
             "dx_gemm_ms": round(dx_ms, 4), "dx_tflops": round(tf_dx, 2),
             "dx_frac_of_sustained_peak": round(tf_dx / peak_t, 4),
             "dw_ms": round(avg("bwd_dw"), 4), "scatter_add_ms": round(avg("combine"), 4),
+            "router_ms": round(avg("router_dlogits") + avg("router_dwr") + avg("router_dx"), 4),
             "note": "dA' = dO W_down^T (dO gathered by token; dS and the SwiGLU backward in the "
                     "epilogue: reads h, writes d_h), d_w reduction, dX_perm = (dG|dU) "
-                    "(W_gate|W_up)^T, scatter-add to tokens; TFLOP/s on 2*d*n (dA') and "
-                    "4*d*n (dX) per kept slot"}
+                    "(W_gate|W_up)^T, scatter-add to tokens, router backward (d_logits, "
+                    "d_W_r, d_bias, its d_x term); TFLOP/s on 2*d*n (dA') and 4*d*n (dX) per "
+                    "kept slot"}
 
 
 # ------------------------------------------------------------------ our arm
