@@ -508,7 +508,9 @@ def backward_figure(tdr, cfg, s, x, w_r, wg, wu, wd, bias, world, peak_t, steps=
             "dx_gemm_ms": round(dx_ms, 4), "dx_tflops": round(tf_dx, 2),
             "dx_frac_of_sustained_peak": round(tf_dx / peak_t, 4),
             "dw_ms": round(avg("bwd_dw"), 4), "scatter_add_ms": round(avg("combine"), 4),
-            "router_ms": round(avg("router_dlogits") + avg("router_dwr") + avg("router_dx"), 4),
+            "router_ms": {"d_logits": round(avg("router_dlogits"), 4),
+                          "d_w_r_and_bias": round(avg("router_dwr"), 4),
+                          "d_x_term": round(avg("router_dx"), 4)},
             "note": "dA' = dO W_down^T (dO gathered by token; dS and the SwiGLU backward in the "
                     "epilogue: reads h, writes d_h), d_w reduction, dX_perm = (dG|dU) "
                     "(W_gate|W_up)^T, scatter-add to tokens, router backward (d_logits, "

@@ -13,7 +13,7 @@
 // Three kernels: one warp per token for dL/dl (the K selections are held one per lane and
 // broadcast by shuffles; a warp max and sum give the plain softmax); d_W_r and d_bias by
 // CTAs that own 32 columns of W_r and EC experts and sum over all tokens in a fixed order
-// (eight token groups, then the groups in order: deterministic); the input-gradient term
+// (sixteen token groups, then the groups in order: deterministic); the input-gradient term
 // by CTAs that own 64 columns of d with that slice of W_r in shared memory, 8 threads per
 // token row slice, fp32 sums added to the bf16 d_x.
 #include <math.h>
@@ -78,32 +78,43 @@ __global__ void __launch_bounds__(256) router_dlogits_kernel(
 }
 
 // d_W_r[j, e] = sum_t x[t, j] dl[t, e]; d_bias[e] = sum_t dl[t, e] (CTAs of column block 0).
-// CTA: 32 columns of x (one per lane) x EC experts; warp w sums the tokens t = w (mod 8).
+// CTA: 32 columns of x (one per lane) x EC experts; warp w of the 16 sums the tokens
+// t = w (mod 16), eight tokens' loads issued before any is used.
+constexpr int kDwrWarps = 16;
+constexpr int kDwrUnroll = 8;
+
 template <int EC>
-__global__ void __launch_bounds__(256) router_dwr_kernel(const bf16* __restrict__ x,
-                                                         const float* __restrict__ dl, int T,
-                                                         int d, int E, float* __restrict__ d_w_r,
-                                                         float* __restrict__ d_bias) {
-  __shared__ float red[8][32][EC + 1];
-  __shared__ float redb[8][EC + 1];
+__global__ void __launch_bounds__(kDwrWarps * 32) router_dwr_kernel(
+    const bf16* __restrict__ x, const float* __restrict__ dl, int T, int d, int E,
+    float* __restrict__ d_w_r, float* __restrict__ d_bias) {
+  __shared__ float red[kDwrWarps][32][EC + 1];
+  __shared__ float redb[kDwrWarps][EC + 1];
   pdl_wait();  // the previous kernel in the stream has completed
   pdl_trigger();
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int j = blockIdx.x * 32 + lane;  // column of x / row of W_r
   const int e0 = blockIdx.y * EC;
   const bool bias_cta = blockIdx.x == 0 && d_bias != nullptr;
+  const bool ecol = lane < EC && e0 + lane < E;
   float acc[EC], accb[EC];
 #pragma unroll
   for (int q = 0; q < EC; ++q) acc[q] = accb[q] = 0.f;
-  for (int t = warp; t < T; t += 8) {
-    const float xv = j < d ? __bfloat162float(x[(size_t)t * d + j]) : 0.f;
-    const float dv = (lane < EC && e0 + lane < E) ? dl[(size_t)t * E + e0 + lane] : 0.f;
+  for (int t0 = warp; t0 < T; t0 += kDwrWarps * kDwrUnroll) {
+    float xv[kDwrUnroll], dv[kDwrUnroll];
 #pragma unroll
-    for (int q = 0; q < EC; ++q) {
-      const float dq = __shfl_sync(0xffffffffu, dv, q);
-      acc[q] = fmaf(xv, dq, acc[q]);
-      if (bias_cta) accb[q] += dq;
+    for (int u = 0; u < kDwrUnroll; ++u) {
+      const int t = t0 + u * kDwrWarps;
+      xv[u] = (t < T && j < d) ? __bfloat162float(x[(size_t)t * d + j]) : 0.f;
+      dv[u] = (t < T && ecol) ? dl[(size_t)t * E + e0 + lane] : 0.f;
     }
+#pragma unroll
+    for (int u = 0; u < kDwrUnroll; ++u)
+#pragma unroll
+      for (int q = 0; q < EC; ++q) {
+        const float dq = __shfl_sync(0xffffffffu, dv[u], q);
+        acc[q] = fmaf(xv[u], dq, acc[q]);
+        if (bias_cta) accb[q] += dq;
+      }
   }
 #pragma unroll
   for (int q = 0; q < EC; ++q) red[warp][lane][q] = acc[q];
@@ -111,18 +122,18 @@ __global__ void __launch_bounds__(256) router_dwr_kernel(const bf16* __restrict_
 #pragma unroll
     for (int q = 0; q < EC; ++q) redb[warp][q] = accb[q];
   __syncthreads();
-  for (int i = threadIdx.x; i < 32 * EC; i += 256) {
+  for (int i = threadIdx.x; i < 32 * EC; i += kDwrWarps * 32) {
     const int c = i / EC, q = i % EC;
     float v = 0.f;
 #pragma unroll
-    for (int w = 0; w < 8; ++w) v += red[w][c][q];  // token groups in order
+    for (int w = 0; w < kDwrWarps; ++w) v += red[w][c][q];  // token groups in order
     const int jj = blockIdx.x * 32 + c, e = e0 + q;
     if (jj < d && e < E) d_w_r[(size_t)jj * E + e] = v;
   }
   if (bias_cta && threadIdx.x < EC && e0 + (int)threadIdx.x < E) {
     float v = 0.f;
 #pragma unroll
-    for (int w = 0; w < 8; ++w) v += redb[w][threadIdx.x];
+    for (int w = 0; w < kDwrWarps; ++w) v += redb[w][threadIdx.x];
     d_bias[e0 + threadIdx.x] = v;
   }
 }
@@ -154,22 +165,29 @@ __global__ void __launch_bounds__(256) router_dx_kernel(const bf16* __restrict__
 #pragma unroll
     for (int c = 0; c < 8; ++c) acc[c] = 0.f;
     const float* dlt = dl + (size_t)t * E;
-    for (int e = 0; e < E; ++e) {
-      const float v = dlt[e];
-      const float4 w0 = *reinterpret_cast<const float4*>(wsl + e * 64 + sub * 8);
-      const float4 w1 = *reinterpret_cast<const float4*>(wsl + e * 64 + sub * 8 + 4);
-      acc[0] = fmaf(v, w0.x, acc[0]);
-      acc[1] = fmaf(v, w0.y, acc[1]);
-      acc[2] = fmaf(v, w0.z, acc[2]);
-      acc[3] = fmaf(v, w0.w, acc[3]);
-      acc[4] = fmaf(v, w1.x, acc[4]);
-      acc[5] = fmaf(v, w1.y, acc[5]);
-      acc[6] = fmaf(v, w1.z, acc[6]);
-      acc[7] = fmaf(v, w1.w, acc[7]);
-    }
     uint4* px = reinterpret_cast<uint4*>(d_x + (size_t)t * d + jj);
+    const uint4 old = *px;  // issued before the sums that follow
+    for (int ec = 0; ec < E; ec += 8) {  // eight of the token's d_logits loaded together
+      float v[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) v[u] = ec + u < E ? dlt[ec + u] : 0.f;
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        if (ec + u >= E) continue;
+        const float4 w0 = *reinterpret_cast<const float4*>(wsl + (ec + u) * 64 + sub * 8);
+        const float4 w1 = *reinterpret_cast<const float4*>(wsl + (ec + u) * 64 + sub * 8 + 4);
+        acc[0] = fmaf(v[u], w0.x, acc[0]);
+        acc[1] = fmaf(v[u], w0.y, acc[1]);
+        acc[2] = fmaf(v[u], w0.z, acc[2]);
+        acc[3] = fmaf(v[u], w0.w, acc[3]);
+        acc[4] = fmaf(v[u], w1.x, acc[4]);
+        acc[5] = fmaf(v[u], w1.y, acc[5]);
+        acc[6] = fmaf(v[u], w1.z, acc[6]);
+        acc[7] = fmaf(v[u], w1.w, acc[7]);
+      }
+    }
     float cur[8];
-    unpack16(*px, cur, bf16());
+    unpack16(old, cur, bf16());
 #pragma unroll
     for (int c = 0; c < 8; ++c) cur[c] += acc[c];
     *px = pack16(cur, bf16());
@@ -193,17 +211,15 @@ moe_status launch_router_backward(const moe_shape& s, const void* x, const void*
     if ((r = launch_end(K_ROUTER_DLOGITS, st)) != MOE_OK) return r;
   }
   {
-    const int EC = E <= 8 ? 8 : (E <= 16 ? 16 : 32);
+    const int EC = E <= 8 ? 8 : 16;
     const dim3 grid((unsigned)((d + 31) / 32), (unsigned)((E + EC - 1) / EC));
+    const dim3 block(kDwrWarps * 32);
     launch_begin(K_ROUTER_DWR, st);
     if (EC == 8)
-      launch_kernel(router_dwr_kernel<8>, grid, dim3(256), 0, st, 1, (const bf16*)x,
-                    (const float*)d_logits, T, d, E, d_w_r, d_bias);
-    else if (EC == 16)
-      launch_kernel(router_dwr_kernel<16>, grid, dim3(256), 0, st, 1, (const bf16*)x,
+      launch_kernel(router_dwr_kernel<8>, grid, block, 0, st, 1, (const bf16*)x,
                     (const float*)d_logits, T, d, E, d_w_r, d_bias);
     else
-      launch_kernel(router_dwr_kernel<32>, grid, dim3(256), 0, st, 1, (const bf16*)x,
+      launch_kernel(router_dwr_kernel<16>, grid, block, 0, st, 1, (const bf16*)x,
                     (const float*)d_logits, T, d, E, d_w_r, d_bias);
     if ((r = launch_end(K_ROUTER_DWR, st)) != MOE_OK) return r;
   }
