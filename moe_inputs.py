@@ -180,6 +180,75 @@ def make_inputs(cfg: MoEConfig, with_experts: bool = True) -> MoEInputs:
     return inp
 
 
+# --------------------------------------------------------------------------- atomic experts
+_KEY_WROW, _KEY_WCOL, _KEY_WIN, _KEY_WOUT, _KEY_PLOGITS = 7, 8, 9, 10, 11
+
+
+@dataclass(frozen=True)
+class OmniConfig:
+    """Fine-grained (rank-1, "atomic") experts behind a Cartesian-product router:
+    N = n_rows * n_cols experts, each a pair of d-vectors (w_in, w_out); top-K
+    per token. Sizes of the "Two upstream innovations of MoE: Routing-Free and
+    OmniMoE" page, section 4: 102,400 experts per layer on a 320 x 320 grid, K
+    from 512 to 4096, 4096 tokens through a ~200M-parameter layer (2 N d =
+    210M at d = 1024)."""
+
+    name: str
+    T: int
+    d: int
+    n_rows: int
+    n_cols: int
+    K: int
+    renormalize: bool = True
+    logits_given: bool = False  # seeded fp32 row/column logits instead of x W
+    seed: int = 0
+    x_std: float = 1.0
+    w_std: float = 0.02
+    logits_std: float = 1.0
+
+    @property
+    def N(self) -> int:
+        return self.n_rows * self.n_cols
+
+    @property
+    def A(self) -> int:
+        return self.T * self.K
+
+
+OMNI_SMALL = OmniConfig("omni_small", T=256, d=256, n_rows=32, n_cols=32, K=64)
+OMNI_102K = OmniConfig("omni_102k", T=4096, d=1024, n_rows=320, n_cols=320, K=512)
+OMNI_CONFIGS = {c.name: c for c in (OMNI_SMALL, OMNI_102K)}
+
+
+@dataclass
+class OmniInputs:
+    cfg: OmniConfig
+    x: torch.Tensor                       # [T, d] bf16
+    w_row: Optional[torch.Tensor] = None  # [d, n_rows] bf16
+    w_col: Optional[torch.Tensor] = None  # [d, n_cols] bf16
+    w_in: Optional[torch.Tensor] = None   # [N, d] bf16
+    w_out: Optional[torch.Tensor] = None  # [N, d] bf16
+    logits: Optional[torch.Tensor] = None  # [T, n_rows + n_cols] fp32 (logits_given)
+
+
+def make_omni_inputs(cfg: OmniConfig, with_experts: bool = True) -> OmniInputs:
+    """Host tensors of one atomic-expert workload: x ~ N(0, 1), router and expert
+    tables ~ N(0, 0.02), drawn in fp32 in the order x, W_row, W_col, W_in, W_out
+    and rounded to bf16; or, with ``logits_given``, N(0, 1) fp32 logits."""
+    s = cfg.seed
+    x = _cast(normal((cfg.T, cfg.d), cfg.x_std, s, _KEY_X), "bf16")
+    inp = OmniInputs(cfg, x=x)
+    if cfg.logits_given:
+        inp.logits = normal((cfg.T, cfg.n_rows + cfg.n_cols), cfg.logits_std, s, _KEY_PLOGITS)
+    else:
+        inp.w_row = _cast(normal((cfg.d, cfg.n_rows), cfg.w_std, s, _KEY_WROW), "bf16")
+        inp.w_col = _cast(normal((cfg.d, cfg.n_cols), cfg.w_std, s, _KEY_WCOL), "bf16")
+    if with_experts:
+        inp.w_in = _cast(normal((cfg.N, cfg.d), cfg.w_std, s, _KEY_WIN), "bf16")
+        inp.w_out = _cast(normal((cfg.N, cfg.d), cfg.w_std, s, _KEY_WOUT), "bf16")
+    return inp
+
+
 def random_small_config(rng: np.random.Generator, dtype: str = "f32", name: str = "rand",
                         max_T: int = 64) -> MoEConfig:
     """A random tiny shape for property tests (both sides get the same draw)."""
