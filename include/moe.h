@@ -324,6 +324,85 @@ moe_status moe_backward_router(const moe_shape* shape, const void* x, const void
                                void* d_x, moe_stream_t stream);
 
 /* ----------------------------------------------------------------------------
+ * Atomic (rank-1) experts behind a Cartesian-product router, run expert-centric
+ * ("Two upstream innovations of MoE: Routing-Free and OmniMoE", chatdocs.ruinique.com,
+ * sections 2.1-2.3 and 3.2).
+ * N = n_rows * n_cols experts; expert i = (i_r, i_c), i = i_r * n_cols + i_c, is a pair of
+ * d-vectors w_in[i], w_out[i] (two [N, d] bf16 tables, section 2.1). Per token t:
+ *   p_r = x_t W_row, p_c = x_t W_col   (W_row [d, n_rows], W_col [d, n_cols] bf16; the
+ *       logits are one [T, n_rows + n_cols] fp32 array, row axis first; section 2.2);
+ *   selection: the K experts with the largest fl32(p_r[i_r] + p_c[i_c]), descending, ties
+ *       to the lower id. The pair's score LogSoftmax(p_r)_{i_r} + LogSoftmax(p_c)_{i_c}
+ *       differs from that sum by a per-token constant, so the ranking is the same;
+ *   weights: renormalize != 0: softmax of the scores over the K selected; renormalize == 0:
+ *       softmax(p_r)_{i_r} * softmax(p_c)_{i_c}, the factorised probability over all N;
+ *   y_t = sum_k w_{t,k} silu(x_t . w_in[i_k]) w_out[i_k]   (bf16 out, fp32 sums).
+ * Reading: the page instantiates the expert's nonlinearity as "SwiGLU"; an atomic expert has
+ * one input vector, so it is read as SiLU, the gating nonlinearity of SwiGLU.
+ * Limits: T >= 0, T * K < 2^31; 1 <= n_rows, n_cols <= 1024, N <= 2^20; 1 <= K <=
+ * min(N, 4096); d % 256 == 0 with d / 256 in 1..8 or 16. The router GEMM (logits_in NULL)
+ * also needs n_rows % 8 == 0, n_cols % 8 == 0. Tables, x, out and logits_out 16-byte aligned.
+ */
+typedef struct {
+  int32_t T, d, n_rows, n_cols, K;
+  int32_t renormalize; /* != 0: weights renormalised over the K selected */
+} moe_omni_shape;
+
+/* Byte offsets inside the workspace of moe_omni_forward (each 256-byte aligned). */
+typedef struct {
+  size_t logits;         /* fp32 [T, n_rows + n_cols] */
+  size_t topk_ids;       /* int32 [T, K] */
+  size_t topk_w;         /* fp32 [T, K] */
+  size_t counts;         /* int32 [N] tasks per expert */
+  size_t offsets;        /* int32 [N + 1] */
+  size_t assign_to_perm; /* int32 [T * K] */
+  size_t perm_to_assign; /* int32 [T * K] */
+  size_t h;              /* fp32 [T * K] per-task scalar w_{t,k} silu(x_t . w_in[i_k]) */
+  size_t scratch;        /* the schedule's scratch */
+  size_t total;
+} moe_omni_layout;
+
+/* Workspace bytes of moe_omni_forward and moe_omni_schedule (0 for an invalid shape). */
+size_t moe_omni_workspace_size(const moe_omni_shape* shape);
+moe_status moe_omni_workspace_layout(const moe_omni_shape* shape, moe_omni_layout* layout);
+
+/* moe_omni_route - router GEMM (tcgen05), then the K best experts of each token over the
+ * whole grid and their weights (section 2.2).
+ *   logits_in [T, n_rows + n_cols] fp32 or NULL; when NULL, x [T, d], w_row and w_col are
+ *   read and the logits written to logits_out (required then); otherwise x, w_row, w_col
+ *   and logits_out are ignored. topk_ids [T, K] int32, topk_w [T, K] fp32 out, slot 0 best.
+ * The selection equals a brute-force sort of all N pair sums (ties to the lower id). */
+moe_status moe_omni_route(const moe_omni_shape* shape, const void* x, const void* w_row,
+                          const void* w_col, const float* logits_in, float* logits_out,
+                          int32_t* topk_ids, float* topk_w, moe_stream_t stream);
+
+/* moe_omni_schedule - the task list in (expert, token) order (section 2.3): counts [N]
+ * (tasks per expert), offsets [N + 1] (exclusive scan), perm_to_assign [T * K] (slot ->
+ * flat assignment t * K + k, ascending token inside an expert), assign_to_perm [T * K] (the
+ * inverse). Deterministic. workspace: moe_omni_workspace_size bytes (its scratch part is
+ * used). An expert id outside [0, N) is skipped and reported as MOE_ERR_DEVICE_INDEX. */
+moe_status moe_omni_schedule(const moe_omni_shape* shape, const int32_t* topk_ids, int32_t* counts,
+                             int32_t* offsets, int32_t* assign_to_perm, int32_t* perm_to_assign,
+                             void* workspace, size_t ws_bytes, moe_stream_t stream);
+
+/* moe_omni_experts - the experts, given the routing and the schedule:
+ *   h[t * K + k] = topk_w[t, k] * silu(x_t . w_in[i_{t,k}])   computed expert-centric: each
+ *       expert's w_in row is read once and meets all of its tokens' rows (section 2.3);
+ *   out[t] = sum_k h[t * K + k] * w_out[i_{t,k}]   gathered per token, k in order.
+ * x [T, d], w_in/w_out [N, d] bf16; h [T * K] fp32 out; out [T, d] bf16 out. */
+moe_status moe_omni_experts(const moe_omni_shape* shape, const void* x, const void* w_in,
+                            const void* w_out, const int32_t* topk_ids, const float* topk_w,
+                            const int32_t* offsets, const int32_t* perm_to_assign, float* h,
+                            void* out, moe_stream_t stream);
+
+/* moe_omni_forward - route + schedule + experts with every intermediate in `workspace`
+ * (layout from moe_omni_workspace_layout). logits_in as in moe_omni_route. */
+moe_status moe_omni_forward(const moe_omni_shape* shape, const void* x, const void* w_row,
+                            const void* w_col, const float* logits_in, const void* w_in,
+                            const void* w_out, void* out, void* workspace, size_t ws_bytes,
+                            moe_stream_t stream);
+
+/* ----------------------------------------------------------------------------
  * Device status: synchronises `stream`, returns the first device-side fault
  * recorded since the last call (MOE_OK if none) and clears it.
  */

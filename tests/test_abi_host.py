@@ -139,3 +139,61 @@ def test_token_rounding_shape_checks(lib):
     r = lib.moe_permute(ctypes.byref(ok), dummy, dummy, dummy, dummy, dummy, None, None, dummy,
                         1 << 30, None)
     assert r == 2  # rounding needs the logits: not available to moe_permute
+
+
+# ------------------------------------------------------------------ atomic experts
+@pytest.mark.parametrize("kw,code", [
+    (dict(T=16, d=200, n_rows=8, n_cols=8, K=4), 1),      # d not a multiple of 256
+    (dict(T=16, d=256, n_rows=8, n_cols=8, K=65), 1),     # K > N
+    (dict(T=16, d=256, n_rows=0, n_cols=8, K=1), 1),      # empty axis
+    (dict(T=-1, d=256, n_rows=8, n_cols=8, K=4), 1),      # negative T
+    (dict(T=16, d=2304, n_rows=8, n_cols=8, K=4), 2),     # d / 256 = 9: no kernel variant
+    (dict(T=16, d=256, n_rows=2048, n_cols=8, K=4), 2),   # axis above 1024
+    (dict(T=16, d=256, n_rows=1024, n_cols=1024, K=5000), 2),  # K above 4096
+])
+def test_omni_bad_shapes_rejected_on_host(lib, kw, code):
+    s = tdr.make_omni_shape(**kw)
+    assert lib.moe_omni_workspace_size(ctypes.byref(s)) == 0
+    r = lib.moe_omni_forward(ctypes.byref(s), None, None, None, None, None, None, None, None, 0,
+                             None)
+    assert r == code
+
+
+def test_omni_workspace_layout_is_host_arithmetic(lib):
+    T, d, nr, nc, K = 4096, 1024, 320, 320, 512
+    s = tdr.make_omni_shape(T, d, nr, nc, K)
+    L = tdr.omni_workspace_layout(s)
+    N, M = nr * nc, T * K
+    assert L.logits == 0 and L.topk_ids >= T * (nr + nc) * 4
+    assert L.h - L.perm_to_assign >= M * 4 and L.scratch - L.h >= M * 4
+    assert L.total >= L.scratch + (2 * N + M) * 4
+    for f in ("topk_ids", "topk_w", "counts", "offsets", "assign_to_perm", "perm_to_assign",
+              "h", "scratch", "total"):
+        assert getattr(L, f) % 256 == 0
+    assert lib.moe_omni_workspace_size(ctypes.byref(s)) == L.total
+
+
+def test_omni_argument_checks_on_host(lib):
+    s = tdr.make_omni_shape(16, 256, 12, 8, 4)  # n_rows not a multiple of 8: no router GEMM
+    dummy = ctypes.c_void_p(256)  # never dereferenced: every check below fails first
+    # missing outputs
+    assert lib.moe_omni_route(ctypes.byref(s), dummy, dummy, dummy, None, dummy, None, None,
+                              None) == 1
+    # the router GEMM needs both axes in multiples of 8
+    assert lib.moe_omni_route(ctypes.byref(s), dummy, dummy, dummy, None, dummy, dummy, dummy,
+                              None) == 2
+    # no logits at all
+    assert lib.moe_omni_route(ctypes.byref(s), None, None, None, None, None, dummy, dummy,
+                              None) == 1
+    # schedule and forward without a workspace
+    assert lib.moe_omni_schedule(ctypes.byref(s), dummy, dummy, dummy, dummy, dummy, None, 0,
+                                 None) == 4
+    assert lib.moe_omni_forward(ctypes.byref(s), dummy, dummy, dummy, None, dummy, dummy, dummy,
+                                None, 0, None) == 4
+    # experts without the scalar buffer
+    assert lib.moe_omni_experts(ctypes.byref(s), dummy, dummy, dummy, dummy, dummy, dummy, dummy,
+                                None, dummy, None) == 1
+    # T = 0 is a no-op
+    z = tdr.make_omni_shape(0, 256, 8, 8, 4)
+    assert lib.moe_omni_route(ctypes.byref(z), None, None, None, None, None, None, None,
+                              None) == 0

@@ -43,8 +43,21 @@ class moe_workspace_layout(ctypes.Structure):
         "total")]
 
 
+class moe_omni_shape(ctypes.Structure):
+    _fields_ = [("T", ctypes.c_int32), ("d", ctypes.c_int32), ("n_rows", ctypes.c_int32),
+                ("n_cols", ctypes.c_int32), ("K", ctypes.c_int32),
+                ("renormalize", ctypes.c_int32)]
+
+
+class moe_omni_layout(ctypes.Structure):
+    _fields_ = [(f, ctypes.c_size_t) for f in (
+        "logits", "topk_ids", "topk_w", "counts", "offsets", "assign_to_perm",
+        "perm_to_assign", "h", "scratch", "total")]
+
+
 _P = ctypes.c_void_p
 _S = ctypes.POINTER(moe_shape)
+_O = ctypes.POINTER(moe_omni_shape)
 _SIGS = {
     "moe_permute_workspace_size": (ctypes.c_size_t, [_S]),
     "moe_forward_workspace_size": (ctypes.c_size_t, [_S]),
@@ -63,6 +76,13 @@ _SIGS = {
     "moe_backward_router": (ctypes.c_int, [_S, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P]),
     "moe_backward": (ctypes.c_int, [_S, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P,
                                     ctypes.c_size_t, _P]),
+    "moe_omni_workspace_size": (ctypes.c_size_t, [_O]),
+    "moe_omni_workspace_layout": (ctypes.c_int, [_O, ctypes.POINTER(moe_omni_layout)]),
+    "moe_omni_route": (ctypes.c_int, [_O, _P, _P, _P, _P, _P, _P, _P, _P]),
+    "moe_omni_schedule": (ctypes.c_int, [_O, _P, _P, _P, _P, _P, _P, ctypes.c_size_t, _P]),
+    "moe_omni_experts": (ctypes.c_int, [_O, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P]),
+    "moe_omni_forward": (ctypes.c_int, [_O, _P, _P, _P, _P, _P, _P, _P, _P, ctypes.c_size_t,
+                                        _P]),
     "moe_get_device_status": (ctypes.c_int, [_P]),
     "moe_status_string": (ctypes.c_char_p, [ctypes.c_int]),
     "moe_profile_enable": (ctypes.c_int, [ctypes.c_int]),
@@ -456,6 +476,139 @@ def workspace_views(shape: moe_shape, workspace: torch.Tensor) -> dict:
                 perm_to_assign=view(L.perm_to_assign, A, torch.int32, (A,), 4),
                 a_act=view(L.a_act, A * n, dt, (A, n), eb),
                 y_perm=view(L.y_perm, A * d, dt, (A, d), eb))
+
+
+# ------------------------------------------------------------------ atomic experts
+def make_omni_shape(T: int, d: int, n_rows: int, n_cols: int, K: int,
+                    renormalize: bool = True) -> moe_omni_shape:
+    """N = n_rows * n_cols rank-1 experts on a Cartesian grid, top-K per token."""
+    return moe_omni_shape(T, d, n_rows, n_cols, K, 1 if renormalize else 0)
+
+
+def omni_workspace_size(shape: moe_omni_shape) -> int:
+    return int(load_library().moe_omni_workspace_size(ctypes.byref(shape)))
+
+
+def omni_workspace_layout(shape: moe_omni_shape) -> moe_omni_layout:
+    L = moe_omni_layout()
+    _check(load_library().moe_omni_workspace_layout(ctypes.byref(shape), ctypes.byref(L)),
+           "moe_omni_workspace_layout")
+    return L
+
+
+def omni_route(shape: moe_omni_shape, x=None, w_row=None, w_col=None, logits_in=None,
+               logits_out=None, topk_ids=None, topk_w=None):
+    """moe_omni_route. Returns (topk_ids [T,K] int32, topk_w [T,K] fp32, logits or None)."""
+    lib = load_library()
+    T, K, P = shape.T, shape.K, shape.n_rows + shape.n_cols
+    dev = (logits_in if logits_in is not None else x).device
+    if logits_in is None:
+        _dev(x, "x", torch.bfloat16, (T, shape.d))
+        _dev(w_row, "w_row", torch.bfloat16, (shape.d, shape.n_rows))
+        _dev(w_col, "w_col", torch.bfloat16, (shape.d, shape.n_cols))
+        if logits_out is None:
+            logits_out = torch.empty(T, P, dtype=torch.float32, device=dev)
+        _dev(logits_out, "logits_out", torch.float32, (T, P))
+    else:
+        _dev(logits_in, "logits_in", torch.float32, (T, P))
+    if topk_ids is None:
+        topk_ids = torch.empty(T, K, dtype=torch.int32, device=dev)
+    if topk_w is None:
+        topk_w = torch.empty(T, K, dtype=torch.float32, device=dev)
+    _check(lib.moe_omni_route(ctypes.byref(shape), _ptr(x), _ptr(w_row), _ptr(w_col),
+                              _ptr(logits_in), _ptr(logits_out), _ptr(topk_ids), _ptr(topk_w),
+                              _stream()), "moe_omni_route")
+    return topk_ids, topk_w, logits_out
+
+
+def omni_schedule(shape: moe_omni_shape, topk_ids, workspace=None):
+    """moe_omni_schedule. Returns dict(counts, offsets, assign_to_perm, perm_to_assign)."""
+    lib = load_library()
+    T, K = shape.T, shape.K
+    N = shape.n_rows * shape.n_cols
+    dev = topk_ids.device
+    _dev(topk_ids, "topk_ids", torch.int32, (T, K))
+    counts = torch.empty(N, dtype=torch.int32, device=dev)
+    offsets = torch.empty(N + 1, dtype=torch.int32, device=dev)
+    a2p = torch.empty(T * K, dtype=torch.int32, device=dev)
+    p2a = torch.empty(T * K, dtype=torch.int32, device=dev)
+    if workspace is None:
+        workspace = torch.empty(omni_workspace_size(shape), dtype=torch.uint8, device=dev)
+    _check(lib.moe_omni_schedule(ctypes.byref(shape), _ptr(topk_ids), _ptr(counts),
+                                 _ptr(offsets), _ptr(a2p), _ptr(p2a), _ptr(workspace),
+                                 workspace.numel(), _stream()), "moe_omni_schedule")
+    return dict(counts=counts, offsets=offsets, assign_to_perm=a2p, perm_to_assign=p2a)
+
+
+def omni_experts(shape: moe_omni_shape, x, w_in, w_out, topk_ids, topk_w, offsets,
+                 perm_to_assign, h=None, out=None):
+    """moe_omni_experts. Returns (out [T, d] bf16, h [T*K] fp32)."""
+    lib = load_library()
+    T, K, d = shape.T, shape.K, shape.d
+    N = shape.n_rows * shape.n_cols
+    _dev(x, "x", torch.bfloat16, (T, d))
+    _dev(w_in, "w_in", torch.bfloat16, (N, d))
+    _dev(w_out, "w_out", torch.bfloat16, (N, d))
+    _dev(topk_ids, "topk_ids", torch.int32, (T, K))
+    _dev(topk_w, "topk_w", torch.float32, (T, K))
+    _dev(offsets, "offsets", torch.int32, (N + 1,))
+    _dev(perm_to_assign, "perm_to_assign", torch.int32, (T * K,))
+    if h is None:
+        h = torch.empty(T * K, dtype=torch.float32, device=x.device)
+    if out is None:
+        out = torch.empty(T, d, dtype=torch.bfloat16, device=x.device)
+    _dev(h, "h", torch.float32, (T * K,))
+    _dev(out, "out", torch.bfloat16, (T, d))
+    _check(lib.moe_omni_experts(ctypes.byref(shape), _ptr(x), _ptr(w_in), _ptr(w_out),
+                                _ptr(topk_ids), _ptr(topk_w), _ptr(offsets),
+                                _ptr(perm_to_assign), _ptr(h), _ptr(out), _stream()),
+           "moe_omni_experts")
+    return out, h
+
+
+def omni_forward(shape: moe_omni_shape, x, w_row, w_col, w_in, w_out, logits_in=None,
+                 out=None, workspace=None):
+    """moe_omni_forward. Returns (out [T, d] bf16, workspace)."""
+    lib = load_library()
+    T, d = shape.T, shape.d
+    N = shape.n_rows * shape.n_cols
+    _dev(x, "x", torch.bfloat16, (T, d))
+    if logits_in is None:
+        _dev(w_row, "w_row", torch.bfloat16, (d, shape.n_rows))
+        _dev(w_col, "w_col", torch.bfloat16, (d, shape.n_cols))
+    else:
+        _dev(logits_in, "logits_in", torch.float32, (T, shape.n_rows + shape.n_cols))
+    _dev(w_in, "w_in", torch.bfloat16, (N, d))
+    _dev(w_out, "w_out", torch.bfloat16, (N, d))
+    if out is None:
+        out = torch.empty(T, d, dtype=torch.bfloat16, device=x.device)
+    _dev(out, "out", torch.bfloat16, (T, d))
+    if workspace is None:
+        workspace = torch.empty(omni_workspace_size(shape), dtype=torch.uint8, device=x.device)
+    _check(lib.moe_omni_forward(ctypes.byref(shape), _ptr(x), _ptr(w_row), _ptr(w_col),
+                                _ptr(logits_in), _ptr(w_in), _ptr(w_out), _ptr(out),
+                                _ptr(workspace), workspace.numel(), _stream()),
+           "moe_omni_forward")
+    return out, workspace
+
+
+def omni_workspace_views(shape: moe_omni_shape, workspace: torch.Tensor) -> dict:
+    """Typed views of moe_omni_forward's intermediates inside its workspace."""
+    L = omni_workspace_layout(shape)
+    T, K = shape.T, shape.K
+    N, P, M = shape.n_rows * shape.n_cols, shape.n_rows + shape.n_cols, shape.T * shape.K
+
+    def view(off, count, dtype, shp):
+        return workspace[off:off + count * 4].view(dtype).view(*shp)
+
+    return dict(logits=view(L.logits, T * P, torch.float32, (T, P)),
+                topk_ids=view(L.topk_ids, M, torch.int32, (T, K)),
+                topk_w=view(L.topk_w, M, torch.float32, (T, K)),
+                counts=view(L.counts, N, torch.int32, (N,)),
+                offsets=view(L.offsets, N + 1, torch.int32, (N + 1,)),
+                assign_to_perm=view(L.assign_to_perm, M, torch.int32, (M,)),
+                perm_to_assign=view(L.perm_to_assign, M, torch.int32, (M,)),
+                h=view(L.h, M, torch.float32, (M,)))
 
 
 def device_status() -> int:

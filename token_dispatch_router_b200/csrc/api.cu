@@ -98,7 +98,8 @@ const char* kKernelNames[K_COUNT] = {
     "down_tc",      "gateup_simt",   "down_simt",      "combine",     "selftest_timeout",
     "route_tc",     "permute_small", "gateup_tc2",   "down_tc2",
     "permute_cluster", "route_permute", "tile_round", "bwd_act", "bwd_dw", "bwd_dx",
-    "router_dlogits", "router_dwr", "router_dx"};
+    "router_dlogits", "router_dwr", "router_dx", "omni_logits", "omni_topk", "omni_count",
+    "omni_scan", "omni_scatter", "omni_sort", "omni_act", "omni_out"};
 
 struct ProfRec {
   int kid;

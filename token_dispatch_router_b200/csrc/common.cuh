@@ -110,6 +110,14 @@ enum KernelId {
   K_ROUTER_DLOGITS,
   K_ROUTER_DWR,
   K_ROUTER_DX,
+  K_OMNI_LOGITS,
+  K_OMNI_TOPK,
+  K_OMNI_COUNT,
+  K_OMNI_SCAN,
+  K_OMNI_SCATTER,
+  K_OMNI_SORT,
+  K_OMNI_ACT,
+  K_OMNI_OUT,
   K_COUNT
 };
 
