@@ -360,6 +360,16 @@ __device__ void pick_digit(const int* hist, int need, bool desc, int* out_digit,
   }
 }
 
+// Adds the lanes' votes to a shared histogram with one atomic per distinct bin of the warp
+// (pair sums of one token fall into few bins, so per-lane atomics would serialise). Every
+// lane of the warp calls it (uniform control flow).
+__device__ __forceinline__ void hist_add_warp(int* hist, bool pred, uint32_t bin) {
+  const uint32_t key = pred ? bin : 0xFFFFFFFFu;
+  const unsigned peers = __match_any_sync(0xffffffffu, key);
+  if (pred && (threadIdx.x & 31) == (unsigned)(__ffs(peers) - 1))
+    atomicAdd(&hist[bin], __popc(peers));
+}
+
 struct TopkArgs {
   const float* logits;  // [T, nr + nc]
   int32_t* ids;         // [T, K]
@@ -441,9 +451,10 @@ __global__ void __launch_bounds__(TK_THREADS) omni_topk_kernel(const TopkArgs g)
     for (int r = warp; r < R; r += TK_WARPS) {
       const int Lr = min(nc, K / (r + 1));
       const float a = sv_r[r];
-      for (int c = lane; c < Lr; c += 32) {
-        const uint32_t key = ord_key(a + sv_c[c]);
-        if ((key & pmask) == prefix) atomicAdd(&hist[(key >> shift) & 255], 1);
+      for (int c0 = 0; c0 < Lr; c0 += 32) {
+        const int c = c0 + lane;
+        const uint32_t key = c < Lr ? ord_key(a + sv_c[c]) : 0u;
+        hist_add_warp(hist, c < Lr && (key & pmask) == prefix, (key >> shift) & 255);
       }
     }
     __syncthreads();
@@ -507,9 +518,11 @@ __global__ void __launch_bounds__(TK_THREADS) omni_topk_kernel(const TopkArgs g)
       for (int r = warp; r < nr; r += TK_WARPS) {
         const uint32_t rid = (uint32_t)sid_r[r] * (uint32_t)nc;
         const int c0 = s_gt[r];
-        for (int c = lane; c < s_tie[r]; c += 32) {
-          const uint32_t id = rid + (uint32_t)sid_c[c0 + c];
-          if ((id & imask) == ipre) atomicAdd(&hist[(id >> shift) & 255], 1);
+        const int nt = s_tie[r];
+        for (int cb = 0; cb < nt; cb += 32) {
+          const int c = cb + lane;
+          const uint32_t id = c < nt ? rid + (uint32_t)sid_c[c0 + c] : 0u;
+          hist_add_warp(hist, c < nt && (id & imask) == ipre, (id >> shift) & 255);
         }
       }
       __syncthreads();
@@ -606,41 +619,82 @@ __global__ void omni_count_kernel(const int32_t* ids, long long M, int N, int32_
   }
 }
 
-// One CTA of 1024 threads: offsets = exclusive scan of counts (offsets[N] = total).
-__global__ void __launch_bounds__(1024) omni_scan_kernel(const int32_t* counts, int N,
-                                                         int32_t* offsets) {
-  __shared__ int wsum[32];
-  pdl_wait();
-  pdl_trigger();
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int chunk = (N + 1023) / 1024;
-  const int lo = min(N, tid * chunk), hi = min(N, lo + chunk);
-  int s = 0;
-  for (int i = lo; i < hi; ++i) s += counts[i];
-  int incl = s;
+constexpr int kScanTile = 4096;  // counts per CTA of the offsets scan: 1024 threads x 4
+
+// Block-wide inclusive scan of one int per thread (1024 threads); returns the inclusive
+// value and leaves the block total in *total.
+__device__ int block_incl_scan(int v, int* ws, int* total) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  int x = v;
 #pragma unroll
   for (int o = 1; o < 32; o <<= 1) {
-    const int v = __shfl_up_sync(0xffffffffu, incl, o);
-    if (lane >= o) incl += v;
+    const int u = __shfl_up_sync(0xffffffffu, x, o);
+    if (lane >= o) x += u;
   }
-  if (lane == 31) wsum[warp] = incl;
+  if (lane == 31) ws[warp] = x;
   __syncthreads();
   if (warp == 0) {
-    int v = wsum[lane], iv = v;
+    const int wv = ws[lane];
+    int y = wv;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
-      const int u = __shfl_up_sync(0xffffffffu, iv, o);
-      if (lane >= o) iv += u;
+      const int u = __shfl_up_sync(0xffffffffu, y, o);
+      if (lane >= o) y += u;
     }
-    wsum[lane] = iv - v;
+    ws[lane] = y - wv;
+    if (lane == 31) *total = y;
   }
   __syncthreads();
-  int run = wsum[warp] + incl - s;
-  for (int i = lo; i < hi; ++i) {
-    offsets[i] = run;
-    run += counts[i];
+  return x + ws[warp];
+}
+
+// Pass 1: the count total of each 4096-expert tile.
+__global__ void __launch_bounds__(1024) omni_scan_sums_kernel(const int32_t* counts, int N,
+                                                              int32_t* sums) {
+  __shared__ int ws[32];
+  __shared__ int total;
+  pdl_wait();
+  pdl_trigger();
+  const int base = blockIdx.x * kScanTile + threadIdx.x * 4;
+  int v = 0;
+#pragma unroll
+  for (int q = 0; q < 4; ++q)
+    if (base + q < N) v += counts[base + q];
+  block_incl_scan(v, ws, &total);
+  if (threadIdx.x == 0) sums[blockIdx.x] = total;
+}
+
+// Pass 2: offsets = exclusive scan of counts; each tile adds the totals of the tiles before
+// it (at most 256 of them); the last tile writes offsets[N].
+__global__ void __launch_bounds__(1024) omni_scan_write_kernel(const int32_t* counts, int N,
+                                                               const int32_t* sums,
+                                                               int32_t* offsets) {
+  __shared__ int ws[32];
+  __shared__ int total, carry;
+  pdl_wait();
+  pdl_trigger();
+  const int lane = threadIdx.x & 31;
+  if (threadIdx.x < 32) {
+    int c = 0;
+    for (int i = lane; i < (int)blockIdx.x; i += 32) c += sums[i];
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) c += __shfl_xor_sync(0xffffffffu, c, o);
+    if (lane == 0) carry = c;
   }
-  if (tid == 1023) offsets[N] = run;
+  const int base = blockIdx.x * kScanTile + threadIdx.x * 4;
+  int v[4], sum = 0;
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    v[q] = base + q < N ? counts[base + q] : 0;
+    sum += v[q];
+  }
+  int run = block_incl_scan(sum, ws, &total) - sum + carry;
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    if (base + q < N) offsets[base + q] = run;
+    run += v[q];
+  }
+  if (blockIdx.x == gridDim.x - 1 && threadIdx.x == 0) offsets[N] = carry + total;
 }
 
 __global__ void omni_scatter_kernel(const int32_t* ids, long long M, int N, const int32_t* offsets,
@@ -763,17 +817,6 @@ __global__ void __launch_bounds__(1024) omni_bigsort_kernel(const int32_t* offse
 }
 
 // ------------------------------------------------------------------ experts
-__device__ __forceinline__ float dot8(const uint4& a, const uint4& b) {
-  const uint32_t x[4] = {a.x, a.y, a.z, a.w}, y[4] = {b.x, b.y, b.z, b.w};
-  float s = 0.f;
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    s = fmaf(__uint_as_float(x[i] << 16), __uint_as_float(y[i] << 16), s);
-    s = fmaf(__uint_as_float(x[i] & 0xffff0000u), __uint_as_float(y[i] & 0xffff0000u), s);
-  }
-  return s;
-}
-
 __device__ __forceinline__ uint4 ldg_nc(const uint4* p) {
   uint4 v;
   asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0, %1, %2, %3}, [%4];"
@@ -782,9 +825,77 @@ __device__ __forceinline__ uint4 ldg_nc(const uint4* p) {
   return v;
 }
 
-// A warp per expert (grid-stride): w_in[e] is loaded once into registers (CH 16-byte
-// vectors per lane, d = 256 CH), then its tasks' token rows stream past it, U at a time.
-template <int CH, int U>
+__device__ __forceinline__ void cp_async_commit() {
+  asm volatile("cp.async.commit_group;" ::: "memory");
+}
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+__device__ __forceinline__ uint4 lds16(uint32_t addr) {
+  uint4 v;
+  asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "r"(addr)
+               : "memory");
+  return v;
+}
+
+// Shared memory of one warp in the row-streaming kernels: R rows of d bf16 (CH 16-byte
+// vectors per lane).
+template <int CH, int R>
+struct RowRing {
+  static constexpr int ROW = CH * 32 * 16;
+  static constexpr int BYTES = R * ROW;
+};
+
+// acc + (x.lo * w.lo) + (x.hi * w.hi) for two packed bf16 pairs, fp32 accumulation: the
+// mixed-precision FMA takes the bf16 halves directly (a bf16 product is exact in fp32).
+__device__ __forceinline__ float fma_bf16x2(uint32_t x, uint32_t w, float acc) {
+  asm("{\n\t.reg .b16 xl, xh, wl, wh;\n\t"
+      "mov.b32 {xl, xh}, %1;\n\tmov.b32 {wl, wh}, %2;\n\t"
+      "fma.rn.f32.bf16 %0, xl, wl, %0;\n\tfma.rn.f32.bf16 %0, xh, wh, %0;\n\t}"
+      : "+f"(acc)
+      : "r"(x), "r"(w));
+  return acc;
+}
+
+// acc.{x, y} += {w.lo, w.hi} * hh.{x, y}: a packed bf16 pair widened to fp32 and one
+// two-lane fp32 FMA.
+__device__ __forceinline__ void fma2_bf16(uint32_t w, uint64_t hh, uint64_t& acc) {
+  asm("{\n\t.reg .b32 lo, hi;\n\t.reg .b64 v;\n\t"
+      "shl.b32 lo, %1, 16;\n\tand.b32 hi, %1, 0xffff0000;\n\t"
+      "mov.b64 v, {lo, hi};\n\tfma.rn.f32x2 %0, v, %2, %0;\n\t}"
+      : "+l"(acc)
+      : "r"(w), "l"(hh));
+}
+
+// Sums v[i] over the 32 lanes for all i at once (a butterfly that halves the values held at
+// each step: 31 shuffles for 32 sums); lane l returns the sum of v[l].
+__device__ __forceinline__ float transpose_reduce32(float (&v)[32]) {
+  const int lane = threadIdx.x & 31;
+#pragma unroll
+  for (int sft = 16; sft >= 1; sft >>= 1) {
+    const bool upper = (lane & sft) != 0;
+#pragma unroll
+    for (int i = 0; i < sft; ++i) {
+      const float send = upper ? v[i] : v[i + sft];
+      const float keep = upper ? v[i + sft] : v[i];
+      v[i] = keep + __shfl_xor_sync(0xffffffffu, send, sft);
+    }
+  }
+  return v[0];
+}
+
+// Expert-centric scalars. The expert-major task list is cut into equal contiguous ranges,
+// one per warp. A warp keeps the current expert's w_in row in registers (loaded once per
+// expert it meets) and streams its tasks' token rows from L2 through an R-deep cp.async
+// ring in shared memory; each lane copies and later reads only its own 16-byte columns,
+// so the ring needs no synchronisation beyond the lane's own cp.async groups. Tasks go in
+// batches of 32: each lane keeps 32 partial dot products, one transposed reduction gives
+// lane l the dot product of task l, and lane l writes that task's scalar
+// h[a] = topk_w[a] * silu(x_{a / K} . w_in[e]).
+template <int CH, int R>
 __global__ void __launch_bounds__(256) omni_act_kernel(const bf16* __restrict__ x,
                                                        const bf16* __restrict__ w_in,
                                                        const int32_t* __restrict__ offsets,
@@ -792,149 +903,204 @@ __global__ void __launch_bounds__(256) omni_act_kernel(const bf16* __restrict__ 
                                                        const float* __restrict__ topk_w,
                                                        float* __restrict__ h, int N, int K, int d,
                                                        int M, unsigned* status) {
+  using Ring = RowRing<CH, R>;
+  extern __shared__ __align__(16) uint8_t sm_act[];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, wpc = blockDim.x >> 5;
+  const uint32_t rbase = saddr(sm_act + (size_t)warp * Ring::BYTES);
   pdl_wait();
   pdl_trigger();
-  const int lane = threadIdx.x & 31;
-  const int nw = (gridDim.x * blockDim.x) >> 5;
-  for (int e = (blockIdx.x * blockDim.x + threadIdx.x) >> 5; e < N; e += nw) {
-    const int p0 = offsets[e], p1 = offsets[e + 1];
-    if (p0 == p1) continue;
-    if (p0 < 0 || p1 < p0 || p1 > M) {
-      if (lane == 0) report(status, MOE_ERR_DEVICE_INDEX);
-      continue;
-    }
-    uint4 wv[CH];
-    const uint4* wrow = reinterpret_cast<const uint4*>(w_in + (size_t)e * d);
-#pragma unroll
-    for (int j = 0; j < CH; ++j) wv[j] = ldg_nc(wrow + lane + 32 * j);
-    for (int p = p0; p < p1; p += U) {
-      int a[U];
-      uint4 xv[U][CH];
-#pragma unroll
-      for (int u = 0; u < U; ++u) {
-        a[u] = p + u < p1 ? p2a[p + u] : -1;
-        if (a[u] >= M) {
-          if (lane == 0) report(status, MOE_ERR_DEVICE_INDEX);
-          a[u] = -1;
-        }
-      }
-#pragma unroll
-      for (int u = 0; u < U; ++u) {
-        if (a[u] >= 0) {
-          const uint4* xr = reinterpret_cast<const uint4*>(x + (size_t)(a[u] / K) * d);
-#pragma unroll
-          for (int j = 0; j < CH; ++j) xv[u][j] = ldg_nc(xr + lane + 32 * j);
-        } else {
-#pragma unroll
-          for (int j = 0; j < CH; ++j) xv[u][j] = make_uint4(0, 0, 0, 0);
-        }
-      }
-      float s[U];
-#pragma unroll
-      for (int u = 0; u < U; ++u) {
-        float acc = 0.f;
-#pragma unroll
-        for (int j = 0; j < CH; ++j) acc += dot8(wv[j], xv[u][j]);
-        s[u] = acc;
-      }
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1)
-#pragma unroll
-        for (int u = 0; u < U; ++u) s[u] += __shfl_xor_sync(0xffffffffu, s[u], o);
-#pragma unroll
-      for (int u = 0; u < U; ++u)
-        if (lane == u && a[u] >= 0) h[a[u]] = topk_w[a[u]] * (s[u] / (1.f + expf(-s[u])));
-    }
+  const long long nw = (long long)gridDim.x * wpc, gw = (long long)blockIdx.x * wpc + warp;
+  const long long per = (((long long)M + nw - 1) / nw + 31) & ~31LL;
+  const int P0 = (int)min((long long)M, gw * per), P1 = (int)min((long long)M, gw * per + per);
+  if (P0 >= P1) return;
+  if (offsets[N] != M) {  // the schedule must cover every task
+    if (lane == 0) report(status, MOE_ERR_DEVICE_INDEX);
+    return;
   }
+  int lo = 0, hi = N - 1;  // the expert owning slot P0: last e with offsets[e] <= P0
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (offsets[mid] <= P0) lo = mid;
+    else hi = mid - 1;
+  }
+  int e = lo, e_end = offsets[e + 1];
+  uint4 wv[CH];
+  {
+    const uint4* wr = reinterpret_cast<const uint4*>(w_in + (size_t)e * d);
+#pragma unroll
+    for (int j = 0; j < CH; ++j) wv[j] = ldg_nc(wr + lane + 32 * j);
+  }
+  // issue side: lane l holds the token of task ibase + l (-1: none or invalid)
+  int ibase = P0 - 32, itok = -1;
+  auto issue = [&](int q) {
+    if (q < P1) {
+      if (q >= ibase + 32) {
+        ibase = q;
+        const int a = q + lane < P1 ? p2a[q + lane] : -1;
+        itok = (unsigned)a < (unsigned)M ? a / K : -1;
+      }
+      const int t = __shfl_sync(0xffffffffu, itok, q - ibase);
+      if (t >= 0) {
+        const uint8_t* src = reinterpret_cast<const uint8_t*>(x + (size_t)t * d);
+        const uint32_t dst = rbase + ((q - P0) % R) * Ring::ROW;
+#pragma unroll
+        for (int j = 0; j < CH; ++j) cp_async16(dst + (lane + 32 * j) * 16, src + (lane + 32 * j) * 16);
+      }
+    }
+    cp_async_commit();
+  };
+#pragma unroll
+  for (int i = 0; i < R; ++i) issue(P0 + i);
+  for (int base = P0; base < P1; base += 32) {
+    int ca = base + lane < P1 ? p2a[base + lane] : -1;  // this lane's task of the batch
+    if (ca >= M) {
+      report(status, MOE_ERR_DEVICE_INDEX);
+      ca = -1;
+    }
+    const float cw = ca >= 0 ? topk_w[ca] : 0.f;
+    float v[32];
+#pragma unroll
+    for (int i = 0; i < 32; ++i) {
+      const int p = base + i;
+      float acc = 0.f;
+      if (p < P1) {
+        if (p >= e_end) {  // next expert with tasks
+          while (p >= e_end && e < N - 1) {
+            ++e;
+            e_end = offsets[e + 1];
+          }
+          const uint4* wr = reinterpret_cast<const uint4*>(w_in + (size_t)e * d);
+#pragma unroll
+          for (int j = 0; j < CH; ++j) wv[j] = ldg_nc(wr + lane + 32 * j);
+        }
+        cp_async_wait<R - 1>();
+        const uint32_t src = rbase + ((p - P0) % R) * Ring::ROW;
+        float a0 = 0.f, a1 = 0.f;
+#pragma unroll
+        for (int j = 0; j < CH; ++j) {
+          const uint4 xv = lds16(src + (lane + 32 * j) * 16);
+          a0 = fma_bf16x2(xv.x, wv[j].x, a0);
+          a1 = fma_bf16x2(xv.y, wv[j].y, a1);
+          a0 = fma_bf16x2(xv.z, wv[j].z, a0);
+          a1 = fma_bf16x2(xv.w, wv[j].w, a1);
+        }
+        acc = a0 + a1;
+        issue(p + R);
+      }
+      v[i] = acc;
+    }
+    const float sdot = transpose_reduce32(v);
+    if (ca >= 0) h[ca] = cw * (sdot / (1.f + expf(-sdot)));
+  }
+  cp_async_wait<0>();
 }
 
-// WPT warps per token; warp w takes k in blocks of 32 (w, w + WPT, ...); each lane keeps
-// 8 CH fp32 partial sums; the warps' partials are added in warp order.
-template <int CH, int U, int WPT>
+// Token-centric output. A CTA takes one token at a time; its WPT warps split the token's K
+// tasks into contiguous chunks, stream the w_out rows through R-deep cp.async rings and keep
+// 8 CH fp32 sums per lane; the warps' sums are then added in warp order (deterministic).
+template <int CH, int R, int WPT>
 __global__ void __launch_bounds__(WPT * 32) omni_out_kernel(const bf16* __restrict__ w_out,
                                                             const int32_t* __restrict__ ids,
                                                             const float* __restrict__ h,
                                                             bf16* __restrict__ out, int T, int K,
                                                             int d, int N, unsigned* status) {
-  extern __shared__ __align__(16) float part[];  // [WPT][d]
+  using Ring = RowRing<CH, R>;
+  static_assert(Ring::BYTES >= CH * 32 * 8 * 4, "a warp's ring holds its partial row");
+  extern __shared__ __align__(16) uint8_t sm_out[];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  uint8_t* rg = sm_out + (size_t)warp * Ring::BYTES;
+  const uint32_t rbase = saddr(rg);
   pdl_wait();
   pdl_trigger();
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int kc = (K + WPT - 1) / WPT;
   for (int t = blockIdx.x; t < T; t += gridDim.x) {
-    float acc[CH][8];
+    const int k0 = min(K, warp * kc), k1 = min(K, k0 + kc);
+    const int32_t* tid_ = ids + (size_t)t * K;
+    const float* th = h + (size_t)t * K;
+    uint64_t acc[CH][4];  // fp32 pairs (columns 2i, 2i + 1 of each 8-column chunk)
 #pragma unroll
     for (int j = 0; j < CH; ++j)
 #pragma unroll
-      for (int q = 0; q < 8; ++q) acc[j][q] = 0.f;
-    for (int k0 = warp * 32; k0 < K; k0 += WPT * 32) {
-      const int nk = min(32, K - k0);
-      int e = -1;
-      float hv = 0.f;
-      if (lane < nk) {
-        e = ids[(size_t)t * K + k0 + lane];
-        hv = h[(size_t)t * K + k0 + lane];
-        if ((unsigned)e >= (unsigned)N) {
-          report(status, MOE_ERR_DEVICE_INDEX);
-          e = -1;
+      for (int q = 0; q < 4; ++q) acc[j][q] = 0ull;
+    int ibase = k0, ewin = k0 + lane < k1 ? tid_[k0 + lane] : -1;
+    int cbase = k0, cwin = ewin;
+    float hwin = k0 + lane < k1 ? th[k0 + lane] : 0.f;
+    auto issue = [&](int q) {
+      if (q < k1) {
+        if (q >= ibase + 32) {
+          ibase = q;
+          ewin = q + lane < k1 ? tid_[q + lane] : -1;
+        }
+        const int e = __shfl_sync(0xffffffffu, ewin, q - ibase);
+        if ((unsigned)e < (unsigned)N) {
+          const uint8_t* src = reinterpret_cast<const uint8_t*>(w_out + (size_t)e * d);
+          const int slot = (q - k0) % R;
+#pragma unroll
+          for (int j = 0; j < CH; ++j)
+            cp_async16(rbase + slot * Ring::ROW + (lane + 32 * j) * 16, src + (lane + 32 * j) * 16);
         }
       }
-      for (int jj = 0; jj < nk; jj += U) {
-        uint4 v[U][CH];
-        float hh[U];
+      cp_async_commit();
+    };
 #pragma unroll
-        for (int u = 0; u < U; ++u) {
-          const int src = jj + u;
-          const int eu = __shfl_sync(0xffffffffu, e, src & 31);
-          hh[u] = __shfl_sync(0xffffffffu, hv, src & 31);
-          if (src < nk && eu >= 0) {
-            const uint4* vr = reinterpret_cast<const uint4*>(w_out + (size_t)eu * d);
-#pragma unroll
-            for (int j = 0; j < CH; ++j) v[u][j] = ldg_nc(vr + lane + 32 * j);
-          } else {
-            hh[u] = 0.f;
-#pragma unroll
-            for (int j = 0; j < CH; ++j) v[u][j] = make_uint4(0, 0, 0, 0);
-          }
-        }
-#pragma unroll
-        for (int u = 0; u < U; ++u) {
-#pragma unroll
-          for (int j = 0; j < CH; ++j) {
-            const uint32_t wd[4] = {v[u][j].x, v[u][j].y, v[u][j].z, v[u][j].w};
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-              acc[j][2 * i] = fmaf(hh[u], __uint_as_float(wd[i] << 16), acc[j][2 * i]);
-              acc[j][2 * i + 1] = fmaf(hh[u], __uint_as_float(wd[i] & 0xffff0000u), acc[j][2 * i + 1]);
-            }
-          }
-        }
+    for (int i = 0; i < R; ++i) issue(k0 + i);
+    for (int p = k0; p < k1; ++p) {
+      if (p >= cbase + 32) {
+        cbase = p;
+        cwin = p + lane < k1 ? tid_[p + lane] : -1;
+        hwin = p + lane < k1 ? th[p + lane] : 0.f;
       }
+      const int e = __shfl_sync(0xffffffffu, cwin, p - cbase);
+      const float hv = __shfl_sync(0xffffffffu, hwin, p - cbase);
+      uint64_t hh;
+      asm("mov.b64 %0, {%1, %1};" : "=l"(hh) : "f"(hv));
+      cp_async_wait<R - 1>();
+      if ((unsigned)e < (unsigned)N) {
+        const int slot = (p - k0) % R;
+#pragma unroll
+        for (int j = 0; j < CH; ++j) {
+          const uint4 v = lds16(rbase + slot * Ring::ROW + (lane + 32 * j) * 16);
+          fma2_bf16(v.x, hh, acc[j][0]);
+          fma2_bf16(v.y, hh, acc[j][1]);
+          fma2_bf16(v.z, hh, acc[j][2]);
+          fma2_bf16(v.w, hh, acc[j][3]);
+        }
+      } else if (lane == 0) {
+        report(status, MOE_ERR_DEVICE_INDEX);
+      }
+      issue(p + R);
     }
+    cp_async_wait<0>();
+    // this warp's partial row, [d] fp32, into its own (now idle) ring
+    float* part = reinterpret_cast<float*>(rg);
 #pragma unroll
     for (int j = 0; j < CH; ++j) {
-      float4* dst = reinterpret_cast<float4*>(part + (size_t)warp * d + (lane + 32 * j) * 8);
-      dst[0] = make_float4(acc[j][0], acc[j][1], acc[j][2], acc[j][3]);
-      dst[1] = make_float4(acc[j][4], acc[j][5], acc[j][6], acc[j][7]);
+      uint4* dst = reinterpret_cast<uint4*>(part + (lane + 32 * j) * 8);
+      dst[0] = make_uint4((uint32_t)acc[j][0], (uint32_t)(acc[j][0] >> 32), (uint32_t)acc[j][1],
+                          (uint32_t)(acc[j][1] >> 32));
+      dst[1] = make_uint4((uint32_t)acc[j][2], (uint32_t)(acc[j][2] >> 32), (uint32_t)acc[j][3],
+                          (uint32_t)(acc[j][3] >> 32));
     }
     __syncthreads();
     for (int c8 = threadIdx.x; c8 < d / 8; c8 += WPT * 32) {
-      float s[8];
+      float sum[8];
 #pragma unroll
-      for (int q = 0; q < 8; ++q) s[q] = 0.f;
+      for (int q = 0; q < 8; ++q) sum[q] = 0.f;
 #pragma unroll
       for (int w = 0; w < WPT; ++w) {
-        const float4* src = reinterpret_cast<const float4*>(part + (size_t)w * d + c8 * 8);
+        const float4* src =
+            reinterpret_cast<const float4*>(sm_out + (size_t)w * Ring::BYTES) + c8 * 2;
         const float4 x0 = src[0], x1 = src[1];
-        s[0] += x0.x;
-        s[1] += x0.y;
-        s[2] += x0.z;
-        s[3] += x0.w;
-        s[4] += x1.x;
-        s[5] += x1.y;
-        s[6] += x1.z;
-        s[7] += x1.w;
+        sum[0] += x0.x;
+        sum[1] += x0.y;
+        sum[2] += x0.z;
+        sum[3] += x0.w;
+        sum[4] += x1.x;
+        sum[5] += x1.y;
+        sum[6] += x1.z;
+        sum[7] += x1.w;
       }
-      *reinterpret_cast<uint4*>(out + (size_t)t * d + c8 * 8) = pack16(s, bf16());
+      *reinterpret_cast<uint4*>(out + (size_t)t * d + c8 * 8) = pack16(sum, bf16());
     }
     __syncthreads();
   }
@@ -972,28 +1138,43 @@ int axis_tile(int n) {  // columns per tile for an axis of n: a multiple of 64, 
   return ((per + 63) / 64) * 64;
 }
 
-template <int CH, int U>
+template <typename Kern>
+int resident_ctas(Kern k, int threads, int smem) {
+  int n = 0;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, k, threads, smem) != cudaSuccess || n < 1)
+    n = 1;
+  return n;
+}
+
+template <int CH, int R>
 moe_status launch_act_ch(const moe_omni_shape& s, const void* x, const void* w_in,
                          const int32_t* offsets, const int32_t* p2a, const float* topk_w, float* h,
                          cudaStream_t st) {
   const int N = s.n_rows * s.n_cols;
-  const int grid = grid_cap((long long)N * 32, 256, 8);
+  constexpr int BYTES = RowRing<CH, R>::BYTES;
+  const int warps = max(1, min(8, (64 * 1024) / BYTES));
+  const int smem = warps * BYTES;
+  auto kern = omni_act_kernel<CH, R>;
+  if (!set_smem(kern, smem)) return MOE_ERR_CUDA;
+  const int grid = sm_count() * resident_ctas(kern, warps * 32, smem);
   launch_begin(K_OMNI_ACT, st);
-  launch_kernel(omni_act_kernel<CH, U>, dim3((unsigned)grid), dim3(256), 0, st, 1u, (const bf16*)x,
+  launch_kernel(kern, dim3((unsigned)grid), dim3(warps * 32), (size_t)smem, st, 1u, (const bf16*)x,
                 (const bf16*)w_in, offsets, p2a, topk_w, h, N, s.K, s.d, s.T * s.K,
                 device_status_ptr());
   return launch_end(K_OMNI_ACT, st);
 }
 
-template <int CH, int U, int WPT>
+template <int CH, int R, int WPT>
 moe_status launch_out_ch(const moe_omni_shape& s, const void* w_out, const int32_t* ids,
                          const float* h, void* out, cudaStream_t st) {
   const int N = s.n_rows * s.n_cols;
-  const int smem = WPT * s.d * 4;
-  auto kern = omni_out_kernel<CH, U, WPT>;
+  const int smem = WPT * RowRing<CH, R>::BYTES;
+  auto kern = omni_out_kernel<CH, R, WPT>;
   if (!set_smem(kern, smem)) return MOE_ERR_CUDA;
+  const int cap = sm_count() * resident_ctas(kern, WPT * 32, smem);
+  const int grid = s.T < cap ? s.T : cap;
   launch_begin(K_OMNI_OUT, st);
-  launch_kernel(kern, dim3((unsigned)s.T), dim3(WPT * 32), (size_t)smem, st, 1u, (const bf16*)w_out,
+  launch_kernel(kern, dim3((unsigned)grid), dim3(WPT * 32), (size_t)smem, st, 1u, (const bf16*)w_out,
                 ids, h, (bf16*)out, s.T, s.K, s.d, N, device_status_ptr());
   return launch_end(K_OMNI_OUT, st);
 }
@@ -1054,10 +1235,11 @@ moe_status launch_omni_topk(const moe_omni_shape& s, const float* logits, int32_
   return launch_end(K_OMNI_TOPK, st);
 }
 
-// Scratch of the schedule: cursor [N], unsorted slots [T K], queued experts [N], queue length.
+// Scratch of the schedule: cursor [N], unsorted slots [T K], queued experts [N], queue length
+// (64 ints), the scan's tile totals (256).
 size_t omni_schedule_scratch_bytes(const moe_omni_shape& s) {
   const size_t N = (size_t)s.n_rows * s.n_cols, M = (size_t)s.T * s.K;
-  return (N + M + N + 64) * 4;
+  return (N + M + N + 64 + 256) * 4;
 }
 
 moe_status launch_omni_schedule(const moe_omni_shape& s, const int32_t* ids, int32_t* counts,
@@ -1069,6 +1251,7 @@ moe_status launch_omni_schedule(const moe_omni_shape& s, const int32_t* ids, int
   int32_t* tmp = cursor + N;
   int32_t* big_list = tmp + M;
   int32_t* big_count = big_list + N;
+  int32_t* scan_sums = big_count + 64;
   unsigned* status = device_status_ptr();
   moe_status r;
   launch_begin(K_OMNI_COUNT, st);
@@ -1079,8 +1262,14 @@ moe_status launch_omni_schedule(const moe_omni_shape& s, const int32_t* ids, int
   launch_kernel(omni_count_kernel, dim3((unsigned)grid_cap(M, 256, 8)), dim3(256), 0, st, 1u, ids, M,
                 N, counts, status);
   if ((r = launch_end(K_OMNI_COUNT, st)) != MOE_OK) return r;
+  const int scan_tiles = (N + kScanTile - 1) / kScanTile;
   launch_begin(K_OMNI_SCAN, st);
-  launch_kernel(omni_scan_kernel, dim3(1), dim3(1024), 0, st, 1u, (const int32_t*)counts, N, offsets);
+  launch_kernel(omni_scan_sums_kernel, dim3((unsigned)scan_tiles), dim3(1024), 0, st, 1u,
+                (const int32_t*)counts, N, scan_sums);
+  if ((r = launch_end(K_OMNI_SCAN, st)) != MOE_OK) return r;
+  launch_begin(K_OMNI_SCAN, st);
+  launch_kernel(omni_scan_write_kernel, dim3((unsigned)scan_tiles), dim3(1024), 0, st, 1u,
+                (const int32_t*)counts, N, (const int32_t*)scan_sums, offsets);
   if ((r = launch_end(K_OMNI_SCAN, st)) != MOE_OK) return r;
   launch_begin(K_OMNI_SCATTER, st);
   launch_kernel(omni_scatter_kernel, dim3((unsigned)grid_cap(M, 256, 8)), dim3(256), 0, st, 1u, ids,
@@ -1105,29 +1294,29 @@ moe_status launch_omni_act(const moe_omni_shape& s, const void* x, const void* w
                            float* h, cudaStream_t st) {
   switch (s.d / 256) {
     case 1: return launch_act_ch<1, 8>(s, x, w_in, offsets, p2a, topk_w, h, st);
-    case 2: return launch_act_ch<2, 8>(s, x, w_in, offsets, p2a, topk_w, h, st);
+    case 2: return launch_act_ch<2, 6>(s, x, w_in, offsets, p2a, topk_w, h, st);
     case 3: return launch_act_ch<3, 4>(s, x, w_in, offsets, p2a, topk_w, h, st);
     case 4: return launch_act_ch<4, 4>(s, x, w_in, offsets, p2a, topk_w, h, st);
-    case 5: return launch_act_ch<5, 2>(s, x, w_in, offsets, p2a, topk_w, h, st);
+    case 5: return launch_act_ch<5, 4>(s, x, w_in, offsets, p2a, topk_w, h, st);
     case 6: return launch_act_ch<6, 2>(s, x, w_in, offsets, p2a, topk_w, h, st);
     case 7: return launch_act_ch<7, 2>(s, x, w_in, offsets, p2a, topk_w, h, st);
     case 8: return launch_act_ch<8, 2>(s, x, w_in, offsets, p2a, topk_w, h, st);
-    default: return launch_act_ch<16, 1>(s, x, w_in, offsets, p2a, topk_w, h, st);
+    default: return launch_act_ch<16, 2>(s, x, w_in, offsets, p2a, topk_w, h, st);
   }
 }
 
 moe_status launch_omni_out(const moe_omni_shape& s, const void* w_out, const int32_t* ids,
                            const float* h, void* out, cudaStream_t st) {
   switch (s.d / 256) {
-    case 1: return launch_out_ch<1, 8, 8>(s, w_out, ids, h, out, st);
-    case 2: return launch_out_ch<2, 4, 8>(s, w_out, ids, h, out, st);
-    case 3: return launch_out_ch<3, 4, 8>(s, w_out, ids, h, out, st);
-    case 4: return launch_out_ch<4, 4, 8>(s, w_out, ids, h, out, st);
-    case 5: return launch_out_ch<5, 2, 8>(s, w_out, ids, h, out, st);
-    case 6: return launch_out_ch<6, 2, 8>(s, w_out, ids, h, out, st);
+    case 1: return launch_out_ch<1, 8, 4>(s, w_out, ids, h, out, st);
+    case 2: return launch_out_ch<2, 6, 4>(s, w_out, ids, h, out, st);
+    case 3: return launch_out_ch<3, 4, 4>(s, w_out, ids, h, out, st);
+    case 4: return launch_out_ch<4, 4, 4>(s, w_out, ids, h, out, st);
+    case 5: return launch_out_ch<5, 4, 4>(s, w_out, ids, h, out, st);
+    case 6: return launch_out_ch<6, 2, 4>(s, w_out, ids, h, out, st);
     case 7: return launch_out_ch<7, 2, 4>(s, w_out, ids, h, out, st);
     case 8: return launch_out_ch<8, 2, 4>(s, w_out, ids, h, out, st);
-    default: return launch_out_ch<16, 1, 4>(s, w_out, ids, h, out, st);
+    default: return launch_out_ch<16, 2, 4>(s, w_out, ids, h, out, st);
   }
 }
 
