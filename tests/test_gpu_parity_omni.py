@@ -60,6 +60,7 @@ def check_route(lg, nr, K, renorm, ids_gpu, w_gpu, tokens=None):
 @pytest.mark.parametrize("T,nr,nc,K", [
     (64, 8, 8, 1), (64, 8, 8, 64), (100, 16, 24, 40), (33, 32, 32, 200), (40, 320, 320, 512),
     (20, 13, 7, 50), (17, 1000, 3, 100), (12, 64, 64, 4096), (9, 1024, 1024, 300),
+    (5, 1024, 1024, 4096),  # staircase above the shared-memory key store: keys recomputed
 ])
 @pytest.mark.parametrize("renorm", [True, False])
 def test_route_on_given_logits(cuda_lib, T, nr, nc, K, renorm):

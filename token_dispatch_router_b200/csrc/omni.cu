@@ -186,48 +186,53 @@ __host__ __device__ inline int pow2_at_least(int n) {
   return p;
 }
 
-// Shared-memory layout of omni_topk (byte offsets; host and device agree).
+constexpr int kStairMax = 16384;  // staircase keys kept in shared memory (else recomputed)
+
+// Shared-memory layout of omni_topk (byte offsets), computed on the host and passed in.
+// The staircase: row r of the sorted grid keeps columns [0, min(nc, K / (r + 1))), for
+// r < min(nr, K); `stair` is its size.
 struct TopkSmem {
   int PP, KP;  // padded axis length and padded K (powers of two)
+  int stair, stored;  // staircase size; keys kept in shared memory (1) or recomputed (0)
   int o_rk, o_ck, o_sel, o_raw_r, o_raw_c, o_sv_r, o_sv_c, o_sid_r, o_sid_c, o_gt, o_tie,
-      o_gpos, o_tpos, o_hist, o_misc, total;
-  __host__ __device__ TopkSmem(int nr, int nc, int K) {
-    PP = pow2_at_least(nr > nc ? nr : nc);
-    KP = pow2_at_least(K);
-    int o = 0;
-    o_rk = o;
-    o += PP * 8;
-    o_ck = o;
-    o += PP * 8;
-    o_sel = o;
-    o += KP * 8;
-    o_raw_r = o;
-    o += nr * 4;
-    o_raw_c = o;
-    o += nc * 4;
-    o_sv_r = o;
-    o += nr * 4;
-    o_sv_c = o;
-    o += nc * 4;
-    o_sid_r = o;
-    o += nr * 4;
-    o_sid_c = o;
-    o += nc * 4;
-    o_gt = o;
-    o += nr * 4;
-    o_tie = o;
-    o += nr * 4;
-    o_gpos = o;
-    o += nr * 4;
-    o_tpos = o;
-    o += nr * 4;
-    o_hist = o;
-    o += 256 * 4;
-    o_misc = o;
-    o += 64 * 4;
-    total = o;
-  }
+      o_gpos, o_tpos, o_soff, o_skeys, o_hist, o_misc, total;
 };
+
+TopkSmem topk_smem_layout(int nr, int nc, int K) {
+  TopkSmem L;
+  L.PP = pow2_at_least(nr > nc ? nr : nc);
+  L.KP = pow2_at_least(K);
+  const int R = nr < K ? nr : K;
+  long long st = 0;
+  for (int r = 0; r < R; ++r) st += (nc < K / (r + 1)) ? nc : K / (r + 1);
+  L.stair = (int)st;
+  L.stored = st <= kStairMax;
+  int o = 0;
+  auto take = [&](int bytes) {
+    const int at = o;
+    o += (bytes + 15) & ~15;
+    return at;
+  };
+  L.o_rk = take(L.PP * 8);
+  L.o_ck = take(L.PP * 8);
+  L.o_sel = take(L.KP * 8);
+  L.o_raw_r = take(nr * 4);
+  L.o_raw_c = take(nc * 4);
+  L.o_sv_r = take(nr * 4);
+  L.o_sv_c = take(nc * 4);
+  L.o_sid_r = take(nr * 4);
+  L.o_sid_c = take(nc * 4);
+  L.o_gt = take(nr * 4);
+  L.o_tie = take(nr * 4);
+  L.o_gpos = take((nr + 1) * 4);
+  L.o_tpos = take((nr + 1) * 4);
+  L.o_soff = take((R + 1) * 4);
+  L.o_skeys = take(L.stored ? L.stair * 4 : 0);
+  L.o_hist = take(256 * 4);
+  L.o_misc = take(64 * 4);
+  L.total = o;
+  return L;
+}
 
 // Bitonic sort, descending, of n (a power of two) keys in shared memory; every thread calls.
 __device__ void bitonic_desc(uint64_t* a, uint64_t* b, int n) {
@@ -376,11 +381,12 @@ struct TopkArgs {
   float* w;             // [T, K]
   int T, nr, nc, K, renorm;
   unsigned* status;
+  TopkSmem L;
 };
 
 __global__ void __launch_bounds__(TK_THREADS) omni_topk_kernel(const TopkArgs g) {
   extern __shared__ __align__(16) uint8_t sm[];
-  const TopkSmem L(g.nr, g.nc, g.K);
+  const TopkSmem& L = g.L;
   uint64_t* rk = (uint64_t*)(sm + L.o_rk);
   uint64_t* ck = (uint64_t*)(sm + L.o_ck);
   uint64_t* sel = (uint64_t*)(sm + L.o_sel);
@@ -394,6 +400,8 @@ __global__ void __launch_bounds__(TK_THREADS) omni_topk_kernel(const TopkArgs g)
   int* s_tie = (int*)(sm + L.o_tie);
   int* gpos = (int*)(sm + L.o_gpos);
   int* tpos = (int*)(sm + L.o_tpos);
+  int* soff = (int*)(sm + L.o_soff);
+  uint32_t* skeys = (uint32_t*)(sm + L.o_skeys);
   int* hist = (int*)(sm + L.o_hist);
   int* misc = (int*)(sm + L.o_misc);  // [0..63]: scan partials, totals, digits, counters
   float* red = (float*)(sm + L.o_hist);  // reused after the selection
@@ -439,6 +447,35 @@ __global__ void __launch_bounds__(TK_THREADS) omni_topk_kernel(const TopkArgs g)
 
   // 2. threshold key: the K-th largest pair-sum key over the staircase of sorted ranks
   const int R = min(nr, K);
+  if (L.stored) {  // the staircase's keys, flattened row after row, in shared memory
+    for (int r = tid; r < R; r += TK_THREADS) s_gt[r] = min(nc, K / (r + 1));
+    __syncthreads();
+    block_exscan2(s_gt, s_gt, soff, s_tie, R, misc, misc + 48);
+    if (tid == 0) soff[R] = L.stair;
+    __syncthreads();
+    const int per = (L.stair + TK_THREADS - 1) / TK_THREADS;
+    int f = tid * per;
+    const int f1 = min(L.stair, f + per);
+    if (f < f1) {
+      int lo = 0, hi = R - 1;  // the row of f: last r with soff[r] <= f (rows are not empty)
+      while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (soff[mid] <= f) lo = mid;
+        else hi = mid - 1;
+      }
+      int r = lo, c = f - soff[lo], rend = soff[lo + 1];
+      float a = sv_r[r];
+      for (; f < f1; ++f, ++c) {
+        if (f == rend) {
+          ++r;
+          c = 0;
+          rend = soff[r + 1];
+          a = sv_r[r];
+        }
+        skeys[f] = ord_key(a + sv_c[c]);
+      }
+    }
+  }
   uint32_t prefix = 0, pmask = 0;
   int need = K;
   if (tid == 0) {
@@ -448,13 +485,19 @@ __global__ void __launch_bounds__(TK_THREADS) omni_topk_kernel(const TopkArgs g)
   for (int shift = 24; shift >= 0; shift -= 8) {
     for (int i = tid; i < 256; i += TK_THREADS) hist[i] = 0;
     __syncthreads();
-    for (int r = warp; r < R; r += TK_WARPS) {
-      const int Lr = min(nc, K / (r + 1));
-      const float a = sv_r[r];
-      for (int c0 = 0; c0 < Lr; c0 += 32) {
-        const int c = c0 + lane;
-        const uint32_t key = c < Lr ? ord_key(a + sv_c[c]) : 0u;
-        hist_add_warp(hist, c < Lr && (key & pmask) == prefix, (key >> shift) & 255);
+    if (L.stored) {
+      for (int f = tid; f < L.stair; f += TK_THREADS) {
+        const uint32_t key = skeys[f];
+        if ((key & pmask) == prefix) atomicAdd(&hist[(key >> shift) & 255], 1);
+      }
+    } else {
+      for (int r = warp; r < R; r += TK_WARPS) {
+        const int Lr = min(nc, K / (r + 1));
+        const float a = sv_r[r];
+        for (int c = lane; c < Lr; c += 32) {
+          const uint32_t key = ord_key(a + sv_c[c]);
+          if ((key & pmask) == prefix) atomicAdd(&hist[(key >> shift) & 255], 1);
+        }
       }
     }
     __syncthreads();
@@ -490,23 +533,36 @@ __global__ void __launch_bounds__(TK_THREADS) omni_topk_kernel(const TopkArgs g)
   block_exscan2(s_gt, s_tie, gpos, tpos, nr, misc, misc + 48);
   const int gt_total = misc[48], tie_total = misc[49];
   const int take = K - gt_total;  // pairs taken at the threshold, 1 <= take <= tie_total
+  if (tid == 0) {
+    gpos[nr] = gt_total;
+    tpos[nr] = tie_total;
+  }
 
-  // 4. the winners: every pair above the threshold, then the `take` lowest ids at it
+  // 4. the winners: every pair above the threshold, then the `take` lowest ids at it; one
+  // thread per output slot finds its row by a binary search over the row offsets
   for (int i = tid; i < L.KP; i += TK_THREADS) sel[i] = 0;
   __syncthreads();
-  for (int r = warp; r < nr; r += TK_WARPS) {
-    const float a = sv_r[r];
-    const uint32_t rid = (uint32_t)sid_r[r] * (uint32_t)nc;
-    for (int c = lane; c < s_gt[r]; c += 32)
-      if (gpos[r] + c < K) sel[gpos[r] + c] = composite(ord_key(a + sv_c[c]), rid + (uint32_t)sid_c[c]);
+  for (int k = tid; k < min(gt_total, K); k += TK_THREADS) {
+    int lo = 0, hi = nr - 1;
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      if (gpos[mid] <= k) lo = mid;
+      else hi = mid - 1;
+    }
+    const int c = k - gpos[lo];
+    sel[k] = composite(ord_key(sv_r[lo] + sv_c[c]), (uint32_t)sid_r[lo] * (uint32_t)nc + (uint32_t)sid_c[c]);
   }
   if (take == tie_total) {
-    for (int r = warp; r < nr; r += TK_WARPS) {
-      const uint32_t rid = (uint32_t)sid_r[r] * (uint32_t)nc;
-      const int c0 = s_gt[r];
-      for (int c = lane; c < s_tie[r]; c += 32)
-        if (gt_total + tpos[r] + c < K)
-          sel[gt_total + tpos[r] + c] = composite(theta, rid + (uint32_t)sid_c[c0 + c]);
+    for (int k = tid; k < tie_total; k += TK_THREADS) {
+      int lo = 0, hi = nr - 1;
+      while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (tpos[mid] <= k) lo = mid;
+        else hi = mid - 1;
+      }
+      const int c = s_gt[lo] + (k - tpos[lo]);
+      if (gt_total + k < K)
+        sel[gt_total + k] = composite(theta, (uint32_t)sid_r[lo] * (uint32_t)nc + (uint32_t)sid_c[c]);
     }
   } else {
     // radix select (ascending) of the take-th smallest id among the pairs at the threshold
@@ -1214,11 +1270,10 @@ moe_status launch_omni_logits(const moe_omni_shape& s, const void* x, const void
   }
 }
 
-int omni_topk_smem(const moe_omni_shape& s) { return TopkSmem(s.n_rows, s.n_cols, s.K).total; }
-
 moe_status launch_omni_topk(const moe_omni_shape& s, const float* logits, int32_t* ids, float* w,
                             cudaStream_t st) {
-  const int smem = omni_topk_smem(s);
+  const TopkSmem L = topk_smem_layout(s.n_rows, s.n_cols, s.K);
+  const int smem = L.total;
   if (!set_smem(omni_topk_kernel, smem)) return MOE_ERR_CUDA;
   TopkArgs a;
   a.logits = logits;
@@ -1230,6 +1285,7 @@ moe_status launch_omni_topk(const moe_omni_shape& s, const float* logits, int32_
   a.K = s.K;
   a.renorm = s.renormalize;
   a.status = device_status_ptr();
+  a.L = L;
   launch_begin(K_OMNI_TOPK, st);
   launch_kernel(omni_topk_kernel, dim3((unsigned)s.T), dim3(TK_THREADS), (size_t)smem, st, 1u, a);
   return launch_end(K_OMNI_TOPK, st);
