@@ -52,6 +52,8 @@ def parse():
                     help="tokens in the CPU oracle sample (0: the workload's whole batch)")
     ap.add_argument("--ref-tokens", type=int, default=64,
                     help="tokens per step of the reference arm (the CPU oracle)")
+    ap.add_argument("--only", choices=["atomic_experts"], default=None,
+                    help="run one secondary figure alone and print it (for profiling)")
     return ap.parse_args()
 
 
@@ -157,7 +159,8 @@ class ClockSampler:
                 "samples": len(sm)}
 
 
-# Source file of each kernel a profiles/ record may describe; the shared headers count too.
+# Source file of each kernel a profiles/ record may describe; the shared headers count too
+# (kernel_ids.h, the profiler's host-side kernel numbering, holds no device code).
 KERNEL_SOURCES = {"gateup_tc": "ffn_tc.cu", "down_tc": "ffn_tc.cu", "gateup_tc2": "ffn_tc2.cu",
                   "down_tc2": "ffn_tc2.cu", "route_tc": "route_tc.cu", "combine": "combine.cu",
                   "gather_rows": "permute.cu", "permute_cluster": "permute.cu"}
@@ -519,9 +522,84 @@ def backward_figure(tdr, cfg, s, x, w_r, wg, wu, wd, bias, world, peak_t, steps=
 
 
 # ------------------------------------------------------------------ our arm
+def atomic_experts_bytes(c) -> dict:
+    """Algorithmic HBM bytes of one atomic-expert forward (each tensor read or written once)
+    and the row gathers its two expert kernels make (one d-row per task and side)."""
+    T, d, K, N, P = c.T, c.d, c.K, c.N, c.n_rows + c.n_cols
+    M = T * K
+    hbm = (T * d * 2 + d * P * 2          # x, the two router tables
+           + 2 * T * P * 4                # logits written, read by the top-K
+           + 2 * M * 4 + 2 * M * 4        # ids and weights written; ids read by the schedule
+           + N * 4 * 2 + (N + 1) * 4 + 2 * M * 4  # counts, offsets, both task maps
+           + N * d * 2 + M * 4 * 3        # w_in once; task map, weights, scalars (act)
+           + N * d * 2 + M * 8 + T * d * 2)  # w_out once, ids and scalars, out (gather)
+    return {"hbm_bytes": int(hbm), "row_gather_bytes": int(2 * M * d * 2)}
+
+
+def atomic_experts_figure(tdr, world, peaks, n=10):
+    """Fine-grained (rank-1) experts behind a Cartesian-product router: the 4096-token layer
+    with 320 x 320 = 102,400 experts, K = 512, d = 1024, through moe_omni_forward. One
+    forward per L2 flush, CUDA events; per-kernel times from the library's event profiler."""
+    c = mi.OMNI_102K
+    inp = mi.make_omni_inputs(c)
+    s = tdr.make_omni_shape(c.T, c.d, c.n_rows, c.n_cols, c.K, c.renormalize)
+    x, wr, wc, wi, wo = (t.cuda() for t in (inp.x, inp.w_row, inp.w_col, inp.w_in, inp.w_out))
+    ws = torch.empty(tdr.omni_workspace_size(s), dtype=torch.uint8, device=x.device)
+    out = torch.empty(c.T, c.d, dtype=torch.bfloat16, device=x.device)
+
+    def once():
+        tdr.omni_forward(s, x, wr, wc, wi, wo, out=out, workspace=ws)
+
+    flush = torch.ones(64 << 20, dtype=torch.int64, device=x.device)
+    for _ in range(3):
+        once()
+    torch.cuda.synchronize()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(n)]
+    for a, b in ev:
+        flush.sum()
+        hold_gpu()
+        a.record()
+        once()
+        b.record()
+    torch.cuda.synchronize()
+    ms = max_over_ranks(sum(a.elapsed_time(b) for a, b in ev) / n, world)
+    del flush
+    prof = tdr.Profiler()
+    with prof:
+        for _ in range(n):
+            once()
+        torch.cuda.synchronize()
+    if tdr.device_status() != 0:
+        raise RuntimeError("device status set during the atomic-expert runs")
+    kern = {k: round(v[1] / n * 1e3, 1) for k, v in prof.results().items()}
+    counts = tdr.omni_workspace_views(s, ws)["counts"]
+    active = int((counts > 0).sum().item())
+    nb = atomic_experts_bytes(c)
+    peak = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
+    gbs = nb["hbm_bytes"] / (ms / 1e3) / 1e9
+    half = nb["row_gather_bytes"] / 2
+    gather = {k: round(half / (kern[k] / 1e6) / 1e12, 2) for k in ("omni_act", "omni_out")
+              if k in kern}
+    return {"workload": c.name, "T": c.T, "d": c.d, "grid": [c.n_rows, c.n_cols], "N": c.N,
+            "K": c.K, "ms": round(ms, 4), "tokens_per_s": c.T * world / (ms / 1e3),
+            "kernels_us": kern, "hbm_bytes": nb["hbm_bytes"], "hbm_gbs": round(gbs, 1),
+            "hbm_frac": round(gbs / peak, 4), "row_gather_bytes": nb["row_gather_bytes"],
+            "row_gather_tbs": gather, "active_experts": active,
+            "reuse_tasks_per_active_expert": round(c.T * c.K / max(active, 1), 2),
+            "note": "one forward per L2 flush (expert tables 420 MB > L2); hbm_frac counts each "
+                    "tensor once; the expert kernels are bound by 2 KB row gathers "
+                    "(row_gather_tbs: TB/s of rows moved per kernel)"}
+
+
 def run_ours(args, rank, world, local):
     import token_dispatch_router_b200 as tdr
     tdr.load_library()  # fails loudly if the CUDA library is missing
+    if args.only == "atomic_experts":
+        fig = atomic_experts_figure(tdr, world, load_peaks()[0], n=max(1, args.steps))
+        if rank == 0:
+            print(json.dumps({"atomic_experts": fig}), flush=True)
+        return
     cfg = mi.CONFIGS[args.workload]
     dt = torch.bfloat16 if cfg.dtype == "bf16" else torch.float32
     inp = mi.make_inputs(cfg)
@@ -649,6 +727,7 @@ def run_ours(args, rank, world, local):
     dd = decode_dispatch(tdr, world)
     tr = token_rounding_figure(tdr, cfg, x, w_r, wg, wu, wd, bias, world)
     bw = backward_figure(tdr, cfg, s, x, w_r, wg, wu, wd, bias, world, peak_t)
+    ae = atomic_experts_figure(tdr, world, peaks)
 
     # ---- per-kernel breakdown (ms per step) and the two secondary figures of the metric
     per_kernel = {k: round(ms / args.steps, 4) for k, (n, ms) in kern.items()}
@@ -663,7 +742,7 @@ def run_ours(args, rank, world, local):
                    "n": cfg.n, "global_batch": cfg.T * world, "parallelism": f"replicas{world}",
                    "l2": "inputs larger than L2: the 2.82 GB of expert weights stream every step"},
         "roofline": roofline, "gemm": gemm, "dispatch_combine": dc, "decode_dispatch": dd,
-        "token_rounding": tr, "backward_act": bw,
+        "token_rounding": tr, "backward_act": bw, "atomic_experts": ae,
         "kernel_ms_per_step": per_kernel,
         "gpu_launches": int(launches), "e2e": e2e,
     }

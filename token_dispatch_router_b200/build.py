@@ -37,7 +37,8 @@ def _sources():
 
 
 def _deps():
-    return _sources() + glob.glob(os.path.join(CSRC, "*.cuh")) + [
+    return _sources() + glob.glob(os.path.join(CSRC, "*.cuh")) + glob.glob(
+        os.path.join(CSRC, "*.h")) + [
         os.path.join(ROOT, "include", "moe.h"), os.path.abspath(__file__)]
 
 

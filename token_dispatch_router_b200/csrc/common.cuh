@@ -8,6 +8,7 @@
 
 #include <utility>
 
+#include "kernel_ids.h"
 #include "moe.h"
 
 namespace moe {
@@ -84,43 +85,6 @@ __device__ __forceinline__ uint64_t globaltimer_ns() {
 }
 
 // ---------------------------------------------------------------- host side
-// Kernel ids of the opt-in profiler (order = moe_kernel_name).
-enum KernelId {
-  K_ROUTE = 0,
-  K_HIST,
-  K_SCAN,
-  K_SCATTER,
-  K_GATHER,
-  K_GATEUP_TC,
-  K_DOWN_TC,
-  K_GATEUP_SIMT,
-  K_DOWN_SIMT,
-  K_COMBINE,
-  K_SELFTEST,
-  K_ROUTE_TC,
-  K_PERMUTE_SMALL,
-  K_GATEUP_TC2,
-  K_DOWN_TC2,
-  K_PERMUTE_CLUSTER,
-  K_ROUTE_PERMUTE,
-  K_TILE_ROUND,
-  K_BWD_ACT,
-  K_BWD_DW,
-  K_BWD_DX,
-  K_ROUTER_DLOGITS,
-  K_ROUTER_DWR,
-  K_ROUTER_DX,
-  K_OMNI_LOGITS,
-  K_OMNI_TOPK,
-  K_OMNI_COUNT,
-  K_OMNI_SCAN,
-  K_OMNI_SCATTER,
-  K_OMNI_SORT,
-  K_OMNI_ACT,
-  K_OMNI_OUT,
-  K_COUNT
-};
-
 unsigned int* device_status_ptr();  // status word of the current device
 int sm_count();                     // SMs of the current device (cached)
 void launch_begin(int kernel_id, cudaStream_t s);
