@@ -43,6 +43,7 @@ struct RouteArgs {
   int32_t* topk_ids;
   float* topk_w;
   int T, E, K, renorm, kblocks, S;
+  int rows;  // tokens per tile (<= 128): a tile's MMA rows past it belong to the next tile
   unsigned* status;
   unsigned long long limit_ns;
 };
@@ -220,7 +221,7 @@ __global__ void __launch_bounds__(R_THREADS) route_tc_kernel(const __grid_consta
       const uint32_t fb = saddr(&full[stage]);
       mbar_expect_tx(fb, STAGE);
       const uint32_t a = saddr(ring + stage * STAGE);
-      tma_load_2d(a, &tmX, kb * RBK, tile * RBM, fb);
+      tma_load_2d(a, &tmX, kb * RBK, tile * g.rows, fb);
 #pragma unroll
       for (int c = 0; c < NCH; ++c) tma_load_2d(a + RA_BYTES + c * RB_CHUNK, &tmW, c * 64, kb * RBK, fb);
       if (++stage == RSTAGES) {
@@ -286,7 +287,7 @@ __global__ void __launch_bounds__(R_THREADS) route_tc_kernel(const __grid_consta
     cluster_sync();
   } else {
     if (S > 1) cluster_sync();  // partials of ranks 1..S-1 are in their shared memory
-    const int t = tile * RBM + r;
+    const int t = tile * g.rows + r;
     const int E = g.E, K = g.K;
     // Outputs are staged in this CTA's (idle) ring and written back coalesced: the tile's
     // logits rows are one contiguous [128, E] block, its ids and weights [128, K] blocks.
@@ -363,8 +364,8 @@ __global__ void __launch_bounds__(R_THREADS) route_tc_kernel(const __grid_consta
       }
     }
     __syncthreads();
-    const int rows = min(RBM, g.T - tile * RBM);
-    const size_t t0 = (size_t)tile * RBM;
+    const int rows = min(g.rows, g.T - tile * g.rows);
+    const size_t t0 = (size_t)tile * g.rows;
     if (g.logits_out != nullptr)
       for (int i = tid; i < rows * E; i += R_THREADS)
         g.logits_out[t0 * E + i] = st_l[(i / E) * (E + 1) + i % E];
@@ -408,8 +409,36 @@ bool make_map_2d(CUtensorMap* m, const void* ptr, uint64_t inner, uint64_t outer
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// Clusters of S CTAs of this kernel that can be resident at once (clusters stay inside one
+// GPC, so this can be below SMs / S); cached per instantiation and S.
+template <typename Kern>
+int active_clusters(Kern kern, int smem, int S) {
+  static int cache[9] = {0};
+  if (S < 1 || S > 8) return 1;
+  if (cache[S] == 0) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)S);
+    cfg.blockDim = dim3(R_THREADS);
+    cfg.dynamicSmemBytes = (size_t)smem;
+    cudaLaunchAttribute attr;
+    attr.id = cudaLaunchAttributeClusterDimension;
+    attr.val.clusterDim.x = (unsigned)S;
+    attr.val.clusterDim.y = 1;
+    attr.val.clusterDim.z = 1;
+    cfg.attrs = &attr;
+    cfg.numAttrs = 1;
+    int n = 0;
+    if (cudaOccupancyMaxActiveClusters(&n, kern, &cfg) != cudaSuccess || n < 1) {
+      cudaGetLastError();
+      n = 1;
+    }
+    cache[S] = n;
+  }
+  return cache[S];
+}
+
 template <int N, int KM>
-moe_status launch_nk(const CUtensorMap& mx, const CUtensorMap& mw, const RouteArgs& a, int tiles,
+moe_status launch_nk(const CUtensorMap& mx, const CUtensorMap& mw, RouteArgs a, int tiles,
                     cudaStream_t st) {
   constexpr int NCH = (N + 63) / 64;
   constexpr int STAGE = RA_BYTES + NCH * RB_CHUNK;
@@ -417,6 +446,16 @@ moe_status launch_nk(const CUtensorMap& mx, const CUtensorMap& mw, const RouteAr
   auto kern = route_tc_kernel<N, KM>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
     return MOE_ERR_CUDA;
+  // With fewer 128-token tiles than clusters that fit at once, shorter tiles (at least 64
+  // tokens) put more SMs to work; the MMA still computes 128 rows, the surplus unwritten.
+  if (a.S > 1) {
+    const int fit = active_clusters(kern, smem, a.S);
+    const int want = min(fit, (a.T + 63) / 64);
+    if (want > tiles) {
+      a.rows = (a.T + want - 1) / want;
+      tiles = (a.T + a.rows - 1) / a.rows;
+    }
+  }
   launch_begin(K_ROUTE_TC, st);
   launch_kernel(kern, dim3((unsigned)(tiles * a.S)), dim3(R_THREADS), (size_t)smem, st,
                 (unsigned)a.S, mx, mw, a);
@@ -471,6 +510,7 @@ moe_status launch_route_tc(const moe_shape& s, const void* x, const void* w_r, c
   a.renorm = s.renormalize;
   a.kblocks = kblocks;
   a.S = S;
+  a.rows = RBM;
   a.status = device_status_ptr();
   a.limit_ns = kWaitLimitNs;
   // instantiations cover N up to the next of 16/32/64/128/256; columns past E read zeros
