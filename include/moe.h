@@ -355,8 +355,8 @@ typedef struct {
   size_t topk_w;         /* fp32 [T, K] */
   size_t counts;         /* int32 [N] tasks per expert */
   size_t offsets;        /* int32 [N + 1] */
-  size_t assign_to_perm; /* int32 [T * K] */
-  size_t perm_to_assign; /* int32 [T * K] */
+  size_t assign_to_perm; /* int32 [T * K] (not written by moe_omni_forward) */
+  size_t perm_to_assign; /* int32 [T * K], grouped by expert */
   size_t h;              /* fp32 [T * K] per-task scalar w_{t,k} silu(x_t . w_in[i_k]) */
   size_t scratch;        /* the schedule's scratch */
   size_t total;
@@ -396,7 +396,10 @@ moe_status moe_omni_experts(const moe_omni_shape* shape, const void* x, const vo
                             void* out, moe_stream_t stream);
 
 /* moe_omni_forward - route + schedule + experts with every intermediate in `workspace`
- * (layout from moe_omni_workspace_layout). logits_in as in moe_omni_route. */
+ * (layout from moe_omni_workspace_layout). logits_in as in moe_omni_route. The experts need
+ * the tasks grouped by expert only, so inside the workspace perm_to_assign is grouped by
+ * expert with the order inside an expert unspecified, and assign_to_perm is not written
+ * (moe_omni_schedule gives the stable order); the output does not depend on that order. */
 moe_status moe_omni_forward(const moe_omni_shape* shape, const void* x, const void* w_row,
                             const void* w_col, const float* logits_in, const void* w_in,
                             const void* w_out, void* out, void* workspace, size_t ws_bytes,

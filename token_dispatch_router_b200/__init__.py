@@ -593,7 +593,8 @@ def omni_forward(shape: moe_omni_shape, x, w_row, w_col, w_in, w_out, logits_in=
 
 
 def omni_workspace_views(shape: moe_omni_shape, workspace: torch.Tensor) -> dict:
-    """Typed views of moe_omni_forward's intermediates inside its workspace."""
+    """Typed views of moe_omni_forward's intermediates inside its workspace (perm_to_assign
+    grouped by expert, any order inside an expert; assign_to_perm is not written)."""
     L = omni_workspace_layout(shape)
     T, K = shape.T, shape.K
     N, P, M = shape.n_rows * shape.n_cols, shape.n_rows + shape.n_cols, shape.T * shape.K

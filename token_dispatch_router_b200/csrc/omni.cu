@@ -200,8 +200,8 @@ struct TopkSmem {
 
 TopkSmem topk_smem_layout(int nr, int nc, int K) {
   TopkSmem L;
-  L.PP = pow2_at_least(nr > nc ? nr : nc);
-  L.KP = pow2_at_least(K);
+  L.PP = pow2_at_least(max(256, nr > nc ? nr : nc));  // the sorts work on 256 x 2^i keys
+  L.KP = pow2_at_least(max(256, K));
   const int R = nr < K ? nr : K;
   long long st = 0;
   for (int r = 0; r < R; ++r) st += (nc < K / (r + 1)) ? nc : K / (r + 1);
@@ -234,30 +234,88 @@ TopkSmem topk_smem_layout(int nr, int nc, int K) {
   return L;
 }
 
-// Bitonic sort, descending, of n (a power of two) keys in shared memory; every thread calls.
-__device__ void bitonic_desc(uint64_t* a, uint64_t* b, int n) {
-  for (int k = 2; k <= n; k <<= 1) {
-    for (int j = k >> 1; j > 0; j >>= 1) {
+// Bitonic sort, descending, of n = 256 * PER keys in shared memory by the CTA's 256 threads.
+// Warp w owns the block [w B, (w + 1) B), B = 32 PER, one key per lane in each of PER
+// slots. Stages whose partner lies in the same block run in registers (partner j < 32
+// lanes away: a shuffle; j >= 32: another slot of the same lane); only the stages with
+// j >= B exchange through shared memory. Every thread calls.
+template <int PER>
+__device__ __forceinline__ void reg_stage(uint64_t (&v)[PER], int base, int k, int j) {
+  const int lane = threadIdx.x & 31;
+  if (j >= 32) {
+    const int js = j >> 5;
+#pragma unroll
+    for (int sl = 0; sl < PER; ++sl) {
+      if ((sl & js) == 0) {
+        const int i = base + sl * 32 + lane;
+        const bool desc = (i & k) == 0;
+        const uint64_t x = v[sl], y = v[sl | js];
+        if (desc ? (x < y) : (x > y)) {
+          v[sl] = y;
+          v[sl | js] = x;
+        }
+      }
+    }
+  } else {
+    const bool lower = (lane & j) == 0;
+#pragma unroll
+    for (int sl = 0; sl < PER; ++sl) {
+      const int i = base + sl * 32 + lane;
+      const bool desc = (i & k) == 0;
+      const uint64_t y = __shfl_xor_sync(0xffffffffu, v[sl], j);
+      const bool keep_max = lower == desc;
+      v[sl] = keep_max ? (v[sl] > y ? v[sl] : y) : (v[sl] < y ? v[sl] : y);
+    }
+  }
+}
+
+template <int PER>
+__device__ void bitonic_desc_t(uint64_t* a) {
+  constexpr int B = 32 * PER, n = 8 * B;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int base = warp * B;
+  uint64_t v[PER];
+#pragma unroll
+  for (int sl = 0; sl < PER; ++sl) v[sl] = a[base + sl * 32 + lane];
+#pragma unroll
+  for (int k = 2; k <= B; k <<= 1)
+#pragma unroll
+    for (int j = k >> 1; j > 0; j >>= 1) reg_stage<PER>(v, base, k, j);
+#pragma unroll
+  for (int sl = 0; sl < PER; ++sl) a[base + sl * 32 + lane] = v[sl];
+  __syncthreads();
+  for (int k = 2 * B; k <= n; k <<= 1) {
+    for (int j = k >> 1; j >= B; j >>= 1) {
       for (int p = threadIdx.x; p < (n >> 1); p += blockDim.x) {
         const int i = ((p & ~(j - 1)) << 1) | (p & (j - 1));
         const int l = i + j;
         const bool desc = (i & k) == 0;
-        uint64_t x = a[i], y = a[l];
+        const uint64_t x = a[i], y = a[l];
         if (desc ? (x < y) : (x > y)) {
           a[i] = y;
           a[l] = x;
         }
-        if (b != nullptr) {
-          x = b[i];
-          y = b[l];
-          if (desc ? (x < y) : (x > y)) {
-            b[i] = y;
-            b[l] = x;
-          }
-        }
       }
       __syncthreads();
     }
+#pragma unroll
+    for (int sl = 0; sl < PER; ++sl) v[sl] = a[base + sl * 32 + lane];
+#pragma unroll
+    for (int j = B >> 1; j > 0; j >>= 1) reg_stage<PER>(v, base, k, j);
+#pragma unroll
+    for (int sl = 0; sl < PER; ++sl) a[base + sl * 32 + lane] = v[sl];
+    __syncthreads();
+  }
+}
+
+// n is a power of two from 256 to 4096.
+__device__ void bitonic_desc(uint64_t* a, int n) {
+  switch (n >> 8) {
+    case 1: bitonic_desc_t<1>(a); break;
+    case 2: bitonic_desc_t<2>(a); break;
+    case 4: bitonic_desc_t<4>(a); break;
+    case 8: bitonic_desc_t<8>(a); break;
+    default: bitonic_desc_t<16>(a); break;
   }
 }
 
@@ -381,6 +439,7 @@ struct TopkArgs {
   float* w;             // [T, K]
   int T, nr, nc, K, renorm;
   unsigned* status;
+  int32_t* counts;  // [N] or NULL: tasks per expert, counted as the ids are written
   TopkSmem L;
 };
 
@@ -432,7 +491,8 @@ __global__ void __launch_bounds__(TK_THREADS) omni_topk_kernel(const TopkArgs g)
     }
   }
   __syncthreads();
-  bitonic_desc(rk, ck, L.PP);
+  bitonic_desc(rk, L.PP);
+  bitonic_desc(ck, L.PP);
   for (int i = tid; i < nr; i += TK_THREADS) {
     const int id = (int)(0xFFFFFFFFu - (uint32_t)rk[i]);
     sid_r[i] = id;
@@ -604,7 +664,7 @@ __global__ void __launch_bounds__(TK_THREADS) omni_topk_kernel(const TopkArgs g)
     }
   }
   __syncthreads();
-  bitonic_desc(sel, nullptr, L.KP);
+  bitonic_desc(sel, L.KP);
   // every slot below K holds a pair unless the logits held a NaN: such a slot decodes to
   // expert 0 and the fault is reported
   const uint32_t N = (uint32_t)nr * (uint32_t)nc;
@@ -644,6 +704,7 @@ __global__ void __launch_bounds__(TK_THREADS) omni_topk_kernel(const TopkArgs g)
     if (g.renorm) w = expf(a + b - v0) / zr;
     else w = (expf(a - mr) / zr) * (expf(b - mc) / zc);
     g.ids[(size_t)t * K + k] = (int32_t)id;
+    if (g.counts != nullptr) atomicAdd(&g.counts[id], 1);
     g.w[(size_t)t * K + k] = w;
   }
 }
@@ -1271,7 +1332,7 @@ moe_status launch_omni_logits(const moe_omni_shape& s, const void* x, const void
 }
 
 moe_status launch_omni_topk(const moe_omni_shape& s, const float* logits, int32_t* ids, float* w,
-                            cudaStream_t st) {
+                            int32_t* counts, cudaStream_t st) {
   const TopkSmem L = topk_smem_layout(s.n_rows, s.n_cols, s.K);
   const int smem = L.total;
   if (!set_smem(omni_topk_kernel, smem)) return MOE_ERR_CUDA;
@@ -1285,6 +1346,7 @@ moe_status launch_omni_topk(const moe_omni_shape& s, const float* logits, int32_
   a.K = s.K;
   a.renorm = s.renormalize;
   a.status = device_status_ptr();
+  a.counts = counts;
   a.L = L;
   launch_begin(K_OMNI_TOPK, st);
   launch_kernel(omni_topk_kernel, dim3((unsigned)s.T), dim3(TK_THREADS), (size_t)smem, st, 1u, a);
@@ -1298,9 +1360,26 @@ size_t omni_schedule_scratch_bytes(const moe_omni_shape& s) {
   return (N + M + N + 64 + 256) * 4;
 }
 
+// Zeroes the schedule's per-expert counts and cursors and its queue length.
+moe_status launch_omni_zero(const moe_omni_shape& s, int32_t* counts, void* scratch,
+                            cudaStream_t st) {
+  const int N = s.n_rows * s.n_cols;
+  const long long M = (long long)s.T * s.K;
+  int32_t* cursor = (int32_t*)scratch;
+  int32_t* big_count = cursor + N + M + N;
+  launch_begin(K_OMNI_COUNT, st);
+  launch_kernel(omni_zero_kernel, dim3((unsigned)grid_cap(N, 256, 4)), dim3(256), 0, st, 1u, counts,
+                cursor, (long long)N, big_count);
+  return launch_end(K_OMNI_COUNT, st);
+}
+
+// The task list grouped by expert. counted: counts were zeroed and filled already (by the
+// top-K kernel). stable: each expert's slots sorted by assignment id (= token) and
+// assign_to_perm written; otherwise the order inside an expert is the order the scatter
+// claimed the slots in, and assign_to_perm is not written.
 moe_status launch_omni_schedule(const moe_omni_shape& s, const int32_t* ids, int32_t* counts,
                                 int32_t* offsets, int32_t* a2p, int32_t* p2a, void* scratch,
-                                cudaStream_t st) {
+                                bool counted, bool stable, cudaStream_t st) {
   const int N = s.n_rows * s.n_cols;
   const long long M = (long long)s.T * s.K;
   int32_t* cursor = (int32_t*)scratch;
@@ -1310,14 +1389,13 @@ moe_status launch_omni_schedule(const moe_omni_shape& s, const int32_t* ids, int
   int32_t* scan_sums = big_count + 64;
   unsigned* status = device_status_ptr();
   moe_status r;
-  launch_begin(K_OMNI_COUNT, st);
-  launch_kernel(omni_zero_kernel, dim3((unsigned)grid_cap(N, 256, 4)), dim3(256), 0, st, 1u, counts,
-                cursor, (long long)N, big_count);
-  if ((r = launch_end(K_OMNI_COUNT, st)) != MOE_OK) return r;
-  launch_begin(K_OMNI_COUNT, st);
-  launch_kernel(omni_count_kernel, dim3((unsigned)grid_cap(M, 256, 8)), dim3(256), 0, st, 1u, ids, M,
-                N, counts, status);
-  if ((r = launch_end(K_OMNI_COUNT, st)) != MOE_OK) return r;
+  if (!counted) {
+    if ((r = launch_omni_zero(s, counts, scratch, st)) != MOE_OK) return r;
+    launch_begin(K_OMNI_COUNT, st);
+    launch_kernel(omni_count_kernel, dim3((unsigned)grid_cap(M, 256, 8)), dim3(256), 0, st, 1u, ids,
+                  M, N, counts, status);
+    if ((r = launch_end(K_OMNI_COUNT, st)) != MOE_OK) return r;
+  }
   const int scan_tiles = (N + kScanTile - 1) / kScanTile;
   launch_begin(K_OMNI_SCAN, st);
   launch_kernel(omni_scan_sums_kernel, dim3((unsigned)scan_tiles), dim3(1024), 0, st, 1u,
@@ -1329,8 +1407,9 @@ moe_status launch_omni_schedule(const moe_omni_shape& s, const int32_t* ids, int
   if ((r = launch_end(K_OMNI_SCAN, st)) != MOE_OK) return r;
   launch_begin(K_OMNI_SCATTER, st);
   launch_kernel(omni_scatter_kernel, dim3((unsigned)grid_cap(M, 256, 8)), dim3(256), 0, st, 1u, ids,
-                M, N, (const int32_t*)offsets, cursor, tmp);
+                M, N, (const int32_t*)offsets, cursor, stable ? tmp : p2a);
   if ((r = launch_end(K_OMNI_SCATTER, st)) != MOE_OK) return r;
+  if (!stable) return MOE_OK;
   launch_begin(K_OMNI_SORT, st);
   launch_kernel(omni_segsort_kernel, dim3((unsigned)grid_cap((long long)N * 32, 256, 8)), dim3(256), 0,
                 st, 1u, (const int32_t*)offsets, N, (const int32_t*)tmp, p2a, a2p, big_list,
@@ -1427,7 +1506,7 @@ bool al16(const void* p) { return ((uintptr_t)p & 15) == 0; }
 
 moe_status omni_route_impl(const moe_omni_shape& s, const void* x, const void* w_row,
                            const void* w_col, const float* logits_in, float* logits_out,
-                           int32_t* ids, float* w, cudaStream_t st) {
+                           int32_t* ids, float* w, int32_t* counts, cudaStream_t st) {
   const float* lg = logits_in;
   if (lg == nullptr) {
     if (!x || !w_row || !w_col || !logits_out) return MOE_ERR_INVALID_ARG;
@@ -1437,7 +1516,7 @@ moe_status omni_route_impl(const moe_omni_shape& s, const void* x, const void* w
     if (r != MOE_OK) return r;
     lg = logits_out;
   }
-  return launch_omni_topk(s, lg, ids, w, st);
+  return launch_omni_topk(s, lg, ids, w, counts, st);
 }
 
 }  // namespace
@@ -1469,7 +1548,7 @@ moe_status moe_omni_route(const moe_omni_shape* s, const void* x, const void* w_
   if (r != MOE_OK) return r;
   if (s->T == 0) return MOE_OK;
   if (!topk_ids || !topk_w) return MOE_ERR_INVALID_ARG;
-  return omni_route_impl(*s, x, w_row, w_col, logits_in, logits_out, topk_ids, topk_w,
+  return omni_route_impl(*s, x, w_row, w_col, logits_in, logits_out, topk_ids, topk_w, nullptr,
                          (cudaStream_t)stream);
 }
 
@@ -1484,7 +1563,7 @@ moe_status moe_omni_schedule(const moe_omni_shape* s, const int32_t* topk_ids, i
   omni_layout(*s, &L);
   if (workspace == nullptr || ws_bytes < L.total) return MOE_ERR_WORKSPACE;
   return launch_omni_schedule(*s, topk_ids, counts, offsets, assign_to_perm, perm_to_assign,
-                              (uint8_t*)workspace + L.scratch, (cudaStream_t)stream);
+                              (uint8_t*)workspace + L.scratch, false, true, (cudaStream_t)stream);
 }
 
 moe_status moe_omni_experts(const moe_omni_shape* s, const void* x, const void* w_in,
@@ -1524,8 +1603,13 @@ moe_status moe_omni_forward(const moe_omni_shape* s, const void* x, const void* 
   int32_t* p2a = (int32_t*)(ws + L.perm_to_assign);
   float* h = (float*)(ws + L.h);
   const cudaStream_t st = (cudaStream_t)stream;
-  if ((r = omni_route_impl(*s, x, w_row, w_col, logits_in, logits, ids, w, st)) != MOE_OK) return r;
-  if ((r = launch_omni_schedule(*s, ids, counts, offsets, a2p, p2a, ws + L.scratch, st)) != MOE_OK)
+  // counts are zeroed first and filled by the top-K kernel; the experts need the tasks
+  // grouped by expert only, so the order inside an expert is left as the scatter made it
+  if ((r = launch_omni_zero(*s, counts, ws + L.scratch, st)) != MOE_OK) return r;
+  if ((r = omni_route_impl(*s, x, w_row, w_col, logits_in, logits, ids, w, counts, st)) != MOE_OK)
+    return r;
+  if ((r = launch_omni_schedule(*s, ids, counts, offsets, a2p, p2a, ws + L.scratch, true, false,
+                                st)) != MOE_OK)
     return r;
   return moe_omni_experts(s, x, w_in, w_out, ids, w, offsets, p2a, h, out, stream);
 }
