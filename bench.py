@@ -52,7 +52,7 @@ def parse():
                     help="tokens in the CPU oracle sample (0: the workload's whole batch)")
     ap.add_argument("--ref-tokens", type=int, default=64,
                     help="tokens per step of the reference arm (the CPU oracle)")
-    ap.add_argument("--only", choices=["atomic_experts"], default=None,
+    ap.add_argument("--only", choices=["atomic_experts", "backward"], default=None,
                     help="run one secondary figure alone and print it (for profiling)")
     return ap.parse_args()
 
@@ -615,6 +615,15 @@ def run_ours(args, rank, world, local):
 
     def step():
         tdr.forward(s, x, w_r, wg, wu, wd, bias=bias, out=out, workspace=ws)
+
+    if args.only == "backward":
+        peaks = load_peaks()[0]
+        peak_t = float(peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"]))
+        fig = backward_figure(tdr, cfg, s, x, w_r, wg, wu, wd, bias, world, peak_t,
+                              steps=max(1, args.steps))
+        if rank == 0:
+            print(json.dumps({"backward_act": fig}), flush=True)
+        return
 
     for _ in range(max(3, args.warmup)):
         step()
