@@ -573,6 +573,24 @@ def atomic_experts_figure(tdr, world, peaks, n=10):
     if tdr.device_status() != 0:
         raise RuntimeError("device status set during the atomic-expert runs")
     kern = {k: round(v[1] / n * 1e3, 1) for k, v in prof.results().items()}
+    # the page's output side for comparison: expert-centric scatter-add (atomic fp32 rows)
+    tdr.omni_set_output_mode(1)
+    try:
+        for _ in range(2):
+            once()
+        torch.cuda.synchronize()
+        prof2 = tdr.Profiler()
+        with prof2:
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            for _ in range(n):
+                once()
+            e1.record()
+            torch.cuda.synchronize()
+        scatter = {"ms_back_to_back": round(max_over_ranks(e0.elapsed_time(e1) / n, world), 4),
+                   "output_us": round(prof2.results()["omni_out"][1] / n * 1e3, 1)}
+    finally:
+        tdr.omni_set_output_mode(0)
     counts = tdr.omni_workspace_views(s, ws)["counts"]
     active = int((counts > 0).sum().item())
     nb = atomic_experts_bytes(c)
@@ -585,11 +603,13 @@ def atomic_experts_figure(tdr, world, peaks, n=10):
             "K": c.K, "ms": round(ms, 4), "tokens_per_s": c.T * world / (ms / 1e3),
             "kernels_us": kern, "hbm_bytes": nb["hbm_bytes"], "hbm_gbs": round(gbs, 1),
             "hbm_frac": round(gbs / peak, 4), "row_gather_bytes": nb["row_gather_bytes"],
-            "row_gather_tbs": gather, "active_experts": active,
+            "row_gather_tbs": gather, "scatter_add_output": scatter, "active_experts": active,
             "reuse_tasks_per_active_expert": round(c.T * c.K / max(active, 1), 2),
             "note": "one forward per L2 flush (expert tables 420 MB > L2); hbm_frac counts each "
                     "tensor once; the expert kernels are bound by 2 KB row gathers "
-                    "(row_gather_tbs: TB/s of rows moved per kernel)"}
+                    "(row_gather_tbs: TB/s of rows moved per kernel); scatter_add_output: the "
+                    "same forward with the expert-centric scatter-add on the output side "
+                    "(zero, atomic fp32 rows, bf16 rounding), back to back"}
 
 
 def run_ours(args, rank, world, local):

@@ -359,6 +359,7 @@ typedef struct {
   size_t perm_to_assign; /* int32 [T * K], grouped by expert */
   size_t h;              /* fp32 [T * K] per-task scalar w_{t,k} silu(x_t . w_in[i_k]) */
   size_t scratch;        /* the schedule's scratch */
+  size_t y32;            /* fp32 [T, d] output accumulator (scatter-add output mode) */
   size_t total;
 } moe_omni_layout;
 
@@ -404,6 +405,14 @@ moe_status moe_omni_forward(const moe_omni_shape* shape, const void* x, const vo
                             const void* w_col, const float* logits_in, const void* w_in,
                             const void* w_out, void* out, void* workspace, size_t ws_bytes,
                             moe_stream_t stream);
+
+/* Output side of moe_omni_forward (process-wide, not thread safe): 0 (default) = token-centric
+ * gather, y_t = sum_k h w_out[i_k] summed per token in slot order (deterministic); 1 = the
+ * page's expert-centric scatter-add (section 2.3): each expert's w_out row is read once and
+ * h * w_out[e] is added into its tokens' fp32 rows with atomic vector reductions, then
+ * rounded to bf16 (the fp32 sum order, and so the last bits, vary from run to run). */
+moe_status moe_omni_set_output_mode(int mode);
+int moe_omni_get_output_mode(void);
 
 /* ----------------------------------------------------------------------------
  * Device status: synchronises `stream`, returns the first device-side fault

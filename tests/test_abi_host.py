@@ -166,9 +166,9 @@ def test_omni_workspace_layout_is_host_arithmetic(lib):
     N, M = nr * nc, T * K
     assert L.logits == 0 and L.topk_ids >= T * (nr + nc) * 4
     assert L.h - L.perm_to_assign >= M * 4 and L.scratch - L.h >= M * 4
-    assert L.total >= L.scratch + (2 * N + M) * 4
+    assert L.y32 >= L.scratch + (2 * N + M) * 4 and L.total >= L.y32 + T * d * 4
     for f in ("topk_ids", "topk_w", "counts", "offsets", "assign_to_perm", "perm_to_assign",
-              "h", "scratch", "total"):
+              "h", "scratch", "y32", "total"):
         assert getattr(L, f) % 256 == 0
     assert lib.moe_omni_workspace_size(ctypes.byref(s)) == L.total
 
@@ -193,6 +193,8 @@ def test_omni_argument_checks_on_host(lib):
     # experts without the scalar buffer
     assert lib.moe_omni_experts(ctypes.byref(s), dummy, dummy, dummy, dummy, dummy, dummy, dummy,
                                 None, dummy, None) == 1
+    # output modes: 0 and 1 only
+    assert lib.moe_omni_set_output_mode(2) == 1 and lib.moe_omni_get_output_mode() == 0
     # T = 0 is a no-op
     z = tdr.make_omni_shape(0, 256, 8, 8, 4)
     assert lib.moe_omni_route(ctypes.byref(z), None, None, None, None, None, None, None,

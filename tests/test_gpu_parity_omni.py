@@ -172,8 +172,17 @@ def test_experts_given_routing(cuda_lib, T, d, nr, nc, K):
     assert_bf16_close(out.float().cpu().numpy(), y_ref, "out")
 
 
+@pytest.fixture(params=[0, 1], ids=["gather_out", "scatter_add_out"])
+def output_mode(request, cuda_lib):
+    """Run a forward test with the token-centric gather and with the expert-centric
+    scatter-add on the output side."""
+    cuda_lib.omni_set_output_mode(request.param)
+    yield request.param
+    cuda_lib.omni_set_output_mode(0)
+
+
 @pytest.mark.parametrize("renorm", [True, False])
-def test_forward_small(cuda_lib, renorm):
+def test_forward_small(cuda_lib, renorm, output_mode):
     tdr = cuda_lib
     c = cfg_of(256, 256, 32, 32, 64, renorm)
     inp = mi.make_omni_inputs(c)
@@ -203,7 +212,7 @@ def test_forward_small(cuda_lib, renorm):
     assert_bf16_close(out.float().cpu().numpy(), y_ec, "out (expert-centric oracle)")
 
 
-def test_forward_102k_experts_sampled_tokens(cuda_lib):
+def test_forward_102k_experts_sampled_tokens(cuda_lib, output_mode):
     """The 4096-token layer with 320 x 320 = 102,400 experts, K = 512, d = 1024: every
     routing output is checked on 12 sampled tokens (brute force over all N pairs), the
     schedule by its invariants and counts, the output on the same tokens."""

@@ -52,7 +52,7 @@ class moe_omni_shape(ctypes.Structure):
 class moe_omni_layout(ctypes.Structure):
     _fields_ = [(f, ctypes.c_size_t) for f in (
         "logits", "topk_ids", "topk_w", "counts", "offsets", "assign_to_perm",
-        "perm_to_assign", "h", "scratch", "total")]
+        "perm_to_assign", "h", "scratch", "y32", "total")]
 
 
 _P = ctypes.c_void_p
@@ -83,6 +83,8 @@ _SIGS = {
     "moe_omni_experts": (ctypes.c_int, [_O, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P]),
     "moe_omni_forward": (ctypes.c_int, [_O, _P, _P, _P, _P, _P, _P, _P, _P, ctypes.c_size_t,
                                         _P]),
+    "moe_omni_set_output_mode": (ctypes.c_int, [ctypes.c_int]),
+    "moe_omni_get_output_mode": (ctypes.c_int, []),
     "moe_get_device_status": (ctypes.c_int, [_P]),
     "moe_status_string": (ctypes.c_char_p, [ctypes.c_int]),
     "moe_profile_enable": (ctypes.c_int, [ctypes.c_int]),
@@ -590,6 +592,15 @@ def omni_forward(shape: moe_omni_shape, x, w_row, w_col, w_in, w_out, logits_in=
                                 _ptr(workspace), workspace.numel(), _stream()),
            "moe_omni_forward")
     return out, workspace
+
+
+def omni_set_output_mode(mode: int) -> None:
+    """0 = token-centric gather (default, deterministic); 1 = expert-centric scatter-add."""
+    _check(load_library().moe_omni_set_output_mode(int(mode)), "moe_omni_set_output_mode")
+
+
+def omni_get_output_mode() -> int:
+    return int(load_library().moe_omni_get_output_mode())
 
 
 def omni_workspace_views(shape: moe_omni_shape, workspace: torch.Tensor) -> dict:

@@ -1223,6 +1223,104 @@ __global__ void __launch_bounds__(WPT * 32) omni_out_kernel(const bf16* __restri
   }
 }
 
+// The page's output side (section 2.3: results added back per token by scatter-add), kept
+// as a measured alternative to the token-centric gather: each warp owns an equal range of
+// the expert-major task list, keeps the current expert's w_out row in registers and adds
+// h[a] * w_out[e] into the token's fp32 row with vector reductions (red.global.add.v4.f32).
+// The sum order is the order the reductions land in, so results vary in the last bits.
+__global__ void omni_zero_f32_kernel(float4* __restrict__ y, long long n4) {
+  pdl_wait();
+  pdl_trigger();
+  for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < n4;
+       i += (long long)gridDim.x * blockDim.x)
+    y[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+}
+
+__device__ __forceinline__ void red_add_v4(float* dst, float a, float b, float c, float d) {
+  asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(dst), "f"(a), "f"(b), "f"(c),
+               "f"(d)
+               : "memory");
+}
+
+template <int CH>
+__global__ void __launch_bounds__(256) omni_scatter_out_kernel(const bf16* __restrict__ w_out,
+                                                               const int32_t* __restrict__ offsets,
+                                                               const int32_t* __restrict__ p2a,
+                                                               const float* __restrict__ h,
+                                                               float* __restrict__ y32, int N,
+                                                               int K, int d, int M,
+                                                               unsigned* status) {
+  pdl_wait();
+  pdl_trigger();
+  const int lane = threadIdx.x & 31, wpc = blockDim.x >> 5;
+  const long long nw = (long long)gridDim.x * wpc, gw = (long long)blockIdx.x * wpc + (threadIdx.x >> 5);
+  const long long per = ((long long)M + nw - 1) / nw;
+  const int P0 = (int)min((long long)M, gw * per), P1 = (int)min((long long)M, gw * per + per);
+  if (P0 >= P1) return;
+  if (offsets[N] != M) {
+    if (lane == 0) report(status, MOE_ERR_DEVICE_INDEX);
+    return;
+  }
+  int lo = 0, hi = N - 1;
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (offsets[mid] <= P0) lo = mid;
+    else hi = mid - 1;
+  }
+  int e = lo, e_end = offsets[e + 1];
+  uint4 wv[CH];
+  {
+    const uint4* wr = reinterpret_cast<const uint4*>(w_out + (size_t)e * d);
+#pragma unroll
+    for (int j = 0; j < CH; ++j) wv[j] = ldg_nc(wr + lane + 32 * j);
+  }
+  for (int base = P0; base < P1; base += 32) {
+    const int a = base + lane < P1 ? p2a[base + lane] : -1;
+    const bool ok = (unsigned)a < (unsigned)M;
+    const int tl = ok ? a / K : -1;
+    const float hl = ok ? h[a] : 0.f;
+    const int n = min(32, P1 - base);
+    for (int i = 0; i < n; ++i) {
+      const int p = base + i;
+      if (p >= e_end) {
+        while (p >= e_end && e < N - 1) {
+          ++e;
+          e_end = offsets[e + 1];
+        }
+        const uint4* wr = reinterpret_cast<const uint4*>(w_out + (size_t)e * d);
+#pragma unroll
+        for (int j = 0; j < CH; ++j) wv[j] = ldg_nc(wr + lane + 32 * j);
+      }
+      const int t = __shfl_sync(0xffffffffu, tl, i);
+      const float hv = __shfl_sync(0xffffffffu, hl, i);
+      if (t < 0) {
+        if (lane == 0) report(status, MOE_ERR_DEVICE_INDEX);
+        continue;
+      }
+      float* row = y32 + (size_t)t * d;
+#pragma unroll
+      for (int j = 0; j < CH; ++j) {
+        float f[8];
+        unpack16(wv[j], f, bf16());
+        float* dst = row + (lane + 32 * j) * 8;
+        red_add_v4(dst, hv * f[0], hv * f[1], hv * f[2], hv * f[3]);
+        red_add_v4(dst + 4, hv * f[4], hv * f[5], hv * f[6], hv * f[7]);
+      }
+    }
+  }
+}
+
+__global__ void omni_to_bf16_kernel(const float4* __restrict__ y32, uint2* __restrict__ out,
+                                    long long n4) {
+  pdl_wait();
+  pdl_trigger();
+  for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < n4;
+       i += (long long)gridDim.x * blockDim.x) {
+    const float4 v = y32[i];
+    out[i] = make_uint2(pack_bf16x2(v.x, v.y), pack_bf16x2(v.z, v.w));
+  }
+}
+
 // ------------------------------------------------------------------ host launchers
 template <typename Kern>
 bool set_smem(Kern k, int bytes) {
@@ -1455,6 +1553,46 @@ moe_status launch_omni_out(const moe_omni_shape& s, const void* w_out, const int
   }
 }
 
+int g_omni_output_mode = 0;  // 0 token-centric gather, 1 expert-centric scatter-add
+
+moe_status launch_omni_out_scatter(const moe_omni_shape& s, const void* w_out,
+                                   const int32_t* offsets, const int32_t* p2a, const float* h,
+                                   float* y32, void* out, cudaStream_t st) {
+  const int N = s.n_rows * s.n_cols;
+  const long long n4 = (long long)s.T * s.d / 4;
+  moe_status r;
+  launch_begin(K_OMNI_OUT, st);
+  launch_kernel(omni_zero_f32_kernel, dim3((unsigned)grid_cap(n4, 256, 8)), dim3(256), 0, st, 1u,
+                (float4*)y32, n4);
+  if ((r = launch_end(K_OMNI_OUT, st)) != MOE_OK) return r;
+  const int grid = sm_count() * 8;
+  launch_begin(K_OMNI_OUT, st);
+  switch (s.d / 256) {
+#define OMNI_SCATTER_CASE(C)                                                                      \
+  case C:                                                                                         \
+    launch_kernel(omni_scatter_out_kernel<C>, dim3((unsigned)grid), dim3(256), 0, st, 1u,         \
+                  (const bf16*)w_out, offsets, p2a, h, y32, N, s.K, s.d, s.T * s.K,               \
+                  device_status_ptr());                                                           \
+    break;
+    OMNI_SCATTER_CASE(1)
+    OMNI_SCATTER_CASE(2)
+    OMNI_SCATTER_CASE(3)
+    OMNI_SCATTER_CASE(4)
+    OMNI_SCATTER_CASE(5)
+    OMNI_SCATTER_CASE(6)
+    OMNI_SCATTER_CASE(7)
+    OMNI_SCATTER_CASE(8)
+    default:
+      OMNI_SCATTER_CASE(16)
+#undef OMNI_SCATTER_CASE
+  }
+  if ((r = launch_end(K_OMNI_OUT, st)) != MOE_OK) return r;
+  launch_begin(K_OMNI_OUT, st);
+  launch_kernel(omni_to_bf16_kernel, dim3((unsigned)grid_cap(n4, 256, 8)), dim3(256), 0, st, 1u,
+                (const float4*)y32, (uint2*)out, n4);
+  return launch_end(K_OMNI_OUT, st);
+}
+
 }  // namespace moe
 
 // ------------------------------------------------------------------ C ABI
@@ -1499,6 +1637,8 @@ void omni_layout(const moe_omni_shape& s, moe_omni_layout* L) {
   o = al256(o + M * 4);
   L->scratch = o;
   o = al256(o + omni_schedule_scratch_bytes(s));
+  L->y32 = o;
+  o = al256(o + T * (size_t)s.d * 4);
   L->total = o;
 }
 
@@ -1611,7 +1751,19 @@ moe_status moe_omni_forward(const moe_omni_shape* s, const void* x, const void* 
   if ((r = launch_omni_schedule(*s, ids, counts, offsets, a2p, p2a, ws + L.scratch, true, false,
                                 st)) != MOE_OK)
     return r;
-  return moe_omni_experts(s, x, w_in, w_out, ids, w, offsets, p2a, h, out, stream);
+  if (g_omni_output_mode == 0)
+    return moe_omni_experts(s, x, w_in, w_out, ids, w, offsets, p2a, h, out, stream);
+  if (!al16(x) || !al16(w_in) || !al16(w_out) || !al16(out)) return MOE_ERR_INVALID_ARG;
+  if ((r = launch_omni_act(*s, x, w_in, offsets, p2a, w, h, st)) != MOE_OK) return r;
+  return launch_omni_out_scatter(*s, w_out, offsets, p2a, h, (float*)(ws + L.y32), out, st);
 }
+
+moe_status moe_omni_set_output_mode(int mode) {
+  if (mode < 0 || mode > 1) return MOE_ERR_INVALID_ARG;
+  g_omni_output_mode = mode;
+  return MOE_OK;
+}
+
+int moe_omni_get_output_mode(void) { return g_omni_output_mode; }
 
 }  // extern "C"
