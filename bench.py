@@ -52,6 +52,9 @@ def parse():
                     help="tokens in the CPU oracle sample (0: the workload's whole batch)")
     ap.add_argument("--ref-tokens", type=int, default=64,
                     help="tokens per step of the reference arm (the CPU oracle)")
+    ap.add_argument("--ffn-variant", type=int, default=0, choices=[0, 1, 2, 3],
+                    help="grouped-GEMM tile variant (moe_set_ffn_variant): 0 automatic, 1 "
+                         "single-CTA, 2 CTA pairs, 3 CTA pairs with the rows gathered first")
     ap.add_argument("--only", choices=["atomic_experts", "backward"], default=None,
                     help="run one secondary figure alone and print it (for profiling)")
     return ap.parse_args()
@@ -615,6 +618,7 @@ def atomic_experts_figure(tdr, world, peaks, n=10):
 def run_ours(args, rank, world, local):
     import token_dispatch_router_b200 as tdr
     tdr.load_library()  # fails loudly if the CUDA library is missing
+    tdr.set_ffn_variant(args.ffn_variant)
     if args.only == "atomic_experts":
         fig = atomic_experts_figure(tdr, world, load_peaks()[0], n=max(1, args.steps))
         if rank == 0:
@@ -758,6 +762,7 @@ def run_ours(args, rank, world, local):
     bw = backward_figure(tdr, cfg, s, x, w_r, wg, wu, wd, bias, world, peak_t)
     ae = atomic_experts_figure(tdr, world, peaks)
 
+    weights_gb = 3 * cfg.E * cfg.d * cfg.n * (2 if dt == torch.bfloat16 else 4) / 1e9
     # ---- per-kernel breakdown (ms per step) and the two secondary figures of the metric
     per_kernel = {k: round(ms / args.steps, 4) for k, (n, ms) in kern.items()}
     gemm = {"achieved_tflops": round(ach_gemm, 2), "frac": round(ach_gemm / peak_t, 4),
@@ -769,7 +774,9 @@ def run_ours(args, rank, world, local):
         if dt == torch.bfloat16 else "f32", "data": "synthetic",
         "config": {"workload": cfg.name, "T": cfg.T, "d": cfg.d, "E": cfg.E, "K": cfg.K,
                    "n": cfg.n, "global_batch": cfg.T * world, "parallelism": f"replicas{world}",
-                   "l2": "inputs larger than L2: the 2.82 GB of expert weights stream every step"},
+                   "ffn_variant": args.ffn_variant,
+                   "l2": f"inputs larger than L2: the {weights_gb:.2f} GB of expert weights "
+                         "stream every step"},
         "roofline": roofline, "gemm": gemm, "dispatch_combine": dc, "decode_dispatch": dd,
         "token_rounding": tr, "backward_act": bw, "atomic_experts": ae,
         "kernel_ms_per_step": per_kernel,
