@@ -315,7 +315,8 @@ moe_status moe_backward(const moe_shape* shape, const void* d_out, const float* 
  *   x [T, d], w_r [d, E] bf16; logits [T, E] fp32 (read only when renormalize == 0);
  *   topk_ids, topk_w [T, K] from the forward; d_w [T, K] from moe_backward;
  *   d_logits [T, E] fp32 out (also the intermediate); d_w_r [d, E] fp32 out;
- *   d_bias [E] fp32 out or NULL; d_x [T, d] bf16 in/out or NULL (16-byte aligned).
+ *   d_bias [E] fp32 out or NULL; d_x [T, d] bf16 in/out or NULL (16-byte aligned); with
+ *   E > 16, x 16-byte aligned too.
  * Sums over tokens run in a fixed order (deterministic). bf16 only.
  */
 moe_status moe_backward_router(const moe_shape* shape, const void* x, const void* w_r,

@@ -600,9 +600,10 @@ def test_backward_act_full_size_sampled_slots(cuda_lib):
 
 
 @pytest.mark.parametrize("renorm", [True, False])
-def test_backward_router_matches_oracle(cuda_lib, renorm):
+@pytest.mark.parametrize("E,K", [(16, 3), (40, 4), (128, 8)])  # > 16: the tiled kernels
+def test_backward_router_matches_oracle(cuda_lib, renorm, E, K):
     tdr = cuda_lib
-    T, d, n, E, K = 700, 256, 128, 16, 3
+    T, d, n = 700, 256, 128
     cfg = mi.MoEConfig("rbwd", T=T, d=d, E=E, K=K, n=n, dtype="bf16", seed=77)
     inp = mi.make_inputs(cfg)
     bias = mi.zipf_bias(E, 1.2, 1.75)

@@ -503,6 +503,7 @@ moe_status moe_backward_router(const moe_shape* s, const void* x, const void* w_
   if (!x || !w_r || !topk_ids || !topk_w || !d_w || !d_logits || !d_w_r) return MOE_ERR_INVALID_ARG;
   if (!s->renormalize && logits == nullptr) return MOE_ERR_INVALID_ARG;  // the plain softmax
   if (d_x != nullptr && !aligned16(d_x)) return MOE_ERR_INVALID_ARG;
+  if (s->E > 16 && !aligned16(x)) return MOE_ERR_INVALID_ARG;  // 16-byte row loads of x
   return launch_router_backward(*s, x, w_r, logits, topk_ids, topk_w, d_w, d_logits, d_w_r,
                                 d_bias, d_x, (cudaStream_t)stream);
 }

@@ -15,7 +15,8 @@
 // CTAs that own 32 columns of W_r and EC experts and sum over all tokens in a fixed order
 // (sixteen token groups, then the groups in order: deterministic); the input-gradient term
 // by CTAs that own 64 columns of d with that slice of W_r in shared memory, 8 threads per
-// token row slice, fp32 sums added to the bf16 d_x.
+// token row slice, fp32 sums added to the bf16 d_x. Routers with more than 16 experts use
+// register-tiled forms of the last two (below), whose work per token grows with E.
 #include <math.h>
 
 #include "common.cuh"
@@ -194,6 +195,201 @@ __global__ void __launch_bounds__(256) router_dx_kernel(const bf16* __restrict__
   }
 }
 
+// ---- wide routers (E > 16): register-tiled CUDA-core GEMMs, fp32 throughout.
+// d_W_r = x^T dl: a 64 (columns of x) x 64 (experts) tile per cluster of 4 CTAs; each CTA
+// sums a quarter of the tokens (chunks of 32 staged in shared memory, a 4 x 4 register tile
+// per thread), then CTA rank 0 adds the four partial tiles in rank order through
+// distributed shared memory (deterministic, no global scratch). d_bias comes from the
+// column-tile-0 clusters the same way.
+constexpr int kWt = 64, kWk = 32, kWsplit = 4;
+
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+  return (uint32_t)__cvta_generic_to_shared(p);
+}
+__device__ __forceinline__ uint32_t cta_rank_in_cluster() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+__device__ __forceinline__ void cluster_barrier() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::
+                   : "memory");
+}
+__device__ __forceinline__ float ld_peer_f32(const float* local, uint32_t rank) {
+  uint32_t remote;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(remote) : "r"(smem_u32(local)), "r"(rank));
+  float v;
+  asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(remote) : "memory");
+  return v;
+}
+
+__global__ void __launch_bounds__(256) router_dwr_tiled_kernel(const bf16* __restrict__ x,
+                                                               const float* __restrict__ dl,
+                                                               int T, int d, int E,
+                                                               float* __restrict__ d_w_r,
+                                                               float* __restrict__ d_bias) {
+  __shared__ __align__(16) float xs[kWk][kWt];  // [token][column]
+  __shared__ __align__(16) float ds[kWk][kWt];  // [token][expert]
+  __shared__ __align__(16) float part[kWt][kWt + 1];
+  __shared__ float partb[kWt];
+  pdl_wait();  // the previous kernel in the stream has completed
+  pdl_trigger();
+  const uint32_t rank = cta_rank_in_cluster();
+  const int tile = blockIdx.x / kWsplit;
+  const int e_tiles = (E + kWt - 1) / kWt;
+  const int jt = tile / e_tiles, et = tile % e_tiles;
+  const int j0 = jt * kWt, e0 = et * kWt;
+  const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;  // 16 x 16 threads, 4 x 4 each
+  const bool bias = d_bias != nullptr && jt == 0;
+  const int per = (T + kWsplit - 1) / kWsplit;
+  const int t_begin = (int)rank * per, t_end = min(T, t_begin + per);
+  float acc[4][4], accb[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    accb[i] = 0.f;
+#pragma unroll
+    for (int q = 0; q < 4; ++q) acc[i][q] = 0.f;
+  }
+  // loaders: x chunk 32 x 64 bf16 = one 8-element vector per thread; dl chunk 32 x 64 fp32 =
+  // eight values per thread; the next chunk's loads are issued before this chunk's sums
+  const int lr = threadIdx.x >> 3, lc = (threadIdx.x & 7) * 8;
+  uint4 xr = make_uint4(0, 0, 0, 0);
+  float dr[8];
+  auto load = [&](int t0) {
+    const int t = t0 + lr;
+    xr = t < t_end ? *reinterpret_cast<const uint4*>(x + (size_t)t * d + j0 + lc)
+                   : make_uint4(0, 0, 0, 0);
+#pragma unroll
+    for (int c = 0; c < 8; ++c) {
+      const int e = e0 + lc + c;
+      dr[c] = (t < t_end && e < E) ? dl[(size_t)t * E + e] : 0.f;
+    }
+  };
+  if (t_begin < t_end) load(t_begin);
+  for (int t0 = t_begin; t0 < t_end; t0 += kWk) {
+    {
+      float f[8];
+      unpack16(xr, f, bf16());
+#pragma unroll
+      for (int c = 0; c < 8; ++c) {
+        xs[lr][lc + c] = f[c];
+        ds[lr][lc + c] = dr[c];
+      }
+    }
+    __syncthreads();
+    if (t0 + kWk < t_end) load(t0 + kWk);
+#pragma unroll 8
+    for (int kk = 0; kk < kWk; ++kk) {
+      const float4 a = *reinterpret_cast<const float4*>(&xs[kk][ty * 4]);
+      const float4 b = *reinterpret_cast<const float4*>(&ds[kk][tx * 4]);
+      const float av[4] = {a.x, a.y, a.z, a.w}, bv[4] = {b.x, b.y, b.z, b.w};
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int q = 0; q < 4; ++q) acc[i][q] = fmaf(av[i], bv[q], acc[i][q]);
+      if (bias && ty == 0)
+#pragma unroll
+        for (int q = 0; q < 4; ++q) accb[q] += bv[q];
+    }
+    __syncthreads();
+  }
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+#pragma unroll
+    for (int q = 0; q < 4; ++q) part[ty * 4 + i][tx * 4 + q] = acc[i][q];
+  if (bias && ty == 0)
+#pragma unroll
+    for (int q = 0; q < 4; ++q) partb[tx * 4 + q] = accb[q];
+  cluster_barrier();  // every rank's partial tile is in its shared memory
+  if (rank == 0) {
+    for (int i = threadIdx.x; i < kWt * kWt; i += 256) {
+      const int r = i / kWt, c = i % kWt;
+      float v = part[r][c];
+      for (uint32_t q = 1; q < kWsplit; ++q) v += ld_peer_f32(&part[r][c], q);  // rank order
+      const int j = j0 + r, e = e0 + c;
+      if (j < d && e < E) d_w_r[(size_t)j * E + e] = v;
+    }
+    if (bias && threadIdx.x < kWt) {
+      float v = partb[threadIdx.x];
+      for (uint32_t q = 1; q < kWsplit; ++q) v += ld_peer_f32(&partb[threadIdx.x], q);
+      const int e = e0 + (int)threadIdx.x;
+      if (e < E) d_bias[e] = v;
+    }
+  }
+  cluster_barrier();  // the peers' tiles have been read; they may exit
+}
+
+// d_x[t, j] += sum_e dl[t, e] W_r[j, e]: a CTA owns 64 tokens and kDxCols columns. Its
+// tokens' dl rows are staged once in shared memory (expert-major), then each 64-column tile
+// sums over the experts in chunks of 32 (the W_r chunk staged expert-major, the next
+// chunk's loads issued before this chunk's sums), a 4 x 4 register tile per thread; fp32
+// sums added to the bf16 d_x.
+constexpr int kDxCols = 512;
+
+__global__ void __launch_bounds__(256) router_dx_tiled_kernel(const bf16* __restrict__ w_r,
+                                                              const float* __restrict__ dl,
+                                                              int T, int d, int E, int Ep,
+                                                              bf16* __restrict__ d_x) {
+  extern __shared__ __align__(16) float dsm[];
+  float* ls = dsm;               // [Ep][64]: expert-major dl of the CTA's tokens
+  float* ws = dsm + Ep * kWt;    // [32][64]: expert-major W_r chunk
+  pdl_wait();  // the previous kernel in the stream has completed
+  pdl_trigger();
+  const int t0 = blockIdx.x * kWt;
+  const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;
+  for (int i = threadIdx.x; i < kWt * Ep; i += 256) {
+    const int r = i / Ep, e = i % Ep;  // consecutive threads: consecutive experts of a token
+    ls[e * kWt + r] = (t0 + r < T && e < E) ? dl[(size_t)(t0 + r) * E + e] : 0.f;
+  }
+  const int lr = threadIdx.x >> 2, lc = (threadIdx.x & 3) * 8;
+  float wv[8];
+  for (int j0 = blockIdx.y * kDxCols; j0 < min(d, (int)(blockIdx.y + 1) * kDxCols); j0 += kWt) {
+    auto load = [&](int k0) {
+      const int j = j0 + lr;
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const int e = k0 + lc + u;
+        wv[u] = (j < d && e < E) ? __bfloat162float(w_r[(size_t)j * E + e]) : 0.f;
+      }
+    };
+    float acc[4][4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+      for (int q = 0; q < 4; ++q) acc[i][q] = 0.f;
+    load(0);
+    for (int k0 = 0; k0 < E; k0 += kWk) {
+      __syncthreads();  // the previous chunk's sums are done with ws (and ls is complete)
+#pragma unroll
+      for (int u = 0; u < 8; ++u) ws[(lc + u) * kWt + lr] = wv[u];
+      __syncthreads();
+      if (k0 + kWk < E) load(k0 + kWk);
+#pragma unroll 8
+      for (int kk = 0; kk < kWk; ++kk) {
+        const float4 a = *reinterpret_cast<const float4*>(&ls[(k0 + kk) * kWt + ty * 4]);
+        const float4 b = *reinterpret_cast<const float4*>(&ws[kk * kWt + tx * 4]);
+        const float av[4] = {a.x, a.y, a.z, a.w}, bv[4] = {b.x, b.y, b.z, b.w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+#pragma unroll
+          for (int q = 0; q < 4; ++q) acc[i][q] = fmaf(av[i], bv[q], acc[i][q]);
+      }
+    }
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const int t = t0 + ty * 4 + i, j = j0 + tx * 4;
+      if (t >= T || j >= d) continue;
+      uint2* px = reinterpret_cast<uint2*>(d_x + (size_t)t * d + j);
+      const uint2 old = *px;
+      const float c0 = __uint_as_float(old.x << 16) + acc[i][0];
+      const float c1 = __uint_as_float(old.x & 0xffff0000u) + acc[i][1];
+      const float c2 = __uint_as_float(old.y << 16) + acc[i][2];
+      const float c3 = __uint_as_float(old.y & 0xffff0000u) + acc[i][3];
+      *px = make_uint2(pack_bf16x2(c0, c1), pack_bf16x2(c2, c3));
+    }
+  }
+}
+
 }  // namespace
 
 moe_status launch_router_backward(const moe_shape& s, const void* x, const void* w_r,
@@ -210,7 +406,14 @@ moe_status launch_router_backward(const moe_shape& s, const void* x, const void*
                   d_w, logits, T, E, K, s.renormalize, d_logits);
     if ((r = launch_end(K_ROUTER_DLOGITS, st)) != MOE_OK) return r;
   }
-  {
+  if (E > 16) {
+    const int tiles = ((d + kWt - 1) / kWt) * ((E + kWt - 1) / kWt);
+    launch_begin(K_ROUTER_DWR, st);
+    launch_kernel(router_dwr_tiled_kernel, dim3((unsigned)(tiles * kWsplit)), dim3(256), 0, st,
+                  (unsigned)kWsplit, (const bf16*)x, (const float*)d_logits, T, d, E, d_w_r,
+                  d_bias);
+    if ((r = launch_end(K_ROUTER_DWR, st)) != MOE_OK) return r;
+  } else {
     const int EC = E <= 8 ? 8 : 16;
     const dim3 grid((unsigned)((d + 31) / 32), (unsigned)((E + EC - 1) / EC));
     const dim3 block(kDwrWarps * 32);
@@ -223,7 +426,19 @@ moe_status launch_router_backward(const moe_shape& s, const void* x, const void*
                     (const float*)d_logits, T, d, E, d_w_r, d_bias);
     if ((r = launch_end(K_ROUTER_DWR, st)) != MOE_OK) return r;
   }
-  if (d_x != nullptr) {
+  if (d_x != nullptr && E > 16) {
+    const int Ep = (E + kWk - 1) / kWk * kWk;  // experts padded to whole chunks
+    const int smem = (Ep + kWk) * kWt * (int)sizeof(float);
+    if (cudaFuncSetAttribute(router_dx_tiled_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             smem) != cudaSuccess)
+      return MOE_ERR_CUDA;
+    launch_begin(K_ROUTER_DX, st);
+    launch_kernel(router_dx_tiled_kernel,
+                  dim3((unsigned)((T + kWt - 1) / kWt), (unsigned)((d + kDxCols - 1) / kDxCols)),
+                  dim3(256), (size_t)smem, st, 1, (const bf16*)w_r, (const float*)d_logits, T, d,
+                  E, Ep, (bf16*)d_x);
+    if ((r = launch_end(K_ROUTER_DX, st)) != MOE_OK) return r;
+  } else if (d_x != nullptr) {
     const int smem = 64 * E * (int)sizeof(float);
     if (cudaFuncSetAttribute(router_dx_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              smem) != cudaSuccess)
