@@ -281,6 +281,38 @@ def test_dispatch_matches_oracle_and_the_two_calls(cuda_lib, T, E, K, cf, renorm
     assert_status_ok(tdr)
 
 
+@pytest.mark.parametrize("T,E,K,cf,mat", [
+    (100, 8, 2, 0.0, False), (1000, 8, 2, 0.0, True), (4096, 8, 2, 0.0, True),
+    (4097, 8, 2, 0.9, True), (3000, 64, 6, 0.0, False), (2000, 256, 8, 1.1, True),
+    (8192, 16, 4, 0.0, False), (40000, 8, 2, 0.0, False)])
+def test_dispatch_from_x_matches_oracle(cuda_lib, T, E, K, cf, mat):
+    """moe_dispatch from x and W_r (tensor-core router, then the permutation): equal to the
+    oracle on the router's own logits, with and without capacity drops, with the rows
+    gathered exactly."""
+    tdr = cuda_lib
+    d = 256
+    cfg = mi.MoEConfig("dispatch_x", T=T, d=d, E=E, K=K, n=0, dtype="bf16", seed=T + E)
+    inp = mi.make_inputs(cfg, with_experts=False)
+    s = tdr.make_shape(T, d, E, K, 0, cf, True, torch.bfloat16)
+    x = inp.x.cuda()
+    out = tdr.dispatch(s, x=x, w_r=inp.w_r.cuda(), logits_out=torch.empty(T, E, device="cuda"),
+                       materialize=mat)
+    torch.cuda.synchronize()
+    assert_status_ok(tdr)
+    lg = out["logits_out"].cpu().numpy() if "logits_out" in out else None
+    assert lg is not None
+    ids_ref, w_ref = orc.route(lg, K, True)
+    np.testing.assert_array_equal(out["topk_ids"].cpu().numpy(), ids_ref)
+    assert np.abs(out["topk_w"].cpu().numpy() - w_ref).max() <= W_ABS
+    C = orc.capacity(cf, T, K, E)
+    _, offsets, _, p2a = check_permutation(out, ids_ref, E, C)
+    if mat:
+        nk = int(offsets[-1])
+        xp = out["x_perm"][:nk].cpu()
+        np.testing.assert_array_equal(xp.view(torch.int16).numpy(),
+                                      inp.x[torch.from_numpy(p2a[:nk] // K)].view(torch.int16).numpy())
+
+
 def test_dispatch_materialised_gather_is_exact(cuda_lib):
     tdr = cuda_lib
     rng = np.random.default_rng(17)
