@@ -232,6 +232,75 @@ def cpu_oracle_tokens_per_s(inp, n_tokens: int, start: int = 0, wide=None):
     return n_tokens / dt, dt, wide
 
 
+def cpu_oracle_figures(inp, wide, R: int = 128, n_tok: int = 256, n_omni: int = 16) -> dict:
+    """The oracle, as it stands, on bounded samples of each secondary figure's work (timed on
+    the host beside the GPU figures): the token-rounded layer and the layer's backward on an
+    n_tok-token batch of the bench workload, the dispatch/combine-only pipeline at its decode
+    sizes, and n_omni tokens of the atomic-expert layer. Expert weights are the fp64 copies
+    the CPU baseline made (untimed)."""
+    from oracle import moe_oracle as orc
+    from oracle import omni_oracle as oo
+    cfg = inp.cfg
+    res = {}
+    E = cfg.E
+    class _Experts:  # the per-expert fp64 matrices, indexable like the stacked tensor
+        def __init__(self, mats):
+            self.mats = mats
+            self.shape = (len(mats),) + tuple(mats[0].shape)
+
+        def __getitem__(self, e):
+            return self.mats[e]
+
+    wg = _Experts([wide[e][0] if e in wide else orc.as_f64(inp.w_gate[e]) for e in range(E)])
+    wu = _Experts([wide[e][1] if e in wide else orc.as_f64(inp.w_up[e]) for e in range(E)])
+    wd = _Experts([wide[e][2] if e in wide else orc.as_f64(inp.w_down[e]) for e in range(E)])
+    x = orc.as_f64(inp.x[:n_tok])
+    bias = None if inp.bias is None else inp.bias.numpy()
+    if cfg.capacity_factor <= 0:
+        t0 = time.perf_counter()
+        orc.forward(x, inp.w_r, wg, wu, wd, cfg.K, bias=bias, tile_round=R)
+        dt = time.perf_counter() - t0
+        res["token_rounding"] = {"tokens_per_s": n_tok / dt, "sample": f"{n_tok} tokens, R={R}"}
+    # backward: forward pieces untimed, then the oracle's backward of the expert half + router
+    f = orc.forward(x, inp.w_r, wg, wu, wd, cfg.K, capacity_factor=cfg.capacity_factor, bias=bias)
+    g, u = orc.gate_up_preact(x, f["perm_to_assign"], f["offsets"], cfg.K, wg, wu)
+    d_out = np.random.default_rng(0).standard_normal((n_tok, cfg.d))
+    t0 = time.perf_counter()
+    dG, dU, d_w = orc.backward_act(d_out, f["topk_w"], f["assign_to_perm"], f["perm_to_assign"],
+                                   f["offsets"], cfg.K, wd, g, u)
+    orc.backward_dx(dG, dU, f["assign_to_perm"], f["perm_to_assign"], f["offsets"], cfg.K, n_tok,
+                    wg, wu)
+    orc.backward_router(d_w, f["topk_ids"], f["logits"], x, inp.w_r)
+    dt = time.perf_counter() - t0
+    res["backward_act"] = {"tokens_per_s": n_tok / dt, "sample": f"{n_tok} tokens"}
+    # dispatch / combine only (given logits, identity experts), the decode sizes
+    dcfg = mi.DISPATCH_COMBINE
+    dd = {}
+    for T in (64, 1024):
+        di = mi.make_inputs(dcfg.with_T(T))
+        lg = di.logits.numpy()
+        xd = orc.as_f64(di.x)
+        t0 = time.perf_counter()
+        ids, w = orc.route(lg, dcfg.K)
+        _, offs, a2p, p2a = orc.permute(ids, dcfg.E)
+        xp = orc.gather_rows(xd, p2a, offs, dcfg.K)
+        orc.combine(xp, a2p, w, T, dcfg.K)
+        dd[f"T={T}"] = round((time.perf_counter() - t0) * 1e6, 1)
+    res["decode_dispatch"] = {"us": dd, "sample": "route + permute + gather + combine"}
+    # atomic experts: routing over the whole grid and the outputs of n_omni tokens
+    oc = mi.OMNI_102K
+    oi = mi.make_omni_inputs(oc)
+    toks = np.arange(n_omni)
+    t0 = time.perf_counter()
+    lg = oo.cartesian_logits(oi.x[:n_omni], oi.w_row, oi.w_col)
+    ids, w = oo.cartesian_route(lg, oc.n_rows, oc.K)
+    oo.token_outputs(oi.x[:n_omni], oi.w_in, oi.w_out, ids, w)
+    dt = time.perf_counter() - t0
+    res["atomic_experts"] = {"tokens_per_s": n_omni / dt, "sample": f"{n_omni} tokens of omni_102k"}
+    res["cores"] = cpu_cores()
+    return res
+
+
 def cpu_cores() -> int:
     try:
         return len(os.sched_getaffinity(0))
@@ -787,11 +856,13 @@ def run_ours(args, rank, world, local):
     # ---- CPU oracle baseline (rank 0, N = 1 only)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         ntok = args.cpu_tokens if args.cpu_tokens > 0 else cfg.T
-        v_cpu, dt_cpu, _ = cpu_oracle_tokens_per_s(inp, ntok)
+        v_cpu, dt_cpu, wide = cpu_oracle_tokens_per_s(inp, ntok)
         result["cpu_baseline"] = {
             "value": v_cpu, "unit": "tokens/s", "cores": cpu_cores(), "kind": "oracle",
             "sample": f"{ntok} tokens through the whole layer (oracle numpy fp64, "
                       f"{dt_cpu:.1f} s; expert weights widened to fp64 outside the timing)"}
+        if cfg.dtype == "bf16":
+            result["cpu_oracle_figures"] = cpu_oracle_figures(inp, wide)
     if rank == 0:
         print(json.dumps(result), flush=True)
 
