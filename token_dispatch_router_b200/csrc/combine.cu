@@ -10,7 +10,8 @@
 // the token's K slots and weights are loaded once per lane (same addresses across the warp),
 // then for each pair of slots every lane issues eight independent 128-bit loads (4 vectors
 // x 2 rows; every warp-wide load covers 512 contiguous bytes), accumulates in fp32 in slot
-// order, and writes its four vectors.
+// order, and writes its four vectors. The rows are read with an L2 evict-first policy: each
+// is read exactly once.
 #include "common.cuh"
 
 namespace moe {
@@ -30,6 +31,7 @@ __global__ void __launch_bounds__(256) combine_kernel(const uint4* __restrict__ 
   const long long units = (long long)T * segs;
   const int lane = threadIdx.x & 31;
   const long long warps = (long long)gridDim.x * (blockDim.x >> 5);
+  const uint64_t once = l2_policy_evict_first();  // each row is read exactly once
   for (long long u = (long long)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); u < units;
        u += warps) {
     const long long t = u / segs;
@@ -60,7 +62,8 @@ __global__ void __launch_bounds__(256) combine_kernel(const uint4* __restrict__ 
       for (int h = 0; h < 2; ++h)
 #pragma unroll
         for (int j = 0; j < 4; ++j)
-          if (p[h] >= 0 && v0 + 32 * j < vec_per_row) r[h][j] = y_perm[p[h] * vec_per_row + v0 + 32 * j];
+          if (p[h] >= 0 && v0 + 32 * j < vec_per_row)
+            r[h][j] = ld_global_hint(y_perm + p[h] * vec_per_row + v0 + 32 * j, once);
 #pragma unroll
       for (int h = 0; h < 2; ++h) {
         if (p[h] < 0) continue;

@@ -722,7 +722,9 @@ __global__ void __launch_bounds__(WARPS * 32) route_permute_kernel(
 
 // x_perm[p] = x[perm_to_assign[p] / K] for p < offsets[E]; 16-byte vectors. One warp moves
 // a 2 KB segment (128 vectors) of one row: the row's source token is loaded once per lane
-// and each lane keeps four independent 16-byte loads in flight.
+// and each lane keeps four independent 16-byte loads in flight. The rows are stored with an
+// L2 evict-last policy: the kernel after this one reads them back (67 MB at the Mixtral
+// shape fits in L2).
 __global__ void __launch_bounds__(256) gather_rows_kernel(const uint4* __restrict__ x,
                                                           const int32_t* __restrict__ p2a,
                                                           const int32_t* __restrict__ n_kept_ptr,
@@ -735,6 +737,7 @@ __global__ void __launch_bounds__(256) gather_rows_kernel(const uint4* __restric
   const int segs = (vec_per_row + 127) / 128;
   const long long units = n_kept * segs;
   const int lane = threadIdx.x & 31;
+  const uint64_t keep = l2_policy_evict_last();  // the next kernel reads the rows back
   const long long warps = (long long)gridDim.x * (blockDim.x >> 5);
   for (long long u = (long long)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); u < units;
        u += warps) {
@@ -754,7 +757,7 @@ __global__ void __launch_bounds__(256) gather_rows_kernel(const uint4* __restric
       if (v0 + 32 * j < vec_per_row) r[j] = src[v0 + 32 * j];
 #pragma unroll
     for (int j = 0; j < 4; ++j)
-      if (v0 + 32 * j < vec_per_row) dst[v0 + 32 * j] = r[j];
+      if (v0 + 32 * j < vec_per_row) st_global_hint(dst + v0 + 32 * j, r[j], keep);
   }
 }
 
