@@ -20,6 +20,7 @@
 #include <math.h>
 
 #include "common.cuh"
+#include "tc_ptx.cuh"
 
 namespace moe {
 
@@ -203,26 +204,6 @@ __global__ void __launch_bounds__(256) router_dx_kernel(const bf16* __restrict__
 // column-tile-0 clusters the same way.
 constexpr int kWt = 64, kWk = 32, kWsplit = 4;
 
-__device__ __forceinline__ uint32_t smem_u32(const void* p) {
-  return (uint32_t)__cvta_generic_to_shared(p);
-}
-__device__ __forceinline__ uint32_t cta_rank_in_cluster() {
-  uint32_t r;
-  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
-  return r;
-}
-__device__ __forceinline__ void cluster_barrier() {
-  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::
-                   : "memory");
-}
-__device__ __forceinline__ float ld_peer_f32(const float* local, uint32_t rank) {
-  uint32_t remote;
-  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(remote) : "r"(smem_u32(local)), "r"(rank));
-  float v;
-  asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(remote) : "memory");
-  return v;
-}
-
 __global__ void __launch_bounds__(256) router_dwr_tiled_kernel(const bf16* __restrict__ x,
                                                                const float* __restrict__ dl,
                                                                int T, int d, int E,
@@ -234,7 +215,7 @@ __global__ void __launch_bounds__(256) router_dwr_tiled_kernel(const bf16* __res
   __shared__ float partb[kWt];
   pdl_wait();  // the previous kernel in the stream has completed
   pdl_trigger();
-  const uint32_t rank = cta_rank_in_cluster();
+  const uint32_t rank = ptx::cluster_rank();
   const int tile = blockIdx.x / kWsplit;
   const int e_tiles = (E + kWt - 1) / kWt;
   const int jt = tile / e_tiles, et = tile % e_tiles;
@@ -300,23 +281,25 @@ __global__ void __launch_bounds__(256) router_dwr_tiled_kernel(const bf16* __res
   if (bias && ty == 0)
 #pragma unroll
     for (int q = 0; q < 4; ++q) partb[tx * 4 + q] = accb[q];
-  cluster_barrier();  // every rank's partial tile is in its shared memory
+  ptx::cluster_sync();  // every rank's partial tile is in its shared memory
   if (rank == 0) {
     for (int i = threadIdx.x; i < kWt * kWt; i += 256) {
       const int r = i / kWt, c = i % kWt;
       float v = part[r][c];
-      for (uint32_t q = 1; q < kWsplit; ++q) v += ld_peer_f32(&part[r][c], q);  // rank order
+      for (uint32_t q = 1; q < kWsplit; ++q)  // rank order
+        v += ptx::ld_dsmem_f32(ptx::map_rank(ptx::saddr(&part[r][c]), q));
       const int j = j0 + r, e = e0 + c;
       if (j < d && e < E) d_w_r[(size_t)j * E + e] = v;
     }
     if (bias && threadIdx.x < kWt) {
       float v = partb[threadIdx.x];
-      for (uint32_t q = 1; q < kWsplit; ++q) v += ld_peer_f32(&partb[threadIdx.x], q);
+      for (uint32_t q = 1; q < kWsplit; ++q)
+        v += ptx::ld_dsmem_f32(ptx::map_rank(ptx::saddr(&partb[threadIdx.x]), q));
       const int e = e0 + (int)threadIdx.x;
       if (e < E) d_bias[e] = v;
     }
   }
-  cluster_barrier();  // the peers' tiles have been read; they may exit
+  ptx::cluster_sync();  // the peers' tiles have been read; they may exit
 }
 
 // d_x[t, j] += sum_e dl[t, e] W_r[j, e]: a CTA owns 64 tokens and kDxCols columns. Its

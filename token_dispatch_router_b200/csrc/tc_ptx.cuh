@@ -247,7 +247,12 @@ __device__ __forceinline__ uint32_t map_rank(uint32_t local_addr, uint32_t rank)
   asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(remote) : "r"(local_addr), "r"(rank));
   return remote;
 }
-// 32-bit load from the shared memory of another CTA of the cluster (address from map_rank).
+// 32-bit loads from the shared memory of another CTA of the cluster (address from map_rank).
+__device__ __forceinline__ float ld_dsmem_f32(uint32_t cluster_addr) {
+  float v;
+  asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(cluster_addr) : "memory");
+  return v;
+}
 __device__ __forceinline__ int ld_dsmem_s32(uint32_t cluster_addr) {
   int v;
   asm volatile("ld.shared::cluster.s32 %0, [%1];" : "=r"(v) : "r"(cluster_addr) : "memory");
