@@ -45,7 +45,11 @@ constexpr int GATHER_THREADS = 128;
 constexpr uint32_t TMEM_COLS = 512;
 constexpr int MAXE = 256;
 constexpr int SMEM_TAIL = 4096;
-constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 + SMEM_TAIL;
+// dA' epilogue: per epilogue warp, one 32-row x 32-column chunk of g and of u (then of dG
+// and dU), rows padded to 80 bytes so that a thread reading its own row hits distinct banks
+constexpr int EPI_ROW = 80;
+constexpr int EPI_WARP_BYTES = 2 * 32 * EPI_ROW;
+constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 + SMEM_TAIL + 4 * EPI_WARP_BYTES;
 // kind::f16: D fp32 (bit 4), A and B bf16 (bits 7-9, 10-12), both K-major (bits 15, 16 = 0),
 // N >> 3 at bits 17-22, M >> 4 at bits 24-28
 constexpr uint32_t IDESC =
@@ -112,6 +116,7 @@ __global__ void __launch_bounds__(MODE == 0 ? THREADS_DACT : THREADS_DX, 1)
   int* s_off = (int*)(tmem_slot + 2);
   int* s_cum = s_off + MAXE + 1;
   int* s_mt = s_cum + MAXE + 1;
+  uint8_t* epi = base + STAGES * STAGE_BYTES + SMEM_TAIL;  // dA' epilogue buffers (16-byte aligned)
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int E = g.E;
@@ -367,69 +372,97 @@ __global__ void __launch_bounds__(MODE == 0 ? THREADS_DACT : THREADS_DX, 1)
         continue;
       }
       const float wt = row_ok ? g.topk_w[g.p2a[p]] : 0.f;
-      const bf16* hrow = g.h + (size_t)p * ld;
-      bf16* drow = g.d_h + (size_t)p * ld;
       float ds = 0.f;
-      // g and u of the chunk are loaded one chunk ahead of their use
-      uint4 gq[4], uq[4], gn[4], un[4];
-      auto load_h = [&](int c, uint4 (&gd)[4], uint4 (&ud)[4]) {
-        const int col = t.n0 + c * 32;
-        if (row_ok && col < g.n) {
-          const uint4* gs = reinterpret_cast<const uint4*>(hrow + col);
-          const uint4* us = reinterpret_cast<const uint4*>(hrow + g.n + col);
+      // The warp's 32 rows of a 32-column chunk of g and u are loaded cooperatively (a lane
+      // moves 16 of a row's 64 bytes; one instruction covers 8 whole row segments), put
+      // through the warp's padded buffer so that each thread reads its own row, and dG / dU
+      // go back out the same way. The next chunk's loads are issued before this chunk's math.
+      uint8_t* gbuf = epi + q * EPI_WARP_BYTES;
+      uint8_t* ubuf = gbuf + 32 * EPI_ROW;
+      const int lr = lane >> 2, lc = lane & 3;  // this lane's row (of 8) and 16-byte column
+      uint4 gn[4], un[4];
+      auto load_chunk = [&](int c) {
+        const int col = t.n0 + c * 32 + lc * 8;
 #pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            gd[j] = gs[j];
-            ud[j] = us[j];
+        for (int i = 0; i < 4; ++i) {
+          const int rr = q * 32 + lr + 8 * i;  // row inside the tile
+          if (rr < t.rows && col < g.n) {
+            const bf16* src = g.h + (size_t)(t.m0 + rr) * ld + col;
+            gn[i] = *reinterpret_cast<const uint4*>(src);
+            un[i] = *reinterpret_cast<const uint4*>(src + g.n);
+          } else {
+            gn[i] = make_uint4(0, 0, 0, 0);
+            un[i] = gn[i];
           }
         }
       };
-      load_h(0, gq, uq);
+      load_chunk(0);
 #pragma unroll 1
       for (int c = 0; c < BN / 32; ++c) {
-        uint32_t v[32];
-        tmem_ld32(tb + c * 32, v);
-        if (c + 1 < BN / 32) load_h(c + 1, gn, un);
-        tmem_ld_wait();
-        const int col = t.n0 + c * 32;
-        if (row_ok && col < g.n) {
-          uint32_t pg[16], pu[16];
 #pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            float gf[8], uf[8];
-            unpack16(gq[j], gf, bf16());
-            unpack16(uq[j], uf, bf16());
-#pragma unroll
-            for (int i = 0; i < 8; i += 2) {
-              float dg[2], du[2];
-#pragma unroll
-              for (int h2 = 0; h2 < 2; ++h2) {
-                const float gg = gf[i + h2], uu = uf[i + h2];
-                const float da1 = __uint_as_float(v[8 * j + i + h2]);
-                const float s = __fdividef(1.f, 1.f + __expf(-gg));
-                const float silu = gg * s;
-                ds = fmaf(da1, silu * uu, ds);
-                const float da = wt * da1;
-                dg[h2] = da * uu * s * (1.f + gg * (1.f - s));
-                du[h2] = da * silu;
-              }
-              pg[4 * j + i / 2] = pack_bf16x2(dg[0], dg[1]);
-              pu[4 * j + i / 2] = pack_bf16x2(du[0], du[1]);
-            }
-          }
-          uint4* gd = reinterpret_cast<uint4*>(drow + col);
-          uint4* ud = reinterpret_cast<uint4*>(drow + g.n + col);
-#pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            gd[j] = make_uint4(pg[4 * j], pg[4 * j + 1], pg[4 * j + 2], pg[4 * j + 3]);
-            ud[j] = make_uint4(pu[4 * j], pu[4 * j + 1], pu[4 * j + 2], pu[4 * j + 3]);
-          }
+        for (int i = 0; i < 4; ++i) {
+          *reinterpret_cast<uint4*>(gbuf + (lr + 8 * i) * EPI_ROW + lc * 16) = gn[i];
+          *reinterpret_cast<uint4*>(ubuf + (lr + 8 * i) * EPI_ROW + lc * 16) = un[i];
         }
+        __syncwarp();
+        uint4 gq[4], uq[4];
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
-          gq[j] = gn[j];
-          uq[j] = un[j];
+          gq[j] = *reinterpret_cast<const uint4*>(gbuf + lane * EPI_ROW + j * 16);
+          uq[j] = *reinterpret_cast<const uint4*>(ubuf + lane * EPI_ROW + j * 16);
         }
+        uint32_t v[32];
+        tmem_ld32(tb + c * 32, v);
+        if (c + 1 < BN / 32) load_chunk(c + 1);
+        tmem_ld_wait();
+        const int col = t.n0 + c * 32;
+        uint32_t pg[16], pu[16];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          float gf[8], uf[8];
+          unpack16(gq[j], gf, bf16());
+          unpack16(uq[j], uf, bf16());
+#pragma unroll
+          for (int i = 0; i < 8; i += 2) {
+            float dg[2], du[2];
+#pragma unroll
+            for (int h2 = 0; h2 < 2; ++h2) {
+              const float gg = gf[i + h2], uu = uf[i + h2];
+              const float da1 = __uint_as_float(v[8 * j + i + h2]);
+              const float s = __fdividef(1.f, 1.f + __expf(-gg));
+              const float silu = gg * s;
+              if (row_ok) ds = fmaf(da1, silu * uu, ds);
+              const float da = wt * da1;
+              dg[h2] = da * uu * s * (1.f + gg * (1.f - s));
+              du[h2] = da * silu;
+            }
+            pg[4 * j + i / 2] = pack_bf16x2(dg[0], dg[1]);
+            pu[4 * j + i / 2] = pack_bf16x2(du[0], du[1]);
+          }
+        }
+        __syncwarp();  // every lane has read its g and u rows
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          *reinterpret_cast<uint4*>(gbuf + lane * EPI_ROW + j * 16) =
+              make_uint4(pg[4 * j], pg[4 * j + 1], pg[4 * j + 2], pg[4 * j + 3]);
+          *reinterpret_cast<uint4*>(ubuf + lane * EPI_ROW + j * 16) =
+              make_uint4(pu[4 * j], pu[4 * j + 1], pu[4 * j + 2], pu[4 * j + 3]);
+        }
+        __syncwarp();
+        if (col < g.n) {
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            const int rr = q * 32 + lr + 8 * i;
+            if (rr < t.rows) {
+              bf16* dst = g.d_h + (size_t)(t.m0 + rr) * ld + col + lc * 8;
+              *reinterpret_cast<uint4*>(dst) =
+                  *reinterpret_cast<const uint4*>(gbuf + (lr + 8 * i) * EPI_ROW + lc * 16);
+              *reinterpret_cast<uint4*>(dst + g.n) =
+                  *reinterpret_cast<const uint4*>(ubuf + (lr + 8 * i) * EPI_ROW + lc * 16);
+            }
+          }
+        }
+        __syncwarp();  // the buffer is free for the next chunk
       }
       if (row_ok) g.partial[(size_t)p * g.n_tiles + t.nt] = ds;
       tc_fence_before();
