@@ -51,7 +51,11 @@ constexpr int GATHER_THREADS = 128;
 constexpr uint32_t TMEM_COLS = 512;
 constexpr int MAXE = 256;
 constexpr int SMEM_TAIL = 4096;  // barriers, TMEM slot, abort flag, tile table
-constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 + SMEM_TAIL;
+// epilogue staging: per epilogue warp, its 32 rows of one 32-column output chunk, rows
+// padded to 80 bytes so that a thread writing its own row hits distinct banks
+constexpr int EPI_ROW = 80;
+constexpr int EPI_WARP_BYTES = 32 * EPI_ROW;
+constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 + SMEM_TAIL + 4 * EPI_WARP_BYTES;
 
 // Instruction descriptor, kind::f16: D fp32 (bit 4), A bf16 (bits 7-9 = 1), B bf16
 // (bits 10-12 = 1), A K-major (bit 15 = 0), B MN-major (bit 16 = 1), N >> 3 at bits 17-22,
@@ -216,6 +220,7 @@ __global__ void __launch_bounds__(GATEUP ? THREADS_GATEUP : THREADS_DOWN, 1)
   int* s_off = (int*)(tmem_slot + 2);
   int* s_cum = s_off + MAXE + 1;
   int* s_mt = s_cum + MAXE + 1;
+  uint8_t* epi = base + STAGES * STAGE_BYTES + SMEM_TAIL;  // epilogue staging (16-byte aligned)
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int E = g.E;
@@ -449,6 +454,10 @@ __global__ void __launch_bounds__(GATEUP ? THREADS_GATEUP : THREADS_DOWN, 1)
       const bool row_ok = r < t.rows;
       bf16* orow = g.out + (size_t)(t.m0 + (row_ok ? r : 0)) * g.ld_out;
       if (GATEUP) {
+        // each thread computes its row's 32 columns of a chunk; the warp's 32 rows go out
+        // through its padded buffer, one instruction storing 8 whole 64-byte row segments
+        uint8_t* ebuf = epi + q * EPI_WARP_BYTES;
+        const int lr = lane >> 2, lc = lane & 3;
 #pragma unroll 1
         for (int c = 0; c < 4; ++c) {
           uint32_t gv[32], uv[32];
@@ -456,7 +465,7 @@ __global__ void __launch_bounds__(GATEUP ? THREADS_GATEUP : THREADS_DOWN, 1)
           tmem_ld32(tb + 128 + c * 32, uv);
           tmem_ld_wait();
           const int col = t.n0 + c * 32;
-          if (row_ok && col < g.n_out) {
+          {
             uint32_t pk[16];
 #pragma unroll
             for (int j = 0; j < 16; ++j) {
@@ -466,25 +475,36 @@ __global__ void __launch_bounds__(GATEUP ? THREADS_GATEUP : THREADS_DOWN, 1)
               const float h1 = __fdividef(g1, 1.f + __expf(-g1)) * u1;
               pk[j] = pack_bf16x2(h0, h1);
             }
-            uint4* dst = reinterpret_cast<uint4*>(orow + col);
 #pragma unroll
             for (int j = 0; j < 4; ++j)
-              dst[j] = make_uint4(pk[4 * j], pk[4 * j + 1], pk[4 * j + 2], pk[4 * j + 3]);
-            if (g.h_out != nullptr) {  // keep (g | u) for the backward
-              bf16* hrow = g.h_out + (size_t)(t.m0 + r) * (2 * (size_t)g.n_out);
-              uint4* hg = reinterpret_cast<uint4*>(hrow + col);
-              uint4* hu = reinterpret_cast<uint4*>(hrow + g.n_out + col);
+              *reinterpret_cast<uint4*>(ebuf + lane * EPI_ROW + j * 16) =
+                  make_uint4(pk[4 * j], pk[4 * j + 1], pk[4 * j + 2], pk[4 * j + 3]);
+          }
+          __syncwarp();
+          if (col < g.n_out) {
 #pragma unroll
-              for (int j = 0; j < 4; ++j) {
-                hg[j] = make_uint4(pack_bf16x2(__uint_as_float(gv[8 * j]), __uint_as_float(gv[8 * j + 1])),
-                                   pack_bf16x2(__uint_as_float(gv[8 * j + 2]), __uint_as_float(gv[8 * j + 3])),
-                                   pack_bf16x2(__uint_as_float(gv[8 * j + 4]), __uint_as_float(gv[8 * j + 5])),
-                                   pack_bf16x2(__uint_as_float(gv[8 * j + 6]), __uint_as_float(gv[8 * j + 7])));
-                hu[j] = make_uint4(pack_bf16x2(__uint_as_float(uv[8 * j]), __uint_as_float(uv[8 * j + 1])),
-                                   pack_bf16x2(__uint_as_float(uv[8 * j + 2]), __uint_as_float(uv[8 * j + 3])),
-                                   pack_bf16x2(__uint_as_float(uv[8 * j + 4]), __uint_as_float(uv[8 * j + 5])),
-                                   pack_bf16x2(__uint_as_float(uv[8 * j + 6]), __uint_as_float(uv[8 * j + 7])));
-              }
+            for (int i = 0; i < 4; ++i) {
+              const int rr = q * 32 + lr + 8 * i;
+              if (rr < t.rows)
+                *reinterpret_cast<uint4*>(g.out + (size_t)(t.m0 + rr) * g.ld_out + col + lc * 8) =
+                    *reinterpret_cast<const uint4*>(ebuf + (lr + 8 * i) * EPI_ROW + lc * 16);
+            }
+          }
+          __syncwarp();  // the buffer is free for the next chunk
+          if (row_ok && col < g.n_out && g.h_out != nullptr) {  // keep (g | u) for the backward
+            bf16* hrow = g.h_out + (size_t)(t.m0 + r) * (2 * (size_t)g.n_out);
+            uint4* hg = reinterpret_cast<uint4*>(hrow + col);
+            uint4* hu = reinterpret_cast<uint4*>(hrow + g.n_out + col);
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+              hg[j] = make_uint4(pack_bf16x2(__uint_as_float(gv[8 * j]), __uint_as_float(gv[8 * j + 1])),
+                                 pack_bf16x2(__uint_as_float(gv[8 * j + 2]), __uint_as_float(gv[8 * j + 3])),
+                                 pack_bf16x2(__uint_as_float(gv[8 * j + 4]), __uint_as_float(gv[8 * j + 5])),
+                                 pack_bf16x2(__uint_as_float(gv[8 * j + 6]), __uint_as_float(gv[8 * j + 7])));
+              hu[j] = make_uint4(pack_bf16x2(__uint_as_float(uv[8 * j]), __uint_as_float(uv[8 * j + 1])),
+                                 pack_bf16x2(__uint_as_float(uv[8 * j + 2]), __uint_as_float(uv[8 * j + 3])),
+                                 pack_bf16x2(__uint_as_float(uv[8 * j + 4]), __uint_as_float(uv[8 * j + 5])),
+                                 pack_bf16x2(__uint_as_float(uv[8 * j + 6]), __uint_as_float(uv[8 * j + 7])));
             }
           }
         }
