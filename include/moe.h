@@ -447,6 +447,18 @@ int64_t moe_launch_count(void);
 moe_status moe_set_ffn_variant(int variant);
 int moe_get_ffn_variant(void);
 
+/* Layout of the bf16 tensor-core router (process-wide, not thread safe): 0 = automatic
+ * (currently form 1), 1 = each tile of up to 128 tokens split over the d contraction by a
+ * cluster of up to 8 CTAs (partials added in rank order through distributed shared memory),
+ * 2 = one tile of ceil(T / SMs) tokens per CTA over the whole of d when that is at most 128
+ * tokens (no cluster; otherwise one 128-token tile per CTA). Both compute the same selection
+ * rule; logits differ only by fp32 summation order. Form 2 is slower on B200 (it issues an
+ * M = 128 MMA per 16-wide k step for fewer useful rows); it is kept selectable for
+ * comparison. The pages have no counterpart: a deployment choice. Returns
+ * MOE_ERR_INVALID_ARG for other values. */
+moe_status moe_set_route_layout(int layout);
+int moe_get_route_layout(void);
+
 /* Test hook for the failure-detection path: launches one block that waits on
  * an mbarrier nothing will complete, bounded by `limit_ns` nanoseconds, then
  * records MOE_ERR_TIMEOUT in the device status word and returns (no trap, no

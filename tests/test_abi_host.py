@@ -199,3 +199,13 @@ def test_omni_argument_checks_on_host(lib):
     z = tdr.make_omni_shape(0, 256, 8, 8, 4)
     assert lib.moe_omni_route(ctypes.byref(z), None, None, None, None, None, None, None,
                               None) == 0
+
+
+def test_route_layout_knob_is_host_state(lib):
+    """The router layout knob checks its argument on the host and round-trips."""
+    assert lib.moe_set_route_layout(3) == 1
+    assert lib.moe_set_route_layout(-1) == 1
+    assert lib.moe_set_route_layout(2) == 0
+    assert tdr.get_route_layout() == 2
+    assert lib.moe_set_route_layout(0) == 0
+    assert tdr.get_route_layout() == 0

@@ -79,6 +79,15 @@ def ffn_variant(request, cuda_lib):
     cuda_lib.set_ffn_variant(0)
 
 
+@pytest.fixture(params=[0, 2], ids=["route_split", "route_tile_per_cta"])
+def route_layout(request, cuda_lib):
+    """Run a router test in both layouts of the tensor-core router (tiles split over
+    clusters, one tile per CTA over the whole of d)."""
+    cuda_lib.set_route_layout(request.param)
+    yield request.param
+    cuda_lib.set_route_layout(0)
+
+
 def inputs_for(cfg):
     if cfg.name not in _INPUTS:
         _INPUTS.clear()  # keep one large workload in host memory at a time
@@ -112,8 +121,14 @@ def test_bounded_wait_times_out_and_reports(cuda_lib):
     (1027, 256, 7, 2, "bf16", False, False),
     (9001, 4096, 8, 8, "bf16", True, True),
     (70, 4160, 8, 2, "bf16", False, True),
+    # per tile: 16, 21, 32 and 128 rows when one tile per SM runs over the whole of d
+    (2300, 1024, 16, 4, "bf16", True, True),
+    (3000, 512, 256, 8, "bf16", False, True),
+    (4736, 2048, 32, 4, "bf16", False, True),
+    (18900, 256, 64, 6, "bf16", True, False),
+    (18945, 128, 8, 2, "bf16", False, True),   # 129 rows per SM: split form again
 ])
-def test_route_matches_oracle(cuda_lib, T, d, E, K, dtype, bias, renorm):
+def test_route_matches_oracle(cuda_lib, route_layout, T, d, E, K, dtype, bias, renorm):
     tdr = cuda_lib
     cfg = mi.MoEConfig("route", T=T, d=d, E=E, K=K, n=64, dtype=dtype, seed=T + E)
     inp = mi.make_inputs(cfg, with_experts=False)
@@ -145,7 +160,7 @@ def test_route_ties_go_to_lower_id(cuda_lib):
 
 
 @pytest.mark.parametrize("d", [1024, 4096])
-def test_route_identical_router_columns_tie_exactly(cuda_lib, d):
+def test_route_identical_router_columns_tie_exactly(cuda_lib, route_layout, d):
     """Experts with identical router columns get bit-identical logits from x, so their
     order is decided by the id alone."""
     tdr = cuda_lib

@@ -97,6 +97,8 @@ _SIGS = {
     "moe_selftest_timeout": (ctypes.c_int, [ctypes.c_uint64, _P]),
     "moe_set_ffn_variant": (ctypes.c_int, [ctypes.c_int]),
     "moe_get_ffn_variant": (ctypes.c_int, []),
+    "moe_set_route_layout": (ctypes.c_int, [ctypes.c_int]),
+    "moe_get_route_layout": (ctypes.c_int, []),
 }
 
 _lib: Optional[ctypes.CDLL] = None
@@ -668,6 +670,16 @@ def set_ffn_variant(variant: int) -> None:
 
 def get_ffn_variant() -> int:
     return int(load_library().moe_get_ffn_variant())
+
+
+def set_route_layout(layout: int) -> None:
+    """bf16 router layout: 0 = automatic, 1 = tiles split over clusters, 2 = one tile per
+    CTA over the whole of d."""
+    _check(load_library().moe_set_route_layout(int(layout)), "moe_set_route_layout")
+
+
+def get_route_layout() -> int:
+    return int(load_library().moe_get_route_layout())
 
 
 def launch_count() -> int:

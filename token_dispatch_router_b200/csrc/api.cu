@@ -24,6 +24,7 @@ moe_status launch_combine(const moe_shape& s, const void* y_perm, const int32_t*
                           const float* topk_w, void* out, cudaStream_t st);
 moe_status launch_selftest_timeout(uint64_t limit_ns, cudaStream_t st);
 bool route_tc_supported(const moe_shape& s);
+extern int g_route_layout;
 moe_status launch_ffn_tc_mixed(const moe_shape& s, const void* x, const int32_t* offsets,
                                const int32_t* p2a, const void* w_gate, const void* w_up,
                                const void* w_down, void* a_act, void* y_perm, int gateup_mode,
@@ -582,6 +583,14 @@ moe_status moe_set_ffn_variant(int variant) {
 }
 
 int moe_get_ffn_variant(void) { return g_ffn_variant; }
+
+moe_status moe_set_route_layout(int layout) {
+  if (layout < 0 || layout > 2) return MOE_ERR_INVALID_ARG;
+  g_route_layout = layout;
+  return MOE_OK;
+}
+
+int moe_get_route_layout(void) { return g_route_layout; }
 
 moe_status moe_selftest_timeout(uint64_t limit_ns, moe_stream_t stream) {
   if (limit_ns == 0 || limit_ns > 10000000000ull) return MOE_ERR_INVALID_ARG;

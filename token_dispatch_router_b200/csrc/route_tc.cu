@@ -8,12 +8,17 @@
 //
 // The router GEMM (M = T tokens, N = E experts, K = d) has an arithmetic intensity of about
 // E FLOP per byte of x, so at E >= 32 fp32 FMA units cannot keep up with HBM; tcgen05 can.
-// Layout: one 128-token tile per cluster of S CTAs (S <= 8). The S CTAs split the d
-// contraction (k-blocks of 64); each accumulates its partial 128 x N tile in TMEM
-// (N = E rounded up to 16, fp32), copies it column-major into its shared memory, and
-// after a cluster barrier CTA rank 0 adds the partials of ranks 0..S-1 in that fixed
-// order through distributed shared memory (deterministic, no atomics, no global
-// scratch). Rank 0's 128 threads then own one token each: + bias, optional logits
+// Two layouts. With at least 16 tokens per SM (and at most 128), every CTA owns one tile of
+// ceil(T / SMs) tokens over the whole of d: no cluster, no cross-CTA reduction, and the x
+// tile is loaded with exactly its own rows (the MMA still computes 128 rows; rows past the
+// tile read whatever follows in shared memory and are never used, since a row of D depends
+// on the same row of A only), so a stage holds ceil(rows/8) KB of x and the ring is as deep
+// as shared memory allows. Otherwise one tile of up to 128 tokens per cluster of S CTAs
+// (S <= 8) that split the d contraction (k-blocks of 64); each accumulates its partial
+// 128 x N tile in TMEM (N = E rounded up to 16, fp32), copies it column-major into its
+// shared memory, and after a cluster barrier CTA rank 0 adds the partials of ranks
+// 0..S-1 in that fixed order through distributed shared memory (deterministic, no
+// atomics, no global scratch). Rank 0's 128 threads then own one token each: + bias, optional logits
 // store, register top-K by insertion (value descending, ties to the lower id, +0 == -0),
 // softmax weights over the selected (renormalised) or over all E with an online sum.
 // Roles per CTA (128 threads): warp 0 lane 0 issues the TMA loads (x tile 128 x 64 and
@@ -25,6 +30,8 @@
 #include "common.cuh"
 
 namespace moe {
+
+extern int g_route_layout;  // 0 automatic (split), 1 split over clusters, 2 one tile per CTA
 
 namespace {
 
@@ -44,9 +51,15 @@ struct RouteArgs {
   float* topk_w;
   int T, E, K, renorm, kblocks, S;
   int rows;  // tokens per tile (<= 128): a tile's MMA rows past it belong to the next tile
+  // Shared-memory ring: `stages` slots of `stage_bytes` (x tile of `a_slot` bytes, then the
+  // W_r chunks); each slot's barrier expects `tx_bytes`; barriers start at `bar_off`.
+  int a_slot, stage_bytes, stages, tx_bytes, bar_off;
   unsigned* status;
   unsigned long long limit_ns;
 };
+
+constexpr int R_MAX_STAGES = 32;
+constexpr int R_SMEM_MAX = 227 * 1024;
 
 __device__ __forceinline__ uint32_t saddr(const void* p) {
   return (uint32_t)__cvta_generic_to_shared(p);
@@ -156,21 +169,36 @@ __device__ __forceinline__ void top_insert(float (&bv)[KM], int (&be)[KM], float
   }
 }
 
+// Columns c0..c0+15 of this warp's 32 TMEM lanes (zeros when the CTA accumulated nothing).
+__device__ __forceinline__ void tmem_cols16(uint32_t trow, int c0, bool have, float (&lv)[16]) {
+  uint32_t v[16];
+  tmem_ld16(trow + (uint32_t)c0, v);
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+  for (int j = 0; j < 16; ++j) lv[j] = have ? __uint_as_float(v[j]) : 0.f;
+}
+__device__ __forceinline__ uint32_t elect_one() {
+  uint32_t p = 0;
+  asm volatile(
+      "{\n\t.reg .pred P;\n\t.reg .b32 R;\n\telect.sync R|P, 0xffffffff;\n\t"
+      "selp.u32 %0, 1, 0, P;\n\t}\n"
+      : "=r"(p));
+  return p;
+}
+
 template <int N, int KM>  // MMA N = E rounded up to 16; KM >= K, a power of two <= 8
 __global__ void __launch_bounds__(R_THREADS) route_tc_kernel(const __grid_constant__ CUtensorMap tmX,
                                                              const __grid_constant__ CUtensorMap tmW,
                                                              const RouteArgs g) {
   constexpr int NCH = (N + 63) / 64;         // B chunks of 64 experts
-  constexpr int B_BYTES = NCH * RB_CHUNK;
-  constexpr int STAGE = RA_BYTES + B_BYTES;
-  constexpr int RSTAGES = route_stages(N);
   constexpr uint32_t TCOLS = N <= 32 ? 32 : (N <= 64 ? 64 : (N <= 128 ? 128 : 256));
   constexpr uint32_t IDESC = (1u << 4) | (1u << 7) | (1u << 10) | (1u << 16) |
                              ((uint32_t)(N >> 3) << 17) | ((uint32_t)(RBM >> 4) << 24);
   extern __shared__ uint8_t smem_raw[];
   uint8_t* base = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
   uint8_t* ring = base;
-  uint64_t* bars = (uint64_t*)(base + RSTAGES * STAGE);
+  const int RSTAGES = g.stages, STAGE = g.stage_bytes, A_SLOT = g.a_slot;
+  uint64_t* bars = (uint64_t*)(base + g.bar_off);
   uint64_t* full = bars;
   uint64_t* empty = bars + RSTAGES;
   uint64_t* accf = bars + 2 * RSTAGES;
@@ -182,6 +210,9 @@ __global__ void __launch_bounds__(R_THREADS) route_tc_kernel(const __grid_consta
   const int tile = (int)cluster_id_x();
   const int S = g.S;
   const int kb0 = (int)(rank * g.kblocks / S), kb1 = (int)((rank + 1) * g.kblocks / S);
+  // Tiles start their k-blocks at different points of the range (and wrap), so that the
+  // CTAs do not all read the same W_r rows from the same L2 lines at the same time.
+  const int nkb = kb1 - kb0, rot = nkb > 0 ? tile % nkb : 0;
 
   if (tid == 32) {  // fetch both tensor maps while the barriers are set up
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmX)) : "memory");
@@ -210,58 +241,79 @@ __global__ void __launch_bounds__(R_THREADS) route_tc_kernel(const __grid_consta
   pdl_wait();  // the previous kernel in the stream has completed
   pdl_trigger();
 
-  if (warp == 0 && lane == 0) {
+  // Producer (warp 0) and MMA issuer (warp 1) run their loops warp-uniformly: lane 0 waits
+  // on the barrier and broadcasts the outcome, one elected lane issues. A single-lane loop
+  // issued about a third fewer small-N MMAs per cycle (the loop, not the tensor pipe, limits
+  // the rate at N = 16).
+  if (warp == 0) {
     int stage = 0;
     uint32_t phase = 0;
-    for (int kb = kb0; kb < kb1; ++kb) {
-      if (!mbar_wait(saddr(&empty[stage]), phase ^ 1u, g.status, g.limit_ns)) {
+    for (int i = 0; i < nkb; ++i) {
+      const int kb = kb0 + (i + rot) % nkb;
+      int w = 0;
+      if (lane == 0) w = mbar_wait(saddr(&empty[stage]), phase ^ 1u, g.status, g.limit_ns);
+      if (!__shfl_sync(0xffffffffu, w, 0)) {
         ok = false;
         break;
       }
-      const uint32_t fb = saddr(&full[stage]);
-      mbar_expect_tx(fb, STAGE);
-      const uint32_t a = saddr(ring + stage * STAGE);
-      tma_load_2d(a, &tmX, kb * RBK, tile * g.rows, fb);
+      if (elect_one()) {
+        const uint32_t fb = saddr(&full[stage]);
+        mbar_expect_tx(fb, (uint32_t)g.tx_bytes);
+        const uint32_t a = saddr(ring + stage * STAGE);
+        tma_load_2d(a, &tmX, kb * RBK, tile * g.rows, fb);
 #pragma unroll
-      for (int c = 0; c < NCH; ++c) tma_load_2d(a + RA_BYTES + c * RB_CHUNK, &tmW, c * 64, kb * RBK, fb);
+        for (int c = 0; c < NCH; ++c)
+          tma_load_2d(a + A_SLOT + c * RB_CHUNK, &tmW, c * 64, kb * RBK, fb);
+      }
+      __syncwarp();
       if (++stage == RSTAGES) {
         stage = 0;
         phase ^= 1u;
       }
     }
-  } else if (warp == 1 && lane == 0) {
+  } else if (warp == 1) {
+    // Descriptors of stage 0; a stage (and a 16-wide k step) moves the start-address field,
+    // which holds shared-memory byte addresses / 16 (below 2^14, so adding does not carry).
+    const uint64_t ad0 = desc_sw128(saddr(ring), 16, 1024);
+    const uint64_t bd0 = desc_sw128(saddr(ring) + A_SLOT, RB_CHUNK, 1024);
     int stage = 0;
     uint32_t phase = 0;
-    for (int kb = kb0; kb < kb1; ++kb) {
-      if (!mbar_wait(saddr(&full[stage]), phase, g.status, g.limit_ns)) {
+    for (int i = 0; i < nkb; ++i) {
+      int w = 0;
+      if (lane == 0) w = mbar_wait(saddr(&full[stage]), phase, g.status, g.limit_ns);
+      if (!__shfl_sync(0xffffffffu, w, 0)) {
         ok = false;
         break;
       }
       asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-      const uint32_t a = saddr(ring + stage * STAGE);
+      if (elect_one()) {
+        const uint64_t so = (uint64_t)((stage * STAGE) >> 4);
 #pragma unroll
-      for (int kk = 0; kk < RBK / 16; ++kk) {
-        const uint64_t ad = desc_sw128(a + kk * 32, 16, 1024);
-        const uint64_t bd = desc_sw128(a + RA_BYTES + kk * 2048, RB_CHUNK, 1024);
-        const uint32_t acc = (kb > kb0 || kk > 0) ? 1u : 0u;
+        for (int kk = 0; kk < RBK / 16; ++kk) {
+          const uint32_t acc = (i | kk) != 0 ? 1u : 0u;
+          asm volatile(
+              "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+              "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(tmem),
+              "l"(ad0 + so + (uint64_t)(kk * 2)), "l"(bd0 + so + (uint64_t)(kk * 128)),
+              "r"(IDESC), "r"(acc)
+              : "memory");
+        }
         asm volatile(
-            "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
-            "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(tmem),
-            "l"(ad), "l"(bd), "r"(IDESC), "r"(acc)
+            "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+                saddr(&empty[stage]))
             : "memory");
       }
-      asm volatile(
-          "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
-              saddr(&empty[stage]))
-          : "memory");
+      __syncwarp();
       if (++stage == RSTAGES) {
         stage = 0;
         phase ^= 1u;
       }
     }
-    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
-                     saddr(accf))
-                 : "memory");
+    if (elect_one())
+      asm volatile(
+          "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+              saddr(accf))
+          : "memory");
   }
   __syncwarp();
   // every thread: the accumulator of this CTA is complete (bounded)
@@ -277,11 +329,10 @@ __global__ void __launch_bounds__(R_THREADS) route_tc_kernel(const __grid_consta
     // publish this CTA's partial (column-major) for rank 0, then wait until it was read
 #pragma unroll
     for (int c0 = 0; c0 < N; c0 += 16) {
-      uint32_t v[16];
-      tmem_ld16(trow + c0, v);
-      asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+      float lv[16];
+      tmem_cols16(trow, c0, have, lv);
 #pragma unroll
-      for (int j = 0; j < 16; ++j) part[(c0 + j) * RBM + r] = have ? __uint_as_float(v[j]) : 0.f;
+      for (int j = 0; j < 16; ++j) part[(c0 + j) * RBM + r] = lv[j];
     }
     cluster_sync();
     cluster_sync();
@@ -302,14 +353,11 @@ __global__ void __launch_bounds__(R_THREADS) route_tc_kernel(const __grid_consta
       be[k] = -1;
     }
     float m = -INFINITY, ssum = 0.f;  // online max / sum of exp for the plain softmax
+    const bool live = warp * 32 < g.rows;  // warp-uniform: this warp holds rows of the tile
 #pragma unroll 1
-    for (int c0 = 0; c0 < N; c0 += 16) {
-      uint32_t v[16];
-      tmem_ld16(trow + c0, v);
-      asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+    for (int c0 = 0; live && c0 < N; c0 += 16) {
       float lv[16];
-#pragma unroll
-      for (int j = 0; j < 16; ++j) lv[j] = have ? __uint_as_float(v[j]) : 0.f;
+      tmem_cols16(trow, c0, have, lv);
       // partials of the other ranks, added in rank order; up to four ranks' loads in flight
       for (int q0 = 1; q0 < S; q0 += 4) {
         float pv[4][16];
@@ -348,7 +396,7 @@ __global__ void __launch_bounds__(R_THREADS) route_tc_kernel(const __grid_consta
         }
       }
     }
-    if (t < g.T) {
+    if (live && t < g.T) {
       const float top = bv[0];
       float den = 0.f;
 #pragma unroll
@@ -437,18 +485,49 @@ int active_clusters(Kern kern, int smem, int S) {
   return cache[S];
 }
 
+// Shared-memory ring for N-wide W_r chunks. own: one tile of `rows` tokens per CTA, x slots
+// of ceil(rows/8) KB and as many stages as fit (the last slot's 128-row MMA read may run
+// 16 KB past its start, so the ring is padded to cover it); otherwise 128-row x slots at
+// route_stages(N) deep. Returns the dynamic shared memory size, or 0 if the epilogue's
+// staging buffers would not fit in the ring.
+int ring_layout(int N, int E, int K, bool own, int rows, RouteArgs& a) {
+  const int nch = (N + 63) / 64;
+  a.a_slot = own ? ((rows + 7) / 8) * 1024 : RA_BYTES;
+  a.stage_bytes = a.a_slot + nch * RB_CHUNK;
+  a.tx_bytes = own ? rows * 128 + nch * RB_CHUNK : a.stage_bytes;
+  auto ring_of = [&](int st) { return max(st * a.stage_bytes, (st - 1) * a.stage_bytes + RA_BYTES); };
+  auto smem_of = [&](int st) { return 1024 + ring_of(st) + (2 * st + 2) * 8; };
+  int st = own ? R_MAX_STAGES : route_stages(N);
+  if (own)
+    while (st > 2 && smem_of(st) > R_SMEM_MAX) --st;
+  a.stages = st;
+  a.bar_off = ring_of(st);
+  const int staging = RBM * (E + 1) * 4 + 2 * RBM * K * 4;
+  const int partials = N * RBM * 4;
+  if (smem_of(st) > R_SMEM_MAX || ring_of(st) < staging || ring_of(st) < partials) return 0;
+  return smem_of(st);
+}
+
 template <int N, int KM>
-moe_status launch_nk(const CUtensorMap& mx, const CUtensorMap& mw, RouteArgs a, int tiles,
-                    cudaStream_t st) {
-  constexpr int NCH = (N + 63) / 64;
-  constexpr int STAGE = RA_BYTES + NCH * RB_CHUNK;
-  const int smem = route_stages(N) * STAGE + 1024 + 256;
+moe_status launch_nk(const void* x, const void* w_r, RouteArgs a, int tiles, bool own,
+                     cudaStream_t st) {
   auto kern = route_tc_kernel<N, KM>;
+  int smem = own ? ring_layout(N, a.E, a.K, true, a.rows, a) : 0;
+  if (smem == 0 && own) {  // the ring does not fit: one 128-token tile per CTA, no split
+    own = false;
+    a.rows = RBM;
+    a.S = 1;
+    tiles = (a.T + RBM - 1) / RBM;
+  }
+  if (smem == 0) {  // one tile of up to 128 tokens per cluster of S CTAs
+    smem = ring_layout(N, a.E, a.K, false, RBM, a);
+    if (smem == 0) return MOE_ERR_UNSUPPORTED;
+  }
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
     return MOE_ERR_CUDA;
   // With fewer 128-token tiles than clusters that fit at once, shorter tiles (at least 64
   // tokens) put more SMs to work; the MMA still computes 128 rows, the surplus unwritten.
-  if (a.S > 1) {
+  if (!own && a.S > 1) {
     const int fit = active_clusters(kern, smem, a.S);
     const int want = min(fit, (a.T + 63) / 64);
     if (want > tiles) {
@@ -456,6 +535,10 @@ moe_status launch_nk(const CUtensorMap& mx, const CUtensorMap& mw, RouteArgs a, 
       tiles = (a.T + a.rows - 1) / a.rows;
     }
   }
+  CUtensorMap mx, mw;
+  if (!make_map_2d(&mx, x, (uint64_t)(a.kblocks * RBK), (uint64_t)a.T, 64, own ? a.rows : RBM))
+    return MOE_ERR_CUDA;
+  if (!make_map_2d(&mw, w_r, (uint64_t)a.E, (uint64_t)(a.kblocks * RBK), 64, 64)) return MOE_ERR_CUDA;
   launch_begin(K_ROUTE_TC, st);
   launch_kernel(kern, dim3((unsigned)(tiles * a.S)), dim3(R_THREADS), (size_t)smem, st,
                 (unsigned)a.S, mx, mw, a);
@@ -463,16 +546,18 @@ moe_status launch_nk(const CUtensorMap& mx, const CUtensorMap& mw, RouteArgs a, 
 }
 
 template <int KM>
-moe_status launch_n(int N, const CUtensorMap& mx, const CUtensorMap& mw, const RouteArgs& a,
-                    int tiles, cudaStream_t st) {
-  if (N <= 16) return launch_nk<16, KM>(mx, mw, a, tiles, st);
-  if (N <= 32) return launch_nk<32, KM>(mx, mw, a, tiles, st);
-  if (N <= 64) return launch_nk<64, KM>(mx, mw, a, tiles, st);
-  if (N <= 128) return launch_nk<128, KM>(mx, mw, a, tiles, st);
-  return launch_nk<256, KM>(mx, mw, a, tiles, st);
+moe_status launch_n(int N, const void* x, const void* w_r, const RouteArgs& a, int tiles,
+                    bool own, cudaStream_t st) {
+  if (N <= 16) return launch_nk<16, KM>(x, w_r, a, tiles, own, st);
+  if (N <= 32) return launch_nk<32, KM>(x, w_r, a, tiles, own, st);
+  if (N <= 64) return launch_nk<64, KM>(x, w_r, a, tiles, own, st);
+  if (N <= 128) return launch_nk<128, KM>(x, w_r, a, tiles, own, st);
+  return launch_nk<256, KM>(x, w_r, a, tiles, own, st);
 }
 
 }  // namespace
+
+int g_route_layout = 0;
 
 bool route_tc_supported(const moe_shape& s) {
   return s.dtype == MOE_BF16 && s.E % 8 == 0 && s.E <= 256 && s.K <= KMAX && s.d % 64 == 0;
@@ -480,25 +565,29 @@ bool route_tc_supported(const moe_shape& s) {
 
 moe_status launch_route_tc(const moe_shape& s, const void* x, const void* w_r, const float* bias,
                            float* logits_out, int32_t* ids, float* w, cudaStream_t st) {
-  const int tiles = (s.T + RBM - 1) / RBM;
+  int tiles = (s.T + RBM - 1) / RBM;
   const int kblocks = s.d / RBK;
-  // Split d over S CTAs so that about one CTA per SM works, but never beyond the CTAs that
-  // can be resident at once (a second wave costs more than the split saves).
-  const int npad = ((s.E + 15) / 16) * 16;
-  const int nmma = npad <= 16 ? 16 : npad <= 32 ? 32 : npad <= 64 ? 64 : npad <= 128 ? 128 : 256;
-  const int smem_cta =
-      route_stages(nmma) * (RA_BYTES + ((nmma + 63) / 64) * RB_CHUNK) + 1024 + 256;
-  const int per_sm = (227 * 1024) / smem_cta;
-  int S = (sm_count() + tiles - 1) / tiles;
-  const int resident = sm_count() * (per_sm > 0 ? per_sm : 1);
-  if (S > resident / tiles) S = resident / tiles;
-  if (S > 8) S = 8;
-  if (S > kblocks) S = kblocks;
-  if (S < 1) S = 1;
   const int N = ((s.E + 15) / 16) * 16;  // MMA N (a multiple of 16 for M = 128)
-  CUtensorMap mx, mw;
-  if (!make_map_2d(&mx, x, (uint64_t)s.d, (uint64_t)s.T, 64, 128)) return MOE_ERR_CUDA;
-  if (!make_map_2d(&mw, w_r, (uint64_t)s.E, (uint64_t)s.d, 64, 64)) return MOE_ERR_CUDA;
+  const int nmma = N <= 16 ? 16 : N <= 32 ? 32 : N <= 64 ? 64 : N <= 128 ? 128 : 256;
+  // On request, one tile of ceil(T / SMs) <= 128 tokens per CTA over the whole of d (no
+  // split, no cluster). Not the default: it issues one M = 128 MMA per 16-wide k step for
+  // fewer useful rows, and the MMA issue loop, not HBM, bounds this kernel.
+  const int rows_own = (s.T + sm_count() - 1) / sm_count();
+  const bool own = g_route_layout == 2 && rows_own <= RBM;
+  int S = 1;
+  if (!own) {
+    // Split d over S CTAs so that about one CTA per SM works, but never beyond the CTAs
+    // that can be resident at once (a second wave costs more than the split saves).
+    const int smem_cta =
+        route_stages(nmma) * (RA_BYTES + ((nmma + 63) / 64) * RB_CHUNK) + 1024 + 256;
+    const int per_sm = R_SMEM_MAX / smem_cta;
+    S = (sm_count() + tiles - 1) / tiles;
+    const int resident = sm_count() * (per_sm > 0 ? per_sm : 1);
+    if (S > resident / tiles) S = resident / tiles;
+    if (S > 8) S = 8;
+    if (S > kblocks) S = kblocks;
+    if (S < 1) S = 1;
+  }
   RouteArgs a;
   a.bias = bias;
   a.logits_out = logits_out;
@@ -510,13 +599,14 @@ moe_status launch_route_tc(const moe_shape& s, const void* x, const void* w_r, c
   a.renorm = s.renormalize;
   a.kblocks = kblocks;
   a.S = S;
-  a.rows = RBM;
+  a.rows = own ? rows_own : RBM;
+  if (own) tiles = (s.T + a.rows - 1) / a.rows;
   a.status = device_status_ptr();
   a.limit_ns = kWaitLimitNs;
   // instantiations cover N up to the next of 16/32/64/128/256; columns past E read zeros
-  if (s.K <= 2) return launch_n<2>(N, mx, mw, a, tiles, st);
-  if (s.K <= 4) return launch_n<4>(N, mx, mw, a, tiles, st);
-  return launch_n<8>(N, mx, mw, a, tiles, st);
+  if (s.K <= 2) return launch_n<2>(N, x, w_r, a, tiles, own, st);
+  if (s.K <= 4) return launch_n<4>(N, x, w_r, a, tiles, own, st);
+  return launch_n<8>(N, x, w_r, a, tiles, own, st);
 }
 
 }  // namespace moe
