@@ -54,6 +54,7 @@ struct RouteArgs {
   // Shared-memory ring: `stages` slots of `stage_bytes` (x tile of `a_slot` bytes, then the
   // W_r chunks); each slot's barrier expects `tx_bytes`; barriers start at `bar_off`.
   int a_slot, stage_bytes, stages, tx_bytes, bar_off;
+  int vec_logits;  // logits_out is 16-byte aligned: the split form stores rows as float4
   unsigned* status;
   unsigned long long limit_ns;
 };
@@ -124,6 +125,12 @@ __device__ __forceinline__ uint32_t cluster_id_x() {
   uint32_t r;
   asm volatile("mov.u32 %0, %%clusterid.x;" : "=r"(r));
   return r;
+}
+__device__ __forceinline__ void cluster_arrive() {
+  asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void cluster_wait() {
+  asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
 }
 __device__ __forceinline__ void cluster_sync() {
   asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::
@@ -325,8 +332,12 @@ __global__ void __launch_bounds__(R_THREADS) route_tc_kernel(const __grid_consta
   const int r = warp * 32 + lane;  // token row of this thread inside the tile
   const uint32_t trow = tmem + ((uint32_t)(warp * 32) << 16);
 
-  if (S > 1 && rank != 0) {
-    // publish this CTA's partial (column-major) for rank 0, then wait until it was read
+  if (S > 1) {
+    // Every rank publishes its partial (column-major), then after one cluster barrier each
+    // rank finishes a contiguous share of the tile's rows, one thread per row, adding the S
+    // partials in rank order through distributed shared memory (the same fp32 sum in the
+    // same order whichever rank does it). A rank arrives on the closing barrier as soon as
+    // its remote reads are done and waits on it only before exiting.
 #pragma unroll
     for (int c0 = 0; c0 < N; c0 += 16) {
       float lv[16];
@@ -335,9 +346,90 @@ __global__ void __launch_bounds__(R_THREADS) route_tc_kernel(const __grid_consta
       for (int j = 0; j < 16; ++j) part[(c0 + j) * RBM + r] = lv[j];
     }
     cluster_sync();
-    cluster_sync();
+    const int share = (g.rows + S - 1) / S;
+    const int row = (int)rank * share + tid;
+    const bool mine = tid < share && row < g.rows;
+    const int t = tile * g.rows + row;
+    const int E = g.E, K = g.K;
+    float bv[KM];
+    int be[KM];
+#pragma unroll
+    for (int k = 0; k < KM; ++k) {
+      bv[k] = -INFINITY;
+      be[k] = -1;
+    }
+    float m = -INFINITY, ssum = 0.f;  // online max / sum of exp for the plain softmax
+    if (mine && t < g.T) {
+      const uint32_t own = saddr(&part[row]);
+#pragma unroll 1
+      for (int c0 = 0; c0 < N && c0 < E; c0 += 16) {
+        float lv[16];
+        for (int q0 = 0; q0 < S; q0 += 4) {  // up to four ranks' loads in flight
+          float pv[4][16];
+#pragma unroll
+          for (int qq = 0; qq < 4; ++qq) {
+            if (q0 + qq < S) {
+              const uint32_t rb = map_rank(own + (uint32_t)(c0 * RBM * 4), (uint32_t)(q0 + qq));
+#pragma unroll
+              for (int j = 0; j < 16; ++j) pv[qq][j] = ld_dsmem(rb + (uint32_t)(j * RBM * 4));
+            }
+          }
+#pragma unroll
+          for (int qq = 0; qq < 4; ++qq)
+            if (q0 + qq < S)
+#pragma unroll
+              for (int j = 0; j < 16; ++j) lv[j] = q0 + qq == 0 ? pv[0][j] : lv[j] + pv[qq][j];
+        }
+#pragma unroll
+        for (int j = 0; j < 16; ++j) {
+          const int e = c0 + j;
+          if (e < E) {
+            if (g.bias != nullptr) lv[j] += g.bias[e];
+            top_insert<KM>(bv, be, lv[j], e);
+            if (!g.renorm) {
+              if (lv[j] > m) {
+                ssum = ssum * expf(m - lv[j]) + 1.f;
+                m = lv[j];
+              } else {
+                ssum += expf(lv[j] - m);
+              }
+            }
+          }
+        }
+        if (g.logits_out != nullptr) {  // E is a multiple of 8: whole groups of four
+          float* dst = g.logits_out + (size_t)t * E + c0;
+#pragma unroll
+          for (int j4 = 0; j4 < 4; ++j4) {
+            if (c0 + 4 * j4 < E) {
+              if (g.vec_logits)
+                *reinterpret_cast<float4*>(dst + 4 * j4) =
+                    make_float4(lv[4 * j4], lv[4 * j4 + 1], lv[4 * j4 + 2], lv[4 * j4 + 3]);
+              else
+#pragma unroll
+                for (int u = 0; u < 4; ++u) dst[4 * j4 + u] = lv[4 * j4 + u];
+            }
+          }
+        }
+      }
+    }
+    cluster_arrive();  // this rank's reads of its peers' partials are done
+    if (mine && t < g.T) {
+      const float top = bv[0];
+      float den = 0.f;
+#pragma unroll
+      for (int k = 0; k < KM; ++k)
+        if (k < K) den += expf(bv[k] - top);
+      if (!g.renorm) den = ssum * expf(m - top);
+#pragma unroll
+      for (int k = 0; k < KM; ++k) {
+        if (k < K) {
+          g.topk_ids[(size_t)t * K + k] = be[k];
+          g.topk_w[(size_t)t * K + k] = expf(bv[k] - top) / den;
+        }
+      }
+    }
+    cluster_wait();  // no CTA exits while a peer may still read its partials
   } else {
-    if (S > 1) cluster_sync();  // partials of ranks 1..S-1 are in their shared memory
     const int t = tile * g.rows + r;
     const int E = g.E, K = g.K;
     // Outputs are staged in this CTA's (idle) ring and written back coalesced: the tile's
@@ -358,23 +450,6 @@ __global__ void __launch_bounds__(R_THREADS) route_tc_kernel(const __grid_consta
     for (int c0 = 0; live && c0 < N; c0 += 16) {
       float lv[16];
       tmem_cols16(trow, c0, have, lv);
-      // partials of the other ranks, added in rank order; up to four ranks' loads in flight
-      for (int q0 = 1; q0 < S; q0 += 4) {
-        float pv[4][16];
-#pragma unroll
-        for (int qq = 0; qq < 4; ++qq) {
-          if (q0 + qq < S) {
-            const uint32_t rbase = map_rank(saddr(&part[c0 * RBM + r]), (uint32_t)(q0 + qq));
-#pragma unroll
-            for (int j = 0; j < 16; ++j) pv[qq][j] = ld_dsmem(rbase + (uint32_t)(j * RBM * 4));
-          }
-        }
-#pragma unroll
-        for (int qq = 0; qq < 4; ++qq)
-          if (q0 + qq < S)
-#pragma unroll
-            for (int j = 0; j < 16; ++j) lv[j] += pv[qq][j];
-      }
 #pragma unroll
       for (int j = 0; j < 16; ++j) {
         const int e = c0 + j;
@@ -421,7 +496,6 @@ __global__ void __launch_bounds__(R_THREADS) route_tc_kernel(const __grid_consta
       g.topk_ids[t0 * K + i] = st_i[i];
       g.topk_w[t0 * K + i] = st_w[i];
     }
-    if (S > 1) cluster_sync();  // peers may exit now
   }
   (void)ok;
   asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
@@ -600,6 +674,7 @@ moe_status launch_route_tc(const moe_shape& s, const void* x, const void* w_r, c
   a.kblocks = kblocks;
   a.S = S;
   a.rows = own ? rows_own : RBM;
+  a.vec_logits = ((uintptr_t)logits_out & 15) == 0;
   if (own) tiles = (s.T + a.rows - 1) / a.rows;
   a.status = device_status_ptr();
   a.limit_ns = kWaitLimitNs;
