@@ -8,22 +8,27 @@
 //
 // The router GEMM (M = T tokens, N = E experts, K = d) has an arithmetic intensity of about
 // E FLOP per byte of x, so at E >= 32 fp32 FMA units cannot keep up with HBM; tcgen05 can.
-// Two layouts. With at least 16 tokens per SM (and at most 128), every CTA owns one tile of
-// ceil(T / SMs) tokens over the whole of d: no cluster, no cross-CTA reduction, and the x
-// tile is loaded with exactly its own rows (the MMA still computes 128 rows; rows past the
-// tile read whatever follows in shared memory and are never used, since a row of D depends
-// on the same row of A only), so a stage holds ceil(rows/8) KB of x and the ring is as deep
-// as shared memory allows. Otherwise one tile of up to 128 tokens per cluster of S CTAs
-// (S <= 8) that split the d contraction (k-blocks of 64); each accumulates its partial
-// 128 x N tile in TMEM (N = E rounded up to 16, fp32), copies it column-major into its
-// shared memory, and after a cluster barrier CTA rank 0 adds the partials of ranks
-// 0..S-1 in that fixed order through distributed shared memory (deterministic, no
-// atomics, no global scratch). Rank 0's 128 threads then own one token each: + bias, optional logits
+// Default layout: one tile of up to 128 tokens per cluster of S CTAs (S <= 8) that split
+// the d contraction (k-blocks of 64); each accumulates its partial 128 x N tile in TMEM
+// (N = E rounded up to 16, fp32) and copies it column-major into its shared memory. After
+// a cluster barrier every rank finishes a contiguous share of the tile's rows, one thread
+// per row, adding the partials of ranks 0..S-1 in that fixed order through distributed
+// shared memory (deterministic, no atomics, no global scratch): + bias, optional logits
 // store, register top-K by insertion (value descending, ties to the lower id, +0 == -0),
-// softmax weights over the selected (renormalised) or over all E with an online sum.
-// Roles per CTA (128 threads): warp 0 lane 0 issues the TMA loads (x tile 128 x 64 and
-// the W_r tile 64 x N, 128-byte swizzle), warp 1 lane 0 issues the MMAs (M=128, N, K=16,
-// A K-major, B MN-major), then all four warps read TMEM (warp w owns lanes 32w..32w+31).
+// softmax weights over the selected (renormalised) or over all E with an online sum. With
+// S = 1 the CTA's 128 threads own one row each and stage the outputs for coalesced stores.
+// On request (moe_set_route_layout(2)) every CTA owns one tile of ceil(T / SMs) <= 128
+// tokens over the whole of d instead: no cluster; the x tile is loaded with exactly its own
+// rows (the MMA still computes 128 rows; rows past the tile read whatever follows in shared
+// memory and are never used, since a row of D depends on the same row of A only), so a
+// stage holds ceil(rows/8) KB of x and the ring is as deep as shared memory allows. It is
+// slower: the kernel is bound by issuing its small-N MMAs, and that form issues one per
+// 16-wide k step for fewer useful rows.
+// Roles per CTA (128 threads): warp 0 issues the TMA loads (x tile rows x 64 and the W_r
+// tile 64 x N, 128-byte swizzle), warp 1 the MMAs (M=128, N, K=16, A K-major, B MN-major),
+// both as warp-uniform loops with one elected lane issuing; then all four warps read TMEM
+// (warp w owns lanes 32w..32w+31). Each tile starts its k-blocks at a different offset so
+// that the CTAs do not all read the same W_r lines at once.
 // Every mbarrier wait is bounded; on expiry the status word records MOE_ERR_TIMEOUT.
 #include <math.h>
 
