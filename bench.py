@@ -53,7 +53,7 @@ def parse():
     ap.add_argument("--ref-tokens", type=int, default=64,
                     help="tokens per step of the reference arm (the CPU oracle)")
     ap.add_argument("--ffn-variant", type=int, default=0, choices=[0, 1, 2, 3],
-                    help="grouped-GEMM tile variant (moe_set_ffn_variant): 0 automatic, 1 "
+                    help="grouped-GEMM tile variant (moe_shape.ffn_variant): 0 automatic, 1 "
                          "single-CTA, 2 CTA pairs, 3 CTA pairs with the rows gathered first")
     ap.add_argument("--only", choices=["atomic_experts", "backward"], default=None,
                     help="run one secondary figure alone and print it (for profiling)")
@@ -646,23 +646,24 @@ def atomic_experts_figure(tdr, world, peaks, n=10):
         raise RuntimeError("device status set during the atomic-expert runs")
     kern = {k: round(v[1] / n * 1e3, 1) for k, v in prof.results().items()}
     # the page's output side for comparison: expert-centric scatter-add (atomic fp32 rows)
-    tdr.omni_set_output_mode(1)
-    try:
-        for _ in range(2):
-            once()
+    s_sc = tdr.make_omni_shape(c.T, c.d, c.n_rows, c.n_cols, c.K, c.renormalize, output_mode=1)
+
+    def once_scatter():
+        tdr.omni_forward(s_sc, x, wr, wc, wi, wo, out=out, workspace=ws)
+
+    for _ in range(2):
+        once_scatter()
+    torch.cuda.synchronize()
+    prof2 = tdr.Profiler()
+    with prof2:
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(n):
+            once_scatter()
+        e1.record()
         torch.cuda.synchronize()
-        prof2 = tdr.Profiler()
-        with prof2:
-            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            e0.record()
-            for _ in range(n):
-                once()
-            e1.record()
-            torch.cuda.synchronize()
-        scatter = {"ms_back_to_back": round(max_over_ranks(e0.elapsed_time(e1) / n, world), 4),
-                   "output_us": round(prof2.results()["omni_out"][1] / n * 1e3, 1)}
-    finally:
-        tdr.omni_set_output_mode(0)
+    scatter = {"ms_back_to_back": round(max_over_ranks(e0.elapsed_time(e1) / n, world), 4),
+               "output_us": round(prof2.results()["omni_out"][1] / n * 1e3, 1)}
     counts = tdr.omni_workspace_views(s, ws)["counts"]
     active = int((counts > 0).sum().item())
     nb = atomic_experts_bytes(c)
@@ -687,7 +688,6 @@ def atomic_experts_figure(tdr, world, peaks, n=10):
 def run_ours(args, rank, world, local):
     import token_dispatch_router_b200 as tdr
     tdr.load_library()  # fails loudly if the CUDA library is missing
-    tdr.set_ffn_variant(args.ffn_variant)
     if args.only == "atomic_experts":
         fig = atomic_experts_figure(tdr, world, load_peaks()[0], n=max(1, args.steps))
         if rank == 0:
@@ -701,7 +701,8 @@ def run_ours(args, rank, world, local):
     w_r = inp.w_r.to(dev)
     wg, wu, wd = inp.w_gate.to(dev), inp.w_up.to(dev), inp.w_down.to(dev)
     bias = None if inp.bias is None else inp.bias.to(dev)
-    s = tdr.make_shape(cfg.T, cfg.d, cfg.E, cfg.K, cfg.n, cfg.capacity_factor, True, dt)
+    s = tdr.make_shape(cfg.T, cfg.d, cfg.E, cfg.K, cfg.n, cfg.capacity_factor, True, dt,
+                       ffn_variant=args.ffn_variant)
     ws = torch.empty(tdr.forward_workspace_size(s), dtype=torch.uint8, device=dev)
     out = torch.empty(cfg.T, cfg.d, dtype=dt, device=dev)
     stream = torch.cuda.current_stream()

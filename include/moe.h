@@ -78,6 +78,14 @@ typedef struct {
   int32_t renormalize;
   int32_t dtype;      /* moe_dtype */
   int32_t tile_round; /* 0, or the row tile R that each expert's kept count is rounded to */
+  int32_t ffn_variant; /* tiles of the bf16 grouped GEMMs (a deployment choice; the pages have
+                        * no counterpart): 0 = automatic, 1 = single-CTA 128 x 256 tiles,
+                        * 2 = CTA pairs (256 x 256 tiles on two SMs, tcgen05 cta_group::2)
+                        * with the gate/up rows gathered inside the GEMM, 3 = CTA pairs with
+                        * the gate/up rows first copied expert-major into the y_perm buffer
+                        * by one gather kernel. All compute the same result; other values
+                        * return MOE_ERR_INVALID_ARG. A per-call field: calls on different
+                        * streams or threads may choose differently. */
 } moe_shape;
 
 /* ----------------------------------------------------------------------------
@@ -347,6 +355,14 @@ moe_status moe_backward_router(const moe_shape* shape, const void* x, const void
 typedef struct {
   int32_t T, d, n_rows, n_cols, K;
   int32_t renormalize; /* != 0: weights renormalised over the K selected */
+  int32_t output_mode; /* output side of moe_omni_forward (moe_omni_experts always gathers,
+                        * having no workspace for the fp32 sums): 0 = token-centric
+                        * gather, y_t = sum_k h w_out[i_k] summed per token in slot order
+                        * (deterministic); 1 = the page's expert-centric scatter-add (section
+                        * 2.3): each expert's w_out row is read once and h * w_out[e] is added
+                        * into its tokens' fp32 rows with atomic vector reductions, then
+                        * rounded to bf16 (the fp32 sum order, and so the last bits, vary from
+                        * run to run). Other values return MOE_ERR_INVALID_ARG. */
 } moe_omni_shape;
 
 /* Byte offsets inside the workspace of moe_omni_forward (each 256-byte aligned). */
@@ -407,14 +423,6 @@ moe_status moe_omni_forward(const moe_omni_shape* shape, const void* x, const vo
                             const void* w_out, void* out, void* workspace, size_t ws_bytes,
                             moe_stream_t stream);
 
-/* Output side of moe_omni_forward (process-wide, not thread safe): 0 (default) = token-centric
- * gather, y_t = sum_k h w_out[i_k] summed per token in slot order (deterministic); 1 = the
- * page's expert-centric scatter-add (section 2.3): each expert's w_out row is read once and
- * h * w_out[e] is added into its tokens' fp32 rows with atomic vector reductions, then
- * rounded to bf16 (the fp32 sum order, and so the last bits, vary from run to run). */
-moe_status moe_omni_set_output_mode(int mode);
-int moe_omni_get_output_mode(void);
-
 /* ----------------------------------------------------------------------------
  * Device status: synchronises `stream`, returns the first device-side fault
  * recorded since the last call (MOE_OK if none) and clears it.
@@ -436,28 +444,6 @@ int moe_kernel_count(void);
 const char* moe_kernel_name(int id);
 moe_status moe_profile_query(int id, int64_t* launches, double* total_ms);
 int64_t moe_launch_count(void);
-
-/* Tile variant of the bf16 grouped GEMMs (process-wide, not thread safe): 0 = automatic,
- * 1 = always single-CTA 128 x 256 tiles, 2 = always CTA pairs (256 x 256 tiles on two SMs,
- * tcgen05 cta_group::2) with the gate/up A rows gathered inside the GEMM, 3 = CTA pairs with
- * the gate/up A rows first copied expert-major into the y_perm buffer by one gather kernel
- * and loaded from there by TMA. All compute the same result; the choice trades row padding
- * (256-row tiles pad more) and the extra copy against traffic per SM (pairs move a third
- * less). */
-moe_status moe_set_ffn_variant(int variant);
-int moe_get_ffn_variant(void);
-
-/* Layout of the bf16 tensor-core router (process-wide, not thread safe): 0 = automatic
- * (currently form 1), 1 = each tile of up to 128 tokens split over the d contraction by a
- * cluster of up to 8 CTAs (partials added in rank order through distributed shared memory),
- * 2 = one tile of ceil(T / SMs) tokens per CTA over the whole of d when that is at most 128
- * tokens (no cluster; otherwise one 128-token tile per CTA). Both compute the same selection
- * rule; logits differ only by fp32 summation order. Form 2 is slower on B200 (it issues an
- * M = 128 MMA per 16-wide k step for fewer useful rows); it is kept selectable for
- * comparison. The pages have no counterpart: a deployment choice. Returns
- * MOE_ERR_INVALID_ARG for other values. */
-moe_status moe_set_route_layout(int layout);
-int moe_get_route_layout(void);
 
 /* Test hook for the failure-detection path: launches one block that waits on
  * an mbarrier nothing will complete, bounded by `limit_ns` nanoseconds, then

@@ -7,6 +7,7 @@ import re
 import subprocess
 
 import pytest
+import torch
 
 import token_dispatch_router_b200 as tdr
 
@@ -193,19 +194,30 @@ def test_omni_argument_checks_on_host(lib):
     # experts without the scalar buffer
     assert lib.moe_omni_experts(ctypes.byref(s), dummy, dummy, dummy, dummy, dummy, dummy, dummy,
                                 None, dummy, None) == 1
-    # output modes: 0 and 1 only
-    assert lib.moe_omni_set_output_mode(2) == 1 and lib.moe_omni_get_output_mode() == 0
+    # output modes: 0 and 1 only (a field of the shape, checked per call)
+    bad = tdr.make_omni_shape(16, 256, 8, 8, 4, output_mode=2)
+    assert lib.moe_omni_workspace_size(ctypes.byref(bad)) == 0
+    assert lib.moe_omni_forward(ctypes.byref(bad), dummy, dummy, dummy, None, dummy, dummy, dummy,
+                                dummy, 1 << 30, None) == 1
     # T = 0 is a no-op
     z = tdr.make_omni_shape(0, 256, 8, 8, 4)
     assert lib.moe_omni_route(ctypes.byref(z), None, None, None, None, None, None, None,
                               None) == 0
 
 
-def test_route_layout_knob_is_host_state(lib):
-    """The router layout knob checks its argument on the host and round-trips."""
-    assert lib.moe_set_route_layout(3) == 1
-    assert lib.moe_set_route_layout(-1) == 1
-    assert lib.moe_set_route_layout(2) == 0
-    assert tdr.get_route_layout() == 2
-    assert lib.moe_set_route_layout(0) == 0
-    assert tdr.get_route_layout() == 0
+@pytest.mark.parametrize("variant,code", [(0, 0), (3, 0), (4, 1), (-1, 1)])
+def test_ffn_variant_is_a_checked_shape_field(lib, variant, code):
+    """The grouped-GEMM tile variant travels with each call's shape (no process-wide state):
+    valid values size a workspace, others are rejected on the host."""
+    s = tdr.make_shape(64, 128, 8, 2, 128, 0.0, True, torch.bfloat16, ffn_variant=variant)
+    size = lib.moe_forward_workspace_size(ctypes.byref(s))
+    assert (size > 0) == (code == 0)
+    if code:
+        assert lib.moe_grouped_ffn(ctypes.byref(s), *([ctypes.c_void_p(256)] * 8), None) == code
+
+
+def test_no_process_wide_switches_exported(lib):
+    """Variant and output-mode selection are per-call shape fields, not library state."""
+    for name in ("moe_set_ffn_variant", "moe_get_ffn_variant", "moe_set_route_layout",
+                 "moe_get_route_layout", "moe_omni_set_output_mode", "moe_omni_get_output_mode"):
+        assert not hasattr(lib, name), name

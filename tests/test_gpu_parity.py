@@ -25,10 +25,10 @@ def cuda(t):
     return None if t is None else t.cuda()
 
 
-def shape_of(cfg, tdr, T=None):
+def shape_of(cfg, tdr, T=None, ffn_variant=0):
     dt = torch.bfloat16 if cfg.dtype == "bf16" else torch.float32
     return tdr.make_shape(cfg.T if T is None else T, cfg.d, cfg.E, cfg.K, cfg.n,
-                          cfg.capacity_factor, True, dt)
+                          cfg.capacity_factor, True, dt, ffn_variant=ffn_variant)
 
 
 def assert_status_ok(tdr):
@@ -71,21 +71,10 @@ _INPUTS = {}
 
 
 @pytest.fixture(params=[1, 2, 3], ids=["single_cta", "cta_pair", "cta_pair_tma_a"])
-def ffn_variant(request, cuda_lib):
+def ffn_variant(request):
     """Run a test with the single-CTA grouped GEMM, the CTA-pair one gathering its rows, and
-    the CTA-pair one reading rows copied expert-major beforehand."""
-    cuda_lib.set_ffn_variant(request.param)
-    yield request.param
-    cuda_lib.set_ffn_variant(0)
-
-
-@pytest.fixture(params=[0, 2], ids=["route_split", "route_tile_per_cta"])
-def route_layout(request, cuda_lib):
-    """Run a router test in both layouts of the tensor-core router (tiles split over
-    clusters, one tile per CTA over the whole of d)."""
-    cuda_lib.set_route_layout(request.param)
-    yield request.param
-    cuda_lib.set_route_layout(0)
+    the CTA-pair one reading rows copied expert-major beforehand (the shape's ffn_variant)."""
+    return request.param
 
 
 def inputs_for(cfg):
@@ -128,7 +117,7 @@ def test_bounded_wait_times_out_and_reports(cuda_lib):
     (18900, 256, 64, 6, "bf16", True, False),
     (18945, 128, 8, 2, "bf16", False, True),   # 129 rows per SM: split form again
 ])
-def test_route_matches_oracle(cuda_lib, route_layout, T, d, E, K, dtype, bias, renorm):
+def test_route_matches_oracle(cuda_lib, T, d, E, K, dtype, bias, renorm):
     tdr = cuda_lib
     cfg = mi.MoEConfig("route", T=T, d=d, E=E, K=K, n=64, dtype=dtype, seed=T + E)
     inp = mi.make_inputs(cfg, with_experts=False)
@@ -160,7 +149,7 @@ def test_route_ties_go_to_lower_id(cuda_lib):
 
 
 @pytest.mark.parametrize("d", [1024, 4096])
-def test_route_identical_router_columns_tie_exactly(cuda_lib, route_layout, d):
+def test_route_identical_router_columns_tie_exactly(cuda_lib, d):
     """Experts with identical router columns get bit-identical logits from x, so their
     order is decided by the id alone."""
     tdr = cuda_lib
@@ -368,11 +357,11 @@ def test_combine_matches_oracle(cuda_lib, dtype):
 
 
 # ------------------------------------------------------------------ grouped FFN
-def _ffn_case(tdr, T, d, n, E, K, cf, dtype, seed):
+def _ffn_case(tdr, T, d, n, E, K, cf, dtype, seed, ffn_variant=0):
     cfg = mi.MoEConfig("ffn", T=T, d=d, E=E, K=K, n=n, dtype=dtype, capacity_factor=cf,
                        seed=seed)
     inp = mi.make_inputs(cfg)
-    s = shape_of(cfg, tdr)
+    s = shape_of(cfg, tdr, ffn_variant=ffn_variant)
     lo = torch.empty(T, E, dtype=torch.float32, device="cuda")
     ids, w, _ = tdr.route(s, cuda(inp.x), cuda(inp.w_r), logits_out=lo)
     perm = tdr.permute(s, ids)
@@ -407,7 +396,8 @@ def test_grouped_ffn_fp32_tiny_workload(cuda_lib):
 ])
 def test_grouped_ffn_bf16_tensor_cores(cuda_lib, ffn_variant, T, d, n, E, K, cf):
     tdr = cuda_lib
-    a, a_ref, y, y_ref, out, out_ref = _ffn_case(tdr, T, d, n, E, K, cf, "bf16", T + d)
+    a, a_ref, y, y_ref, out, out_ref = _ffn_case(tdr, T, d, n, E, K, cf, "bf16", T + d,
+                                                 ffn_variant)
     assert_bf16_close(a, a_ref, "a_act")
     assert_bf16_close(y, y_ref, "y_perm")
     assert_bf16_close(out, out_ref, "out")
@@ -438,7 +428,7 @@ def test_forward_full_size_workloads(cuda_lib, ffn_variant, name):
     tdr = cuda_lib
     cfg = mi.CONFIGS[name]
     inp = inputs_for(cfg)
-    s = shape_of(cfg, tdr)
+    s = shape_of(cfg, tdr, ffn_variant=ffn_variant)
     out, ws = tdr.forward(s, cuda(inp.x), cuda(inp.w_r), cuda(inp.w_gate), cuda(inp.w_up),
                           cuda(inp.w_down), bias=cuda(inp.bias))
     torch.cuda.synchronize()
@@ -712,7 +702,7 @@ def test_forward_edge_cases(cuda_lib, ffn_variant):
         cfg = mi.MoEConfig("edge", T=T, d=d, E=E, K=K, n=n, dtype="bf16", capacity_factor=cf,
                            seed=T + E)
         inp = mi.make_inputs(cfg)
-        s = shape_of(cfg, tdr)
+        s = shape_of(cfg, tdr, ffn_variant=ffn_variant)
         logits = None
         if force:
             lg = np.zeros((T, E), np.float32)
@@ -732,7 +722,7 @@ def test_forward_edge_cases(cuda_lib, ffn_variant):
         else:
             assert_bf16_close(got, ref["out"], f"edge T={T} E={E} cf={cf}")
         assert_status_ok(tdr)
-    s0 = tdr.make_shape(0, 64, 4, 2, 64, 0.0, True, torch.bfloat16)
+    s0 = tdr.make_shape(0, 64, 4, 2, 64, 0.0, True, torch.bfloat16, ffn_variant=ffn_variant)
     z = torch.empty(0, 64, dtype=torch.bfloat16, device="cuda")
     w = torch.zeros(64, 4, dtype=torch.bfloat16, device="cuda")
     wg = torch.zeros(4, 64, 64, dtype=torch.bfloat16, device="cuda")

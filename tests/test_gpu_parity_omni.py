@@ -26,8 +26,8 @@ def cfg_of(T, d, nr, nc, K, renorm=True, logits_given=False, seed=0):
                          renormalize=renorm, logits_given=logits_given, seed=seed)
 
 
-def shape_of(tdr, c):
-    return tdr.make_omni_shape(c.T, c.d, c.n_rows, c.n_cols, c.K, c.renormalize)
+def shape_of(tdr, c, output_mode=0):
+    return tdr.make_omni_shape(c.T, c.d, c.n_rows, c.n_cols, c.K, c.renormalize, output_mode)
 
 
 def rel_errors(got, ref):
@@ -173,12 +173,10 @@ def test_experts_given_routing(cuda_lib, T, d, nr, nc, K):
 
 
 @pytest.fixture(params=[0, 1], ids=["gather_out", "scatter_add_out"])
-def output_mode(request, cuda_lib):
+def output_mode(request):
     """Run a forward test with the token-centric gather and with the expert-centric
-    scatter-add on the output side."""
-    cuda_lib.omni_set_output_mode(request.param)
-    yield request.param
-    cuda_lib.omni_set_output_mode(0)
+    scatter-add on the output side (the shape's output_mode)."""
+    return request.param
 
 
 @pytest.mark.parametrize("renorm", [True, False])
@@ -186,7 +184,7 @@ def test_forward_small(cuda_lib, renorm, output_mode):
     tdr = cuda_lib
     c = cfg_of(256, 256, 32, 32, 64, renorm)
     inp = mi.make_omni_inputs(c)
-    s = shape_of(tdr, c)
+    s = shape_of(tdr, c, output_mode)
     out, ws = tdr.omni_forward(s, inp.x.cuda(), inp.w_row.cuda(), inp.w_col.cuda(),
                                inp.w_in.cuda(), inp.w_out.cuda())
     torch.cuda.synchronize()
@@ -219,7 +217,7 @@ def test_forward_102k_experts_sampled_tokens(cuda_lib, output_mode):
     tdr = cuda_lib
     c = mi.OMNI_102K
     inp = mi.make_omni_inputs(c)
-    s = shape_of(tdr, c)
+    s = shape_of(tdr, c, output_mode)
     out, ws = tdr.omni_forward(s, inp.x.cuda(), inp.w_row.cuda(), inp.w_col.cuda(),
                                inp.w_in.cuda(), inp.w_out.cuda())
     torch.cuda.synchronize()

@@ -33,7 +33,8 @@ class moe_shape(ctypes.Structure):
     _fields_ = [("T", ctypes.c_int32), ("d", ctypes.c_int32), ("E", ctypes.c_int32),
                 ("K", ctypes.c_int32), ("n", ctypes.c_int32),
                 ("capacity_factor", ctypes.c_float), ("renormalize", ctypes.c_int32),
-                ("dtype", ctypes.c_int32), ("tile_round", ctypes.c_int32)]
+                ("dtype", ctypes.c_int32), ("tile_round", ctypes.c_int32),
+                ("ffn_variant", ctypes.c_int32)]
 
 
 class moe_workspace_layout(ctypes.Structure):
@@ -46,7 +47,7 @@ class moe_workspace_layout(ctypes.Structure):
 class moe_omni_shape(ctypes.Structure):
     _fields_ = [("T", ctypes.c_int32), ("d", ctypes.c_int32), ("n_rows", ctypes.c_int32),
                 ("n_cols", ctypes.c_int32), ("K", ctypes.c_int32),
-                ("renormalize", ctypes.c_int32)]
+                ("renormalize", ctypes.c_int32), ("output_mode", ctypes.c_int32)]
 
 
 class moe_omni_layout(ctypes.Structure):
@@ -83,8 +84,6 @@ _SIGS = {
     "moe_omni_experts": (ctypes.c_int, [_O, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P]),
     "moe_omni_forward": (ctypes.c_int, [_O, _P, _P, _P, _P, _P, _P, _P, _P, ctypes.c_size_t,
                                         _P]),
-    "moe_omni_set_output_mode": (ctypes.c_int, [ctypes.c_int]),
-    "moe_omni_get_output_mode": (ctypes.c_int, []),
     "moe_get_device_status": (ctypes.c_int, [_P]),
     "moe_status_string": (ctypes.c_char_p, [ctypes.c_int]),
     "moe_profile_enable": (ctypes.c_int, [ctypes.c_int]),
@@ -95,10 +94,6 @@ _SIGS = {
                                          ctypes.POINTER(ctypes.c_double)]),
     "moe_launch_count": (ctypes.c_int64, []),
     "moe_selftest_timeout": (ctypes.c_int, [ctypes.c_uint64, _P]),
-    "moe_set_ffn_variant": (ctypes.c_int, [ctypes.c_int]),
-    "moe_get_ffn_variant": (ctypes.c_int, []),
-    "moe_set_route_layout": (ctypes.c_int, [ctypes.c_int]),
-    "moe_get_route_layout": (ctypes.c_int, []),
 }
 
 _lib: Optional[ctypes.CDLL] = None
@@ -127,11 +122,15 @@ def _check(code: int, where: str) -> None:
 
 
 def make_shape(T: int, d: int, E: int, K: int, n: int = 0, capacity_factor: float = 0.0,
-               renormalize: bool = True, dtype=torch.bfloat16, tile_round: int = 0) -> moe_shape:
-    """tile_round = R > 0 rounds each expert's kept count down to whole R-row tiles."""
+               renormalize: bool = True, dtype=torch.bfloat16, tile_round: int = 0,
+               ffn_variant: int = 0) -> moe_shape:
+    """tile_round = R > 0 rounds each expert's kept count down to whole R-row tiles.
+    ffn_variant selects the bf16 grouped-GEMM tiles: 0 = automatic, 1 = single-CTA 128 x 256
+    tiles, 2 = CTA-pair 256 x 256 tiles with the gate/up rows gathered in the GEMM, 3 = CTA
+    pairs with the rows copied first (all compute the same result)."""
     dt = MOE_BF16 if dtype == torch.bfloat16 else MOE_F32
     return moe_shape(T, d, E, K, n, float(capacity_factor), 1 if renormalize else 0, dt,
-                     int(tile_round))
+                     int(tile_round), int(ffn_variant))
 
 
 def _ptr(t: Optional[torch.Tensor]):
@@ -484,9 +483,11 @@ def workspace_views(shape: moe_shape, workspace: torch.Tensor) -> dict:
 
 # ------------------------------------------------------------------ atomic experts
 def make_omni_shape(T: int, d: int, n_rows: int, n_cols: int, K: int,
-                    renormalize: bool = True) -> moe_omni_shape:
-    """N = n_rows * n_cols rank-1 experts on a Cartesian grid, top-K per token."""
-    return moe_omni_shape(T, d, n_rows, n_cols, K, 1 if renormalize else 0)
+                    renormalize: bool = True, output_mode: int = 0) -> moe_omni_shape:
+    """N = n_rows * n_cols rank-1 experts on a Cartesian grid, top-K per token. output_mode
+    (moe_omni_forward): 0 = token-centric gather (deterministic), 1 = expert-centric
+    scatter-add."""
+    return moe_omni_shape(T, d, n_rows, n_cols, K, 1 if renormalize else 0, int(output_mode))
 
 
 def omni_workspace_size(shape: moe_omni_shape) -> int:
@@ -596,15 +597,6 @@ def omni_forward(shape: moe_omni_shape, x, w_row, w_col, w_in, w_out, logits_in=
     return out, workspace
 
 
-def omni_set_output_mode(mode: int) -> None:
-    """0 = token-centric gather (default, deterministic); 1 = expert-centric scatter-add."""
-    _check(load_library().moe_omni_set_output_mode(int(mode)), "moe_omni_set_output_mode")
-
-
-def omni_get_output_mode() -> int:
-    return int(load_library().moe_omni_get_output_mode())
-
-
 def omni_workspace_views(shape: moe_omni_shape, workspace: torch.Tensor) -> dict:
     """Typed views of moe_omni_forward's intermediates inside its workspace (perm_to_assign
     grouped by expert, any order inside an expert; assign_to_perm is not written)."""
@@ -660,26 +652,6 @@ class Profiler:
             if n.value:
                 out[self.lib.moe_kernel_name(i).decode()] = (int(n.value), float(ms.value))
         return out
-
-
-def set_ffn_variant(variant: int) -> None:
-    """0 = automatic, 1 = single-CTA 128 x 256 tiles, 2 = CTA-pair 256 x 256 tiles with
-    the gate/up rows gathered in the GEMM, 3 = CTA pairs with the rows copied first."""
-    _check(load_library().moe_set_ffn_variant(int(variant)), "moe_set_ffn_variant")
-
-
-def get_ffn_variant() -> int:
-    return int(load_library().moe_get_ffn_variant())
-
-
-def set_route_layout(layout: int) -> None:
-    """bf16 router layout: 0 = automatic, 1 = tiles split over clusters, 2 = one tile per
-    CTA over the whole of d."""
-    _check(load_library().moe_set_route_layout(int(layout)), "moe_set_route_layout")
-
-
-def get_route_layout() -> int:
-    return int(load_library().moe_get_route_layout())
 
 
 def launch_count() -> int:

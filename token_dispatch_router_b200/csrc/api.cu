@@ -24,7 +24,6 @@ moe_status launch_combine(const moe_shape& s, const void* y_perm, const int32_t*
                           const float* topk_w, void* out, cudaStream_t st);
 moe_status launch_selftest_timeout(uint64_t limit_ns, cudaStream_t st);
 bool route_tc_supported(const moe_shape& s);
-extern int g_route_layout;
 moe_status launch_ffn_tc_mixed(const moe_shape& s, const void* x, const int32_t* offsets,
                                const int32_t* p2a, const void* w_gate, const void* w_up,
                                const void* w_down, void* a_act, void* y_perm, int gateup_mode,
@@ -158,6 +157,7 @@ moe_status check_shape(const moe_shape* s, bool need_d, bool need_ffn) {
   if (isnan(s->capacity_factor)) return MOE_ERR_INVALID_ARG;
   if (s->tile_round < 0 || (s->tile_round > 0 && s->capacity_factor > 0.f))
     return MOE_ERR_INVALID_ARG;  // token rounding and a capacity limit are exclusive
+  if (s->ffn_variant < 0 || s->ffn_variant > 3) return MOE_ERR_INVALID_ARG;
   if (need_d) {
     if (s->d < 64 || s->d % 64 != 0) return MOE_ERR_INVALID_ARG;
   }
@@ -202,17 +202,15 @@ bool layout_of(const moe_shape& s, moe_workspace_layout* L) {
 
 bool aligned16(const void* p) { return ((uintptr_t)p & 15) == 0; }
 
-int g_ffn_variant = 0;  // 0 auto, 1 single-CTA tiles, 2 CTA-pair tiles, 3 CTA pairs, A by TMA
-
-// Automatic choice, from measurements on B200: the gate/up GEMM runs single-CTA tiles
-// (its gathered A operand gains nothing from pairing, and 256-row tiles pad twice as many
-// rows); the down GEMM runs on CTA pairs once experts average at least 512 rows, where the
-// pair's deeper pipeline beats the extra padding.
+// Tile variant (moe_shape.ffn_variant). Automatic choice, from measurements on B200: the
+// gate/up GEMM runs single-CTA tiles (its gathered A operand gains nothing from pairing, and
+// 256-row tiles pad twice as many rows); the down GEMM runs on CTA pairs once experts
+// average at least 512 rows, where the pair's deeper pipeline beats the extra padding.
 bool use_pair_down(const moe_shape& s) {
-  if (g_ffn_variant != 0) return g_ffn_variant >= 2;
+  if (s.ffn_variant != 0) return s.ffn_variant >= 2;
   return (long long)s.T * s.K >= 512LL * s.E;
 }
-int gateup_mode() { return g_ffn_variant == 2 ? 1 : g_ffn_variant == 3 ? 2 : 0; }
+int gateup_mode(const moe_shape& s) { return s.ffn_variant == 2 ? 1 : s.ffn_variant == 3 ? 2 : 0; }
 
 }  // namespace
 }  // namespace moe
@@ -422,7 +420,7 @@ moe_status moe_grouped_ffn(const moe_shape* s, const void* x, const int32_t* off
     return MOE_ERR_INVALID_ARG;
   if (s->dtype == MOE_BF16)
     return launch_ffn_tc_mixed(*s, x, offsets, perm_to_assign, w_gate, w_up, w_down, a_act, y_perm,
-                               gateup_mode(), use_pair_down(*s), nullptr, (cudaStream_t)stream);
+                               gateup_mode(*s), use_pair_down(*s), nullptr, (cudaStream_t)stream);
   return launch_ffn_simt(*s, x, offsets, perm_to_assign, w_gate, w_up, w_down, a_act, y_perm,
                          (cudaStream_t)stream);
 }
@@ -575,22 +573,6 @@ int64_t moe_launch_count(void) {
   std::lock_guard<std::mutex> lk(g_prof_mu);
   return g_launches;
 }
-
-moe_status moe_set_ffn_variant(int variant) {
-  if (variant < 0 || variant > 3) return MOE_ERR_INVALID_ARG;
-  g_ffn_variant = variant;
-  return MOE_OK;
-}
-
-int moe_get_ffn_variant(void) { return g_ffn_variant; }
-
-moe_status moe_set_route_layout(int layout) {
-  if (layout < 0 || layout > 2) return MOE_ERR_INVALID_ARG;
-  g_route_layout = layout;
-  return MOE_OK;
-}
-
-int moe_get_route_layout(void) { return g_route_layout; }
 
 moe_status moe_selftest_timeout(uint64_t limit_ns, moe_stream_t stream) {
   if (limit_ns == 0 || limit_ns > 10000000000ull) return MOE_ERR_INVALID_ARG;

@@ -1553,8 +1553,6 @@ moe_status launch_omni_out(const moe_omni_shape& s, const void* w_out, const int
   }
 }
 
-int g_omni_output_mode = 0;  // 0 token-centric gather, 1 expert-centric scatter-add
-
 moe_status launch_omni_out_scatter(const moe_omni_shape& s, const void* w_out,
                                    const int32_t* offsets, const int32_t* p2a, const float* h,
                                    float* y32, void* out, cudaStream_t st) {
@@ -1605,6 +1603,7 @@ moe_status check_omni(const moe_omni_shape* s) {
   if (s == nullptr) return MOE_ERR_INVALID_ARG;
   if (s->T < 0 || s->n_rows < 1 || s->n_cols < 1 || s->K < 1 || s->d < 256 || s->d % 256 != 0)
     return MOE_ERR_INVALID_ARG;
+  if (s->output_mode < 0 || s->output_mode > 1) return MOE_ERR_INVALID_ARG;
   const long long N = (long long)s->n_rows * s->n_cols;
   if (s->K > N) return MOE_ERR_INVALID_ARG;
   if (s->n_rows > 1024 || s->n_cols > 1024 || N > (1LL << 20) || s->K > 4096)
@@ -1751,19 +1750,11 @@ moe_status moe_omni_forward(const moe_omni_shape* s, const void* x, const void* 
   if ((r = launch_omni_schedule(*s, ids, counts, offsets, a2p, p2a, ws + L.scratch, true, false,
                                 st)) != MOE_OK)
     return r;
-  if (g_omni_output_mode == 0)
+  if (s->output_mode == 0)
     return moe_omni_experts(s, x, w_in, w_out, ids, w, offsets, p2a, h, out, stream);
   if (!al16(x) || !al16(w_in) || !al16(w_out) || !al16(out)) return MOE_ERR_INVALID_ARG;
   if ((r = launch_omni_act(*s, x, w_in, offsets, p2a, w, h, st)) != MOE_OK) return r;
   return launch_omni_out_scatter(*s, w_out, offsets, p2a, h, (float*)(ws + L.y32), out, st);
 }
-
-moe_status moe_omni_set_output_mode(int mode) {
-  if (mode < 0 || mode > 1) return MOE_ERR_INVALID_ARG;
-  g_omni_output_mode = mode;
-  return MOE_OK;
-}
-
-int moe_omni_get_output_mode(void) { return g_omni_output_mode; }
 
 }  // extern "C"

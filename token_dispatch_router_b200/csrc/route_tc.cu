@@ -1,116 +1,85 @@
 // Router on the tensor cores for bf16 shapes: logits = x W_r (+ bias) with tcgen05, then
-// softmax and top-K in the epilogue, one token per thread.
+// softmax and top-K in the epilogue.
 //
 // "How AI chips support MoE", chapter 4, section 4.2: the gate is a small dense linear map
 // that every token passes through and that the experts wait on; section 4.3: top-K is a
 // partial sort per token. "Two upstream innovations of MoE: Routing-Free and OmniMoE",
 // section 1.1: Router -> Softmax -> TopK.
 //
-// The router GEMM (M = T tokens, N = E experts, K = d) has an arithmetic intensity of about
-// E FLOP per byte of x, so at E >= 32 fp32 FMA units cannot keep up with HBM; tcgen05 can.
-// Default layout: one tile of up to 128 tokens per cluster of S CTAs (S <= 8) that split
-// the d contraction (k-blocks of 64); each accumulates its partial 128 x N tile in TMEM
-// (N = E rounded up to 16, fp32) and copies it column-major into its shared memory. After
-// a cluster barrier every rank finishes a contiguous share of the tile's rows, one thread
-// per row, adding the partials of ranks 0..S-1 in that fixed order through distributed
-// shared memory (deterministic, no atomics, no global scratch): + bias, optional logits
-// store, register top-K by insertion (value descending, ties to the lower id, +0 == -0),
-// softmax weights over the selected (renormalised) or over all E with an online sum. With
-// S = 1 the CTA's 128 threads own one row each and stage the outputs for coalesced stores.
-// On request (moe_set_route_layout(2)) every CTA owns one tile of ceil(T / SMs) <= 128
-// tokens over the whole of d instead: no cluster; the x tile is loaded with exactly its own
-// rows (the MMA still computes 128 rows; rows past the tile read whatever follows in shared
-// memory and are never used, since a row of D depends on the same row of A only), so a
-// stage holds ceil(rows/8) KB of x and the ring is as deep as shared memory allows. It is
-// slower: the kernel is bound by issuing its small-N MMAs, and that form issues one per
-// 16-wide k step for fewer useful rows.
-// Roles per CTA (128 threads): warp 0 issues the TMA loads (x tile rows x 64 and the W_r
-// tile 64 x N, 128-byte swizzle), warp 1 the MMAs (M=128, N, K=16, A K-major, B MN-major),
-// both as warp-uniform loops with one elected lane issuing; then all four warps read TMEM
-// (warp w owns lanes 32w..32w+31). Each tile starts its k-blocks at a different offset so
-// that the CTAs do not all read the same W_r lines at once.
-// Every mbarrier wait is bounded; on expiry the status word records MOE_ERR_TIMEOUT.
+// The product is computed transposed, D[e, t] = sum_k W_r[k, e] x[t, k]: experts on the
+// MMA's M (one 128-row M tile per 128 experts; rows past E are never read) and tokens on its
+// N (up to 256 per instruction). The router's contraction d is long and its output narrow,
+// so the kernel's cost is the number of tcgen05.mma instructions one thread issues per CTA,
+// (d / S / 16) per M tile, not their size: putting 256 tokens on N instead of 128 on M
+// halves that count, and an instruction of N = 256 costs the tensor pipe no more than the
+// issue loop sustains.
+// Layout: one tile of up to 256 tokens per cluster of S CTAs (S = 1, 2, 4 or 8) that split
+// the d contraction into contiguous ranges of 64-wide k-blocks. Operands: A = W_r rows
+// [64 k][64 e] as MN-major 128-byte-swizzled chunks (one TMA box per chunk, experts past E
+// zero-filled); B = the x tile [rows][64 k], K-major, 128-byte swizzle. The partial
+// D[e, t] (fp32, TMEM lanes = experts, columns = tokens) is copied to shared memory as
+// [e][t] rows; after a cluster barrier every rank finishes a contiguous share of the tile's
+// tokens, G threads per token (each owning experts g, g + G, ...), adding the partials of
+// ranks 0..S-1 in that order through distributed shared memory (deterministic: the same
+// fp32 sum in the same order whichever rank does it), + bias, optional logits store, a
+// register top-KM list per thread (value descending, ties to the lower id, +0 == -0), the G
+// lists merged by a bitonic network over shuffles, softmax weights over the selected
+// (renormalised) or over all E (online sum, merged the same way).
+// Roles (256 threads): warp 0 issues the TMA loads, warp 1 the MMAs, both as warp-uniform
+// loops with one elected lane issuing; warps 4m..4m+3 read M tile m from TMEM (warp w owns
+// lanes 32 (w % 4) ...); all eight warps reduce. Each tile starts its k-blocks at a
+// different offset so that the CTAs do not all read the same W_r lines at once.
+// Every mbarrier wait is bounded; on expiry the status word records MOE_ERR_TIMEOUT and the
+// CTA skips its remaining work (cluster barriers are still passed, so no peer waits).
 #include <math.h>
 
-#include "common.cuh"
+#include <mutex>
+
+#include "tc_ptx.cuh"
 
 namespace moe {
 
-extern int g_route_layout;  // 0 automatic (split), 1 split over clusters, 2 one tile per CTA
-
 namespace {
 
-constexpr int RBM = 128, RBK = 64;
-constexpr int RA_BYTES = RBM * RBK * 2;  // 16 KB
-constexpr int RB_CHUNK = RBK * 64 * 2;   // 8 KB: 64 k-rows x 64 experts
-constexpr int R_THREADS = 128;
-constexpr int KMAX = 8;
+using namespace ptx;
 
-// Pipeline depth: the x stream is latency-bound per CTA, so small-N stages (24 KB) go 8 deep.
-__host__ __device__ constexpr int route_stages(int N) { return N <= 64 ? 8 : (N <= 128 ? 6 : 4); }
+constexpr int RBK = 64;                  // k per stage: one 128-byte swizzle atom of bf16
+constexpr int RCHUNK = RBK * 64 * 2;     // 8 KB: A chunk of 64 k-rows x 64 experts
+constexpr int R_THREADS = 256;
+constexpr int KMAX = 8;
+constexpr int R_SMEM_MAX = 227 * 1024;
+constexpr int R_MAX_STAGES = 8;
 
 struct RouteArgs {
   const float* bias;
   float* logits_out;
   int32_t* topk_ids;
   float* topk_w;
-  int T, E, K, renorm, kblocks, S;
-  int rows;  // tokens per tile (<= 128): a tile's MMA rows past it belong to the next tile
-  // Shared-memory ring: `stages` slots of `stage_bytes` (x tile of `a_slot` bytes, then the
-  // W_r chunks); each slot's barrier expects `tx_bytes`; barriers start at `bar_off`.
-  int a_slot, stage_bytes, stages, tx_bytes, bar_off;
-  int vec_logits;  // logits_out is 16-byte aligned: the split form stores rows as float4
+  int T, E, K, renorm;
+  int kblocks;   // d / 64
+  int S;         // CTAs of a cluster splitting d
+  int rows;      // tokens per tile (<= 256); tile i holds tokens [i rows, (i + 1) rows)
+  int nmma;      // the MMA's N: rows rounded up to 16
+  int a_chunks;  // W_r chunks loaded per stage: ceil(E / 64)
+  int a_slot;    // bytes of a stage's A slot: 16 KB per M tile
+  int stage_bytes, stages, tx_bytes, bar_off;
+  int ps;        // row stride (floats) of the partial tile part[e][t] in shared memory
+  int G;         // threads per token in the epilogue (1, 2, 4 or 8)
+  int vec_logits;  // G == 1 and logits_out 16-byte aligned: rows stored as float4
   unsigned* status;
   unsigned long long limit_ns;
 };
 
-constexpr int R_MAX_STAGES = 32;
-constexpr int R_SMEM_MAX = 227 * 1024;
-
-__device__ __forceinline__ uint32_t saddr(const void* p) {
-  return (uint32_t)__cvta_generic_to_shared(p);
-}
-__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
-  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
-}
-__device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
-  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes)
-               : "memory");
-}
-__device__ __forceinline__ bool mbar_try(uint32_t bar, uint32_t parity) {
-  uint32_t ok;
+__device__ __forceinline__ uint32_t elect_one() {
+  uint32_t p = 0;
   asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-      "selp.u32 %0, 1, 0, p;\n\t}\n"
-      : "=r"(ok)
-      : "r"(bar), "r"(parity)
-      : "memory");
-  return ok != 0;
+      "{\n\t.reg .pred P;\n\t.reg .b32 R;\n\telect.sync R|P, 0xffffffff;\n\t"
+      "selp.u32 %0, 1, 0, P;\n\t}\n"
+      : "=r"(p));
+  return p;
 }
-__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, unsigned* status,
-                                          uint64_t limit) {
-  if (mbar_try(bar, parity)) return true;
-  const uint64_t t0 = globaltimer_ns();
-  while (!mbar_try(bar, parity)) {
-    if (globaltimer_ns() - t0 > limit) {
-      report(status, MOE_ERR_TIMEOUT);
-      return false;
-    }
-  }
-  return true;
-}
-__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, int c0, int c1,
-                                            uint32_t bar) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes"
-      " [%0], [%1, {%2, %3}], [%4];" ::"r"(dst),
-      "l"((uint64_t)map), "r"(c0), "r"(c1), "r"(bar)
-      : "memory");
-}
-__device__ __forceinline__ uint64_t desc_sw128(uint32_t addr, uint32_t lbo, uint32_t sbo) {
-  return (uint64_t)((addr >> 4) & 0x3FFFu) | ((uint64_t)((lbo >> 4) & 0x3FFFu) << 16) |
-         ((uint64_t)((sbo >> 4) & 0x3FFFu) << 32) | (1ull << 46) | (2ull << 61);
+__device__ __forceinline__ void cluster_wait() {
+  asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
 }
 __device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&v)[16]) {
   asm volatile(
@@ -121,91 +90,146 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&v)[16]) {
         "=r"(v[14]), "=r"(v[15])
       : "r"(taddr));
 }
-__device__ __forceinline__ uint32_t cluster_rank() {
-  uint32_t r;
-  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
-  return r;
+__device__ __forceinline__ void st_shared_v4(uint32_t addr, float a, float b, float c, float d) {
+  asm volatile("st.shared.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "f"(a), "f"(b), "f"(c),
+               "f"(d)
+               : "memory");
 }
-__device__ __forceinline__ uint32_t cluster_id_x() {
-  uint32_t r;
-  asm volatile("mov.u32 %0, %%clusterid.x;" : "=r"(r));
-  return r;
-}
-__device__ __forceinline__ void cluster_arrive() {
-  asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
-}
-__device__ __forceinline__ void cluster_wait() {
-  asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
-}
-__device__ __forceinline__ void cluster_sync() {
-  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::
-                   : "memory");
-}
-// Address of the same shared-memory location in CTA `rank` of this cluster.
-__device__ __forceinline__ uint32_t map_rank(uint32_t local_addr, uint32_t rank) {
-  uint32_t remote;
-  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(remote) : "r"(local_addr), "r"(rank));
-  return remote;
-}
-__device__ __forceinline__ float ld_dsmem(uint32_t remote_addr) {
+__device__ __forceinline__ float ld_shared_f32(uint32_t addr) {
   float v;
-  asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(remote_addr) : "memory");
+  asm volatile("ld.shared.f32 %0, [%1];" : "=f"(v) : "r"(addr) : "memory");
   return v;
 }
 
-// Top-KM list (KM = 2, 4 or 8 >= K), descending by (value, then lower id); empty slots
-// have id -1. Ids arrive in ascending order, so an existing entry with an equal value stays
-// above the new one (ties go to the lower id, +0 == -0). The top-K is the first K slots.
-// Every index is a compile-time constant, so the list lives in registers.
+// (value, id) order of the selection: a ranks above b when its value is larger, or equal
+// (+0 == -0) with a lower id; an empty slot (id < 0) ranks below everything.
+__device__ __forceinline__ bool ranks_above(float av, int ae, float bv, int be) {
+  if (ae < 0) return false;
+  if (be < 0) return true;
+  return av > bv || (av == bv && ae < be);
+}
+
+// Top-KM list (KM = 2, 4 or 8 >= K), best first, empty slots (id -1) hold -inf. This
+// thread's ids arrive in ascending order, so a value equal to a listed one goes below it
+// (ties to the lower id, +0 == -0): only a strictly larger value moves an entry down. The
+// values shift by min/max (slot j keeps the larger of its own value and the smaller of the
+// slot above and the new value), the ids follow the same comparisons. Compile-time indices
+// only; the common case, a value that does not enter, costs one compare and a branch.
 template <int KM>
 __device__ __forceinline__ void top_insert(float (&bv)[KM], int (&be)[KM], float v, int e) {
-  if (be[KM - 1] >= 0 && !(v > bv[KM - 1])) return;  // does not enter
-  bool above[KM];  // the entry in slot j stays above the new one
+  if (!(v > bv[KM - 1]) && be[KM - 1] >= 0) return;  // does not enter
+  bool gt[KM];  // the new value ranks above the entry in slot j
 #pragma unroll
-  for (int j = 0; j < KM; ++j) above[j] = be[j] >= 0 && !(v > bv[j]);
+  for (int j = 0; j < KM; ++j) gt[j] = be[j] < 0 || v > bv[j];
 #pragma unroll
   for (int j = KM - 1; j >= 1; --j) {
-    if (!above[j]) {
-      if (above[j - 1]) {
-        bv[j] = v;
-        be[j] = e;
-      } else {
-        bv[j] = bv[j - 1];
-        be[j] = be[j - 1];
+    be[j] = gt[j] ? (gt[j - 1] ? be[j - 1] : e) : be[j];
+    bv[j] = gt[j] ? (gt[j - 1] ? bv[j - 1] : v) : bv[j];
+  }
+  if (gt[0]) {
+    be[0] = e;
+    bv[0] = v;
+  }
+}
+
+// Merge this thread's sorted list with that of the lane `mask` away (same token group):
+// c[i] = better of a[i] and b[KM-1-i] holds the KM best of both lists as a bitonic
+// sequence, which log2(KM) half-cleaner stages sort. Both lanes end with the same list.
+template <int KM>
+__device__ __forceinline__ void top_merge(float (&bv)[KM], int (&be)[KM], int mask) {
+  float ov[KM];
+  int oe[KM];
+#pragma unroll
+  for (int j = 0; j < KM; ++j) {
+    ov[j] = __shfl_xor_sync(0xffffffffu, bv[j], mask);
+    oe[j] = __shfl_xor_sync(0xffffffffu, be[j], mask);
+  }
+#pragma unroll
+  for (int j = 0; j < KM; ++j) {
+    if (!ranks_above(bv[j], be[j], ov[KM - 1 - j], oe[KM - 1 - j])) {
+      bv[j] = ov[KM - 1 - j];
+      be[j] = oe[KM - 1 - j];
+    }
+  }
+#pragma unroll
+  for (int h = KM / 2; h >= 1; h /= 2) {
+#pragma unroll
+    for (int j = 0; j < KM; ++j) {
+      if ((j & h) == 0) {
+        if (ranks_above(bv[j + h], be[j + h], bv[j], be[j])) {
+          const float tv = bv[j];
+          const int te = be[j];
+          bv[j] = bv[j + h];
+          be[j] = be[j + h];
+          bv[j + h] = tv;
+          be[j + h] = te;
+        }
       }
     }
   }
-  if (!above[0]) {
-    bv[0] = v;
-    be[0] = e;
+}
+
+// Eight of one token's experts, e = e0 + G j: their partials from every rank (loaded first,
+// S x 8 loads in flight, at addresses clamped into the tile so that no load sits behind a
+// branch), added in rank order, + bias, into the thread's top-K list and plain-softmax sums,
+// and stored as logits. FULL: all eight experts exist (no per-expert checks).
+template <int KM, int S, bool FULL>
+__device__ __forceinline__ void route_batch(float (&bv)[KM], int (&be)[KM], float& mx, float& ssum,
+                                            const uint32_t (&rbase)[S], uint32_t colb, int e0,
+                                            const RouteArgs& g, float* lrow) {
+  const int E = g.E, G = g.G;
+  float pv[S][8];
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    const int e = FULL ? e0 + G * j : min(e0 + G * j, E - 1);
+    const uint32_t off = colb + (uint32_t)(e * g.ps * 4);
+#pragma unroll
+    for (int q = 0; q < S; ++q)
+      pv[q][j] = S > 1 ? ld_dsmem_f32(rbase[q] + off) : ld_shared_f32(rbase[q] + off);
+  }
+  float lv[8];
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    float l = pv[0][j];
+#pragma unroll
+    for (int q = 1; q < S; ++q) l += pv[q][j];
+    const int e = e0 + G * j;
+    if (g.bias != nullptr) l += g.bias[FULL ? e : min(e, E - 1)];
+    lv[j] = l;
+  }
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    const int e = e0 + G * j;
+    if (FULL || e < E) {
+      top_insert<KM>(bv, be, lv[j], e);
+      if (!g.renorm) {
+        if (lv[j] > mx) {
+          ssum = ssum * expf(mx - lv[j]) + 1.f;
+          mx = lv[j];
+        } else {
+          ssum += expf(lv[j] - mx);
+        }
+      }
+    }
+  }
+  if (lrow != nullptr) {
+    if (FULL && G == 1 && g.vec_logits) {  // e = e0 + j: two whole float4 groups
+      *reinterpret_cast<float4*>(lrow + e0) = make_float4(lv[0], lv[1], lv[2], lv[3]);
+      *reinterpret_cast<float4*>(lrow + e0 + 4) = make_float4(lv[4], lv[5], lv[6], lv[7]);
+    } else {
+#pragma unroll
+      for (int j = 0; j < 8; ++j)
+        if (FULL || e0 + G * j < E) lrow[e0 + G * j] = lv[j];
+    }
   }
 }
 
-// Columns c0..c0+15 of this warp's 32 TMEM lanes (zeros when the CTA accumulated nothing).
-__device__ __forceinline__ void tmem_cols16(uint32_t trow, int c0, bool have, float (&lv)[16]) {
-  uint32_t v[16];
-  tmem_ld16(trow + (uint32_t)c0, v);
-  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
-#pragma unroll
-  for (int j = 0; j < 16; ++j) lv[j] = have ? __uint_as_float(v[j]) : 0.f;
-}
-__device__ __forceinline__ uint32_t elect_one() {
-  uint32_t p = 0;
-  asm volatile(
-      "{\n\t.reg .pred P;\n\t.reg .b32 R;\n\telect.sync R|P, 0xffffffff;\n\t"
-      "selp.u32 %0, 1, 0, P;\n\t}\n"
-      : "=r"(p));
-  return p;
-}
-
-template <int N, int KM>  // MMA N = E rounded up to 16; KM >= K, a power of two <= 8
-__global__ void __launch_bounds__(R_THREADS) route_tc_kernel(const __grid_constant__ CUtensorMap tmX,
-                                                             const __grid_constant__ CUtensorMap tmW,
-                                                             const RouteArgs g) {
-  constexpr int NCH = (N + 63) / 64;         // B chunks of 64 experts
-  constexpr uint32_t TCOLS = N <= 32 ? 32 : (N <= 64 ? 64 : (N <= 128 ? 128 : 256));
-  constexpr uint32_t IDESC = (1u << 4) | (1u << 7) | (1u << 10) | (1u << 16) |
-                             ((uint32_t)(N >> 3) << 17) | ((uint32_t)(RBM >> 4) << 24);
+// MT: M tiles of 128 experts (1 or 2); KM >= K, a power of two <= 8; S: CTAs of a cluster
+// splitting d (1, 2, 4 or 8).
+template <int MT, int KM, int S>
+__global__ void __launch_bounds__(R_THREADS, 1)
+    route_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmW,
+                    const RouteArgs g) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* base = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
   uint8_t* ring = base;
@@ -215,15 +239,12 @@ __global__ void __launch_bounds__(R_THREADS) route_tc_kernel(const __grid_consta
   uint64_t* empty = bars + RSTAGES;
   uint64_t* accf = bars + 2 * RSTAGES;
   uint32_t* tmem_slot = (uint32_t*)(bars + 2 * RSTAGES + 1);
-  float* part = (float*)ring;  // after the mainloop: this CTA's partial, [N][128]
+  constexpr uint32_t TCOLS = MT == 1 ? 256 : 512;  // accumulator m at column 256 m
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const uint32_t rank = cluster_rank();
-  const int tile = (int)cluster_id_x();
-  const int S = g.S;
+  const uint32_t rank = S > 1 ? cluster_rank() : 0u;
+  const int tile = S > 1 ? (int)cluster_id_x() : (int)blockIdx.x;
   const int kb0 = (int)(rank * g.kblocks / S), kb1 = (int)((rank + 1) * g.kblocks / S);
-  // Tiles start their k-blocks at different points of the range (and wrap), so that the
-  // CTAs do not all read the same W_r rows from the same L2 lines at the same time.
   const int nkb = kb1 - kb0, rot = nkb > 0 ? tile % nkb : 0;
 
   if (tid == 32) {  // fetch both tensor maps while the barriers are set up
@@ -236,46 +257,27 @@ __global__ void __launch_bounds__(R_THREADS) route_tc_kernel(const __grid_consta
       mbar_init(saddr(&empty[s]), 1);
     }
     mbar_init(saddr(accf), 1);
-    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    mbar_init_fence();
   }
-  if (warp == 1) {
-    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
-                     saddr(tmem_slot)),
-                 "r"(TCOLS)
-                 : "memory");
-    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
-  }
-  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
   __syncthreads();
-  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-  const uint32_t tmem = *tmem_slot;
-  bool ok = true;
   pdl_wait();  // the previous kernel in the stream has completed
   pdl_trigger();
 
-  // Producer (warp 0) and MMA issuer (warp 1) run their loops warp-uniformly: lane 0 waits
-  // on the barrier and broadcasts the outcome, one elected lane issues. A single-lane loop
-  // issued about a third fewer small-N MMAs per cycle (the loop, not the tensor pipe, limits
-  // the rate at N = 16).
+  // The producer starts loading at once; the MMA warp allocates the accumulators meanwhile.
   if (warp == 0) {
     int stage = 0;
     uint32_t phase = 0;
     for (int i = 0; i < nkb; ++i) {
       const int kb = kb0 + (i + rot) % nkb;
       int w = 0;
-      if (lane == 0) w = mbar_wait(saddr(&empty[stage]), phase ^ 1u, g.status, g.limit_ns);
-      if (!__shfl_sync(0xffffffffu, w, 0)) {
-        ok = false;
-        break;
-      }
+      if (lane == 0) w = mbar_wait(saddr(&empty[stage]), phase ^ 1u, nullptr, g.status, g.limit_ns);
+      if (!__shfl_sync(0xffffffffu, w, 0)) break;
       if (elect_one()) {
         const uint32_t fb = saddr(&full[stage]);
         mbar_expect_tx(fb, (uint32_t)g.tx_bytes);
         const uint32_t a = saddr(ring + stage * STAGE);
-        tma_load_2d(a, &tmX, kb * RBK, tile * g.rows, fb);
-#pragma unroll
-        for (int c = 0; c < NCH; ++c)
-          tma_load_2d(a + A_SLOT + c * RB_CHUNK, &tmW, c * 64, kb * RBK, fb);
+        tma_load_2d(a + A_SLOT, &tmX, kb * RBK, tile * g.rows, fb);
+        for (int c = 0; c < g.a_chunks; ++c) tma_load_2d(a + c * RCHUNK, &tmW, c * 64, kb * RBK, fb);
       }
       __syncwarp();
       if (++stage == RSTAGES) {
@@ -284,36 +286,37 @@ __global__ void __launch_bounds__(R_THREADS) route_tc_kernel(const __grid_consta
       }
     }
   } else if (warp == 1) {
+    tmem_alloc<1>(saddr(tmem_slot), TCOLS);
+    tc_fence_before();
+    __syncwarp();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
     // Descriptors of stage 0; a stage (and a 16-wide k step) moves the start-address field,
     // which holds shared-memory byte addresses / 16 (below 2^14, so adding does not carry).
-    const uint64_t ad0 = desc_sw128(saddr(ring), 16, 1024);
-    const uint64_t bd0 = desc_sw128(saddr(ring) + A_SLOT, RB_CHUNK, 1024);
+    // A (MN-major): 64-expert chunks 8 KB apart, 8-row k groups 1 KB apart, a k step = 16
+    // rows = 2 KB. B (K-major): 128-byte rows, 8-row groups 1 KB apart, a k step = 32 bytes.
+    const uint64_t ad0 = desc_sw128(saddr(ring), RCHUNK, 1024);
+    const uint64_t bd0 = desc_sw128(saddr(ring) + A_SLOT, 16, 1024);
+    const uint32_t idesc = (1u << 4) | (1u << 7) | (1u << 10) | (1u << 15) |
+                           ((uint32_t)(g.nmma >> 3) << 17) | ((uint32_t)(128 >> 4) << 24);
     int stage = 0;
     uint32_t phase = 0;
     for (int i = 0; i < nkb; ++i) {
       int w = 0;
-      if (lane == 0) w = mbar_wait(saddr(&full[stage]), phase, g.status, g.limit_ns);
-      if (!__shfl_sync(0xffffffffu, w, 0)) {
-        ok = false;
-        break;
-      }
-      asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+      if (lane == 0) w = mbar_wait(saddr(&full[stage]), phase, nullptr, g.status, g.limit_ns);
+      if (!__shfl_sync(0xffffffffu, w, 0)) break;
+      tc_fence_after();
       if (elect_one()) {
         const uint64_t so = (uint64_t)((stage * STAGE) >> 4);
 #pragma unroll
         for (int kk = 0; kk < RBK / 16; ++kk) {
-          const uint32_t acc = (i | kk) != 0 ? 1u : 0u;
-          asm volatile(
-              "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
-              "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(tmem),
-              "l"(ad0 + so + (uint64_t)(kk * 2)), "l"(bd0 + so + (uint64_t)(kk * 128)),
-              "r"(IDESC), "r"(acc)
-              : "memory");
+#pragma unroll
+          for (int m = 0; m < MT; ++m)
+            tc_mma<1>(tmem + (uint32_t)(256 * m),
+                      ad0 + so + (uint64_t)(m * (2 * RCHUNK >> 4) + kk * 128),
+                      bd0 + so + (uint64_t)(kk * 2), idesc, (i | kk) != 0 ? 1u : 0u);
         }
-        asm volatile(
-            "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
-                saddr(&empty[stage]))
-            : "memory");
+        tc_commit<1>(saddr(&empty[stage]));
       }
       __syncwarp();
       if (++stage == RSTAGES) {
@@ -321,41 +324,70 @@ __global__ void __launch_bounds__(R_THREADS) route_tc_kernel(const __grid_consta
         phase ^= 1u;
       }
     }
-    if (elect_one())
-      asm volatile(
-          "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
-              saddr(accf))
-          : "memory");
+    if (elect_one()) tc_commit<1>(saddr(accf));
   }
   __syncwarp();
-  // every thread: the accumulator of this CTA is complete (bounded)
-  int w_ok = 0;
-  if (lane == 0) w_ok = mbar_wait(saddr(accf), 0, g.status, g.limit_ns);
-  w_ok = __shfl_sync(0xffffffffu, w_ok, 0);
-  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-  const bool have = w_ok && (kb1 > kb0);
-  const int r = warp * 32 + lane;  // token row of this thread inside the tile
-  const uint32_t trow = tmem + ((uint32_t)(warp * 32) << 16);
 
-  if (S > 1) {
-    // Every rank publishes its partial (column-major), then after one cluster barrier each
-    // rank finishes a contiguous share of the tile's rows, one thread per row, adding the S
-    // partials in rank order through distributed shared memory (the same fp32 sum in the
-    // same order whichever rank does it). A rank arrives on the closing barrier as soon as
-    // its remote reads are done and waits on it only before exiting.
+  // ---- the partial tile to shared memory: part[e][t], e < E, t < nmma (row stride ps)
+  int w_ok = 0;
+  if (lane == 0) w_ok = mbar_wait(saddr(accf), 0, nullptr, g.status, g.limit_ns);
+  w_ok = __shfl_sync(0xffffffffu, w_ok, 0);
+  tc_fence_before();
+  __syncthreads();  // the ring is free (every MMA has completed); the TMEM address is set
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const bool have = w_ok && nkb > 0;  // this CTA accumulated a partial
+  const uint32_t part = saddr(ring);
+  {
+    // warp w reads TMEM lanes 32 (w % 4) ...; with one M tile, warps w and w + 4 take
+    // alternate 64-column blocks of the same lanes; four 16-column loads, then one wait
+    const int q = warp & 3;
+    const int m = MT == 1 ? 0 : warp >> 2;
+    const int c_first = MT == 1 ? 64 * (warp >> 2) : 0, c_step = MT == 1 ? 128 : 64;
+    const int e = 128 * m + 32 * q + lane;
+    if (128 * m + 32 * q < g.E) {  // warp-uniform: this warp holds experts
+      const uint32_t trow = tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)(256 * m);
+      for (int c0 = c_first; c0 < g.nmma; c0 += c_step) {
+        uint32_t v[4][16];
 #pragma unroll
-    for (int c0 = 0; c0 < N; c0 += 16) {
-      float lv[16];
-      tmem_cols16(trow, c0, have, lv);
+        for (int h = 0; h < 4; ++h)
+          if (c0 + 16 * h < g.nmma) tmem_ld16(trow + (uint32_t)(c0 + 16 * h), v[h]);
+        tmem_ld_wait();
+        if (e < g.E) {
 #pragma unroll
-      for (int j = 0; j < 16; ++j) part[(c0 + j) * RBM + r] = lv[j];
+          for (int h = 0; h < 4; ++h) {
+            if (c0 + 16 * h < g.nmma) {
+              const uint32_t dst = part + (uint32_t)((e * g.ps + c0 + 16 * h) * 4);
+#pragma unroll
+              for (int j = 0; j < 16; j += 4)
+                st_shared_v4(dst + j * 4, have ? __uint_as_float(v[h][j]) : 0.f,
+                             have ? __uint_as_float(v[h][j + 1]) : 0.f,
+                             have ? __uint_as_float(v[h][j + 2]) : 0.f,
+                             have ? __uint_as_float(v[h][j + 3]) : 0.f);
+            }
+          }
+        }
+      }
     }
-    cluster_sync();
-    const int share = (g.rows + S - 1) / S;
-    const int row = (int)rank * share + tid;
-    const bool mine = tid < share && row < g.rows;
-    const int t = tile * g.rows + row;
-    const int E = g.E, K = g.K;
+  }
+  if (S > 1)
+    cluster_sync();  // every rank's partial is in its shared memory
+  else
+    __syncthreads();
+
+  // ---- this rank's share of the tile's tokens: G threads per token (thread gi owns experts
+  // gi, gi + G, ...), R_THREADS / G tokens a pass
+  const int E = g.E, K = g.K, G = g.G;
+  const int share = (g.rows + S - 1) / S;
+  const int tl = tid / G, gi = tid % G;
+  uint32_t rbase[S];  // the partial tile of each rank, in the cluster's shared window
+#pragma unroll
+  for (int q = 0; q < S; ++q) rbase[q] = S > 1 ? map_rank(part, (uint32_t)q) : part;
+  const bool whole = E % (8 * G) == 0;  // every batch of eight experts is whole
+  for (int p0 = 0; p0 < share; p0 += R_THREADS / G) {
+    const int col = (int)rank * share + p0 + tl;  // token column inside the tile
+    const int t = tile * g.rows + col;
+    const bool mine = p0 + tl < share && col < g.rows && t < g.T;
     float bv[KM];
     int be[KM];
 #pragma unroll
@@ -363,68 +395,38 @@ __global__ void __launch_bounds__(R_THREADS) route_tc_kernel(const __grid_consta
       bv[k] = -INFINITY;
       be[k] = -1;
     }
-    float m = -INFINITY, ssum = 0.f;  // online max / sum of exp for the plain softmax
-    if (mine && t < g.T) {
-      const uint32_t own = saddr(&part[row]);
+    float mx = -INFINITY, ssum = 0.f;  // online max / sum of exp for the plain softmax
+    if (mine) {
+      float* lrow = g.logits_out != nullptr ? g.logits_out + (size_t)t * E : nullptr;
 #pragma unroll 1
-      for (int c0 = 0; c0 < N && c0 < E; c0 += 16) {
-        float lv[16];
-        for (int q0 = 0; q0 < S; q0 += 4) {  // up to four ranks' loads in flight
-          float pv[4][16];
-#pragma unroll
-          for (int qq = 0; qq < 4; ++qq) {
-            if (q0 + qq < S) {
-              const uint32_t rb = map_rank(own + (uint32_t)(c0 * RBM * 4), (uint32_t)(q0 + qq));
-#pragma unroll
-              for (int j = 0; j < 16; ++j) pv[qq][j] = ld_dsmem(rb + (uint32_t)(j * RBM * 4));
-            }
-          }
-#pragma unroll
-          for (int qq = 0; qq < 4; ++qq)
-            if (q0 + qq < S)
-#pragma unroll
-              for (int j = 0; j < 16; ++j) lv[j] = q0 + qq == 0 ? pv[0][j] : lv[j] + pv[qq][j];
-        }
-#pragma unroll
-        for (int j = 0; j < 16; ++j) {
-          const int e = c0 + j;
-          if (e < E) {
-            if (g.bias != nullptr) lv[j] += g.bias[e];
-            top_insert<KM>(bv, be, lv[j], e);
-            if (!g.renorm) {
-              if (lv[j] > m) {
-                ssum = ssum * expf(m - lv[j]) + 1.f;
-                m = lv[j];
-              } else {
-                ssum += expf(lv[j] - m);
-              }
-            }
-          }
-        }
-        if (g.logits_out != nullptr) {  // E is a multiple of 8: whole groups of four
-          float* dst = g.logits_out + (size_t)t * E + c0;
-#pragma unroll
-          for (int j4 = 0; j4 < 4; ++j4) {
-            if (c0 + 4 * j4 < E) {
-              if (g.vec_logits)
-                *reinterpret_cast<float4*>(dst + 4 * j4) =
-                    make_float4(lv[4 * j4], lv[4 * j4 + 1], lv[4 * j4 + 2], lv[4 * j4 + 3]);
-              else
-#pragma unroll
-                for (int u = 0; u < 4; ++u) dst[4 * j4 + u] = lv[4 * j4 + u];
-            }
-          }
+      for (int e0 = gi; e0 < E; e0 += 8 * G) {  // eight of this thread's experts at a time
+        if (whole)
+          route_batch<KM, S, true>(bv, be, mx, ssum, rbase, (uint32_t)(col * 4), e0, g, lrow);
+        else
+          route_batch<KM, S, false>(bv, be, mx, ssum, rbase, (uint32_t)(col * 4), e0, g, lrow);
+      }
+    }
+    // merge the G lists of a token (lanes G tl .. G tl + G - 1 of one warp)
+    for (int h = 1; h < G; h <<= 1) {
+      top_merge<KM>(bv, be, h);
+      if (!g.renorm) {
+        const float om = __shfl_xor_sync(0xffffffffu, mx, h);
+        const float os = __shfl_xor_sync(0xffffffffu, ssum, h);
+        const float nm = fmaxf(mx, om);
+        if (nm != -INFINITY) {
+          ssum = (mx == -INFINITY ? 0.f : ssum * expf(mx - nm)) +
+                 (om == -INFINITY ? 0.f : os * expf(om - nm));
+          mx = nm;
         }
       }
     }
-    cluster_arrive();  // this rank's reads of its peers' partials are done
-    if (mine && t < g.T) {
+    if (mine && gi == 0) {
       const float top = bv[0];
       float den = 0.f;
 #pragma unroll
       for (int k = 0; k < KM; ++k)
         if (k < K) den += expf(bv[k] - top);
-      if (!g.renorm) den = ssum * expf(m - top);
+      if (!g.renorm) den = ssum * expf(mx - top);
 #pragma unroll
       for (int k = 0; k < KM; ++k) {
         if (k < K) {
@@ -433,82 +435,19 @@ __global__ void __launch_bounds__(R_THREADS) route_tc_kernel(const __grid_consta
         }
       }
     }
-    cluster_wait();  // no CTA exits while a peer may still read its partials
-  } else {
-    const int t = tile * g.rows + r;
-    const int E = g.E, K = g.K;
-    // Outputs are staged in this CTA's (idle) ring and written back coalesced: the tile's
-    // logits rows are one contiguous [128, E] block, its ids and weights [128, K] blocks.
-    float* st_l = (float*)ring;                         // [128][E + 1]
-    int32_t* st_i = (int32_t*)(st_l + RBM * (E + 1));   // [128][K]
-    float* st_w = (float*)(st_i + RBM * K);             // [128][K]
-    float bv[KM];
-    int be[KM];
-#pragma unroll
-    for (int k = 0; k < KM; ++k) {
-      bv[k] = -INFINITY;
-      be[k] = -1;
-    }
-    float m = -INFINITY, ssum = 0.f;  // online max / sum of exp for the plain softmax
-    const bool live = warp * 32 < g.rows;  // warp-uniform: this warp holds rows of the tile
-#pragma unroll 1
-    for (int c0 = 0; live && c0 < N; c0 += 16) {
-      float lv[16];
-      tmem_cols16(trow, c0, have, lv);
-#pragma unroll
-      for (int j = 0; j < 16; ++j) {
-        const int e = c0 + j;
-        float l = lv[j];
-        if (e < E) {
-          if (g.bias != nullptr) l += g.bias[e];
-          if (t < g.T) {
-            st_l[r * (E + 1) + e] = l;
-            top_insert<KM>(bv, be, l, e);
-            if (!g.renorm) {
-              if (l > m) {
-                ssum = ssum * expf(m - l) + 1.f;
-                m = l;
-              } else {
-                ssum += expf(l - m);
-              }
-            }
-          }
-        }
-      }
-    }
-    if (live && t < g.T) {
-      const float top = bv[0];
-      float den = 0.f;
-#pragma unroll
-      for (int k = 0; k < KM; ++k)
-        if (k < K) den += expf(bv[k] - top);
-      if (!g.renorm) den = ssum * expf(m - top);
-#pragma unroll
-      for (int k = 0; k < KM; ++k) {
-        if (k < K) {
-          st_i[r * K + k] = be[k];
-          st_w[r * K + k] = expf(bv[k] - top) / den;
-        }
-      }
-    }
-    __syncthreads();
-    const int rows = min(g.rows, g.T - tile * g.rows);
-    const size_t t0 = (size_t)tile * g.rows;
-    if (g.logits_out != nullptr)
-      for (int i = tid; i < rows * E; i += R_THREADS)
-        g.logits_out[t0 * E + i] = st_l[(i / E) * (E + 1) + i % E];
-    for (int i = tid; i < rows * K; i += R_THREADS) {
-      g.topk_ids[t0 * K + i] = st_i[i];
-      g.topk_w[t0 * K + i] = st_w[i];
-    }
   }
-  (void)ok;
-  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+  if (S > 1) {
+    // This rank's reads of its peers' partials are done (their values are in registers): a
+    // relaxed arrive, so that it does not wait for this thread's global stores; then no CTA
+    // exits while a peer may still read its partial.
+    asm volatile("barrier.cluster.arrive.relaxed.aligned;" ::: "memory");
+    cluster_wait();
+  }
+  tc_fence_before();
   __syncthreads();
   if (warp == 1) {
-    asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(TCOLS)
-                 : "memory");
+    tc_fence_after();
+    tmem_dealloc<1>(tmem, TCOLS);
   }
 }
 
@@ -536,107 +475,145 @@ bool make_map_2d(CUtensorMap* m, const void* ptr, uint64_t inner, uint64_t outer
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// Clusters of S CTAs of this kernel that can be resident at once (clusters stay inside one
-// GPC, so this can be below SMs / S); cached per instantiation and S.
-template <typename Kern>
-int active_clusters(Kern kern, int smem, int S) {
-  static int cache[9] = {0};
-  if (S < 1 || S > 8) return 1;
-  if (cache[S] == 0) {
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3((unsigned)S);
-    cfg.blockDim = dim3(R_THREADS);
-    cfg.dynamicSmemBytes = (size_t)smem;
-    cudaLaunchAttribute attr;
-    attr.id = cudaLaunchAttributeClusterDimension;
-    attr.val.clusterDim.x = (unsigned)S;
-    attr.val.clusterDim.y = 1;
-    attr.val.clusterDim.z = 1;
-    cfg.attrs = &attr;
-    cfg.numAttrs = 1;
-    int n = 0;
-    if (cudaOccupancyMaxActiveClusters(&n, kern, &cfg) != cudaSuccess || n < 1) {
-      cudaGetLastError();
-      n = 1;
-    }
-    cache[S] = n;
-  }
-  return cache[S];
-}
-
-// Shared-memory ring for N-wide W_r chunks. own: one tile of `rows` tokens per CTA, x slots
-// of ceil(rows/8) KB and as many stages as fit (the last slot's 128-row MMA read may run
-// 16 KB past its start, so the ring is padded to cover it); otherwise 128-row x slots at
-// route_stages(N) deep. Returns the dynamic shared memory size, or 0 if the epilogue's
-// staging buffers would not fit in the ring.
-int ring_layout(int N, int E, int K, bool own, int rows, RouteArgs& a) {
-  const int nch = (N + 63) / 64;
-  a.a_slot = own ? ((rows + 7) / 8) * 1024 : RA_BYTES;
-  a.stage_bytes = a.a_slot + nch * RB_CHUNK;
-  a.tx_bytes = own ? rows * 128 + nch * RB_CHUNK : a.stage_bytes;
-  auto ring_of = [&](int st) { return max(st * a.stage_bytes, (st - 1) * a.stage_bytes + RA_BYTES); };
-  auto smem_of = [&](int st) { return 1024 + ring_of(st) + (2 * st + 2) * 8; };
-  int st = own ? R_MAX_STAGES : route_stages(N);
-  if (own)
-    while (st > 2 && smem_of(st) > R_SMEM_MAX) --st;
+// Stage layout for `rows` tokens: A slot (16 KB per M tile) then the x tile (nmma rows of
+// 128 B); as many stages as fit, at most R_MAX_STAGES; the partial tile [E][ps] must fit in
+// the ring. Returns the dynamic shared memory size, or 0 if it does not fit.
+int ring_layout(int MT, int E, int rows, RouteArgs& a) {
+  a.nmma = ((rows + 15) / 16) * 16;
+  a.a_chunks = (E + 63) / 64;
+  a.a_slot = MT * 2 * RCHUNK;
+  a.stage_bytes = a.a_slot + a.nmma * 128;
+  a.tx_bytes = a.a_chunks * RCHUNK + rows * 128;
+  a.ps = a.nmma + 4;  // v4 stores of 32 lanes land on 8 distinct bank groups
+  auto smem_of = [&](int st) { return 1024 + st * a.stage_bytes + (2 * st + 2) * 8; };
+  int st = R_MAX_STAGES;
+  while (st > 2 && smem_of(st) > R_SMEM_MAX) --st;
   a.stages = st;
-  a.bar_off = ring_of(st);
-  const int staging = RBM * (E + 1) * 4 + 2 * RBM * K * 4;
-  const int partials = N * RBM * 4;
-  if (smem_of(st) > R_SMEM_MAX || ring_of(st) < staging || ring_of(st) < partials) return 0;
+  a.bar_off = st * a.stage_bytes;
+  if (smem_of(st) > R_SMEM_MAX || E * a.ps * 4 > a.bar_off) return 0;
   return smem_of(st);
 }
 
-template <int N, int KM>
-moe_status launch_nk(const void* x, const void* w_r, RouteArgs a, int tiles, bool own,
-                     cudaStream_t st) {
-  auto kern = route_tc_kernel<N, KM>;
-  int smem = own ? ring_layout(N, a.E, a.K, true, a.rows, a) : 0;
-  if (smem == 0 && own) {  // the ring does not fit: one 128-token tile per CTA, no split
-    own = false;
-    a.rows = RBM;
-    a.S = 1;
-    tiles = (a.T + RBM - 1) / RBM;
+// Clusters of S CTAs of `kern` that can be resident at once (clusters stay inside one GPC,
+// so this can be below SMs / S); cached per device, kernel, S and shared-memory size.
+int active_clusters(const void* kern, int smem, int S) {
+  struct Entry {
+    const void* kern;
+    int dev, S, smem, n;
+  };
+  static std::mutex mu;
+  static Entry cache[64];
+  static int used = 0;
+  int dev = 0;
+  cudaGetDevice(&dev);
+  std::lock_guard<std::mutex> lk(mu);
+  for (int i = 0; i < used; ++i)
+    if (cache[i].kern == kern && cache[i].dev == dev && cache[i].S == S && cache[i].smem == smem)
+      return cache[i].n;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)S);
+  cfg.blockDim = dim3(R_THREADS);
+  cfg.dynamicSmemBytes = (size_t)smem;
+  cudaLaunchAttribute attr;
+  attr.id = cudaLaunchAttributeClusterDimension;
+  attr.val.clusterDim.x = (unsigned)S;
+  attr.val.clusterDim.y = 1;
+  attr.val.clusterDim.z = 1;
+  cfg.attrs = &attr;
+  cfg.numAttrs = 1;
+  int n = 0;
+  if (cudaOccupancyMaxActiveClusters(&n, kern, &cfg) != cudaSuccess || n < 1) {
+    cudaGetLastError();
+    n = 1;
   }
-  if (smem == 0) {  // one tile of up to 128 tokens per cluster of S CTAs
-    smem = ring_layout(N, a.E, a.K, false, RBM, a);
-    if (smem == 0) return MOE_ERR_UNSUPPORTED;
-  }
-  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+  if (used < 64) cache[used++] = Entry{kern, dev, S, smem, n};
+  return n;
+}
+
+template <int MT, int KM, int S>
+const void* kernel_for() {
+  return (const void*)route_tc_kernel<MT, KM, S>;
+}
+
+template <int MT, int KM, int S>
+moe_status launch_cfg(const moe_shape& s, const void* x, const void* w_r, const RouteArgs& a,
+                      int tiles, int smem, cudaStream_t st) {
+  auto kern = route_tc_kernel<MT, KM, S>;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, R_SMEM_MAX) !=
+      cudaSuccess)
     return MOE_ERR_CUDA;
-  // With fewer 128-token tiles than clusters that fit at once, shorter tiles (at least 64
-  // tokens) put more SMs to work; the MMA still computes 128 rows, the surplus unwritten.
-  if (!own && a.S > 1) {
-    const int fit = active_clusters(kern, smem, a.S);
-    const int want = min(fit, (a.T + 63) / 64);
-    if (want > tiles) {
-      a.rows = (a.T + want - 1) / want;
-      tiles = (a.T + a.rows - 1) / a.rows;
-    }
-  }
   CUtensorMap mx, mw;
-  if (!make_map_2d(&mx, x, (uint64_t)(a.kblocks * RBK), (uint64_t)a.T, 64, own ? a.rows : RBM))
+  if (!make_map_2d(&mx, x, (uint64_t)(a.kblocks * RBK), (uint64_t)s.T, 64, (uint32_t)a.rows))
     return MOE_ERR_CUDA;
-  if (!make_map_2d(&mw, w_r, (uint64_t)a.E, (uint64_t)(a.kblocks * RBK), 64, 64)) return MOE_ERR_CUDA;
+  if (!make_map_2d(&mw, w_r, (uint64_t)s.E, (uint64_t)(a.kblocks * RBK), 64, 64))
+    return MOE_ERR_CUDA;
   launch_begin(K_ROUTE_TC, st);
-  launch_kernel(kern, dim3((unsigned)(tiles * a.S)), dim3(R_THREADS), (size_t)smem, st,
-                (unsigned)a.S, mx, mw, a);
+  launch_kernel(kern, dim3((unsigned)(tiles * S)), dim3(R_THREADS), (size_t)smem, st,
+                (unsigned)S, mx, mw, a);
   return launch_end(K_ROUTE_TC, st);
 }
 
-template <int KM>
-moe_status launch_n(int N, const void* x, const void* w_r, const RouteArgs& a, int tiles,
-                    bool own, cudaStream_t st) {
-  if (N <= 16) return launch_nk<16, KM>(x, w_r, a, tiles, own, st);
-  if (N <= 32) return launch_nk<32, KM>(x, w_r, a, tiles, own, st);
-  if (N <= 64) return launch_nk<64, KM>(x, w_r, a, tiles, own, st);
-  if (N <= 128) return launch_nk<128, KM>(x, w_r, a, tiles, own, st);
-  return launch_nk<256, KM>(x, w_r, a, tiles, own, st);
+template <int MT, int KM>
+moe_status launch_mk(const moe_shape& s, const void* x, const void* w_r, RouteArgs a,
+                     cudaStream_t st) {
+  // Tiles of up to 256 tokens (fewer when E * (rows + 4) floats would not fit the ring).
+  int max_rows = 256;
+  RouteArgs probe = a;
+  while (max_rows > 16 && ring_layout(MT, s.E, max_rows, probe) == 0) max_rows -= 16;
+  const int smem_max = ring_layout(MT, s.E, max_rows, probe);
+  if (smem_max == 0) return MOE_ERR_UNSUPPORTED;
+  // Split d over the largest S in {8, 4, 2, 1} (each rank keeping at least two k-blocks)
+  // whose clusters, all resident at once, hold every 256-token tile; then shorten the tiles
+  // so that the resident clusters are all used (at least 16 tokens a tile).
+  const void* kern_s[4] = {kernel_for<MT, KM, 1>(), kernel_for<MT, KM, 2>(),
+                           kernel_for<MT, KM, 4>(), kernel_for<MT, KM, 8>()};
+  const int tiles0 = (s.T + max_rows - 1) / max_rows;
+  int S = 1, fit = sm_count();
+  for (int si = 3; si >= 1; --si) {
+    const int cand = 1 << si;
+    if (2 * cand > a.kblocks) continue;
+    if (cudaFuncSetAttribute(kern_s[si], cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             R_SMEM_MAX) != cudaSuccess)
+      return MOE_ERR_CUDA;
+    const int f = active_clusters(kern_s[si], smem_max, cand);
+    if (f >= tiles0) {
+      S = cand;
+      fit = f;
+      break;
+    }
+  }
+  int tiles = fit;
+  if (tiles < tiles0) tiles = tiles0;
+  if (tiles > (s.T + 15) / 16) tiles = (s.T + 15) / 16;
+  a.rows = (s.T + tiles - 1) / tiles;
+  if (a.rows > max_rows) a.rows = max_rows;
+  tiles = (s.T + a.rows - 1) / a.rows;
+  a.S = S;
+  const int smem = ring_layout(MT, s.E, a.rows, a);
+  if (smem == 0) return MOE_ERR_UNSUPPORTED;
+  // Threads per token: one up to 32 experts, then enough for about 32 experts each (their
+  // top-K lists merged by shuffles).
+  int G = 1;
+  while (G < 8 && 32 * G < s.E) G *= 2;
+  a.G = G;
+  a.vec_logits = G == 1 && ((uintptr_t)a.logits_out & 15) == 0;
+  switch (S) {
+    case 8: return launch_cfg<MT, KM, 8>(s, x, w_r, a, tiles, smem, st);
+    case 4: return launch_cfg<MT, KM, 4>(s, x, w_r, a, tiles, smem, st);
+    case 2: return launch_cfg<MT, KM, 2>(s, x, w_r, a, tiles, smem, st);
+    default: return launch_cfg<MT, KM, 1>(s, x, w_r, a, tiles, smem, st);
+  }
+}
+
+template <int MT>
+moe_status launch_m(const moe_shape& s, const void* x, const void* w_r, const RouteArgs& a,
+                    cudaStream_t st) {
+  if (s.K <= 2) return launch_mk<MT, 2>(s, x, w_r, a, st);
+  if (s.K <= 4) return launch_mk<MT, 4>(s, x, w_r, a, st);
+  return launch_mk<MT, 8>(s, x, w_r, a, st);
 }
 
 }  // namespace
-
-int g_route_layout = 0;
 
 bool route_tc_supported(const moe_shape& s) {
   return s.dtype == MOE_BF16 && s.E % 8 == 0 && s.E <= 256 && s.K <= KMAX && s.d % 64 == 0;
@@ -644,30 +621,7 @@ bool route_tc_supported(const moe_shape& s) {
 
 moe_status launch_route_tc(const moe_shape& s, const void* x, const void* w_r, const float* bias,
                            float* logits_out, int32_t* ids, float* w, cudaStream_t st) {
-  int tiles = (s.T + RBM - 1) / RBM;
-  const int kblocks = s.d / RBK;
-  const int N = ((s.E + 15) / 16) * 16;  // MMA N (a multiple of 16 for M = 128)
-  const int nmma = N <= 16 ? 16 : N <= 32 ? 32 : N <= 64 ? 64 : N <= 128 ? 128 : 256;
-  // On request, one tile of ceil(T / SMs) <= 128 tokens per CTA over the whole of d (no
-  // split, no cluster). Not the default: it issues one M = 128 MMA per 16-wide k step for
-  // fewer useful rows, and the MMA issue loop, not HBM, bounds this kernel.
-  const int rows_own = (s.T + sm_count() - 1) / sm_count();
-  const bool own = g_route_layout == 2 && rows_own <= RBM;
-  int S = 1;
-  if (!own) {
-    // Split d over S CTAs so that about one CTA per SM works, but never beyond the CTAs
-    // that can be resident at once (a second wave costs more than the split saves).
-    const int smem_cta =
-        route_stages(nmma) * (RA_BYTES + ((nmma + 63) / 64) * RB_CHUNK) + 1024 + 256;
-    const int per_sm = R_SMEM_MAX / smem_cta;
-    S = (sm_count() + tiles - 1) / tiles;
-    const int resident = sm_count() * (per_sm > 0 ? per_sm : 1);
-    if (S > resident / tiles) S = resident / tiles;
-    if (S > 8) S = 8;
-    if (S > kblocks) S = kblocks;
-    if (S < 1) S = 1;
-  }
-  RouteArgs a;
+  RouteArgs a = {};
   a.bias = bias;
   a.logits_out = logits_out;
   a.topk_ids = ids;
@@ -676,17 +630,11 @@ moe_status launch_route_tc(const moe_shape& s, const void* x, const void* w_r, c
   a.E = s.E;
   a.K = s.K;
   a.renorm = s.renormalize;
-  a.kblocks = kblocks;
-  a.S = S;
-  a.rows = own ? rows_own : RBM;
-  a.vec_logits = ((uintptr_t)logits_out & 15) == 0;
-  if (own) tiles = (s.T + a.rows - 1) / a.rows;
+  a.kblocks = s.d / RBK;
   a.status = device_status_ptr();
   a.limit_ns = kWaitLimitNs;
-  // instantiations cover N up to the next of 16/32/64/128/256; columns past E read zeros
-  if (s.K <= 2) return launch_n<2>(N, x, w_r, a, tiles, own, st);
-  if (s.K <= 4) return launch_n<4>(N, x, w_r, a, tiles, own, st);
-  return launch_n<8>(N, x, w_r, a, tiles, own, st);
+  if (s.E <= 128) return launch_m<1>(s, x, w_r, a, st);
+  return launch_m<2>(s, x, w_r, a, st);
 }
 
 }  // namespace moe
