@@ -36,7 +36,7 @@ import moe_inputs as mi  # noqa: E402
 
 METRIC = "MoE layer fwd tokens/s at 1 B200; dispatch+combine GB/s and GEMM % of peak"
 PEAKS_FILE = os.path.join(ROOT, "MEASURED_PEAKS.json")
-PROFILES_DIR = os.path.join(ROOT, "profiles")
+RECORDS_FILE = os.path.join(ROOT, "profiles", "records.json")
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 
@@ -55,7 +55,12 @@ def parse():
     ap.add_argument("--ffn-variant", type=int, default=0, choices=[0, 1, 2, 3],
                     help="grouped-GEMM tile variant (moe_shape.ffn_variant): 0 automatic, 1 "
                          "single-CTA, 2 CTA pairs, 3 CTA pairs with the rows gathered first")
-    ap.add_argument("--only", choices=["atomic_experts", "backward"], default=None,
+    ap.add_argument("--no-secondary", action="store_true",
+                    help="only the layer forward, its roofline, dispatch + combine and e2e (no "
+                         "decode, rounding, backward, atomic-expert or other-workload figures)")
+    ap.add_argument("--no-workloads", action="store_true",
+                    help="skip the fine-grained and skewed workload figures")
+    ap.add_argument("--only", choices=["atomic_experts", "backward", "dispatch"], default=None,
                     help="run one secondary figure alone and print it (for profiling)")
     return ap.parse_args()
 
@@ -179,19 +184,18 @@ def kernel_source_hash(kernel: str) -> str:
 
 
 def traffic_for(kernel: str, workload: str):
-    """ncu DRAM bytes per launch for `kernel` from a `bench-record:` line of a profiles/*.md
-    summary, reported only if it was taken on the current kernel source."""
-    import glob
+    """ncu DRAM bytes per launch for `kernel` from profiles/records.json, reported only if the
+    record was taken on the current kernel source."""
+    try:
+        with open(RECORDS_FILE) as f:
+            recs = json.load(f)["records"]
+    except (OSError, ValueError, KeyError):
+        return None
     want = kernel_source_hash(kernel)
-    for path in sorted(glob.glob(os.path.join(PROFILES_DIR, "*.md"))):
-        with open(path) as f:
-            for line in f:
-                if not line.startswith("bench-record:"):
-                    continue
-                kv = dict(item.split("=", 1) for item in line.split()[1:] if "=" in item)
-                if (kv.get("workload") == workload and kv.get("kernel") == kernel
-                        and kv.get("source_hash") == want):
-                    return int(kv["bytes_per_launch"])
+    for r in recs:
+        if r.get("workload") == workload and r.get("kernel") == kernel and \
+                r.get("source_hash") == want:
+            return int(r["bytes_per_launch"])
     return None
 
 
@@ -593,6 +597,68 @@ def backward_figure(tdr, cfg, s, x, w_r, wg, wu, wd, bias, world, peak_t, steps=
                     "kept slot"}
 
 
+def workload_figure(tdr, name, world, peak_t, steps=20):
+    """The layer forward at one of the other bf16 workloads (fine-grained: 128 small uneven
+    experts; skewed: Zipf-biased routing with a capacity limit): `steps` forwards back to back
+    (their weights, 1.2-1.6 GB, stream from HBM every step), CUDA events, per-kernel times from
+    the library's event profiler. Reports the grouped GEMMs against the sustained bf16 peak on
+    algorithmic FLOPs (kept rows only), the share of gate/up tile rows that is padding, and
+    the share of the step spent routing and permuting."""
+    cfg = mi.CONFIGS[name]
+    inp = mi.make_inputs(cfg)
+    dev = torch.device("cuda", torch.cuda.current_device())
+    x, w_r = inp.x.to(dev), inp.w_r.to(dev)
+    wg, wu, wd = inp.w_gate.to(dev), inp.w_up.to(dev), inp.w_down.to(dev)
+    bias = None if inp.bias is None else inp.bias.to(dev)
+    del inp
+    s = tdr.make_shape(cfg.T, cfg.d, cfg.E, cfg.K, cfg.n, cfg.capacity_factor, True,
+                       torch.bfloat16)
+    ws = torch.empty(tdr.forward_workspace_size(s), dtype=torch.uint8, device=dev)
+    out = torch.empty(cfg.T, cfg.d, dtype=torch.bfloat16, device=dev)
+
+    def step():
+        tdr.forward(s, x, w_r, wg, wu, wd, bias=bias, out=out, workspace=ws)
+
+    for _ in range(3):
+        step()
+    torch.cuda.synchronize()
+    prof = tdr.Profiler()
+    with prof:
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(steps):
+            step()
+        e1.record()
+        torch.cuda.synchronize()
+    if tdr.device_status() != 0:
+        raise RuntimeError(f"device status set during the {name} runs")
+    ms = max_over_ranks(e0.elapsed_time(e1) / steps, world)
+    kern = prof.results()
+    offs = tdr.workspace_views(s, ws)["offsets"].cpu().numpy()
+    kept = np.diff(offs)
+    a_kept = int(offs[-1])
+    tile_rows = int(sum(-(-int(c) // 128) * 128 for c in kept))
+
+    def avg(*names):
+        return sum(kern.get(k, (0, 0.0))[1] for k in names) / steps
+
+    g_ms = avg("gateup_tc", "gateup_tc2")
+    d_ms = avg("down_tc", "down_tc2")
+    fg, fd = 4.0 * cfg.d * cfg.n * a_kept, 2.0 * cfg.d * cfg.n * a_kept
+    tg = fg / (g_ms / 1e3) / 1e12 if g_ms > 0 else 0.0
+    td = fd / (d_ms / 1e3) / 1e12 if d_ms > 0 else 0.0
+    rp = avg("route_tc", "route", "permute_small", "permute_cluster", "hist", "scan", "scatter")
+    del x, wg, wu, wd, ws
+    torch.cuda.empty_cache()
+    return {"ms": round(ms, 4), "tok_s": round(cfg.T * world / (ms / 1e3)),
+            "gateup_ms": round(g_ms, 4), "gateup_tflops": round(tg, 1),
+            "gateup_frac": round(tg / peak_t, 4), "down_ms": round(d_ms, 4),
+            "down_tflops": round(td, 1), "down_frac": round(td / peak_t, 4),
+            "kept": a_kept, "pad_share": round(1.0 - a_kept / max(tile_rows, 1), 4),
+            "route_ms": round(avg("route_tc", "route"), 4),
+            "route_permute_share": round(rp / ms, 4), "combine_ms": round(avg("combine"), 4)}
+
+
 # ------------------------------------------------------------------ our arm
 def atomic_experts_bytes(c) -> dict:
     """Algorithmic HBM bytes of one atomic-expert forward (each tensor read or written once)
@@ -695,6 +761,18 @@ def run_ours(args, rank, world, local):
         return
     cfg = mi.CONFIGS[args.workload]
     dt = torch.bfloat16 if cfg.dtype == "bf16" else torch.float32
+    if args.only == "dispatch":  # the dispatch + combine sequence alone (no expert weights)
+        inp = mi.make_inputs(cfg, with_experts=False)
+        dev = torch.device("cuda", torch.cuda.current_device())
+        x, w_r = inp.x.to(dev), inp.w_r.to(dev)
+        bias = None if inp.bias is None else inp.bias.to(dev)
+        s = tdr.make_shape(cfg.T, cfg.d, cfg.E, cfg.K, cfg.n, cfg.capacity_factor, True, dt)
+        with ClockSampler(local) as dc_clocks:
+            dc = dispatch_combine(tdr, s, cfg, x, w_r, bias, args.steps, world, load_peaks()[0])
+        dc["clocks"] = dc_clocks.summary()
+        if rank == 0:
+            print(json.dumps({"dispatch_combine": dc}), flush=True)
+        return
     inp = mi.make_inputs(cfg)
     dev = torch.device("cuda", torch.cuda.current_device())
     x = inp.x.to(dev)
@@ -718,6 +796,15 @@ def run_ours(args, rank, world, local):
         if rank == 0:
             print(json.dumps({"backward_act": fig}), flush=True)
         return
+
+    # ---- dispatch + combine byte stream at the layer's shape (route, permute with the
+    # gathered rows materialised, combine of those rows as identity experts): measured first,
+    # on its own, before the GEMM-bound steps heat the GPU into its power cap, with its own
+    # clock record
+    peaks = load_peaks()[0]
+    with ClockSampler(local) as dc_clocks:
+        dc = dispatch_combine(tdr, s, cfg, x, w_r, bias, args.steps, world, peaks)
+    dc["clocks"] = dc_clocks.summary()
 
     for _ in range(max(3, args.warmup)):
         step()
@@ -768,10 +855,8 @@ def run_ours(args, rank, world, local):
     roofline = {"bound": "tensor", "kernel": g_name, "achieved": round(ach_g, 2),
                 "peak": peak_t, "unit": "TFLOP/s", "frac": round(ach_g / peak_t, 4),
                 "traffic": traffic_for(g_name, cfg.name),
-                "peak_source": f"{peak_src} bf16_tflops_sustained (kernel timed inside a long "
-                               "step loop)",
-                "algorithmic": "4*d*n*A_kept FLOP per launch (gate and up GEMMs)",
-                "avg_launch_ms": round(avg_g, 4)}
+                "peak_source": f"{peak_src} sustained bf16",
+                "flop_per_launch": flops_gateup, "avg_launch_ms": round(avg_g, 4)}
 
     # ---- end to end through the public API with host buffers: every step uploads its input
     # from pinned host memory and downloads its output. Uploads and downloads run on their
@@ -818,54 +903,102 @@ def run_ours(args, rank, world, local):
     e2e_ms = max_over_ranks(e0.elapsed_time(e1), world)
     assert torch.equal(out_host[(e2e_steps - 1) % 2], out.cpu()), "e2e output differs"
     elem = 2 if dt == torch.bfloat16 else 4
-    e2e = {"value": cfg.T * world * e2e_steps / (e2e_ms / 1e3), "unit": "tokens/s",
+    # public API (token_dispatch_router_b200.forward); pinned host input uploaded and output
+    # downloaded every step on separate streams, double-buffered
+    e2e = {"value": round(cfg.T * world * e2e_steps / (e2e_ms / 1e3), 1), "unit": "tokens/s",
            "h2d_bytes_per_step": cfg.T * cfg.d * elem, "d2h_bytes_per_step": cfg.T * cfg.d * elem,
-           "steps": e2e_steps,
-           "how": "public API (token_dispatch_router_b200.forward); pinned host input uploaded "
-                  "and output downloaded every step on separate streams, double-buffered"}
+           "steps": e2e_steps}
 
     # ---- dispatch + combine byte stream at the same shape (route, permute with the gathered
     # rows materialised, combine of those rows as identity experts): the unfused traffic
-    dc = dispatch_combine(tdr, s, cfg, x, w_r, bias, args.steps, world, peaks)
-    dd = decode_dispatch(tdr, world)
-    tr = token_rounding_figure(tdr, cfg, x, w_r, wg, wu, wd, bias, world)
-    bw = backward_figure(tdr, cfg, s, x, w_r, wg, wu, wd, bias, world, peak_t)
-    ae = atomic_experts_figure(tdr, world, peaks)
+    dd = tr = bw = ae = None
+    if not args.no_secondary:
+        dd = decode_dispatch(tdr, world)
+        tr = token_rounding_figure(tdr, cfg, x, w_r, wg, wu, wd, bias, world)
+        bw = backward_figure(tdr, cfg, s, x, w_r, wg, wu, wd, bias, world, peak_t)
+        ae = atomic_experts_figure(tdr, world, peaks)
+
+    wl = {}
+    if cfg.name == "mixtral_bf16" and not (args.no_workloads or args.no_secondary):
+        for other in ("fine_grained_bf16", "skewed_capacity_bf16"):
+            wl[other] = workload_figure(tdr, other, world, peak_t)
 
     weights_gb = 3 * cfg.E * cfg.d * cfg.n * (2 if dt == torch.bfloat16 else 4) / 1e9
-    # ---- per-kernel breakdown (ms per step) and the two secondary figures of the metric
     per_kernel = {k: round(ms / args.steps, 4) for k, (n, ms) in kern.items()}
-    gemm = {"achieved_tflops": round(ach_gemm, 2), "frac": round(ach_gemm / peak_t, 4),
-            "gateup_tflops": round(ach_g, 2), "down_tflops": round(ach_d, 2)}
+    # One compact JSON line (no spaces, short keys, no prose): the driver keeps the last few
+    # thousand characters of the output, so the headline figures come last.
     result = {
-        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
-        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
+        "metric": METRIC, "value": round(value, 1), "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_step, 5),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16"
         if dt == torch.bfloat16 else "f32", "data": "synthetic",
         "config": {"workload": cfg.name, "T": cfg.T, "d": cfg.d, "E": cfg.E, "K": cfg.K,
                    "n": cfg.n, "global_batch": cfg.T * world, "parallelism": f"replicas{world}",
                    "ffn_variant": args.ffn_variant,
-                   "l2": f"inputs larger than L2: the {weights_gb:.2f} GB of expert weights "
-                         "stream every step"},
-        "roofline": roofline, "gemm": gemm, "dispatch_combine": dc, "decode_dispatch": dd,
-        "token_rounding": tr, "backward_act": bw, "atomic_experts": ae,
-        "kernel_ms_per_step": per_kernel,
-        "gpu_launches": int(launches), "e2e": e2e,
+                   "l2": f"{weights_gb:.2f} GB of weights stream each step (> L2)"},
     }
-    result["clocks"] = clocks.summary()
-
+    if bw:
+        result["backward"] = {"ms": bw["ms_per_call"], "dact_ms": bw["dact_gemm_ms"],
+                              "dact_frac": bw["dact_frac_of_sustained_peak"],
+                              "dx_ms": bw["dx_gemm_ms"], "dx_frac": bw["dx_frac_of_sustained_peak"],
+                              "router_ms": round(sum(bw["router_ms"].values()), 4)}
+    if ae:
+        ku = ae["kernels_us"]
+        result["atomic_experts"] = {"workload": ae["workload"], "ms": ae["ms"],
+                                    "tok_s": round(ae["tokens_per_s"]), "hbm_frac": ae["hbm_frac"],
+                                    "topk_us": ku.get("omni_topk"), "act_us": ku.get("omni_act"),
+                                    "out_us": ku.get("omni_out"),
+                                    "scatter_out_us": ae["scatter_add_output"]["output_us"]}
+    if tr:
+        result["token_rounding"] = {"R": tr["R"], "plain_ms": tr["plain"]["ms_per_step"],
+                                    "rounded_ms": tr["rounded"]["ms_per_step"],
+                                    "speedup": tr["speedup"], "kept_share": tr["kept_share"]}
+    if dd:
+        result["decode_dispatch_us"] = {"cols": "two_calls,moe_dispatch",
+                                        **{k.split("=")[1]: [v["two_calls_us"],
+                                                             v["moe_dispatch_us"]]
+                                           for k, v in dd["latency"].items()}}
     # ---- CPU oracle baseline (rank 0, N = 1 only)
+    cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         ntok = args.cpu_tokens if args.cpu_tokens > 0 else cfg.T
         v_cpu, dt_cpu, wide = cpu_oracle_tokens_per_s(inp, ntok)
-        result["cpu_baseline"] = {
-            "value": v_cpu, "unit": "tokens/s", "cores": cpu_cores(), "kind": "oracle",
-            "sample": f"{ntok} tokens through the whole layer (oracle numpy fp64, "
-                      f"{dt_cpu:.1f} s; expert weights widened to fp64 outside the timing)"}
-        if cfg.dtype == "bf16":
-            result["cpu_oracle_figures"] = cpu_oracle_figures(inp, wide)
+        cpu = {"value": round(v_cpu, 1), "unit": "tokens/s", "cores": cpu_cores(),
+               "kind": "oracle",
+               "sample": f"{ntok} tokens, whole layer, numpy fp64, {dt_cpu:.1f} s"}
+        if cfg.dtype == "bf16" and not args.no_secondary:
+            cf = cpu_oracle_figures(inp, wide)
+            result["cpu_oracle_figures"] = {
+                "token_rounding_tok_s": round(cf["token_rounding"]["tokens_per_s"], 1)
+                if "token_rounding" in cf else None,
+                "backward_tok_s": round(cf["backward_act"]["tokens_per_s"], 1),
+                "decode_us": cf["decode_dispatch"]["us"],
+                "atomic_tok_s": round(cf["atomic_experts"]["tokens_per_s"], 1)}
+    result["kernel_ms_per_step"] = per_kernel
+    if wl:
+        result["workloads"] = wl
+    result["gemm"] = {"tflops": round(ach_gemm, 1), "frac": round(ach_gemm / peak_t, 4),
+                      "gateup_tflops": round(ach_g, 1), "gateup_frac": round(ach_g / peak_t, 4),
+                      "down_tflops": round(ach_d, 1), "down_frac": round(ach_d / peak_t, 4)}
+    kd = dc["kernels_ms_with_events"]
+    result["dispatch_combine"] = {"bytes": dc["bytes"], "ms": dc["ms"],
+                                  "gbs": dc["achieved_gbs"], "frac": dc["frac"],
+                                  "peak_gbs": dc["peak_gbs"], "ms_warm": dc["ms_back_to_back"],
+                                  "route_ms": kd.get("route_tc", kd.get("route")),
+                                  "permute_ms": round(sum(v for k, v in kd.items() if k in (
+                                      "permute_small", "permute_cluster", "hist", "scan",
+                                      "scatter")), 4),
+                                  "gather_ms": kd.get("gather_rows"), "combine_ms": kd.get("combine"),
+                                  "sm_mhz": dc["clocks"]["sm_mhz"],
+                                  "clock_reasons": dc["clocks"]["reasons"]}
+    result["roofline"] = roofline
+    result["e2e"] = e2e
+    result["clocks"] = clocks.summary()
+    if cpu is not None:
+        result["cpu_baseline"] = cpu
+    result["gpu_launches"] = int(launches)
     if rank == 0:
-        print(json.dumps(result), flush=True)
+        print(json.dumps(result, separators=(",", ":")), flush=True)
 
 
 def main():

@@ -165,20 +165,24 @@ moe_status moe_permute(const moe_shape* shape, const int32_t* topk_ids, int32_t*
  * library holds until the process exits. It allocates nothing and calls no allocating
  * routine. Results are identical to moe_permute.
  *  - Limit: needs 2 * ceil(T*K / 1024) * E * 4 bytes of scratch (= moe_permute_workspace_size
- *    minus its 256-byte slack); larger problems return MOE_ERR_UNSUPPORTED and enqueue
- *    nothing. With the default 1 MiB: T*K up to about 0.5 million assignments at E = 256,
- *    2 million at E = 64.
+ *    minus its 256-byte slack) when T*K > 32768; smaller problems run in one CTA or one
+ *    cluster and use none of it. Problems beyond the limit return MOE_ERR_UNSUPPORTED and
+ *    enqueue nothing. With the 1 MiB array: T*K up to about 0.5 million assignments at
+ *    E = 256, 2 million at E = 64.
  *  - Set-up: the first call on each device (with that device current) resolves the array's
- *    device address with cudaGetSymbolAddress; make that first call before any stream
- *    capture.
+ *    device address with cudaGetSymbolAddress. That call, or any earlier call into the
+ *    library on the device, may also be when the CUDA driver loads the library's module
+ *    and places the array in device memory (lazy module loading), which can allocate and
+ *    synchronise. So make the first call on each device at start-up, before any stream
+ *    capture and before the allocation-free part of the program. The resolved address is
+ *    kept for the life of the process; after cudaDeviceReset on a device it is stale and
+ *    the library must not be used on that device again.
  *  - Sharing: every call uses the same array, which keeps the last call's contents (the
  *    kernels overwrite every entry they read, so nothing must start at zero). Calls whose
  *    kernels overlap on the GPU (other streams, other host threads) race on it: serialise
  *    them.
  */
-#ifndef MOE_PERMUTE_STATIC_SCRATCH_BYTES
-#define MOE_PERMUTE_STATIC_SCRATCH_BYTES (1u << 20)
-#endif
+#define MOE_PERMUTE_STATIC_SCRATCH_BYTES (1u << 20) /* fixed when the library is built */
 moe_status moe_permute_static(const moe_shape* shape, const int32_t* topk_ids, int32_t* counts,
                               int32_t* offsets, int32_t* assign_to_perm, int32_t* perm_to_assign,
                               const void* x, void* x_perm, moe_stream_t stream);

@@ -254,6 +254,29 @@ def grouped_ffn(x, perm_to_assign, offsets, K: int, w_gate, w_up, w_down):
     return a_act, y_perm
 
 
+def grouped_ffn_rows(slots, x, perm_to_assign, offsets, K: int, w_gate, w_up, w_down):
+    """grouped_ffn for chosen expert-major slots only (the sampled full-size check): row p of
+    a_act and y_perm, with p's expert found from offsets and its token perm_to_assign[p] // K.
+    The slots of one expert run together, so each expert's weights are widened once.
+    Returns (a_rows, y_rows) in the order of `slots`, fp64."""
+    slots = np.asarray(slots, dtype=np.int64)
+    off = np.asarray(offsets, dtype=np.int64)
+    n = w_gate.shape[2]
+    d = w_down.shape[2]
+    a_rows = np.zeros((slots.size, n), dtype=F64)
+    y_rows = np.zeros((slots.size, d), dtype=F64)
+    by_expert = {}
+    for i, p in enumerate(slots):
+        by_expert.setdefault(expert_of_slot(off, int(p)), []).append(i)
+    for e, idx in by_expert.items():
+        tok = np.asarray(perm_to_assign, dtype=np.int64)[slots[idx]] // K
+        xr = as_f64(x[tok])
+        a = swiglu(xr @ as_f64(w_gate[e]), xr @ as_f64(w_up[e]))
+        a_rows[idx] = a
+        y_rows[idx] = a @ as_f64(w_down[e])
+    return a_rows, y_rows
+
+
 def gate_up_preact(x, perm_to_assign, offsets, K: int, w_gate, w_up):
     """[P5] 3 item 3: the pre-activations of the kept slots, g[p] = x[tok(p)] W_gate[e] and
     u[p] = x[tok(p)] W_up[e] (fp64), which the backward below reads."""

@@ -298,6 +298,24 @@ def test_layer_with_capacity_equals_dense_with_dropped_gates_zeroed():
     np.testing.assert_allclose(res["out"], dense, rtol=1e-12, atol=1e-12)
 
 
+def test_grouped_ffn_rows_are_rows_of_grouped_ffn():
+    """The chosen-slot form returns exactly the rows the whole grouped FFN computes (same
+    slots, any order, slots of several experts mixed), on a small routed problem."""
+    g = np.random.default_rng(3)
+    T, d, n, E, K = 40, 16, 24, 5, 2
+    bf = lambda a: torch.from_numpy(a.astype(np.float32)).to(torch.bfloat16)  # noqa: E731
+    x = bf(g.standard_normal((T, d)))  # bf16 tensors, as the workloads hold them
+    wg, wu, wd = (bf(g.standard_normal((E, d, n))), bf(g.standard_normal((E, d, n))),
+                  bf(g.standard_normal((E, n, d))))
+    ids, _ = orc.route(g.standard_normal((T, E)).astype(np.float32), K)
+    _, offsets, _, p2a = orc.permute(ids, E, orc.capacity(1.2, T, K, E))
+    a_all, y_all = orc.grouped_ffn(x, p2a, offsets, K, wg, wu, wd)
+    slots = g.permutation(int(offsets[-1]))[:30]
+    a_rows, y_rows = orc.grouped_ffn_rows(slots, x, p2a, offsets, K, wg, wu, wd)
+    np.testing.assert_allclose(a_rows, a_all[slots], rtol=1e-13, atol=1e-13)
+    np.testing.assert_allclose(y_rows, y_all[slots], rtol=1e-13, atol=1e-12)
+
+
 def test_identity_experts_give_back_x():
     """Dispatch/combine-only workload: identity experts, sum of weights 1 => out = x."""
     cfg = mi.DISPATCH_COMBINE.with_T(64)

@@ -1,9 +1,13 @@
-"""moe_permute_static: the permute entry point for callers that may not allocate device
-memory while they run (its scratch is a fixed device array inside the library, not a
-caller workspace). Called through the C ABI and checked against moe_permute, the
-workspace entry point, on two calls in a row; the second call is smaller than the first,
-so stale contents of the shared array would show up as a mismatch. This file sorts last
-so that a run stopping at the first failure has already run every other test."""
+"""moe_permute_static: the permute entry point for callers that may not allocate device memory
+while they run (a serving engine whose memory plan is fixed at start-up, an embedded runtime
+with a fixed arena): its scratch is a fixed device array inside the library, not a caller
+workspace. Called through the C ABI and checked against moe_permute, the workspace entry
+point, on calls in a row that all take the chunked path whose histogram, scan and scatter
+kernels keep per-chunk counts and rank bases in that array (more than 32768 assignments, and
+more than 8192 chunk-experts, so the scan is not fused into the scatter). The second call is
+smaller than the first, so entries the first call left behind would show up as a mismatch if
+any kernel read one it had not written. This file sorts last so that a run stopping at the
+first failure has already run every other test."""
 import ctypes
 
 import numpy as np
@@ -11,6 +15,8 @@ import pytest
 import torch
 
 pytestmark = pytest.mark.gpu
+
+LIMIT = 1 << 20  # MOE_PERMUTE_STATIC_SCRATCH_BYTES
 
 
 def _ids(rng, T, E, K):
@@ -29,11 +35,16 @@ def _call_static(tdr, shape, ids, x, x_perm, outs):
         ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
 
 
-@pytest.mark.parametrize("calls", [[(20000, 64, 6, 0.0, 256), (3001, 32, 4, 1.1, 128)]])
+@pytest.mark.parametrize("calls", [[(40000, 256, 8, 0.0, 128), (10000, 128, 8, 1.1, 64),
+                                    (12000, 128, 6, 0.0, 64)]])
 def test_static_scratch_permute_matches_workspace_permute(cuda_lib, calls):
     tdr = cuda_lib
     rng = np.random.default_rng(77)
-    for T, E, K, cf, d in calls:  # two calls in a row, the second smaller
+    for T, E, K, cf, d in calls:  # calls in a row, each smaller than the one before
+        A = T * K
+        chunks = -(-A // 1024)
+        assert A > 32768 and chunks * E > 8192  # the unfused chunked path
+        assert 2 * chunks * E * 4 <= LIMIT
         ids = _ids(rng, T, E, K).cuda()
         x = torch.randn(T, d).to(torch.bfloat16).cuda()
         s = tdr.make_shape(T, d, E, K, 64, cf, True, torch.bfloat16)

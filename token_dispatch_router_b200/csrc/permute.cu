@@ -1033,10 +1033,13 @@ moe_status launch_permute_rounded(const moe_shape& s, const int32_t* ids, const 
 // embedded runtime with a fixed arena, or code that runs where cudaMalloc would synchronise
 // the device. Their permute scratch lives in this file-scope device array instead of a
 // caller workspace. Every GPU that loads the library holds it until the process exits.
-// All calls share it and it keeps the last call's contents; the histogram kernel writes
-// every per-chunk count and the scan kernel every rank base before either is read, so
-// nothing in it has to start at zero. Calls whose kernels overlap on the GPU (different
-// streams, or several host threads) race on it and must be serialised by the caller.
+// All calls share it and it keeps the last call's contents. Problems of up to kClusterMax
+// assignments (one CTA or one cluster) use none of it; larger ones use the per-chunk
+// counts, written by the histogram kernel before the scan or the scatter reads them, and,
+// when the scan is not fused into the scatter, the rank bases, written by the scan kernel
+// before the scatter reads them: nothing in it has to start at zero. Calls whose kernels
+// overlap on the GPU (different streams, or several host threads) race on it and must be
+// serialised by the caller.
 static __device__ __align__(256) unsigned char g_permute_static_scratch[kPermuteStaticScratchBytes];
 
 namespace {
@@ -1045,7 +1048,8 @@ void* g_static_ptr[64];  // device address of the array, per device
 }  // namespace
 
 // Device address of the static scratch on the current device. The first call on a device
-// resolves it with cudaGetSymbolAddress (with that device current); later calls reuse it.
+// resolves it with cudaGetSymbolAddress (with that device current); later calls reuse it
+// (it stays valid until the device is reset, which the library does not support).
 static moe_status static_scratch_ptr(void** out) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return MOE_ERR_CUDA;
