@@ -60,7 +60,8 @@ def parse():
                          "decode, rounding, backward, atomic-expert or other-workload figures)")
     ap.add_argument("--no-workloads", action="store_true",
                     help="skip the fine-grained and skewed workload figures")
-    ap.add_argument("--only", choices=["atomic_experts", "backward", "dispatch"], default=None,
+    ap.add_argument("--only", choices=["atomic_experts", "backward", "dispatch", "decode"],
+                    default=None,
                     help="run one secondary figure alone and print it (for profiling)")
     return ap.parse_args()
 
@@ -441,7 +442,9 @@ def decode_dispatch(tdr, world, Ts=(64, 256, 512, 1024)):
         cfg = base.with_T(T)
         inp = mi.make_inputs(cfg)
         x, lg = inp.x.to(dev), inp.logits.to(dev)
-        s = tdr.make_shape(T, cfg.d, cfg.E, cfg.K, 64, 0.0, True, torch.bfloat16)
+        shapes = {f: tdr.make_shape(T, cfg.d, cfg.E, cfg.K, 64, 0.0, True, torch.bfloat16,
+                                    route_topk=f) for f in (1, 2)}
+        s = shapes[1]
         pws = torch.empty(max(tdr.permute_workspace_size(s), 256), dtype=torch.uint8, device=dev)
         out = torch.empty(T, cfg.d, dtype=x.dtype, device=dev)
         bufs = {}
@@ -451,33 +454,42 @@ def decode_dispatch(tdr, world, Ts=(64, 256, 512, 1024)):
             p = tdr.permute(s, ids, x=x, materialize=True, workspace=pws)
             tdr.combine(s, p["x_perm"], p["assign_to_perm"], w, out=out)
 
-        def one_call():
-            r = tdr.dispatch(s, x=x, logits_in=lg, materialize=True, workspace=pws, out=bufs)
-            bufs.update(r)
-            tdr.combine(s, r["x_perm"], r["assign_to_perm"], r["topk_w"], out=out)
+        def one_call(form):
+            def fn():
+                r = tdr.dispatch(shapes[form], x=x, logits_in=lg, materialize=True,
+                                 workspace=pws, out=bufs)
+                bufs.update(r)
+                tdr.combine(s, r["x_perm"], r["assign_to_perm"], r["topk_w"], out=out)
+            return fn
 
-        row = {}
-        for name, fn in (("two_calls_us", two_calls), ("moe_dispatch_us", one_call)):
+        variants = (("two_calls_us", two_calls), ("dispatch_rounds_us", one_call(1)),
+                    ("dispatch_bitonic_us", one_call(2)))
+        for _, fn in variants:
             for _ in range(3):
                 fn()
-            torch.cuda.synchronize()
-            n = 50
-            ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-                  for _ in range(n)]
-            for a, b in ev:
-                flush.sum()
-                hold_gpu()
-                a.record()
-                fn()
-                b.record()
-            torch.cuda.synchronize()
-            row[name] = round(1e3 * max_over_ranks(sum(a.elapsed_time(b) for a, b in ev) / n,
-                                                   world), 2)
+        torch.cuda.synchronize()
+        # blocks of 10 flushed sequences, the variants interleaved block by block (the clock
+        # drifts), the median of every variant's sequences
+        times = {name: [] for name, _ in variants}
+        for _ in range(5):
+            for name, fn in variants:
+                ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                      for _ in range(10)]
+                for a, b in ev:
+                    flush.sum()
+                    hold_gpu()
+                    a.record()
+                    fn()
+                    b.record()
+                torch.cuda.synchronize()
+                times[name] += [a.elapsed_time(b) for a, b in ev]
+        row = {name: round(1e3 * max_over_ranks(statistics.median(v), world), 2)
+               for name, v in times.items()}
         res[f"T={T}"] = row
     del flush
-    return {"workload": "dispatch_combine (E=64 K=6 d=4096 bf16, given logits)", "latency": res,
-            "note": "route + permute with x_perm + combine, one sequence per L2-flushed "
-                    "iteration, CUDA events, launch gaps included"}
+    # route + permute with x_perm + combine, one sequence per L2-flushed iteration, CUDA
+    # events, launch gaps included; moe_dispatch with either top-K form of its one launch
+    return {"workload": "dispatch_combine (E=64 K=6 d=4096 bf16, given logits)", "latency": res}
 
 
 def token_rounding_figure(tdr, cfg, x, w_r, wg, wu, wd, bias, world, R=128, rounds=5, per=10):
@@ -761,6 +773,17 @@ def run_ours(args, rank, world, local):
         return
     cfg = mi.CONFIGS[args.workload]
     dt = torch.bfloat16 if cfg.dtype == "bf16" else torch.float32
+    if args.only == "decode":  # the decode-regime dispatch latencies alone
+        a = torch.randn(4096, 4096, device="cuda", dtype=torch.bfloat16)
+        t_end = time.time() + 0.5  # bring the clocks up first
+        while time.time() < t_end:
+            a @ a
+        torch.cuda.synchronize()
+        del a
+        dd = decode_dispatch(tdr, world)
+        if rank == 0:
+            print(json.dumps({"decode_dispatch": dd}), flush=True)
+        return
     if args.only == "dispatch":  # the dispatch + combine sequence alone (no expert weights)
         inp = mi.make_inputs(cfg, with_experts=False)
         dev = torch.device("cuda", torch.cuda.current_device())
@@ -954,9 +977,10 @@ def run_ours(args, rank, world, local):
                                     "rounded_ms": tr["rounded"]["ms_per_step"],
                                     "speedup": tr["speedup"], "kept_share": tr["kept_share"]}
     if dd:
-        result["decode_dispatch_us"] = {"cols": "two_calls,moe_dispatch",
+        result["decode_dispatch_us"] = {"cols": "two_calls,dispatch_rounds,dispatch_bitonic",
                                         **{k.split("=")[1]: [v["two_calls_us"],
-                                                             v["moe_dispatch_us"]]
+                                                             v["dispatch_rounds_us"],
+                                                             v["dispatch_bitonic_us"]]
                                            for k, v in dd["latency"].items()}}
     # ---- CPU oracle baseline (rank 0, N = 1 only)
     cpu = None

@@ -86,6 +86,16 @@ typedef struct {
                         * by one gather kernel. All compute the same result; other values
                         * return MOE_ERR_INVALID_ARG. A per-call field: calls on different
                         * streams or threads may choose differently. */
+  int32_t route_topk;  /* top-K form of the warp-per-token routers (fp32 x, given logits, the
+                        * one-launch route + permute of moe_dispatch), a per-call field:
+                        * 0 = automatic (currently form 1, measured faster), 1 = K rounds of a
+                        * warp arg-max, 2 = bitonic merges ("How AI chips support MoE",
+                        * chapter 4, section 4.3: a bitonic network for few experts): lane l
+                        * holds experts l and l + 32 as a sorted pair and five shuffle merges
+                        * give every lane the token's top-K; applies for E <= 64 and K <= 8,
+                        * otherwise form 1 runs. Both give the same ids and weights. The bf16
+                        * tensor-core router keeps its per-thread insertion lists. Other values
+                        * return MOE_ERR_INVALID_ARG. */
 } moe_shape;
 
 /* ----------------------------------------------------------------------------

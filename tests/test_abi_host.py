@@ -221,3 +221,10 @@ def test_no_process_wide_switches_exported(lib):
     for name in ("moe_set_ffn_variant", "moe_get_ffn_variant", "moe_set_route_layout",
                  "moe_get_route_layout", "moe_omni_set_output_mode", "moe_omni_get_output_mode"):
         assert not hasattr(lib, name), name
+
+
+@pytest.mark.parametrize("form,ok", [(0, True), (1, True), (2, True), (3, False)])
+def test_route_topk_is_a_checked_shape_field(lib, form, ok):
+    """The top-K form of the warp-per-token routers is a per-call shape field."""
+    s = tdr.make_shape(64, 128, 8, 2, 128, 0.0, True, torch.bfloat16, route_topk=form)
+    assert (lib.moe_forward_workspace_size(ctypes.byref(s)) > 0) == ok

@@ -77,6 +77,13 @@ def ffn_variant(request):
     return request.param
 
 
+@pytest.fixture(params=[1, 2], ids=["topk_rounds", "topk_bitonic"])
+def route_topk(request):
+    """Run a warp-per-token routing test with K rounds of a warp arg-max and with the bitonic
+    merges (the shape's route_topk; the bitonic form applies for E <= 64 and K <= 8)."""
+    return request.param
+
+
 def inputs_for(cfg):
     if cfg.name not in _INPUTS:
         _INPUTS.clear()  # keep one large workload in host memory at a time
@@ -135,14 +142,15 @@ def test_route_matches_oracle(cuda_lib, T, d, E, K, dtype, bias, renorm):
     assert_status_ok(tdr)
 
 
-def test_route_ties_go_to_lower_id(cuda_lib):
+@pytest.mark.parametrize("E,K", [(64, 6), (40, 8), (32, 2), (128, 4)])
+def test_route_ties_go_to_lower_id(cuda_lib, route_topk, E, K):
     tdr = cuda_lib
     g = np.random.default_rng(5)
-    T, E, K = 777, 64, 6
+    T = 777
     lg = g.integers(-2, 3, size=(T, E)).astype(np.float32)  # heavy ties
     lg[0] = 0.0
     lg[1, ::2] = -0.0  # signed zeros tie with +0
-    s = tdr.make_shape(T, 64, E, K, 64, 0.0, True, torch.bfloat16)
+    s = tdr.make_shape(T, 64, E, K, 64, 0.0, True, torch.bfloat16, route_topk=route_topk)
     ids, w, lo = tdr.route(s, logits_in=torch.from_numpy(lg).cuda(),
                            logits_out=torch.empty(T, E, device="cuda"))
     np.testing.assert_array_equal(lo.cpu().numpy(), lg)
@@ -177,11 +185,12 @@ def test_route_identical_router_columns_tie_exactly(cuda_lib, d):
 
 
 @pytest.mark.parametrize("T", mi.DISPATCH_COMBINE_T)
-def test_route_given_logits_sweep(cuda_lib, T):
+def test_route_given_logits_sweep(cuda_lib, route_topk, T):
     tdr = cuda_lib
     cfg = mi.DISPATCH_COMBINE.with_T(T)
     inp = mi.make_inputs(cfg)
-    s = shape_of(cfg, tdr)
+    s = tdr.make_shape(T, cfg.d, cfg.E, cfg.K, cfg.n, cfg.capacity_factor, True,
+                       torch.bfloat16, route_topk=route_topk)
     ids, w, _ = tdr.route(s, logits_in=cuda(inp.logits))
     check_routing(tdr, inp.logits, ids, w, cfg.K)
     assert_status_ok(tdr)
@@ -261,7 +270,8 @@ def test_permute_flags_out_of_range_ids(cuda_lib):
     (683, 64, 6, 0.0, True, False),     # 4098 assignments: the two-call path
     (1365, 64, 6, 1.25, True, False),
 ])
-def test_dispatch_matches_oracle_and_the_two_calls(cuda_lib, T, E, K, cf, renorm, ties):
+def test_dispatch_matches_oracle_and_the_two_calls(cuda_lib, route_topk, T, E, K, cf, renorm,
+                                                   ties):
     tdr = cuda_lib
     rng = np.random.default_rng(T * 7 + E)
     if ties:
@@ -269,7 +279,7 @@ def test_dispatch_matches_oracle_and_the_two_calls(cuda_lib, T, E, K, cf, renorm
         lg[0, ::2] = -0.0
     else:
         lg = rng.standard_normal((T, E)).astype(np.float32)
-    s = tdr.make_shape(T, 64, E, K, 64, cf, renorm, torch.bfloat16)
+    s = tdr.make_shape(T, 64, E, K, 64, cf, renorm, torch.bfloat16, route_topk=route_topk)
     lgd = torch.from_numpy(lg).cuda()
     lo = torch.empty(T, E, device="cuda")
     out = tdr.dispatch(s, logits_in=lgd, logits_out=lo)
@@ -320,16 +330,22 @@ def test_dispatch_from_x_matches_oracle(cuda_lib, T, E, K, cf, mat):
                                       inp.x[torch.from_numpy(p2a[:nk] // K)].view(torch.int16).numpy())
 
 
-def test_dispatch_materialised_gather_is_exact(cuda_lib):
+@pytest.mark.parametrize("T,E,K,d,cf", [
+    (300, 16, 3, 256, 0.9),     # rows copied by the one-launch kernel (small gather)
+    (64, 64, 6, 4096, 0.0),     # the dispatch workload at T = 64: 3 MB, still in one launch
+    (7, 64, 6, 4096, 0.5),      # fewer tokens than CTAs; capacity drops
+    (256, 64, 6, 4096, 0.0),    # 12.6 MB: the separate gather kernel
+    (500, 8, 2, 320, 1.0),      # ragged row (40 vectors)
+])
+def test_dispatch_materialised_gather_is_exact(cuda_lib, route_topk, T, E, K, d, cf):
     tdr = cuda_lib
-    rng = np.random.default_rng(17)
-    T, E, K, d = 300, 16, 3, 256
+    rng = np.random.default_rng(17 + T)
     lg = rng.standard_normal((T, E)).astype(np.float32)
     x = torch.randn(T, d).to(torch.bfloat16)
-    s = tdr.make_shape(T, d, E, K, 64, 0.9, True, torch.bfloat16)
+    s = tdr.make_shape(T, d, E, K, 64, cf, True, torch.bfloat16, route_topk=route_topk)
     out = tdr.dispatch(s, x=x.cuda(), logits_in=torch.from_numpy(lg).cuda(), materialize=True)
     ids_ref, _ = orc.route(lg, K, True)
-    _, offsets, _, p2a = check_permutation(out, ids_ref, E, orc.capacity(0.9, T, K, E))
+    _, offsets, _, p2a = check_permutation(out, ids_ref, E, orc.capacity(cf, T, K, E))
     nk = int(offsets[-1])
     ref = orc.gather_rows(x.float().numpy(), p2a, offsets, K)
     np.testing.assert_array_equal(out["x_perm"][:nk].float().cpu().numpy(), ref)

@@ -34,7 +34,7 @@ class moe_shape(ctypes.Structure):
                 ("K", ctypes.c_int32), ("n", ctypes.c_int32),
                 ("capacity_factor", ctypes.c_float), ("renormalize", ctypes.c_int32),
                 ("dtype", ctypes.c_int32), ("tile_round", ctypes.c_int32),
-                ("ffn_variant", ctypes.c_int32)]
+                ("ffn_variant", ctypes.c_int32), ("route_topk", ctypes.c_int32)]
 
 
 class moe_workspace_layout(ctypes.Structure):
@@ -123,14 +123,16 @@ def _check(code: int, where: str) -> None:
 
 def make_shape(T: int, d: int, E: int, K: int, n: int = 0, capacity_factor: float = 0.0,
                renormalize: bool = True, dtype=torch.bfloat16, tile_round: int = 0,
-               ffn_variant: int = 0) -> moe_shape:
+               ffn_variant: int = 0, route_topk: int = 0) -> moe_shape:
     """tile_round = R > 0 rounds each expert's kept count down to whole R-row tiles.
     ffn_variant selects the bf16 grouped-GEMM tiles: 0 = automatic, 1 = single-CTA 128 x 256
     tiles, 2 = CTA-pair 256 x 256 tiles with the gate/up rows gathered in the GEMM, 3 = CTA
-    pairs with the rows copied first (all compute the same result)."""
+    pairs with the rows copied first (all compute the same result). route_topk selects the
+    top-K form of the warp-per-token routers: 0 = automatic, 1 = K rounds of a warp arg-max,
+    2 = bitonic merges (E <= 64, K <= 8)."""
     dt = MOE_BF16 if dtype == torch.bfloat16 else MOE_F32
     return moe_shape(T, d, E, K, n, float(capacity_factor), 1 if renormalize else 0, dt,
-                     int(tile_round), int(ffn_variant))
+                     int(tile_round), int(ffn_variant), int(route_topk))
 
 
 def _ptr(t: Optional[torch.Tensor]):

@@ -46,7 +46,9 @@ moe_status launch_route_tc(const moe_shape& s, const void* x, const void* w_r, c
 bool route_permute_fusable(const moe_shape& s, const float* logits_in);
 moe_status launch_route_permute(const moe_shape& s, const float* logits_in, float* logits_out,
                                 int32_t* ids, float* w, int32_t* counts, int32_t* offsets,
-                                int32_t* a2p, int32_t* p2a, cudaStream_t st);
+                                int32_t* a2p, int32_t* p2a, const void* x, void* x_perm,
+                                cudaStream_t st);
+bool route_permute_gathers(const moe_shape& s);
 moe_status launch_gather_rows(const moe_shape& s, const void* x, const int32_t* p2a,
                               const int32_t* offsets, void* x_perm, cudaStream_t st);
 moe_status launch_permute_rounded(const moe_shape& s, const int32_t* ids, const float* logits,
@@ -158,6 +160,7 @@ moe_status check_shape(const moe_shape* s, bool need_d, bool need_ffn) {
   if (s->tile_round < 0 || (s->tile_round > 0 && s->capacity_factor > 0.f))
     return MOE_ERR_INVALID_ARG;  // token rounding and a capacity limit are exclusive
   if (s->ffn_variant < 0 || s->ffn_variant > 3) return MOE_ERR_INVALID_ARG;
+  if (s->route_topk < 0 || s->route_topk > 2) return MOE_ERR_INVALID_ARG;
   if (need_d) {
     if (s->d < 64 || s->d % 64 != 0) return MOE_ERR_INVALID_ARG;
   }
@@ -245,7 +248,8 @@ moe_status forward_impl(const moe_shape* s, const void* x, const void* w_r, cons
                                     (int32_t*)(ws + L.round_counts), st)) != MOE_OK)
       return r;
   } else if (route_permute_fusable(*s, logits_in)) {
-    if ((r = launch_route_permute(*s, logits_in, logits, ids, w, counts, offsets, a2p, p2a, st)) !=
+    if ((r = launch_route_permute(*s, logits_in, logits, ids, w, counts, offsets, a2p, p2a,
+                                  nullptr, nullptr, st)) !=
         MOE_OK)
       return r;
   } else {
@@ -400,10 +404,13 @@ moe_status moe_dispatch(const moe_shape* s, const void* x, const void* w_r, cons
   const size_t need = permute_scratch_bytes(*s);
   if (need > 0 && (workspace == nullptr || ws_bytes < need)) return MOE_ERR_WORKSPACE;
   const cudaStream_t st = (cudaStream_t)stream;
+  // small gathers are copied by the one-launch kernel itself
+  const bool fuse_gather = gather && route_permute_gathers(*s);
   if ((r = launch_route_permute(*s, logits_in, logits_out, topk_ids, topk_w, counts, offsets,
-                                assign_to_perm, perm_to_assign, st)) != MOE_OK)
+                                assign_to_perm, perm_to_assign, fuse_gather ? x : nullptr,
+                                fuse_gather ? x_perm : nullptr, st)) != MOE_OK)
     return r;
-  if (gather) return launch_gather_rows(*s, x, perm_to_assign, offsets, x_perm, st);
+  if (gather && !fuse_gather) return launch_gather_rows(*s, x, perm_to_assign, offsets, x_perm, st);
   return MOE_OK;
 }
 

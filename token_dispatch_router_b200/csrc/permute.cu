@@ -24,8 +24,10 @@
 // Problems of at most kSmallMax assignments run all three phases in one CTA.
 // Inside an expert the slots follow ascending flat index a = t*K + k, i.e. token order.
 #include <mutex>
+#include <type_traits>
 
 #include "tc_ptx.cuh"
+#include "topk.cuh"
 
 namespace moe {
 
@@ -520,12 +522,13 @@ moe_status launch_cluster_permute(const int32_t* ids, long long A, int E, long l
 constexpr long long kFusedMax = 4096;  // assignments (above, the two launches were faster)
 constexpr int kFusedTpw = 4;           // tokens a warp routes
 
-template <int WARPS, int ITERS>
+template <int WARPS, int ITERS, int FORM>
 __global__ void __launch_bounds__(WARPS * 32) route_permute_kernel(
     const float* __restrict__ logits_in, float* __restrict__ logits_out, int T, int E, int K,
     int renorm, int tpc, long long cap, int C, int32_t* __restrict__ topk_ids,
     float* __restrict__ topk_w, int32_t* __restrict__ counts, int32_t* __restrict__ offsets,
-    int32_t* __restrict__ assign_to_perm, int32_t* __restrict__ perm_to_assign) {
+    int32_t* __restrict__ assign_to_perm, int32_t* __restrict__ perm_to_assign,
+    const uint4* __restrict__ x, uint4* __restrict__ x_perm, int vec_per_row) {
   constexpr int NT = WARPS * 32;
   constexpr int CHUNK = NT * ITERS;  // assignments a CTA can own
   static_assert(NT >= kMaxE, "one thread per expert in the scan");
@@ -564,60 +567,23 @@ __global__ void __launch_bounds__(WARPS * 32) route_permute_kernel(
     if (r >= ntok) break;  // warp-uniform
     const int t = t0 + r;
     float v[8];
-    bool taken[8];
 #pragma unroll
     for (int j = 0; j < 8; ++j) {
       const int e = lane + 32 * j;
       v[j] = lv[i][j];
-      taken[j] = (e >= E);
       if (logits_out != nullptr && e < E) logits_out[(size_t)t * E + e] = v[j];
     }
-    float vmax = 0.f, selv = 0.f;
-    int sele = 0;
-    for (int k = 0; k < K; ++k) {
-      float bv = -INFINITY;
-      int be = 0x7fffffff;
-#pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        const int e = lane + 32 * j;
-        if (!taken[j] && (v[j] > bv || (v[j] == bv && e < be))) {
-          bv = v[j];
-          be = e;
-        }
-      }
-#pragma unroll
-      for (int off = 16; off > 0; off >>= 1) {
-        const float ov = __shfl_xor_sync(0xffffffffu, bv, off);
-        const int oe = __shfl_xor_sync(0xffffffffu, be, off);
-        if (ov > bv || (ov == bv && oe < be)) {
-          bv = ov;
-          be = oe;
-        }
-      }
-#pragma unroll
-      for (int j = 0; j < 8; ++j)
-        if (lane + 32 * j == be) taken[j] = true;
-      if (k == 0) vmax = bv;
-      if (lane == k) {
-        selv = bv;
-        sele = be;
-      }
-    }
-    const float ex = (lane < K) ? expf(selv - vmax) : 0.f;
-    float den;
-    if (renorm) {
-      den = ex;
+    int sele;
+    float selw;
+    if (E <= 64) {  // two logits a lane: the bitonic form applies
+      const float v2[2] = {v[0], v[1]};
+      warp_route_token<2, FORM>(v2, E, K, renorm, sele, selw);
     } else {
-      den = 0.f;
-#pragma unroll
-      for (int j = 0; j < 8; ++j)
-        if (lane + 32 * j < E) den += expf(v[j] - vmax);
+      warp_route_token<8, TOPK_ROUNDS>(v, E, K, renorm, sele, selw);
     }
-#pragma unroll
-    for (int off = 16; off > 0; off >>= 1) den += __shfl_xor_sync(0xffffffffu, den, off);
     if (lane < K) {
       topk_ids[(size_t)t * K + lane] = sele;
-      topk_w[(size_t)t * K + lane] = ex / den;
+      topk_w[(size_t)t * K + lane] = selw;
       sid[r * K + lane] = sele;
     }
   }
@@ -697,6 +663,7 @@ __global__ void __launch_bounds__(WARPS * 32) route_permute_kernel(
   }
   __syncthreads();
   const unsigned lt = lanemask_lt();
+  int pos[ITERS];  // each assignment's slot, -1 if dropped
 #pragma unroll
   for (int it = 0; it < ITERS; ++it) {
     const int l = l0 + it * 32 + lane;
@@ -715,6 +682,33 @@ __global__ void __launch_bounds__(WARPS * 32) route_permute_kernel(
         perm_to_assign[p] = (int32_t)a;
       }
       assign_to_perm[a] = p;
+    }
+    pos[it] = id >= 0 && (cap < 0 || r < cap) ? offs[id] + r : -1;
+  }
+  if (x_perm != nullptr) {
+    // the rows of this CTA's kept assignments, x_perm[p] = x[t] (a warp per row, four
+    // 16-byte vectors a lane in flight)
+    __syncthreads();  // every warp's ids have left sid
+#pragma unroll
+    for (int it = 0; it < ITERS; ++it) {
+      const int l = l0 + it * 32 + lane;
+      if (l < na) sid[l] = pos[it];
+    }
+    __syncthreads();
+    for (int l = warp; l < na; l += WARPS) {
+      const int p = sid[l];
+      if (p < 0) continue;
+      const uint4* src = x + (size_t)((a0 + l) / K) * vec_per_row;
+      uint4* dst = x_perm + (size_t)p * vec_per_row;
+      for (int v0 = lane; v0 < vec_per_row; v0 += 128) {
+        uint4 q[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+          if (v0 + 32 * j < vec_per_row) q[j] = src[v0 + 32 * j];
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+          if (v0 + 32 * j < vec_per_row) dst[v0 + 32 * j] = q[j];
+      }
     }
   }
   if (C > 1) cluster_wait();  // every CTA has finished reading this CTA's counts
@@ -855,13 +849,16 @@ moe_status launch_gather_rows(const moe_shape& s, const void* x, const int32_t* 
 }
 
 namespace {
-// CTAs of the fused kernel: about 32 tokens per CTA up to 8 CTAs; 8 warps per CTA, or 32
-// when a CTA owns more than 32 tokens (routing runs one token per warp at a time); false if
-// a warp would own more assignments than the instantiated shapes hold (4 x 32 with 8 warps,
-// 2 x 32 with 32)
-bool fused_grid(const moe_shape& s, int* C_out, int* tpc_out, int* warps_out, int* iters_out) {
+// CTAs of the fused kernel: about 32 tokens per CTA up to 8 CTAs (at least min_ctas, one token
+// each at least); 8 warps per CTA, or 32 when a CTA owns more than 32 tokens (routing runs one
+// token per warp at a time); false if a warp would own more assignments than the
+// instantiated shapes hold (4 x 32 with 8 warps, 2 x 32 with 32)
+bool fused_grid(const moe_shape& s, int min_ctas, int* C_out, int* tpc_out, int* warps_out,
+                int* iters_out) {
   int C = (s.T + 31) / 32;
+  if (C < min_ctas) C = min_ctas;
   if (C > kClusterMaxCtas) C = kClusterMaxCtas;
+  if (C > s.T) C = s.T;
   if (C < 1) C = 1;
   const int tpc = (s.T + C - 1) / C;
   const int warps = tpc > 32 ? 32 : 8;
@@ -875,37 +872,55 @@ bool fused_grid(const moe_shape& s, int* C_out, int* tpc_out, int* warps_out, in
   *iters_out = per <= lanes ? 1 : per <= 2 * lanes ? 2 : 4;
   return true;
 }
+// The gathered rows are copied by the fused kernel itself (its C <= 8 CTAs) up to this many
+// bytes; beyond, the many-CTA gather kernel is faster.
+constexpr long long kFusedGatherMax = 4ll << 20;
 }  // namespace
 
 bool route_permute_fusable(const moe_shape& s, const float* logits_in) {
   int C, tpc, warps, iters;
   return logits_in != nullptr && s.T > 0 && s.E <= kMaxE && s.K <= 32 &&
-         (long long)s.T * s.K <= kFusedMax && fused_grid(s, &C, &tpc, &warps, &iters);
+         (long long)s.T * s.K <= kFusedMax && fused_grid(s, 1, &C, &tpc, &warps, &iters);
+}
+
+bool route_permute_gathers(const moe_shape& s) {
+  const long long eb = s.dtype == MOE_BF16 ? 2 : 4;
+  return (long long)s.T * s.K * s.d * eb <= kFusedGatherMax;
 }
 
 moe_status launch_route_permute(const moe_shape& s, const float* logits_in, float* logits_out,
                                 int32_t* ids, float* w, int32_t* counts, int32_t* offsets,
-                                int32_t* a2p, int32_t* p2a, cudaStream_t st) {
+                                int32_t* a2p, int32_t* p2a, const void* x, void* x_perm,
+                                cudaStream_t st) {
   const long long cap =
       (s.capacity_factor > 0.f)
           ? (long long)ceil((double)s.capacity_factor * (double)s.T * (double)s.K / (double)s.E)
           : -1;
   int C, tpc, warps, iters;
-  if (!fused_grid(s, &C, &tpc, &warps, &iters)) return MOE_ERR_UNSUPPORTED;
+  // a fused gather shares the copy over all eight CTAs
+  if (!fused_grid(s, x_perm != nullptr ? kClusterMaxCtas : 1, &C, &tpc, &warps, &iters))
+    return MOE_ERR_UNSUPPORTED;
+  const int vec_per_row = s.d * (s.dtype == MOE_BF16 ? 2 : 4) / 16;
+  const bool bitonic = route_topk_form(s.route_topk, s.E, s.K) == TOPK_BITONIC;
   launch_begin(K_ROUTE_PERMUTE, st);
   auto go = [&](auto kern, int nwarps) {
     launch_kernel(kern, dim3((unsigned)C), dim3(nwarps * 32), 0, st, (unsigned)C, logits_in,
                   logits_out, s.T, s.E, s.K, s.renormalize, tpc, cap, C, ids, w, counts, offsets,
-                  a2p, p2a);
+                  a2p, p2a, (const uint4*)x, (uint4*)x_perm, vec_per_row);
   };
-  if (warps == 8) {
-    if (iters == 1) go(route_permute_kernel<8, 1>, 8);
-    else if (iters == 2) go(route_permute_kernel<8, 2>, 8);
-    else go(route_permute_kernel<8, 4>, 8);
-  } else {
-    if (iters == 1) go(route_permute_kernel<32, 1>, 32);
-    else go(route_permute_kernel<32, 2>, 32);
-  }
+  auto shape = [&](auto form) {
+    constexpr int F = decltype(form)::value;
+    if (warps == 8) {
+      if (iters == 1) go(route_permute_kernel<8, 1, F>, 8);
+      else if (iters == 2) go(route_permute_kernel<8, 2, F>, 8);
+      else go(route_permute_kernel<8, 4, F>, 8);
+    } else {
+      if (iters == 1) go(route_permute_kernel<32, 1, F>, 32);
+      else go(route_permute_kernel<32, 2, F>, 32);
+    }
+  };
+  if (bitonic) shape(std::integral_constant<int, TOPK_BITONIC>());
+  else shape(std::integral_constant<int, TOPK_ROUNDS>());
   return launch_end(K_ROUTE_PERMUTE, st);
 }
 

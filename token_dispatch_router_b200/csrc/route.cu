@@ -8,12 +8,15 @@
 // One CTA owns TM tokens. Phase 1 is a register-tiled fp32 FMA GEMM (x tile and W_r tile
 // staged through shared memory, fp32 accumulation) that leaves the TM x E logits in shared
 // memory; with logits_in the tile is loaded instead. Phase 2 gives one warp per token: each
-// lane holds E/32 logits in registers and K rounds of a warp arg-max under the total order
-// (value descending, id ascending) pick the top-K. Selection compares fp32 logits, so +0 and
-// -0 tie. Weights: exp(l - l_max) over the selected (renormalised) or over all E.
+// lane holds E/32 logits in registers and the top-K under the total order (value descending,
+// id ascending) comes from K rounds of a warp arg-max or, for E <= 64 and K <= 8, from the
+// bitonic merges of the lanes' sorted lists (moe_shape.route_topk). Selection compares fp32
+// logits, so +0 and -0 tie. Weights: exp(l - l_max) over the selected (renormalised) or over
+// all E.
 #include <math.h>
 
 #include "common.cuh"
+#include "topk.cuh"
 
 namespace moe {
 
@@ -22,7 +25,7 @@ namespace {
 constexpr int kThreads = 256;
 constexpr int kDK = 64;
 
-template <typename Tin, int CT, int CPT, int RPT>
+template <typename Tin, int CT, int CPT, int RPT, int FORM>
 __global__ void __launch_bounds__(kThreads) route_kernel(
     const Tin* __restrict__ x, const Tin* __restrict__ w_r, const float* __restrict__ bias,
     const float* __restrict__ logits_in, float* __restrict__ logits_out,
@@ -117,59 +120,17 @@ __global__ void __launch_bounds__(kThreads) route_kernel(
     const int t = t0 + r;
     if (t >= T) break;
     float v[VPL];
-    bool taken[VPL];
 #pragma unroll
     for (int j = 0; j < VPL; ++j) {
       const int e = lane + 32 * j;
       v[j] = (e < E) ? lg[r * LDL + e] : -INFINITY;
-      taken[j] = (e >= E);
     }
-    float vmax = 0.f, selv = 0.f;
-    int sele = 0;
-    for (int k = 0; k < K; ++k) {
-      float bv = -INFINITY;
-      int be = 0x7fffffff;
-#pragma unroll
-      for (int j = 0; j < VPL; ++j) {
-        const int e = lane + 32 * j;
-        if (!taken[j] && (v[j] > bv || (v[j] == bv && e < be))) {
-          bv = v[j];
-          be = e;
-        }
-      }
-#pragma unroll
-      for (int off = 16; off > 0; off >>= 1) {
-        const float ov = __shfl_xor_sync(0xffffffffu, bv, off);
-        const int oe = __shfl_xor_sync(0xffffffffu, be, off);
-        if (ov > bv || (ov == bv && oe < be)) {
-          bv = ov;
-          be = oe;
-        }
-      }
-#pragma unroll
-      for (int j = 0; j < VPL; ++j)
-        if (lane + 32 * j == be) taken[j] = true;
-      if (k == 0) vmax = bv;
-      if (lane == k) {
-        selv = bv;
-        sele = be;
-      }
-    }
-    const float ex = (lane < K) ? expf(selv - vmax) : 0.f;
-    float den;
-    if (renorm) {
-      den = ex;
-    } else {
-      den = 0.f;
-#pragma unroll
-      for (int j = 0; j < VPL; ++j)
-        if (lane + 32 * j < E) den += expf(v[j] - vmax);
-    }
-#pragma unroll
-    for (int off = 16; off > 0; off >>= 1) den += __shfl_xor_sync(0xffffffffu, den, off);
+    int sele;
+    float selw;
+    warp_route_token<VPL, FORM>(v, E, K, renorm, sele, selw);
     if (lane < K) {
       topk_ids[(size_t)t * K + lane] = sele;
-      topk_w[(size_t)t * K + lane] = ex / den;
+      topk_w[(size_t)t * K + lane] = selw;
     }
   }
 }
@@ -183,7 +144,9 @@ moe_status launch_route_t(const moe_shape& s, const void* x, const void* w_r, co
   constexpr int EP = CT * CPT;
   size_t smem = (size_t)TM * (EP + 1) * sizeof(float);
   if (logits_in == nullptr) smem += ((size_t)TM * (kDK + 1) + (size_t)kDK * EP) * sizeof(float);
-  auto kern = route_kernel<Tin, CT, CPT, RPT>;
+  const bool bitonic = route_topk_form(s.route_topk, s.E, s.K) == TOPK_BITONIC;
+  auto kern = bitonic ? route_kernel<Tin, CT, CPT, RPT, TOPK_BITONIC>
+                      : route_kernel<Tin, CT, CPT, RPT, TOPK_ROUNDS>;
   if (smem > 48 * 1024) {
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
         cudaSuccess)

@@ -36,6 +36,7 @@
 #include <mutex>
 
 #include "tc_ptx.cuh"
+#include "topk.cuh"
 
 namespace moe {
 
@@ -99,74 +100,6 @@ __device__ __forceinline__ float ld_shared_f32(uint32_t addr) {
   float v;
   asm volatile("ld.shared.f32 %0, [%1];" : "=f"(v) : "r"(addr) : "memory");
   return v;
-}
-
-// (value, id) order of the selection: a ranks above b when its value is larger, or equal
-// (+0 == -0) with a lower id; an empty slot (id < 0) ranks below everything.
-__device__ __forceinline__ bool ranks_above(float av, int ae, float bv, int be) {
-  if (ae < 0) return false;
-  if (be < 0) return true;
-  return av > bv || (av == bv && ae < be);
-}
-
-// Top-KM list (KM = 2, 4 or 8 >= K), best first, empty slots (id -1) hold -inf. This
-// thread's ids arrive in ascending order, so a value equal to a listed one goes below it
-// (ties to the lower id, +0 == -0): only a strictly larger value moves an entry down. The
-// values shift by min/max (slot j keeps the larger of its own value and the smaller of the
-// slot above and the new value), the ids follow the same comparisons. Compile-time indices
-// only; the common case, a value that does not enter, costs one compare and a branch.
-template <int KM>
-__device__ __forceinline__ void top_insert(float (&bv)[KM], int (&be)[KM], float v, int e) {
-  if (!(v > bv[KM - 1]) && be[KM - 1] >= 0) return;  // does not enter
-  bool gt[KM];  // the new value ranks above the entry in slot j
-#pragma unroll
-  for (int j = 0; j < KM; ++j) gt[j] = be[j] < 0 || v > bv[j];
-#pragma unroll
-  for (int j = KM - 1; j >= 1; --j) {
-    be[j] = gt[j] ? (gt[j - 1] ? be[j - 1] : e) : be[j];
-    bv[j] = gt[j] ? (gt[j - 1] ? bv[j - 1] : v) : bv[j];
-  }
-  if (gt[0]) {
-    be[0] = e;
-    bv[0] = v;
-  }
-}
-
-// Merge this thread's sorted list with that of the lane `mask` away (same token group):
-// c[i] = better of a[i] and b[KM-1-i] holds the KM best of both lists as a bitonic
-// sequence, which log2(KM) half-cleaner stages sort. Both lanes end with the same list.
-template <int KM>
-__device__ __forceinline__ void top_merge(float (&bv)[KM], int (&be)[KM], int mask) {
-  float ov[KM];
-  int oe[KM];
-#pragma unroll
-  for (int j = 0; j < KM; ++j) {
-    ov[j] = __shfl_xor_sync(0xffffffffu, bv[j], mask);
-    oe[j] = __shfl_xor_sync(0xffffffffu, be[j], mask);
-  }
-#pragma unroll
-  for (int j = 0; j < KM; ++j) {
-    if (!ranks_above(bv[j], be[j], ov[KM - 1 - j], oe[KM - 1 - j])) {
-      bv[j] = ov[KM - 1 - j];
-      be[j] = oe[KM - 1 - j];
-    }
-  }
-#pragma unroll
-  for (int h = KM / 2; h >= 1; h /= 2) {
-#pragma unroll
-    for (int j = 0; j < KM; ++j) {
-      if ((j & h) == 0) {
-        if (ranks_above(bv[j + h], be[j + h], bv[j], be[j])) {
-          const float tv = bv[j];
-          const int te = be[j];
-          bv[j] = bv[j + h];
-          be[j] = be[j + h];
-          bv[j + h] = tv;
-          be[j + h] = te;
-        }
-      }
-    }
-  }
 }
 
 // Eight of one token's experts, e = e0 + G j: their partials from every rank (loaded first,
