@@ -151,6 +151,102 @@ def tile_round_keep(topk_ids_, logits_f32, E: int, R: int) -> np.ndarray:
     return keep
 
 
+def tile_round_select(topk_ids_, logits_f32, E: int, R: int, mode: str = "down"):
+    """[P5] 6.5 with rounding in either direction (the library's reading: the page says
+    only that expert token counts are brought closer to kernel-friendly tile shapes).
+    For expert e with c routed assignments and r = c mod R != 0:
+      down    - c >= R: drop its r weakest assignments (tile_round_keep); c < R: keep all;
+      up      - add the m = min(R - r, T - c) tokens that did not route to e with the
+                largest router logit for e (equal logits: the earlier token), each gaining
+                one more slot;
+      nearest - down when r <= R - r, else up.
+    Returns (keep [T, K] bool, add_tok [n], add_exp [n]); the added assignments are
+    listed by expert, then by ascending token."""
+    if mode not in ("down", "up", "nearest"):
+        raise ValueError(mode)
+    ids = np.asarray(topk_ids_, dtype=np.int64)
+    lg = np.asarray(logits_f32, dtype=np.float32)
+    T, K = ids.shape
+    keep = np.ones((T, K), dtype=bool)
+    add_tok, add_exp = [], []
+    if R <= 1:
+        return keep, np.zeros(0, np.int64), np.zeros(0, np.int64)
+    for e in range(E):
+        tok, slot = np.nonzero(ids == e)  # ascending token
+        c = tok.size
+        r = c % R
+        if r == 0:
+            continue
+        up = mode == "up" or (mode == "nearest" and r > R - r)
+        if not up:
+            if c >= R:
+                order = np.lexsort((-tok, lg[tok, e].astype(F64)))  # weakest first
+                drop = order[:r]
+                keep[tok[drop], slot[drop]] = False
+            continue
+        routed = np.zeros(T, dtype=bool)
+        routed[tok] = True
+        cand = np.nonzero(~routed)[0]
+        m = min(R - r, cand.size)
+        if m == 0:
+            continue
+        # strongest first: larger logit, then the earlier token
+        order = np.lexsort((cand, -lg[cand, e].astype(F64)))
+        chosen = np.sort(cand[order[:m]])
+        add_tok.extend(chosen.tolist())
+        add_exp.extend([e] * m)
+    return keep, np.asarray(add_tok, np.int64), np.asarray(add_exp, np.int64)
+
+
+def round_weights(logits_f32, topk_ids_, add_tok, add_exp, renormalize: bool = True):
+    """Weights after rounding up: each token's selection is its K routed experts plus the
+    experts it was added to. Renormalised: w = exp(l - l_max) / (sum over the enlarged
+    selection of exp(l_j - l_max)) (they still sum to 1); plain: softmax(l) over all E at
+    every selected expert (the routed weights are unchanged). Dropped assignments keep
+    their place in the sum (reading 6: no re-renormalisation). fp64, rounded to fp32.
+    Returns (topk_w [T, K], add_w [n])."""
+    lg = np.asarray(logits_f32, dtype=np.float32).astype(F64)
+    ids = np.asarray(topk_ids_, dtype=np.int64)
+    T, K = ids.shape
+    add_tok = np.asarray(add_tok, np.int64)
+    add_exp = np.asarray(add_exp, np.int64)
+    w = np.zeros((T, K), dtype=F64)
+    add_w = np.zeros(add_tok.size, dtype=F64)
+    for t in range(T):
+        extra = np.nonzero(add_tok == t)[0]
+        sel = np.concatenate([ids[t], add_exp[extra]])
+        if renormalize:
+            top = lg[t, ids[t, 0]]
+            z = np.exp(lg[t, sel] - top)
+            p = z / z.sum()
+        else:
+            m = lg[t].max()
+            p = np.exp(lg[t, sel] - m) / np.exp(lg[t] - m).sum()
+        w[t] = p[:K]
+        add_w[extra] = p[K:]
+    return w.astype(np.float32), add_w.astype(np.float32)
+
+
+def permute_ext(ids_ext, E: int):
+    """The stable permutation over an extended assignment list (routed assignments a =
+    t*K + k first, then the added ones): expert-major, ascending flat index inside an
+    expert; -1 marks an assignment that does not exist (dropped). Returns (offsets,
+    assign_to_perm, perm_to_assign) over len(ids_ext) assignments."""
+    ids = np.asarray(ids_ext, dtype=np.int64).reshape(-1)
+    A = ids.size
+    offsets = np.zeros(E + 1, dtype=np.int64)
+    members = [np.nonzero(ids == e)[0] for e in range(E)]
+    for e in range(E):
+        offsets[e + 1] = offsets[e] + members[e].size
+    p2a = np.full(A, -1, dtype=np.int64)
+    a2p = np.full(A, -1, dtype=np.int64)
+    for e in range(E):
+        for r, a in enumerate(members[e]):
+            p2a[offsets[e] + r] = a
+            a2p[a] = offsets[e] + r
+    return offsets.astype(np.int32), a2p.astype(np.int32), p2a.astype(np.int32)
+
+
 def permute(topk_ids_, E: int, C: Optional[int] = None, keep=None):
     """[P1] 3 (counting + prefix sum), [P2] 2.3 (sort tasks by (expert, token)),
     [P5] 11 (expert-major metadata).
@@ -415,19 +511,63 @@ def combine(y_perm, assign_to_perm, topk_w, T: int, K: int) -> np.ndarray:
     return out
 
 
+def slot_tokens(perm_to_assign, n_kept: int, K: int, T: int, add_tok) -> np.ndarray:
+    """Token of each kept expert-major slot over the extended assignment list: a < T*K is
+    token a // K, an added assignment a = T*K + j is add_tok[j]."""
+    p2a = np.asarray(perm_to_assign, dtype=np.int64)[:n_kept]
+    add_tok = np.asarray(add_tok, np.int64)
+    A0 = T * K
+    return np.where(p2a < A0, p2a // K, add_tok[np.maximum(p2a - A0, 0)] if add_tok.size else 0)
+
+
+def combine_ext(y_perm, assign_to_perm, topk_w, T: int, K: int, add_tok, add_w) -> np.ndarray:
+    """combine over the extended assignments: out[t] = sum_k w[t,k] y[slot(t*K+k)] (k order,
+    dropped slots add nothing), then the token's added assignments in expert order
+    (= their order in the added list), w y[slot(T*K+j)]. fp64."""
+    y = as_f64(y_perm)
+    a2p = np.asarray(assign_to_perm, dtype=np.int64)
+    out = combine(y, a2p[:T * K], topk_w, T, K)
+    add_tok = np.asarray(add_tok, np.int64)
+    aw = as_f64(add_w)
+    for j in range(add_tok.size):
+        p = a2p[T * K + j]
+        if p >= 0:
+            out[add_tok[j]] += aw[j] * y[p]
+    return out
+
+
 # --------------------------------------------------------------------------- layer
 def forward(x, w_r, w_gate, w_up, w_down, K: int, capacity_factor: float = 0.0,
-            bias=None, logits=None, renormalize: bool = True, tile_round: int = 0):
+            bias=None, logits=None, renormalize: bool = True, tile_round: int = 0,
+            round_mode: str = "down"):
     """The whole layer forward ([P5] section 3 pipeline), every intermediate kept.
 
     ``logits`` (fp32 [T, E]) replaces x . W_r + bias when given: this is how
     ids/counts/permutation parity is checked on identical logits. ``tile_round``
-    = R > 0 applies token rounding to R-row tiles (see tile_round_keep)."""
+    = R > 0 applies token rounding to R-row tiles (see tile_round_keep); round_mode "up"
+    or "nearest" may add assignments (see tile_round_select), laid out after the routed
+    ones (a = T*K + j) and reported in add_tok / add_exp / add_w."""
     T = x.shape[0]
     lg = router_logits(x, w_r, bias) if logits is None else np.asarray(logits, np.float32)
     E = lg.shape[1]
     ids, w = route(lg, K, renormalize)
     C = capacity(capacity_factor, T, K, E)
+    if tile_round > 0 and round_mode != "down":
+        if C is not None:
+            raise ValueError("token rounding and a capacity limit are exclusive")
+        keep, add_tok, add_exp = tile_round_select(ids, lg, E, tile_round, round_mode)
+        counts = np.bincount(ids.reshape(-1), minlength=E).astype(np.int32)
+        ids_ext = np.concatenate([np.where(keep, ids, -1).reshape(-1), add_exp])
+        offsets, a2p, p2a = permute_ext(ids_ext, E)
+        w, add_w = round_weights(lg, ids, add_tok, add_exp, renormalize)
+        n_kept = int(offsets[-1])
+        tok = slot_tokens(p2a, n_kept, K, T, add_tok)
+        a_act, y_perm = grouped_ffn(x, tok, offsets, 1, w_gate, w_up, w_down)
+        out = combine_ext(y_perm, a2p, w, T, K, add_tok, add_w)
+        return dict(logits=lg, topk_ids=ids, topk_w=w, counts=counts, offsets=offsets,
+                    assign_to_perm=a2p, perm_to_assign=p2a, a_act=a_act, y_perm=y_perm,
+                    out=out, capacity=C, add_tok=add_tok, add_exp=add_exp, add_w=add_w,
+                    slot_tokens=tok)
     keep = None
     if tile_round > 0:
         if C is not None:

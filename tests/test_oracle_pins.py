@@ -523,6 +523,162 @@ def test_token_rounding_planted_mistake_is_caught(monkeypatch):
     assert not np.array_equal(wrong, _rounding_brute_force(ids, lg, E, R))
 
 
+# ------------------------------------------------------------------ token rounding up / nearest
+def _up_case():
+    # T = 6, E = 2, K = 1: routed e0 = {0, 1, 4, 5} (t5 ties 2 = 2: the lower id), e1 = {2, 3}
+    return np.array([[5, 1], [4, 2], [0, 3], [3, 3.5], [1, 0], [2, 2]], dtype=np.float32)
+
+
+def test_rounding_up_hand_worked():
+    """R = 4: e0 holds 4 (unchanged); e1 holds 2 and gains 2 of t0 (1), t1 (2), t4 (0),
+    t5 (2): t1 and t5 (equal logits, both taken). Renormalised weights over the enlarged
+    selections: t1 {e0, e1} = softmax(4, 2), t5 {e0, e1} = softmax(2, 2) = (1/2, 1/2)."""
+    lg = _up_case()
+    ids, _ = orc.route(lg, 1)
+    np.testing.assert_array_equal(ids[:, 0], [0, 0, 1, 1, 0, 0])
+    keep, at, ae = orc.tile_round_select(ids, lg, 2, 4, "up")
+    assert keep.all()
+    np.testing.assert_array_equal(at, [1, 5])
+    np.testing.assert_array_equal(ae, [1, 1])
+    w, aw = orc.round_weights(lg, ids, at, ae)
+    s1 = 1.0 / (1.0 + math.exp(-2.0))
+    np.testing.assert_allclose([w[1, 0], aw[0]], [s1, 1.0 - s1], rtol=1e-6)
+    np.testing.assert_allclose([w[5, 0], aw[1]], [0.5, 0.5], rtol=1e-7)
+    np.testing.assert_allclose(w[[0, 2, 3, 4], 0], 1.0)
+    # nearest: e1 has r = 2 = R - r: rounds down, and with c < R it keeps all (no change)
+    keep, at, ae = orc.tile_round_select(ids, lg, 2, 4, "nearest")
+    assert keep.all() and at.size == 0
+
+
+def test_rounding_nearest_hand_worked():
+    """R = 4, e1 routed 3 times (r = 3 > R - r = 1): nearest rounds up by one, the best
+    non-routed token for e1; e0 routed 5 times (r = 1): nearest drops its weakest."""
+    lg = np.array([[9, 1], [8, 2], [0, 7], [1, 6], [2, 5], [7, 4], [6, 3], [5, 0]],
+                  dtype=np.float32)
+    ids, _ = orc.route(lg, 1)
+    np.testing.assert_array_equal(ids[:, 0], [0, 0, 1, 1, 1, 0, 0, 0])
+    keep, at, ae = orc.tile_round_select(ids, lg, 2, 4, "nearest")
+    # e0 = {0, 1, 5, 6, 7} with logits 9, 8, 7, 6, 5: drop t7 (the weakest)
+    np.testing.assert_array_equal(keep[:, 0], [True] * 7 + [False])
+    # e1 gains the best of t0 (1), t1 (2), t5 (4), t6 (3), t7 (0): t5
+    np.testing.assert_array_equal(at, [5])
+    np.testing.assert_array_equal(ae, [1])
+
+
+def _is_top_m(cand, chosen, score):
+    """Brute force over pairs: every chosen token ranks above every unchosen candidate
+    (larger logit, or equal logit and earlier token)."""
+    ch = set(int(c) for c in chosen)
+    for c in ch:
+        for u in cand:
+            u = int(u)
+            if u in ch:
+                continue
+            if not (score[c] > score[u] or (score[c] == score[u] and c < u)):
+                return False
+    return True
+
+
+@pytest.mark.parametrize("seed", range(6))
+def test_rounding_up_adds_the_best_non_routed_tokens(seed):
+    g = np.random.default_rng(100 + seed)
+    T, E, K, R = 30, 5, 2, 7
+    lg = g.integers(-3, 4, size=(T, E)).astype(np.float32)  # ties on purpose
+    ids, _ = orc.route(lg, K)
+    keep, at, ae = orc.tile_round_select(ids, lg, E, R, "up")
+    assert keep.all()
+    for e in range(E):
+        routed = np.unique(np.nonzero(ids == e)[0])
+        c = routed.size
+        chosen = at[ae == e]
+        cand = np.setdiff1d(np.arange(T), routed)
+        want = 0 if c % R == 0 else min(R - c % R, cand.size)
+        assert chosen.size == want
+        assert np.all(np.diff(chosen) > 0) and not np.isin(chosen, routed).any()
+        assert _is_top_m(cand, chosen, lg[:, e])
+        final = c + chosen.size
+        assert final % R == 0 or final == T
+
+
+@pytest.mark.parametrize("seed", range(4))
+def test_rounding_nearest_invariants(seed):
+    g = np.random.default_rng(200 + seed)
+    T, E, K, R = 60, 6, 2, 8
+    lg = g.standard_normal((T, E)).astype(np.float32)
+    ids, _ = orc.route(lg, K)
+    keep, at, ae = orc.tile_round_select(ids, lg, E, R, "nearest")
+    down_keep = orc.tile_round_keep(ids, lg, E, R)
+    for e in range(E):
+        c = int((ids == e).sum())
+        r = c % R
+        final = int((keep & (ids == e)).sum()) + int((ae == e).sum())
+        if r == 0:
+            assert final == c
+        elif r <= R - r:  # down: the down rule's result for this expert
+            assert final == (c if c < R else c - r)
+            np.testing.assert_array_equal(keep[ids == e], down_keep[ids == e])
+        else:
+            assert final == min(c + R - r, T)
+    # mode "down" is tile_round_keep with nothing added
+    k2, at2, _ = orc.tile_round_select(ids, lg, E, R, "down")
+    np.testing.assert_array_equal(k2, down_keep)
+    assert at2.size == 0
+
+
+@pytest.mark.parametrize("renorm", [True, False])
+def test_rounded_up_layer_equals_dense_sum_with_enlarged_gates(renorm):
+    """The layer with added assignments equals the dense sum over all E experts gated by
+    each token's weights over its enlarged selection (0 elsewhere), and the renormalised
+    weights of a token sum to one."""
+    g = np.random.default_rng(7)
+    T, d, n, E, K, R = 24, 16, 32, 4, 2, 5
+    x = g.standard_normal((T, d))
+    w_r = 0.5 * g.standard_normal((d, E))
+    wg, wu, wd = (0.3 * g.standard_normal((E, d, n)), 0.3 * g.standard_normal((E, d, n)),
+                  0.3 * g.standard_normal((E, n, d)))
+    f = orc.forward(x, w_r, wg, wu, wd, K, renormalize=renorm, tile_round=R, round_mode="up")
+    at, ae, aw = f["add_tok"], f["add_exp"], f["add_w"]
+    assert at.size > 0
+    gate = np.zeros((T, E))
+    for t in range(T):
+        for k in range(K):
+            gate[t, f["topk_ids"][t, k]] = f["topk_w"][t, k]
+    for j in range(at.size):
+        gate[at[j], ae[j]] = aw[j]
+    if renorm:
+        np.testing.assert_allclose(gate.sum(axis=1), 1.0, rtol=1e-6)
+    dense = np.zeros((T, d))
+    for e in range(E):
+        dense += gate[:, e:e + 1] * orc.expert_ffn(x, wg[e], wu[e], wd[e])
+    np.testing.assert_allclose(f["out"], dense, rtol=1e-9, atol=1e-9)
+    counts = np.diff(f["offsets"])
+    assert np.all((counts % R == 0) | (counts == T))
+
+
+def test_rounding_up_planted_mistakes_are_caught(monkeypatch):
+    """A tie rule reversed inside the selection, and added weights over the routed
+    denominator only, both fail the pins above."""
+    lg = _up_case()
+    ids, _ = orc.route(lg, 1)
+    real = np.lexsort
+
+    def later_token_first(keys):  # the selection's tie-break inverted
+        return real((-np.asarray(keys[0]),) + tuple(keys[1:]))
+
+    # R = 3: e1 (routed 2) gains one token, t1 and t5 tie at 2: the earlier one, t1
+    _, at, ae = orc.tile_round_select(ids, lg, 2, 3, "up")
+    np.testing.assert_array_equal(at[ae == 1], [1])
+    monkeypatch.setattr(orc.np, "lexsort", later_token_first)
+    _, at, ae = orc.tile_round_select(ids, lg, 2, 3, "up")
+    monkeypatch.undo()
+    assert not np.array_equal(at[ae == 1], [1])
+    # weights of the added slot over the routed selection only: the token's weights no
+    # longer sum to one
+    w, aw = orc.round_weights(lg, ids, [1, 5], [1, 1])
+    wrong = math.exp(2.0 - 4.0)  # exp(l_add - l_top) / (routed sum = 1)
+    assert abs(w[1, 0] + wrong - 1.0) > 1e-3 and abs(w[1, 0] + aw[0] - 1.0) < 1e-6
+
+
 # ------------------------------------------------------------------ backward (expert half)
 def _autograd_backward(x, lg, wg, wu, wd, K, cf, d_out):
     """The same layer written with torch ops in fp64 and differentiated by autograd: the
