@@ -65,19 +65,31 @@ typedef enum { MOE_F32 = 0, MOE_BF16 = 1 } moe_dtype;
  * K <= 32, T >= 0, T * K < 2^31, d % 64 == 0 (router tiles, TMA boxes);
  * n % 64 == 0 for MOE_BF16 and n % 16 == 0 for MOE_F32.
  * tile_round = R > 0: tile-aware token rounding (SonicMoE explainer, section 6.5, names
- * it without a rule; this is the library's reading): an expert with c >= R routed
- * assignments keeps R * floor(c / R) of them, the ones with the largest router logit for
- * that expert (equal logits: the earlier token stays), and drops the rest like capacity
- * overflow (assign_to_perm = -1, no re-normalisation); an expert with c < R keeps all.
- * Nothing is added. Needs the router logits, so it applies in moe_forward and
- * moe_dispatch (moe_permute returns MOE_ERR_UNSUPPORTED); exclusive with
- * capacity_factor > 0. 0 = off. */
+ * it without a rule; this is the library's reading), in the direction tile_round_mode gives
+ * (0 = down, 1 = up, 2 = nearest). For expert e with c routed assignments, r = c mod R != 0:
+ *   down: with c >= R, e keeps R * floor(c / R) of them, the ones with the largest router
+ *     logit for e (equal logits: the earlier token stays), and drops the rest like capacity
+ *     overflow (assign_to_perm = -1, no re-normalisation); with c < R it keeps all;
+ *   up: e gains the min(R - r, T - c) tokens that did not route to it with the largest
+ *     router logit for it (equal logits: the earlier token), each such token gaining one
+ *     more slot; a token's weights are then computed over its enlarged selection
+ *     (renormalised: they still sum to 1; plain softmax: unchanged for its routed experts);
+ *   nearest: down when r <= R - r, else up.
+ * Added assignments follow the routed ones in the flat numbering, a = T*K + j for the j-th
+ * added (listed by expert, then ascending token), so that assign_to_perm / perm_to_assign
+ * span T*K + E*(R-1) entries with rounding up or to the nearest tile. Needs the router
+ * logits, so rounding applies in moe_forward (every direction) and moe_dispatch (down only;
+ * the other directions return MOE_ERR_UNSUPPORTED there, as moe_permute does for any
+ * rounding, and moe_forward_h); exclusive with capacity_factor > 0. 0 = off. Up and nearest
+ * need T <= 131072 (one bit a token in shared memory) and T*K + E*(R-1) < 2^31, else
+ * MOE_ERR_UNSUPPORTED. */
 typedef struct {
   int32_t T, d, E, K, n;
   float capacity_factor;
   int32_t renormalize;
   int32_t dtype;      /* moe_dtype */
   int32_t tile_round; /* 0, or the row tile R that each expert's kept count is rounded to */
+  int32_t tile_round_mode; /* 0 = round down, 1 = up, 2 = to the nearest tile (see above) */
   int32_t ffn_variant; /* tiles of the bf16 grouped GEMMs (a deployment choice; the pages have
                         * no counterpart): 0 = automatic, 1 = single-CTA 128 x 256 tiles,
                         * 2 = CTA pairs (256 x 256 tiles on two SMs, tcgen05 cta_group::2)
@@ -106,7 +118,8 @@ typedef struct {
  *   the rounded copy of the ids and the kept counts (used by moe_dispatch).
  * moe_forward_workspace_size: everything moe_forward keeps between kernels:
  *   logits, top-K ids and weights, counts, offsets, both permutation indices,
- *   the permute scratch, a_act[T*K, n] and y_perm[T*K, d].
+ *   the permute scratch, a_act[n_assign, n] and y_perm[n_assign, d] (n_assign = T*K, or
+ *   T*K + E*(R-1) with rounding up or to the nearest tile) and the rounding buffers.
  */
 size_t moe_permute_workspace_size(const moe_shape* shape);
 size_t moe_forward_workspace_size(const moe_shape* shape);
@@ -277,7 +290,15 @@ moe_status moe_forward(const moe_shape* shape, const void* x, const void* w_r, c
 /* Byte offsets of the intermediates inside moe_forward's workspace. */
 typedef struct {
   size_t logits, topk_ids, topk_w, counts, offsets, assign_to_perm, perm_to_assign,
-      permute_scratch, a_act, y_perm, round_ids, round_counts, total;
+      permute_scratch, a_act, y_perm, round_ids, round_counts;
+  /* rounding up or to the nearest tile (else equal to total, zero-sized): the added
+   * assignments' tokens add_tok [E*(R-1)] int32 (-1 past the last one), their weights
+   * add_w [E*(R-1)] fp32, each token's added assignments add_ptr [T+1] / add_idx
+   * [E*(R-1)] (indices j into add_tok, ascending per token), a per-token cursor
+   * add_cursor [T], and the token of every expert-major slot slot_token [T*K + E*(R-1)]. */
+  size_t add_tok, add_w, add_ptr, add_idx, add_cursor, slot_token;
+  size_t n_assign; /* entries of assign_to_perm / perm_to_assign: T*K, or T*K + E*(R-1) */
+  size_t total;
 } moe_workspace_layout;
 moe_status moe_forward_workspace_layout(const moe_shape* shape, moe_workspace_layout* layout);
 

@@ -228,3 +228,52 @@ def test_route_topk_is_a_checked_shape_field(lib, form, ok):
     """The top-K form of the warp-per-token routers is a per-call shape field."""
     s = tdr.make_shape(64, 128, 8, 2, 128, 0.0, True, torch.bfloat16, route_topk=form)
     assert (lib.moe_forward_workspace_size(ctypes.byref(s)) > 0) == ok
+
+
+@pytest.mark.parametrize("mode,ok", [(0, True), (1, True), (2, True), (3, False), (-1, False)])
+def test_tile_round_mode_is_a_checked_shape_field(lib, mode, ok):
+    """The rounding direction is a per-call shape field: 0 down, 1 up, 2 nearest."""
+    s = tdr.make_shape(64, 128, 8, 2, 128, 0.0, True, torch.bfloat16, tile_round=16,
+                       tile_round_mode=mode)
+    assert (lib.moe_forward_workspace_size(ctypes.byref(s)) > 0) == ok
+
+
+def test_rounding_up_layout_spans_the_added_assignments(lib):
+    """Rounding up or to the nearest tile lays out T*K + E*(R-1) entries in both maps, the
+    activations and the expert outputs, plus the added-assignment lists; rounding down and
+    no rounding lay out T*K."""
+    T, d, E, K, n, R = 1000, 128, 8, 2, 128, 16
+    lays = {}
+    for mode in (0, 1, 2):
+        s = tdr.make_shape(T, d, E, K, n, 0.0, True, torch.bfloat16, tile_round=R,
+                           tile_round_mode=mode)
+        lays[mode] = tdr.forward_workspace_layout(s)
+    assert lays[0].n_assign == T * K
+    for mode in (1, 2):
+        L = lays[mode]
+        assert L.n_assign == T * K + E * (R - 1)
+        assert L.y_perm - L.a_act >= L.n_assign * n * 2
+        assert L.add_w - L.add_tok >= E * (R - 1) * 4
+        assert L.add_idx - L.add_ptr >= (T + 1) * 4
+        assert L.total - L.slot_token >= L.n_assign * 4
+        offs = [L.logits, L.topk_ids, L.topk_w, L.counts, L.offsets, L.assign_to_perm,
+                L.perm_to_assign, L.permute_scratch, L.a_act, L.y_perm, L.round_ids,
+                L.round_counts, L.add_tok, L.add_w, L.add_ptr, L.add_idx, L.add_cursor,
+                L.slot_token, L.total]
+        assert offs == sorted(offs) and all(o % 256 == 0 for o in offs)
+    plain = tdr.forward_workspace_layout(tdr.make_shape(T, d, E, K, n, 0.0, True,
+                                                        torch.bfloat16))
+    assert plain.n_assign == T * K and plain.slot_token == plain.total
+
+
+def test_rounding_up_limits(lib):
+    """Up and nearest: one bit a token in shared memory (T <= 131072); moe_dispatch only
+    rounds down."""
+    big = tdr.make_shape(131073, 128, 8, 2, 128, 0.0, True, torch.bfloat16, tile_round=16,
+                         tile_round_mode=1)
+    assert lib.moe_forward_workspace_size(ctypes.byref(big)) == 0
+    edge = tdr.make_shape(131072, 128, 8, 2, 128, 0.0, True, torch.bfloat16, tile_round=16,
+                          tile_round_mode=1)
+    assert lib.moe_forward_workspace_size(ctypes.byref(edge)) > 0
+    down = tdr.make_shape(131073, 128, 8, 2, 128, 0.0, True, torch.bfloat16, tile_round=16)
+    assert lib.moe_forward_workspace_size(ctypes.byref(down)) > 0

@@ -613,6 +613,177 @@ def test_token_rounding_rejected_where_it_cannot_apply(cuda_lib):
         tdr.dispatch(bad, logits_in=torch.zeros(64, 8, device="cuda"))
 
 
+# ------------------------------------------------------------------ token rounding up / nearest
+def _check_rounded_up(tdr, s, v, ref, R, T, E, K, f32):
+    """Every intermediate of a forward that rounds up or to the nearest tile against the
+    oracle's: the discrete ones exactly, the weights within W_ABS, the rows within the
+    dtype's bar. Returns the number of added assignments."""
+    ids_ref = ref["topk_ids"]
+    np.testing.assert_array_equal(v["topk_ids"].cpu().numpy(), ids_ref)
+    np.testing.assert_array_equal(v["counts"].cpu().numpy(), ref["counts"])
+    NA = E * (R - 1)
+    n_add = ref["add_tok"].size
+    assert n_add <= NA
+    keep = (ref["assign_to_perm"][:T * K] >= 0).reshape(T, K)
+    ids_ext = np.full(T * K + NA, -1, np.int64)
+    ids_ext[:T * K] = np.where(keep, ids_ref, -1).reshape(-1)
+    ids_ext[T * K:T * K + n_add] = ref["add_exp"]
+    np.testing.assert_array_equal(v["round_ids"].cpu().numpy(), ids_ext)
+    add_tok = v["add_tok"].cpu().numpy()
+    np.testing.assert_array_equal(add_tok[:n_add], ref["add_tok"])
+    assert np.all(add_tok[n_add:] == -1)
+    offsets = ref["offsets"]
+    np.testing.assert_array_equal(v["offsets"].cpu().numpy(), offsets)
+    a2p_ref = np.full(T * K + NA, -1, np.int64)
+    a2p_ref[:ref["assign_to_perm"].size] = ref["assign_to_perm"]
+    np.testing.assert_array_equal(v["assign_to_perm"].cpu().numpy(), a2p_ref)
+    nk = int(offsets[-1])
+    np.testing.assert_array_equal(v["perm_to_assign"].cpu().numpy()[:nk],
+                                  ref["perm_to_assign"][:nk])
+    np.testing.assert_array_equal(v["slot_token"].cpu().numpy()[:nk], ref["slot_tokens"])
+    assert np.abs(v["topk_w"].cpu().numpy().astype(np.float64) - ref["topk_w"]).max() <= W_ABS
+    if n_add:
+        got_aw = v["add_w"].cpu().numpy()[:n_add].astype(np.float64)
+        assert np.abs(got_aw - ref["add_w"]).max() <= W_ABS
+    # the token-major lists: each token's added entries, ascending
+    ptr = v["add_ptr"].cpu().numpy()
+    idx = v["add_idx"].cpu().numpy()
+    assert ptr[0] == 0 and ptr[-1] == n_add
+    for t in np.unique(ref["add_tok"])[:64]:
+        np.testing.assert_array_equal(idx[ptr[t]:ptr[t + 1]],
+                                      np.nonzero(ref["add_tok"] == t)[0])
+    return n_add
+
+
+@pytest.mark.parametrize("T,d,n,E,K,R,mode,dtype,renorm,ties", [
+    (1000, 128, 128, 8, 2, 64, "up", "bf16", True, False),
+    (1000, 128, 128, 8, 2, 64, "nearest", "bf16", True, False),
+    (3001, 64, 64, 32, 4, 128, "up", "bf16", True, True),     # integer logits: ties
+    (300, 64, 64, 4, 1, 128, "up", "bf16", False, False),     # c < R: every expert gains
+    (200, 64, 128, 8, 2, 256, "up", "bf16", True, False),     # R > T: every token everywhere
+    (500, 64, 64, 16, 3, 16, "nearest", "f32", True, False),  # the fp32 grouped FFN
+    (16384, 64, 64, 128, 8, 128, "nearest", "bf16", True, False),  # chunked permutation
+    (129, 64, 64, 3, 1, 1, "up", "bf16", True, False),        # R = 1 changes nothing
+])
+def test_forward_token_rounding_up_matches_oracle(cuda_lib, T, d, n, E, K, R, mode, dtype,
+                                                  renorm, ties):
+    tdr = cuda_lib
+    cfg = mi.MoEConfig("round_up", T=T, d=d, E=E, K=K, n=n, dtype=dtype, seed=T + R)
+    inp = mi.make_inputs(cfg)
+    rng = np.random.default_rng(T + E + R)
+    if ties:
+        lg = rng.integers(-3, 4, size=(T, E)).astype(np.float32)
+    else:
+        lg = rng.standard_normal((T, E)).astype(np.float32)
+    dt = torch.bfloat16 if dtype == "bf16" else torch.float32
+    m = {"up": 1, "nearest": 2}[mode]
+    s = tdr.make_shape(T, d, E, K, n, 0.0, renorm, dt, tile_round=R, tile_round_mode=m)
+    out, ws = tdr.forward(s, cuda(inp.x), None, cuda(inp.w_gate), cuda(inp.w_up),
+                          cuda(inp.w_down), logits_in=torch.from_numpy(lg).cuda())
+    torch.cuda.synchronize()
+    assert_status_ok(tdr)
+    v = tdr.workspace_views(s, ws)
+    ref = orc.forward(inp.x, None, inp.w_gate, inp.w_up, inp.w_down, K, logits=lg,
+                      renormalize=renorm, tile_round=R, round_mode=mode)
+    if R == 1:  # nothing to round: the plain forward, its workspace without added entries
+        plain = orc.forward(inp.x, None, inp.w_gate, inp.w_up, inp.w_down, K, logits=lg,
+                            renormalize=renorm)
+        assert ref["add_tok"].size == 0 and "add_tok" not in v
+        np.testing.assert_array_equal(v["offsets"].cpu().numpy(), plain["offsets"])
+        np.testing.assert_array_equal(v["assign_to_perm"].cpu().numpy(),
+                                      plain["assign_to_perm"])
+        assert_bf16_close(out.float().cpu().numpy(), ref["out"], "out")
+        return
+    n_add = _check_rounded_up(tdr, s, v, ref, R, T, E, K, dtype == "f32")
+    nk = int(ref["offsets"][-1])
+    got = [v["a_act"][:nk].float().cpu().numpy(), v["y_perm"][:nk].float().cpu().numpy(),
+           out.float().cpu().numpy()]
+    for g, r, what in zip(got, (ref["a_act"], ref["y_perm"], ref["out"]),
+                          ("a_act", "y_perm", "out")):
+        if dtype == "f32":
+            assert np.abs(g - r).max() <= F32_ABS, what
+        else:
+            assert_bf16_close(g, r, what)
+    kept = np.diff(ref["offsets"])
+    if R > 1 and mode == "up":
+        assert n_add > 0
+        assert all(k % R == 0 or k == T for k in kept)
+    if R > T:
+        assert np.all(kept == T)  # every expert holds every token
+
+
+def _added_rows(tokens, x, w_gate, w_up, w_down, add_tok, add_exp, add_w):
+    """The added assignments' share of out[t] for the chosen tokens, in expert order."""
+    tokens = np.asarray(tokens, np.int64)
+    extra = np.zeros((tokens.size, w_down.shape[2]), np.float64)
+    for i, t in enumerate(tokens):
+        for j in np.nonzero(add_tok == t)[0]:
+            e = int(add_exp[j])
+            extra[i] += float(add_w[j]) * orc.expert_ffn(orc.as_f64(x[t:t + 1]), w_gate[e],
+                                                         w_up[e], w_down[e])[0]
+    return extra
+
+
+@pytest.mark.parametrize("mode", [1, 2], ids=["up", "nearest"])
+def test_forward_token_rounding_up_full_size(cuda_lib, mode):
+    """The Mixtral-like workload rounded up or to the nearest 128-row tile, routed from x:
+    the discrete intermediates in full, the layer output on sampled tokens (a token that
+    gained an expert among them)."""
+    tdr = cuda_lib
+    cfg = mi.CONFIGS["mixtral_bf16"]
+    inp = inputs_for(cfg)
+    R = 128
+    s = tdr.make_shape(cfg.T, cfg.d, cfg.E, cfg.K, cfg.n, 0.0, True, torch.bfloat16,
+                       tile_round=R, tile_round_mode=mode)
+    out, ws = tdr.forward(s, cuda(inp.x), cuda(inp.w_r), cuda(inp.w_gate), cuda(inp.w_up),
+                          cuda(inp.w_down))
+    torch.cuda.synchronize()
+    assert_status_ok(tdr)
+    v = tdr.workspace_views(s, ws)
+    lg = v["logits"].cpu().numpy()
+    ids_ref, _ = orc.route(lg, cfg.K, True)
+    np.testing.assert_array_equal(v["topk_ids"].cpu().numpy(), ids_ref)
+    keep, add_tok, add_exp = orc.tile_round_select(ids_ref, lg, cfg.E, R,
+                                                   {1: "up", 2: "nearest"}[mode])
+    ids_ext = np.concatenate([np.where(keep, ids_ref, -1).reshape(-1), add_exp])
+    offsets, a2p, p2a = orc.permute_ext(ids_ext, cfg.E)
+    w_ref, add_w = orc.round_weights(lg, ids_ref, add_tok, add_exp, True)
+    np.testing.assert_array_equal(v["offsets"].cpu().numpy(), offsets)
+    np.testing.assert_array_equal(v["assign_to_perm"].cpu().numpy()[:a2p.size], a2p)
+    np.testing.assert_array_equal(v["add_tok"].cpu().numpy()[:add_tok.size], add_tok)
+    nk = int(offsets[-1])
+    np.testing.assert_array_equal(v["slot_token"].cpu().numpy()[:nk],
+                                  orc.slot_tokens(p2a, nk, cfg.K, cfg.T, add_tok))
+    assert np.abs(v["topk_w"].cpu().numpy().astype(np.float64) - w_ref).max() <= W_ABS
+    assert np.abs(v["add_w"].cpu().numpy()[:add_w.size] - add_w).max() <= W_ABS
+    assert add_tok.size > 0 and np.all(np.diff(offsets) % R == 0)
+    rng = np.random.default_rng(13)
+    tokens = np.unique(np.concatenate([rng.choice(cfg.T, size=10, replace=False),
+                                       add_tok[:3], np.nonzero((~keep).any(1))[0][:2]]))
+    ref_rows = orc.forward_rows(tokens, inp.x, inp.w_gate, inp.w_up, inp.w_down, ids_ref, w_ref,
+                                a2p[:cfg.T * cfg.K], cfg.K)
+    ref_rows += _added_rows(tokens, inp.x, inp.w_gate, inp.w_up, inp.w_down, add_tok, add_exp,
+                            add_w)
+    assert_bf16_close(out[torch.from_numpy(tokens).cuda()].float().cpu().numpy(), ref_rows,
+                      "rounded-up forward out")
+
+
+def test_token_rounding_up_rejected_where_it_cannot_apply(cuda_lib):
+    """Up and nearest run in moe_forward only: moe_dispatch and moe_forward_h refuse them."""
+    tdr = cuda_lib
+    T, d, E, K, n = 64, 64, 8, 2, 64
+    s = tdr.make_shape(T, d, E, K, n, 0.0, True, torch.bfloat16, tile_round=16,
+                       tile_round_mode=1)
+    lg = torch.randn(T, E, device="cuda")
+    with pytest.raises(tdr.MoEError):
+        tdr.dispatch(s, logits_in=lg)
+    x = torch.randn(T, d, device="cuda").to(torch.bfloat16)
+    wg = torch.randn(E, d, n, device="cuda").to(torch.bfloat16)
+    wd = torch.randn(E, n, d, device="cuda").to(torch.bfloat16)
+    with pytest.raises(tdr.MoEError):
+        tdr.forward_h(s, x, None, wg, wg, wd, logits_in=lg)
+
+
 # ------------------------------------------------------------------ backward (expert half)
 def _bwd_case(tdr, cfg, seed):
     inp = mi.make_inputs(cfg)

@@ -34,13 +34,15 @@ class moe_shape(ctypes.Structure):
                 ("K", ctypes.c_int32), ("n", ctypes.c_int32),
                 ("capacity_factor", ctypes.c_float), ("renormalize", ctypes.c_int32),
                 ("dtype", ctypes.c_int32), ("tile_round", ctypes.c_int32),
-                ("ffn_variant", ctypes.c_int32), ("route_topk", ctypes.c_int32)]
+                ("tile_round_mode", ctypes.c_int32), ("ffn_variant", ctypes.c_int32),
+                ("route_topk", ctypes.c_int32)]
 
 
 class moe_workspace_layout(ctypes.Structure):
     _fields_ = [(f, ctypes.c_size_t) for f in (
         "logits", "topk_ids", "topk_w", "counts", "offsets", "assign_to_perm",
         "perm_to_assign", "permute_scratch", "a_act", "y_perm", "round_ids", "round_counts",
+        "add_tok", "add_w", "add_ptr", "add_idx", "add_cursor", "slot_token", "n_assign",
         "total")]
 
 
@@ -123,8 +125,11 @@ def _check(code: int, where: str) -> None:
 
 def make_shape(T: int, d: int, E: int, K: int, n: int = 0, capacity_factor: float = 0.0,
                renormalize: bool = True, dtype=torch.bfloat16, tile_round: int = 0,
-               ffn_variant: int = 0, route_topk: int = 0) -> moe_shape:
-    """tile_round = R > 0 rounds each expert's kept count down to whole R-row tiles.
+               ffn_variant: int = 0, route_topk: int = 0,
+               tile_round_mode: int = 0) -> moe_shape:
+    """tile_round = R > 0 rounds each expert's count to whole R-row tiles: tile_round_mode
+    0 = down (drops its weakest assignments), 1 = up (adds the strongest tokens that did not
+    route to it), 2 = to the nearest tile; up and nearest run in moe_forward only.
     ffn_variant selects the bf16 grouped-GEMM tiles: 0 = automatic, 1 = single-CTA 128 x 256
     tiles, 2 = CTA-pair 256 x 256 tiles with the gate/up rows gathered in the GEMM, 3 = CTA
     pairs with the rows copied first (all compute the same result). route_topk selects the
@@ -132,7 +137,7 @@ def make_shape(T: int, d: int, E: int, K: int, n: int = 0, capacity_factor: floa
     2 = bitonic merges (E <= 64, K <= 8)."""
     dt = MOE_BF16 if dtype == torch.bfloat16 else MOE_F32
     return moe_shape(T, d, E, K, n, float(capacity_factor), 1 if renormalize else 0, dt,
-                     int(tile_round), int(ffn_variant), int(route_topk))
+                     int(tile_round), int(tile_round_mode), int(ffn_variant), int(route_topk))
 
 
 def _ptr(t: Optional[torch.Tensor]):
@@ -465,22 +470,31 @@ def workspace_views(shape: moe_shape, workspace: torch.Tensor) -> dict:
     """Typed views of moe_forward's intermediates inside its workspace."""
     L = forward_workspace_layout(shape)
     T, E, K, d, n = shape.T, shape.E, shape.K, shape.d, shape.n
-    A = T * K
+    A = int(L.n_assign)  # T * K, plus E * (R - 1) added entries when rounding up
     dt = _act_dtype(shape)
     eb = 2 if dt == torch.bfloat16 else 4
 
     def view(off, count, dtype, shp, esz):
         return workspace[off:off + count * esz].view(dtype).view(*shp)
 
-    return dict(logits=view(L.logits, T * E, torch.float32, (T, E), 4),
-                topk_ids=view(L.topk_ids, A, torch.int32, (T, K), 4),
-                topk_w=view(L.topk_w, A, torch.float32, (T, K), 4),
-                counts=view(L.counts, E, torch.int32, (E,), 4),
-                offsets=view(L.offsets, E + 1, torch.int32, (E + 1,), 4),
-                assign_to_perm=view(L.assign_to_perm, A, torch.int32, (A,), 4),
-                perm_to_assign=view(L.perm_to_assign, A, torch.int32, (A,), 4),
-                a_act=view(L.a_act, A * n, dt, (A, n), eb),
-                y_perm=view(L.y_perm, A * d, dt, (A, d), eb))
+    v = dict(logits=view(L.logits, T * E, torch.float32, (T, E), 4),
+             topk_ids=view(L.topk_ids, T * K, torch.int32, (T, K), 4),
+             topk_w=view(L.topk_w, T * K, torch.float32, (T, K), 4),
+             counts=view(L.counts, E, torch.int32, (E,), 4),
+             offsets=view(L.offsets, E + 1, torch.int32, (E + 1,), 4),
+             assign_to_perm=view(L.assign_to_perm, A, torch.int32, (A,), 4),
+             perm_to_assign=view(L.perm_to_assign, A, torch.int32, (A,), 4),
+             a_act=view(L.a_act, A * n, dt, (A, n), eb),
+             y_perm=view(L.y_perm, A * d, dt, (A, d), eb))
+    if A > T * K:  # rounding up or to the nearest tile
+        NA = A - T * K
+        v.update(round_ids=view(L.round_ids, A, torch.int32, (A,), 4),
+                 add_tok=view(L.add_tok, NA, torch.int32, (NA,), 4),
+                 add_w=view(L.add_w, NA, torch.float32, (NA,), 4),
+                 add_ptr=view(L.add_ptr, T + 1, torch.int32, (T + 1,), 4),
+                 add_idx=view(L.add_idx, NA, torch.int32, (NA,), 4),
+                 slot_token=view(L.slot_token, A, torch.int32, (A,), 4))
+    return v
 
 
 # ------------------------------------------------------------------ atomic experts

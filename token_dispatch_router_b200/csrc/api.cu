@@ -7,6 +7,7 @@
 #include <vector>
 
 #include "common.cuh"
+#include "round.cuh"
 
 namespace moe {
 
@@ -55,6 +56,34 @@ moe_status launch_permute_rounded(const moe_shape& s, const int32_t* ids, const 
                                   int32_t* counts, int32_t* offsets, int32_t* a2p, int32_t* p2a,
                                   const void* x, void* x_perm, void* scratch, int32_t* round_ids,
                                   int32_t* round_counts, cudaStream_t st);
+
+moe_status launch_round_select(const moe_shape& s, const int32_t* counts, const int32_t* offsets0,
+                               const int32_t* p2a0, const float* logits, int32_t* ids_ext,
+                               int32_t* add_tok, cudaStream_t st);
+moe_status launch_round_weights(const moe_shape& s, const float* logits, const int32_t* ids,
+                                const int32_t* ids_add, const int32_t* add_tok, int32_t* cursor,
+                                int32_t* add_ptr, int32_t* add_idx, float* topk_w, float* add_w,
+                                cudaStream_t st);
+moe_status launch_slot_tokens(const moe_shape& s, const int32_t* p2a, const int32_t* offsets,
+                              const int32_t* add_tok, int32_t* slot_tok, cudaStream_t st);
+moe_status launch_combine_added(const moe_shape& s, const void* y_perm, const int32_t* a2p,
+                                const float* topk_w, void* out, const int32_t* add_ptr,
+                                const int32_t* add_idx, const float* add_w, long long n_rows,
+                                cudaStream_t st);
+
+// Rounding up or to the nearest tile: added assignments beyond T * K.
+bool rounds_up(const moe_shape& s) { return s.tile_round > 1 && s.tile_round_mode != 0; }
+// The permutation over the extended assignment list runs as T * K + E * (R - 1)
+// one-assignment "tokens".
+moe_shape ext_shape(const moe_shape& s) {
+  moe_shape e = s;
+  e.T = s.T * s.K + s.E * (s.tile_round - 1);
+  e.K = 1;
+  e.capacity_factor = 0.f;
+  e.tile_round = 0;
+  e.tile_round_mode = 0;
+  return e;
+}
 
 // ------------------------------------------------------------------ device state
 __device__ unsigned int g_device_status;
@@ -159,6 +188,12 @@ moe_status check_shape(const moe_shape* s, bool need_d, bool need_ffn) {
   if (isnan(s->capacity_factor)) return MOE_ERR_INVALID_ARG;
   if (s->tile_round < 0 || (s->tile_round > 0 && s->capacity_factor > 0.f))
     return MOE_ERR_INVALID_ARG;  // token rounding and a capacity limit are exclusive
+  if (s->tile_round_mode < 0 || s->tile_round_mode > 2) return MOE_ERR_INVALID_ARG;
+  if (rounds_up(*s)) {  // added assignments: E * (R - 1) beyond T * K, int32 indices
+    if ((long long)s->T * s->K + (long long)s->E * (s->tile_round - 1) > 0x7fffffffLL)
+      return MOE_ERR_UNSUPPORTED;
+    if (s->T > kRoundUpMaxTokens) return MOE_ERR_UNSUPPORTED;
+  }
   if (s->ffn_variant < 0 || s->ffn_variant > 3) return MOE_ERR_INVALID_ARG;
   if (s->route_topk < 0 || s->route_topk > 2) return MOE_ERR_INVALID_ARG;
   if (need_d) {
@@ -172,7 +207,10 @@ moe_status check_shape(const moe_shape* s, bool need_d, bool need_ffn) {
 }
 
 bool layout_of(const moe_shape& s, moe_workspace_layout* L) {
-  const size_t T = (size_t)s.T, E = (size_t)s.E, K = (size_t)s.K, A = T * K;
+  const size_t T = (size_t)s.T, E = (size_t)s.E, K = (size_t)s.K;
+  const bool up = rounds_up(s);
+  const size_t NA = up ? E * (size_t)(s.tile_round - 1) : 0;  // added assignments at most
+  const size_t A = T * K + NA;                                 // entries of both maps
   const size_t eb = (size_t)elem_bytes(s);
   size_t o = 0;
   L->logits = o;
@@ -190,7 +228,7 @@ bool layout_of(const moe_shape& s, moe_workspace_layout* L) {
   L->perm_to_assign = o;
   o = align256(o + A * 4);
   L->permute_scratch = o;
-  o = align256(o + permute_scratch_bytes(s));
+  o = align256(o + permute_scratch_bytes(up ? ext_shape(s) : s));
   L->a_act = o;
   o = align256(o + A * (size_t)s.n * eb);
   L->y_perm = o;
@@ -199,6 +237,19 @@ bool layout_of(const moe_shape& s, moe_workspace_layout* L) {
   if (s.tile_round > 0) o = align256(o + A * 4);
   L->round_counts = o;
   if (s.tile_round > 0) o = align256(o + E * 4);
+  L->add_tok = o;
+  if (up) o = align256(o + NA * 4);
+  L->add_w = o;
+  if (up) o = align256(o + NA * 4);
+  L->add_ptr = o;
+  if (up) o = align256(o + (T + 1) * 4);
+  L->add_idx = o;
+  if (up) o = align256(o + NA * 4);
+  L->add_cursor = o;
+  if (up) o = align256(o + T * 4);
+  L->slot_token = o;
+  if (up) o = align256(o + A * 4);
+  L->n_assign = A;
   L->total = o;
   return true;
 }
@@ -220,6 +271,65 @@ int gateup_mode(const moe_shape& s) { return s.ffn_variant == 2 ? 1 : s.ffn_vari
 
 namespace moe {
 namespace {
+// The layer forward with token rounding up or to the nearest tile (reading in moe.h).
+// 1. route; 2. the uncapped permutation (raw counts, each expert's assignments in token
+// order); 3. the extended id list: the routed ids, then E * (R - 1) entries of -1, in which
+// each expert drops (rounding down) or gains (rounding up) assignments; 4. the permutation
+// of the extended list as T * K + E * (R - 1) one-assignment rows; 5. the token-major lists
+// of the added assignments and the weights over each enlarged selection; 6. the token of
+// every expert-major slot; 7. the grouped FFN over those rows; 8. combine with the added
+// slots.
+moe_status launch_forward_rounded_up(const moe_shape& s, const void* x, const void* w_r,
+                                     const float* bias, const float* logits_in,
+                                     const void* w_gate, const void* w_up, const void* w_down,
+                                     void* out, uint8_t* ws, const moe_workspace_layout& L,
+                                     bool pair_down, int gateup_mode, cudaStream_t st) {
+  float* logits = (float*)(ws + L.logits);
+  int32_t* ids = (int32_t*)(ws + L.topk_ids);
+  float* w = (float*)(ws + L.topk_w);
+  int32_t* counts = (int32_t*)(ws + L.counts);
+  int32_t* offsets = (int32_t*)(ws + L.offsets);
+  int32_t* a2p = (int32_t*)(ws + L.assign_to_perm);
+  int32_t* p2a = (int32_t*)(ws + L.perm_to_assign);
+  int32_t* ids_ext = (int32_t*)(ws + L.round_ids);
+  int32_t* add_tok = (int32_t*)(ws + L.add_tok);
+  int32_t* slot_tok = (int32_t*)(ws + L.slot_token);
+  const size_t A0 = (size_t)s.T * s.K, NA = (size_t)s.E * (s.tile_round - 1);
+  moe_status r;
+  if ((r = moe_route(&s, x, w_r, bias, logits_in, logits, ids, w, (moe_stream_t)st)) != MOE_OK)
+    return r;
+  if ((r = launch_permute(s, ids, counts, offsets, a2p, p2a, nullptr, nullptr,
+                          ws + L.permute_scratch, st)) != MOE_OK)
+    return r;
+  if (cudaMemcpyAsync(ids_ext, ids, A0 * sizeof(int32_t), cudaMemcpyDeviceToDevice, st) !=
+          cudaSuccess ||
+      cudaMemsetAsync(ids_ext + A0, 0xff, NA * sizeof(int32_t), st) != cudaSuccess ||
+      cudaMemsetAsync(add_tok, 0xff, NA * sizeof(int32_t), st) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  if ((r = launch_round_select(s, counts, offsets, p2a, logits, ids_ext, add_tok, st)) != MOE_OK)
+    return r;
+  const moe_shape xs = ext_shape(s);
+  if ((r = launch_permute(xs, ids_ext, (int32_t*)(ws + L.round_counts), offsets, a2p, p2a,
+                          nullptr, nullptr, ws + L.permute_scratch, st)) != MOE_OK)
+    return r;
+  if ((r = launch_round_weights(s, logits, ids, ids_ext + A0, add_tok,
+                                (int32_t*)(ws + L.add_cursor), (int32_t*)(ws + L.add_ptr),
+                                (int32_t*)(ws + L.add_idx), w, (float*)(ws + L.add_w), st)) !=
+      MOE_OK)
+    return r;
+  if ((r = launch_slot_tokens(s, p2a, offsets, add_tok, slot_tok, st)) != MOE_OK) return r;
+  // the grouped FFN sees the extended list as one-assignment rows whose token is slot_tok[p]
+  r = s.dtype == MOE_BF16 ? launch_ffn_tc_mixed(xs, x, offsets, slot_tok, w_gate, w_up, w_down,
+                                                ws + L.a_act, ws + L.y_perm, gateup_mode,
+                                                pair_down, nullptr, st)
+                          : launch_ffn_simt(xs, x, offsets, slot_tok, w_gate, w_up, w_down,
+                                            ws + L.a_act, ws + L.y_perm, st);
+  if (r != MOE_OK) return r;
+  return launch_combine_added(s, ws + L.y_perm, a2p, w, out, (const int32_t*)(ws + L.add_ptr),
+                              (const int32_t*)(ws + L.add_idx), (const float*)(ws + L.add_w),
+                              (long long)(A0 + NA), st);
+}
+
 moe_status forward_impl(const moe_shape* s, const void* x, const void* w_r, const float* bias,
                         const float* logits_in, const void* w_gate, const void* w_up,
                         const void* w_down, void* out, void* h_out, void* workspace,
@@ -241,6 +351,14 @@ moe_status forward_impl(const moe_shape* s, const void* x, const void* w_r, cons
   int32_t* offsets = (int32_t*)(ws + L.offsets);
   int32_t* a2p = (int32_t*)(ws + L.assign_to_perm);
   int32_t* p2a = (int32_t*)(ws + L.perm_to_assign);
+  if (rounds_up(*s)) {  // added assignments: the extended path
+    if (h_out != nullptr) return MOE_ERR_UNSUPPORTED;
+    if (s->dtype == MOE_BF16 &&
+        (!aligned16(x) || !aligned16(w_gate) || !aligned16(w_up) || !aligned16(w_down)))
+      return MOE_ERR_INVALID_ARG;
+    return launch_forward_rounded_up(*s, x, w_r, bias, logits_in, w_gate, w_up, w_down, out, ws,
+                                     L, use_pair_down(*s), gateup_mode(*s), st);
+  }
   if (s->tile_round > 0) {
     if ((r = moe_route(s, x, w_r, bias, logits_in, logits, ids, w, stream)) != MOE_OK) return r;
     if ((r = launch_permute_rounded(*s, ids, logits, counts, offsets, a2p, p2a, nullptr, nullptr,
@@ -379,6 +497,7 @@ moe_status moe_dispatch(const moe_shape* s, const void* x, const void* w_r, cons
   if (!topk_ids || !topk_w || !counts || !offsets || !assign_to_perm || !perm_to_assign)
     return MOE_ERR_INVALID_ARG;
   if (gather && (x == nullptr || !aligned16(x) || !aligned16(x_perm))) return MOE_ERR_INVALID_ARG;
+  if (rounds_up(*s)) return MOE_ERR_UNSUPPORTED;  // added assignments: moe_forward only
   if (s->tile_round > 0) {  // route, then the rounded permutation on the logits it saw
     const float* lg = logits_in != nullptr ? logits_in : logits_out;
     if (lg == nullptr) return MOE_ERR_INVALID_ARG;  // rounding reads the logits

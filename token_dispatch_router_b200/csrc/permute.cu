@@ -28,6 +28,7 @@
 
 #include "tc_ptx.cuh"
 #include "topk.cuh"
+#include "round.cuh"
 
 namespace moe {
 
@@ -948,30 +949,22 @@ __device__ __forceinline__ uint64_t round_key(const int32_t* p2a, const float* l
   return ((uint64_t)u << 32) | (uint64_t)(0xffffffffu - (uint32_t)t);
 }
 
-__global__ void __launch_bounds__(256) tile_round_kernel(const int32_t* __restrict__ counts,
-                                                         const int32_t* __restrict__ offsets,
-                                                         const int32_t* __restrict__ p2a,
-                                                         const float* __restrict__ logits,
-                                                         int K, int E, int R,
-                                                         int32_t* __restrict__ round_ids) {
-  __shared__ unsigned hist[256];
-  __shared__ unsigned long long s_pre;
-  __shared__ int s_need;
-  pdl_wait();  // the previous kernel in the stream has completed
-  pdl_trigger();
-  const int e = blockIdx.x, tid = threadIdx.x;
-  const int c = counts[e];
-  if (c < R || c % R == 0) return;  // uniform across the CTA
-  const int off = offsets[e];
+// The need-th smallest (1-based) of the distinct 64-bit keys key_of(j) over the j < n for
+// which key_of returns true: an 8-pass radix select, 8 bits a pass, a 256-bin shared
+// histogram, the bin found by warp 0's shuffle scan and ballot. Every thread of the
+// 256-thread CTA calls it.
+template <typename KeyOf>
+__device__ uint64_t radix_select_u64(int n, int need, KeyOf key_of, unsigned* hist,
+                                     unsigned long long* s_pre, int* s_need) {
+  const int tid = threadIdx.x;
   uint64_t pre = 0;
-  int need = c % R;  // rank of the wanted key among the keys matching `pre` so far
   for (int d = 7; d >= 0; --d) {
     const uint64_t hi = d == 7 ? 0ull : (~0ull << (8 * (d + 1)));
     hist[tid] = 0;
     __syncthreads();
-    for (int j = tid; j < c; j += 256) {
-      const uint64_t key = round_key(p2a, logits, off + j, K, E, e);
-      if (((key ^ pre) & hi) == 0) atomicAdd(&hist[(key >> (8 * d)) & 255u], 1u);
+    for (int j = tid; j < n; j += 256) {
+      uint64_t key;
+      if (key_of(j, key) && ((key ^ pre) & hi) == 0) atomicAdd(&hist[(key >> (8 * d)) & 255u], 1u);
     }
     __syncthreads();
     if (tid < 32) {  // warp 0: the bin where the running count reaches `need`
@@ -1001,19 +994,270 @@ __global__ void __launch_bounds__(256) tile_round_kernel(const int32_t* __restri
           }
           run += v[q];
         }
-        s_need = need - (int)run;
-        s_pre = pre | ((uint64_t)b << (8 * d));
+        *s_need = need - (int)run;
+        *s_pre = pre | ((uint64_t)b << (8 * d));
       }
     }
     __syncthreads();
-    pre = s_pre;
-    need = s_need;
+    pre = *s_pre;
+    need = *s_need;
     __syncthreads();
   }
-  // `pre` is the m-th smallest key: drop it and every smaller one
+  return pre;
+}
+
+__global__ void __launch_bounds__(256) tile_round_kernel(const int32_t* __restrict__ counts,
+                                                         const int32_t* __restrict__ offsets,
+                                                         const int32_t* __restrict__ p2a,
+                                                         const float* __restrict__ logits,
+                                                         int K, int E, int R,
+                                                         int32_t* __restrict__ round_ids) {
+  __shared__ unsigned hist[256];
+  __shared__ unsigned long long s_pre;
+  __shared__ int s_need;
+  pdl_wait();  // the previous kernel in the stream has completed
+  pdl_trigger();
+  const int e = blockIdx.x, tid = threadIdx.x;
+  const int c = counts[e];
+  if (c < R || c % R == 0) return;  // uniform across the CTA
+  const int off = offsets[e];
+  // the (c mod R)-th smallest key: it and every smaller one are dropped
+  const uint64_t pre = radix_select_u64(
+      c, c % R,
+      [&](int j, uint64_t& key) {
+        key = round_key(p2a, logits, off + j, K, E, e);
+        return true;
+      },
+      hist, &s_pre, &s_need);
   for (int j = tid; j < c; j += 256) {
     const uint64_t key = round_key(p2a, logits, off + j, K, E, e);
     if (key <= pre) round_ids[p2a[off + j]] = -1;
+  }
+}
+
+// Rounding up or to the nearest tile (reading in moe.h): the tokens expert e gains, as a
+// count, from its routed count c (0 when it rounds down or is whole).
+__device__ __forceinline__ int round_adds(int c, int R, int mode, int T) {
+  const int r = c % R;
+  if (r == 0 || !(mode == 1 || (mode == 2 && r > R - r))) return 0;
+  return min(R - r, T - c);
+}
+
+// One CTA per expert, after an uncapped permutation (e's routed assignments in token order
+// at p2a0[offsets0[e] ...]). An expert that rounds down drops its weakest assignments in the
+// extended id list (as tile_round_kernel); one that rounds up gains the m best tokens that
+// did not route to it: a shared bitmap marks its routed tokens, each other token's key is
+// (its logit for e as an order-preserving integer) << 32 | (2^32 - 1 - t), so larger keys
+// are stronger and all distinct; a radix select finds the m-th largest, and the tokens at or
+// above it are written in ascending order to add_tok[base ...] and as e into
+// ids_ext[T*K + base ...], base = the tokens gained by the experts before e.
+__global__ void __launch_bounds__(256) round_select_kernel(
+    const int32_t* __restrict__ counts, const int32_t* __restrict__ offsets0,
+    const int32_t* __restrict__ p2a0, const float* __restrict__ logits, int T, int K, int E,
+    int R, int mode, int32_t* __restrict__ ids_ext, int32_t* __restrict__ add_tok) {
+  __shared__ uint32_t routed[kRoundUpMaxTokens / 32];
+  __shared__ unsigned hist[256];
+  __shared__ unsigned long long s_pre;
+  __shared__ int s_need, s_base;
+  __shared__ int wsum[8];
+  pdl_wait();  // the previous kernel in the stream has completed
+  pdl_trigger();
+  const int e = blockIdx.x, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int c = counts[e];
+  const int r = c % R;
+  if (r == 0) return;  // uniform across the CTA
+  const int off = offsets0[e];
+  const bool up = mode == 1 || (mode == 2 && r > R - r);
+  if (!up) {
+    if (c < R) return;
+    const uint64_t pre = radix_select_u64(
+        c, r,
+        [&](int j, uint64_t& key) {
+          key = round_key(p2a0, logits, off + j, K, E, e);
+          return true;
+        },
+        hist, &s_pre, &s_need);
+    for (int j = tid; j < c; j += 256) {
+      const uint64_t key = round_key(p2a0, logits, off + j, K, E, e);
+      if (key <= pre) ids_ext[p2a0[off + j]] = -1;
+    }
+    return;
+  }
+  const int m = min(R - r, T - c);
+  if (tid == 0) s_base = 0;
+  for (int i = tid; i < T / 32 + 1 && i < kRoundUpMaxTokens / 32; i += 256) routed[i] = 0;
+  __syncthreads();
+  for (int i = tid; i < e; i += 256) atomicAdd(&s_base, round_adds(counts[i], R, mode, T));
+  for (int j = tid; j < c; j += 256) {
+    const int t = p2a0[off + j] / K;
+    atomicOr(&routed[t >> 5], 1u << (t & 31));
+  }
+  __syncthreads();
+  const int base = s_base;
+  if (m <= 0) return;
+  auto key_of = [&](int t, uint64_t& key) {
+    if ((routed[t >> 5] >> (t & 31)) & 1u) return false;
+    float v = logits[(size_t)t * E + e];
+    if (v == 0.f) v = 0.f;  // -0 and +0 are one value
+    uint32_t u = __float_as_uint(v);
+    u = (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+    key = ((uint64_t)u << 32) | (uint64_t)(0xffffffffu - (uint32_t)t);
+    return true;
+  };
+  // the m-th largest of the T - c candidate keys = their (T - c - m + 1)-th smallest
+  const uint64_t theta = radix_select_u64(T, T - c - m + 1, key_of, hist, &s_pre, &s_need);
+  // the chosen tokens in ascending order, 256 at a time
+  int run = 0;
+  for (int t0 = 0; t0 < T; t0 += 256) {
+    const int t = t0 + tid;
+    uint64_t key = 0;
+    const bool chosen = t < T && key_of(t, key) && key >= theta;
+    const unsigned bal = __ballot_sync(0xffffffffu, chosen);
+    if (lane == 0) wsum[warp] = __popc(bal);
+    __syncthreads();
+    int before = run, total = 0;
+    for (int w = 0; w < 8; ++w) {
+      if (w < warp) before += wsum[w];
+      total += wsum[w];
+    }
+    if (chosen) {
+      const int pos = base + before + __popc(bal & lanemask_lt());
+      add_tok[pos] = t;
+      ids_ext[(size_t)T * K + pos] = e;
+    }
+    run += total;
+    __syncthreads();
+  }
+}
+
+// Token-major view of the added assignments: counts per token (atomics on counters that
+// start at zero; the counts do not depend on the order).
+__global__ void __launch_bounds__(256) round_count_kernel(const int32_t* __restrict__ ids_add,
+                                                          const int32_t* __restrict__ add_tok,
+                                                          int NA, int T, int32_t* cnt,
+                                                          unsigned* status) {
+  pdl_wait();  // the previous kernel in the stream has completed
+  pdl_trigger();
+  const int j = blockIdx.x * 256 + threadIdx.x;
+  if (j >= NA || ids_add[j] < 0) return;
+  const int t = add_tok[j];
+  if (t < 0 || t >= T) {
+    report(status, MOE_ERR_DEVICE_INDEX);
+    return;
+  }
+  atomicAdd(&cnt[t], 1);
+}
+
+// add_ptr = exclusive scan of the per-token counts (one CTA of 1024 threads, each scanning a
+// contiguous run); the counters are zeroed again for the fill.
+__global__ void __launch_bounds__(1024) round_scan_kernel(int32_t* cnt, int T,
+                                                          int32_t* __restrict__ add_ptr) {
+  __shared__ int wsum[32];
+  pdl_wait();  // the previous kernel in the stream has completed
+  pdl_trigger();
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int per = (T + 1023) / 1024;
+  const int b = tid * per, e = min(T, b + per);
+  int sum = 0;
+  for (int t = b; t < e; ++t) sum += cnt[t];
+  int incl = sum;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += y;
+  }
+  if (lane == 31) wsum[warp] = incl;
+  __syncthreads();
+  if (warp == 0) {
+    int v = wsum[lane], iv = v;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, iv, o);
+      if (lane >= o) iv += y;
+    }
+    wsum[lane] = iv - v;
+  }
+  __syncthreads();
+  int run = wsum[warp] + incl - sum;
+  for (int t = b; t < e; ++t) {
+    add_ptr[t] = run;
+    run += cnt[t];
+    cnt[t] = 0;
+  }
+  if (tid == 1023) add_ptr[T] = run;
+}
+
+// Each added assignment into its token's list (atomic cursors: any order here, sorted by
+// the weights kernel).
+__global__ void __launch_bounds__(256) round_fill_kernel(const int32_t* __restrict__ ids_add,
+                                                         const int32_t* __restrict__ add_tok,
+                                                         int NA, int T,
+                                                         const int32_t* __restrict__ add_ptr,
+                                                         int32_t* cursor,
+                                                         int32_t* __restrict__ add_idx) {
+  pdl_wait();  // the previous kernel in the stream has completed
+  pdl_trigger();
+  const int j = blockIdx.x * 256 + threadIdx.x;
+  if (j >= NA || ids_add[j] < 0) return;
+  const int t = add_tok[j];
+  if (t < 0 || t >= T) return;
+  add_idx[add_ptr[t] + atomicAdd(&cursor[t], 1)] = j;
+}
+
+// Weights of a token that gained assignments, over its enlarged selection (reading in
+// moe.h): its added list sorted ascending (= expert order), then, renormalised,
+// w = exp(l - l_top) / (sum over the K routed and the added of exp(l_j - l_top)), summed in
+// slot order then list order; plain softmax: the added ones get softmax(l) over all E, the
+// routed ones keep theirs. One thread per token.
+__global__ void __launch_bounds__(256) round_weights_kernel(
+    const float* __restrict__ logits, const int32_t* __restrict__ ids, int T, int K, int E,
+    int renorm, const int32_t* __restrict__ ids_add, const int32_t* __restrict__ add_ptr,
+    int32_t* __restrict__ add_idx, float* __restrict__ topk_w, float* __restrict__ add_w) {
+  pdl_wait();  // the previous kernel in the stream has completed
+  pdl_trigger();
+  const int t = blockIdx.x * 256 + threadIdx.x;
+  if (t >= T) return;
+  const int lo = add_ptr[t], hi = add_ptr[t + 1];
+  if (hi == lo) return;
+  for (int i = lo + 1; i < hi; ++i) {  // insertion sort (a token gains a few at most)
+    const int v = add_idx[i];
+    int k = i - 1;
+    while (k >= lo && add_idx[k] > v) {
+      add_idx[k + 1] = add_idx[k];
+      --k;
+    }
+    add_idx[k + 1] = v;
+  }
+  const float* lg = logits + (size_t)t * E;
+  const float top = lg[ids[(size_t)t * K]];
+  if (renorm) {
+    float den = 0.f;
+    for (int k = 0; k < K; ++k) den += expf(lg[ids[(size_t)t * K + k]] - top);
+    for (int i = lo; i < hi; ++i) den += expf(lg[ids_add[add_idx[i]]] - top);
+    for (int k = 0; k < K; ++k)
+      topk_w[(size_t)t * K + k] = expf(lg[ids[(size_t)t * K + k]] - top) / den;
+    for (int i = lo; i < hi; ++i) add_w[add_idx[i]] = expf(lg[ids_add[add_idx[i]]] - top) / den;
+  } else {
+    float den = 0.f;  // the plain softmax over all E (the top logit is the maximum)
+    for (int q = 0; q < E; ++q) den += expf(lg[q] - top);
+    for (int i = lo; i < hi; ++i) add_w[add_idx[i]] = expf(lg[ids_add[add_idx[i]]] - top) / den;
+  }
+}
+
+// The token of every kept expert-major slot: a < T*K is token a / K, an added a = T*K + j
+// is add_tok[j].
+__global__ void __launch_bounds__(256) slot_token_kernel(const int32_t* __restrict__ p2a,
+                                                         const int32_t* __restrict__ n_kept_ptr,
+                                                         int T, int K,
+                                                         const int32_t* __restrict__ add_tok,
+                                                         int32_t* __restrict__ slot_tok) {
+  pdl_wait();  // the previous kernel in the stream has completed
+  pdl_trigger();
+  const int n_kept = *n_kept_ptr;
+  const long long A0 = (long long)T * K;
+  for (int p = blockIdx.x * 256 + threadIdx.x; p < n_kept; p += gridDim.x * 256) {
+    const long long a = p2a[p];
+    slot_tok[p] = a < A0 ? (int32_t)(a / K) : add_tok[a - A0];
   }
 }
 
@@ -1040,6 +1284,54 @@ moe_status launch_permute_rounded(const moe_shape& s, const int32_t* ids, const 
   if ((r = launch_end(K_TILE_ROUND, st)) != MOE_OK) return r;
   // 3. the final permutation of what is kept (its counts are the kept ones: not returned)
   return launch_permute(s, round_ids, round_counts, offsets, a2p, p2a, x, x_perm, scratch, st);
+}
+
+moe_status launch_round_select(const moe_shape& s, const int32_t* counts, const int32_t* offsets0,
+                               const int32_t* p2a0, const float* logits, int32_t* ids_ext,
+                               int32_t* add_tok, cudaStream_t st) {
+  if (s.T > kRoundUpMaxTokens) return MOE_ERR_UNSUPPORTED;
+  launch_begin(K_TILE_ROUND, st);
+  launch_kernel(round_select_kernel, dim3((unsigned)s.E), dim3(256), 0, st, 1, counts, offsets0,
+                p2a0, logits, s.T, s.K, s.E, s.tile_round, s.tile_round_mode, ids_ext, add_tok);
+  return launch_end(K_TILE_ROUND, st);
+}
+
+moe_status launch_round_weights(const moe_shape& s, const float* logits, const int32_t* ids,
+                                const int32_t* ids_add, const int32_t* add_tok, int32_t* cursor,
+                                int32_t* add_ptr, int32_t* add_idx, float* topk_w, float* add_w,
+                                cudaStream_t st) {
+  const int NA = s.E * (s.tile_round - 1);
+  moe_status r;
+  if (cudaMemsetAsync(cursor, 0, sizeof(int32_t) * (size_t)s.T, st) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  const unsigned gb = (unsigned)((NA + 255) / 256);
+  launch_begin(K_TILE_ROUND, st);
+  launch_kernel(round_count_kernel, dim3(gb), dim3(256), 0, st, 1, ids_add, add_tok, NA, s.T,
+                cursor, device_status_ptr());
+  if ((r = launch_end(K_TILE_ROUND, st)) != MOE_OK) return r;
+  launch_begin(K_TILE_ROUND, st);
+  launch_kernel(round_scan_kernel, dim3(1), dim3(1024), 0, st, 1, cursor, s.T, add_ptr);
+  if ((r = launch_end(K_TILE_ROUND, st)) != MOE_OK) return r;
+  launch_begin(K_TILE_ROUND, st);
+  launch_kernel(round_fill_kernel, dim3(gb), dim3(256), 0, st, 1, ids_add, add_tok, NA, s.T,
+                (const int32_t*)add_ptr, cursor, add_idx);
+  if ((r = launch_end(K_TILE_ROUND, st)) != MOE_OK) return r;
+  launch_begin(K_TILE_ROUND, st);
+  launch_kernel(round_weights_kernel, dim3((unsigned)((s.T + 255) / 256)), dim3(256), 0, st, 1,
+                logits, ids, s.T, s.K, s.E, s.renormalize, ids_add, (const int32_t*)add_ptr,
+                add_idx, topk_w, add_w);
+  return launch_end(K_TILE_ROUND, st);
+}
+
+moe_status launch_slot_tokens(const moe_shape& s, const int32_t* p2a, const int32_t* offsets,
+                              const int32_t* add_tok, int32_t* slot_tok, cudaStream_t st) {
+  const long long A = (long long)s.T * s.K + (long long)s.E * (s.tile_round - 1);
+  long long blocks = (A + 255) / 256;
+  if (blocks > (long long)sm_count() * 8) blocks = (long long)sm_count() * 8;
+  launch_begin(K_TILE_ROUND, st);
+  launch_kernel(slot_token_kernel, dim3((unsigned)blocks), dim3(256), 0, st, 1, p2a,
+                offsets + s.E, s.T, s.K, add_tok, slot_tok);
+  return launch_end(K_TILE_ROUND, st);
 }
 
 // ------------------------------------------------------------------ no-allocation variant
