@@ -60,7 +60,8 @@ def parse():
                          "decode, rounding, backward, atomic-expert or other-workload figures)")
     ap.add_argument("--no-workloads", action="store_true",
                     help="skip the fine-grained and skewed workload figures")
-    ap.add_argument("--only", choices=["atomic_experts", "backward", "dispatch", "decode"],
+    ap.add_argument("--only", choices=["atomic_experts", "backward", "dispatch", "decode",
+                                       "rounding"],
                     default=None,
                     help="run one secondary figure alone and print it (for profiling)")
     return ap.parse_args()
@@ -493,19 +494,24 @@ def decode_dispatch(tdr, world, Ts=(64, 256, 512, 1024)):
 
 
 def token_rounding_figure(tdr, cfg, x, w_r, wg, wu, wd, bias, world, R=128, rounds=5, per=10):
-    """The layer with tile-aware token rounding (each expert's kept rows rounded down to whole
-    R-row tiles, its weakest assignments dropped) against the plain layer: blocks of `per`
-    steps alternate between the two `rounds` times (the power-capped clock drifts), CUDA
-    events; reports both step times, the kept share of the assignments and the 128-row
-    tile rows the gate/up GEMM computes in each case."""
+    """The layer with tile-aware token rounding to whole R-row tiles, in each direction (down:
+    an expert's weakest assignments dropped; up: the strongest tokens that did not route to it
+    added; nearest: whichever is closer), against the plain layer: blocks of `per` steps
+    alternate between the four `rounds` times (the power-capped clock drifts), CUDA events;
+    reports each step time, the rows each expert-major list holds (kept plus added) and the
+    128-row tile rows the gate/up GEMM computes in each case."""
     if cfg.capacity_factor > 0:
         return None
     dev = x.device
     dt = x.dtype
     out = torch.empty(cfg.T, cfg.d, dtype=dt, device=dev)
     shapes = {"plain": tdr.make_shape(cfg.T, cfg.d, cfg.E, cfg.K, cfg.n, 0.0, True, dt),
-              "rounded": tdr.make_shape(cfg.T, cfg.d, cfg.E, cfg.K, cfg.n, 0.0, True, dt,
-                                        tile_round=R)}
+              "down": tdr.make_shape(cfg.T, cfg.d, cfg.E, cfg.K, cfg.n, 0.0, True, dt,
+                                     tile_round=R),
+              "up": tdr.make_shape(cfg.T, cfg.d, cfg.E, cfg.K, cfg.n, 0.0, True, dt,
+                                   tile_round=R, tile_round_mode=1),
+              "nearest": tdr.make_shape(cfg.T, cfg.d, cfg.E, cfg.K, cfg.n, 0.0, True, dt,
+                                        tile_round=R, tile_round_mode=2)}
     wss = {k: torch.empty(tdr.forward_workspace_size(v), dtype=torch.uint8, device=dev)
            for k, v in shapes.items()}
     ms = {k: 0.0 for k in shapes}
@@ -522,6 +528,14 @@ def token_rounding_figure(tdr, cfg, x, w_r, wg, wu, wd, bias, world, R=128, roun
             e1.record()
             torch.cuda.synchronize()
             ms[k] += e0.elapsed_time(e1)
+    kern = {}
+    for k in shapes:  # per-kernel device time, a separate pass under the event profiler
+        prof = tdr.Profiler()
+        with prof:
+            for _ in range(per):
+                tdr.forward(shapes[k], x, w_r, wg, wu, wd, bias=bias, out=out, workspace=wss[k])
+            torch.cuda.synchronize()
+        kern[k] = {n: round(v[1] / per * 1e3, 1) for n, v in prof.results().items()}
     if tdr.device_status() != 0:
         raise RuntimeError("device status set during the token-rounding runs")
     res = {}
@@ -532,12 +546,14 @@ def token_rounding_figure(tdr, cfg, x, w_r, wg, wu, wd, bias, world, R=128, roun
         res[k] = {"ms_per_step": round(step, 4),
                   "tokens_per_s": cfg.T * world / (step / 1e3),
                   "kept_assignments": int(offs[-1]),
-                  "gemm_tile_rows": int(sum(-(-int(c) // 128) * 128 for c in kept))}
+                  "gemm_tile_rows": int(sum(-(-int(c) // 128) * 128 for c in kept)),
+                  "kernels_us": kern[k]}
     res["R"] = R
-    res["kept_share"] = round(res["rounded"]["kept_assignments"] / (cfg.T * cfg.K), 4)
-    res["speedup"] = round(res["plain"]["ms_per_step"] / res["rounded"]["ms_per_step"], 4)
-    res["note"] = ("a different layer output: the dropped assignments add nothing; same "
-                   "weights, inputs and kernels otherwise")
+    for k in ("down", "up", "nearest"):
+        res[k]["row_share"] = round(res[k]["kept_assignments"] / (cfg.T * cfg.K), 4)
+        res[k]["speedup"] = round(res["plain"]["ms_per_step"] / res[k]["ms_per_step"], 4)
+    res["note"] = ("each a different layer output: dropped assignments add nothing, added ones "
+                   "add their weighted expert output; same weights, inputs and kernels otherwise")
     return res
 
 
@@ -811,6 +827,11 @@ def run_ours(args, rank, world, local):
     def step():
         tdr.forward(s, x, w_r, wg, wu, wd, bias=bias, out=out, workspace=ws)
 
+    if args.only == "rounding":
+        fig = token_rounding_figure(tdr, cfg, x, w_r, wg, wu, wd, bias, world)
+        if rank == 0:
+            print(json.dumps({"token_rounding": fig}), flush=True)
+        return
     if args.only == "backward":
         peaks = load_peaks()[0]
         peak_t = float(peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"]))
@@ -974,8 +995,10 @@ def run_ours(args, rank, world, local):
                                     "scatter_out_us": ae["scatter_add_output"]["output_us"]}
     if tr:
         result["token_rounding"] = {"R": tr["R"], "plain_ms": tr["plain"]["ms_per_step"],
-                                    "rounded_ms": tr["rounded"]["ms_per_step"],
-                                    "speedup": tr["speedup"], "kept_share": tr["kept_share"]}
+                                    **{f"{k}_ms": tr[k]["ms_per_step"]
+                                       for k in ("down", "up", "nearest")},
+                                    **{f"{k}_rows": tr[k]["row_share"]
+                                       for k in ("down", "up", "nearest")}}
     if dd:
         result["decode_dispatch_us"] = {"cols": "two_calls,dispatch_rounds,dispatch_bitonic",
                                         **{k.split("=")[1]: [v["two_calls_us"],

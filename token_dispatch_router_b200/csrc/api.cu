@@ -60,12 +60,13 @@ moe_status launch_permute_rounded(const moe_shape& s, const int32_t* ids, const 
 moe_status launch_round_select(const moe_shape& s, const int32_t* counts, const int32_t* offsets0,
                                const int32_t* p2a0, const float* logits, int32_t* ids_ext,
                                int32_t* add_tok, cudaStream_t st);
-moe_status launch_round_weights(const moe_shape& s, const float* logits, const int32_t* ids,
-                                const int32_t* ids_add, const int32_t* add_tok, int32_t* cursor,
-                                int32_t* add_ptr, int32_t* add_idx, float* topk_w, float* add_w,
-                                cudaStream_t st);
-moe_status launch_slot_tokens(const moe_shape& s, const int32_t* p2a, const int32_t* offsets,
-                              const int32_t* add_tok, int32_t* slot_tok, cudaStream_t st);
+moe_status launch_round_lists(const moe_shape& s, const int32_t* ids_add, const int32_t* add_tok,
+                              int32_t* cursor, int32_t* add_ptr, int32_t* add_idx,
+                              cudaStream_t st);
+moe_status launch_round_finish(const moe_shape& s, const int32_t* p2a, const int32_t* offsets,
+                               const float* logits, const int32_t* ids, const int32_t* ids_add,
+                               const int32_t* add_tok, const int32_t* add_ptr, int32_t* add_idx,
+                               int32_t* slot_tok, float* topk_w, float* add_w, cudaStream_t st);
 moe_status launch_combine_added(const moe_shape& s, const void* y_perm, const int32_t* a2p,
                                 const float* topk_w, void* out, const int32_t* add_ptr,
                                 const int32_t* add_idx, const float* add_w, long long n_rows,
@@ -273,8 +274,9 @@ namespace moe {
 namespace {
 // The layer forward with token rounding up or to the nearest tile (reading in moe.h).
 // 1. route; 2. the uncapped permutation (raw counts, each expert's assignments in token
-// order); 3. the extended id list: the routed ids, then E * (R - 1) entries of -1, in which
-// each expert drops (rounding down) or gains (rounding up) assignments; 4. the permutation
+// order); 3. the extended id list: the routed ids, less those an expert that rounds down
+// drops, then E * (R - 1) entries holding the added assignments' experts (-1 past the
+// last); 4. the permutation
 // of the extended list as T * K + E * (R - 1) one-assignment rows; 5. the token-major lists
 // of the added assignments and the weights over each enlarged selection; 6. the token of
 // every expert-major slot; 7. the grouped FFN over those rows; 8. combine with the added
@@ -301,23 +303,20 @@ moe_status launch_forward_rounded_up(const moe_shape& s, const void* x, const vo
   if ((r = launch_permute(s, ids, counts, offsets, a2p, p2a, nullptr, nullptr,
                           ws + L.permute_scratch, st)) != MOE_OK)
     return r;
-  if (cudaMemcpyAsync(ids_ext, ids, A0 * sizeof(int32_t), cudaMemcpyDeviceToDevice, st) !=
-          cudaSuccess ||
-      cudaMemsetAsync(ids_ext + A0, 0xff, NA * sizeof(int32_t), st) != cudaSuccess ||
-      cudaMemsetAsync(add_tok, 0xff, NA * sizeof(int32_t), st) != cudaSuccess)
-    return MOE_ERR_CUDA;
   if ((r = launch_round_select(s, counts, offsets, p2a, logits, ids_ext, add_tok, st)) != MOE_OK)
     return r;
   const moe_shape xs = ext_shape(s);
   if ((r = launch_permute(xs, ids_ext, (int32_t*)(ws + L.round_counts), offsets, a2p, p2a,
                           nullptr, nullptr, ws + L.permute_scratch, st)) != MOE_OK)
     return r;
-  if ((r = launch_round_weights(s, logits, ids, ids_ext + A0, add_tok,
-                                (int32_t*)(ws + L.add_cursor), (int32_t*)(ws + L.add_ptr),
-                                (int32_t*)(ws + L.add_idx), w, (float*)(ws + L.add_w), st)) !=
-      MOE_OK)
+  int32_t* add_ptr = (int32_t*)(ws + L.add_ptr);
+  int32_t* add_idx = (int32_t*)(ws + L.add_idx);
+  if ((r = launch_round_lists(s, ids_ext + A0, add_tok, (int32_t*)(ws + L.add_cursor), add_ptr,
+                              add_idx, st)) != MOE_OK)
     return r;
-  if ((r = launch_slot_tokens(s, p2a, offsets, add_tok, slot_tok, st)) != MOE_OK) return r;
+  if ((r = launch_round_finish(s, p2a, offsets, logits, ids, ids_ext + A0, add_tok, add_ptr,
+                               add_idx, slot_tok, w, (float*)(ws + L.add_w), st)) != MOE_OK)
+    return r;
   // the grouped FFN sees the extended list as one-assignment rows whose token is slot_tok[p]
   r = s.dtype == MOE_BF16 ? launch_ffn_tc_mixed(xs, x, offsets, slot_tok, w_gate, w_up, w_down,
                                                 ws + L.a_act, ws + L.y_perm, gateup_mode,
@@ -325,9 +324,8 @@ moe_status launch_forward_rounded_up(const moe_shape& s, const void* x, const vo
                           : launch_ffn_simt(xs, x, offsets, slot_tok, w_gate, w_up, w_down,
                                             ws + L.a_act, ws + L.y_perm, st);
   if (r != MOE_OK) return r;
-  return launch_combine_added(s, ws + L.y_perm, a2p, w, out, (const int32_t*)(ws + L.add_ptr),
-                              (const int32_t*)(ws + L.add_idx), (const float*)(ws + L.add_w),
-                              (long long)(A0 + NA), st);
+  return launch_combine_added(s, ws + L.y_perm, a2p, w, out, add_ptr, add_idx,
+                              (const float*)(ws + L.add_w), (long long)(A0 + NA), st);
 }
 
 moe_status forward_impl(const moe_shape* s, const void* x, const void* w_r, const float* bias,

@@ -23,6 +23,7 @@
 //             me); rank < C -> slot offsets[e] + rank, else dropped (-1).
 // Problems of at most kSmallMax assignments run all three phases in one CTA.
 // Inside an expert the slots follow ascending flat index a = t*K + k, i.e. token order.
+#include <algorithm>
 #include <mutex>
 #include <type_traits>
 
@@ -927,42 +928,33 @@ moe_status launch_route_permute(const moe_shape& s, const float* logits_in, floa
 
 // ------------------------------------------------------------------ token rounding
 // Tile-aware token rounding (SonicMoE explainer, section 6.5; the rule is the library's
-// reading): an expert with c >= R routed assignments keeps R * floor(c / R) of them, those
-// with the largest router logit for it (equal logits: the earlier token stays), and drops
-// the m = c mod R weakest. One CTA per expert, after an uncapped permutation (its slots
-// [offsets[e], offsets[e] + c) hold the assignments in token order): each slot's key is
-// (logit as an order-preserving 32-bit integer, +0 for both zeros) << 32 | (2^32 - 1 - t),
-// so ascending keys run from the weakest assignment up and every key is distinct; an
-// 8-pass radix select (8 bits a pass, a 256-bin shared histogram) finds the m-th smallest
-// key, and every slot at or below it marks its assignment -1 in the copy of the ids that
-// the second permutation reads.
+// reading, stated in moe.h). One CTA per expert e, after an uncapped permutation (its slots
+// [offsets[e], offsets[e] + c) hold its c routed assignments in token order). Keys are
+// (logit for e as an order-preserving 32-bit integer, +0 for both zeros) << 32 |
+// (2^32 - 1 - t): ascending keys run from the weakest token up and every key is distinct.
+// Rounding down drops the c mod R smallest keys of e's routed tokens; rounding up adds the
+// m largest keys among the tokens that did not route to e. Both place a threshold with a
+// radix select over the keys, cached in shared memory when they fit.
 namespace {
 
-__device__ __forceinline__ uint64_t round_key(const int32_t* p2a, const float* logits, int slot,
-                                              int K, int E, int e) {
-  const int a = p2a[slot];
-  const int t = a / K;
-  float v = logits[(size_t)t * E + e];
-  if (v == 0.f) v = 0.f;  // -0 and +0 are one value
-  uint32_t u = __float_as_uint(v);
-  u = (u & 0x80000000u) ? ~u : (u | 0x80000000u);  // ascending order of the floats
-  return ((uint64_t)u << 32) | (uint64_t)(0xffffffffu - (uint32_t)t);
-}
-
-// The need-th smallest (1-based) of the distinct 64-bit keys key_of(j) over the j < n for
-// which key_of returns true: an 8-pass radix select, 8 bits a pass, a 256-bin shared
-// histogram, the bin found by warp 0's shuffle scan and ballot. Every thread of the
-// 256-thread CTA calls it.
-template <typename KeyOf>
-__device__ uint64_t radix_select_u64(int n, int need, KeyOf key_of, unsigned* hist,
-                                     unsigned long long* s_pre, int* s_need) {
+// A threshold on the distinct 64-bit keys key_of(j) over the j < n for which key_of returns
+// true, placed at the need-th smallest (1-based) of them, q: GE returns theta with
+// {key >= theta} = {key >= q}; otherwise theta with {key <= theta} = {key <= q}. An 8-pass
+// radix select, 8 bits a pass from the top, a 256-bin shared histogram, the bin found by
+// warp 0's shuffle scan and ballot; it stops early once q's bin is known to lie wholly on
+// the selected side (GE: q is the bin's smallest key; else its largest), which for
+// continuous logits happens after two or three passes. Every thread of the NT-thread CTA
+// calls it.
+template <int NT, bool GE, typename KeyOf>
+__device__ uint64_t radix_threshold(int n, int need, KeyOf key_of, unsigned* hist,
+                                    unsigned long long* s_pre, int* s_need, int* s_done) {
   const int tid = threadIdx.x;
   uint64_t pre = 0;
   for (int d = 7; d >= 0; --d) {
     const uint64_t hi = d == 7 ? 0ull : (~0ull << (8 * (d + 1)));
-    hist[tid] = 0;
+    for (int b = tid; b < 256; b += NT) hist[b] = 0;
     __syncthreads();
-    for (int j = tid; j < n; j += 256) {
+    for (int j = tid; j < n; j += NT) {
       uint64_t key;
       if (key_of(j, key) && ((key ^ pre) & hi) == 0) atomicAdd(&hist[(key >> (8 * d)) & 255u], 1u);
     }
@@ -984,131 +976,158 @@ __device__ uint64_t radix_select_u64(int n, int need, KeyOf key_of, unsigned* hi
       const unsigned excl = incl - ls;
       const unsigned hit = __ballot_sync(0xffffffffu, excl < (unsigned)need && incl >= (unsigned)need);
       if (lane == __ffs(hit) - 1) {
-        unsigned run = excl;
+        unsigned run = excl, cnt = v[7];
         int b = lane * 8 + 7;
 #pragma unroll
         for (int q = 0; q < 8; ++q) {
           if (run + v[q] >= (unsigned)need) {
             b = lane * 8 + q;
+            cnt = v[q];
             break;
           }
           run += v[q];
         }
-        *s_need = need - (int)run;
-        *s_pre = pre | ((uint64_t)b << (8 * d));
+        const int nn = need - (int)run;  // q's rank inside bin b
+        uint64_t p = pre | ((uint64_t)b << (8 * d));
+        const bool done = d == 0 || (GE ? nn == 1 : nn == (int)cnt);
+        if (done && !GE && d > 0) p |= (1ull << (8 * d)) - 1;  // every lower digit at its top
+        *s_need = nn;
+        *s_pre = p;
+        *s_done = done;
       }
     }
     __syncthreads();
     pre = *s_pre;
     need = *s_need;
+    const bool done = *s_done;
     __syncthreads();
+    if (done) break;
   }
   return pre;
 }
 
-__global__ void __launch_bounds__(256) tile_round_kernel(const int32_t* __restrict__ counts,
-                                                         const int32_t* __restrict__ offsets,
-                                                         const int32_t* __restrict__ p2a,
-                                                         const float* __restrict__ logits,
-                                                         int K, int E, int R,
-                                                         int32_t* __restrict__ round_ids) {
-  __shared__ unsigned hist[256];
-  __shared__ unsigned long long s_pre;
-  __shared__ int s_need;
-  pdl_wait();  // the previous kernel in the stream has completed
-  pdl_trigger();
-  const int e = blockIdx.x, tid = threadIdx.x;
-  const int c = counts[e];
-  if (c < R || c % R == 0) return;  // uniform across the CTA
-  const int off = offsets[e];
-  // the (c mod R)-th smallest key: it and every smaller one are dropped
-  const uint64_t pre = radix_select_u64(
-      c, c % R,
-      [&](int j, uint64_t& key) {
-        key = round_key(p2a, logits, off + j, K, E, e);
-        return true;
-      },
-      hist, &s_pre, &s_need);
-  for (int j = tid; j < c; j += 256) {
-    const uint64_t key = round_key(p2a, logits, off + j, K, E, e);
-    if (key <= pre) round_ids[p2a[off + j]] = -1;
-  }
-}
+// Threads of the selection kernel: its loops are latency-bound with one CTA per expert.
+constexpr int kRoundThreads = 1024;
 
-// Rounding up or to the nearest tile (reading in moe.h): the tokens expert e gains, as a
-// count, from its routed count c (0 when it rounds down or is whole).
+// Rounding up or to the nearest tile: the tokens expert e gains, as a count, from its routed
+// count c (0 when it rounds down or is whole).
 __device__ __forceinline__ int round_adds(int c, int R, int mode, int T) {
   const int r = c % R;
   if (r == 0 || !(mode == 1 || (mode == 2 && r > R - r))) return 0;
   return min(R - r, T - c);
 }
 
-// One CTA per expert, after an uncapped permutation (e's routed assignments in token order
-// at p2a0[offsets0[e] ...]). An expert that rounds down drops its weakest assignments in the
-// extended id list (as tile_round_kernel); one that rounds up gains the m best tokens that
-// did not route to it: a shared bitmap marks its routed tokens, each other token's key is
-// (its logit for e as an order-preserving integer) << 32 | (2^32 - 1 - t), so larger keys
-// are stronger and all distinct; a radix select finds the m-th largest, and the tokens at or
-// above it are written in ascending order to add_tok[base ...] and as e into
-// ids_ext[T*K + base ...], base = the tokens gained by the experts before e.
-__global__ void __launch_bounds__(256) round_select_kernel(
+__device__ __forceinline__ uint32_t ord_logit(float v) {
+  if (v == 0.f) v = 0.f;  // -0 and +0 are one value
+  const uint32_t u = __float_as_uint(v);
+  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);  // ascending order of the floats
+}
+
+// Writes the extended id list ids_ext [T*K + NA] whole (NA = 0 when only rounding down).
+// Each CTA writes its expert's routed entries: e, or -1 for those an expert that rounds
+// down drops. An expert that rounds up (mode 1, or 2 with r > R - r) gains the m =
+// min(R - r, T - c) strongest tokens that did not route to it (a shared bitmap marks its
+// routed ones); they are written in ascending order to add_tok[base ...] and as e into
+// ids_ext[T*K + base ...], base = the tokens gained by the experts before e. CTA 0 sets the
+// unused tail of both added lists to -1. The keys live in the dynamic shared memory (cap
+// bytes) when they fit: 32 bits a token when rounding up (the token is the index), 64 bits
+// a routed slot when rounding down.
+__global__ void __launch_bounds__(kRoundThreads) round_select_kernel(
     const int32_t* __restrict__ counts, const int32_t* __restrict__ offsets0,
     const int32_t* __restrict__ p2a0, const float* __restrict__ logits, int T, int K, int E,
-    int R, int mode, int32_t* __restrict__ ids_ext, int32_t* __restrict__ add_tok) {
+    int R, int mode, int NA, int cap, int32_t* __restrict__ ids_ext,
+    int32_t* __restrict__ add_tok) {
+  extern __shared__ __align__(16) uint8_t round_cache[];
   __shared__ uint32_t routed[kRoundUpMaxTokens / 32];
   __shared__ unsigned hist[256];
   __shared__ unsigned long long s_pre;
-  __shared__ int s_need, s_base;
-  __shared__ int wsum[8];
+  __shared__ int s_need, s_base, s_total, s_done;
+  __shared__ int wsum[kRoundThreads / 32];
   pdl_wait();  // the previous kernel in the stream has completed
   pdl_trigger();
   const int e = blockIdx.x, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const size_t A0 = (size_t)T * K;
   const int c = counts[e];
   const int r = c % R;
-  if (r == 0) return;  // uniform across the CTA
   const int off = offsets0[e];
-  const bool up = mode == 1 || (mode == 2 && r > R - r);
+  if (NA > 0) {
+    if (tid == 0) s_base = s_total = 0;
+    __syncthreads();
+    for (int i = tid; i < E; i += kRoundThreads) {
+      const int v = round_adds(counts[i], R, mode, T);
+      if (i < e) atomicAdd(&s_base, v);
+      atomicAdd(&s_total, v);
+    }
+    __syncthreads();
+    if (e == 0)
+      for (int j = s_total + tid; j < NA; j += kRoundThreads) {
+        ids_ext[A0 + j] = -1;
+        add_tok[j] = -1;
+      }
+  }
+  const bool up = NA > 0 && r != 0 && (mode == 1 || (mode == 2 && r > R - r));
   if (!up) {
-    if (c < R) return;
-    const uint64_t pre = radix_select_u64(
-        c, r,
-        [&](int j, uint64_t& key) {
-          key = round_key(p2a0, logits, off + j, K, E, e);
-          return true;
-        },
-        hist, &s_pre, &s_need);
-    for (int j = tid; j < c; j += 256) {
-      const uint64_t key = round_key(p2a0, logits, off + j, K, E, e);
-      if (key <= pre) ids_ext[p2a0[off + j]] = -1;
+    if (r == 0 || c < R) {  // whole tiles, or too few to drop: every routed entry stays
+      for (int j = tid; j < c; j += kRoundThreads) ids_ext[p2a0[off + j]] = e;
+      return;
+    }
+    uint64_t* kc = reinterpret_cast<uint64_t*>(round_cache);
+    const bool cached = (long long)c * 8 <= cap;  // uniform across the CTA
+    if (cached) {
+      for (int j = tid; j < c; j += kRoundThreads) {
+        const int t = p2a0[off + j] / K;
+        kc[j] = ((uint64_t)ord_logit(logits[(size_t)t * E + e]) << 32) |
+                (uint64_t)(0xffffffffu - (uint32_t)t);
+      }
+      __syncthreads();
+    }
+    auto key_of = [&](int j, uint64_t& key) {
+      if (cached) {
+        key = kc[j];
+      } else {
+        const int t = p2a0[off + j] / K;
+        key = ((uint64_t)ord_logit(logits[(size_t)t * E + e]) << 32) |
+              (uint64_t)(0xffffffffu - (uint32_t)t);
+      }
+      return true;
+    };
+    // the r-th smallest key: it and every smaller one are dropped
+    const uint64_t pre = radix_threshold<kRoundThreads, false>(c, r, key_of, hist, &s_pre, &s_need, &s_done);
+    for (int j = tid; j < c; j += kRoundThreads) {
+      uint64_t key;
+      key_of(j, key);
+      ids_ext[p2a0[off + j]] = key <= pre ? -1 : e;
     }
     return;
   }
+  const int base = s_base;
   const int m = min(R - r, T - c);
-  if (tid == 0) s_base = 0;
-  for (int i = tid; i < T / 32 + 1 && i < kRoundUpMaxTokens / 32; i += 256) routed[i] = 0;
+  for (int i = tid; i < T / 32 + 1 && i < kRoundUpMaxTokens / 32; i += kRoundThreads) routed[i] = 0;
+  uint32_t* uc = reinterpret_cast<uint32_t*>(round_cache);
+  const bool cached = (long long)T * 4 <= cap;  // uniform across the CTA
+  if (cached)
+    for (int t = tid; t < T; t += kRoundThreads) uc[t] = ord_logit(logits[(size_t)t * E + e]);
   __syncthreads();
-  for (int i = tid; i < e; i += 256) atomicAdd(&s_base, round_adds(counts[i], R, mode, T));
-  for (int j = tid; j < c; j += 256) {
-    const int t = p2a0[off + j] / K;
+  for (int j = tid; j < c; j += kRoundThreads) {
+    const int a = p2a0[off + j];
+    ids_ext[a] = e;
+    const int t = a / K;
     atomicOr(&routed[t >> 5], 1u << (t & 31));
   }
   __syncthreads();
-  const int base = s_base;
   if (m <= 0) return;
   auto key_of = [&](int t, uint64_t& key) {
     if ((routed[t >> 5] >> (t & 31)) & 1u) return false;
-    float v = logits[(size_t)t * E + e];
-    if (v == 0.f) v = 0.f;  // -0 and +0 are one value
-    uint32_t u = __float_as_uint(v);
-    u = (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+    const uint32_t u = cached ? uc[t] : ord_logit(logits[(size_t)t * E + e]);
     key = ((uint64_t)u << 32) | (uint64_t)(0xffffffffu - (uint32_t)t);
     return true;
   };
   // the m-th largest of the T - c candidate keys = their (T - c - m + 1)-th smallest
-  const uint64_t theta = radix_select_u64(T, T - c - m + 1, key_of, hist, &s_pre, &s_need);
-  // the chosen tokens in ascending order, 256 at a time
+  const uint64_t theta =
+      radix_threshold<kRoundThreads, true>(T, T - c - m + 1, key_of, hist, &s_pre, &s_need, &s_done);
+  // the chosen tokens in ascending order, kRoundThreads at a time
   int run = 0;
-  for (int t0 = 0; t0 < T; t0 += 256) {
+  for (int t0 = 0; t0 < T; t0 += kRoundThreads) {
     const int t = t0 + tid;
     uint64_t key = 0;
     const bool chosen = t < T && key_of(t, key) && key >= theta;
@@ -1116,152 +1135,162 @@ __global__ void __launch_bounds__(256) round_select_kernel(
     if (lane == 0) wsum[warp] = __popc(bal);
     __syncthreads();
     int before = run, total = 0;
-    for (int w = 0; w < 8; ++w) {
+    for (int w = 0; w < kRoundThreads / 32; ++w) {
       if (w < warp) before += wsum[w];
       total += wsum[w];
     }
     if (chosen) {
       const int pos = base + before + __popc(bal & lanemask_lt());
       add_tok[pos] = t;
-      ids_ext[(size_t)T * K + pos] = e;
+      ids_ext[A0 + pos] = e;
     }
     run += total;
     __syncthreads();
   }
 }
 
-// Token-major view of the added assignments: counts per token (atomics on counters that
-// start at zero; the counts do not depend on the order).
-__global__ void __launch_bounds__(256) round_count_kernel(const int32_t* __restrict__ ids_add,
-                                                          const int32_t* __restrict__ add_tok,
-                                                          int NA, int T, int32_t* cnt,
-                                                          unsigned* status) {
-  pdl_wait();  // the previous kernel in the stream has completed
-  pdl_trigger();
-  const int j = blockIdx.x * 256 + threadIdx.x;
-  if (j >= NA || ids_add[j] < 0) return;
-  const int t = add_tok[j];
-  if (t < 0 || t >= T) {
-    report(status, MOE_ERR_DEVICE_INDEX);
-    return;
-  }
-  atomicAdd(&cnt[t], 1);
-}
-
-// add_ptr = exclusive scan of the per-token counts (one CTA of 1024 threads, each scanning a
-// contiguous run); the counters are zeroed again for the fill.
-__global__ void __launch_bounds__(1024) round_scan_kernel(int32_t* cnt, int T,
-                                                          int32_t* __restrict__ add_ptr) {
+// Token-major lists of the added assignments, in one CTA of 1024 threads whose phases are
+// separated by block barriers (a few thousand entries):
+//   1. per-token counts of the added assignments (atomics on zeroed counters);
+//   2. add_ptr = their exclusive scan (each thread a contiguous run of tokens, the runs'
+//      sums scanned across the block); the counters are zeroed again;
+//   3. each added assignment into its token's list at an atomic cursor (any order; the
+//      finishing kernel sorts each list).
+__global__ void __launch_bounds__(1024) round_lists_kernel(const int32_t* __restrict__ ids_add,
+                                                           const int32_t* __restrict__ add_tok,
+                                                           int NA, int T, int32_t* cnt,
+                                                           int32_t* add_ptr, int32_t* add_idx,
+                                                           unsigned* status) {
   __shared__ int wsum[32];
   pdl_wait();  // the previous kernel in the stream has completed
   pdl_trigger();
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int per = (T + 1023) / 1024;
-  const int b = tid * per, e = min(T, b + per);
-  int sum = 0;
-  for (int t = b; t < e; ++t) sum += cnt[t];
-  int incl = sum;
-#pragma unroll
-  for (int o = 1; o < 32; o <<= 1) {
-    const int y = __shfl_up_sync(0xffffffffu, incl, o);
-    if (lane >= o) incl += y;
-  }
-  if (lane == 31) wsum[warp] = incl;
+  for (int t = tid; t < T; t += 1024) cnt[t] = 0;
   __syncthreads();
-  if (warp == 0) {
-    int v = wsum[lane], iv = v;
+  for (int j = tid; j < NA; j += 1024) {  // 1. counts
+    if (ids_add[j] < 0) continue;
+    const int t = add_tok[j];
+    if (t < 0 || t >= T) {
+      report(status, MOE_ERR_DEVICE_INDEX);
+      continue;
+    }
+    atomicAdd(&cnt[t], 1);
+  }
+  __syncthreads();
+  {  // 2. exclusive scan
+    const int per = (T + 1023) / 1024;
+    const int b = tid * per, e = min(T, b + per);
+    int sum = 0;
+    for (int t = b; t < e; ++t) sum += cnt[t];
+    int incl = sum;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
-      const int y = __shfl_up_sync(0xffffffffu, iv, o);
-      if (lane >= o) iv += y;
+      const int y = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += y;
     }
-    wsum[lane] = iv - v;
+    if (lane == 31) wsum[warp] = incl;
+    __syncthreads();
+    if (warp == 0) {
+      const int v = wsum[lane];
+      int iv = v;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, iv, o);
+        if (lane >= o) iv += y;
+      }
+      wsum[lane] = iv - v;
+    }
+    __syncthreads();
+    int run = wsum[warp] + incl - sum;
+    for (int t = b; t < e; ++t) {
+      add_ptr[t] = run;
+      run += cnt[t];
+      cnt[t] = 0;
+    }
+    if (tid == 1023) add_ptr[T] = run;
   }
   __syncthreads();
-  int run = wsum[warp] + incl - sum;
-  for (int t = b; t < e; ++t) {
-    add_ptr[t] = run;
-    run += cnt[t];
-    cnt[t] = 0;
+  for (int j = tid; j < NA; j += 1024) {  // 3. fill
+    if (ids_add[j] < 0) continue;
+    const int t = add_tok[j];
+    if (t < 0 || t >= T) continue;
+    add_idx[add_ptr[t] + atomicAdd(&cnt[t], 1)] = j;
   }
-  if (tid == 1023) add_ptr[T] = run;
+  __syncthreads();
 }
 
-// Each added assignment into its token's list (atomic cursors: any order here, sorted by
-// the weights kernel).
-__global__ void __launch_bounds__(256) round_fill_kernel(const int32_t* __restrict__ ids_add,
-                                                         const int32_t* __restrict__ add_tok,
-                                                         int NA, int T,
-                                                         const int32_t* __restrict__ add_ptr,
-                                                         int32_t* cursor,
-                                                         int32_t* __restrict__ add_idx) {
-  pdl_wait();  // the previous kernel in the stream has completed
-  pdl_trigger();
-  const int j = blockIdx.x * 256 + threadIdx.x;
-  if (j >= NA || ids_add[j] < 0) return;
-  const int t = add_tok[j];
-  if (t < 0 || t >= T) return;
-  add_idx[add_ptr[t] + atomicAdd(&cursor[t], 1)] = j;
-}
-
-// Weights of a token that gained assignments, over its enlarged selection (reading in
-// moe.h): its added list sorted ascending (= expert order), then, renormalised,
-// w = exp(l - l_top) / (sum over the K routed and the added of exp(l_j - l_top)), summed in
-// slot order then list order; plain softmax: the added ones get softmax(l) over all E, the
-// routed ones keep theirs. One thread per token.
-__global__ void __launch_bounds__(256) round_weights_kernel(
-    const float* __restrict__ logits, const int32_t* __restrict__ ids, int T, int K, int E,
-    int renorm, const int32_t* __restrict__ ids_add, const int32_t* __restrict__ add_ptr,
-    int32_t* __restrict__ add_idx, float* __restrict__ topk_w, float* __restrict__ add_w) {
-  pdl_wait();  // the previous kernel in the stream has completed
-  pdl_trigger();
-  const int t = blockIdx.x * 256 + threadIdx.x;
-  if (t >= T) return;
-  const int lo = add_ptr[t], hi = add_ptr[t + 1];
-  if (hi == lo) return;
-  for (int i = lo + 1; i < hi; ++i) {  // insertion sort (a token gains a few at most)
-    const int v = add_idx[i];
-    int k = i - 1;
-    while (k >= lo && add_idx[k] > v) {
-      add_idx[k + 1] = add_idx[k];
-      --k;
-    }
-    add_idx[k + 1] = v;
-  }
-  const float* lg = logits + (size_t)t * E;
-  const float top = lg[ids[(size_t)t * K]];
-  if (renorm) {
-    float den = 0.f;
-    for (int k = 0; k < K; ++k) den += expf(lg[ids[(size_t)t * K + k]] - top);
-    for (int i = lo; i < hi; ++i) den += expf(lg[ids_add[add_idx[i]]] - top);
-    for (int k = 0; k < K; ++k)
-      topk_w[(size_t)t * K + k] = expf(lg[ids[(size_t)t * K + k]] - top) / den;
-    for (int i = lo; i < hi; ++i) add_w[add_idx[i]] = expf(lg[ids_add[add_idx[i]]] - top) / den;
-  } else {
-    float den = 0.f;  // the plain softmax over all E (the top logit is the maximum)
-    for (int q = 0; q < E; ++q) den += expf(lg[q] - top);
-    for (int i = lo; i < hi; ++i) add_w[add_idx[i]] = expf(lg[ids_add[add_idx[i]]] - top) / den;
-  }
-}
-
-// The token of every kept expert-major slot: a < T*K is token a / K, an added a = T*K + j
-// is add_tok[j].
-__global__ void __launch_bounds__(256) slot_token_kernel(const int32_t* __restrict__ p2a,
-                                                         const int32_t* __restrict__ n_kept_ptr,
-                                                         int T, int K,
-                                                         const int32_t* __restrict__ add_tok,
-                                                         int32_t* __restrict__ slot_tok) {
+// The rest of rounding up, one thread per entry over max(T, n_kept) (both independent):
+//   p < n_kept: the token of expert-major slot p (a < T*K is token a / K, an added
+//     a = T*K + j is add_tok[j]);
+//   t < T with added assignments: its list sorted ascending (= expert order), then,
+//     renormalised, w = exp(l - l_top) / (sum over the K routed and the added of
+//     exp(l_j - l_top)) summed in slot order then list order, l_top the logit of its first
+//     routed expert (the largest); plain softmax: the added ones get softmax(l) over all E,
+//     the routed ones keep theirs.
+__global__ void __launch_bounds__(256) round_finish_kernel(
+    const int32_t* __restrict__ p2a, const int32_t* __restrict__ n_kept_ptr, int T, int K, int E,
+    int renorm, const float* __restrict__ logits, const int32_t* __restrict__ ids,
+    const int32_t* __restrict__ ids_add, const int32_t* __restrict__ add_tok,
+    const int32_t* __restrict__ add_ptr, int32_t* __restrict__ add_idx,
+    int32_t* __restrict__ slot_tok, float* __restrict__ topk_w, float* __restrict__ add_w) {
   pdl_wait();  // the previous kernel in the stream has completed
   pdl_trigger();
   const int n_kept = *n_kept_ptr;
   const long long A0 = (long long)T * K;
-  for (int p = blockIdx.x * 256 + threadIdx.x; p < n_kept; p += gridDim.x * 256) {
-    const long long a = p2a[p];
-    slot_tok[p] = a < A0 ? (int32_t)(a / K) : add_tok[a - A0];
+  const int n = max(n_kept, T);
+  for (int i = blockIdx.x * 256 + threadIdx.x; i < n; i += gridDim.x * 256) {
+    if (i < n_kept) {
+      const long long a = p2a[i];
+      slot_tok[i] = a < A0 ? (int32_t)(a / K) : add_tok[a - A0];
+    }
+    if (i >= T) continue;
+    const int t = i;
+    const int lo = add_ptr[t], hi = add_ptr[t + 1];
+    if (hi == lo) continue;
+    for (int q = lo + 1; q < hi; ++q) {  // insertion sort (a token gains a few at most)
+      const int v = add_idx[q];
+      int k = q - 1;
+      while (k >= lo && add_idx[k] > v) {
+        add_idx[k + 1] = add_idx[k];
+        --k;
+      }
+      add_idx[k + 1] = v;
+    }
+    const float* lg = logits + (size_t)t * E;
+    const float top = lg[ids[(size_t)t * K]];
+    float den = 0.f;
+    if (renorm) {
+      for (int k = 0; k < K; ++k) den += expf(lg[ids[(size_t)t * K + k]] - top);
+      for (int q = lo; q < hi; ++q) den += expf(lg[ids_add[add_idx[q]]] - top);
+      for (int k = 0; k < K; ++k)
+        topk_w[(size_t)t * K + k] = expf(lg[ids[(size_t)t * K + k]] - top) / den;
+    } else {  // the plain softmax over all E (the top logit is the maximum)
+      for (int q = 0; q < E; ++q) den += expf(lg[q] - top);
+    }
+    for (int q = lo; q < hi; ++q) add_w[add_idx[q]] = expf(lg[ids_add[add_idx[q]]] - top) / den;
   }
 }
 
 }  // namespace
+
+// Dynamic shared memory of the selection kernel: up to 192 KB of cached keys (8 bytes a
+// token bounds both directions), beside its 17 KB of static arrays.
+constexpr int kRoundCacheMax = 192 * 1024;
+
+moe_status launch_round_select_kernel(const moe_shape& s, const int32_t* counts,
+                                      const int32_t* offsets0, const int32_t* p2a0,
+                                      const float* logits, int mode, int NA, int32_t* ids_ext,
+                                      int32_t* add_tok, cudaStream_t st) {
+  const int cap = (int)std::min<long long>(kRoundCacheMax, (long long)s.T * 8);
+  if (cudaFuncSetAttribute(round_select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           kRoundCacheMax) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  launch_begin(K_TILE_ROUND, st);
+  launch_kernel(round_select_kernel, dim3((unsigned)s.E), dim3(kRoundThreads), (size_t)cap, st, 1, counts,
+                offsets0, p2a0, logits, s.T, s.K, s.E, s.tile_round, mode, NA, cap, ids_ext,
+                add_tok);
+  return launch_end(K_TILE_ROUND, st);
+}
 
 moe_status launch_permute_rounded(const moe_shape& s, const int32_t* ids, const float* logits,
                                   int32_t* counts, int32_t* offsets, int32_t* a2p, int32_t* p2a,
@@ -1273,15 +1302,9 @@ moe_status launch_permute_rounded(const moe_shape& s, const int32_t* ids, const 
       MOE_OK)
     return r;
   // 2. the ids again, with the rounded-away assignments set to -1
-  const size_t A = (size_t)s.T * s.K;
-  if (cudaMemcpyAsync(round_ids, ids, A * sizeof(int32_t), cudaMemcpyDeviceToDevice, st) !=
-      cudaSuccess)
-    return MOE_ERR_CUDA;
-  launch_begin(K_TILE_ROUND, st);
-  launch_kernel(tile_round_kernel, dim3((unsigned)s.E), dim3(256), 0, st, 1,
-                (const int32_t*)counts, (const int32_t*)offsets, (const int32_t*)p2a, logits, s.K,
-                s.E, s.tile_round, round_ids);
-  if ((r = launch_end(K_TILE_ROUND, st)) != MOE_OK) return r;
+  if ((r = launch_round_select_kernel(s, counts, offsets, p2a, logits, 0, 0, round_ids, nullptr,
+                                      st)) != MOE_OK)
+    return r;
   // 3. the final permutation of what is kept (its counts are the kept ones: not returned)
   return launch_permute(s, round_ids, round_counts, offsets, a2p, p2a, x, x_perm, scratch, st);
 }
@@ -1290,47 +1313,30 @@ moe_status launch_round_select(const moe_shape& s, const int32_t* counts, const 
                                const int32_t* p2a0, const float* logits, int32_t* ids_ext,
                                int32_t* add_tok, cudaStream_t st) {
   if (s.T > kRoundUpMaxTokens) return MOE_ERR_UNSUPPORTED;
+  return launch_round_select_kernel(s, counts, offsets0, p2a0, logits, s.tile_round_mode,
+                                    s.E * (s.tile_round - 1), ids_ext, add_tok, st);
+}
+
+moe_status launch_round_lists(const moe_shape& s, const int32_t* ids_add, const int32_t* add_tok,
+                              int32_t* cursor, int32_t* add_ptr, int32_t* add_idx,
+                              cudaStream_t st) {
   launch_begin(K_TILE_ROUND, st);
-  launch_kernel(round_select_kernel, dim3((unsigned)s.E), dim3(256), 0, st, 1, counts, offsets0,
-                p2a0, logits, s.T, s.K, s.E, s.tile_round, s.tile_round_mode, ids_ext, add_tok);
+  launch_kernel(round_lists_kernel, dim3(1), dim3(1024), 0, st, 1, ids_add, add_tok,
+                s.E * (s.tile_round - 1), s.T, cursor, add_ptr, add_idx, device_status_ptr());
   return launch_end(K_TILE_ROUND, st);
 }
 
-moe_status launch_round_weights(const moe_shape& s, const float* logits, const int32_t* ids,
-                                const int32_t* ids_add, const int32_t* add_tok, int32_t* cursor,
-                                int32_t* add_ptr, int32_t* add_idx, float* topk_w, float* add_w,
-                                cudaStream_t st) {
-  const int NA = s.E * (s.tile_round - 1);
-  moe_status r;
-  if (cudaMemsetAsync(cursor, 0, sizeof(int32_t) * (size_t)s.T, st) != cudaSuccess)
-    return MOE_ERR_CUDA;
-  const unsigned gb = (unsigned)((NA + 255) / 256);
-  launch_begin(K_TILE_ROUND, st);
-  launch_kernel(round_count_kernel, dim3(gb), dim3(256), 0, st, 1, ids_add, add_tok, NA, s.T,
-                cursor, device_status_ptr());
-  if ((r = launch_end(K_TILE_ROUND, st)) != MOE_OK) return r;
-  launch_begin(K_TILE_ROUND, st);
-  launch_kernel(round_scan_kernel, dim3(1), dim3(1024), 0, st, 1, cursor, s.T, add_ptr);
-  if ((r = launch_end(K_TILE_ROUND, st)) != MOE_OK) return r;
-  launch_begin(K_TILE_ROUND, st);
-  launch_kernel(round_fill_kernel, dim3(gb), dim3(256), 0, st, 1, ids_add, add_tok, NA, s.T,
-                (const int32_t*)add_ptr, cursor, add_idx);
-  if ((r = launch_end(K_TILE_ROUND, st)) != MOE_OK) return r;
-  launch_begin(K_TILE_ROUND, st);
-  launch_kernel(round_weights_kernel, dim3((unsigned)((s.T + 255) / 256)), dim3(256), 0, st, 1,
-                logits, ids, s.T, s.K, s.E, s.renormalize, ids_add, (const int32_t*)add_ptr,
-                add_idx, topk_w, add_w);
-  return launch_end(K_TILE_ROUND, st);
-}
-
-moe_status launch_slot_tokens(const moe_shape& s, const int32_t* p2a, const int32_t* offsets,
-                              const int32_t* add_tok, int32_t* slot_tok, cudaStream_t st) {
+moe_status launch_round_finish(const moe_shape& s, const int32_t* p2a, const int32_t* offsets,
+                               const float* logits, const int32_t* ids, const int32_t* ids_add,
+                               const int32_t* add_tok, const int32_t* add_ptr, int32_t* add_idx,
+                               int32_t* slot_tok, float* topk_w, float* add_w, cudaStream_t st) {
   const long long A = (long long)s.T * s.K + (long long)s.E * (s.tile_round - 1);
-  long long blocks = (A + 255) / 256;
+  long long blocks = (std::max<long long>(A, s.T) + 255) / 256;
   if (blocks > (long long)sm_count() * 8) blocks = (long long)sm_count() * 8;
   launch_begin(K_TILE_ROUND, st);
-  launch_kernel(slot_token_kernel, dim3((unsigned)blocks), dim3(256), 0, st, 1, p2a,
-                offsets + s.E, s.T, s.K, add_tok, slot_tok);
+  launch_kernel(round_finish_kernel, dim3((unsigned)blocks), dim3(256), 0, st, 1, p2a,
+                offsets + s.E, s.T, s.K, s.E, s.renormalize, logits, ids, ids_add, add_tok,
+                add_ptr, add_idx, slot_tok, topk_w, add_w);
   return launch_end(K_TILE_ROUND, st);
 }
 
