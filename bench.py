@@ -618,7 +618,8 @@ def backward_figure(tdr, cfg, s, x, w_r, wg, wu, wd, bias, world, peak_t, steps=
             "router_ms": {"d_logits": round(avg("router_dlogits"), 4),
                           "d_w_r_and_bias": round(avg("router_dwr"), 4),
                           "d_x_term": round(avg("router_dx"), 4)},
-            "note": "dA' = dO W_down^T (dO gathered by token; dS and the SwiGLU backward in the "
+            "note": "dA' = dO W_down^T (dO rows by token: copied expert-major first when "
+                    "n >= 4096, else gathered in the GEMM; dS and the SwiGLU backward in the "
                     "epilogue: reads h, writes d_h), d_w reduction, dX_perm = (dG|dU) "
                     "(W_gate|W_up)^T, scatter-add to tokens, router backward (d_logits, "
                     "d_W_r, d_bias, its d_x term); TFLOP/s on 2*d*n (dA') and 4*d*n (dX) per "

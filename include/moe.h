@@ -327,7 +327,9 @@ moe_status moe_forward_workspace_layout(const moe_shape* shape, moe_workspace_la
  *   h [T*K, 2n] from moe_forward_h; d_h [T*K, 2n] bf16 out; d_w [T, K] fp32 out;
  *   d_x [T, d] bf16 out or NULL;
  *   workspace >= moe_backward_workspace_size(shape), 256-byte aligned (per-slot partial
- *   sums, and the dX_perm rows).
+ *   sums, and one [T*K, d] row buffer: the dO rows copied expert-major for the dA' GEMM
+ *   when shape.ffn_variant is 3, or 0 with n >= 4096 (1 and 2 gather them inside the
+ *   GEMM), then the dX_perm rows).
  * d_w sums each slot's 256-column parts in a fixed order (deterministic). The router's
  * own backward (through the softmax and top-K to the logits, W_r and x) and the weight
  * gradients are not computed. bf16 only; d_out, w_*, h, d_h, d_x 16-byte aligned.

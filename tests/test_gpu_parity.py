@@ -785,9 +785,9 @@ def test_token_rounding_up_rejected_where_it_cannot_apply(cuda_lib):
 
 
 # ------------------------------------------------------------------ backward (expert half)
-def _bwd_case(tdr, cfg, seed):
+def _bwd_case(tdr, cfg, seed, ffn_variant=0, input_grad=True):
     inp = mi.make_inputs(cfg)
-    s = shape_of(cfg, tdr)
+    s = shape_of(cfg, tdr, ffn_variant=ffn_variant)
     out_h, ws, h = tdr.forward_h(s, cuda(inp.x), cuda(inp.w_r), cuda(inp.w_gate), cuda(inp.w_up),
                                  cuda(inp.w_down), bias=cuda(inp.bias))
     v = tdr.workspace_views(s, ws)
@@ -796,22 +796,26 @@ def _bwd_case(tdr, cfg, seed):
         torch.bfloat16)
     d_h, d_w, d_x = tdr.backward(s, d_out.cuda(), v["topk_w"], v["offsets"], v["perm_to_assign"],
                                  v["assign_to_perm"], cuda(inp.w_down), h,
-                                 w_gate=cuda(inp.w_gate), w_up=cuda(inp.w_up), input_grad=True)
+                                 w_gate=cuda(inp.w_gate), w_up=cuda(inp.w_up),
+                                 input_grad=input_grad)
     torch.cuda.synchronize()
     assert_status_ok(tdr)
     return inp, s, out_h, v, h, d_out, d_h, d_w, d_x
 
 
+@pytest.mark.parametrize("bwd_rows", [3, 1], ids=["rows_copied", "rows_gathered"])
 @pytest.mark.parametrize("T,d,n,E,K,cf", [
     (300, 128, 128, 8, 2, 0.0),
     (513, 256, 384, 4, 2, 0.8),    # a half n-tile, capacity drops
     (1000, 512, 768, 16, 4, 0.0),
 ])
-def test_backward_act_matches_oracle(cuda_lib, T, d, n, E, K, cf):
+def test_backward_act_matches_oracle(cuda_lib, bwd_rows, T, d, n, E, K, cf):
+    """dA' with the dO rows copied expert-major first (ffn_variant 3) and gathered inside the
+    GEMM (ffn_variant 1); the full-size case below takes the automatic choice (copied)."""
     tdr = cuda_lib
     cfg = mi.MoEConfig("bwd", T=T, d=d, E=E, K=K, n=n, dtype="bf16", capacity_factor=cf,
                        seed=T + n)
-    inp, s, out_h, v, h, d_out, d_h, d_w, d_x = _bwd_case(tdr, cfg, 5)
+    inp, s, out_h, v, h, d_out, d_h, d_w, d_x = _bwd_case(tdr, cfg, 5, ffn_variant=bwd_rows)
     # the forward is the plain one, and h holds the pre-activations
     out_plain, _ = tdr.forward(s, cuda(inp.x), cuda(inp.w_r), cuda(inp.w_gate), cuda(inp.w_up),
                                cuda(inp.w_down))
@@ -834,6 +838,18 @@ def test_backward_act_matches_oracle(cuda_lib, T, d, n, E, K, cf):
     assert_bf16_close(d_x.float().cpu().numpy(), dx_ref, "d_x")
     if cf > 0:
         assert np.all(d_w.cpu().numpy().reshape(-1)[a2p < 0] == 0)
+
+
+def test_backward_without_input_grad_matches_with(cuda_lib):
+    """moe_backward without d_x (the row buffer still holds the copied dO rows) gives the
+    same d_h and d_w as with it."""
+    tdr = cuda_lib
+    cfg = mi.MoEConfig("bwd", T=700, d=256, E=8, K=2, n=256, dtype="bf16", seed=3)
+    _, _, _, _, _, _, d_h1, d_w1, _ = _bwd_case(tdr, cfg, 6, ffn_variant=3, input_grad=True)
+    _, _, _, _, _, _, d_h0, d_w0, d_x0 = _bwd_case(tdr, cfg, 6, ffn_variant=3,
+                                                   input_grad=False)
+    assert d_x0 is None
+    assert torch.equal(d_h0, d_h1) and torch.equal(d_w0, d_w1)
 
 
 def test_backward_act_full_size_sampled_slots(cuda_lib):

@@ -16,7 +16,10 @@
 //   warp 0     TMA producer: the B tile, 256 rows of W_down[e] (n) x 64 of d, one
 //              K-major box (128-byte swizzle), into a 4-stage ring (48 KB a stage);
 //   warps 6-9  the gathered A tile: 128 rows of dO (row = perm_to_assign[p] / K) x 64 of
-//              d by cp.async into the swizzled K-major layout;
+//              d by cp.async into the swizzled K-major layout (MODE 0); or (MODE 2) the dO
+//              rows are first copied expert-major into a scratch buffer and the producer
+//              loads the A tile from there by TMA, which leaves the load/store units to the
+//              epilogue;
 //   warp 1     TMEM allocation and the MMA thread (both operands K-major);
 //   warps 2-5  epilogue: one TMEM lane = one slot per thread; dG and dU (bf16) into
 //              d_h[p] = (dG | dU), and this tile's 256-column part of dS into
@@ -97,11 +100,13 @@ __device__ __forceinline__ Tile decode(int w, const int* s_off, const int* s_cum
 // MODE 0 (dA'): A = rows of dO gathered by token, B = W_down[e] (K = d), epilogue above.
 // MODE 1 (dX): A = the (dG | dU) rows by TMA, B = W_gate[e] for the first n of K and W_up[e]
 // for the second (K = 2n), both read K-major in place; epilogue: bf16 dX_perm rows.
+// MODE 2 (dA'): as MODE 0 with A = the dO rows copied expert-major beforehand, by TMA.
 template <int MODE>
 __global__ void __launch_bounds__(MODE == 0 ? THREADS_DACT : THREADS_DX, 1)
     grouped_gemm_bwd(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                      const __grid_constant__ CUtensorMap tmB2, const BwdArgs g) {
   constexpr int THREADS = MODE == 0 ? THREADS_DACT : THREADS_DX;
+  constexpr bool GATHER = MODE == 0;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* base = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
   uint8_t* ring = base;
@@ -121,8 +126,8 @@ __global__ void __launch_bounds__(MODE == 0 ? THREADS_DACT : THREADS_DX, 1)
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int E = g.E;
   // TMA expect_tx (+ the gather threads' cp.async arrivals in MODE 0)
-  constexpr uint32_t FULL_COUNT = MODE == 0 ? 1 + GATHER_THREADS : 1;
-  constexpr uint32_t TMA_BYTES = MODE == 0 ? B_BYTES : STAGE_BYTES;
+  constexpr uint32_t FULL_COUNT = GATHER ? 1 + GATHER_THREADS : 1;
+  constexpr uint32_t TMA_BYTES = GATHER ? B_BYTES : STAGE_BYTES;
 
   if (tid == 0) {
     for (int s = 0; s < STAGES; ++s) {
@@ -139,10 +144,10 @@ __global__ void __launch_bounds__(MODE == 0 ? THREADS_DACT : THREADS_DX, 1)
   }
   if (tid == 32) {
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmB)) : "memory");
-    if (MODE == 1) {
+    if (!GATHER)
       asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmA)) : "memory");
+    if (MODE == 1)
       asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmB2)) : "memory");
-    }
   }
   if (warp == 1) tmem_alloc<1>(saddr(tmem_slot), TMEM_COLS);
   pdl_wait();  // the previous kernel in the stream has completed
@@ -204,7 +209,10 @@ __global__ void __launch_bounds__(MODE == 0 ? THREADS_DACT : THREADS_DX, 1)
           const uint32_t fb = saddr(&full[stage]);
           const uint32_t a_dst = saddr(ring + stage * STAGE_BYTES);
           mbar_expect_tx(fb, TMA_BYTES);
-          if (MODE == 0) {
+          if (GATHER) {
+            tma_load_3d(a_dst + A_BYTES, &tmB, kb * BK, t.n0, t.e, fb);
+          } else if (MODE == 2) {
+            tma_load_2d(a_dst, &tmA, kb * BK, t.m0, fb);
             tma_load_3d(a_dst + A_BYTES, &tmB, kb * BK, t.n0, t.e, fb);
           } else {
             tma_load_2d(a_dst, &tmA, kb * BK, t.m0, fb);
@@ -250,7 +258,7 @@ __global__ void __launch_bounds__(MODE == 0 ? THREADS_DACT : THREADS_DX, 1)
             ok = false;
             break;
           }
-          if (MODE == 0) fence_proxy_async_smem();  // cp.async (generic) writes -> MMA reads
+          if (GATHER) fence_proxy_async_smem();  // cp.async (generic) writes -> MMA reads
           tc_fence_after();
           const uint32_t a_addr = saddr(ring + stage * STAGE_BYTES);
           const uint32_t b_addr = a_addr + A_BYTES;
@@ -273,7 +281,7 @@ __global__ void __launch_bounds__(MODE == 0 ? THREADS_DACT : THREADS_DX, 1)
       while (!mbar_try(saddr(done), 0) && globaltimer_ns() - t0 < limit) {
       }
     }
-  } else if (MODE == 0 && warp >= GATHER_WARP0) {
+  } else if (GATHER && warp >= GATHER_WARP0) {
     // ------------------------------------------------------------ A gather: rows of dO
     const int gw = warp - GATHER_WARP0;
     const int c = lane & 7;
@@ -500,15 +508,32 @@ size_t align256b(size_t v) { return (v + 255) & ~(size_t)255; }
 
 // Scratch: the per-slot partial sums of dS, then (when the input gradient is wanted) the
 // dX_perm rows.
-size_t backward_scratch_bytes(const moe_shape& s, bool with_dx) {
+// The dO rows are copied expert-major before the dA' GEMM (ffn_variant 3), or gathered
+// inside it (1, 2). Automatic (0): copied when n >= 4096. The in-GEMM gather shares the
+// load/store units with this epilogue's h reads and d_h writes; at n = 14336 the TMA-fed
+// GEMM measured 0.870 ms against 0.950 ms, while the copy costs 4 T K d bytes of traffic
+// (about 15 us there), a share of the GEMM that grows as n shrinks.
+bool backward_copies_rows(const moe_shape& s) {
+  return s.ffn_variant == 3 || (s.ffn_variant == 0 && s.n >= 4096);
+}
+
+// Scratch: the per-slot partial sums of d_w, then (at backward_rows_offset) one
+// [T*K, d] bf16 row buffer: the copied dO rows for the dA' GEMM, later the dX_perm rows.
+size_t backward_rows_offset(const moe_shape& s) {
   const size_t n_tiles = (size_t)(s.n + BN - 1) / BN;
-  size_t b = align256b((size_t)s.T * s.K * n_tiles * sizeof(float));
-  if (with_dx) b += align256b((size_t)s.T * s.K * s.d * 2);
+  return align256b((size_t)s.T * s.K * n_tiles * sizeof(float));
+}
+
+size_t backward_scratch_bytes(const moe_shape& s, bool with_dx) {
+  size_t b = backward_rows_offset(s);
+  if (with_dx || backward_copies_rows(s)) b += align256b((size_t)s.T * s.K * s.d * 2);
   return b;
 }
 
 moe_status launch_combine(const moe_shape& s, const void* y_perm, const int32_t* a2p,
                           const float* topk_w, void* out, cudaStream_t st);
+moe_status launch_gather_rows(const moe_shape& s, const void* x, const int32_t* p2a,
+                              const int32_t* offsets, void* x_perm, cudaStream_t st);
 
 moe_status launch_backward(const moe_shape& s, const void* d_out, const float* topk_w,
                            const int32_t* offsets, const int32_t* p2a, const int32_t* a2p,
@@ -544,14 +569,30 @@ moe_status launch_backward(const moe_shape& s, const void* d_out, const float* t
   a.T = s.T;
   a.status = device_status_ptr();
   a.limit_ns = kWaitLimitNs;
-  if (cudaFuncSetAttribute(grouped_gemm_bwd<0>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           SMEM_BYTES) != cudaSuccess)
-    return MOE_ERR_CUDA;
-  launch_begin(K_BWD_ACT, st);
-  launch_kernel(grouped_gemm_bwd<0>, dim3((unsigned)sm_count()), dim3(THREADS_DACT),
-                (size_t)SMEM_BYTES, st, 1, none, mb, none, a);
-  moe_status r = launch_end(K_BWD_ACT, st);
-  if (r != MOE_OK) return r;
+  bf16* rows = (bf16*)((uint8_t*)scratch + backward_rows_offset(s));
+  moe_status r;
+  if (backward_copies_rows(s)) {  // dO rows expert-major, then the GEMM loads them by TMA
+    if ((r = launch_gather_rows(s, d_out, p2a, offsets, rows, st)) != MOE_OK) return r;
+    CUtensorMap ma;
+    const uint64_t dims[2] = {(uint64_t)s.d, (uint64_t)A};
+    const uint64_t str[1] = {(uint64_t)s.d * 2};
+    const uint32_t box[2] = {BK, BM};
+    if (!make_map(&ma, rows, 2, dims, str, box)) return MOE_ERR_CUDA;
+    if (cudaFuncSetAttribute(grouped_gemm_bwd<2>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             SMEM_BYTES) != cudaSuccess)
+      return MOE_ERR_CUDA;
+    launch_begin(K_BWD_ACT, st);
+    launch_kernel(grouped_gemm_bwd<2>, dim3((unsigned)sm_count()), dim3(THREADS_DX),
+                  (size_t)SMEM_BYTES, st, 1, ma, mb, none, a);
+  } else {
+    if (cudaFuncSetAttribute(grouped_gemm_bwd<0>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             SMEM_BYTES) != cudaSuccess)
+      return MOE_ERR_CUDA;
+    launch_begin(K_BWD_ACT, st);
+    launch_kernel(grouped_gemm_bwd<0>, dim3((unsigned)sm_count()), dim3(THREADS_DACT),
+                  (size_t)SMEM_BYTES, st, 1, none, mb, none, a);
+  }
+  if ((r = launch_end(K_BWD_ACT, st)) != MOE_OK) return r;
   long long blocks = (A + 255) / 256;
   if (blocks > (long long)sm_count() * 8) blocks = (long long)sm_count() * 8;
   launch_begin(K_BWD_DW, st);
@@ -560,7 +601,7 @@ moe_status launch_backward(const moe_shape& s, const void* d_out, const float* t
   if ((r = launch_end(K_BWD_DW, st)) != MOE_OK) return r;
   if (d_x == nullptr) return MOE_OK;
   // input gradient: dX_perm = (dG | dU) [W_gate | W_up]^T per expert, then the scatter-add
-  bf16* dx_perm = (bf16*)((uint8_t*)scratch + backward_scratch_bytes(s, false));
+  bf16* dx_perm = rows;
   CUtensorMap ma, mg, mu;
   {
     const uint64_t dims[2] = {2 * (uint64_t)s.n, (uint64_t)A};
