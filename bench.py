@@ -434,7 +434,7 @@ def decode_dispatch(tdr, world, Ts=(64, 256, 512, 1024)):
     """Dispatch workload (given N(0,1) logits, E=64 K=6 d=4096 bf16) in the decode regime:
     route + permute with x_perm materialised + combine of those rows, per L2-flushed
     sequence with CUDA events around it, through the two calls (moe_route, moe_permute) and
-    through moe_dispatch (one kernel for routing and permutation)."""
+    through moe_dispatch (the same kernels from one call) with either top-K form."""
     base = mi.CONFIGS["dispatch_combine"]
     dev = torch.device("cuda", torch.cuda.current_device())
     flush = torch.ones(64 << 20, dtype=torch.int64, device=dev)
@@ -489,7 +489,7 @@ def decode_dispatch(tdr, world, Ts=(64, 256, 512, 1024)):
         res[f"T={T}"] = row
     del flush
     # route + permute with x_perm + combine, one sequence per L2-flushed iteration, CUDA
-    # events, launch gaps included; moe_dispatch with either top-K form of its one launch
+    # events, launch gaps included; moe_dispatch with either top-K form of the router
     return {"workload": "dispatch_combine (E=64 K=6 d=4096 bf16, given logits)", "latency": res}
 
 

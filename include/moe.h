@@ -217,10 +217,11 @@ moe_status moe_permute_static(const moe_shape* shape, const int32_t* topk_ids, i
  * the pages describe no separate dispatch operation, this is a launch-count saving for
  * the decode regime. Arguments are the union of both calls' (x serves the router and
  * the optional gather); every output equals what moe_route then moe_permute write.
- * When logits_in is given, T*K <= 4096, E <= 256 and K <= 32, one kernel (one
- * cluster of up to 8 CTAs) routes and permutes without a round trip of the ids through
- * global memory; otherwise the two calls' kernels run in turn. bias is added only to
- * x W_r, as in moe_route.
+ * When logits_in is given, T <= 128, T*K <= 2048, E <= 256 and K <= 32, one kernel (one
+ * CTA) routes and permutes without a round trip of the ids through global memory;
+ * otherwise the two calls' kernels run in turn. A requested x_perm is then copied by
+ * the gather kernel of moe_permute, over the whole GPU. bias is added only to x W_r, as
+ * in moe_route.
  *   workspace, ws_bytes  >= moe_permute_workspace_size(shape)
  * Errors: those of moe_route and moe_permute.
  */

@@ -109,7 +109,7 @@ def test_dispatch_argument_checks_on_host(lib):
     r = lib.moe_dispatch(ctypes.byref(s), None, None, None, dummy, None, None, dummy, dummy,
                          dummy, dummy, dummy, None, None, 0, None)
     assert r == 1
-    # routable from the given logits in one kernel, but no workspace for the permute scratch
+    # given logits, but no workspace for the permute scratch
     r = lib.moe_dispatch(ctypes.byref(s), None, None, None, dummy, None, dummy, dummy, dummy,
                          dummy, dummy, dummy, None, None, 0, None)
     assert r == 4

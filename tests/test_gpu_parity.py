@@ -264,11 +264,13 @@ def test_permute_flags_out_of_range_ids(cuda_lib):
     (1024, 64, 6, 0.0, True, False),
     (1, 1, 1, 0.0, True, False),
     (33, 8, 2, 1.0, False, False),
-    (682, 64, 6, 1.25, True, False),    # 4092 assignments over 8 ragged CTAs of 32 warps
-    (128, 256, 32, 0.0, True, True),    # E = 256, K = 32, integer logits (ties)
-    (800, 37, 5, 0.5, False, True),     # 4000 assignments
-    (683, 64, 6, 0.0, True, False),     # 4098 assignments: the two-call path
-    (1365, 64, 6, 1.25, True, False),
+    (128, 200, 16, 1.25, True, False),  # capacity drops
+    (100, 256, 11, 0.3, False, True),
+    (64, 256, 32, 0.0, True, True),     # E = 256, K = 32, integer logits (ties)
+    (128, 256, 32, 0.0, True, True),
+    (800, 37, 5, 0.5, False, True),
+    (1365, 64, 6, 1.25, True, False),   # the cluster permutation
+    (7000, 64, 6, 0.0, True, False),    # the chunked permutation, four tokens a router warp
 ])
 def test_dispatch_matches_oracle_and_the_two_calls(cuda_lib, route_topk, T, E, K, cf, renorm,
                                                    ties):

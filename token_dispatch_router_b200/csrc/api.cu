@@ -44,12 +44,6 @@ moe_status launch_permute_static(const moe_shape& s, const int32_t* ids, int32_t
                                  void* x_perm, cudaStream_t st);
 moe_status launch_route_tc(const moe_shape& s, const void* x, const void* w_r, const float* bias,
                            float* logits_out, int32_t* ids, float* w, cudaStream_t st);
-bool route_permute_fusable(const moe_shape& s, const float* logits_in);
-moe_status launch_route_permute(const moe_shape& s, const float* logits_in, float* logits_out,
-                                int32_t* ids, float* w, int32_t* counts, int32_t* offsets,
-                                int32_t* a2p, int32_t* p2a, const void* x, void* x_perm,
-                                cudaStream_t st);
-bool route_permute_gathers(const moe_shape& s);
 moe_status launch_gather_rows(const moe_shape& s, const void* x, const int32_t* p2a,
                               const int32_t* offsets, void* x_perm, cudaStream_t st);
 moe_status launch_permute_rounded(const moe_shape& s, const int32_t* ids, const float* logits,
@@ -129,7 +123,7 @@ const char* kKernelNames[K_COUNT] = {
     "route",        "hist",          "scan",           "scatter",     "gather_rows", "gateup_tc",
     "down_tc",      "gateup_simt",   "down_simt",      "combine",     "selftest_timeout",
     "route_tc",     "permute_small", "gateup_tc2",   "down_tc2",
-    "permute_cluster", "route_permute", "tile_round", "bwd_act", "bwd_dw", "bwd_dx",
+    "permute_cluster", "tile_round", "bwd_act", "bwd_dw", "bwd_dx",
     "router_dlogits", "router_dwr", "router_dx", "omni_logits", "omni_topk", "omni_count",
     "omni_scan", "omni_scatter", "omni_sort", "omni_act", "omni_out"};
 
@@ -363,11 +357,6 @@ moe_status forward_impl(const moe_shape* s, const void* x, const void* w_r, cons
                                     ws + L.permute_scratch, (int32_t*)(ws + L.round_ids),
                                     (int32_t*)(ws + L.round_counts), st)) != MOE_OK)
       return r;
-  } else if (route_permute_fusable(*s, logits_in)) {
-    if ((r = launch_route_permute(*s, logits_in, logits, ids, w, counts, offsets, a2p, p2a,
-                                  nullptr, nullptr, st)) !=
-        MOE_OK)
-      return r;
   } else {
     if ((r = moe_route(s, x, w_r, bias, logits_in, logits, ids, w, stream)) != MOE_OK) return r;
     if ((r = launch_permute(*s, ids, counts, offsets, a2p, p2a, nullptr, nullptr,
@@ -512,23 +501,13 @@ moe_status moe_dispatch(const moe_shape* s, const void* x, const void* w_r, cons
                                   (int32_t*)(ws + sb + align256((size_t)s->T * s->K * 4)),
                                   (cudaStream_t)stream);
   }
-  if (!route_permute_fusable(*s, logits_in)) {
-    if ((r = moe_route(s, x, w_r, bias, logits_in, logits_out, topk_ids, topk_w, stream)) != MOE_OK)
-      return r;
-    return moe_permute(s, topk_ids, counts, offsets, assign_to_perm, perm_to_assign,
-                       gather ? x : nullptr, x_perm, workspace, ws_bytes, stream);
-  }
+  // every argument is checked before the first launch
   const size_t need = permute_scratch_bytes(*s);
   if (need > 0 && (workspace == nullptr || ws_bytes < need)) return MOE_ERR_WORKSPACE;
-  const cudaStream_t st = (cudaStream_t)stream;
-  // small gathers are copied by the one-launch kernel itself
-  const bool fuse_gather = gather && route_permute_gathers(*s);
-  if ((r = launch_route_permute(*s, logits_in, logits_out, topk_ids, topk_w, counts, offsets,
-                                assign_to_perm, perm_to_assign, fuse_gather ? x : nullptr,
-                                fuse_gather ? x_perm : nullptr, st)) != MOE_OK)
+  if ((r = moe_route(s, x, w_r, bias, logits_in, logits_out, topk_ids, topk_w, stream)) != MOE_OK)
     return r;
-  if (gather && !fuse_gather) return launch_gather_rows(*s, x, perm_to_assign, offsets, x_perm, st);
-  return MOE_OK;
+  return moe_permute(s, topk_ids, counts, offsets, assign_to_perm, perm_to_assign,
+                     gather ? x : nullptr, x_perm, workspace, ws_bytes, stream);
 }
 
 moe_status moe_grouped_ffn(const moe_shape* s, const void* x, const int32_t* offsets,

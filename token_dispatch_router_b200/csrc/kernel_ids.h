@@ -22,7 +22,6 @@ enum KernelId {
   K_GATEUP_TC2,
   K_DOWN_TC2,
   K_PERMUTE_CLUSTER,
-  K_ROUTE_PERMUTE,
   K_TILE_ROUND,
   K_BWD_ACT,
   K_BWD_DW,

@@ -507,214 +507,9 @@ moe_status launch_cluster_permute(const int32_t* ids, long long A, int E, long l
   return launch_end(K_PERMUTE_CLUSTER, st);
 }
 
-// Routing and permutation in one launch, for given router logits and at most
-// kFusedMax assignments (the decode regime: up to several hundred tokens).
-// "How AI chips support MoE", chapter 4, sections 4.2-4.3 (softmax, top-K) and
-// "Operators & compilers: MoE routing and sparse kernels", section 3 (count, prefix sum,
-// scatter): the steps are those of the router and of the cluster permute above, run by one
-// cluster of C <= 8 CTAs of 8 or 32 warps without a round trip of the ids through global
-// memory.
-// CTA c owns the tokens [c * tpc, (c + 1) * tpc) and so the assignments
-// [c * tpc * K, (c + 1) * tpc * K). Routing: one warp per token, each lane holding up to 8
-// logits (e = lane + 32 j), K rounds of a warp arg-max under (value descending, id
-// ascending; +0 == -0), weights exp(l - l_max) over the selected (renormalised) or over all
-// E; the ids also go to shared memory. Permutation: each warp owns ITERS x 32 of the CTA's
-// assignments, and the histogram, cluster exchange of counts, scan and scatter follow the
-// cluster permute exactly.
-constexpr long long kFusedMax = 4096;  // assignments (above, the two launches were faster)
-constexpr int kFusedTpw = 4;           // tokens a warp routes
+}  // namespace
 
-template <int WARPS, int ITERS, int FORM>
-__global__ void __launch_bounds__(WARPS * 32) route_permute_kernel(
-    const float* __restrict__ logits_in, float* __restrict__ logits_out, int T, int E, int K,
-    int renorm, int tpc, long long cap, int C, int32_t* __restrict__ topk_ids,
-    float* __restrict__ topk_w, int32_t* __restrict__ counts, int32_t* __restrict__ offsets,
-    int32_t* __restrict__ assign_to_perm, int32_t* __restrict__ perm_to_assign,
-    const uint4* __restrict__ x, uint4* __restrict__ x_perm, int vec_per_row) {
-  constexpr int NT = WARPS * 32;
-  constexpr int CHUNK = NT * ITERS;  // assignments a CTA can own
-  static_assert(NT >= kMaxE, "one thread per expert in the scan");
-  __shared__ int rows[WARPS][kMaxE];
-  __shared__ int ctot[kMaxE];
-  __shared__ int cbase[kMaxE];
-  __shared__ int offs[kMaxE];
-  __shared__ int wsum[kMaxE / 32];
-  __shared__ int sid[CHUNK];  // this CTA's ids, in flat assignment order
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const uint32_t rank = C > 1 ? ptx::cluster_rank() : 0u;
-  const int t0 = (int)rank * tpc;
-  const int ntok = max(0, min(tpc, T - t0));
-  const int na = ntok * K;                      // assignments of this CTA
-  const long long a0 = (long long)t0 * K;       // the first one's flat index
-  for (int i = tid; i < WARPS * kMaxE; i += NT) (&rows[0][0])[i] = 0;
-  pdl_wait();  // the previous kernel in the stream has completed
-  pdl_trigger();
-
-  // ---------------------------------------------------------------- routing
-  // a warp routes the tokens warp, warp + WARPS, ... (at most kFusedTpw); all their logits
-  // are loaded before the first is ranked
-  float lv[kFusedTpw][8];
-#pragma unroll
-  for (int i = 0; i < kFusedTpw; ++i) {
-    const int r = warp + i * WARPS;
-#pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      const int e = lane + 32 * j;
-      lv[i][j] = (r < ntok && e < E) ? logits_in[(size_t)(t0 + r) * E + e] : -INFINITY;
-    }
-  }
-#pragma unroll
-  for (int i = 0; i < kFusedTpw; ++i) {
-    const int r = warp + i * WARPS;
-    if (r >= ntok) break;  // warp-uniform
-    const int t = t0 + r;
-    float v[8];
-#pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      const int e = lane + 32 * j;
-      v[j] = lv[i][j];
-      if (logits_out != nullptr && e < E) logits_out[(size_t)t * E + e] = v[j];
-    }
-    int sele;
-    float selw;
-    if (E <= 64) {  // two logits a lane: the bitonic form applies
-      const float v2[2] = {v[0], v[1]};
-      warp_route_token<2, FORM>(v2, E, K, renorm, sele, selw);
-    } else {
-      warp_route_token<8, TOPK_ROUNDS>(v, E, K, renorm, sele, selw);
-    }
-    if (lane < K) {
-      topk_ids[(size_t)t * K + lane] = sele;
-      topk_w[(size_t)t * K + lane] = selw;
-      sid[r * K + lane] = sele;
-    }
-  }
-  __syncthreads();  // the CTA's ids are in shared memory; rows are zeroed
-
-  // ---------------------------------------------------------------- permutation
-  const int l0 = warp * 32 * ITERS;  // this warp's slice of the CTA's assignments
-  int v[ITERS];
-#pragma unroll
-  for (int it = 0; it < ITERS; ++it) {
-    const int l = l0 + it * 32 + lane;
-    v[it] = l < na ? sid[l] : -1;
-  }
-  int* row = rows[warp];
-#pragma unroll
-  for (int it = 0; it < ITERS; ++it) {
-    const unsigned m = __match_any_sync(0xffffffffu, v[it]);
-    if (v[it] >= 0 && lane == __ffs(m) - 1) row[v[it]] += __popc(m);
-    __syncwarp();
-  }
-  __syncthreads();
-  for (int e = warp; e < E; e += WARPS) {
-    const int c = lane < WARPS ? rows[lane][e] : 0;
-    int incl = c;
-#pragma unroll
-    for (int off = 1; off < 32; off <<= 1) {
-      const int y = __shfl_up_sync(0xffffffffu, incl, off);
-      if (lane >= off) incl += y;
-    }
-    if (lane < WARPS) rows[lane][e] = incl - c;
-    if (lane == 31) ctot[e] = incl;
-  }
-  if (C > 1) ptx::cluster_sync();  // every CTA's totals are complete
-  else __syncthreads();
-  int total = 0;
-  if (tid < E) {
-    int cv[kClusterMaxCtas];
-    const uint32_t mine = ptx::saddr(&ctot[tid]);
-#pragma unroll
-    for (int q = 0; q < kClusterMaxCtas; ++q)
-      cv[q] = q == (int)rank ? ctot[tid]
-              : q < C        ? ptx::ld_dsmem_s32(ptx::map_rank(mine, (uint32_t)q))
-                             : 0;
-    int before = 0;
-#pragma unroll
-    for (int q = 0; q < kClusterMaxCtas; ++q) {
-      if (q < (int)rank) before += cv[q];
-      total += cv[q];
-    }
-    cbase[tid] = before;
-    if (rank == 0) counts[tid] = total;
-  }
-  if (C > 1) cluster_arrive();  // remote reads done (waited on before exit)
-  int kept = 0, incl = 0;
-  if (tid < kMaxE) {
-    kept = (tid < E) ? (int)((cap >= 0 && total > cap) ? cap : total) : 0;
-    incl = kept;
-#pragma unroll
-    for (int off = 1; off < 32; off <<= 1) {
-      const int y = __shfl_up_sync(0xffffffffu, incl, off);
-      if (lane >= off) incl += y;
-    }
-    if (lane == 31) wsum[warp] = incl;
-  }
-  __syncthreads();
-  if (tid < kMaxE) {
-    int pre = 0;
-    for (int w = 0; w < warp; ++w) pre += wsum[w];
-    incl += pre;
-    if (tid < E) {
-      offs[tid] = incl - kept;
-      if (rank == 0) {
-        offsets[tid] = incl - kept;
-        if (tid == E - 1) offsets[E] = incl;
-      }
-    }
-  }
-  __syncthreads();
-  const unsigned lt = lanemask_lt();
-  int pos[ITERS];  // each assignment's slot, -1 if dropped
-#pragma unroll
-  for (int it = 0; it < ITERS; ++it) {
-    const int l = l0 + it * 32 + lane;
-    const long long a = a0 + l;
-    const int id = v[it];
-    const unsigned m = __match_any_sync(0xffffffffu, id);
-    int r = 0;
-    if (id >= 0) r = cbase[id] + row[id] + __popc(m & lt);
-    __syncwarp();
-    if (id >= 0 && lane == __ffs(m) - 1) row[id] += __popc(m);
-    __syncwarp();
-    if (id >= 0) {
-      int p = -1;
-      if (cap < 0 || r < cap) {
-        p = offs[id] + r;
-        perm_to_assign[p] = (int32_t)a;
-      }
-      assign_to_perm[a] = p;
-    }
-    pos[it] = id >= 0 && (cap < 0 || r < cap) ? offs[id] + r : -1;
-  }
-  if (x_perm != nullptr) {
-    // the rows of this CTA's kept assignments, x_perm[p] = x[t] (a warp per row, four
-    // 16-byte vectors a lane in flight)
-    __syncthreads();  // every warp's ids have left sid
-#pragma unroll
-    for (int it = 0; it < ITERS; ++it) {
-      const int l = l0 + it * 32 + lane;
-      if (l < na) sid[l] = pos[it];
-    }
-    __syncthreads();
-    for (int l = warp; l < na; l += WARPS) {
-      const int p = sid[l];
-      if (p < 0) continue;
-      const uint4* src = x + (size_t)((a0 + l) / K) * vec_per_row;
-      uint4* dst = x_perm + (size_t)p * vec_per_row;
-      for (int v0 = lane; v0 < vec_per_row; v0 += 128) {
-        uint4 q[4];
-#pragma unroll
-        for (int j = 0; j < 4; ++j)
-          if (v0 + 32 * j < vec_per_row) q[j] = src[v0 + 32 * j];
-#pragma unroll
-        for (int j = 0; j < 4; ++j)
-          if (v0 + 32 * j < vec_per_row) dst[v0 + 32 * j] = q[j];
-      }
-    }
-  }
-  if (C > 1) cluster_wait();  // every CTA has finished reading this CTA's counts
-}
+namespace {
 
 // x_perm[p] = x[perm_to_assign[p] / K] for p < offsets[E]; 16-byte vectors. One warp moves
 // a 2 KB segment (128 vectors) of one row: the row's source token is loaded once per lane
@@ -848,82 +643,6 @@ moe_status launch_gather_rows(const moe_shape& s, const void* x, const int32_t* 
                 p2a, (const int32_t*)(offsets + s.E), s.K, s.T, vec_per_row, (uint4*)x_perm,
                 device_status_ptr());
   return launch_end(K_GATHER, st);
-}
-
-namespace {
-// CTAs of the fused kernel: about 32 tokens per CTA up to 8 CTAs (at least min_ctas, one token
-// each at least); 8 warps per CTA, or 32 when a CTA owns more than 32 tokens (routing runs one
-// token per warp at a time); false if a warp would own more assignments than the
-// instantiated shapes hold (4 x 32 with 8 warps, 2 x 32 with 32)
-bool fused_grid(const moe_shape& s, int min_ctas, int* C_out, int* tpc_out, int* warps_out,
-                int* iters_out) {
-  int C = (s.T + 31) / 32;
-  if (C < min_ctas) C = min_ctas;
-  if (C > kClusterMaxCtas) C = kClusterMaxCtas;
-  if (C > s.T) C = s.T;
-  if (C < 1) C = 1;
-  const int tpc = (s.T + C - 1) / C;
-  const int warps = tpc > 32 ? 32 : 8;
-  if (tpc > warps * kFusedTpw) return false;
-  const long long per = (long long)tpc * s.K;  // assignments per CTA
-  const long long lanes = (long long)warps * 32;
-  if (per > lanes * (warps == 32 ? 2 : 4)) return false;  // the instantiated shapes
-  *C_out = C;
-  *tpc_out = tpc;
-  *warps_out = warps;
-  *iters_out = per <= lanes ? 1 : per <= 2 * lanes ? 2 : 4;
-  return true;
-}
-// The gathered rows are copied by the fused kernel itself (its C <= 8 CTAs) up to this many
-// bytes; beyond, the many-CTA gather kernel is faster.
-constexpr long long kFusedGatherMax = 4ll << 20;
-}  // namespace
-
-bool route_permute_fusable(const moe_shape& s, const float* logits_in) {
-  int C, tpc, warps, iters;
-  return logits_in != nullptr && s.T > 0 && s.E <= kMaxE && s.K <= 32 &&
-         (long long)s.T * s.K <= kFusedMax && fused_grid(s, 1, &C, &tpc, &warps, &iters);
-}
-
-bool route_permute_gathers(const moe_shape& s) {
-  const long long eb = s.dtype == MOE_BF16 ? 2 : 4;
-  return (long long)s.T * s.K * s.d * eb <= kFusedGatherMax;
-}
-
-moe_status launch_route_permute(const moe_shape& s, const float* logits_in, float* logits_out,
-                                int32_t* ids, float* w, int32_t* counts, int32_t* offsets,
-                                int32_t* a2p, int32_t* p2a, const void* x, void* x_perm,
-                                cudaStream_t st) {
-  const long long cap =
-      (s.capacity_factor > 0.f)
-          ? (long long)ceil((double)s.capacity_factor * (double)s.T * (double)s.K / (double)s.E)
-          : -1;
-  int C, tpc, warps, iters;
-  // a fused gather shares the copy over all eight CTAs
-  if (!fused_grid(s, x_perm != nullptr ? kClusterMaxCtas : 1, &C, &tpc, &warps, &iters))
-    return MOE_ERR_UNSUPPORTED;
-  const int vec_per_row = s.d * (s.dtype == MOE_BF16 ? 2 : 4) / 16;
-  const bool bitonic = route_topk_form(s.route_topk, s.E, s.K) == TOPK_BITONIC;
-  launch_begin(K_ROUTE_PERMUTE, st);
-  auto go = [&](auto kern, int nwarps) {
-    launch_kernel(kern, dim3((unsigned)C), dim3(nwarps * 32), 0, st, (unsigned)C, logits_in,
-                  logits_out, s.T, s.E, s.K, s.renormalize, tpc, cap, C, ids, w, counts, offsets,
-                  a2p, p2a, (const uint4*)x, (uint4*)x_perm, vec_per_row);
-  };
-  auto shape = [&](auto form) {
-    constexpr int F = decltype(form)::value;
-    if (warps == 8) {
-      if (iters == 1) go(route_permute_kernel<8, 1, F>, 8);
-      else if (iters == 2) go(route_permute_kernel<8, 2, F>, 8);
-      else go(route_permute_kernel<8, 4, F>, 8);
-    } else {
-      if (iters == 1) go(route_permute_kernel<32, 1, F>, 32);
-      else go(route_permute_kernel<32, 2, F>, 32);
-    }
-  };
-  if (bitonic) shape(std::integral_constant<int, TOPK_BITONIC>());
-  else shape(std::integral_constant<int, TOPK_ROUNDS>());
-  return launch_end(K_ROUTE_PERMUTE, st);
 }
 
 // ------------------------------------------------------------------ token rounding

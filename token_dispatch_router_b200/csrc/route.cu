@@ -7,7 +7,9 @@
 //
 // One CTA owns TM tokens. Phase 1 is a register-tiled fp32 FMA GEMM (x tile and W_r tile
 // staged through shared memory, fp32 accumulation) that leaves the TM x E logits in shared
-// memory; with logits_in the tile is loaded instead. Phase 2 gives one warp per token: each
+// memory. Given logits skip phase 1 and shared memory: a warp loads its tokens' logits
+// straight into registers, all of them before the first is ranked, over enough CTAs to
+// spread a small batch across the SMs. Phase 2 gives one warp per token: each
 // lane holds E/32 logits in registers and the top-K under the total order (value descending,
 // id ascending) comes from K rounds of a warp arg-max or, for E <= 64 and K <= 8, from the
 // bitonic merges of the lanes' sorted lists (moe_shape.route_topk). Selection compares fp32
@@ -135,6 +137,75 @@ __global__ void __launch_bounds__(kThreads) route_kernel(
   }
 }
 
+// Given logits: warp w of CTA b ranks tokens (8 b + w) TPW ... + TPW - 1.
+template <int VPL, int TPW, int FORM>
+__global__ void __launch_bounds__(kThreads) route_given_kernel(
+    const float* __restrict__ logits_in, float* __restrict__ logits_out,
+    int32_t* __restrict__ topk_ids, float* __restrict__ topk_w, int T, int E, int K, int renorm) {
+  pdl_wait();  // the previous kernel in the stream has completed
+  pdl_trigger();
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const long long tw0 = ((long long)blockIdx.x * (kThreads / 32) + warp) * TPW;
+  float v[TPW][VPL];
+#pragma unroll
+  for (int i = 0; i < TPW; ++i) {
+    const long long t = tw0 + i;
+#pragma unroll
+    for (int j = 0; j < VPL; ++j) {
+      const int e = lane + 32 * j;
+      v[i][j] = (t < T && e < E) ? logits_in[t * E + e] : -INFINITY;
+    }
+  }
+#pragma unroll
+  for (int i = 0; i < TPW; ++i) {
+    const long long t = tw0 + i;
+    if (t >= T) break;  // warp-uniform
+    if (logits_out != nullptr && logits_out != logits_in) {
+#pragma unroll
+      for (int j = 0; j < VPL; ++j) {
+        const int e = lane + 32 * j;
+        if (e < E) logits_out[t * E + e] = v[i][j];
+      }
+    }
+    int sele;
+    float selw;
+    warp_route_token<VPL, FORM>(v[i], E, K, renorm, sele, selw);
+    if (lane < K) {
+      topk_ids[t * K + lane] = sele;
+      topk_w[t * K + lane] = selw;
+    }
+  }
+}
+
+template <int VPL>
+moe_status launch_route_given_v(const moe_shape& s, const float* logits_in, float* logits_out,
+                                int32_t* ids, float* w, cudaStream_t st) {
+  const bool bitonic = VPL <= 2 && route_topk_form(s.route_topk, s.E, s.K) == TOPK_BITONIC;
+  // one token a warp while that leaves CTAs for fewer than four waves of the SMs, else four
+  const bool four = (long long)s.T >= 4LL * 8 * 4 * sm_count();
+  const int tpw = four ? 4 : 1;
+  const long long grid = ((long long)s.T + 8LL * tpw - 1) / (8LL * tpw);
+  auto launch = [&](auto kern) {
+    launch_begin(K_ROUTE, st);
+    launch_kernel(kern, dim3((unsigned)grid), dim3(kThreads), 0, st, 1, logits_in, logits_out,
+                  ids, w, s.T, s.E, s.K, s.renormalize);
+    return launch_end(K_ROUTE, st);
+  };
+  if (bitonic)
+    return four ? launch(route_given_kernel<VPL, 4, TOPK_BITONIC>)
+                : launch(route_given_kernel<VPL, 1, TOPK_BITONIC>);
+  return four ? launch(route_given_kernel<VPL, 4, TOPK_ROUNDS>)
+              : launch(route_given_kernel<VPL, 1, TOPK_ROUNDS>);
+}
+
+moe_status launch_route_given(const moe_shape& s, const float* logits_in, float* logits_out,
+                              int32_t* ids, float* w, cudaStream_t st) {
+  if (s.E <= 32) return launch_route_given_v<1>(s, logits_in, logits_out, ids, w, st);
+  if (s.E <= 64) return launch_route_given_v<2>(s, logits_in, logits_out, ids, w, st);
+  if (s.E <= 128) return launch_route_given_v<4>(s, logits_in, logits_out, ids, w, st);
+  return launch_route_given_v<8>(s, logits_in, logits_out, ids, w, st);
+}
+
 template <typename Tin, int CT, int CPT, int RPT>
 moe_status launch_route_t(const moe_shape& s, const void* x, const void* w_r, const float* bias,
                           const float* logits_in, float* logits_out, int32_t* ids, float* w,
@@ -177,6 +248,8 @@ moe_status launch_route_dt(const moe_shape& s, const void* x, const void* w_r, c
 moe_status launch_route(const moe_shape& s, const void* x, const void* w_r, const float* bias,
                         const float* logits_in, float* logits_out, int32_t* ids, float* w,
                         cudaStream_t st) {
+  if (s.T == 0) return MOE_OK;
+  if (logits_in != nullptr) return launch_route_given(s, logits_in, logits_out, ids, w, st);
   if (s.dtype == MOE_BF16)
     return launch_route_dt<bf16>(s, x, w_r, bias, logits_in, logits_out, ids, w, st);
   return launch_route_dt<float>(s, x, w_r, bias, logits_in, logits_out, ids, w, st);
