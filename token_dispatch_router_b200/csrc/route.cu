@@ -5,9 +5,9 @@
 // section 4.2: the gate is a small dense linear map every token passes through; 4.3: the
 // top-K is a partial sort per token.
 //
-// One CTA owns TM tokens. Phase 1 is a register-tiled fp32 FMA GEMM (x tile and W_r tile
-// staged through shared memory, fp32 accumulation) that leaves the TM x E logits in shared
-// memory. Given logits skip phase 1 and shared memory: a warp loads its tokens' logits
+// From x: one CTA owns TM tokens. Phase 1 is a register-tiled fp32 FMA GEMM (x tile and W_r
+// tile staged through shared memory, fp32 accumulation) that leaves the TM x E logits in
+// shared memory. Given logits skip phase 1 and shared memory: a warp loads its tokens' logits
 // straight into registers, all of them before the first is ranked, over enough CTAs to
 // spread a small batch across the SMs. Phase 2 gives one warp per token: each
 // lane holds E/32 logits in registers and the top-K under the total order (value descending,
@@ -30,9 +30,8 @@ constexpr int kDK = 64;
 template <typename Tin, int CT, int CPT, int RPT, int FORM>
 __global__ void __launch_bounds__(kThreads) route_kernel(
     const Tin* __restrict__ x, const Tin* __restrict__ w_r, const float* __restrict__ bias,
-    const float* __restrict__ logits_in, float* __restrict__ logits_out,
-    int32_t* __restrict__ topk_ids, float* __restrict__ topk_w, int T, int d, int E, int K,
-    int renorm) {
+    float* __restrict__ logits_out, int32_t* __restrict__ topk_ids, float* __restrict__ topk_w,
+    int T, int d, int E, int K, int renorm) {
   pdl_wait();  // the previous kernel in the stream has completed
   pdl_trigger();
   constexpr int RT = kThreads / CT;
@@ -45,7 +44,7 @@ __global__ void __launch_bounds__(kThreads) route_kernel(
   const int tid = threadIdx.x;
   const int t0 = blockIdx.x * TM;
 
-  if (logits_in == nullptr) {
+  {
     constexpr int VEC = Vec16<Tin>::N;
     float* xs = lg + TM * LDL;          // [TM][kDK + 1]
     float* ws = xs + TM * (kDK + 1);    // [kDK][EP]
@@ -100,16 +99,10 @@ __global__ void __launch_bounds__(kThreads) route_kernel(
         const float bb = (bias != nullptr && e < E) ? bias[e] : 0.f;
         lg[(tr + i * RT) * LDL + e] = acc[i][j] + bb;
       }
-  } else {
-    for (int i = tid; i < TM * E; i += kThreads) {
-      const int r = i / E, c = i % E;
-      const int t = t0 + r;
-      lg[r * LDL + c] = (t < T) ? logits_in[(size_t)t * E + c] : 0.f;
-    }
   }
   __syncthreads();
 
-  if (logits_out != nullptr && logits_out != logits_in) {
+  if (logits_out != nullptr) {
     for (int i = tid; i < TM * E; i += kThreads) {
       const int r = i / E, c = i % E;
       const int t = t0 + r;
@@ -208,13 +201,12 @@ moe_status launch_route_given(const moe_shape& s, const float* logits_in, float*
 
 template <typename Tin, int CT, int CPT, int RPT>
 moe_status launch_route_t(const moe_shape& s, const void* x, const void* w_r, const float* bias,
-                          const float* logits_in, float* logits_out, int32_t* ids, float* w,
-                          cudaStream_t st) {
+                          float* logits_out, int32_t* ids, float* w, cudaStream_t st) {
   constexpr int RT = kThreads / CT;
   constexpr int TM = RT * RPT;
   constexpr int EP = CT * CPT;
-  size_t smem = (size_t)TM * (EP + 1) * sizeof(float);
-  if (logits_in == nullptr) smem += ((size_t)TM * (kDK + 1) + (size_t)kDK * EP) * sizeof(float);
+  const size_t smem =
+      ((size_t)TM * (EP + 1) + (size_t)TM * (kDK + 1) + (size_t)kDK * EP) * sizeof(float);
   const bool bitonic = route_topk_form(s.route_topk, s.E, s.K) == TOPK_BITONIC;
   auto kern = bitonic ? route_kernel<Tin, CT, CPT, RPT, TOPK_BITONIC>
                       : route_kernel<Tin, CT, CPT, RPT, TOPK_ROUNDS>;
@@ -227,20 +219,19 @@ moe_status launch_route_t(const moe_shape& s, const void* x, const void* w_r, co
   if (grid == 0) return MOE_OK;
   launch_begin(K_ROUTE, st);
   launch_kernel(kern, dim3((unsigned)grid), dim3(kThreads), smem, st, 1, (const Tin*)x,
-                (const Tin*)w_r, bias, logits_in, logits_out, ids, w, s.T, s.d, s.E, s.K,
-                s.renormalize);
+                (const Tin*)w_r, bias, logits_out, ids, w, s.T, s.d, s.E, s.K, s.renormalize);
   return launch_end(K_ROUTE, st);
 }
 
 template <typename Tin>
 moe_status launch_route_dt(const moe_shape& s, const void* x, const void* w_r, const float* bias,
-                           const float* li, float* lo, int32_t* ids, float* w, cudaStream_t st) {
-  if (s.E <= 8) return launch_route_t<Tin, 8, 1, 2>(s, x, w_r, bias, li, lo, ids, w, st);
-  if (s.E <= 16) return launch_route_t<Tin, 16, 1, 4>(s, x, w_r, bias, li, lo, ids, w, st);
-  if (s.E <= 32) return launch_route_t<Tin, 32, 1, 8>(s, x, w_r, bias, li, lo, ids, w, st);
-  if (s.E <= 64) return launch_route_t<Tin, 32, 2, 8>(s, x, w_r, bias, li, lo, ids, w, st);
-  if (s.E <= 128) return launch_route_t<Tin, 32, 4, 4>(s, x, w_r, bias, li, lo, ids, w, st);
-  return launch_route_t<Tin, 32, 8, 2>(s, x, w_r, bias, li, lo, ids, w, st);
+                           float* lo, int32_t* ids, float* w, cudaStream_t st) {
+  if (s.E <= 8) return launch_route_t<Tin, 8, 1, 2>(s, x, w_r, bias, lo, ids, w, st);
+  if (s.E <= 16) return launch_route_t<Tin, 16, 1, 4>(s, x, w_r, bias, lo, ids, w, st);
+  if (s.E <= 32) return launch_route_t<Tin, 32, 1, 8>(s, x, w_r, bias, lo, ids, w, st);
+  if (s.E <= 64) return launch_route_t<Tin, 32, 2, 8>(s, x, w_r, bias, lo, ids, w, st);
+  if (s.E <= 128) return launch_route_t<Tin, 32, 4, 4>(s, x, w_r, bias, lo, ids, w, st);
+  return launch_route_t<Tin, 32, 8, 2>(s, x, w_r, bias, lo, ids, w, st);
 }
 
 }  // namespace
@@ -250,9 +241,8 @@ moe_status launch_route(const moe_shape& s, const void* x, const void* w_r, cons
                         cudaStream_t st) {
   if (s.T == 0) return MOE_OK;
   if (logits_in != nullptr) return launch_route_given(s, logits_in, logits_out, ids, w, st);
-  if (s.dtype == MOE_BF16)
-    return launch_route_dt<bf16>(s, x, w_r, bias, logits_in, logits_out, ids, w, st);
-  return launch_route_dt<float>(s, x, w_r, bias, logits_in, logits_out, ids, w, st);
+  if (s.dtype == MOE_BF16) return launch_route_dt<bf16>(s, x, w_r, bias, logits_out, ids, w, st);
+  return launch_route_dt<float>(s, x, w_r, bias, logits_out, ids, w, st);
 }
 
 }  // namespace moe
