@@ -1115,77 +1115,79 @@ __global__ void __launch_bounds__(256) omni_act_kernel(const bf16* __restrict__ 
 // Token-centric output. A CTA takes one token at a time; its WPT warps split the token's K
 // tasks into contiguous chunks, stream the w_out rows through R-deep cp.async rings and keep
 // 8 CH fp32 sums per lane; the warps' sums are then added in warp order (deterministic).
+// One pass takes only the tasks whose expert lies in [elo, ehi) (a warp first compacts its
+// chunk's (expert, scalar) pairs into shared memory): with the w_out table cut into slabs
+// that fit in L2, each pass gathers its rows from L2 instead of DRAM. The first pass starts
+// from zero, the others from the fp32 row y32[t] the previous one left; the last writes
+// bf16 out[t], the others y32[t].
 template <int CH, int R, int WPT>
 __global__ void __launch_bounds__(WPT * 32) omni_out_kernel(const bf16* __restrict__ w_out,
                                                             const int32_t* __restrict__ ids,
                                                             const float* __restrict__ h,
-                                                            bf16* __restrict__ out, int T, int K,
-                                                            int d, int N, unsigned* status) {
+                                                            bf16* __restrict__ out, float* y32,
+                                                            int T, int K, int d, int N, int elo,
+                                                            int ehi, int first, int last,
+                                                            unsigned* status) {
   using Ring = RowRing<CH, R>;
   static_assert(Ring::BYTES >= CH * 32 * 8 * 4, "a warp's ring holds its partial row");
   extern __shared__ __align__(16) uint8_t sm_out[];
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int kc = (K + WPT - 1) / WPT;
   uint8_t* rg = sm_out + (size_t)warp * Ring::BYTES;
   const uint32_t rbase = saddr(rg);
+  int2* list = reinterpret_cast<int2*>(sm_out + (size_t)WPT * Ring::BYTES) + (size_t)warp * kc;
+  const unsigned lt = lanemask_lt();
   pdl_wait();
   pdl_trigger();
-  const int kc = (K + WPT - 1) / WPT;
   for (int t = blockIdx.x; t < T; t += gridDim.x) {
     const int k0 = min(K, warp * kc), k1 = min(K, k0 + kc);
     const int32_t* tid_ = ids + (size_t)t * K;
     const float* th = h + (size_t)t * K;
+    // this pass's tasks of the chunk, in k order
+    int nv = 0;
+    for (int q0 = k0; q0 < k1; q0 += 32) {
+      const int q = q0 + lane;
+      const int e = q < k1 ? tid_[q] : 0;
+      const float hv = q < k1 ? th[q] : 0.f;
+      if (q < k1 && (unsigned)e >= (unsigned)N) report(status, MOE_ERR_DEVICE_INDEX);
+      const bool in = q < k1 && e >= elo && e < ehi;
+      const unsigned b = __ballot_sync(0xffffffffu, in);
+      if (in) list[nv + __popc(b & lt)] = make_int2(e, __float_as_int(hv));
+      nv += __popc(b);
+    }
+    __syncwarp();
     uint64_t acc[CH][4];  // fp32 pairs (columns 2i, 2i + 1 of each 8-column chunk)
 #pragma unroll
     for (int j = 0; j < CH; ++j)
 #pragma unroll
       for (int q = 0; q < 4; ++q) acc[j][q] = 0ull;
-    int ibase = k0, ewin = k0 + lane < k1 ? tid_[k0 + lane] : -1;
-    int cbase = k0, cwin = ewin;
-    float hwin = k0 + lane < k1 ? th[k0 + lane] : 0.f;
-    auto issue = [&](int q) {
-      if (q < k1) {
-        if (q >= ibase + 32) {
-          ibase = q;
-          ewin = q + lane < k1 ? tid_[q + lane] : -1;
-        }
-        const int e = __shfl_sync(0xffffffffu, ewin, q - ibase);
-        if ((unsigned)e < (unsigned)N) {
-          const uint8_t* src = reinterpret_cast<const uint8_t*>(w_out + (size_t)e * d);
-          const int slot = (q - k0) % R;
+    auto issue = [&](int i) {
+      if (i < nv) {
+        const uint8_t* src = reinterpret_cast<const uint8_t*>(w_out + (size_t)list[i].x * d);
+        const int slot = i % R;
 #pragma unroll
-          for (int j = 0; j < CH; ++j)
-            cp_async16(rbase + slot * Ring::ROW + (lane + 32 * j) * 16, src + (lane + 32 * j) * 16);
-        }
+        for (int j = 0; j < CH; ++j)
+          cp_async16(rbase + slot * Ring::ROW + (lane + 32 * j) * 16, src + (lane + 32 * j) * 16);
       }
       cp_async_commit();
     };
 #pragma unroll
-    for (int i = 0; i < R; ++i) issue(k0 + i);
-    for (int p = k0; p < k1; ++p) {
-      if (p >= cbase + 32) {
-        cbase = p;
-        cwin = p + lane < k1 ? tid_[p + lane] : -1;
-        hwin = p + lane < k1 ? th[p + lane] : 0.f;
-      }
-      const int e = __shfl_sync(0xffffffffu, cwin, p - cbase);
-      const float hv = __shfl_sync(0xffffffffu, hwin, p - cbase);
+    for (int i = 0; i < R; ++i) issue(i);
+    for (int i = 0; i < nv; ++i) {
+      const float hv = __int_as_float(list[i].y);
       uint64_t hh;
       asm("mov.b64 %0, {%1, %1};" : "=l"(hh) : "f"(hv));
       cp_async_wait<R - 1>();
-      if ((unsigned)e < (unsigned)N) {
-        const int slot = (p - k0) % R;
+      const int slot = i % R;
 #pragma unroll
-        for (int j = 0; j < CH; ++j) {
-          const uint4 v = lds16(rbase + slot * Ring::ROW + (lane + 32 * j) * 16);
-          fma2_bf16(v.x, hh, acc[j][0]);
-          fma2_bf16(v.y, hh, acc[j][1]);
-          fma2_bf16(v.z, hh, acc[j][2]);
-          fma2_bf16(v.w, hh, acc[j][3]);
-        }
-      } else if (lane == 0) {
-        report(status, MOE_ERR_DEVICE_INDEX);
+      for (int j = 0; j < CH; ++j) {
+        const uint4 v = lds16(rbase + slot * Ring::ROW + (lane + 32 * j) * 16);
+        fma2_bf16(v.x, hh, acc[j][0]);
+        fma2_bf16(v.y, hh, acc[j][1]);
+        fma2_bf16(v.z, hh, acc[j][2]);
+        fma2_bf16(v.w, hh, acc[j][3]);
       }
-      issue(p + R);
+      issue(i + R);
     }
     cp_async_wait<0>();
     // this warp's partial row, [d] fp32, into its own (now idle) ring
@@ -1201,8 +1203,21 @@ __global__ void __launch_bounds__(WPT * 32) omni_out_kernel(const bf16* __restri
     __syncthreads();
     for (int c8 = threadIdx.x; c8 < d / 8; c8 += WPT * 32) {
       float sum[8];
+      float4* yrow = reinterpret_cast<float4*>(y32 + (size_t)t * d) + c8 * 2;
+      if (first) {
 #pragma unroll
-      for (int q = 0; q < 8; ++q) sum[q] = 0.f;
+        for (int q = 0; q < 8; ++q) sum[q] = 0.f;
+      } else {
+        const float4 y0 = yrow[0], y1 = yrow[1];
+        sum[0] = y0.x;
+        sum[1] = y0.y;
+        sum[2] = y0.z;
+        sum[3] = y0.w;
+        sum[4] = y1.x;
+        sum[5] = y1.y;
+        sum[6] = y1.z;
+        sum[7] = y1.w;
+      }
 #pragma unroll
       for (int w = 0; w < WPT; ++w) {
         const float4* src =
@@ -1217,7 +1232,12 @@ __global__ void __launch_bounds__(WPT * 32) omni_out_kernel(const bf16* __restri
         sum[6] += x1.z;
         sum[7] += x1.w;
       }
-      *reinterpret_cast<uint4*>(out + (size_t)t * d + c8 * 8) = pack16(sum, bf16());
+      if (last) {
+        *reinterpret_cast<uint4*>(out + (size_t)t * d + c8 * 8) = pack16(sum, bf16());
+      } else {
+        yrow[0] = make_float4(sum[0], sum[1], sum[2], sum[3]);
+        yrow[1] = make_float4(sum[4], sum[5], sum[6], sum[7]);
+      }
     }
     __syncthreads();
   }
@@ -1379,19 +1399,34 @@ moe_status launch_act_ch(const moe_omni_shape& s, const void* x, const void* w_i
   return launch_end(K_OMNI_ACT, st);
 }
 
+// w_out bytes a slab of the output gather may hold (it then stays in L2 between the tokens
+// that read it): a 105 MB half of a 210 MB table measured as fast as a table that fits.
+constexpr size_t kSlabBytes = 112u << 20;
+
 template <int CH, int R, int WPT>
 moe_status launch_out_ch(const moe_omni_shape& s, const void* w_out, const int32_t* ids,
-                         const float* h, void* out, cudaStream_t st) {
+                         const float* h, void* out, float* y32, cudaStream_t st) {
   const int N = s.n_rows * s.n_cols;
-  const int smem = WPT * RowRing<CH, R>::BYTES;
+  const int kc = (s.K + WPT - 1) / WPT;
+  const int smem = WPT * (RowRing<CH, R>::BYTES + kc * 8);
   auto kern = omni_out_kernel<CH, R, WPT>;
   if (!set_smem(kern, smem)) return MOE_ERR_CUDA;
   const int cap = sm_count() * resident_ctas(kern, WPT * 32, smem);
   const int grid = s.T < cap ? s.T : cap;
-  launch_begin(K_OMNI_OUT, st);
-  launch_kernel(kern, dim3((unsigned)grid), dim3(WPT * 32), (size_t)smem, st, 1u, (const bf16*)w_out,
-                ids, h, (bf16*)out, s.T, s.K, s.d, N, device_status_ptr());
-  return launch_end(K_OMNI_OUT, st);
+  // slabs of the expert table when there is an fp32 row to carry the sums between them
+  const size_t table = (size_t)N * s.d * 2;
+  const int S = (y32 != nullptr && table > kSlabBytes) ? (int)((table + kSlabBytes - 1) / kSlabBytes)
+                                                       : 1;
+  for (int p = 0; p < S; ++p) {
+    const int elo = (int)((long long)N * p / S), ehi = (int)((long long)N * (p + 1) / S);
+    launch_begin(K_OMNI_OUT, st);
+    launch_kernel(kern, dim3((unsigned)grid), dim3(WPT * 32), (size_t)smem, st, 1u,
+                  (const bf16*)w_out, ids, h, (bf16*)out, y32, s.T, s.K, s.d, N, elo, ehi,
+                  p == 0 ? 1 : 0, p == S - 1 ? 1 : 0, device_status_ptr());
+    const moe_status r = launch_end(K_OMNI_OUT, st);
+    if (r != MOE_OK) return r;
+  }
+  return MOE_OK;
 }
 
 }  // namespace
@@ -1539,17 +1574,17 @@ moe_status launch_omni_act(const moe_omni_shape& s, const void* x, const void* w
 }
 
 moe_status launch_omni_out(const moe_omni_shape& s, const void* w_out, const int32_t* ids,
-                           const float* h, void* out, cudaStream_t st) {
+                           const float* h, void* out, float* y32, cudaStream_t st) {
   switch (s.d / 256) {
-    case 1: return launch_out_ch<1, 8, 4>(s, w_out, ids, h, out, st);
-    case 2: return launch_out_ch<2, 6, 4>(s, w_out, ids, h, out, st);
-    case 3: return launch_out_ch<3, 4, 4>(s, w_out, ids, h, out, st);
-    case 4: return launch_out_ch<4, 4, 4>(s, w_out, ids, h, out, st);
-    case 5: return launch_out_ch<5, 4, 4>(s, w_out, ids, h, out, st);
-    case 6: return launch_out_ch<6, 2, 4>(s, w_out, ids, h, out, st);
-    case 7: return launch_out_ch<7, 2, 4>(s, w_out, ids, h, out, st);
-    case 8: return launch_out_ch<8, 2, 4>(s, w_out, ids, h, out, st);
-    default: return launch_out_ch<16, 2, 4>(s, w_out, ids, h, out, st);
+    case 1: return launch_out_ch<1, 8, 4>(s, w_out, ids, h, out, y32, st);
+    case 2: return launch_out_ch<2, 6, 4>(s, w_out, ids, h, out, y32, st);
+    case 3: return launch_out_ch<3, 4, 4>(s, w_out, ids, h, out, y32, st);
+    case 4: return launch_out_ch<4, 4, 4>(s, w_out, ids, h, out, y32, st);
+    case 5: return launch_out_ch<5, 4, 4>(s, w_out, ids, h, out, y32, st);
+    case 6: return launch_out_ch<6, 2, 4>(s, w_out, ids, h, out, y32, st);
+    case 7: return launch_out_ch<7, 2, 4>(s, w_out, ids, h, out, y32, st);
+    case 8: return launch_out_ch<8, 2, 4>(s, w_out, ids, h, out, y32, st);
+    default: return launch_out_ch<16, 2, 4>(s, w_out, ids, h, out, y32, st);
   }
 }
 
@@ -1717,7 +1752,7 @@ moe_status moe_omni_experts(const moe_omni_shape* s, const void* x, const void* 
   if (!al16(x) || !al16(w_in) || !al16(w_out) || !al16(out)) return MOE_ERR_INVALID_ARG;
   const cudaStream_t st = (cudaStream_t)stream;
   if ((r = launch_omni_act(*s, x, w_in, offsets, perm_to_assign, topk_w, h, st)) != MOE_OK) return r;
-  return launch_omni_out(*s, w_out, topk_ids, h, out, st);
+  return launch_omni_out(*s, w_out, topk_ids, h, out, nullptr, st);  // no fp32 rows: one pass
 }
 
 moe_status moe_omni_forward(const moe_omni_shape* s, const void* x, const void* w_row,
@@ -1750,10 +1785,10 @@ moe_status moe_omni_forward(const moe_omni_shape* s, const void* x, const void* 
   if ((r = launch_omni_schedule(*s, ids, counts, offsets, a2p, p2a, ws + L.scratch, true, false,
                                 st)) != MOE_OK)
     return r;
-  if (s->output_mode == 0)
-    return moe_omni_experts(s, x, w_in, w_out, ids, w, offsets, p2a, h, out, stream);
   if (!al16(x) || !al16(w_in) || !al16(w_out) || !al16(out)) return MOE_ERR_INVALID_ARG;
   if ((r = launch_omni_act(*s, x, w_in, offsets, p2a, w, h, st)) != MOE_OK) return r;
+  if (s->output_mode == 0)  // gathered per token, in L2-sized slabs of w_out
+    return launch_omni_out(*s, w_out, ids, h, out, (float*)(ws + L.y32), st);
   return launch_omni_out_scatter(*s, w_out, offsets, p2a, h, (float*)(ws + L.y32), out, st);
 }
 
