@@ -666,6 +666,9 @@ def _check_rounded_up(tdr, s, v, ref, R, T, E, K, f32):
     (500, 64, 64, 16, 3, 16, "nearest", "f32", True, False),  # the fp32 grouped FFN
     (16384, 64, 64, 128, 8, 128, "nearest", "bf16", True, False),  # chunked permutation
     (129, 64, 64, 3, 1, 1, "up", "bf16", True, False),        # R = 1 changes nothing
+    (1, 64, 64, 8, 2, 16, "up", "bf16", True, False),         # one token: nothing to add
+    (700, 64, 64, 8, 8, 64, "nearest", "bf16", True, False),  # K = E: every token everywhere
+    (900, 64, 128, 16, 4, 32, "nearest", "bf16", False, True),  # plain softmax, ties
 ])
 def test_forward_token_rounding_up_matches_oracle(cuda_lib, T, d, n, E, K, R, mode, dtype,
                                                   renorm, ties):
@@ -707,11 +710,11 @@ def test_forward_token_rounding_up_matches_oracle(cuda_lib, T, d, n, E, K, R, mo
         else:
             assert_bf16_close(g, r, what)
     kept = np.diff(ref["offsets"])
-    if R > 1 and mode == "up":
+    if R > 1 and mode == "up" and T >= R:
         assert n_add > 0
         assert all(k % R == 0 or k == T for k in kept)
-    if R > T:
-        assert np.all(kept == T)  # every expert holds every token
+    if R > T and mode == "up":  # every expert with a routed token holds every token
+        assert np.all((kept == T) | (kept == 0))
 
 
 def _added_rows(tokens, x, w_gate, w_up, w_down, add_tok, add_exp, add_w):
