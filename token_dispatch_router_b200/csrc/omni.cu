@@ -987,21 +987,26 @@ __device__ __forceinline__ void fma2_bf16(uint32_t w, uint64_t hh, uint64_t& acc
       : "r"(w), "l"(hh));
 }
 
-// Sums v[i] over the 32 lanes for all i at once (a butterfly that halves the values held at
-// each step: 31 shuffles for 32 sums); lane l returns the sum of v[l].
-__device__ __forceinline__ float transpose_reduce32(float (&v)[32]) {
+// Sums v[i] over the 32 lanes for all NB values at once: a butterfly that halves the values
+// held at each step (lane masks 16, 8, ...), then plain sums over the lane bits left; lane l
+// returns the sum of v[l / (32 / NB)]. NB = 8: 9 shuffles for 8 sums.
+template <int NB>
+__device__ __forceinline__ float transpose_reduce(float (&v)[NB]) {
   const int lane = threadIdx.x & 31;
 #pragma unroll
-  for (int sft = 16; sft >= 1; sft >>= 1) {
+  for (int half = NB / 2, sft = 16; half >= 1; half >>= 1, sft >>= 1) {
     const bool upper = (lane & sft) != 0;
 #pragma unroll
-    for (int i = 0; i < sft; ++i) {
-      const float send = upper ? v[i] : v[i + sft];
-      const float keep = upper ? v[i + sft] : v[i];
+    for (int i = 0; i < half; ++i) {
+      const float send = upper ? v[i] : v[i + half];
+      const float keep = upper ? v[i + half] : v[i];
       v[i] = keep + __shfl_xor_sync(0xffffffffu, send, sft);
     }
   }
-  return v[0];
+  float s = v[0];
+#pragma unroll
+  for (int sft = 32 / NB / 2; sft >= 1; sft >>= 1) s += __shfl_xor_sync(0xffffffffu, s, sft);
+  return s;
 }
 
 // Expert-centric scalars. The expert-major task list is cut into equal contiguous ranges,
@@ -1009,9 +1014,11 @@ __device__ __forceinline__ float transpose_reduce32(float (&v)[32]) {
 // expert it meets) and streams its tasks' token rows from L2 through an R-deep cp.async
 // ring in shared memory; each lane copies and later reads only its own 16-byte columns,
 // so the ring needs no synchronisation beyond the lane's own cp.async groups. Tasks go in
-// batches of 32: each lane keeps 32 partial dot products, one transposed reduction gives
-// lane l the dot product of task l, and lane l writes that task's scalar
-// h[a] = topk_w[a] * silu(x_{a / K} . w_in[e]).
+// batches of 8: each lane keeps 8 partial dot products, one transposed reduction gives
+// lanes 4i .. 4i + 3 the dot product of task i, and lane 4i writes that task's scalar
+// h[a] = topk_w[a] * silu(x_{a / K} . w_in[e]). (Batches of 32, one task a lane, kept the
+// unrolled loop too large for the instruction cache: no-instruction stalls led the warp
+// state profile.)
 template <int CH, int R>
 __global__ void __launch_bounds__(256) omni_act_kernel(const bf16* __restrict__ x,
                                                        const bf16* __restrict__ w_in,
@@ -1068,16 +1075,18 @@ __global__ void __launch_bounds__(256) omni_act_kernel(const bf16* __restrict__ 
   };
 #pragma unroll
   for (int i = 0; i < R; ++i) issue(P0 + i);
-  for (int base = P0; base < P1; base += 32) {
-    int ca = base + lane < P1 ? p2a[base + lane] : -1;  // this lane's task of the batch
+  constexpr int NB = 8;  // tasks a batch; lanes 4i .. 4i + 3 receive task i's sum
+  for (int base = P0; base < P1; base += NB) {
+    const int mine = base + (lane >> 2);
+    int ca = (lane & 3) == 0 && mine < P1 ? p2a[mine] : -1;  // the task this lane writes
     if (ca >= M) {
       report(status, MOE_ERR_DEVICE_INDEX);
       ca = -1;
     }
     const float cw = ca >= 0 ? topk_w[ca] : 0.f;
-    float v[32];
+    float v[NB];
 #pragma unroll
-    for (int i = 0; i < 32; ++i) {
+    for (int i = 0; i < NB; ++i) {
       const int p = base + i;
       float acc = 0.f;
       if (p < P1) {
@@ -1106,7 +1115,7 @@ __global__ void __launch_bounds__(256) omni_act_kernel(const bf16* __restrict__ 
       }
       v[i] = acc;
     }
-    const float sdot = transpose_reduce32(v);
+    const float sdot = transpose_reduce<NB>(v);
     if (ca >= 0) h[ca] = cw * (sdot / (1.f + expf(-sdot)));
   }
   cp_async_wait<0>();
