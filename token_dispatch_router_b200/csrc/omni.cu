@@ -1573,7 +1573,7 @@ moe_status launch_omni_act(const moe_omni_shape& s, const void* x, const void* w
     case 1: return launch_act_ch<1, 8>(s, x, w_in, offsets, p2a, topk_w, h, st);
     case 2: return launch_act_ch<2, 6>(s, x, w_in, offsets, p2a, topk_w, h, st);
     case 3: return launch_act_ch<3, 4>(s, x, w_in, offsets, p2a, topk_w, h, st);
-    case 4: return launch_act_ch<4, 4>(s, x, w_in, offsets, p2a, topk_w, h, st);
+    case 4: return launch_act_ch<4, 3>(s, x, w_in, offsets, p2a, topk_w, h, st);
     case 5: return launch_act_ch<5, 4>(s, x, w_in, offsets, p2a, topk_w, h, st);
     case 6: return launch_act_ch<6, 2>(s, x, w_in, offsets, p2a, topk_w, h, st);
     case 7: return launch_act_ch<7, 2>(s, x, w_in, offsets, p2a, topk_w, h, st);
