@@ -17,6 +17,7 @@ struct GemmArgs {
   int out_tile;  // output columns per tile (128 gate/up, 256 down)
   int n_tiles;
   int kblocks;   // contraction / 64
+  int kb_split;  // backward dX: k-blocks below it read the first B map, the rest the second
   int E, K, T;
   unsigned* status;
   unsigned long long limit_ns;

@@ -532,6 +532,13 @@ size_t backward_scratch_bytes(const moe_shape& s, bool with_dx) {
 
 moe_status launch_combine(const moe_shape& s, const void* y_perm, const int32_t* a2p,
                           const float* topk_w, void* out, cudaStream_t st);
+moe_status launch_ffn_tc2_gemm(int mode, const CUtensorMap& a, const CUtensorMap& b0,
+                               const CUtensorMap& b1, const GemmArgs& args, cudaStream_t st);
+
+// dX on CTA pairs (256-row tiles) when a pair variant is asked for (ffn_variant 2 or 3),
+// else on single CTAs: at the Mixtral-like shape the pairs measured slower (1.75-1.79
+// against 1.64-1.67 ms), their 256-row tiles padding twice the rows of the 128-row ones.
+bool backward_pair_dx(const moe_shape& s) { return s.ffn_variant >= 2; }
 moe_status launch_gather_rows(const moe_shape& s, const void* x, const int32_t* p2a,
                               const int32_t* offsets, void* x_perm, cudaStream_t st);
 
@@ -602,6 +609,39 @@ moe_status launch_backward(const moe_shape& s, const void* d_out, const float* t
   if (d_x == nullptr) return MOE_OK;
   // input gradient: dX_perm = (dG | dU) [W_gate | W_up]^T per expert, then the scatter-add
   bf16* dx_perm = rows;
+  if (backward_pair_dx(s)) {
+    CUtensorMap pa, pg, pu;
+    {
+      const uint64_t dims[2] = {2 * (uint64_t)s.n, (uint64_t)A};
+      const uint64_t str[1] = {2 * (uint64_t)s.n * 2};
+      const uint32_t box[2] = {BK, 128};
+      if (!make_map(&pa, d_h, 2, dims, str, box)) return MOE_ERR_CUDA;
+    }
+    {
+      const uint64_t dims[3] = {(uint64_t)s.n, (uint64_t)s.d, (uint64_t)s.E};
+      const uint64_t str[2] = {(uint64_t)s.n * 2, (uint64_t)s.d * s.n * 2};
+      const uint32_t box[3] = {BK, 128, 1};  // this CTA's 128 of the pair's 256 output columns
+      if (!make_map(&pg, w_gate, 3, dims, str, box)) return MOE_ERR_CUDA;
+      if (!make_map(&pu, w_up, 3, dims, str, box)) return MOE_ERR_CUDA;
+    }
+    GemmArgs ga = {};
+    ga.offsets = offsets;
+    ga.p2a = p2a;
+    ga.out = dx_perm;
+    ga.ld_out = s.d;
+    ga.n_out = s.d;
+    ga.out_tile = 256;
+    ga.n_tiles = (s.d + 255) / 256;
+    ga.kblocks = 2 * s.n / BK;
+    ga.kb_split = s.n / BK;
+    ga.E = s.E;
+    ga.K = s.K;
+    ga.T = s.T;
+    ga.status = device_status_ptr();
+    ga.limit_ns = kWaitLimitNs;
+    if ((r = launch_ffn_tc2_gemm(3, pa, pg, pu, ga, st)) != MOE_OK) return r;
+    return launch_combine(s, dx_perm, a2p, nullptr, d_x, st);  // unit weights: a plain sum
+  }
   CUtensorMap ma, mg, mu;
   {
     const uint64_t dims[2] = {2 * (uint64_t)s.n, (uint64_t)A};

@@ -663,6 +663,7 @@ static moe_status prepare_ffn(const moe_shape& s, const void* x, const int32_t* 
   ga.out_tile = 128;
   ga.n_tiles = (s.n + 127) / 128;
   ga.kblocks = s.d / BK;
+  ga.kb_split = ga.kblocks;
   GemmArgs& gd = f.down;
   gd = ga;
   gd.out = (bf16*)y_perm;
@@ -671,6 +672,7 @@ static moe_status prepare_ffn(const moe_shape& s, const void* x, const int32_t* 
   gd.out_tile = BN;
   gd.n_tiles = (s.d + BN - 1) / BN;
   gd.kblocks = s.n / BK;
+  gd.kb_split = gd.kblocks;
   return MOE_OK;
 }
 

@@ -11,6 +11,9 @@
 //   gate/up: rank 0 holds the W_gate columns n0..n0+127, rank 1 the W_up columns, so every
 //   thread still finds its row's (gate, up) pairs in TMEM columns c and 128 + c.
 //   down:    rank r holds W_down columns n0 + 128 r .. + 127.
+//   backward dX (MODE 3): dX_perm = (dG | dU) (W_gate | W_up)^T: A = the d_h rows by TMA,
+//   B K-major (rank r holds rows n0 + 128 r .. + 127 of W_gate[e], or of W_up[e] for the
+//   second half of the contraction, read in place as the transposes).
 // Synchronisation: TMA loads of both CTAs (.cta_group::2) complete on the leader's full
 // barrier; gate/up gathers by cp.async complete on the leader's barrier directly (leader)
 // or on a local barrier that one peer thread relays to the leader after a proxy fence
@@ -42,6 +45,7 @@ constexpr int MAXE = 256;
 constexpr int SMEM_TAIL = 4096;
 constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 + SMEM_TAIL;
 constexpr uint32_t IDESC = idesc_bf16(PAIR_M, BN);
+constexpr uint32_t IDESC_BK = IDESC & ~(1u << 16);  // B K-major (backward dX)
 
 
 struct Tile2 {
@@ -69,7 +73,8 @@ __device__ __forceinline__ Tile2 decode2(int w, const int* s_off, const int* s_c
 
 // MODE 0: down GEMM (A = the activations, by TMA); 1: gate/up GEMM with the A rows
 // gathered from x by cp.async; 2: gate/up GEMM with A = rows already gathered into an
-// expert-major buffer, by TMA (no gather warps, no relay).
+// expert-major buffer, by TMA (no gather warps, no relay); 3: backward dX (A = the d_h
+// rows by TMA, B K-major from W_gate then W_up).
 template <int MODE>
 __global__ void __launch_bounds__(MODE == 1 ? THREADS_GATEUP : THREADS_DOWN, 1)
     grouped_gemm_tc2(const __grid_constant__ CUtensorMap tmA,
@@ -91,7 +96,8 @@ __global__ void __launch_bounds__(MODE == 1 ? THREADS_GATEUP : THREADS_DOWN, 1)
   int* s_cum = s_off + MAXE + 1;
   int* s_mt = s_cum + MAXE + 1;
 
-  constexpr bool GATEUP = MODE != 0;
+  constexpr bool GATEUP = MODE == 1 || MODE == 2;
+  constexpr bool BKMAJOR = MODE == 3;
   constexpr bool GATHER = MODE == 1;
   constexpr int NTHREADS = GATHER ? THREADS_GATEUP : THREADS_DOWN;
   // leader's full[s]: the leader's expect_tx arrival for the TMA bytes of both CTAs (+ the
@@ -184,7 +190,13 @@ __global__ void __launch_bounds__(MODE == 1 ? THREADS_GATEUP : THREADS_DOWN, 1)
         const uint32_t a_dst = saddr(ring + stage * STAGE_BYTES);
         const uint32_t b_dst = a_dst + A_BYTES;
         if (!GATHER && lane == 0) tma_load_2d_pair(a_dst, &tmA, kb * BK, t.m0, fb);
-        if (lane < 2) {
+        if (BKMAJOR) {
+          if (lane == 0) {
+            const bool first = kb < g.kb_split;
+            tma_load_3d_pair(b_dst, first ? &tmB0 : &tmB1, (first ? kb : kb - g.kb_split) * BK,
+                             t.n0 + (int)rank * 128, t.e, fb);
+          }
+        } else if (lane < 2) {
           if (GATEUP)
             tma_load_3d_pair(b_dst + lane * B_CHUNK, leader ? &tmB0 : &tmB1, t.n0 + lane * 64,
                              kb * BK, t.e, fb);
@@ -239,8 +251,9 @@ __global__ void __launch_bounds__(MODE == 1 ? THREADS_GATEUP : THREADS_DOWN, 1)
 #pragma unroll
           for (int kk = 0; kk < BK / 16; ++kk) {
             const uint64_t ad = desc_sw128(a_addr + kk * 32, 16, 1024);
-            const uint64_t bd = desc_sw128(b_addr + kk * 2048, B_CHUNK, 1024);
-            tc_mma<2>(d_tmem, ad, bd, IDESC, (kb | kk) != 0 ? 1u : 0u);
+            const uint64_t bd = BKMAJOR ? desc_sw128(b_addr + kk * 32, 16, 1024)
+                                        : desc_sw128(b_addr + kk * 2048, B_CHUNK, 1024);
+            tc_mma<2>(d_tmem, ad, bd, BKMAJOR ? IDESC_BK : IDESC, (kb | kk) != 0 ? 1u : 0u);
           }
           tc_commit<2>(saddr(&empty[stage]));
           tc_commit<2>(map_rank(saddr(&empty[stage]), 1));
@@ -433,6 +446,7 @@ moe_status launch_ffn_tc2_gemm(int mode, const CUtensorMap& a, const CUtensorMap
                                const CUtensorMap& b1, const GemmArgs& args, cudaStream_t st) {
   if (mode == 1) return run_gemm2<1>(a, b0, b1, args, st, K_GATEUP_TC2);
   if (mode == 2) return run_gemm2<2>(a, b0, b1, args, st, K_GATEUP_TC2);
+  if (mode == 3) return run_gemm2<3>(a, b0, b1, args, st, K_BWD_DX);
   return run_gemm2<0>(a, b0, b1, args, st, K_DOWN_TC2);
 }
 
