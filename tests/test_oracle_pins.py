@@ -397,7 +397,7 @@ def test_planted_mistakes_are_caught(monkeypatch):
 
 # ------------------------------------------------------------------ token rounding
 # SonicMoE explainer (gitcode.csdn.net), section 6.5 names tile-aware token rounding
-# without a rule; the rule pinned here is this build's reading: an expert with c >= R
+# without a rule; the rule pinned here is the library's reading: an expert with c >= R
 # routed assignments keeps R * floor(c / R) of them, the ones with the largest logit for
 # that expert (equal logits: the earlier token stays), experts with c < R keep all.
 def _hand_logits():
