@@ -913,7 +913,7 @@ def test_backward_act_full_size_sampled_slots(cuda_lib):
 
 
 @pytest.mark.parametrize("renorm", [True, False])
-@pytest.mark.parametrize("E,K", [(16, 3), (40, 4), (128, 8)])  # > 16: the tiled kernels
+@pytest.mark.parametrize("E,K", [(16, 3), (40, 4), (128, 8)])  # > 16: the tensor-core forms
 def test_backward_router_matches_oracle(cuda_lib, renorm, E, K):
     tdr = cuda_lib
     T, d, n = 700, 256, 128
@@ -946,6 +946,55 @@ def test_backward_router_matches_oracle(cuda_lib, renorm, E, K):
         mask = np.zeros((T, E), bool)
         np.put_along_axis(mask, ids, True, axis=1)
         assert np.all(d_logits.cpu().numpy()[~mask] == 0)
+
+
+@pytest.mark.parametrize("T,d,E,K,renorm,with_bias,misalign_w_r", [
+    (5, 192, 24, 2, True, True, False),        # one block of tokens: most ranks sum nothing
+    (1000, 320, 200, 8, False, True, False),   # 4 expert chunks; the last column tile half out
+    (2049, 128, 64, 4, True, False, False),    # one expert chunk, no bias
+    (300, 256, 136, 6, False, True, False),    # 3 expert chunks, E not a multiple of 32
+    (4100, 2048, 128, 8, True, True, False),   # 16 column tiles x 8 token ranges
+    (700, 256, 36, 3, True, True, False),      # E % 8 != 0: the CUDA-core forms
+    (700, 256, 64, 4, True, True, True),       # W_r not 16-byte aligned: CUDA-core d_x term
+])
+def test_backward_router_forms(cuda_lib, T, d, E, K, renorm, with_bias, misalign_w_r):
+    """moe_backward_router against the oracle over the shapes that select its kernel forms:
+    d_W_r, d_bias and the d_x term (added to a non-zero d_x) for uneven token blocks, partial
+    column tiles, 1-4 expert chunks, and the CUDA-core fallbacks."""
+    tdr = cuda_lib
+    rng = np.random.default_rng(T + d + E)
+    x = torch.from_numpy(rng.standard_normal((T, d)).astype(np.float32)).to(torch.bfloat16)
+    w_r = torch.from_numpy((0.05 * rng.standard_normal((d, E))).astype(np.float32)).to(
+        torch.bfloat16)
+    logits = torch.from_numpy(rng.standard_normal((T, E)).astype(np.float32))
+    d_w = torch.from_numpy(rng.standard_normal((T, K)).astype(np.float32))
+    s = tdr.make_shape(T, d, E, K, 64, 0.0, renorm, torch.bfloat16)
+    ids, w, _ = tdr.route(s, logits_in=logits.cuda())
+    ref = orc.backward_router(d_w.numpy(), ids.cpu().numpy(), logits.numpy(), x, w_r, renorm)
+    # a d_x to add to, at a tenth of the router term's spread (its bf16 rounding stays small
+    # against the term)
+    d_x0 = torch.from_numpy((0.1 * ref[3].std() * rng.standard_normal((T, d))).astype(
+        np.float32)).to(torch.bfloat16)
+    w_r_dev = w_r.cuda()
+    if misalign_w_r:  # the same values 2 bytes past a 16-byte boundary
+        buf = torch.empty(d * E + 8, dtype=torch.bfloat16, device="cuda")
+        w_r_dev = buf[1:1 + d * E].view(d, E)
+        w_r_dev.copy_(w_r.cuda())
+        assert w_r_dev.data_ptr() % 16 != 0
+    d_x = d_x0.cuda()
+    d_logits, d_w_r, d_bias = tdr.backward_router(s, x.cuda(), w_r_dev, ids, w, d_w.cuda(),
+                                                  logits=logits.cuda(), d_x=d_x,
+                                                  with_bias=with_bias)
+    torch.cuda.synchronize()
+    assert_status_ok(tdr)
+    np.testing.assert_allclose(d_logits.cpu().numpy(), ref[0], rtol=1e-4, atol=1e-6)
+    np.testing.assert_allclose(d_w_r.cpu().numpy(), ref[1], rtol=1e-3, atol=1e-4)
+    if with_bias:
+        np.testing.assert_allclose(d_bias.cpu().numpy(), ref[2], rtol=1e-3, atol=1e-4)
+    else:
+        assert d_bias is None
+    assert_bf16_close(d_x.float().cpu().numpy() - d_x0.float().numpy(), ref[3],
+                      "router term of d_x")
 
 
 @pytest.mark.parametrize("T", mi.DISPATCH_COMBINE_T)

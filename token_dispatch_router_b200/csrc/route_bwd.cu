@@ -375,6 +375,13 @@ __global__ void __launch_bounds__(256) router_dx_tiled_kernel(const bf16* __rest
 
 }  // namespace
 
+// route_bwd_tc.cu: the tensor-core forms of d_W_r (with d_bias) and of the d_x term; they
+// set *used = false for the shapes and alignments they do not take.
+moe_status launch_router_dwr_tc(const moe_shape& s, const void* x, const float* d_logits,
+                                float* d_w_r, float* d_bias, cudaStream_t st, bool* used);
+moe_status launch_router_dx_tc(const moe_shape& s, const void* w_r, const float* d_logits,
+                               void* d_x, cudaStream_t st, bool* used);
+
 moe_status launch_router_backward(const moe_shape& s, const void* x, const void* w_r,
                                   const float* logits, const int32_t* ids, const float* topk_w,
                                   const float* d_w, float* d_logits, float* d_w_r,
@@ -389,14 +396,17 @@ moe_status launch_router_backward(const moe_shape& s, const void* x, const void*
                   d_w, logits, T, E, K, s.renormalize, d_logits);
     if ((r = launch_end(K_ROUTER_DLOGITS, st)) != MOE_OK) return r;
   }
-  if (E > 16) {
+  bool tc = false;
+  if (E > 16 && (r = launch_router_dwr_tc(s, x, d_logits, d_w_r, d_bias, st, &tc)) != MOE_OK)
+    return r;
+  if (E > 16 && !tc) {  // the CUDA-core forms for the other wide routers
     const int tiles = ((d + kWt - 1) / kWt) * ((E + kWt - 1) / kWt);
     launch_begin(K_ROUTER_DWR, st);
     launch_kernel(router_dwr_tiled_kernel, dim3((unsigned)(tiles * kWsplit)), dim3(256), 0, st,
                   (unsigned)kWsplit, (const bf16*)x, (const float*)d_logits, T, d, E, d_w_r,
                   d_bias);
     if ((r = launch_end(K_ROUTER_DWR, st)) != MOE_OK) return r;
-  } else {
+  } else if (E <= 16) {
     const int EC = E <= 8 ? 8 : 16;
     const dim3 grid((unsigned)((d + 31) / 32), (unsigned)((E + EC - 1) / EC));
     const dim3 block(kDwrWarps * 32);
@@ -409,7 +419,11 @@ moe_status launch_router_backward(const moe_shape& s, const void* x, const void*
                     (const float*)d_logits, T, d, E, d_w_r, d_bias);
     if ((r = launch_end(K_ROUTER_DWR, st)) != MOE_OK) return r;
   }
-  if (d_x != nullptr && E > 16) {
+  tc = false;
+  if (d_x != nullptr && E > 16 &&
+      (r = launch_router_dx_tc(s, w_r, d_logits, d_x, st, &tc)) != MOE_OK)
+    return r;
+  if (d_x != nullptr && E > 16 && !tc) {
     const int Ep = (E + kWk - 1) / kWk * kWk;  // experts padded to whole chunks
     const int smem = (Ep + kWk) * kWt * (int)sizeof(float);
     if (cudaFuncSetAttribute(router_dx_tiled_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -421,7 +435,7 @@ moe_status launch_router_backward(const moe_shape& s, const void* x, const void*
                   dim3(256), (size_t)smem, st, 1, (const bf16*)w_r, (const float*)d_logits, T, d,
                   E, Ep, (bf16*)d_x);
     if ((r = launch_end(K_ROUTER_DX, st)) != MOE_OK) return r;
-  } else if (d_x != nullptr) {
+  } else if (d_x != nullptr && E <= 16) {
     const int smem = 64 * E * (int)sizeof(float);
     if (cudaFuncSetAttribute(router_dx_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              smem) != cudaSuccess)
