@@ -363,7 +363,10 @@ moe_status moe_backward(const moe_shape* shape, const void* d_out, const float* 
  *   d_logits [T, E] fp32 out (also the intermediate); d_w_r [d, E] fp32 out;
  *   d_bias [E] fp32 out or NULL; d_x [T, d] bf16 in/out or NULL (16-byte aligned); with
  *   E > 16, x 16-byte aligned too.
- * Sums over tokens run in a fixed order (deterministic). bf16 only.
+ * Sums over tokens run in a fixed order (deterministic). bf16 only. With 17..256 experts,
+ * E % 8 == 0 and w_r, d_logits 16-byte aligned, both contractions run on the tensor cores
+ * with each d_logits value split into two bf16 terms (hi = bf16(v), lo = bf16(v - hi):
+ * |v - hi - lo| <= 2^-16 |v|), so the sums keep fp32 accuracy.
  */
 moe_status moe_backward_router(const moe_shape* shape, const void* x, const void* w_r,
                                const float* logits, const int32_t* topk_ids, const float* topk_w,

@@ -15,8 +15,9 @@
 // CTAs that own 32 columns of W_r and EC experts and sum over all tokens in a fixed order
 // (sixteen token groups, then the groups in order: deterministic); the input-gradient term
 // by CTAs that own 64 columns of d with that slice of W_r in shared memory, 8 threads per
-// token row slice, fp32 sums added to the bf16 d_x. Routers with more than 16 experts use
-// register-tiled forms of the last two (below), whose work per token grows with E.
+// token row slice, fp32 sums added to the bf16 d_x. Routers with more than 16 experts run
+// the last two on the tensor cores (route_bwd_tc.cu) where E % 8 == 0 and the operands are
+// 16-byte aligned, else in the register-tiled forms below.
 #include <math.h>
 
 #include "common.cuh"
