@@ -29,13 +29,17 @@
 // threads): warp 0 issues the x loads, warp 1 the MMAs, warps 2-9 convert; warps 2-5 read
 // the accumulator (warp w may read TMEM lanes 32 (w % 4) ...).
 //
-// d_x (router_dx_tc_kernel): D[t, j] = sum_e dL/dl[t, e] W_r[j, e], 128 tokens on M and 128
-// columns of d on N, K = experts (at most 256, so one shot: no ring). A = the tile's dL/dl
-// rows as hi and lo terms (K-major, converted by all threads, one float4 each), B = W_r rows
-// by TMA (K-major: W_r is [d, E] with E innermost). The tile's d_x values are loaded at the
-// start (whole 128-byte row segments per 8 threads); after the MMAs the sums go through
-// shared memory in two 64-column halves, so that the read-add-store of d_x runs on the same
-// row-contiguous pattern, rounding once as the CUDA-core form does.
+// d_x: D[t, j] = sum_e dL/dl[t, e] W_r[j, e], 128 tokens on M and 128 columns of d on N,
+// K = experts (at most 256: one shot per tile). A = the tile's dL/dl rows as hi and lo terms
+// (K-major, converted by all threads, one float4 each), B = W_r rows by TMA (K-major: W_r is
+// [d, E] with E innermost); the sums are added to the bf16 d_x and rounded once, as the
+// CUDA-core form does. Two kernels:
+//  - E <= 128, router_dx_tc_stream_kernel: one CTA per token tile converts A once and
+//    streams the column tiles, d_x moving by TMA through a 3-stage ring (described below);
+//  - E > 128, router_dx_tc_kernel: one CTA per 128 x 128 tile (A and B leave no room for the
+//    ring); the tile's d_x values are loaded at the start (whole 128-byte row segments per 8
+//    threads) and after the MMAs the sums go through shared memory in two 64-column halves,
+//    so that the read-add-store of d_x runs on that row-contiguous pattern.
 //
 // Every mbarrier wait is bounded: on expiry the status word records MOE_ERR_TIMEOUT, the
 // abort flag makes the CTA's other waits give up, nothing is stored, and the TMEM and the
